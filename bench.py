@@ -1,0 +1,377 @@
+#!/usr/bin/env python
+"""Benchmark of the displaced-patch UNet layer step on B200: layer-steps/s and latent px/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--impl ours|reference]
+
+One "step" is one displaced layer step (dfp_step with is_sync = 0) of the
+workload: GN1 statistics + corrected merge, GN1 apply + SiLU, halo refresh,
+conv3x3, GN2 statistics + merge + apply, Q/K/V projection, displaced attention,
+output projection.  The run first executes the synchronous warm-up steps of the
+schedule (untimed), then W displaced warm-up steps, then K timed displaced steps,
+each bracketed by CUDA events on the library's stream; L2 is flushed (a 512 MB
+write) between timed steps, outside the events.  With N > 1 (torchrun) every
+rank runs an independent replica (the layer step does not shard on one GPU
+each: replicas only); value = total steps of all ranks / max over ranks of the
+summed step time.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (numpy fp64) on the host cores instead:
+the same metric on the same workload, full (unsampled) displaced steps.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from patch_diffusion_unet_b200 import configs, inputs  # noqa: E402
+
+METRIC = "displaced-patch layer-steps/s & latent px/s on 1 B200; % tensor/HBM roofline"
+UNIT = "layer-steps/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--profile-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return PEAKS_FALLBACK, "fallback"
+
+
+# ---------------------------------------------------------------------------- work model
+
+def work_model(cfg):
+    """Algorithmic FLOPs / bytes per launch of each kernel of one layer step."""
+    H, W, C, N, heads = cfg["H"], cfg["W"], cfg["C"], cfg["n_patches"], cfg["heads"]
+    L, d = H * W, cfg["head_dim"]
+    e = 2 if cfg["dtype"] == "bf16" else 4
+    R = H // N
+    return {
+        "gn1 statistics": ("hbm", L * C * e),
+        "gn1 apply": ("hbm", 2 * L * C * e),
+        "halo refresh": ("hbm", 2 * 2 * (N - 1) * W * C * e),
+        "conv (tcgen05)": ("tensor", 2.0 * L * C * 9 * C),
+        "gn2 statistics": ("hbm", L * C * e),
+        "gn2 apply": ("hbm", 2 * L * C * e),
+        "qkv (tcgen05)": ("tensor", 2.0 * L * C * 3 * C),
+        "attention (tcgen05)": ("tensor", 4.0 * L * L * d * heads),
+        "out projection (tcgen05)": ("tensor", 2.0 * L * C * C),
+        "_total_flops": 2.0 * L * C * 9 * C + 2.0 * L * C * 4 * C + 4.0 * L * L * d * heads,
+        "_rows_per_patch": R,
+    }
+
+
+# ---------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    COLS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+            "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+            "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.COLS}", "--format=csv,noheader,nounits",
+                                       "-i", str(gpu_index), "-lms", "200"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        sm, mx, reasons = [], [], set()
+        for line in self.f.read().splitlines():
+            cols = [c.strip() for c in line.split(",")]
+            if len(cols) < 9:
+                continue
+            try:
+                sm.append(float(cols[1]))
+                mx.append(float(cols[2]))
+            except ValueError:
+                continue
+            for name, v in zip(self.NAMES, cols[5:9]):
+                if v == "Active":
+                    reasons.add(name)
+        os.unlink(self.f.name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------- CPU oracle leg
+
+def oracle_displaced_rate(cfg, n_disp=2):
+    """Time the oracle as it stands on full displaced steps of the workload (after one sync step)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    wl = inputs.SyntheticWorkload(cfg)
+    blk = oracle.make_block(cfg, wl.weights, wl.context)
+    blk.step(wl.x(0), 0, 1)
+    t0 = time.perf_counter()
+    for t in range(1, 1 + n_disp):
+        blk.step(wl.x(t), t, 0)
+    dt = time.perf_counter() - t0
+    return n_disp / dt, threads, dt
+
+
+# ---------------------------------------------------------------------------- main
+
+def dist_setup():
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def run_reference(args, cfg):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    import oracle
+    wl = inputs.SyntheticWorkload(cfg)
+    blk = oracle.make_block(cfg, wl.weights, wl.context)
+    n_sync = cfg["n_sync"]
+    t = 0
+    for t in range(n_sync):
+        blk.step(wl.x(t), t, 1)
+    for _ in range(args.warmup):
+        t += 1
+        blk.step(wl.x(t), t, 0)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        t += 1
+        blk.step(wl.x(t), t, 0)
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    value = args.steps / dt
+    L = cfg["H"] * cfg["W"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "latent_px_per_s": value * L,
+        "config": {"workload": cfg["name"], "H": cfg["H"], "W": cfg["W"], "C": cfg["C"],
+                   "n_patches": cfg["n_patches"], "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{args.steps} full displaced layer steps after {n_sync} sync steps"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    cfg = configs.get(args.config)
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+
+    import torch
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    import torch.distributed as dist
+    from patch_diffusion_unet_b200 import dfp
+
+    dtype = cfg["dtype"]
+    L = cfg["H"] * cfg["W"]
+    wl = inputs.SyntheticWorkload(cfg)
+    blk = dfp.DisplacedPatchBlock(cfg)
+    blk.load_weights(wl.weights)
+    stream = blk.stream
+    n_pool = 16
+    host_x = [inputs.to_torch(wl.x(t), dtype) for t in range(n_pool)]
+    xs = [h.cuda() for h in host_x]
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+
+    def x_of(t):
+        return xs[t % n_pool]
+
+    n_sync = cfg["n_sync"]
+    for t in range(n_sync):
+        blk.step(x_of(t), t, 1)
+    t = n_sync - 1
+    # warm-up: at least W displaced steps and at least ~1.5 s (clocks settle, sampler sees load)
+    gpu_index = os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local] if \
+        os.environ.get("CUDA_VISIBLE_DEVICES") else str(local)
+    sampler = ClockSampler(gpu_index)
+    w_start = time.perf_counter()
+    n_warm = 0
+    while n_warm < args.warmup or time.perf_counter() - w_start < 1.5:
+        t += 1
+        blk.step(x_of(t), t, 0)
+        flush.zero_()
+        n_warm += 1
+        if n_warm % 16 == 0:
+            torch.cuda.synchronize()
+    blk.check_device()
+
+    # ---- timed region
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        t += 1
+        ev[i][0].record(stream)
+        blk.step(x_of(t), t, 0)
+        ev[i][1].record(stream)
+        flush.zero_()
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    blk.check_device()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = float(sum(step_ms))
+    tt = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    total_ms_max = float(tt.item())
+    value = world * args.steps / (total_ms_max / 1e3)
+    launches = blk.launches_per_step()
+
+    # ---- per-kernel durations (separate profiled steps, same stream, L2 flushed between)
+    blk.set_profiling(True)
+    per = {}
+    for _ in range(args.profile_steps):
+        t += 1
+        blk.step(x_of(t), t, 0)
+        for name, ms in blk.kernel_times():
+            per.setdefault(name, []).append(ms)
+        flush.zero_()
+    blk.set_profiling(False)
+    kern_us = {k: 1e3 * statistics.mean(v) for k, v in per.items()}
+
+    # ---- sync step time (for context)
+    sync_ms = None
+
+    # ---- end to end through the host-buffer entry point (pinned host memory)
+    e2e = None
+    if not args.no_e2e:
+        xh = [h.pin_memory() for h in host_x]
+        yh = torch.empty(L, cfg["C"], dtype=xh[0].dtype).pin_memory()
+        for _ in range(3):
+            t += 1
+            blk.step_host(xh[t % n_pool], yh, t, 0)
+        e_total = 0.0
+        n_e = max(10, min(args.steps, 100))
+        for _ in range(n_e):
+            t += 1
+            flush.zero_()
+            torch.cuda.synchronize()
+            w0 = time.perf_counter()
+            blk.step_host(xh[t % n_pool], yh, t, 0)
+            e_total += time.perf_counter() - w0
+        et = torch.tensor([e_total], device="cuda", dtype=torch.float64)
+        if world > 1:
+            dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        nbytes = L * cfg["C"] * (2 if dtype == "bf16" else 4)
+        e2e = {"value": world * n_e / float(et.item()), "unit": UNIT, "h2d_bytes_per_step": nbytes,
+               "d2h_bytes_per_step": nbytes, "steps": n_e}
+
+    # ---- roofline of the dominant kernel
+    pk, pk_src = peaks()
+    wm = work_model(cfg)
+    dom = max(kern_us, key=kern_us.get) if kern_us else None
+    roof = None
+    if dom and dom in wm:
+        bound, work = wm[dom]
+        us = kern_us[dom]
+        if bound == "tensor":
+            ach = work / (us * 1e-6) / 1e12
+            peak = pk.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+            roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                    "frac": ach / peak, "traffic": None, "peak_source": f"{pk_src} bf16 burst",
+                    "work_per_launch": work, "us_per_launch": us}
+        else:
+            ach = work / (us * 1e-6) / 1e9
+            peak = pk.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+            roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
+                    "frac": ach / peak, "traffic": None, "peak_source": f"{pk_src} HBM copy",
+                    "work_per_launch": work, "us_per_launch": us}
+
+    blk.close()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, threads, dt = oracle_displaced_rate(cfg)
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"2 full displaced layer steps of {cfg['name']} after 1 sync step ({dt:.1f} s)"}
+
+    if rank == 0:
+        ms_step = total_ms_max / args.steps
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": n_warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if dtype == "bf16" else "f32", "data": "synthetic",
+            "latent_px_per_s": value * L,
+            "tensor_tflops_per_step": wm["_total_flops"] / (ms_step * 1e-3) / 1e12,
+            "config": {"workload": cfg["name"], "H": cfg["H"], "W": cfg["W"], "C": cfg["C"],
+                       "n_patches": cfg["n_patches"], "heads": cfg["heads"], "parallelism": f"replicas{world}",
+                       "l2": "flushed between timed steps (512 MB write, outside the events)",
+                       "step": "displaced (is_sync=0)"},
+            "gpu_launches": launches * args.steps,
+            "launches_per_step": launches,
+            "kernels_us": {k: round(v, 2) for k, v in kern_us.items()},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "clocks": clocks,
+            "wall_s_timed_region": wall,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

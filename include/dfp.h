@@ -1,0 +1,173 @@
+/*
+ * dfp.h -- C ABI of the displaced-patch UNet layer step on one B200 (libdfp.so).
+ *
+ * The method (DistriFusion, CVPR 2024) splits the latent feature map into N row
+ * patches.  Each patch computes fresh activations for its own rows; the context
+ * it needs from the other patches is read from the previous denoising step:
+ *   - conv3x3 halo rows      (DistriConv2dPP; "DistriFusion源码探秘" source
+ *                             walkthrough, Patch Parallelism section, item 1)
+ *   - self-attention K/V     (DistriSelfAttentionPP; same section, item 2)
+ *   - GroupNorm statistics   (DistriGroupNorm; same section, item 3; the
+ *                             "corrected asynchronous" default of the
+ *                             --sync_mode flag, project README, Benchmarks)
+ * The first steps run synchronously (project README, Overview (c); paper
+ * reading blog, Implementation details).  Here all N patches run inside one
+ * GPU and a double-buffered device-resident cache replaces the all_gather of
+ * the multi-GPU original (walkthrough, forward-pass section; blog, Ablation).
+ *
+ * Conventions for every entry point
+ *   - Returns a dfp_status; never aborts, never exits.  On failure the handle's
+ *     dfp_last_error() text says why (a NULL handle gets a static message).
+ *   - Argument checks run on the host before any launch.
+ *   - Work is enqueued on the handle's CUDA stream; no call blocks on the device
+ *     except dfp_step_host, dfp_copy_out (host destination) and
+ *     dfp_check_device.
+ *   - Tensors are row-major.  The feature map is NHWC with batch 1: [H, W, C].
+ *     Tokens of attention are the pixels in row-major (h, w) order.
+ *   - Patch p (0 <= p < N) owns rows [p*H/N, (p+1)*H/N).
+ *   - One handle is not thread-safe; distinct handles are independent.
+ */
+#ifndef DFP_H
+#define DFP_H
+
+#if defined(__GNUC__)
+#define DFP_API __attribute__((visibility("default")))
+#else
+#define DFP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct dfp_ctx* dfp_handle;
+
+typedef enum {
+  DFP_OK = 0,
+  DFP_E_ARG = 1,          /* a bad pointer, size, name, dtype or shape            */
+  DFP_E_STATE = 2,        /* call out of order (e.g. displaced step, empty cache) */
+  DFP_E_CUDA = 3,         /* a CUDA runtime/driver call or a kernel launch failed */
+  DFP_E_NOMEM = 4,        /* device or host allocation failed                     */
+  DFP_E_UNSUPPORTED = 5,  /* valid request this build does not implement          */
+  DFP_E_DEVICE = 6        /* a kernel reported an error through the device flag   */
+} dfp_status;
+
+typedef enum { DFP_F32 = 0, DFP_BF16 = 1 } dfp_dtype;
+
+typedef enum {
+  DFP_BLOCK_RES_ATTN = 0,   /* GN+SiLU -> conv3x3 -> GN -> self-attention (Q,K,V,O) */
+  DFP_BLOCK_SDXL_STAGE = 1  /* ResNet block + transformer blocks (not built yet)     */
+} dfp_block;
+
+typedef enum {
+  /* est_p = mean_j m_j(t-1) + (m_p(t) - m_p(t-1)), m = (E[x], E[x^2]) per (patch, group) */
+  DFP_GN_CORRECTED = 0,
+  /* est_p = (m_p(t) + sum_{j != p} m_j(t-1)) / N */
+  DFP_GN_STALE_OTHERS = 1
+} dfp_gn_mode;
+
+typedef enum {
+  DFP_CTX_DISPLACED = 0,  /* the method: stale context on displaced steps          */
+  DFP_CTX_NAIVE = 1       /* naive-patch baseline: no cross-patch context at all
+                             (project README, Overview (b))                        */
+} dfp_context;
+
+typedef struct {
+  int H, W, C;          /* feature map; C = heads * head_dim                          */
+  int n_patches;        /* N: H % N == 0; (H/N)*W % 8 == 0                            */
+  int gn_groups;        /* G: C % G == 0                                               */
+  float gn_eps;         /* GroupNorm epsilon                                           */
+  int heads, head_dim;  /* head_dim must be 64                                         */
+  dfp_dtype dtype;      /* storage and MMA operand type; statistics/accumulation fp32 */
+  dfp_block block;
+  dfp_gn_mode gn_mode;
+  dfp_context context;
+  int n_xformer, ffn_inner, ctx_len, ctx_dim;  /* DFP_BLOCK_SDXL_STAGE only           */
+} dfp_config;
+
+typedef struct {
+  const char* name;          /* PyTorch module naming, e.g. "conv1.weight"            */
+  const void* ptr;           /* host or device pointer to the values, contiguous       */
+  int on_device;             /* 1 if ptr is a device pointer                           */
+  dfp_dtype dtype;           /* element type at ptr                                    */
+  int ndim;
+  const long long* shape;    /* PyTorch layout: conv [Cout,Cin,3,3], linear [out,in]   */
+} dfp_tensor;
+
+/* Create a handle for one layer (or stage) configuration and allocate its device
+ * buffers: the double-buffered context caches, intermediates and the output.
+ * cuda_stream: a cudaStream_t (NULL = legacy default stream); all work of this
+ * handle is enqueued on it.  *out receives the handle (NULL on failure).
+ * Errors: DFP_E_ARG for invalid sizes (see dfp_config), DFP_E_UNSUPPORTED for a
+ * block type not built, DFP_E_NOMEM / DFP_E_CUDA for allocation failures. */
+DFP_API dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out);
+
+/* Copy the weights in (host or device source; the library keeps its own re-laid
+ * copy, the caller's memory may be freed after the call returns).  Every weight
+ * of the block must be named exactly once across calls before the first step;
+ * names for DFP_BLOCK_RES_ATTN: gn1.weight gn1.bias conv1.weight conv1.bias
+ * gn2.weight gn2.bias attn.to_q.weight attn.to_k.weight attn.to_v.weight
+ * attn.to_out.weight attn.to_out.bias.  Blocks until the copies are done.
+ * Errors: DFP_E_ARG for an unknown name, wrong shape or dtype. */
+DFP_API dfp_status dfp_load_weights(dfp_handle h, const dfp_tensor* w, int n);
+
+/* One layer step.  x: caller-owned device pointer [H, W, C] of the config dtype,
+ * contiguous; it must stay valid until the stream work completes.
+ * step: 0 starts a new run and must be synchronous (is_sync = 1); otherwise
+ * step must equal the previous step + 1.  is_sync = 1 uses fresh context
+ * everywhere (exact full-image layer); is_sync = 0 uses the previous step's
+ * cached context for every cross-patch read.  Every step refreshes the caches.
+ * Asynchronous: returns once the kernels are enqueued.
+ * Errors: DFP_E_STATE (order, weights missing), DFP_E_ARG, DFP_E_CUDA. */
+DFP_API dfp_status dfp_step(dfp_handle h, const void* x, int step, int is_sync);
+
+/* Same step with HOST buffers: copies x_host ([H,W,C], config dtype; pinned
+ * memory gives asynchronous copies) to the device, runs the step, copies the
+ * output to y_host and waits for the stream. */
+DFP_API dfp_status dfp_step_host(dfp_handle h, const void* x_host, void* y_host, int step, int is_sync);
+
+/* Library-owned device pointer to the last step's output [H*W, C] (config dtype);
+ * valid until the next dfp_step or dfp_destroy. */
+DFP_API dfp_status dfp_output(dfp_handle h, const void** y);
+
+/* Copy an internal buffer of the last step to dst (device or host pointer,
+ * dst_bytes must equal the buffer size, see dfp_buffer_bytes).  Names:
+ * "y" output [L,C]; "slab" GN1+SiLU output with its halo rows [N,H/N+2,W,C];
+ * "h" conv output [H,W,C];
+ * "t" GN2 output [H,W,C]; "q","k","v" this step's projections [heads,L,64];
+ * "o" attention output [L,C]; "gn1","gn2" per-(patch,group) (mean, rstd) fp32
+ * [N,G,2].  Stream-ordered; a host dst makes the call wait for the stream. */
+DFP_API dfp_status dfp_copy_out(dfp_handle h, const char* name, void* dst, long long dst_bytes);
+DFP_API dfp_status dfp_buffer_bytes(dfp_handle h, const char* name, long long* bytes);
+
+/* Wait for the stream and read the device error flag that bounded waits inside
+ * the kernels set instead of hanging.  DFP_OK if clean, DFP_E_DEVICE (flag is
+ * cleared) otherwise, DFP_E_CUDA if a launch failed asynchronously. */
+DFP_API dfp_status dfp_check_device(dfp_handle h);
+
+/* Number of kernel launches one dfp_step of this handle enqueues. */
+DFP_API int dfp_launches_per_step(dfp_handle h);
+
+/* Choose the kernel family for the contractions: 0 = tcgen05/TMA tensor-core
+ * kernels (default for bf16), 1 = SIMT CUDA-core kernels (the only family for
+ * fp32).  Returns DFP_E_UNSUPPORTED for tensor cores with fp32. */
+DFP_API dfp_status dfp_set_kernel_family(dfp_handle h, int family);
+
+/* Per-kernel timing.  With profiling on, dfp_step brackets every kernel launch
+ * with CUDA events recorded on the handle's stream.  dfp_kernel_times waits for
+ * the last step's events and writes up to max_n durations (milliseconds) and the
+ * matching static kernel names; it returns the number of launches timed (0 when
+ * profiling is off or no step ran), or -1 on a CUDA error. */
+DFP_API dfp_status dfp_set_profiling(dfp_handle h, int enable);
+DFP_API int dfp_kernel_times(dfp_handle h, float* ms, const char** names, int max_n);
+
+/* Free everything the handle owns (waits for its stream first).  NULL is a no-op. */
+DFP_API dfp_status dfp_destroy(dfp_handle h);
+
+/* Text of the last error of h (or of the last failed dfp_create when h is NULL). */
+DFP_API const char* dfp_last_error(dfp_handle h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DFP_H */

@@ -1,0 +1,625 @@
+// libdfp host side: the C ABI of include/dfp.h, the handle with its device
+// buffers, weight re-layout, and the fixed launch sequence of one layer step.
+//
+// Device memory of a handle (row-major, batch 1):
+//   slab[2]     [N][R+2][W][C]   GN1+SiLU output with one halo row above/below each
+//                                patch; two buffers alternate by step parity, the other
+//                                one holds the previous step's map (stale context)
+//   h, t        [H*W][C]         conv output, GN2 output
+//   q           [heads][L][64]   this step's queries
+//   k[2], v[2]  [heads][L][64]   keys / values, alternating by step parity
+//   o, y        [L][C]           attention output, block output
+//   mom1/2[2]   [N][G][2] fp32   per-(patch, group) (E[x], E[x^2]) of GN1 / GN2, alternating
+//   coef        [N][C][2] fp32   per-(patch, channel) GroupNorm scale and shift
+//   part        fp32 scratch     per-chunk partial sums of the GroupNorm statistics
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <new>
+#include <set>
+#include <string>
+#include <vector>
+
+#include <cuda_bf16.h>
+
+#include "../../include/dfp.h"
+#include "kernels.h"
+
+using namespace dfp;
+
+namespace {
+
+thread_local std::string g_create_error;
+
+size_t dtype_size(dfp_dtype d) { return d == DFP_BF16 ? 2 : 4; }
+
+float bf16_bits_to_f32(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+uint16_t f32_to_bf16_bits(float f) {
+  // round to nearest even (the inputs handed in are finite)
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  const uint32_t rounding = 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)((u + rounding) >> 16);
+}
+
+}  // namespace
+
+struct dfp_ctx {
+  dfp_config cfg{};
+  cudaStream_t stream = nullptr;
+  std::string err;
+  int R = 0, L = 0, Lp = 0, family = 0;
+  size_t esz = 4;
+  // weights
+  void* w_conv = nullptr;   // [C][9][C]
+  float* b_conv = nullptr;
+  void* w_qkv = nullptr;    // [3C][C]
+  void* w_o = nullptr;      // [C][C]
+  float* b_o = nullptr;
+  float *gn1_g = nullptr, *gn1_b = nullptr, *gn2_g = nullptr, *gn2_b = nullptr;
+  std::set<std::string> loaded;
+  // activations and caches
+  void* slab[2] = {nullptr, nullptr};
+  void *h = nullptr, *t = nullptr, *q = nullptr, *o = nullptr, *y = nullptr, *xin = nullptr;
+  void* kb[2] = {nullptr, nullptr};
+  void* vb[2] = {nullptr, nullptr};
+  float *mom1[2] = {nullptr, nullptr}, *mom2[2] = {nullptr, nullptr};
+  float *coef = nullptr, *dbg1 = nullptr, *dbg2 = nullptr, *part = nullptr;
+  unsigned* counter = nullptr;
+  int* dev_err = nullptr;
+  std::vector<void*> allocs;
+  int last_step = -1;
+  int launches = 0;
+  // per-launch timing (dfp_set_profiling)
+  static constexpr int kMaxEv = 24;
+  bool profiling = false;
+  cudaEvent_t ev[kMaxEv] = {};
+  const char* ev_name[kMaxEv] = {};
+  int n_ev = 0;
+  // TMA descriptors (bf16 only)
+  CUtensorMap m_slab[2], m_wconv, m_t, m_wqkv, m_o, m_wo, m_q, m_k[2], m_v[2];
+  TcGemmPlan conv_plan{}, qkv_plan{}, out_plan{};
+
+  dfp_status fail(dfp_status s, const std::string& msg) {
+    err = msg;
+    return s;
+  }
+  dfp_status cuda_fail(cudaError_t e, const char* where) {
+    err = std::string(where) + ": " + cudaGetErrorString(e);
+    return DFP_E_CUDA;
+  }
+  bool alloc(void** p, size_t bytes) {
+    if (cudaMalloc(p, bytes) != cudaSuccess) { *p = nullptr; return false; }
+    allocs.push_back(*p);
+    return true;
+  }
+};
+
+namespace {
+
+dfp_status check_config(const dfp_config* c, std::string& why) {
+  auto bad = [&](const char* m) { why = m; return DFP_E_ARG; };
+  if (c->H <= 0 || c->W <= 0 || c->C <= 0 || c->n_patches <= 0) return bad("H, W, C, n_patches must be positive");
+  if (c->H % c->n_patches) return bad("H must be a multiple of n_patches");
+  if (c->gn_groups <= 0 || c->C % c->gn_groups) return bad("C must be a multiple of gn_groups");
+  if (c->n_patches * c->gn_groups > 256) return bad("n_patches * gn_groups must be <= 256");
+  if (c->head_dim != 64) return bad("head_dim must be 64");
+  if (c->heads * c->head_dim != c->C) return bad("heads * head_dim must equal C");
+  if (c->C % 64) return bad("C must be a multiple of 64");
+  if (c->C > 4096) return bad("C must be <= 4096");
+  if (c->dtype != DFP_F32 && c->dtype != DFP_BF16) return bad("unknown dtype");
+  if (c->gn_mode != DFP_GN_CORRECTED && c->gn_mode != DFP_GN_STALE_OTHERS) return bad("unknown gn_mode");
+  if (c->context != DFP_CTX_DISPLACED && c->context != DFP_CTX_NAIVE) return bad("unknown context");
+  if (!(c->gn_eps >= 0.f)) return bad("gn_eps must be >= 0");
+  const long long Lp = (long long)(c->H / c->n_patches) * c->W;
+  if (Lp % 8) return bad("(H / n_patches) * W must be a multiple of 8");
+  if ((long long)c->H * c->W * c->C > (1ll << 31)) return bad("feature map too large (H*W*C >= 2^31)");
+  if (c->block == DFP_BLOCK_SDXL_STAGE) { why = "the transformer stage block is not built yet"; return DFP_E_UNSUPPORTED; }
+  if (c->block != DFP_BLOCK_RES_ATTN) return bad("unknown block type");
+  return DFP_OK;
+}
+
+// Conv tile geometry of the implicit GEMM: 128 output pixels = rows_tile x cols_tile.
+void conv_tiles(int R, int W, int& cols_tile, int& rows_tile, int& tiles_per_row) {
+  cols_tile = W < 128 ? W : 128;
+  tiles_per_row = (W + cols_tile - 1) / cols_tile;
+  rows_tile = 128 / cols_tile;
+  if (rows_tile < 1) rows_tile = 1;
+  while (R % rows_tile) --rows_tile;
+}
+
+int pick_bn(int N) {
+  if (N % 128 == 0 && N / 128 >= 8) return 128;
+  if (N % 160 == 0) return 160;
+  if (N % 128 == 0) return 128;
+  return 64;
+}
+
+dfp_status build_tmaps(dfp_ctx* h) {
+  const dfp_config& c = h->cfg;
+  const int C = c.C, W = c.W, N = c.n_patches, R = h->R, L = h->L;
+  bool ok = true;
+  int cols_tile, rows_tile, tpr;
+  conv_tiles(R, W, cols_tile, rows_tile, tpr);
+  for (int i = 0; i < 2; ++i) {
+    const uint64_t dims[4] = {(uint64_t)C, (uint64_t)W, (uint64_t)(R + 2), (uint64_t)N};
+    const uint64_t str[3] = {(uint64_t)C * 2, (uint64_t)W * C * 2, (uint64_t)(R + 2) * W * C * 2};
+    const uint32_t box[4] = {64, (uint32_t)cols_tile, (uint32_t)rows_tile, 1};
+    ok &= encode_tmap_4d(&h->m_slab[i], h->slab[i], dims, str, box);
+  }
+  const int bn_conv = pick_bn(C), bn_qkv = pick_bn(3 * C), bn_out = pick_bn(C);
+  ok &= encode_tmap_2d(&h->m_wconv, h->w_conv, 9ull * C, C, 9ull * C * 2, 64, bn_conv);
+  ok &= encode_tmap_2d(&h->m_t, h->t, C, L, (uint64_t)C * 2, 64, 128);
+  ok &= encode_tmap_2d(&h->m_wqkv, h->w_qkv, C, 3ull * C, (uint64_t)C * 2, 64, bn_qkv);
+  ok &= encode_tmap_2d(&h->m_o, h->o, C, L, (uint64_t)C * 2, 64, 128);
+  ok &= encode_tmap_2d(&h->m_wo, h->w_o, C, C, (uint64_t)C * 2, 64, bn_out);
+  const int heads = c.heads;
+  ok &= encode_tmap_3d(&h->m_q, h->q, 64, L, heads, 128, (uint64_t)L * 128, 64, 128, 1);
+  for (int i = 0; i < 2; ++i) {
+    ok &= encode_tmap_3d(&h->m_k[i], h->kb[i], 64, L, heads, 128, (uint64_t)L * 128, 64, 128, 1);
+    ok &= encode_tmap_3d(&h->m_v[i], h->vb[i], 64, L, heads, 128, (uint64_t)L * 128, 64, 128, 1);
+  }
+  if (!ok) return h->fail(DFP_E_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+  TcGemmPlan& cp = h->conv_plan;
+  cp = TcGemmPlan{};
+  cp.M = L; cp.N = C; cp.K = 9 * C; cp.bn = bn_conv; cp.conv = 1;
+  cp.P = N; cp.R = R; cp.W = W; cp.Cin = C;
+  cp.cols_tile = cols_tile; cp.rows_tile = rows_tile; cp.tiles_per_row = tpr;
+  TcGemmPlan& qp = h->qkv_plan;
+  qp = TcGemmPlan{};
+  qp.M = L; qp.N = 3 * C; qp.K = C; qp.bn = bn_qkv;
+  TcGemmPlan& op = h->out_plan;
+  op = TcGemmPlan{};
+  op.M = L; op.N = C; op.K = C; op.bn = bn_out;
+  return DFP_OK;
+}
+
+// ------------------------------------------------------------------ weights
+struct WeightSpec {
+  const char* name;
+  std::vector<long long> shape;
+};
+
+std::vector<WeightSpec> weight_specs(const dfp_config& c) {
+  const long long C = c.C;
+  return {
+      {"gn1.weight", {C}}, {"gn1.bias", {C}}, {"conv1.weight", {C, C, 3, 3}}, {"conv1.bias", {C}},
+      {"gn2.weight", {C}}, {"gn2.bias", {C}}, {"attn.to_q.weight", {C, C}}, {"attn.to_k.weight", {C, C}},
+      {"attn.to_v.weight", {C, C}}, {"attn.to_out.weight", {C, C}}, {"attn.to_out.bias", {C}},
+  };
+}
+
+// Read n elements of the given dtype from host memory as float.
+void read_as_float(const void* src, dfp_dtype dt, size_t n, std::vector<float>& out) {
+  out.resize(n);
+  if (dt == DFP_F32) {
+    std::memcpy(out.data(), src, n * 4);
+  } else {
+    const uint16_t* s = static_cast<const uint16_t*>(src);
+    for (size_t i = 0; i < n; ++i) out[i] = bf16_bits_to_f32(s[i]);
+  }
+}
+
+// Convert float values to the storage dtype (host bytes).
+std::vector<uint8_t> to_storage(const std::vector<float>& v, dfp_dtype dt) {
+  std::vector<uint8_t> out(v.size() * dtype_size(dt));
+  if (dt == DFP_F32) {
+    std::memcpy(out.data(), v.data(), v.size() * 4);
+  } else {
+    uint16_t* d = reinterpret_cast<uint16_t*>(out.data());
+    for (size_t i = 0; i < v.size(); ++i) d[i] = f32_to_bf16_bits(v[i]);
+  }
+  return out;
+}
+
+template <typename T>
+dfp_status run_step(dfp_ctx* h, const void* x, int step, int is_sync);
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out) {
+  if (!out) { g_create_error = "out is NULL"; return DFP_E_ARG; }
+  *out = nullptr;
+  if (!cfg) { g_create_error = "cfg is NULL"; return DFP_E_ARG; }
+  std::string why;
+  dfp_status st = check_config(cfg, why);
+  if (st != DFP_OK) { g_create_error = why; return st; }
+  dfp_ctx* h = new (std::nothrow) dfp_ctx();
+  if (!h) { g_create_error = "host allocation failed"; return DFP_E_NOMEM; }
+  h->cfg = *cfg;
+  h->stream = static_cast<cudaStream_t>(cuda_stream);
+  h->R = cfg->H / cfg->n_patches;
+  h->L = cfg->H * cfg->W;
+  h->Lp = h->R * cfg->W;
+  h->esz = dtype_size(cfg->dtype);
+  h->family = cfg->dtype == DFP_BF16 ? 0 : 1;
+  const size_t C = cfg->C, N = cfg->n_patches, G = cfg->gn_groups, W = cfg->W, R = h->R, L = h->L;
+  const size_t map = L * C * h->esz;
+  bool ok = true;
+  ok &= h->alloc(&h->w_conv, 9 * C * C * h->esz);
+  ok &= h->alloc((void**)&h->b_conv, C * 4);
+  ok &= h->alloc(&h->w_qkv, 3 * C * C * h->esz);
+  ok &= h->alloc(&h->w_o, C * C * h->esz);
+  ok &= h->alloc((void**)&h->b_o, C * 4);
+  ok &= h->alloc((void**)&h->gn1_g, C * 4);
+  ok &= h->alloc((void**)&h->gn1_b, C * 4);
+  ok &= h->alloc((void**)&h->gn2_g, C * 4);
+  ok &= h->alloc((void**)&h->gn2_b, C * 4);
+  for (int i = 0; i < 2; ++i) {
+    ok &= h->alloc(&h->slab[i], N * (R + 2) * W * C * h->esz);
+    ok &= h->alloc(&h->kb[i], map);
+    ok &= h->alloc(&h->vb[i], map);
+    ok &= h->alloc((void**)&h->mom1[i], N * G * 2 * 4);
+    ok &= h->alloc((void**)&h->mom2[i], N * G * 2 * 4);
+  }
+  ok &= h->alloc(&h->h, map);
+  ok &= h->alloc(&h->t, map);
+  ok &= h->alloc(&h->q, map);
+  ok &= h->alloc(&h->o, map);
+  ok &= h->alloc(&h->y, map);
+  ok &= h->alloc(&h->xin, map);
+  ok &= h->alloc((void**)&h->coef, N * C * 2 * 4);
+  ok &= h->alloc((void**)&h->dbg1, N * G * 2 * 4);
+  ok &= h->alloc((void**)&h->dbg2, N * G * 2 * 4);
+  ok &= h->alloc((void**)&h->part, N * (size_t)gn_stats_chunks((int)N, (int)(R * W)) * G * 2 * 4);
+  ok &= h->alloc((void**)&h->counter, 64);
+  ok &= h->alloc((void**)&h->dev_err, 64);
+  if (!ok) {
+    g_create_error = "device allocation failed";
+    dfp_destroy(h);
+    return DFP_E_NOMEM;
+  }
+  // zero everything the kernels rely on: slab halo rows at the image edges, the
+  // GroupNorm block counter, the device error word, and all caches
+  cudaError_t e = cudaSuccess;
+  for (void* p : {h->slab[0], h->slab[1]})
+    if (e == cudaSuccess) e = cudaMemset(p, 0, N * (R + 2) * W * C * h->esz);
+  for (void* p : {h->kb[0], h->kb[1], h->vb[0], h->vb[1], h->h, h->t, h->q, h->o, h->y})
+    if (e == cudaSuccess) e = cudaMemset(p, 0, map);
+  if (e == cudaSuccess) e = cudaMemset(h->counter, 0, 64);
+  if (e == cudaSuccess) e = cudaMemset(h->dev_err, 0, 64);
+  if (e != cudaSuccess) {
+    g_create_error = std::string("cudaMemset: ") + cudaGetErrorString(e);
+    dfp_destroy(h);
+    return DFP_E_CUDA;
+  }
+  if (cfg->dtype == DFP_BF16) {
+    st = build_tmaps(h);
+    if (st != DFP_OK) {
+      g_create_error = h->err;
+      dfp_destroy(h);
+      return st;
+    }
+  }
+  *out = h;
+  return DFP_OK;
+}
+
+dfp_status dfp_load_weights(dfp_handle h, const dfp_tensor* w, int n) {
+  if (!h) return DFP_E_ARG;
+  if (n < 0 || (n > 0 && !w)) return h->fail(DFP_E_ARG, "bad weight list");
+  const dfp_config& c = h->cfg;
+  const std::vector<WeightSpec> specs = weight_specs(c);
+  for (int i = 0; i < n; ++i) {
+    const dfp_tensor& t = w[i];
+    if (!t.name || !t.ptr) return h->fail(DFP_E_ARG, "weight with NULL name or pointer");
+    const WeightSpec* spec = nullptr;
+    for (const auto& s : specs)
+      if (std::strcmp(s.name, t.name) == 0) spec = &s;
+    if (!spec) return h->fail(DFP_E_ARG, std::string("unknown weight name ") + t.name);
+    if (t.dtype != DFP_F32 && t.dtype != DFP_BF16) return h->fail(DFP_E_ARG, std::string("bad dtype for ") + t.name);
+    if (t.ndim != (int)spec->shape.size() || !t.shape)
+      return h->fail(DFP_E_ARG, std::string("wrong rank for ") + t.name);
+    size_t numel = 1;
+    for (int d = 0; d < t.ndim; ++d) {
+      if (t.shape[d] != spec->shape[d]) return h->fail(DFP_E_ARG, std::string("wrong shape for ") + t.name);
+      numel *= (size_t)t.shape[d];
+    }
+    // bring the values to the host as float
+    std::vector<uint8_t> staging;
+    const void* src = t.ptr;
+    if (t.on_device) {
+      staging.resize(numel * dtype_size(t.dtype));
+      cudaError_t e = cudaMemcpy(staging.data(), t.ptr, staging.size(), cudaMemcpyDeviceToHost);
+      if (e != cudaSuccess) return h->cuda_fail(e, "weight copy to host");
+      src = staging.data();
+    }
+    std::vector<float> v;
+    read_as_float(src, t.dtype, numel, v);
+    const std::string name = t.name;
+    const size_t C = c.C;
+    void* dst = nullptr;
+    std::vector<uint8_t> bytes;
+    size_t offset = 0;
+    if (name == "conv1.weight") {
+      // [Cout][Cin][3][3] -> [Cout][tap][Cin], tap = 3 r + s
+      std::vector<float> r(numel);
+      for (size_t co = 0; co < C; ++co)
+        for (size_t ci = 0; ci < C; ++ci)
+          for (int tap = 0; tap < 9; ++tap) r[(co * 9 + tap) * C + ci] = v[(co * C + ci) * 9 + tap];
+      bytes = to_storage(r, c.dtype);
+      dst = h->w_conv;
+    } else if (name == "attn.to_q.weight" || name == "attn.to_k.weight" || name == "attn.to_v.weight") {
+      const int which = name == "attn.to_q.weight" ? 0 : (name == "attn.to_k.weight" ? 1 : 2);
+      bytes = to_storage(v, c.dtype);
+      dst = h->w_qkv;
+      offset = (size_t)which * C * C * h->esz;
+    } else if (name == "attn.to_out.weight") {
+      bytes = to_storage(v, c.dtype);
+      dst = h->w_o;
+    } else {
+      // fp32 vectors
+      bytes.resize(numel * 4);
+      std::memcpy(bytes.data(), v.data(), numel * 4);
+      if (name == "conv1.bias") dst = h->b_conv;
+      else if (name == "attn.to_out.bias") dst = h->b_o;
+      else if (name == "gn1.weight") dst = h->gn1_g;
+      else if (name == "gn1.bias") dst = h->gn1_b;
+      else if (name == "gn2.weight") dst = h->gn2_g;
+      else if (name == "gn2.bias") dst = h->gn2_b;
+    }
+    cudaError_t e = cudaMemcpy(static_cast<uint8_t*>(dst) + offset, bytes.data(), bytes.size(),
+                               cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return h->cuda_fail(e, "weight copy to device");
+    h->loaded.insert(name);
+  }
+  return DFP_OK;
+}
+
+dfp_status dfp_step(dfp_handle h, const void* x, int step, int is_sync) {
+  if (!h) return DFP_E_ARG;
+  if (!x) return h->fail(DFP_E_ARG, "x is NULL");
+  if (is_sync != 0 && is_sync != 1) return h->fail(DFP_E_ARG, "is_sync must be 0 or 1");
+  if (step < 0) return h->fail(DFP_E_ARG, "step must be >= 0");
+  if (h->loaded.size() != weight_specs(h->cfg).size())
+    return h->fail(DFP_E_STATE, "weights not loaded (every weight must be given before the first step)");
+  if (step == 0 && !is_sync) return h->fail(DFP_E_STATE, "step 0 must be synchronous: the context cache is empty");
+  if (step != 0 && step != h->last_step + 1)
+    return h->fail(DFP_E_STATE, "steps must be consecutive (or restart at 0)");
+  dfp_status st = h->cfg.dtype == DFP_BF16 ? run_step<__nv_bfloat16>(h, x, step, is_sync)
+                                           : run_step<float>(h, x, step, is_sync);
+  if (st == DFP_OK) h->last_step = step;
+  return st;
+}
+
+dfp_status dfp_step_host(dfp_handle h, const void* x_host, void* y_host, int step, int is_sync) {
+  if (!h) return DFP_E_ARG;
+  if (!x_host || !y_host) return h->fail(DFP_E_ARG, "x_host / y_host is NULL");
+  const size_t bytes = (size_t)h->L * h->cfg.C * h->esz;
+  cudaError_t e = cudaMemcpyAsync(h->xin, x_host, bytes, cudaMemcpyHostToDevice, h->stream);
+  if (e != cudaSuccess) return h->cuda_fail(e, "input copy");
+  dfp_status st = dfp_step(h, h->xin, step, is_sync);
+  if (st != DFP_OK) return st;
+  e = cudaMemcpyAsync(y_host, h->y, bytes, cudaMemcpyDeviceToHost, h->stream);
+  if (e != cudaSuccess) return h->cuda_fail(e, "output copy");
+  e = cudaStreamSynchronize(h->stream);
+  if (e != cudaSuccess) return h->cuda_fail(e, "stream synchronize");
+  return DFP_OK;
+}
+
+dfp_status dfp_output(dfp_handle h, const void** y) {
+  if (!h) return DFP_E_ARG;
+  if (!y) return h->fail(DFP_E_ARG, "y is NULL");
+  *y = h->y;
+  return DFP_OK;
+}
+
+static bool buffer_of(dfp_handle h, const char* name, const void** ptr, long long* bytes) {
+  const long long map = (long long)h->L * h->cfg.C * (long long)h->esz;
+  const long long st = (long long)h->cfg.n_patches * h->cfg.gn_groups * 2 * 4;
+  const int cur = h->last_step < 0 ? 0 : (h->last_step & 1);
+  const std::string n = name;
+  if (n == "y") { *ptr = h->y; *bytes = map; }
+  else if (n == "h") { *ptr = h->h; *bytes = map; }
+  else if (n == "t") { *ptr = h->t; *bytes = map; }
+  else if (n == "o") { *ptr = h->o; *bytes = map; }
+  else if (n == "q") { *ptr = h->q; *bytes = map; }
+  else if (n == "k") { *ptr = h->kb[cur]; *bytes = map; }
+  else if (n == "v") { *ptr = h->vb[cur]; *bytes = map; }
+  else if (n == "gn1") { *ptr = h->dbg1; *bytes = st; }
+  else if (n == "gn2") { *ptr = h->dbg2; *bytes = st; }
+  else if (n == "slab") {
+    *ptr = h->slab[cur];
+    *bytes = (long long)h->cfg.n_patches * (h->R + 2) * h->cfg.W * h->cfg.C * (long long)h->esz;
+  } else return false;
+  return true;
+}
+
+dfp_status dfp_buffer_bytes(dfp_handle h, const char* name, long long* bytes) {
+  if (!h) return DFP_E_ARG;
+  if (!name || !bytes) return h->fail(DFP_E_ARG, "NULL argument");
+  const void* p;
+  if (!buffer_of(h, name, &p, bytes)) return h->fail(DFP_E_ARG, std::string("unknown buffer ") + name);
+  return DFP_OK;
+}
+
+dfp_status dfp_copy_out(dfp_handle h, const char* name, void* dst, long long dst_bytes) {
+  if (!h) return DFP_E_ARG;
+  if (!name || !dst) return h->fail(DFP_E_ARG, "NULL argument");
+  const void* p;
+  long long bytes;
+  if (!buffer_of(h, name, &p, &bytes)) return h->fail(DFP_E_ARG, std::string("unknown buffer ") + name);
+  if (dst_bytes != bytes) return h->fail(DFP_E_ARG, "dst_bytes does not match the buffer size");
+  cudaError_t e = cudaMemcpyAsync(dst, p, (size_t)bytes, cudaMemcpyDefault, h->stream);
+  if (e != cudaSuccess) return h->cuda_fail(e, "buffer copy");
+  cudaPointerAttributes attr{};
+  if (cudaPointerGetAttributes(&attr, dst) != cudaSuccess || attr.type != cudaMemoryTypeDevice) {
+    cudaGetLastError();
+    e = cudaStreamSynchronize(h->stream);
+    if (e != cudaSuccess) return h->cuda_fail(e, "stream synchronize");
+  }
+  return DFP_OK;
+}
+
+dfp_status dfp_check_device(dfp_handle h) {
+  if (!h) return DFP_E_ARG;
+  cudaError_t e = cudaStreamSynchronize(h->stream);
+  if (e != cudaSuccess) return h->cuda_fail(e, "stream synchronize");
+  int flag = 0;
+  e = cudaMemcpy(&flag, h->dev_err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return h->cuda_fail(e, "error flag read");
+  if (flag != 0) {
+    cudaMemset(h->dev_err, 0, sizeof(int));
+    return h->fail(DFP_E_DEVICE, "a kernel wait ran past its limit (device error code " + std::to_string(flag) + ")");
+  }
+  return DFP_OK;
+}
+
+int dfp_launches_per_step(dfp_handle h) { return h ? h->launches : -1; }
+
+dfp_status dfp_set_kernel_family(dfp_handle h, int family) {
+  if (!h) return DFP_E_ARG;
+  if (family != 0 && family != 1) return h->fail(DFP_E_ARG, "family must be 0 or 1");
+  if (family == 0 && h->cfg.dtype != DFP_BF16)
+    return h->fail(DFP_E_UNSUPPORTED, "tensor-core kernels need bf16 storage");
+  h->family = family;
+  return DFP_OK;
+}
+
+dfp_status dfp_set_profiling(dfp_handle h, int enable) {
+  if (!h) return DFP_E_ARG;
+  if (enable && !h->ev[0]) {
+    for (int i = 0; i < dfp_ctx::kMaxEv; ++i) {
+      cudaError_t e = cudaEventCreate(&h->ev[i]);
+      if (e != cudaSuccess) return h->cuda_fail(e, "event create");
+    }
+  }
+  h->profiling = enable != 0;
+  h->n_ev = 0;
+  return DFP_OK;
+}
+
+int dfp_kernel_times(dfp_handle h, float* ms, const char** names, int max_n) {
+  if (!h) return -1;
+  if (!h->profiling || h->n_ev < 2) return 0;
+  if (cudaEventSynchronize(h->ev[h->n_ev - 1]) != cudaSuccess) return -1;
+  const int n = h->n_ev - 1;
+  for (int i = 0; i < n && i < max_n; ++i) {
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, h->ev[i], h->ev[i + 1]) != cudaSuccess) return -1;
+    if (ms) ms[i] = t;
+    if (names) names[i] = h->ev_name[i];
+  }
+  return n;
+}
+
+dfp_status dfp_destroy(dfp_handle h) {
+  if (!h) return DFP_OK;
+  cudaStreamSynchronize(h->stream);
+  for (int i = 0; i < dfp_ctx::kMaxEv; ++i)
+    if (h->ev[i]) cudaEventDestroy(h->ev[i]);
+  for (void* p : h->allocs) cudaFree(p);
+  delete h;
+  return DFP_OK;
+}
+
+const char* dfp_last_error(dfp_handle h) {
+  if (!h) return g_create_error.c_str();
+  return h->err.c_str();
+}
+
+}  // extern "C"
+
+// ====================================================================== step scheduler
+namespace {
+
+template <typename T>
+dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
+  const dfp_config& c = h->cfg;
+  const int N = c.n_patches, C = c.C, G = c.gn_groups, W = c.W, R = h->R, L = h->L, Lp = h->Lp;
+  const int cur = step & 1, prv = cur ^ 1;
+  const bool naive = c.context == DFP_CTX_NAIVE;
+  const bool displaced = !is_sync && !naive;
+  cudaStream_t s = h->stream;
+  const T* x = static_cast<const T*>(xv);
+  T* slab = static_cast<T*>(h->slab[cur]);
+  int launches = 0;
+  cudaError_t e;
+  h->n_ev = 0;
+#define DFP_LAUNCH(call, what)                                   \
+  do {                                                           \
+    if (h->profiling && launches + 1 < dfp_ctx::kMaxEv) {        \
+      cudaEventRecord(h->ev[launches], s);                       \
+      h->ev_name[launches] = what;                               \
+    }                                                            \
+    e = (call);                                                  \
+    if (e != cudaSuccess) return h->cuda_fail(e, what);          \
+    ++launches;                                                  \
+  } while (0)
+
+  // ---- GN1 statistics (+ corrected merge) and apply + SiLU into the slab interior
+  GnArgs g{};
+  g.x = x; g.N = N; g.pix_per_patch = Lp; g.C = C; g.G = G; g.eps = c.gn_eps;
+  g.part = h->part; g.counter = h->counter;
+  g.fresh_out = h->mom1[cur]; g.stale = h->mom1[prv];
+  g.gamma = h->gn1_g; g.beta = h->gn1_b; g.coef = h->coef; g.dbg = h->dbg1;
+  g.is_sync = is_sync; g.mode = (int)c.gn_mode; g.naive = naive ? 1 : 0;
+  DFP_LAUNCH(launch_gn_stats_merge<T>(g, s), "gn1 statistics");
+  DFP_LAUNCH(launch_gn_apply<T>(x, slab, h->coef, N, Lp, C, (long long)(R + 2) * W, W, true, s), "gn1 apply");
+  // ---- halo rows: the neighbours' boundary rows, stale (other buffer) on displaced steps
+  if (!naive && N > 1) {
+    const T* src = static_cast<const T*>(displaced ? h->slab[prv] : h->slab[cur]);
+    DFP_LAUNCH(launch_halo_refresh<T>(src, slab, N, R, W, C, s), "halo refresh");
+  }
+  // ---- conv3x3 (+ bias) -> h
+  Epilogue ec{};
+  ec.kind = 0; ec.out = h->h; ec.bias = h->b_conv; ec.ldo = C;
+  if (h->family == 0) {
+    DFP_LAUNCH(launch_tc_gemm(h->conv_plan, h->m_slab[cur], h->m_wconv, ec, h->dev_err, s), "conv (tcgen05)");
+  } else {
+    ConvA cv{slab, N, R, W, C};
+    DFP_LAUNCH(launch_simt_gemm<T>(nullptr, &cv, static_cast<const T*>(h->w_conv), L, C, 9 * C, ec, s), "conv (simt)");
+  }
+  // ---- GN2 (no SiLU) -> t
+  g.x = h->h; g.fresh_out = h->mom2[cur]; g.stale = h->mom2[prv];
+  g.gamma = h->gn2_g; g.beta = h->gn2_b; g.dbg = h->dbg2;
+  DFP_LAUNCH(launch_gn_stats_merge<T>(g, s), "gn2 statistics");
+  DFP_LAUNCH(launch_gn_apply<T>(static_cast<const T*>(h->h), static_cast<T*>(h->t), h->coef, N, Lp, C,
+                                (long long)Lp, 0, false, s), "gn2 apply");
+  // ---- Q, K, V projections; K/V land in this step's cache buffers
+  Epilogue eq{};
+  eq.kind = 1; eq.q = h->q; eq.k = h->kb[cur]; eq.v = h->vb[cur]; eq.L = L; eq.C = C;
+  if (h->family == 0) {
+    DFP_LAUNCH(launch_tc_gemm(h->qkv_plan, h->m_t, h->m_wqkv, eq, h->dev_err, s), "qkv (tcgen05)");
+  } else {
+    DFP_LAUNCH(launch_simt_gemm<T>(static_cast<const T*>(h->t), nullptr, static_cast<const T*>(h->w_qkv), L, 3 * C, C, eq, s), "qkv (simt)");
+  }
+  // ---- displaced attention
+  const int mode = naive ? kAttnNaive : (is_sync ? kAttnSync : kAttnDisplaced);
+  if (h->family == 0) {
+    TcAttnArgs a{};
+    a.L = L; a.Lp = Lp; a.N = N; a.heads = c.heads; a.C = C; a.mode = mode; a.o = h->o; a.err = h->dev_err;
+    DFP_LAUNCH(launch_tc_attention(a, h->m_q, h->m_k[cur], h->m_v[cur], h->m_k[prv], h->m_v[prv], s), "attention (tcgen05)");
+  } else {
+    DFP_LAUNCH(launch_simt_attention<T>(static_cast<const T*>(h->q), static_cast<const T*>(h->kb[cur]),
+                                        static_cast<const T*>(h->vb[cur]), static_cast<const T*>(h->kb[prv]),
+                                        static_cast<const T*>(h->vb[prv]), static_cast<T*>(h->o), L, Lp, N,
+                                        c.heads, C, mode, s), "attention (simt)");
+  }
+  // ---- output projection (+ bias) -> y
+  Epilogue eo{};
+  eo.kind = 0; eo.out = h->y; eo.bias = h->b_o; eo.ldo = C;
+  if (h->family == 0) {
+    DFP_LAUNCH(launch_tc_gemm(h->out_plan, h->m_o, h->m_wo, eo, h->dev_err, s), "out projection (tcgen05)");
+  } else {
+    DFP_LAUNCH(launch_simt_gemm<T>(static_cast<const T*>(h->o), nullptr, static_cast<const T*>(h->w_o), L, C, C, eo, s), "out projection (simt)");
+  }
+#undef DFP_LAUNCH
+  if (h->profiling && launches < dfp_ctx::kMaxEv) {
+    cudaEventRecord(h->ev[launches], s);
+    h->n_ev = launches + 1;
+  }
+  h->launches = launches;
+  return DFP_OK;
+}
+
+}  // namespace

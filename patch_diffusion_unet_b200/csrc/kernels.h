@@ -1,0 +1,92 @@
+// Host-side launchers of libdfp's kernels (internal; not part of the C ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dfp {
+
+// Attention context mode of one launch.
+enum AttnMode : int { kAttnSync = 0, kAttnDisplaced = 1, kAttnNaive = 2 };
+
+// ---------------------------------------------------------------- GroupNorm
+struct GnArgs {
+  const void* x;          // [N * pix_per_patch, C] input map, patch-major rows
+  int N, pix_per_patch, C, G;
+  float eps;
+  float* part;            // scratch [N][n_chunks][G][2] partial (sum x, sum x^2)
+  unsigned* counter;      // scratch, one word, zero between launches
+  float* fresh_out;       // [N][G][2] this step's (E[x], E[x^2]) per (patch, group)
+  const float* stale;     // [N][G][2] moments of step t-1 (read on displaced steps)
+  const float* gamma;     // [C] fp32
+  const float* beta;      // [C] fp32
+  float* coef;            // [N][C][2] per (patch, channel) (scale, shift)
+  float* dbg;             // [N][G][2] (mean, rstd) used, for inspection
+  int is_sync, mode, naive;
+};
+int gn_stats_chunks(int N, int pix_per_patch);
+template <typename T> cudaError_t launch_gn_stats_merge(const GnArgs& a, cudaStream_t s);
+template <typename T>
+cudaError_t launch_gn_apply(const T* x, T* out, const float* coef, int N, int pix_per_patch, int C,
+                            long long out_patch_stride_pix, long long out_pix_off, bool silu,
+                            cudaStream_t s);
+template <typename T>
+cudaError_t launch_halo_refresh(const T* src_slab, T* dst_slab, int N, int R, int W, int C,
+                                cudaStream_t s);
+
+// ---------------------------------------------------------------- GEMM epilogues
+struct Epilogue {
+  int kind;               // 0: out[m, n] = acc + bias[n] (bias may be null); 1: Q/K/V scatter
+  void* out;              // kind 0: [M, ldo]
+  const float* bias;
+  int ldo;
+  void* q; void* k; void* v;  // kind 1: [heads][L][64] each; column n -> (n / C, head, d)
+  int L, C;
+};
+// A operand of the conv: the haloed per-patch slab [N][R+2][W][Cin]; row m of the
+// implicit GEMM is pixel m of the full map, column k = tap * Cin + ci.
+struct ConvA {
+  const void* slab;
+  int N, R, W, Cin;
+};
+
+// SIMT (CUDA-core) contractions: the fp32 path, and a cross-check for bf16.
+template <typename T>
+cudaError_t launch_simt_gemm(const T* A, const ConvA* conv, const T* B, int M, int N, int K,
+                             const Epilogue& epi, cudaStream_t s);
+template <typename T>
+cudaError_t launch_simt_attention(const T* q, const T* kf, const T* vf, const T* ks, const T* vs,
+                                  T* o, int L, int Lp, int N, int heads, int C, int mode,
+                                  cudaStream_t s);
+
+// ---------------------------------------------------------------- tensor-core path (bf16)
+// TMA descriptors are built once per buffer on the host.
+bool encode_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t outer_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+bool encode_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                    uint64_t s1_bytes, uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
+bool encode_tmap_4d(CUtensorMap* m, const void* base, const uint64_t dims[4],
+                    const uint64_t strides_bytes[3], const uint32_t box[4]);
+
+struct TcGemmPlan {
+  int M, N, K;            // GEMM sizes (conv: M = H*W, K = 9*Cin)
+  int bn;                 // N tile (64, 128, 160 or 256)
+  int conv;               // 1: A is the haloed slab (4-D map), 0: plain [M, K] (2-D map)
+  // conv geometry
+  int P, R, W, Cin;       // patches, rows per patch, width, input channels
+  int cols_tile, rows_tile, tiles_per_row;
+};
+cudaError_t launch_tc_gemm(const TcGemmPlan& plan, const CUtensorMap& mapA, const CUtensorMap& mapB,
+                           const Epilogue& epi, int* err, cudaStream_t s);
+
+struct TcAttnArgs {
+  int L, Lp, N, heads, C, mode;
+  void* o;                // [L, C] bf16
+  int* err;
+};
+// maps: q [heads][L][64]; k/v fresh and stale, same shape (box 128 rows x 64)
+cudaError_t launch_tc_attention(const TcAttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mkf,
+                                const CUtensorMap& mvf, const CUtensorMap& mks,
+                                const CUtensorMap& mvs, cudaStream_t s);
+
+}  // namespace dfp
