@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--profile-steps", type=int, default=10)
+    ap.add_argument("--min-warmup-s", type=float, default=1.5,
+                    help="keep warming up until this much wall time has passed (clocks settle)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -70,8 +72,7 @@ def work_model(cfg):
     R = H // N
     return {
         "gn1 statistics": ("hbm", L * C * e),
-        "gn1 apply": ("hbm", 2 * L * C * e),
-        "halo refresh": ("hbm", 2 * 2 * (N - 1) * W * C * e),
+        "gn1 apply + halo": ("hbm", 2 * L * C * e + 2 * 2 * (N - 1) * W * C * e),
         "conv (tcgen05)": ("tensor", 2.0 * L * C * 9 * C),
         "gn2 statistics": ("hbm", L * C * e),
         "gn2 apply": ("hbm", 2 * L * C * e),
@@ -242,7 +243,7 @@ def main():
     sampler = ClockSampler(gpu_index)
     w_start = time.perf_counter()
     n_warm = 0
-    while n_warm < args.warmup or time.perf_counter() - w_start < 1.5:
+    while n_warm < args.warmup or time.perf_counter() - w_start < args.min_warmup_s:
         t += 1
         blk.step(x_of(t), t, 0)
         flush.zero_()

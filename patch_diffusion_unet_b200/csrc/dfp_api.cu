@@ -73,6 +73,10 @@ struct dfp_ctx {
   float *coef = nullptr, *dbg1 = nullptr, *dbg2 = nullptr, *part = nullptr;
   unsigned* counter = nullptr;
   int* dev_err = nullptr;
+  // split-KV attention scratch
+  int attn_splits = 1;
+  float *attn_part_o = nullptr, *attn_part_ml = nullptr;
+  unsigned* attn_counters = nullptr;
   std::vector<void*> allocs;
   int last_step = -1;
   int launches = 0;
@@ -273,6 +277,17 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
   ok &= h->alloc((void**)&h->part, N * (size_t)gn_stats_chunks((int)N, (int)(R * W)) * G * 2 * 4);
   ok &= h->alloc((void**)&h->counter, 64);
   ok &= h->alloc((void**)&h->dev_err, 64);
+  const int n_qt = (h->Lp + 127) / 128;
+  const size_t pairs = (size_t)((n_qt + 1) / 2) * N * cfg->heads;
+  if (cfg->dtype == DFP_BF16) {
+    const int min_tiles = cfg->context == DFP_CTX_NAIVE ? n_qt : (h->L + 127) / 128;
+    h->attn_splits = attention_splits(h->L, h->Lp, (int)N, cfg->heads, min_tiles);
+    if (h->attn_splits > 1) {
+      ok &= h->alloc((void**)&h->attn_part_o, pairs * h->attn_splits * 256 * 64 * 4);
+      ok &= h->alloc((void**)&h->attn_part_ml, pairs * h->attn_splits * 256 * 2 * 4);
+    }
+    ok &= h->alloc((void**)&h->attn_counters, pairs * 4 + 64);
+  }
   if (!ok) {
     g_create_error = "device allocation failed";
     dfp_destroy(h);
@@ -287,6 +302,7 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
     if (e == cudaSuccess) e = cudaMemset(p, 0, map);
   if (e == cudaSuccess) e = cudaMemset(h->counter, 0, 64);
   if (e == cudaSuccess) e = cudaMemset(h->dev_err, 0, 64);
+  if (e == cudaSuccess && h->attn_counters) e = cudaMemset(h->attn_counters, 0, pairs * 4 + 64);
   if (e != cudaSuccess) {
     g_create_error = std::string("cudaMemset: ") + cudaGetErrorString(e);
     dfp_destroy(h);
@@ -564,12 +580,11 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   g.gamma = h->gn1_g; g.beta = h->gn1_b; g.coef = h->coef; g.dbg = h->dbg1;
   g.is_sync = is_sync; g.mode = (int)c.gn_mode; g.naive = naive ? 1 : 0;
   DFP_LAUNCH(launch_gn_stats_merge<T>(g, s), "gn1 statistics");
-  DFP_LAUNCH(launch_gn_apply<T>(x, slab, h->coef, N, Lp, C, (long long)(R + 2) * W, W, true, s), "gn1 apply");
-  // ---- halo rows: the neighbours' boundary rows, stale (other buffer) on displaced steps
-  if (!naive && N > 1) {
-    const T* src = static_cast<const T*>(displaced ? h->slab[prv] : h->slab[cur]);
-    DFP_LAUNCH(launch_halo_refresh<T>(src, slab, N, R, W, C, s), "halo refresh");
-  }
+  // the same kernel fills the halo rows: the neighbours' boundary rows of this step
+  // (sync) or of the previous step (displaced, read from the other slab buffer)
+  const int halo_mode = (naive || N == 1) ? 0 : (displaced ? 2 : 1);
+  DFP_LAUNCH(launch_gn_apply<T>(x, slab, static_cast<const T*>(h->slab[prv]), h->coef, N, Lp, C, W,
+                                (long long)(R + 2) * W, W, true, halo_mode, s), "gn1 apply + halo");
   // ---- conv3x3 (+ bias) -> h
   Epilogue ec{};
   ec.kind = 0; ec.out = h->h; ec.bias = h->b_conv; ec.ldo = C;
@@ -583,8 +598,8 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   g.x = h->h; g.fresh_out = h->mom2[cur]; g.stale = h->mom2[prv];
   g.gamma = h->gn2_g; g.beta = h->gn2_b; g.dbg = h->dbg2;
   DFP_LAUNCH(launch_gn_stats_merge<T>(g, s), "gn2 statistics");
-  DFP_LAUNCH(launch_gn_apply<T>(static_cast<const T*>(h->h), static_cast<T*>(h->t), h->coef, N, Lp, C,
-                                (long long)Lp, 0, false, s), "gn2 apply");
+  DFP_LAUNCH(launch_gn_apply<T>(static_cast<const T*>(h->h), static_cast<T*>(h->t), nullptr, h->coef, N, Lp,
+                                C, W, (long long)Lp, 0, false, 0, s), "gn2 apply");
   // ---- Q, K, V projections; K/V land in this step's cache buffers
   Epilogue eq{};
   eq.kind = 1; eq.q = h->q; eq.k = h->kb[cur]; eq.v = h->vb[cur]; eq.L = L; eq.C = C;
@@ -598,6 +613,8 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   if (h->family == 0) {
     TcAttnArgs a{};
     a.L = L; a.Lp = Lp; a.N = N; a.heads = c.heads; a.C = C; a.mode = mode; a.o = h->o; a.err = h->dev_err;
+    a.splits = h->attn_splits; a.n_qtiles = (Lp + 127) / 128;
+    a.part_o = h->attn_part_o; a.part_ml = h->attn_part_ml; a.counters = h->attn_counters;
     DFP_LAUNCH(launch_tc_attention(a, h->m_q, h->m_k[cur], h->m_v[cur], h->m_k[prv], h->m_v[prv], s), "attention (tcgen05)");
   } else {
     DFP_LAUNCH(launch_simt_attention<T>(static_cast<const T*>(h->q), static_cast<const T*>(h->kb[cur]),

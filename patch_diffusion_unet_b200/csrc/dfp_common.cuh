@@ -22,9 +22,9 @@ enum DeviceError : int {
   kErrWaitAttnO = 6,       // softmax waited too long for P V
 };
 
-// Limit of every spin-wait, in nanoseconds of %globaltimer (a correct kernel
-// waits microseconds at most).
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Limit of every spin-wait, in SM clock cycles (about 2 s at the B200's maximum
+// clock; a correct kernel waits microseconds at most).
+constexpr long long kWaitLimitCycles = 4000000000ll;
 
 // ---------------------------------------------------------------- vectors
 template <typename T> struct VecTraits;
@@ -106,13 +106,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, records `code` in *err and returns false.
+// kWaitLimitCycles (the cycle counter is read once per 64 polls), records `code`
+// in *err and returns false.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err, int code) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const long long t0 = clock64();
+#pragma unroll 1
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (clock64() - t0 > kWaitLimitCycles) {
       atomicCAS(err, 0, code);
       return false;
     }

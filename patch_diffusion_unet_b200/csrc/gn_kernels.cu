@@ -22,22 +22,29 @@ namespace {
 
 constexpr int kGnThreads = 512;
 
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kGnThreads)
 gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
   constexpr int VEC = VecTraits<T>::kN;
-  extern __shared__ float sh[];                 // [2][PL][C] per-thread-row channel sums
+  extern __shared__ float sh[];                 // [2][PL][C] lane sums, then [2][C] channel sums
   __shared__ float s_mom[256 * 2];              // merged fresh moments  [N*G][2]
   __shared__ float s_mr[256 * 2];               // (mean, rstd)          [N*G][2]
   __shared__ int s_last;
   const int C = a.C, G = a.G, N = a.N;
   const int V = C / VEC;
   const int PL = kGnThreads / V;                // pixel lanes
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int vc = tid % V, pl = tid / V;
   const int p = blockIdx.y, chunk = blockIdx.x;
+  float* chan = sh + 2 * PL * C;
 
-  // ---- phase 1: per-channel partial sums of this chunk of patch p
+  // ---- phase 1: per-channel partial sums of this chunk of patch p (8 loads in flight)
   float s1[VEC], s2[VEC];
 #pragma unroll
   for (int i = 0; i < VEC; ++i) s1[i] = s2[i] = 0.f;
@@ -46,12 +53,12 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
     const int pix1 = min(pix0 + pix_per_chunk, a.pix_per_patch);
     const T* base = static_cast<const T*>(a.x) + (size_t)p * a.pix_per_patch * C + vc * VEC;
     int pix = pix0 + pl;
-    for (; pix + 3 * PL < pix1; pix += 4 * PL) {
-      uint4 u[4];
+    for (; pix + 7 * PL < pix1; pix += 8 * PL) {
+      uint4 u[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) u[j] = ld_nc16(base + (size_t)(pix + j * PL) * C);
+      for (int j = 0; j < 8; ++j) u[j] = ld_nc16(base + (size_t)(pix + j * PL) * C);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 8; ++j) {
         float v[VEC];
         unpack16(u[j], v);
 #pragma unroll
@@ -64,20 +71,30 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
 #pragma unroll
       for (int i = 0; i < VEC; ++i) { s1[i] += v[i]; s2[i] = fmaf(v[i], v[i], s2[i]); }
     }
+    float4* d1 = reinterpret_cast<float4*>(sh + pl * C + vc * VEC);
+    float4* d2 = reinterpret_cast<float4*>(sh + PL * C + pl * C + vc * VEC);
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) {
-      sh[pl * C + vc * VEC + i] = s1[i];
-      sh[PL * C + pl * C + vc * VEC + i] = s2[i];
+    for (int i = 0; i < VEC / 4; ++i) {
+      d1[i] = make_float4(s1[4 * i], s1[4 * i + 1], s1[4 * i + 2], s1[4 * i + 3]);
+      d2[i] = make_float4(s2[4 * i], s2[4 * i + 1], s2[4 * i + 2], s2[4 * i + 3]);
     }
   }
   __syncthreads();
-  const int cg = C / G;
-  for (int g = tid; g < G; g += kGnThreads) {
+  for (int c = tid; c < C; c += kGnThreads) {
     float t1 = 0.f, t2 = 0.f;
-    for (int c = g * cg; c < (g + 1) * cg; ++c)
-      for (int l = 0; l < PL; ++l) { t1 += sh[l * C + c]; t2 += sh[PL * C + l * C + c]; }
-    float2* dst = reinterpret_cast<float2*>(a.part) + ((size_t)p * n_chunks + chunk) * G + g;
-    *dst = make_float2(t1, t2);
+    for (int l = 0; l < PL; ++l) { t1 += sh[l * C + c]; t2 += sh[PL * C + l * C + c]; }
+    chan[c] = t1;
+    chan[C + c] = t2;
+  }
+  __syncthreads();
+  const int cg = C / G;
+  for (int g = warp; g < G; g += kGnThreads / 32) {
+    float t1 = 0.f, t2 = 0.f;
+    for (int c = lane; c < cg; c += 32) { t1 += chan[g * cg + c]; t2 += chan[C + g * cg + c]; }
+    t1 = warp_sum(t1);
+    t2 = warp_sum(t2);
+    if (lane == 0)
+      reinterpret_cast<float2*>(a.part)[((size_t)p * n_chunks + chunk) * G + g] = make_float2(t1, t2);
   }
 
   // ---- phase 2: the last block to finish merges every partial in a fixed order
@@ -89,19 +106,25 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
   __threadfence();
 
   const int NG = N * G;                         // <= 256 (checked on the host)
-  const int S = kGnThreads / NG;                // threads per (patch, group)
-  float* red = sh;                              // [S][NG][2] reuse
+  const int S = kGnThreads / NG;                // threads per (patch, group), >= 2
+  float* red = sh;                              // [S][NG][2]
   if (tid < S * NG) {
     const int item = tid % NG, part_id = tid / NG;
     const int pp = item / G, gg = item % G;
     const float2* src = reinterpret_cast<const float2*>(a.part) + (size_t)pp * n_chunks * G + gg;
-    float t1 = 0.f, t2 = 0.f;
-    for (int c = part_id; c < n_chunks; c += S) {
-      const float2 v = __ldcg(src + (size_t)c * G);
-      t1 += v.x; t2 += v.y;
+    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    for (int c = part_id; c < n_chunks; c += 4 * S) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int cc = c + u * S;
+        if (cc < n_chunks) {
+          const float2 v = __ldcg(src + (size_t)cc * G);
+          acc[u].x += v.x; acc[u].y += v.y;
+        }
+      }
     }
-    red[(part_id * NG + item) * 2 + 0] = t1;
-    red[(part_id * NG + item) * 2 + 1] = t2;
+    red[(part_id * NG + item) * 2 + 0] = (acc[0].x + acc[1].x) + (acc[2].x + acc[3].x);
+    red[(part_id * NG + item) * 2 + 1] = (acc[0].y + acc[1].y) + (acc[2].y + acc[3].y);
   }
   __syncthreads();
   const float inv_n = 1.f / ((float)a.pix_per_patch * (float)cg);
@@ -154,11 +177,32 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
 
 __device__ __forceinline__ float silu_f(float y) { return y / (1.f + expf(-y)); }
 
+// Normalise (+SiLU) one chunk of patch p.  With halo_mode != 0 the output is the
+// haloed slab and the kernel also fills the neighbours' halo rows: a patch's
+// first row goes to the bottom halo of patch p-1, its last row to the top halo
+// of patch p+1 -- this step's values on sync steps (halo_mode 1), the previous
+// step's values of the same rows, read from prev_slab, on displaced steps
+// (halo_mode 2).  Halo rows at the image top and bottom stay zero.
+template <typename T>
+__device__ __forceinline__ void write_halos(T* out, const T* prev_slab, const uint4& o, int p, int q,
+                                            int pix_per_patch, int last_row0, int W, int C, int c0,
+                                            long long stride, long long off, bool top_src, bool bot_src,
+                                            int halo_mode) {
+  const bool first = top_src && q < W;
+  const bool last = bot_src && q >= last_row0;
+  if (!first && !last) return;
+  const uint4 hv = halo_mode == 1 ? o : ld_nc16(prev_slab + ((size_t)p * stride + off + q) * C + c0);
+  if (first)   // bottom halo row (slab row R+1) of patch p-1
+    *reinterpret_cast<uint4*>(out + ((size_t)(p - 1) * stride + off + pix_per_patch + q) * C + c0) = hv;
+  if (last)    // top halo row (slab row 0) of patch p+1
+    *reinterpret_cast<uint4*>(out + ((size_t)(p + 1) * stride + (q - last_row0)) * C + c0) = hv;
+}
+
 template <typename T, bool SILU>
 __global__ void __launch_bounds__(kGnThreads)
-gn_apply_kernel(const T* __restrict__ x, T* __restrict__ out, const float* __restrict__ coef,
-                int pix_per_patch, int C, long long out_patch_stride, long long out_off,
-                int pix_per_chunk) {
+gn_apply_kernel(const T* __restrict__ x, T* __restrict__ out, const T* __restrict__ prev_slab,
+                const float* __restrict__ coef, int pix_per_patch, int C, long long out_patch_stride,
+                long long out_off, int pix_per_chunk, int W, int N, int halo_mode) {
   constexpr int VEC = VecTraits<T>::kN;
   const int V = C / VEC;
   const int PL = kGnThreads / V;
@@ -173,21 +217,29 @@ gn_apply_kernel(const T* __restrict__ x, T* __restrict__ out, const float* __res
   const int pix1 = min(pix0 + pix_per_chunk, pix_per_patch);
   const T* src = x + (size_t)p * pix_per_patch * C + vc * VEC;
   T* dst = out + ((size_t)p * out_patch_stride + out_off) * C + vc * VEC;
+  const int last_row0 = pix_per_patch - W;
+  const bool top_src = halo_mode != 0 && p > 0;          // my first row feeds patch p-1
+  const bool bot_src = halo_mode != 0 && p < N - 1;      // my last row feeds patch p+1
   int pix = pix0 + pl;
-  for (; pix + PL < pix1; pix += 2 * PL) {
-    uint4 u0 = ld_nc16(src + (size_t)pix * C);
-    uint4 u1 = ld_nc16(src + (size_t)(pix + PL) * C);
-    float v0[VEC], v1[VEC];
-    unpack16(u0, v0);
-    unpack16(u1, v1);
+  for (; pix + 3 * PL < pix1; pix += 4 * PL) {
+    uint4 u[4];
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) {
-      v0[i] = fmaf(v0[i], sc[i], sf[i]);
-      v1[i] = fmaf(v1[i], sc[i], sf[i]);
-      if (SILU) { v0[i] = silu_f(v0[i]); v1[i] = silu_f(v1[i]); }
+    for (int j = 0; j < 4; ++j) u[j] = ld_nc16(src + (size_t)(pix + j * PL) * C);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float v[VEC];
+      unpack16(u[j], v);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) {
+        v[i] = fmaf(v[i], sc[i], sf[i]);
+        if (SILU) v[i] = silu_f(v[i]);
+      }
+      const uint4 o = pack16(v);
+      const int q = pix + j * PL;
+      *reinterpret_cast<uint4*>(dst + (size_t)q * C) = o;
+      if (halo_mode != 0) write_halos(out, prev_slab, o, p, q, pix_per_patch, last_row0, W, C, vc * VEC,
+                                      out_patch_stride, out_off, top_src, bot_src, halo_mode);
     }
-    *reinterpret_cast<uint4*>(dst + (size_t)pix * C) = pack16(v0);
-    *reinterpret_cast<uint4*>(dst + (size_t)(pix + PL) * C) = pack16(v1);
   }
   for (; pix < pix1; pix += PL) {
     float v[VEC];
@@ -197,7 +249,10 @@ gn_apply_kernel(const T* __restrict__ x, T* __restrict__ out, const float* __res
       v[i] = fmaf(v[i], sc[i], sf[i]);
       if (SILU) v[i] = silu_f(v[i]);
     }
-    *reinterpret_cast<uint4*>(dst + (size_t)pix * C) = pack16(v);
+    const uint4 o = pack16(v);
+    *reinterpret_cast<uint4*>(dst + (size_t)pix * C) = o;
+    if (halo_mode != 0) write_halos(out, prev_slab, o, p, pix, pix_per_patch, last_row0, W, C, vc * VEC,
+                                    out_patch_stride, out_off, top_src, bot_src, halo_mode);
   }
 }
 
@@ -216,9 +271,9 @@ __global__ void halo_refresh_kernel(const T* __restrict__ src, T* __restrict__ d
     reinterpret_cast<uint4*>(d)[i] = ld_nc16(reinterpret_cast<const uint4*>(s) + i);
 }
 
+// Pixels per block: one wave of 512-thread blocks over the whole map.
 int chunk_pixels(int N, int pix_per_patch) {
-  // about two resident 512-thread blocks per SM over the whole map
-  const int target_blocks = 296;
+  const int target_blocks = 148;
   int per = (N * pix_per_patch + target_blocks - 1) / target_blocks;
   if (per < 16) per = 16;
   return per;
@@ -238,7 +293,7 @@ cudaError_t launch_gn_stats_merge(const GnArgs& a, cudaStream_t s) {
   const int n_chunks = (a.pix_per_patch + per - 1) / per;
   const int V = a.C / VEC;
   const int PL = kGnThreads / V;
-  size_t smem = (size_t)2 * PL * a.C * sizeof(float);
+  size_t smem = (size_t)(2 * PL + 2) * a.C * sizeof(float);
   const size_t red = (size_t)kGnThreads * 2 * sizeof(float);
   if (smem < red) smem = red;
   dim3 grid(n_chunks, a.N);
@@ -247,17 +302,19 @@ cudaError_t launch_gn_stats_merge(const GnArgs& a, cudaStream_t s) {
 }
 
 template <typename T>
-cudaError_t launch_gn_apply(const T* x, T* out, const float* coef, int N, int pix_per_patch, int C,
-                            long long out_patch_stride_pix, long long out_pix_off, bool silu,
-                            cudaStream_t s) {
+cudaError_t launch_gn_apply(const T* x, T* out, const T* prev_slab, const float* coef, int N,
+                            int pix_per_patch, int C, int W, long long out_patch_stride_pix,
+                            long long out_pix_off, bool silu, int halo_mode, cudaStream_t s) {
   const int per = chunk_pixels(N, pix_per_patch);
   dim3 grid((pix_per_patch + per - 1) / per, N);
   if (silu)
-    gn_apply_kernel<T, true><<<grid, kGnThreads, 0, s>>>(x, out, coef, pix_per_patch, C,
-                                                         out_patch_stride_pix, out_pix_off, per);
+    gn_apply_kernel<T, true><<<grid, kGnThreads, 0, s>>>(x, out, prev_slab, coef, pix_per_patch, C,
+                                                         out_patch_stride_pix, out_pix_off, per, W, N,
+                                                         halo_mode);
   else
-    gn_apply_kernel<T, false><<<grid, kGnThreads, 0, s>>>(x, out, coef, pix_per_patch, C,
-                                                          out_patch_stride_pix, out_pix_off, per);
+    gn_apply_kernel<T, false><<<grid, kGnThreads, 0, s>>>(x, out, prev_slab, coef, pix_per_patch, C,
+                                                          out_patch_stride_pix, out_pix_off, per, W, N,
+                                                          halo_mode);
   return cudaGetLastError();
 }
 
@@ -277,11 +334,13 @@ cudaError_t launch_halo_refresh(const T* src_slab, T* dst_slab, int N, int R, in
 
 template cudaError_t launch_gn_stats_merge<float>(const GnArgs&, cudaStream_t);
 template cudaError_t launch_gn_stats_merge<__nv_bfloat16>(const GnArgs&, cudaStream_t);
-template cudaError_t launch_gn_apply<float>(const float*, float*, const float*, int, int, int,
-                                            long long, long long, bool, cudaStream_t);
+template cudaError_t launch_gn_apply<float>(const float*, float*, const float*, const float*, int,
+                                            int, int, int, long long, long long, bool, int,
+                                            cudaStream_t);
 template cudaError_t launch_gn_apply<__nv_bfloat16>(const __nv_bfloat16*, __nv_bfloat16*,
-                                                    const float*, int, int, int, long long,
-                                                    long long, bool, cudaStream_t);
+                                                    const __nv_bfloat16*, const float*, int, int,
+                                                    int, int, long long, long long, bool, int,
+                                                    cudaStream_t);
 template cudaError_t launch_halo_refresh<float>(const float*, float*, int, int, int, int,
                                                 cudaStream_t);
 template cudaError_t launch_halo_refresh<__nv_bfloat16>(const __nv_bfloat16*, __nv_bfloat16*, int,

@@ -26,10 +26,12 @@ struct GnArgs {
 };
 int gn_stats_chunks(int N, int pix_per_patch);
 template <typename T> cudaError_t launch_gn_stats_merge(const GnArgs& a, cudaStream_t s);
+// halo_mode: 0 none (plain output), 1 sync (fresh neighbour rows), 2 displaced
+// (the previous step's rows, read from prev_slab)
 template <typename T>
-cudaError_t launch_gn_apply(const T* x, T* out, const float* coef, int N, int pix_per_patch, int C,
-                            long long out_patch_stride_pix, long long out_pix_off, bool silu,
-                            cudaStream_t s);
+cudaError_t launch_gn_apply(const T* x, T* out, const T* prev_slab, const float* coef, int N,
+                            int pix_per_patch, int C, int W, long long out_patch_stride_pix,
+                            long long out_pix_off, bool silu, int halo_mode, cudaStream_t s);
 template <typename T>
 cudaError_t launch_halo_refresh(const T* src_slab, T* dst_slab, int N, int R, int W, int C,
                                 cudaStream_t s);
@@ -83,7 +85,15 @@ struct TcAttnArgs {
   int L, Lp, N, heads, C, mode;
   void* o;                // [L, C] bf16
   int* err;
+  int splits;             // CTAs sharing the KV tile list of one Q-tile pair
+  int n_qtiles;           // ceil(Lp / 128)
+  float* part_o;          // scratch [pairs][splits][256][64] (splits > 1)
+  float* part_ml;         // scratch [pairs][splits][256][2]  (running max, row sum)
+  unsigned* counters;     // scratch [pairs], zero between launches
 };
+// Split count for the KV loop: enough CTAs to fill the GPU (148 SMs) in whole waves,
+// keeping at least 2 KV tiles per split.  min_tiles = fewest KV tiles of any mode used.
+int attention_splits(int L, int Lp, int N, int heads, int min_tiles);
 // maps: q [heads][L][64]; k/v fresh and stale, same shape (box 128 rows x 64)
 cudaError_t launch_tc_attention(const TcAttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mkf,
                                 const CUtensorMap& mvf, const CUtensorMap& mks,

@@ -1,5 +1,5 @@
 // Displaced self-attention on tcgen05 / TMEM / TMA (sm_100a), bf16 operands, fp32
-// softmax and accumulation, head width 64.
+// softmax statistics and accumulation, head width 64.
 //
 // DistriSelfAttentionPP ("DistriFusion源码探秘" source walkthrough, Patch
 // Parallelism section item 2): the queries of patch p attend to all L tokens; the
@@ -9,15 +9,33 @@
 //   sync       [0, L) fresh
 //   displaced  own patch fresh, then [0, p*Lp) stale, then [(p+1)*Lp, L) stale
 //   naive      own patch fresh only (the naive-patch baseline, README Overview (b))
-// Segment boundaries need not be multiples of the 128-key tile: columns past a
-// segment's end are masked to -inf.
+// Segment ends need not be multiples of the 128-key tile: columns past a
+// segment's end are masked.
 //
-// One CTA = one (128-query tile, head).  Warp 0: TMA (Q once, K/V two-stage
-// rings), warp 1: one thread issues S = Q K^T (M=128, N=128, K=64) into TMEM and
-// O_j = P_j V_j (M=128, N=64, K=128; V read MN-major) into a second TMEM region,
-// warps 2-5: one thread per query row reads S from TMEM, runs the online softmax
-// (exp2 on the MUFU), writes P (bf16) to shared memory in the 128-byte swizzle
-// layout the MMA reads, and accumulates O = alpha * O + O_j in registers.
+// CTA layout (384 threads, three warpgroups): two softmax warpgroups, each
+// owning one 128-query tile (thread = query row = TMEM lane); in the third, warp
+// 8 issues TMA (both Q tiles once, K/V through 3-stage rings shared by the
+// groups) and warp 9 issues the MMAs from one thread.  setmaxnreg moves
+// registers from the third warpgroup to the softmax warpgroups so a full row of
+// 128 scores stays in registers.  Per KV tile j and group g:
+//   S_g = Q_g K_j^T            tcgen05.mma, A and B from shared memory, D in TMEM
+//   P_g = exp2(S_g * c - m_g)  softmax threads, written back over S_g in TMEM as
+//                              bf16 pairs (byte-permute truncation)
+//   O_g += P_g [V_j | 1]       tcgen05.mma with A = P from TMEM; the ones block
+//                              appended to V makes the tensor core produce the row
+//                              sums of the same truncated P, so the truncation
+//                              cancels in O / l
+// The groups ping-pong: the MMAs of one group run while the other computes its
+// softmax.  The running maximum is lazy: O and l are rescaled (in TMEM) only
+// when a row's maximum grows by more than 2^8.  Part of the exponentials run as
+// a polynomial on the FMA pipe (range reduction to 2^j * 2^f, |f| <= 1/2, with a
+// degree-3 polynomial for 2^f fitted by weighted least squares on Chebyshev
+// nodes, max relative error 7.5e-5) to offload the MUFU unit.
+//
+// Split-KV: with few query tiles per SM (small maps) the KV tile list of a Q-tile
+// pair is split over `splits` CTAs; each writes its unnormalised O, m and l to a
+// scratch buffer and the last CTA of the pair (arrival counter) merges them in
+// split order, so the result is deterministic.
 #include "dfp_common.cuh"
 #include "kernels.h"
 
@@ -25,11 +43,16 @@ namespace dfp {
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kTileQ = 128;
-constexpr int kTileK = 128;
+constexpr int kThreads = 384;
+constexpr int kRegsSoftmax = 208;               // 256 x 208 + 128 x 80 = 63488 <= 384 x 168 (launch)
+constexpr int kRegsOther = 80;
+constexpr int kTile = 128;
 constexpr uint32_t kTileBytes = 128 * 64 * 2;   // one 128 x 64 bf16 tile
-constexpr uint32_t kTmemCols = 256;             // S: cols [0,128), O_j: cols [128,192)
+constexpr int kStages = 3;
+constexpr int kOCols = 80;                      // 64 outputs + 16 row-sum columns
+constexpr uint32_t kTmemCols = 512;             // S/P: [128g, 128g+128), O: [256+128g, +80)
+constexpr float kRescale = 8.f;                 // lazy rescale threshold (log2 units)
+constexpr int kPolyPer8 = 2;                    // of every 8 columns, this many use the polynomial
 
 struct Segs {
   int n;
@@ -42,7 +65,7 @@ __device__ __forceinline__ Segs make_segs(int mode, int p, int Lp, int L) {
   auto add = [&](int st, int b, int len) {
     if (len <= 0) return;
     s.stale[s.n] = st; s.start[s.n] = b; s.len[s.n] = len;
-    s.tiles[s.n] = (len + kTileK - 1) / kTileK;
+    s.tiles[s.n] = (len + kTile - 1) / kTile;
     s.total += s.tiles[s.n];
     ++s.n;
   };
@@ -58,19 +81,100 @@ __device__ __forceinline__ Segs make_segs(int mode, int p, int Lp, int L) {
   return s;
 }
 
-// tile j -> (stale?, first key row, valid keys)
+// tile j of the segment list -> (stale?, first key row, valid keys)
 __device__ __forceinline__ void seg_tile(const Segs& s, int j, int& stale, int& row, int& valid) {
   int k = 0;
   while (k < s.n - 1 && j >= s.tiles[k]) { j -= s.tiles[k]; ++k; }
   stale = s.stale[k];
-  row = s.start[k] + j * kTileK;
-  valid = min(kTileK, s.len[k] - j * kTileK);
+  row = s.start[k] + j * kTile;
+  valid = min(kTile, s.len[k] - j * kTile);
 }
 
-__device__ __forceinline__ float ex2(float x) {
+__device__ __forceinline__ float ex2_mufu(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe: x = j + f with j = rint(x) (magic-constant rounding),
+// 2^f by a degree-3 polynomial, 2^j added into the exponent field.  x >= -125.
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = __fadd_rn(x, 12582912.f);      // 1.5 * 2^23: j lands in the low mantissa bits
+  const float j = __fadd_rn(t, -12582912.f);
+  const float f = __fadd_rn(x, -j);
+  float p = fmaf(0.0551716648f, f, 0.242611125f);
+  p = fmaf(p, f, 0.693260968f);
+  p = fmaf(p, f, 0.999928057f);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// upper halves of two fp32 words -> one bf16 pair (lo = a, hi = b): truncation
+__device__ __forceinline__ uint32_t pack_trunc(float a, float b) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(__float_as_uint(a)), "r"(__float_as_uint(b)));
+  return r;
+}
+
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+template <int N> __device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N> __device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+__device__ __forceinline__ void named_bar(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Load the 80 O columns (64 outputs + row sums) of this thread's row.
+__device__ __forceinline__ void load_o(uint32_t tO, float (&o)[64], float& l) {
+  uint32_t r[32], r16[16];
+  tmem_ld32(tO, r);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(r[i]);
+  tmem_ld32(tO + 32, r);
+  tmem_ld16(tO + 64, r16);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) o[32 + i] = __uint_as_float(r[i]);
+  l = __uint_as_float(r16[0]);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -79,43 +183,55 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
                     const __grid_constant__ CUtensorMap mvs, const TcAttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                       // 16 KB
-  uint8_t* sK = sQ + kTileBytes;            // 2 x 16 KB
-  uint8_t* sV = sK + 2 * kTileBytes;        // 2 x 16 KB
-  uint8_t* sP = sV + 2 * kTileBytes;        // 32 KB: keys [0,64) then [64,128), each 128 rows x 128 B
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * kTileBytes);
+  uint8_t* sQ = smem;                          // 2 x 16 KB
+  uint8_t* sK = sQ + 2 * kTileBytes;           // kStages x 16 KB
+  uint8_t* sV = sK + kStages * kTileBytes;     // kStages x 16 KB
+  uint8_t* sOnes = sV + kStages * kTileBytes;  // 16 KB of bf16 1.0 (the row-sum columns of B)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOnes + kTileBytes);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;   // [2]
-  uint64_t* k_empty = bars + 3;  // [2]
-  uint64_t* v_full = bars + 5;   // [2]
-  uint64_t* v_empty = bars + 7;  // [2]
-  uint64_t* s_full = bars + 9;
-  uint64_t* p_full = bars + 10;
-  uint64_t* o_full = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + kStages;
+  uint64_t* v_full = k_empty + kStages;
+  uint64_t* v_empty = v_full + kStages;
+  uint64_t* s_full = v_empty + kStages;        // [2]
+  uint64_t* p_full = s_full + 2;               // [2]
+  uint64_t* o_done = p_full + 2;               // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 2);
   __shared__ volatile int s_abort;
+  __shared__ int s_last;
+  __shared__ Segs s_segs;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int head = blockIdx.z, p = blockIdx.y;
-  const int q_local0 = blockIdx.x * kTileQ;
-  const int q_row0 = p * a.Lp + q_local0;
-  const Segs segs = make_segs(a.mode, p, a.Lp, a.L);
-  const int nt = segs.total;
+  const int splits = a.splits;
+  const int split = blockIdx.x % splits, pair = blockIdx.x / splits;
+  const int p = blockIdx.y, head = blockIdx.z;
+  const int qt0 = 2 * pair;
+  const bool activeB = qt0 + 1 < a.n_qtiles;
+  const Segs& segs = s_segs;   // the KV segment list lives in shared memory (registers are precious)
   int* err = a.err;
 
   if (threadIdx.x == 0) {
+    s_segs = make_segs(a.mode, p, a.Lp, a.L);
     s_abort = 0;
     mbar_init(smem_u32(q_full), 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(smem_u32(&k_full[i]), 1); mbar_init(smem_u32(&k_empty[i]), 1);
       mbar_init(smem_u32(&v_full[i]), 1); mbar_init(smem_u32(&v_empty[i]), 1);
     }
-    mbar_init(smem_u32(s_full), 1);
-    mbar_init(smem_u32(p_full), 128);
-    mbar_init(smem_u32(o_full), 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(smem_u32(&s_full[g]), 1);
+      mbar_init(smem_u32(&p_full[g]), 128);
+      mbar_init(smem_u32(&o_done[g]), 1);
+    }
     fence_mbar_init();
   }
-  if (warp == 1) {
+  {
+    uint4* ones = reinterpret_cast<uint4*>(sOnes);
+    for (int i = threadIdx.x; i < (int)(kTileBytes / 16); i += kThreads)
+      ones[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -123,19 +239,24 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_s = tmem, tmem_o = tmem + 128;
+  const int j0 = split * segs.total / splits;
+  const int nt = (split + 1) * segs.total / splits - j0;
 
-  if (warp == 0) {
+  if (warp >= 8) {
+   setmaxnreg_dec<kRegsOther>();
+   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&mq);
-      mbar_arrive_expect_tx(smem_u32(q_full), kTileBytes);
-      tma_load_3d(smem_u32(sQ), &mq, smem_u32(q_full), 0, q_row0, head);
+      const int qrow = p * a.Lp + qt0 * kTile;
+      mbar_arrive_expect_tx(smem_u32(q_full), activeB ? 2 * kTileBytes : kTileBytes);
+      tma_load_3d(smem_u32(sQ), &mq, smem_u32(q_full), 0, qrow, head);
+      if (activeB) tma_load_3d(smem_u32(sQ + kTileBytes), &mq, smem_u32(q_full), 0, qrow + kTile, head);
       int issued = 0;
-      for (int j = 0; j < nt; ++j) {
-        const int s = j & 1, round = j >> 1;
+      for (int jj = 0; jj < nt; ++jj) {
+        const int s = jj % kStages, round = jj / kStages;
         int stale, row, valid;
-        seg_tile(segs, j, stale, row, valid);
+        seg_tile(segs, j0 + jj, stale, row, valid);
         if (round > 0 && !mbar_wait(smem_u32(&k_empty[s]), (round - 1) & 1, err, kErrWaitStageFree)) { s_abort = 1; break; }
         mbar_arrive_expect_tx(smem_u32(&k_full[s]), kTileBytes);
         tma_load_3d(smem_u32(sK + s * kTileBytes), stale ? &mks : &mkf, smem_u32(&k_full[s]), 0, row, head);
@@ -150,122 +271,248 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
         ++issued;
       }
       if (s_abort) {
-        for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) {
-          mbar_wait(smem_u32(&k_full[j & 1]), (j >> 1) & 1, err, kErrWaitTmaFull);
-          mbar_wait(smem_u32(&v_full[j & 1]), (j >> 1) & 1, err, kErrWaitTmaFull);
+        for (int jj = (issued > kStages ? issued - kStages : 0); jj < issued; ++jj) {
+          mbar_wait(smem_u32(&k_full[jj % kStages]), (jj / kStages) & 1, err, kErrWaitTmaFull);
+          mbar_wait(smem_u32(&v_full[jj % kStages]), (jj / kStages) & 1, err, kErrWaitTmaFull);
         }
       }
     }
-  } else if (warp == 1) {
+   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTileK, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 64, false, true);
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTile, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, kOCols, false, true);
+      // group g: S/P at TMEM column 128 g, O at 256 + 128 g; Q tile at sQ + g * 16 KB
+      const uint64_t qd0 = sw128_kmajor_desc(smem_u32(sQ));
+      const int ng = activeB ? 2 : 1;
       bool ok = mbar_wait(smem_u32(q_full), 0, err, kErrWaitTmaFull);
-      const uint64_t qd = sw128_kmajor_desc(smem_u32(sQ));
-      for (int j = 0; ok && j < nt; ++j) {
-        const int s = j & 1, round = j >> 1;
-        if (!mbar_wait(smem_u32(&k_full[s]), round & 1, err, kErrWaitTmaFull)) { ok = false; break; }
-        tc_fence_after();
+      auto issue_s = [&](int g, int s) {
         const uint64_t kd = sw128_kmajor_desc(smem_u32(sK + s * kTileBytes));
+        const uint64_t qd = qd0 + (uint64_t)((g * kTileBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_f16_ss(tmem_s, qd + 2 * kk, kd + 2 * kk, idesc_s, kk != 0);
-        umma_commit(smem_u32(&k_empty[s]));
-        umma_commit(smem_u32(s_full));
-        if (!mbar_wait(smem_u32(p_full), j & 1, err, kErrWaitAttnP)) { ok = false; break; }
-        if (!mbar_wait(smem_u32(&v_full[s]), round & 1, err, kErrWaitTmaFull)) { ok = false; break; }
+        for (int kk = 0; kk < 4; ++kk) umma_f16_ss(tmem + 128 * g, qd + 2 * kk, kd + 2 * kk, idesc_s, kk != 0);
+        umma_commit(smem_u32(&s_full[g]));
+      };
+      if (ok) {
+        if (!mbar_wait(smem_u32(&k_full[0]), 0, err, kErrWaitTmaFull)) ok = false;
         tc_fence_after();
-        const uint64_t vd = sw128_mnmajor_desc(smem_u32(sV + s * kTileBytes));
-        const uint64_t pd0 = sw128_kmajor_desc(smem_u32(sP));
-        const uint64_t pd1 = sw128_kmajor_desc(smem_u32(sP + kTileBytes));
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = (kk < 4 ? pd0 : pd1) + 2 * (kk & 3);
-          const uint64_t bd = vd + (uint64_t)((kk * 16 * 128) >> 4);   // 16 keys = 16 rows of 128 B
-          umma_f16_ss(tmem_o, ad, bd, idesc_o, kk != 0);
+        if (ok) {
+          for (int g = 0; g < ng; ++g) issue_s(g, 0);
+          umma_commit(smem_u32(&k_empty[0]));
         }
+      }
+      for (int jj = 0; ok && jj < nt; ++jj) {
+        const int s = jj % kStages, round = jj / kStages;
+        const int s1 = (jj + 1) % kStages, round1 = (jj + 1) / kStages;
+        const bool more = jj + 1 < nt;
+        // V_j with the ones block as its second 64-column atom (leading byte offset)
+        const uint32_t vaddr = smem_u32(sV + s * kTileBytes);
+        uint64_t vd = sw128_mnmajor_desc(vaddr);
+        vd = (vd & ~(uint64_t(0x3FFF) << 16)) | (uint64_t(((smem_u32(sOnes) - vaddr) >> 4) & 0x3FFF) << 16);
+        if (!mbar_wait(smem_u32(&v_full[s]), round & 1, err, kErrWaitTmaFull)) { ok = false; break; }
+        for (int g = 0; g < ng; ++g) {
+          if (!mbar_wait(smem_u32(&p_full[g]), jj & 1, err, kErrWaitAttnP)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_f16_ts(tmem + 256 + 128 * g, tmem + 128 * g + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4),
+                        idesc_o, (jj | kk) != 0);
+          umma_commit(smem_u32(&o_done[g]));
+          if (more) {
+            if (g == 0 && !mbar_wait(smem_u32(&k_full[s1]), round1 & 1, err, kErrWaitTmaFull)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(g, s1);
+          }
+        }
+        if (!ok) break;
         umma_commit(smem_u32(&v_empty[s]));
-        umma_commit(smem_u32(o_full));
+        if (more) umma_commit(smem_u32(&k_empty[s1]));
       }
       if (!ok) s_abort = 1;
     }
+   }
   } else {
-    // ------------------------------------------------------------ softmax (warps 2..5)
+    setmaxnreg_inc<kRegsSoftmax>();
+    // ------------------------------------------------------------ softmax groups (warps 0..7)
+    const int g = warp >> 2;
     const int sub = warp & 3;
     const int row = sub * 32 + lane;
+    const bool active = g == 0 || activeB;
     const uint32_t lane_off = (uint32_t)(sub * 32) << 16;
+    const uint32_t tS = tmem + 128 * g + lane_off;
+    const uint32_t tO = tmem + 256 + 128 * g + lane_off;
     const float sl2 = 0.125f * 1.4426950408889634f;   // (1/sqrt(64)) * log2(e)
-    float m_run = -INFINITY, l_run = 0.f;
-    float oacc[64];
-#pragma unroll
-    for (int i = 0; i < 64; ++i) oacc[i] = 0.f;
-    uint8_t* prow = sP + row * 128;
-    const int sw = row & 7;
-    for (int j = 0; j < nt; ++j) {
+    float m_used = -INFINITY;
+    bool ok = active;
+    for (int jj = 0; ok && jj < nt; ++jj) {
       int stale, krow, valid;
-      seg_tile(segs, j, stale, krow, valid);
-      if (!mbar_wait(smem_u32(s_full), j & 1, err, kErrWaitAttnS)) { s_abort = 1; break; }
+      seg_tile(segs, j0 + jj, stale, krow, valid);
+      if (!mbar_wait(smem_u32(&s_full[g]), jj & 1, err, kErrWaitAttnS)) { ok = false; s_abort = 1; break; }
       tc_fence_after();
       float sc[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem_s + lane_off + c * 32, r);
-        tmem_wait_ld();
+        tmem_ld32(tS + c * 32, r);
 #pragma unroll
         for (int i = 0; i < 32; ++i) sc[c * 32 + i] = __uint_as_float(r[i]);
       }
-      float mx = -INFINITY;
+      tmem_wait_ld();
+      const bool full_tile = valid == kTile;
+      if (!full_tile) {
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        sc[i] = i < valid ? sc[i] * sl2 : -INFINITY;
-        mx = fmaxf(mx, sc[i]);
+        for (int i = 0; i < 128; ++i) sc[i] = i < valid ? sc[i] : -INFINITY;
       }
-      const float m_new = fmaxf(m_run, mx);
-      const float alpha = ex2(m_run - m_new);
-      float rs = 0.f;
+      float mx[8];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        float pv[8];
+      for (int i = 0; i < 8; ++i) mx[i] = sc[i];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) { pv[e] = ex2(sc[c * 8 + e] - m_new); rs += pv[e]; }
-        const int blk = c >> 3, chunk = c & 7;
-        *reinterpret_cast<uint4*>(prow + blk * kTileBytes + ((chunk ^ sw) << 4)) = pack16(pv);
+      for (int i = 8; i < 128; i += 16) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], sc[i + k], sc[i + 8 + k]);
       }
-      l_run = l_run * alpha + rs;
-      m_run = m_new;
-      fence_proxy_async_smem();
+      const float mrow = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl2;
+      if (jj == 0) {
+        m_used = mrow;
+      } else {
+        const bool need = mrow > m_used + kRescale;
+        if (__any_sync(0xffffffffu, need)) {
+          const float m_new = need ? mrow : m_used;
+          const float alpha = ex2_mufu(m_used - m_new);
+          if (!mbar_wait(smem_u32(&o_done[g]), (jj - 1) & 1, err, kErrWaitAttnO)) { ok = false; s_abort = 1; }
+          tc_fence_after();
+          // O and its row sums (80 columns) times alpha, in five 16-column pieces
+#pragma unroll
+          for (int c = 0; c < kOCols / 16; ++c) {
+            uint32_t r16[16];
+            tmem_ld16(tO + c * 16, r16);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha);
+            tmem_st16(tO + c * 16, r16);
+          }
+          tmem_wait_st();
+          m_used = m_new;
+          if (!ok) break;
+        }
+      }
+      const float nm = -m_used;
+      if (full_tile) {
+        // a fixed share of the exponentials on the FMA pipe, the rest on the MUFU
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float x0 = fmaf(sc[c * 32 + e], sl2, nm);
+            const float x1 = fmaf(sc[c * 32 + e + 1], sl2, nm);
+            float p0, p1;
+            if ((e & 7) < kPolyPer8) { p0 = ex2_poly(x0); p1 = ex2_poly(x1); }
+            else { p0 = ex2_mufu(x0); p1 = ex2_mufu(x1); }
+            pk[e >> 1] = pack_trunc(p0, p1);
+          }
+          tmem_st16(tS + c * 16, pk);
+        }
+      } else {
+        // partial tile: masked columns are -inf, which only the MUFU maps to exactly 0
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2)
+            pk[e >> 1] = pack_trunc(ex2_mufu(fmaf(sc[c * 32 + e], sl2, nm)),
+                                    ex2_mufu(fmaf(sc[c * 32 + e + 1], sl2, nm)));
+          tmem_st16(tS + c * 16, pk);
+        }
+      }
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(p_full));
-      if (!mbar_wait(smem_u32(o_full), j & 1, err, kErrWaitAttnO)) { s_abort = 1; break; }
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem_o + lane_off + c * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) oacc[c * 32 + i] = fmaf(oacc[c * 32 + i], alpha, __uint_as_float(r[i]));
-      }
-      tc_fence_before();
+      mbar_arrive(smem_u32(&p_full[g]));
     }
-    if (!s_abort && q_local0 + row < a.Lp) {
-      const float inv = 1.f / l_run;
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) +
-                                            (size_t)(q_row0 + row) * a.C + head * 64);
+    // ---- epilogue: final O and row sums of this CTA's KV range
+    float o[64], l = 1.f;
+    bool have = false;
+    if (ok && !s_abort) {
+      if (mbar_wait(smem_u32(&o_done[g]), (nt - 1) & 1, err, kErrWaitAttnO)) {
+        tc_fence_after();
+        load_o(tO, o, l);
+        have = true;
+      } else {
+        s_abort = 1;
+      }
+    }
+    const int q_local = (qt0 + g) * kTile + row;
+    const bool row_ok = have && q_local < a.Lp;
+    if (splits == 1) {
+      if (row_ok) {
+        const float inv = 1.f / l;
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) +
+                                              (size_t)(p * a.Lp + q_local) * a.C + head * 64);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float w8[8];
+        for (int c = 0; c < 8; ++c) {
+          float w8[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) w8[e] = oacc[c * 8 + e] * inv;
-        dst[c] = pack16(w8);
+          for (int e = 0; e < 8; ++e) w8[e] = o[c * 8 + e] * inv;
+          dst[c] = pack16(w8);
+        }
+      }
+    } else {
+      // partial results of this split, then the last CTA of the pair merges them
+      const size_t grp = ((size_t)head * a.N + p) * ((a.n_qtiles + 1) / 2) + pair;
+      const size_t slot = (grp * splits + split) * 256 + g * 128 + row;
+      if (have) {
+        float4* po = reinterpret_cast<float4*>(a.part_o + slot * 64);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) po[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        reinterpret_cast<float2*>(a.part_ml)[slot] = make_float2(m_used, l);
+      }
+      __threadfence();
+      named_bar(1, 256);
+      if (threadIdx.x == 0) s_last = atomicAdd(a.counters + grp, 1u) == (unsigned)(splits - 1);
+      named_bar(1, 256);
+      if (s_last) {
+        __threadfence();
+        if (row_ok) {
+          float mm = -INFINITY;
+          for (int s = 0; s < splits; ++s)
+            mm = fmaxf(mm, __ldcg(reinterpret_cast<const float2*>(a.part_ml) + (grp * splits + s) * 256 + g * 128 + row).x);
+          float acc[64], lsum = 0.f;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+          for (int s = 0; s < splits; ++s) {
+            const size_t sl = (grp * splits + s) * 256 + g * 128 + row;
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sl);
+            const float w = ex2_mufu(ml.x - mm);
+            lsum = fmaf(ml.y, w, lsum);
+            const float4* po = reinterpret_cast<const float4*>(a.part_o + sl * 64);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const float4 v = __ldcg(po + c);
+              acc[4 * c] = fmaf(v.x, w, acc[4 * c]);
+              acc[4 * c + 1] = fmaf(v.y, w, acc[4 * c + 1]);
+              acc[4 * c + 2] = fmaf(v.z, w, acc[4 * c + 2]);
+              acc[4 * c + 3] = fmaf(v.w, w, acc[4 * c + 3]);
+            }
+          }
+          const float inv = 1.f / lsum;
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) +
+                                                (size_t)(p * a.Lp + q_local) * a.C + head * 64);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            float w8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w8[e] = acc[c * 8 + e] * inv;
+            dst[c] = pack16(w8);
+          }
+        }
+        if (threadIdx.x == 0) a.counters[grp] = 0u;
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -273,13 +520,30 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
 
 }  // namespace
 
+int attention_splits(int L, int Lp, int N, int heads, int mode_min_tiles) {
+  const int n_qt = (Lp + kTile - 1) / kTile;
+  const int groups = ((n_qt + 1) / 2) * N * heads;
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= 4; ++s) {
+    if (s > 1 && mode_min_tiles / s < 2) break;
+    const long items = (long)groups * s;
+    const long waves = (items + 147) / 148;
+    const double eff = (double)items / (double)(waves * 148);
+    if (eff > best_eff + 0.03) { best_eff = eff; best = s; }
+    if (eff >= 0.85) break;
+  }
+  return best;
+}
+
 cudaError_t launch_tc_attention(const TcAttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mkf,
                                 const CUtensorMap& mvf, const CUtensorMap& mks,
                                 const CUtensorMap& mvs, cudaStream_t s) {
-  const size_t smem = 1024 + 7 * (size_t)kTileBytes + 13 * 8 + 64;
+  const size_t smem = 1024 + (2 + 2 * kStages + 1) * (size_t)kTileBytes + (4 * kStages + 8) * 8 + 64;
   cudaError_t e = cudaFuncSetAttribute(tc_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.Lp + kTileQ - 1) / kTileQ, a.N, a.heads);
+  const int n_qt = (a.Lp + kTile - 1) / kTile;
+  dim3 grid(((n_qt + 1) / 2) * a.splits, a.N, a.heads);
   tc_attention_kernel<<<grid, kThreads, smem, s>>>(mq, mkf, mvf, mks, mvs, a);
   return cudaGetLastError();
 }
