@@ -12,12 +12,14 @@
 // Segment ends need not be multiples of the 128-key tile: columns past a
 // segment's end are masked.
 //
-// CTA layout (384 threads, three warpgroups): two softmax warpgroups, each
-// owning one 128-query tile (thread = query row = TMEM lane); in the third, warp
-// 8 issues TMA (both Q tiles once, K/V through 3-stage rings shared by the
-// groups) and warp 9 issues the MMAs from one thread.  setmaxnreg moves
-// registers from the third warpgroup to the softmax warpgroups so a full row of
-// 128 scores stays in registers.  Per KV tile j and group g:
+// CTA layout (640 threads, five warpgroups): two softmax groups of 8 warps, each
+// owning one 128-query tile.  Warps w and w+4 of a group read the same 32 TMEM
+// lanes (query rows); the first takes key columns 0-63, the second 64-127, and
+// they exchange their partial row maxima through shared memory -- at head width
+// 64 the softmax work per tile is large next to the MMAs, and two threads per
+// row double the latency hiding.  In the fifth warpgroup warp 16 issues TMA
+// (both Q tiles once, K/V through 3-stage rings shared by the groups) and warp
+// 17 issues the MMAs from one thread.  Per KV tile j and group g:
 //   S_g = Q_g K_j^T            tcgen05.mma, A and B from shared memory, D in TMEM
 //   P_g = exp2(S_g * c - m_g)  softmax threads, written back over S_g in TMEM as
 //                              bf16 pairs (byte-permute truncation)
@@ -43,16 +45,16 @@ namespace dfp {
 
 namespace {
 
-constexpr int kThreads = 384;
-constexpr int kRegsSoftmax = 208;               // 256 x 208 + 128 x 80 = 63488 <= 384 x 168 (launch)
-constexpr int kRegsOther = 80;
+constexpr int kThreads = 640;
+constexpr int kSoftmaxThreads = 512;
+constexpr int kWarpTma = 16, kWarpMma = 17;
 constexpr int kTile = 128;
 constexpr uint32_t kTileBytes = 128 * 64 * 2;   // one 128 x 64 bf16 tile
 constexpr int kStages = 3;
 constexpr int kOCols = 80;                      // 64 outputs + 16 row-sum columns
 constexpr uint32_t kTmemCols = 512;             // S/P: [128g, 128g+128), O: [256+128g, +80)
 constexpr float kRescale = 8.f;                 // lazy rescale threshold (log2 units)
-constexpr int kPolyPer8 = 2;                    // of every 8 columns, this many use the polynomial
+constexpr int kPolyPer8 = 3;                    // of every 8 columns, this many use the polynomial
 
 struct Segs {
   int n;
@@ -96,17 +98,48 @@ __device__ __forceinline__ float ex2_mufu(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe: x = j + f with j = rint(x) (magic-constant rounding),
-// 2^f by a degree-3 polynomial, 2^j added into the exponent field.  x >= -125.
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = __fadd_rn(x, 12582912.f);      // 1.5 * 2^23: j lands in the low mantissa bits
-  const float j = __fadd_rn(t, -12582912.f);
-  const float f = __fadd_rn(x, -j);
-  float p = fmaf(0.0551716648f, f, 0.242611125f);
-  p = fmaf(p, f, 0.693260968f);
-  p = fmaf(p, f, 0.999928057f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+// ---- packed fp32x2 arithmetic (two lanes per 64-bit register pair)
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^x for a pair on the FMA pipe, returned as a truncated bf16 pair (lo = first
+// lane): x = j + f with j = rint(x) by magic-constant rounding (1.5 * 2^23 puts j
+// in the low mantissa bits), 2^f by a degree-3 polynomial, 2^j added into the
+// exponent field.  x is clamped to >= -125 so the exponent cannot wrap.
+__device__ __forceinline__ uint32_t ex2_poly_pair_bf16(uint64_t x2) {
+  float x0, x1;
+  f2_split(x2, x0, x1);
+  const uint64_t x = f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = add2(x, f2(12582912.f, 12582912.f));
+  const uint64_t j = add2(t, f2(-12582912.f, -12582912.f));
+  const uint64_t f = fma2(j, f2(-1.f, -1.f), x);
+  uint64_t p = fma2(f2(0.0551716648f, 0.0551716648f), f, f2(0.242611125f, 0.242611125f));
+  p = fma2(p, f, f2(0.693260968f, 0.693260968f));
+  p = fma2(p, f, f2(0.999928057f, 0.999928057f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  const uint32_t r0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
+  const uint32_t r1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(r0), "r"(r1));
+  return r;
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -152,29 +185,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
-template <int N> __device__ __forceinline__ void setmaxnreg_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N> __device__ __forceinline__ void setmaxnreg_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+// Named barrier that also ORs a predicate over the participating threads: every
+// thread leaves with the same answer, so a group can give up collectively.
+__device__ __forceinline__ bool named_bar_or(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(n) : "memory");
+  return r != 0;
 }
 __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
-// Load the 80 O columns (64 outputs + row sums) of this thread's row.
-__device__ __forceinline__ void load_o(uint32_t tO, float (&o)[64], float& l) {
-  uint32_t r[32], r16[16];
-  tmem_ld32(tO, r);
-  tmem_wait_ld();
-#pragma unroll
-  for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(r[i]);
-  tmem_ld32(tO + 32, r);
-  tmem_ld16(tO + 64, r16);
-  tmem_wait_ld();
-#pragma unroll
-  for (int i = 0; i < 32; ++i) o[32 + i] = __uint_as_float(r[i]);
-  l = __uint_as_float(r16[0]);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -200,6 +224,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
   __shared__ volatile int s_abort;
   __shared__ int s_last;
   __shared__ Segs s_segs;
+  __shared__ float s_rowmax[2][2][2][128];   // [tile parity][group][half][row]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int splits = a.splits;
@@ -220,7 +245,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(smem_u32(&s_full[g]), 1);
-      mbar_init(smem_u32(&p_full[g]), 128);
+      mbar_init(smem_u32(&p_full[g]), 256);
       mbar_init(smem_u32(&o_done[g]), 1);
     }
     fence_mbar_init();
@@ -231,7 +256,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
       ones[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
     fence_proxy_async_smem();
   }
-  if (warp == 9) {
+  if (warp == kWarpMma) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -242,9 +267,8 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
   const int j0 = split * segs.total / splits;
   const int nt = (split + 1) * segs.total / splits - j0;
 
-  if (warp >= 8) {
-   setmaxnreg_dec<kRegsOther>();
-   if (warp == 8) {
+  if (warp >= kWarpTma) {
+   if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&mq);
@@ -277,65 +301,84 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
         }
       }
     }
-   } else if (warp == 9) {
+   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      // Per MMA, every operand is a per-tile base plus a compile-time offset (the two
+      // groups and the K slices are unrolled): runtime arithmetic between
+      // tcgen05.mma instructions stalls their issue.
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTile, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, kOCols, false, true);
-      // group g: S/P at TMEM column 128 g, O at 256 + 128 g; Q tile at sQ + g * 16 KB
+      constexpr uint64_t kTileDesc = kTileBytes >> 4;            // one tile in descriptor address units
       const uint64_t qd0 = sw128_kmajor_desc(smem_u32(sQ));
-      const int ng = activeB ? 2 : 1;
+      const uint64_t kd0 = sw128_kmajor_desc(smem_u32(sK));
+      // V stage 0 with the ones block as its second 64-column atom (leading byte offset);
+      // stage st: start address + st tiles, leading byte offset - st tiles
+      uint64_t vd0 = sw128_mnmajor_desc(smem_u32(sV));
+      vd0 = (vd0 & ~(uint64_t(0x3FFF) << 16)) |
+            (uint64_t(((smem_u32(sOnes) - smem_u32(sV)) >> 4) & 0x3FFF) << 16);
+      const bool two = activeB;
       bool ok = mbar_wait(smem_u32(q_full), 0, err, kErrWaitTmaFull);
-      auto issue_s = [&](int g, int s) {
-        const uint64_t kd = sw128_kmajor_desc(smem_u32(sK + s * kTileBytes));
-        const uint64_t qd = qd0 + (uint64_t)((g * kTileBytes) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_f16_ss(tmem + 128 * g, qd + 2 * kk, kd + 2 * kk, idesc_s, kk != 0);
-        umma_commit(smem_u32(&s_full[g]));
-      };
+      // S_g = Q_g K^T, K tile at descriptor kd
+#define DFP_ISSUE_S(G, KD)                                                   \
+      do {                                                                   \
+        const uint64_t qd = qd0 + (uint64_t)(G) * kTileDesc;                 \
+        umma_f16_ss(tmem + 128 * (G), qd, (KD), idesc_s, 0);                 \
+        umma_f16_ss(tmem + 128 * (G), qd + 2, (KD) + 2, idesc_s, 1);         \
+        umma_f16_ss(tmem + 128 * (G), qd + 4, (KD) + 4, idesc_s, 1);         \
+        umma_f16_ss(tmem + 128 * (G), qd + 6, (KD) + 6, idesc_s, 1);         \
+        umma_commit(smem_u32(&s_full[G]));                                   \
+      } while (0)
+      // O_g += P_g [V | 1], V tile at descriptor vd (P read from TMEM over S_g)
+#define DFP_ISSUE_PV(G, VD, ACC0)                                                                \
+      do {                                                                                       \
+        umma_f16_ts(tmem + 256 + 128 * (G), tmem + 128 * (G), (VD), idesc_o, (ACC0));            \
+        _Pragma("unroll") for (int kk = 1; kk < 8; ++kk)                                         \
+          umma_f16_ts(tmem + 256 + 128 * (G), tmem + 128 * (G) + kk * 8, (VD) + (uint64_t)kk * 128, idesc_o, 1); \
+        umma_commit(smem_u32(&o_done[G]));                                                       \
+      } while (0)
+      if (ok && !mbar_wait(smem_u32(&k_full[0]), 0, err, kErrWaitTmaFull)) ok = false;
       if (ok) {
-        if (!mbar_wait(smem_u32(&k_full[0]), 0, err, kErrWaitTmaFull)) ok = false;
         tc_fence_after();
-        if (ok) {
-          for (int g = 0; g < ng; ++g) issue_s(g, 0);
-          umma_commit(smem_u32(&k_empty[0]));
-        }
+        DFP_ISSUE_S(0, kd0);
+        if (two) DFP_ISSUE_S(1, kd0);
+        umma_commit(smem_u32(&k_empty[0]));
       }
       for (int jj = 0; ok && jj < nt; ++jj) {
-        const int s = jj % kStages, round = jj / kStages;
-        const int s1 = (jj + 1) % kStages, round1 = (jj + 1) / kStages;
+        const int st = jj % kStages, st1 = (jj + 1) % kStages;
+        const uint32_t par = (uint32_t)(jj / kStages) & 1u, par1 = (uint32_t)((jj + 1) / kStages) & 1u;
         const bool more = jj + 1 < nt;
-        // V_j with the ones block as its second 64-column atom (leading byte offset)
-        const uint32_t vaddr = smem_u32(sV + s * kTileBytes);
-        uint64_t vd = sw128_mnmajor_desc(vaddr);
-        vd = (vd & ~(uint64_t(0x3FFF) << 16)) | (uint64_t(((smem_u32(sOnes) - vaddr) >> 4) & 0x3FFF) << 16);
-        if (!mbar_wait(smem_u32(&v_full[s]), round & 1, err, kErrWaitTmaFull)) { ok = false; break; }
-        for (int g = 0; g < ng; ++g) {
-          if (!mbar_wait(smem_u32(&p_full[g]), jj & 1, err, kErrWaitAttnP)) { ok = false; break; }
+        const uint32_t acc0 = jj > 0;
+        const uint64_t vd = vd0 + (uint64_t)st * (kTileDesc - (kTileDesc << 16));
+        const uint64_t kd1 = kd0 + (uint64_t)st1 * kTileDesc;
+        if (!mbar_wait(smem_u32(&v_full[st]), par, err, kErrWaitTmaFull)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&p_full[0]), (uint32_t)jj & 1u, err, kErrWaitAttnP)) { ok = false; break; }
+        tc_fence_after();
+        DFP_ISSUE_PV(0, vd, acc0);
+        if (more) {
+          if (!mbar_wait(smem_u32(&k_full[st1]), par1, err, kErrWaitTmaFull)) { ok = false; break; }
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_f16_ts(tmem + 256 + 128 * g, tmem + 128 * g + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4),
-                        idesc_o, (jj | kk) != 0);
-          umma_commit(smem_u32(&o_done[g]));
-          if (more) {
-            if (g == 0 && !mbar_wait(smem_u32(&k_full[s1]), round1 & 1, err, kErrWaitTmaFull)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(g, s1);
-          }
+          DFP_ISSUE_S(0, kd1);
         }
-        if (!ok) break;
-        umma_commit(smem_u32(&v_empty[s]));
-        if (more) umma_commit(smem_u32(&k_empty[s1]));
+        if (two) {
+          if (!mbar_wait(smem_u32(&p_full[1]), (uint32_t)jj & 1u, err, kErrWaitAttnP)) { ok = false; break; }
+          tc_fence_after();
+          DFP_ISSUE_PV(1, vd, acc0);
+          if (more) DFP_ISSUE_S(1, kd1);
+        }
+        umma_commit(smem_u32(&v_empty[st]));
+        if (more) umma_commit(smem_u32(&k_empty[st1]));
       }
+#undef DFP_ISSUE_S
+#undef DFP_ISSUE_PV
       if (!ok) s_abort = 1;
     }
    }
   } else {
-    setmaxnreg_inc<kRegsSoftmax>();
-    // ------------------------------------------------------------ softmax groups (warps 0..7)
-    const int g = warp >> 2;
-    const int sub = warp & 3;
+    // ------------------------------------------------------------ softmax groups (warps 0..15)
+    const int g = warp >> 3;                    // query tile of this warp
+    const int half = (warp >> 2) & 1;           // key columns [64 half, 64 half + 64)
+    const int sub = warp & 3;                   // TMEM lane quadrant
     const int row = sub * 32 + lane;
     const bool active = g == 0 || activeB;
     const uint32_t lane_off = (uint32_t)(sub * 32) << 16;
@@ -344,98 +387,124 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
     const float sl2 = 0.125f * 1.4426950408889634f;   // (1/sqrt(64)) * log2(e)
     float m_used = -INFINITY;
     bool ok = active;
+    // A failed wait only marks the thread; the group leaves the loop together at the
+    // next max-exchange barrier (bar.red.or), so no thread is left waiting there.
+    bool carry = false;                         // a failed wait of the previous tile
     for (int jj = 0; ok && jj < nt; ++jj) {
       int stale, krow, valid;
       seg_tile(segs, j0 + jj, stale, krow, valid);
-      if (!mbar_wait(smem_u32(&s_full[g]), jj & 1, err, kErrWaitAttnS)) { ok = false; s_abort = 1; break; }
+      bool bad = !mbar_wait(smem_u32(&s_full[g]), jj & 1, err, kErrWaitAttnS) || carry;
       tc_fence_after();
-      float sc[128];
+      float sc[64];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
-        tmem_ld32(tS + c * 32, r);
+        tmem_ld32(tS + half * 64 + c * 32, r);
 #pragma unroll
         for (int i = 0; i < 32; ++i) sc[c * 32 + i] = __uint_as_float(r[i]);
       }
       tmem_wait_ld();
+      const int vcols = valid - half * 64;     // valid columns of this half (may be <= 0 or >= 64)
       const bool full_tile = valid == kTile;
       if (!full_tile) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) sc[i] = i < valid ? sc[i] : -INFINITY;
+        for (int i = 0; i < 64; ++i) sc[i] = i < vcols ? sc[i] : -INFINITY;
       }
       float mx[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = sc[i];
+      for (int i = 0; i < 8; ++i) mx[i] = max3(sc[i], sc[8 + i], sc[16 + i]);
 #pragma unroll
-      for (int i = 8; i < 128; i += 16) {
+      for (int i = 24; i < 64; i += 16) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], sc[i + k], sc[i + 8 + k]);
+        for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], sc[i + k], i + 8 + k < 64 ? sc[i + 8 + k] : mx[k]);
       }
-      const float mrow = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl2;
+      const float mhalf = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+      // exchange with the other half of the row (double-buffered by tile parity)
+      s_rowmax[jj & 1][g][half][row] = mhalf;
+      if (named_bar_or(2 + g, 256, bad)) { ok = false; s_abort = 1; break; }
+      const float mrow = fmaxf(mhalf, s_rowmax[jj & 1][g][half ^ 1][row]) * sl2;
       if (jj == 0) {
         m_used = mrow;
       } else {
         const bool need = mrow > m_used + kRescale;
         if (__any_sync(0xffffffffu, need)) {
+          // both halves of a row see the same mrow, so they agree on every decision
           const float m_new = need ? mrow : m_used;
           const float alpha = ex2_mufu(m_used - m_new);
-          if (!mbar_wait(smem_u32(&o_done[g]), (jj - 1) & 1, err, kErrWaitAttnO)) { ok = false; s_abort = 1; }
+          if (!mbar_wait(smem_u32(&o_done[g]), (jj - 1) & 1, err, kErrWaitAttnO)) carry = true;
           tc_fence_after();
-          // O and its row sums (80 columns) times alpha, in five 16-column pieces
+          // O (64 columns) and its row sums (16): half 0 rescales columns 0-39, half 1 40-79
 #pragma unroll
-          for (int c = 0; c < kOCols / 16; ++c) {
-            uint32_t r16[16];
-            tmem_ld16(tO + c * 16, r16);
+          for (int c = 0; c < 5; ++c) {
+            uint32_t r8[8];
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                         : "=r"(r8[0]), "=r"(r8[1]), "=r"(r8[2]), "=r"(r8[3]), "=r"(r8[4]), "=r"(r8[5]),
+                           "=r"(r8[6]), "=r"(r8[7])
+                         : "r"(tO + half * 40 + c * 8));
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha);
-            tmem_st16(tO + c * 16, r16);
+            for (int i = 0; i < 8; ++i) r8[i] = __float_as_uint(__uint_as_float(r8[i]) * alpha);
+            asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                         ::"r"(tO + half * 40 + c * 8), "r"(r8[0]), "r"(r8[1]), "r"(r8[2]), "r"(r8[3]),
+                           "r"(r8[4]), "r"(r8[5]), "r"(r8[6]), "r"(r8[7])
+                         : "memory");
           }
           tmem_wait_st();
           m_used = m_new;
-          if (!ok) break;
         }
       }
       const float nm = -m_used;
       if (full_tile) {
-        // a fixed share of the exponentials on the FMA pipe, the rest on the MUFU
+        // x = s * c - m on pairs (fp32x2); a fixed share of the pairs through the
+        // polynomial on the FMA pipe, the rest through the MUFU
+        const uint64_t sl2x2 = f2(sl2, sl2), nmx2 = f2(nm, nm);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float x0 = fmaf(sc[c * 32 + e], sl2, nm);
-            const float x1 = fmaf(sc[c * 32 + e + 1], sl2, nm);
-            float p0, p1;
-            if ((e & 7) < kPolyPer8) { p0 = ex2_poly(x0); p1 = ex2_poly(x1); }
-            else { p0 = ex2_mufu(x0); p1 = ex2_mufu(x1); }
-            pk[e >> 1] = pack_trunc(p0, p1);
+            const uint64_t x2 = fma2(f2(sc[c * 32 + e], sc[c * 32 + e + 1]), sl2x2, nmx2);
+            if (((e >> 1) & 7) < kPolyPer8) {
+              pk[e >> 1] = ex2_poly_pair_bf16(x2);
+            } else {
+              float x0, x1;
+              f2_split(x2, x0, x1);
+              pk[e >> 1] = pack_trunc(ex2_mufu(x0), ex2_mufu(x1));
+            }
           }
-          tmem_st16(tS + c * 16, pk);
+          tmem_st16(tS + half * 32 + c * 16, pk);
         }
       } else {
         // partial tile: masked columns are -inf, which only the MUFU maps to exactly 0
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2)
             pk[e >> 1] = pack_trunc(ex2_mufu(fmaf(sc[c * 32 + e], sl2, nm)),
                                     ex2_mufu(fmaf(sc[c * 32 + e + 1], sl2, nm)));
-          tmem_st16(tS + c * 16, pk);
+          tmem_st16(tS + half * 32 + c * 16, pk);
         }
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&p_full[g]));
     }
-    // ---- epilogue: final O and row sums of this CTA's KV range
-    float o[64], l = 1.f;
+    // every active thread of the group reaches this barrier exactly once
+    if (active && named_bar_or(2 + g, 256, carry || !ok)) { ok = false; s_abort = 1; }
+    // ---- epilogue: this half's 32 output columns and the row sum
+    float o[32], l = 1.f;
     bool have = false;
     if (ok && !s_abort) {
       if (mbar_wait(smem_u32(&o_done[g]), (nt - 1) & 1, err, kErrWaitAttnO)) {
         tc_fence_after();
-        load_o(tO, o, l);
+        uint32_t r[32], r16[16];
+        tmem_ld32(tO + half * 32, r);
+        tmem_ld16(tO + 64, r16);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(r[i]);
+        l = __uint_as_float(r16[0]);
         have = true;
       } else {
         s_abort = 1;
@@ -443,13 +512,13 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
     }
     const int q_local = (qt0 + g) * kTile + row;
     const bool row_ok = have && q_local < a.Lp;
+    __nv_bfloat16* out_row = static_cast<__nv_bfloat16*>(a.o) + (size_t)(p * a.Lp + q_local) * a.C + head * 64 + half * 32;
     if (splits == 1) {
       if (row_ok) {
         const float inv = 1.f / l;
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) +
-                                              (size_t)(p * a.Lp + q_local) * a.C + head * 64);
+        uint4* dst = reinterpret_cast<uint4*>(out_row);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           float w8[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) w8[e] = o[c * 8 + e] * inv;
@@ -461,32 +530,32 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
       const size_t grp = ((size_t)head * a.N + p) * ((a.n_qtiles + 1) / 2) + pair;
       const size_t slot = (grp * splits + split) * 256 + g * 128 + row;
       if (have) {
-        float4* po = reinterpret_cast<float4*>(a.part_o + slot * 64);
+        float4* po = reinterpret_cast<float4*>(a.part_o + slot * 64 + half * 32);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) po[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-        reinterpret_cast<float2*>(a.part_ml)[slot] = make_float2(m_used, l);
+        for (int c = 0; c < 8; ++c) po[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        if (half == 0) reinterpret_cast<float2*>(a.part_ml)[slot] = make_float2(m_used, l);
       }
       __threadfence();
-      named_bar(1, 256);
+      named_bar(1, kSoftmaxThreads);
       if (threadIdx.x == 0) s_last = atomicAdd(a.counters + grp, 1u) == (unsigned)(splits - 1);
-      named_bar(1, 256);
+      named_bar(1, kSoftmaxThreads);
       if (s_last) {
         __threadfence();
         if (row_ok) {
           float mm = -INFINITY;
-          for (int s = 0; s < splits; ++s)
-            mm = fmaxf(mm, __ldcg(reinterpret_cast<const float2*>(a.part_ml) + (grp * splits + s) * 256 + g * 128 + row).x);
-          float acc[64], lsum = 0.f;
+          for (int s2 = 0; s2 < splits; ++s2)
+            mm = fmaxf(mm, __ldcg(reinterpret_cast<const float2*>(a.part_ml) + (grp * splits + s2) * 256 + g * 128 + row).x);
+          float acc[32], lsum = 0.f;
 #pragma unroll
-          for (int i = 0; i < 64; ++i) acc[i] = 0.f;
-          for (int s = 0; s < splits; ++s) {
-            const size_t sl = (grp * splits + s) * 256 + g * 128 + row;
+          for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+          for (int s2 = 0; s2 < splits; ++s2) {
+            const size_t sl = (grp * splits + s2) * 256 + g * 128 + row;
             const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sl);
             const float w = ex2_mufu(ml.x - mm);
             lsum = fmaf(ml.y, w, lsum);
-            const float4* po = reinterpret_cast<const float4*>(a.part_o + sl * 64);
+            const float4* po = reinterpret_cast<const float4*>(a.part_o + sl * 64 + half * 32);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
+            for (int c = 0; c < 8; ++c) {
               const float4 v = __ldcg(po + c);
               acc[4 * c] = fmaf(v.x, w, acc[4 * c]);
               acc[4 * c + 1] = fmaf(v.y, w, acc[4 * c + 1]);
@@ -495,10 +564,9 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
             }
           }
           const float inv = 1.f / lsum;
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) +
-                                                (size_t)(p * a.Lp + q_local) * a.C + head * 64);
+          uint4* dst = reinterpret_cast<uint4*>(out_row);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < 4; ++c) {
             float w8[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) w8[e] = acc[c * 8 + e] * inv;
@@ -512,7 +580,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

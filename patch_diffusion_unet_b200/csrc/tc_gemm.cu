@@ -123,18 +123,28 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      // The stage ring is unrolled so that every MMA operand is a hoisted descriptor
+      // plus a compile-time offset: runtime arithmetic between tcgen05.mma
+      // instructions stalls their issue.
       constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, false, false);
+      const uint64_t ad0 = sw128_kmajor_desc(smem_u32(sA));
+      const uint64_t bd0 = sw128_kmajor_desc(smem_u32(sB));
       bool ok = true;
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const int s = kb % STAGES, round = kb / STAGES;
-        if (!mbar_wait(smem_u32(&full[s]), round & 1, err, kErrWaitTmaFull)) { ok = false; break; }
-        tc_fence_after();
-        const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * kABytes));
-        const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * kBBytes));
+      for (int kb0 = 0; ok && kb0 < num_kb; kb0 += STAGES) {
+        const uint32_t par = (uint32_t)(kb0 / STAGES) & 1u;
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk)
-          umma_f16_ss(tmem_d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
-        umma_commit(smem_u32(&empty[s]));
+        for (int s = 0; s < STAGES; ++s) {
+          const int kb = kb0 + s;
+          if (kb >= num_kb) break;
+          if (!mbar_wait(smem_u32(&full[s]), par, err, kErrWaitTmaFull)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = ad0 + (uint64_t)((s * kABytes) >> 4);
+          const uint64_t bd = bd0 + (uint64_t)((s * kBBytes) >> 4);
+          umma_f16_ss(tmem_d, ad, bd, idesc, kb > 0);
+#pragma unroll
+          for (int kk = 1; kk < kBK / 16; ++kk) umma_f16_ss(tmem_d, ad + 2 * kk, bd + 2 * kk, idesc, 1);
+          umma_commit(smem_u32(&empty[s]));
+        }
       }
       if (!ok) s_abort = 1;
       umma_commit(smem_u32(accum));
