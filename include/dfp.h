@@ -161,6 +161,36 @@ DFP_API dfp_status dfp_set_kernel_family(dfp_handle h, int family);
 DFP_API dfp_status dfp_set_profiling(dfp_handle h, int enable);
 DFP_API int dfp_kernel_times(dfp_handle h, float* ms, const char** names, int max_n);
 
+/* GroupNorm over N row patches with the displaced (stale/fresh) statistics merge,
+ * normalise and optional SiLU, as ONE call that allocates no memory.  The paper
+ * has no counterpart to this entry point: it exists for callers that cannot
+ * allocate device memory when they need the op (a fixed memory pool that bans the
+ * CUDA allocator, a pre-planned or capped memory region, a latency-critical host
+ * path that must not take allocator locks).
+ *   x, y            device [H, W, C] of dtype (input, output; y may not alias x)
+ *   gamma, beta     device fp32 [C]
+ *   stale_moments   device fp32 [N, G, 2] (E[x], E[x^2]) per (patch, group) of the
+ *                   previous step -- pass the previous call's fresh_moments -- or
+ *                   NULL for a synchronous step (exact full-map statistics)
+ *   fresh_moments   device fp32 [N, G, 2], out: this call's moments
+ *   mean_rstd       device fp32 [N, G, 2], out: the (mean, 1/std) applied, or NULL
+ *   cuda_stream     cudaStream_t the work is enqueued on (asynchronous)
+ * Scratch comes from a fixed 1 MiB array in the library's device memory (held by
+ * every GPU that loads the library until exit).  The first call on a device, with
+ * that device current, looks up the array's device address; make that first call
+ * before any stream capture begins.  All calls share the array and it keeps the
+ * last call's contents (the counter that must start at zero is cleared by every
+ * call), so calls that overlap on the GPU race.  Limits: n_patches * groups <= 256,
+ * n_patches * C <= 81920, and the (patch, group, block) partials <= 98304 floats;
+ * larger requests return DFP_E_ARG with the reason in
+ * dfp_group_norm_noalloc_error().  Never calls cudaMalloc or cudaFree. */
+DFP_API dfp_status dfp_group_norm_noalloc(const void* x, void* y, dfp_dtype dtype, int H, int W, int C,
+                                          int n_patches, int groups, float eps, const float* gamma,
+                                          const float* beta, const float* stale_moments, dfp_gn_mode mode,
+                                          int apply_silu, float* fresh_moments, float* mean_rstd,
+                                          void* cuda_stream);
+DFP_API const char* dfp_group_norm_noalloc_error(void);
+
 /* Free everything the handle owns (waits for its stream first).  NULL is a no-op. */
 DFP_API dfp_status dfp_destroy(dfp_handle h);
 

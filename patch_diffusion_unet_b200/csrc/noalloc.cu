@@ -1,0 +1,134 @@
+// dfp_group_norm_noalloc: the displaced-patch GroupNorm (statistics, stale/fresh
+// merge, normalise, optional SiLU) as a standalone call that allocates nothing.
+//
+// Some callers cannot allocate device memory at the moment they need the op: an
+// engine that owns a fixed memory pool and forbids the CUDA allocator, code that
+// runs where allocation is not allowed (inside a memory-capped or pre-planned
+// region), or a host that must not take the allocator's locks on its critical
+// path.  The regular path (dfp_create / dfp_step) allocates its scratch when the
+// handle is made; this entry point instead takes its scratch -- the per-block
+// partial sums, the block-arrival counter and the per-channel scale/shift -- from
+// one fixed array compiled into the library.  The caller passes only inputs and
+// outputs.
+//
+// The array (g_noalloc_scratch below) is file-scope device memory: every GPU that
+// loads the library holds its 1 MiB until the process exits.  Its host-side name
+// is only a stand-in, so the device address is looked up with
+// cudaGetSymbolAddress, once per device, by the first call made with that device
+// current; make that first call before any stream capture begins.  All calls on a
+// device share the array and it keeps the last call's contents: the counter that
+// must start at zero is cleared by every call, and calls whose work overlaps on
+// the GPU (different streams without ordering) race on the array.
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include <cuda_bf16.h>
+
+#include "../../include/dfp.h"
+#include "kernels.h"
+
+namespace {
+
+// Layout of the scratch, in floats.
+constexpr size_t kCounterFloats = 64;                 // arrival counter (first word), padded
+constexpr size_t kPartFloats = 98304;                 // per-block partial (sum x, sum x^2)
+constexpr size_t kCoefFloats = 163840;                // per-(patch, channel) (scale, shift)
+constexpr size_t kScratchFloats = kCounterFloats + kPartFloats + kCoefFloats;   // 1 MiB
+
+static __device__ __align__(256) float g_noalloc_scratch[kScratchFloats];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+float* g_ptr[kMaxDevices] = {};
+
+thread_local std::string g_noalloc_error;
+
+dfp_status fail(dfp_status s, const std::string& m) {
+  g_noalloc_error = m;
+  return s;
+}
+
+}  // namespace
+
+extern "C" DFP_API const char* dfp_group_norm_noalloc_error(void) { return g_noalloc_error.c_str(); }
+
+extern "C" DFP_API dfp_status dfp_group_norm_noalloc(const void* x, void* y, dfp_dtype dtype, int H, int W,
+                                                     int C, int n_patches, int groups, float eps,
+                                                     const float* gamma, const float* beta,
+                                                     const float* stale_moments, dfp_gn_mode mode,
+                                                     int apply_silu, float* fresh_moments, float* mean_rstd,
+                                                     void* cuda_stream) {
+  // ---- argument checks (host only, before anything reaches the GPU)
+  if (!x || !y || !gamma || !beta || !fresh_moments) return fail(DFP_E_ARG, "x, y, gamma, beta and fresh_moments must be non-NULL");
+  if (dtype != DFP_F32 && dtype != DFP_BF16) return fail(DFP_E_ARG, "unknown dtype");
+  if (H <= 0 || W <= 0 || C <= 0 || n_patches <= 0 || groups <= 0) return fail(DFP_E_ARG, "sizes must be positive");
+  if (H % n_patches) return fail(DFP_E_ARG, "H must be a multiple of n_patches");
+  if (C % groups) return fail(DFP_E_ARG, "C must be a multiple of groups");
+  const int vec = dtype == DFP_BF16 ? 8 : 4;
+  if (C % vec || C / vec > 512) return fail(DFP_E_ARG, "C must be a multiple of 16 bytes of elements and C/vector <= 512");
+  if (n_patches * groups > 256) return fail(DFP_E_ARG, "n_patches * groups must be <= 256");
+  if (mode != DFP_GN_CORRECTED && mode != DFP_GN_STALE_OTHERS) return fail(DFP_E_ARG, "unknown gn mode");
+  if (!(eps >= 0.f)) return fail(DFP_E_ARG, "eps must be >= 0");
+  if ((long long)H * W * C >= (1ll << 31)) return fail(DFP_E_ARG, "feature map too large");
+  const int pix_per_patch = (H / n_patches) * W;
+  const int n_chunks = dfp::gn_stats_chunks(n_patches, pix_per_patch);
+  const size_t part_need = (size_t)n_patches * n_chunks * groups * 2;
+  const size_t coef_need = (size_t)n_patches * C * 2;
+  if (part_need > kPartFloats)
+    return fail(DFP_E_ARG, "too many (patch, group, block) partials for the fixed scratch (" +
+                               std::to_string(part_need) + " > " + std::to_string(kPartFloats) + " floats)");
+  if (coef_need > kCoefFloats)
+    return fail(DFP_E_ARG, "n_patches * C too large for the fixed scratch (2 * n_patches * C must be <= " +
+                               std::to_string(kCoefFloats) + ")");
+
+  // ---- once per device: the device address of the scratch array
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(DFP_E_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(DFP_E_UNSUPPORTED, "device ordinal out of range");
+  float* base;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_ptr[dev]) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess || !p)
+        return fail(DFP_E_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+      g_ptr[dev] = static_cast<float*>(p);
+    }
+    base = g_ptr[dev];
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  unsigned* counter = reinterpret_cast<unsigned*>(base);
+  float* part = base + kCounterFloats;
+  float* coef = part + kPartFloats;
+
+  // the arrival counter must start at zero (the kernel also leaves it at zero)
+  e = cudaMemsetAsync(counter, 0, sizeof(unsigned), s);
+  if (e != cudaSuccess) return fail(DFP_E_CUDA, std::string("counter clear: ") + cudaGetErrorString(e));
+
+  dfp::GnArgs a{};
+  a.x = x; a.N = n_patches; a.pix_per_patch = pix_per_patch; a.C = C; a.G = groups; a.eps = eps;
+  a.part = part; a.counter = counter;
+  a.fresh_out = fresh_moments; a.stale = stale_moments ? stale_moments : fresh_moments;
+  a.gamma = gamma; a.beta = beta; a.coef = coef;
+  a.dbg = mean_rstd ? mean_rstd : coef + coef_need;   // unused tail of the coef region when not wanted
+  a.is_sync = stale_moments ? 0 : 1; a.mode = (int)mode; a.naive = 0;
+  if (!mean_rstd && coef_need + (size_t)n_patches * groups * 2 > kCoefFloats)
+    return fail(DFP_E_ARG, "pass mean_rstd: no room left in the fixed scratch for the statistics");
+  if (dtype == DFP_BF16) {
+    e = dfp::launch_gn_stats_merge<__nv_bfloat16>(a, s);
+    if (e == cudaSuccess)
+      e = dfp::launch_gn_apply<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y),
+                                              nullptr, coef, n_patches, pix_per_patch, C, W, pix_per_patch, 0,
+                                              apply_silu != 0, 0, s);
+  } else {
+    e = dfp::launch_gn_stats_merge<float>(a, s);
+    if (e == cudaSuccess)
+      e = dfp::launch_gn_apply<float>(static_cast<const float*>(x), static_cast<float*>(y), nullptr, coef,
+                                      n_patches, pix_per_patch, C, W, pix_per_patch, 0, apply_silu != 0, 0, s);
+  }
+  if (e != cudaSuccess) return fail(DFP_E_CUDA, std::string("launch: ") + cudaGetErrorString(e));
+  return DFP_OK;
+}

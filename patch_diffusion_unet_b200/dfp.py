@@ -22,7 +22,7 @@ FAMILY_TENSOR_CORE, FAMILY_SIMT = 0, 1
 EXPORTED = ("dfp_create", "dfp_load_weights", "dfp_step", "dfp_step_host", "dfp_output",
             "dfp_copy_out", "dfp_buffer_bytes", "dfp_check_device", "dfp_launches_per_step",
             "dfp_set_kernel_family", "dfp_set_profiling", "dfp_kernel_times", "dfp_destroy",
-            "dfp_last_error")
+            "dfp_last_error", "dfp_group_norm_noalloc", "dfp_group_norm_noalloc_error")
 
 
 class Config(ctypes.Structure):
@@ -61,6 +61,11 @@ def load_library(path=_LIB_PATH):
         "dfp_kernel_times": ([H, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_char_p), ctypes.c_int],
                              ctypes.c_int),
         "dfp_destroy": ([H], ctypes.c_int),
+        "dfp_group_norm_noalloc": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_void_p,
+                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+        "dfp_group_norm_noalloc_error": ([], ctypes.c_char_p),
         "dfp_last_error": ([H], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
