@@ -354,7 +354,9 @@ class SDXLStage(_StepProtocol):
         out = dict(resnet=r.reshape(H, W, C).copy())
         for p, sa, ca in self.blocks:
             r = r + sa(layer_norm(r, w[p + "norm1.weight"], w[p + "norm1.bias"]), is_sync)
+            out[p + "sa"] = r.reshape(H, W, C).copy()
             r = r + ca(layer_norm(r, w[p + "norm2.weight"], w[p + "norm2.bias"]))
+            out[p + "ca"] = r.reshape(H, W, C).copy()
             r = r + self._ffn(p, layer_norm(r, w[p + "norm3.weight"], w[p + "norm3.bias"]))
             out[p + "out"] = r.reshape(H, W, C).copy()
         out["y"] = r

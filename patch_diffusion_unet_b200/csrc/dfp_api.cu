@@ -24,15 +24,19 @@
 #include <cuda_bf16.h>
 
 #include "../../include/dfp.h"
+#include "handle.h"
 #include "kernels.h"
 
 using namespace dfp;
+
+namespace dfp {
+size_t dtype_size(dfp_dtype d) { return d == DFP_BF16 ? 2 : 4; }
+}  // namespace dfp
 
 namespace {
 
 thread_local std::string g_create_error;
 
-size_t dtype_size(dfp_dtype d) { return d == DFP_BF16 ? 2 : 4; }
 
 float bf16_bits_to_f32(uint16_t b) {
   uint32_t u = (uint32_t)b << 16;
@@ -49,61 +53,6 @@ uint16_t f32_to_bf16_bits(float f) {
 }
 
 }  // namespace
-
-struct dfp_ctx {
-  dfp_config cfg{};
-  cudaStream_t stream = nullptr;
-  std::string err;
-  int R = 0, L = 0, Lp = 0, family = 0;
-  size_t esz = 4;
-  // weights
-  void* w_conv = nullptr;   // [C][9][C]
-  float* b_conv = nullptr;
-  void* w_qkv = nullptr;    // [3C][C]
-  void* w_o = nullptr;      // [C][C]
-  float* b_o = nullptr;
-  float *gn1_g = nullptr, *gn1_b = nullptr, *gn2_g = nullptr, *gn2_b = nullptr;
-  std::set<std::string> loaded;
-  // activations and caches
-  void* slab[2] = {nullptr, nullptr};
-  void *h = nullptr, *t = nullptr, *q = nullptr, *o = nullptr, *y = nullptr, *xin = nullptr;
-  void* kb[2] = {nullptr, nullptr};
-  void* vb[2] = {nullptr, nullptr};
-  float *mom1[2] = {nullptr, nullptr}, *mom2[2] = {nullptr, nullptr};
-  float *coef = nullptr, *dbg1 = nullptr, *dbg2 = nullptr, *part = nullptr;
-  unsigned* counter = nullptr;
-  int* dev_err = nullptr;
-  // split-KV attention scratch
-  int attn_splits = 1;
-  float *attn_part_o = nullptr, *attn_part_ml = nullptr;
-  unsigned* attn_counters = nullptr;
-  std::vector<void*> allocs;
-  int last_step = -1;
-  int launches = 0;
-  // per-launch timing (dfp_set_profiling)
-  static constexpr int kMaxEv = 24;
-  bool profiling = false;
-  cudaEvent_t ev[kMaxEv] = {};
-  const char* ev_name[kMaxEv] = {};
-  int n_ev = 0;
-  // TMA descriptors (bf16 only)
-  CUtensorMap m_slab[2], m_wconv, m_t, m_wqkv, m_o, m_wo, m_q, m_k[2], m_v[2];
-  TcGemmPlan conv_plan{}, qkv_plan{}, out_plan{};
-
-  dfp_status fail(dfp_status s, const std::string& msg) {
-    err = msg;
-    return s;
-  }
-  dfp_status cuda_fail(cudaError_t e, const char* where) {
-    err = std::string(where) + ": " + cudaGetErrorString(e);
-    return DFP_E_CUDA;
-  }
-  bool alloc(void** p, size_t bytes) {
-    if (cudaMalloc(p, bytes) != cudaSuccess) { *p = nullptr; return false; }
-    allocs.push_back(*p);
-    return true;
-  }
-};
 
 namespace {
 
@@ -124,8 +73,15 @@ dfp_status check_config(const dfp_config* c, std::string& why) {
   const long long Lp = (long long)(c->H / c->n_patches) * c->W;
   if (Lp % 8) return bad("(H / n_patches) * W must be a multiple of 8");
   if ((long long)c->H * c->W * c->C > (1ll << 31)) return bad("feature map too large (H*W*C >= 2^31)");
-  if (c->block == DFP_BLOCK_SDXL_STAGE) { why = "the transformer stage block is not built yet"; return DFP_E_UNSUPPORTED; }
-  if (c->block != DFP_BLOCK_RES_ATTN) return bad("unknown block type");
+  if (c->block == DFP_BLOCK_SDXL_STAGE) {
+    if (c->dtype != DFP_BF16) { why = "the transformer stage is built for bf16 storage only"; return DFP_E_UNSUPPORTED; }
+    if (c->n_xformer < 1 || c->n_xformer > 2) return bad("n_xformer must be 1 or 2");
+    if (c->ffn_inner <= 0 || c->ffn_inner % 64) return bad("ffn_inner must be a positive multiple of 64");
+    if (c->ctx_len <= 0 || c->ctx_dim <= 0 || c->ctx_dim % 8) return bad("ctx_len > 0 and ctx_dim a positive multiple of 8");
+    if (c->C > 2048) return bad("C must be <= 2048 for the transformer stage");
+  } else if (c->block != DFP_BLOCK_RES_ATTN) {
+    return bad("unknown block type");
+  }
   return DFP_OK;
 }
 
@@ -185,12 +141,13 @@ dfp_status build_tmaps(dfp_ctx* h) {
 }
 
 // ------------------------------------------------------------------ weights
-struct WeightSpec {
-  const char* name;
-  std::vector<long long> shape;
-};
 
-std::vector<WeightSpec> weight_specs(const dfp_config& c) {
+std::vector<WeightSpec> res_attn_weight_specs(const dfp_config& c);
+std::vector<WeightSpec> weight_specs(dfp_ctx* h) {
+  if (h->cfg.block == DFP_BLOCK_SDXL_STAGE) return stage_weight_specs(h->cfg, h->spec_names);
+  return res_attn_weight_specs(h->cfg);
+}
+std::vector<WeightSpec> res_attn_weight_specs(const dfp_config& c) {
   const long long C = c.C;
   return {
       {"gn1.weight", {C}}, {"gn1.bias", {C}}, {"conv1.weight", {C, C, 3, 3}}, {"conv1.bias", {C}},
@@ -248,28 +205,31 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
   h->family = cfg->dtype == DFP_BF16 ? 0 : 1;
   const size_t C = cfg->C, N = cfg->n_patches, G = cfg->gn_groups, W = cfg->W, R = h->R, L = h->L;
   const size_t map = L * C * h->esz;
+  const bool is_stage = cfg->block == DFP_BLOCK_SDXL_STAGE;
   bool ok = true;
-  ok &= h->alloc(&h->w_conv, 9 * C * C * h->esz);
-  ok &= h->alloc((void**)&h->b_conv, C * 4);
-  ok &= h->alloc(&h->w_qkv, 3 * C * C * h->esz);
-  ok &= h->alloc(&h->w_o, C * C * h->esz);
-  ok &= h->alloc((void**)&h->b_o, C * 4);
-  ok &= h->alloc((void**)&h->gn1_g, C * 4);
-  ok &= h->alloc((void**)&h->gn1_b, C * 4);
-  ok &= h->alloc((void**)&h->gn2_g, C * 4);
-  ok &= h->alloc((void**)&h->gn2_b, C * 4);
-  for (int i = 0; i < 2; ++i) {
-    ok &= h->alloc(&h->slab[i], N * (R + 2) * W * C * h->esz);
-    ok &= h->alloc(&h->kb[i], map);
-    ok &= h->alloc(&h->vb[i], map);
-    ok &= h->alloc((void**)&h->mom1[i], N * G * 2 * 4);
-    ok &= h->alloc((void**)&h->mom2[i], N * G * 2 * 4);
+  if (!is_stage) {
+    ok &= h->alloc(&h->w_conv, 9 * C * C * h->esz);
+    ok &= h->alloc((void**)&h->b_conv, C * 4);
+    ok &= h->alloc(&h->w_qkv, 3 * C * C * h->esz);
+    ok &= h->alloc(&h->w_o, C * C * h->esz);
+    ok &= h->alloc((void**)&h->b_o, C * 4);
+    ok &= h->alloc((void**)&h->gn1_g, C * 4);
+    ok &= h->alloc((void**)&h->gn1_b, C * 4);
+    ok &= h->alloc((void**)&h->gn2_g, C * 4);
+    ok &= h->alloc((void**)&h->gn2_b, C * 4);
+    for (int i = 0; i < 2; ++i) {
+      ok &= h->alloc(&h->slab[i], N * (R + 2) * W * C * h->esz);
+      ok &= h->alloc(&h->kb[i], map);
+      ok &= h->alloc(&h->vb[i], map);
+      ok &= h->alloc((void**)&h->mom1[i], N * G * 2 * 4);
+      ok &= h->alloc((void**)&h->mom2[i], N * G * 2 * 4);
+    }
+    ok &= h->alloc(&h->h, map);
+    ok &= h->alloc(&h->t, map);
+    ok &= h->alloc(&h->y, map);
   }
-  ok &= h->alloc(&h->h, map);
-  ok &= h->alloc(&h->t, map);
   ok &= h->alloc(&h->q, map);
   ok &= h->alloc(&h->o, map);
-  ok &= h->alloc(&h->y, map);
   ok &= h->alloc(&h->xin, map);
   ok &= h->alloc((void**)&h->coef, N * C * 2 * 4);
   ok &= h->alloc((void**)&h->dbg1, N * G * 2 * 4);
@@ -296,9 +256,13 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
   // zero everything the kernels rely on: slab halo rows at the image edges, the
   // GroupNorm block counter, the device error word, and all caches
   cudaError_t e = cudaSuccess;
-  for (void* p : {h->slab[0], h->slab[1]})
-    if (e == cudaSuccess) e = cudaMemset(p, 0, N * (R + 2) * W * C * h->esz);
-  for (void* p : {h->kb[0], h->kb[1], h->vb[0], h->vb[1], h->h, h->t, h->q, h->o, h->y})
+  if (!is_stage) {
+    for (void* p : {h->slab[0], h->slab[1]})
+      if (e == cudaSuccess) e = cudaMemset(p, 0, N * (R + 2) * W * C * h->esz);
+    for (void* p : {h->kb[0], h->kb[1], h->vb[0], h->vb[1], h->h, h->t, h->y})
+      if (e == cudaSuccess) e = cudaMemset(p, 0, map);
+  }
+  for (void* p : {h->q, h->o})
     if (e == cudaSuccess) e = cudaMemset(p, 0, map);
   if (e == cudaSuccess) e = cudaMemset(h->counter, 0, 64);
   if (e == cudaSuccess) e = cudaMemset(h->dev_err, 0, 64);
@@ -308,13 +272,15 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
     dfp_destroy(h);
     return DFP_E_CUDA;
   }
-  if (cfg->dtype == DFP_BF16) {
+  if (is_stage) {
+    st = stage_create(h);
+  } else if (cfg->dtype == DFP_BF16) {
     st = build_tmaps(h);
-    if (st != DFP_OK) {
-      g_create_error = h->err;
-      dfp_destroy(h);
-      return st;
-    }
+  }
+  if (st != DFP_OK) {
+    g_create_error = h->err;
+    dfp_destroy(h);
+    return st;
   }
   *out = h;
   return DFP_OK;
@@ -324,7 +290,7 @@ dfp_status dfp_load_weights(dfp_handle h, const dfp_tensor* w, int n) {
   if (!h) return DFP_E_ARG;
   if (n < 0 || (n > 0 && !w)) return h->fail(DFP_E_ARG, "bad weight list");
   const dfp_config& c = h->cfg;
-  const std::vector<WeightSpec> specs = weight_specs(c);
+  const std::vector<WeightSpec> specs = weight_specs(h);
   for (int i = 0; i < n; ++i) {
     const dfp_tensor& t = w[i];
     if (!t.name || !t.ptr) return h->fail(DFP_E_ARG, "weight with NULL name or pointer");
@@ -352,6 +318,13 @@ dfp_status dfp_load_weights(dfp_handle h, const dfp_tensor* w, int n) {
     std::vector<float> v;
     read_as_float(src, t.dtype, numel, v);
     const std::string name = t.name;
+    if (h->stage) {
+      dfp_status lst = DFP_OK;
+      if (!stage_load_weight(h, name, v, lst)) return h->fail(DFP_E_ARG, "unknown weight name " + name);
+      if (lst != DFP_OK) return lst;
+      h->loaded.insert(name);
+      continue;
+    }
     const size_t C = c.C;
     void* dst = nullptr;
     std::vector<uint8_t> bytes;
@@ -388,6 +361,7 @@ dfp_status dfp_load_weights(dfp_handle h, const dfp_tensor* w, int n) {
     if (e != cudaSuccess) return h->cuda_fail(e, "weight copy to device");
     h->loaded.insert(name);
   }
+  if (h->stage) return stage_finish_load(h);
   return DFP_OK;
 }
 
@@ -396,13 +370,14 @@ dfp_status dfp_step(dfp_handle h, const void* x, int step, int is_sync) {
   if (!x) return h->fail(DFP_E_ARG, "x is NULL");
   if (is_sync != 0 && is_sync != 1) return h->fail(DFP_E_ARG, "is_sync must be 0 or 1");
   if (step < 0) return h->fail(DFP_E_ARG, "step must be >= 0");
-  if (h->loaded.size() != weight_specs(h->cfg).size())
+  if (h->loaded.size() != weight_specs(h).size())
     return h->fail(DFP_E_STATE, "weights not loaded (every weight must be given before the first step)");
   if (step == 0 && !is_sync) return h->fail(DFP_E_STATE, "step 0 must be synchronous: the context cache is empty");
   if (step != 0 && step != h->last_step + 1)
     return h->fail(DFP_E_STATE, "steps must be consecutive (or restart at 0)");
-  dfp_status st = h->cfg.dtype == DFP_BF16 ? run_step<__nv_bfloat16>(h, x, step, is_sync)
-                                           : run_step<float>(h, x, step, is_sync);
+  dfp_status st = h->stage ? stage_step(h, x, step, is_sync)
+                 : h->cfg.dtype == DFP_BF16 ? run_step<__nv_bfloat16>(h, x, step, is_sync)
+                                            : run_step<float>(h, x, step, is_sync);
   if (st == DFP_OK) h->last_step = step;
   return st;
 }
@@ -434,6 +409,12 @@ static bool buffer_of(dfp_handle h, const char* name, const void** ptr, long lon
   const long long st = (long long)h->cfg.n_patches * h->cfg.gn_groups * 2 * 4;
   const int cur = h->last_step < 0 ? 0 : (h->last_step & 1);
   const std::string n = name;
+  if (h->stage) {
+    if (stage_buffer(h, n, ptr, bytes)) return true;
+    if (n == "gn1" || n == "gn2") { *ptr = n == "gn1" ? h->dbg1 : h->dbg2; *bytes = st; return true; }
+    if (n == "q" || n == "o") { *ptr = n == "q" ? h->q : h->o; *bytes = map; return true; }
+    return false;
+  }
   if (n == "y") { *ptr = h->y; *bytes = map; }
   else if (n == "h") { *ptr = h->h; *bytes = map; }
   else if (n == "t") { *ptr = h->t; *bytes = map; }
@@ -534,6 +515,7 @@ dfp_status dfp_destroy(dfp_handle h) {
   for (int i = 0; i < dfp_ctx::kMaxEv; ++i)
     if (h->ev[i]) cudaEventDestroy(h->ev[i]);
   for (void* p : h->allocs) cudaFree(p);
+  delete_stage(h->stage);
   delete h;
   return DFP_OK;
 }
@@ -561,16 +543,6 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   int launches = 0;
   cudaError_t e;
   h->n_ev = 0;
-#define DFP_LAUNCH(call, what)                                   \
-  do {                                                           \
-    if (h->profiling && launches + 1 < dfp_ctx::kMaxEv) {        \
-      cudaEventRecord(h->ev[launches], s);                       \
-      h->ev_name[launches] = what;                               \
-    }                                                            \
-    e = (call);                                                  \
-    if (e != cudaSuccess) return h->cuda_fail(e, what);          \
-    ++launches;                                                  \
-  } while (0)
 
   // ---- GN1 statistics (+ corrected merge) and apply + SiLU into the slab interior
   GnArgs g{};
@@ -630,12 +602,7 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   } else {
     DFP_LAUNCH(launch_simt_gemm<T>(static_cast<const T*>(h->o), nullptr, static_cast<const T*>(h->w_o), L, C, C, eo, s), "out projection (simt)");
   }
-#undef DFP_LAUNCH
-  if (h->profiling && launches < dfp_ctx::kMaxEv) {
-    cudaEventRecord(h->ev[launches], s);
-    h->n_ev = launches + 1;
-  }
-  h->launches = launches;
+  DFP_LAUNCH_END();
   return DFP_OK;
 }
 

@@ -272,6 +272,52 @@ __global__ void halo_refresh_kernel(const T* __restrict__ src, T* __restrict__ d
 }
 
 // Pixels per block: one wave of 512-thread blocks over the whole map.
+// Per-token LayerNorm (transformer blocks of the SDXL-style stage): one warp per
+// token, the token's C channels held in registers (16-byte vectors), mean and
+// biased variance by warp butterflies (deterministic), fp32 math, bf16 in/out.
+template <int KMAX>
+__global__ void __launch_bounds__(256)
+layernorm_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ y,
+                 const float* __restrict__ gamma, const float* __restrict__ beta, int L, int C, float eps) {
+  const int tok = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (tok >= L) return;
+  const int nvec = C / 8;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)tok * C);
+  float v[KMAX][8];
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < KMAX; ++k) {
+    const int i = lane + 32 * k;
+    if (i < nvec) {
+      unpack16(ld_nc16(src + i), v[k]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s += v[k][e];
+    }
+  }
+  const float mean = warp_sum(s) / (float)C;
+  float q = 0.f;
+#pragma unroll
+  for (int k = 0; k < KMAX; ++k) {
+    if (lane + 32 * k < nvec) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { const float d = v[k][e] - mean; q = fmaf(d, d, q); }
+    }
+  }
+  const float rstd = 1.f / sqrtf(warp_sum(q) / (float)C + eps);
+  uint4* dst = reinterpret_cast<uint4*>(y + (size_t)tok * C);
+#pragma unroll
+  for (int k = 0; k < KMAX; ++k) {
+    const int i = lane + 32 * k;
+    if (i < nvec) {
+      float o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = (v[k][e] - mean) * rstd * __ldg(gamma + i * 8 + e) + __ldg(beta + i * 8 + e);
+      dst[i] = pack16(o);
+    }
+  }
+}
+
 int chunk_pixels(int N, int pix_per_patch) {
   const int target_blocks = 148;
   int per = (N * pix_per_patch + target_blocks - 1) / target_blocks;
@@ -329,6 +375,19 @@ cudaError_t launch_halo_refresh(const T* src_slab, T* dst_slab, int N, int R, in
   if (bx > 64) bx = 64;
   dim3 grid(bx, 2 * (N - 1));
   halo_refresh_kernel<T><<<grid, threads, 0, s>>>(src_slab, dst_slab, R, W, C);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_layernorm(const void* x, void* y, const float* gamma, const float* beta, int L, int C,
+                             float eps, cudaStream_t s) {
+  if (C % 8 || C > 2048) return cudaErrorInvalidValue;
+  const dim3 grid((L + 7) / 8);
+  const auto* xi = static_cast<const __nv_bfloat16*>(x);
+  auto* yo = static_cast<__nv_bfloat16*>(y);
+  if (C <= 1024)
+    layernorm_kernel<4><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps);
+  else
+    layernorm_kernel<8><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps);
   return cudaGetLastError();
 }
 

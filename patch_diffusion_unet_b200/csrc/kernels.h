@@ -7,7 +7,7 @@
 namespace dfp {
 
 // Attention context mode of one launch.
-enum AttnMode : int { kAttnSync = 0, kAttnDisplaced = 1, kAttnNaive = 2 };
+enum AttnMode : int { kAttnSync = 0, kAttnDisplaced = 1, kAttnNaive = 2, kAttnCross = 3 };
 
 // ---------------------------------------------------------------- GroupNorm
 struct GnArgs {
@@ -36,13 +36,22 @@ template <typename T>
 cudaError_t launch_halo_refresh(const T* src_slab, T* dst_slab, int N, int R, int W, int C,
                                 cudaStream_t s);
 
+// Per-token LayerNorm over C channels (biased variance), bf16 in / out, fp32 math.
+cudaError_t launch_layernorm(const void* x, void* y, const float* gamma, const float* beta, int L, int C,
+                             float eps, cudaStream_t s);
+
 // ---------------------------------------------------------------- GEMM epilogues
 struct Epilogue {
-  int kind;               // 0: out[m, n] = acc + bias[n] (bias may be null); 1: Q/K/V scatter
-  void* out;              // kind 0: [M, ldo]
+  // 0: out[m, n] = acc + bias[n] (+ residual[m, n]); bias / residual may be null
+  // 1: Q/K/V scatter: column n -> (n / C: 0 q, 1 k, 2 v; head; d) into [heads][L][64]
+  // 2: GEGLU: the 128 columns of a tile are 64 values then the 64 matching gates;
+  //    out[m, n0/2 + j] = (v_j + bias) * GELU(g_j + bias), GELU exact (erf)
+  int kind;
+  void* out;              // kinds 0, 2: [M, ldo]
   const float* bias;
+  const void* residual;   // kind 0: [M, ldo] bf16, may alias out (same element read then written)
   int ldo;
-  void* q; void* k; void* v;  // kind 1: [heads][L][64] each; column n -> (n / C, head, d)
+  void* q; void* k; void* v;
   int L, C;
 };
 // A operand of the conv: the haloed per-patch slab [N][R+2][W][Cin]; row m of the
@@ -83,6 +92,7 @@ cudaError_t launch_tc_gemm(const TcGemmPlan& plan, const CUtensorMap& mapA, cons
 
 struct TcAttnArgs {
   int L, Lp, N, heads, C, mode;
+  int kv_len;             // cross-attention: number of context tokens (mode kAttnCross)
   void* o;                // [L, C] bf16
   int* err;
   int splits;             // CTAs sharing the KV tile list of one Q-tile pair

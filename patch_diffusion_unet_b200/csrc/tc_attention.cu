@@ -62,7 +62,7 @@ struct Segs {
   int total;
 };
 
-__device__ __forceinline__ Segs make_segs(int mode, int p, int Lp, int L) {
+__device__ __forceinline__ Segs make_segs(int mode, int p, int Lp, int L, int kv_len) {
   Segs s{};
   auto add = [&](int st, int b, int len) {
     if (len <= 0) return;
@@ -73,6 +73,8 @@ __device__ __forceinline__ Segs make_segs(int mode, int p, int Lp, int L) {
   };
   if (mode == kAttnSync) {
     add(0, 0, L);
+  } else if (mode == kAttnCross) {
+    add(0, 0, kv_len);        // the fixed context: same for every patch, never stale
   } else {
     add(0, p * Lp, Lp);
     if (mode == kAttnDisplaced) {
@@ -236,7 +238,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
   int* err = a.err;
 
   if (threadIdx.x == 0) {
-    s_segs = make_segs(a.mode, p, a.Lp, a.L);
+    s_segs = make_segs(a.mode, p, a.Lp, a.L, a.kv_len);
     s_abort = 0;
     mbar_init(smem_u32(q_full), 1);
     for (int i = 0; i < kStages; ++i) {
@@ -599,7 +601,7 @@ int attention_splits(int L, int Lp, int N, int heads, int mode_min_tiles) {
     const long waves = (items + 147) / 148;
     const double eff = (double)items / (double)(waves * 148);
     if (eff > best_eff + 0.03) { best_eff = eff; best = s; }
-    if (eff >= 0.85) break;
+    if (eff >= 0.7) break;   // each split adds a CTA prologue and a merge: stop early
   }
   return best;
 }

@@ -165,6 +165,33 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     }
     if (!ready || s_abort) gm = -1;
     const uint32_t taddr = tmem_d + ((uint32_t)(sub * 32) << 16);
+    if (BN == 128 && epi.kind == 2) {
+      // GEGLU: columns [0, 64) are values, [64, 128) the gates of the same features
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t rv[32], rg[32];
+        tmem_ld32(taddr + c * 32, rv);
+        tmem_ld32(taddr + 64 + c * 32, rg);
+        tmem_wait_ld();
+        if (gm < 0) continue;
+        const int nv = n0 + c * 32, ng = n0 + 64 + c * 32;
+        float w[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float a = __uint_as_float(rv[i]) + __ldg(epi.bias + nv + i);
+          const float g = __uint_as_float(rg[i]) + __ldg(epi.bias + ng + i);
+          w[i] = a * (0.5f * g * (1.f + erff(g * 0.70710678118654752f)));
+        }
+        uint4* d4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(epi.out) + gm * epi.ldo + n0 / 2 + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float w8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w8[e] = w[i * 8 + e];
+          d4[i] = pack16(w8);
+        }
+      }
+    } else
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
       uint32_t r[32];
@@ -180,6 +207,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         if (epi.bias) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] += __ldg(epi.bias + n + i);
+        }
+        if (epi.residual) {
+          const uint4* r4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(epi.residual) + gm * epi.ldo + n);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float rr[8];
+            unpack16(r4[i], rr);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[i * 8 + e] += rr[e];
+          }
         }
         dst = static_cast<__nv_bfloat16*>(epi.out) + gm * epi.ldo + n;
       } else {

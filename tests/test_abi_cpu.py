@@ -55,12 +55,15 @@ def test_create_rejects_bad_config(over, frag):
     assert not h.value
 
 
-def test_create_rejects_unbuilt_block():
+def test_create_rejects_fp32_stage_and_bad_stage_sizes():
     from patch_diffusion_unet_b200 import dfp
-    cfg = configs.get(4)
-    c = dfp.make_config(cfg)
     h = ctypes.c_void_p()
+    c = dfp.make_config(configs.get(4, dtype="f32"))
     assert dfp.LIB.dfp_create(ctypes.byref(c), None, ctypes.byref(h)) == dfp.E_UNSUPPORTED
+    c = dfp.make_config(configs.get(4, ffn_inner=100))
+    assert dfp.LIB.dfp_create(ctypes.byref(c), None, ctypes.byref(h)) == dfp.E_ARG
+    c = dfp.make_config(configs.get(4, n_xformer=3))
+    assert dfp.LIB.dfp_create(ctypes.byref(c), None, ctypes.byref(h)) == dfp.E_ARG
 
 
 def test_null_arguments():
