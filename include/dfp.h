@@ -175,14 +175,15 @@ DFP_API int dfp_kernel_times(dfp_handle h, float* ms, const char** names, int ma
  *   fresh_moments   device fp32 [N, G, 2], out: this call's moments
  *   mean_rstd       device fp32 [N, G, 2], out: the (mean, 1/std) applied, or NULL
  *   cuda_stream     cudaStream_t the work is enqueued on (asynchronous)
- * Scratch comes from a fixed 1 MiB array in the library's device memory (held by
+ * Scratch comes from a fixed 256 KiB array in the library's device memory (held by
  * every GPU that loads the library until exit).  The first call on a device, with
  * that device current, looks up the array's device address; make that first call
  * before any stream capture begins.  All calls share the array and it keeps the
  * last call's contents (the counter that must start at zero is cleared by every
- * call), so calls that overlap on the GPU race.  Limits: n_patches * groups <= 256,
- * n_patches * C <= 81920, and the (patch, group, block) partials <= 98304 floats;
- * larger requests return DFP_E_ARG with the reason in
+ * call), so calls that overlap on the GPU race.  Limits: n_patches * groups <= 256
+ * and the (patch, group, block) partial sums <= 64960 floats (about
+ * n_patches * groups * 2 * min(148 / n_patches + 1, pixels per patch / 16)); larger
+ * requests return DFP_E_ARG with the reason in
  * dfp_group_norm_noalloc_error().  Never calls cudaMalloc or cudaFree. */
 DFP_API dfp_status dfp_group_norm_noalloc(const void* x, void* y, dfp_dtype dtype, int H, int W, int C,
                                           int n_patches, int groups, float eps, const float* gamma,

@@ -10,7 +10,6 @@
 //   k[2], v[2]  [heads][L][64]   keys / values, alternating by step parity
 //   o, y        [L][C]           attention output, block output
 //   mom1/2[2]   [N][G][2] fp32   per-(patch, group) (E[x], E[x^2]) of GN1 / GN2, alternating
-//   coef        [N][C][2] fp32   per-(patch, channel) GroupNorm scale and shift
 //   part        fp32 scratch     per-chunk partial sums of the GroupNorm statistics
 #include <cmath>
 #include <cstdio>
@@ -94,13 +93,6 @@ void conv_tiles(int R, int W, int& cols_tile, int& rows_tile, int& tiles_per_row
   while (R % rows_tile) --rows_tile;
 }
 
-int pick_bn(int N) {
-  if (N % 128 == 0 && N / 128 >= 8) return 128;
-  if (N % 160 == 0) return 160;
-  if (N % 128 == 0) return 128;
-  return 64;
-}
-
 dfp_status build_tmaps(dfp_ctx* h) {
   const dfp_config& c = h->cfg;
   const int C = c.C, W = c.W, N = c.n_patches, R = h->R, L = h->L;
@@ -113,12 +105,14 @@ dfp_status build_tmaps(dfp_ctx* h) {
     const uint32_t box[4] = {64, (uint32_t)cols_tile, (uint32_t)rows_tile, 1};
     ok &= encode_tmap_4d(&h->m_slab[i], h->slab[i], dims, str, box);
   }
-  const int bn_conv = pick_bn(C), bn_qkv = pick_bn(3 * C), bn_out = pick_bn(C);
-  ok &= encode_tmap_2d(&h->m_wconv, h->w_conv, 9ull * C, C, 9ull * C * 2, 64, bn_conv);
-  ok &= encode_tmap_2d(&h->m_t, h->t, C, L, (uint64_t)C * 2, 64, 128);
-  ok &= encode_tmap_2d(&h->m_wqkv, h->w_qkv, C, 3ull * C, (uint64_t)C * 2, 64, bn_qkv);
-  ok &= encode_tmap_2d(&h->m_o, h->o, C, L, (uint64_t)C * 2, 64, 128);
-  ok &= encode_tmap_2d(&h->m_wo, h->w_o, C, C, (uint64_t)C * 2, 64, bn_out);
+  const int conv_m_tiles = N * (R / rows_tile) * tpr, lin_m_tiles = gemm_m_tiles_plain(L);
+  const int bn_conv = choose_bn(C, conv_m_tiles), bn_qkv = choose_bn(3 * C, lin_m_tiles),
+            bn_out = choose_bn(C, lin_m_tiles);
+  ok &= encode_gemm_rows(&h->m_wconv, h->w_conv, C, 9ull * C, bn_conv);
+  ok &= encode_gemm_rows(&h->m_t, h->t, L, C, 128);
+  ok &= encode_gemm_rows(&h->m_wqkv, h->w_qkv, 3ull * C, C, bn_qkv);
+  ok &= encode_gemm_rows(&h->m_o, h->o, L, C, 128);
+  ok &= encode_gemm_rows(&h->m_wo, h->w_o, C, C, bn_out);
   const int heads = c.heads;
   ok &= encode_tmap_3d(&h->m_q, h->q, 64, L, heads, 128, (uint64_t)L * 128, 64, 128, 1);
   for (int i = 0; i < 2; ++i) {
@@ -231,7 +225,6 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
   ok &= h->alloc(&h->q, map);
   ok &= h->alloc(&h->o, map);
   ok &= h->alloc(&h->xin, map);
-  ok &= h->alloc((void**)&h->coef, N * C * 2 * 4);
   ok &= h->alloc((void**)&h->dbg1, N * G * 2 * 4);
   ok &= h->alloc((void**)&h->dbg2, N * G * 2 * 4);
   ok &= h->alloc((void**)&h->part, N * (size_t)gn_stats_chunks((int)N, (int)(R * W)) * G * 2 * 4);
@@ -549,13 +542,13 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   g.x = x; g.N = N; g.pix_per_patch = Lp; g.C = C; g.G = G; g.eps = c.gn_eps;
   g.part = h->part; g.counter = h->counter;
   g.fresh_out = h->mom1[cur]; g.stale = h->mom1[prv];
-  g.gamma = h->gn1_g; g.beta = h->gn1_b; g.coef = h->coef; g.dbg = h->dbg1;
+  g.gamma = h->gn1_g; g.beta = h->gn1_b; g.dbg = h->dbg1;
   g.is_sync = is_sync; g.mode = (int)c.gn_mode; g.naive = naive ? 1 : 0;
   DFP_LAUNCH(launch_gn_stats_merge<T>(g, s), "gn1 statistics");
   // the same kernel fills the halo rows: the neighbours' boundary rows of this step
   // (sync) or of the previous step (displaced, read from the other slab buffer)
   const int halo_mode = (naive || N == 1) ? 0 : (displaced ? 2 : 1);
-  DFP_LAUNCH(launch_gn_apply<T>(x, slab, static_cast<const T*>(h->slab[prv]), h->coef, N, Lp, C, W,
+  DFP_LAUNCH(launch_gn_apply<T>(x, slab, static_cast<const T*>(h->slab[prv]), h->dbg1, h->gn1_g, h->gn1_b, G, N, Lp, C, W,
                                 (long long)(R + 2) * W, W, true, halo_mode, s), "gn1 apply + halo");
   // ---- conv3x3 (+ bias) -> h
   Epilogue ec{};
@@ -570,7 +563,7 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   g.x = h->h; g.fresh_out = h->mom2[cur]; g.stale = h->mom2[prv];
   g.gamma = h->gn2_g; g.beta = h->gn2_b; g.dbg = h->dbg2;
   DFP_LAUNCH(launch_gn_stats_merge<T>(g, s), "gn2 statistics");
-  DFP_LAUNCH(launch_gn_apply<T>(static_cast<const T*>(h->h), static_cast<T*>(h->t), nullptr, h->coef, N, Lp,
+  DFP_LAUNCH(launch_gn_apply<T>(static_cast<const T*>(h->h), static_cast<T*>(h->t), nullptr, h->dbg2, h->gn2_g, h->gn2_b, G, N, Lp,
                                 C, W, (long long)Lp, 0, false, 0, s), "gn2 apply");
   // ---- Q, K, V projections; K/V land in this step's cache buffers
   Epilogue eq{};

@@ -34,7 +34,6 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
   constexpr int VEC = VecTraits<T>::kN;
   extern __shared__ float sh[];                 // [2][PL][C] lane sums, then [2][C] channel sums
   __shared__ float s_mom[256 * 2];              // merged fresh moments  [N*G][2]
-  __shared__ float s_mr[256 * 2];               // (mean, rstd)          [N*G][2]
   __shared__ int s_last;
   const int C = a.C, G = a.G, N = a.N;
   const int V = C / VEC;
@@ -52,11 +51,12 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
     const int pix0 = chunk * pix_per_chunk;
     const int pix1 = min(pix0 + pix_per_chunk, a.pix_per_patch);
     const T* base = static_cast<const T*>(a.x) + (size_t)p * a.pix_per_patch * C + vc * VEC;
-    int pix = pix0 + pl;
-    for (; pix + 7 * PL < pix1; pix += 8 * PL) {
+    // eight predicated loads in flight per thread, then accumulate in pixel order
+    for (int pix = pix0 + pl; pix < pix1; pix += 8 * PL) {
       uint4 u[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) u[j] = ld_nc16(base + (size_t)(pix + j * PL) * C);
+      for (int j = 0; j < 8; ++j)
+        u[j] = pix + j * PL < pix1 ? ld_nc16(base + (size_t)(pix + j * PL) * C) : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         float v[VEC];
@@ -64,12 +64,6 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
 #pragma unroll
         for (int i = 0; i < VEC; ++i) { s1[i] += v[i]; s2[i] = fmaf(v[i], v[i], s2[i]); }
       }
-    }
-    for (; pix < pix1; pix += PL) {
-      float v[VEC];
-      unpack16(ld_nc16(base + (size_t)pix * C), v);
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) { s1[i] += v[i]; s2[i] = fmaf(v[i], v[i], s2[i]); }
     }
     float4* d1 = reinterpret_cast<float4*>(sh + pl * C + vc * VEC);
     float4* d2 = reinterpret_cast<float4*>(sh + PL * C + pl * C + vc * VEC);
@@ -93,12 +87,13 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
     for (int c = lane; c < cg; c += 32) { t1 += chan[g * cg + c]; t2 += chan[C + g * cg + c]; }
     t1 = warp_sum(t1);
     t2 = warp_sum(t2);
-    if (lane == 0)
+    if (lane == 0) {
       reinterpret_cast<float2*>(a.part)[((size_t)p * n_chunks + chunk) * G + g] = make_float2(t1, t2);
+      __threadfence();                          // only the writers need to publish
+    }
   }
 
   // ---- phase 2: the last block to finish merges every partial in a fixed order
-  __threadfence();
   __syncthreads();
   if (tid == 0) s_last = (atomicAdd(a.counter, 1u) == gridDim.x * gridDim.y - 1);
   __syncthreads();
@@ -160,17 +155,8 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
     }
     const float var = fmaxf(e2 - e1 * e1, 0.f);
     const float rstd = 1.f / sqrtf(var + a.eps);
-    s_mr[tid * 2] = e1;
-    s_mr[tid * 2 + 1] = rstd;
     a.dbg[tid * 2] = e1;
     a.dbg[tid * 2 + 1] = rstd;
-  }
-  __syncthreads();
-  for (int i = tid; i < N * C; i += kGnThreads) {
-    const int pp = i / C, c = i % C, gg = c / cg;
-    const float mean = s_mr[(pp * G + gg) * 2], rstd = s_mr[(pp * G + gg) * 2 + 1];
-    const float sc = a.gamma[c] * rstd;
-    reinterpret_cast<float2*>(a.coef)[i] = make_float2(sc, a.beta[c] - mean * sc);
   }
   if (tid == 0) *a.counter = 0u;
 }
@@ -201,7 +187,8 @@ __device__ __forceinline__ void write_halos(T* out, const T* prev_slab, const ui
 template <typename T, bool SILU>
 __global__ void __launch_bounds__(kGnThreads)
 gn_apply_kernel(const T* __restrict__ x, T* __restrict__ out, const T* __restrict__ prev_slab,
-                const float* __restrict__ coef, int pix_per_patch, int C, long long out_patch_stride,
+                const float* __restrict__ mean_rstd, const float* __restrict__ gamma,
+                const float* __restrict__ beta, int G, int pix_per_patch, int C, long long out_patch_stride,
                 long long out_off, int pix_per_chunk, int W, int N, int halo_mode) {
   constexpr int VEC = VecTraits<T>::kN;
   const int V = C / VEC;
@@ -209,10 +196,16 @@ gn_apply_kernel(const T* __restrict__ x, T* __restrict__ out, const T* __restric
   const int vc = threadIdx.x % V, pl = threadIdx.x / V;
   if (pl >= PL) return;
   const int p = blockIdx.y, chunk = blockIdx.x;
+  // per-channel scale and shift of this thread's channels from the group (mean, rstd)
   float sc[VEC], sf[VEC];
-  const float2* cf = reinterpret_cast<const float2*>(coef) + (size_t)p * C + vc * VEC;
+  const int cg = C / G;
 #pragma unroll
-  for (int i = 0; i < VEC; ++i) { const float2 t = cf[i]; sc[i] = t.x; sf[i] = t.y; }
+  for (int i = 0; i < VEC; ++i) {
+    const int c = vc * VEC + i;
+    const float2 mr = reinterpret_cast<const float2*>(mean_rstd)[p * G + c / cg];
+    sc[i] = __ldg(gamma + c) * mr.y;
+    sf[i] = __ldg(beta + c) - mr.x * sc[i];
+  }
   const int pix0 = chunk * pix_per_chunk;
   const int pix1 = min(pix0 + pix_per_chunk, pix_per_patch);
   const T* src = x + (size_t)p * pix_per_patch * C + vc * VEC;
@@ -220,13 +213,15 @@ gn_apply_kernel(const T* __restrict__ x, T* __restrict__ out, const T* __restric
   const int last_row0 = pix_per_patch - W;
   const bool top_src = halo_mode != 0 && p > 0;          // my first row feeds patch p-1
   const bool bot_src = halo_mode != 0 && p < N - 1;      // my last row feeds patch p+1
-  int pix = pix0 + pl;
-  for (; pix + 3 * PL < pix1; pix += 4 * PL) {
+  for (int pix = pix0 + pl; pix < pix1; pix += 4 * PL) {
     uint4 u[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) u[j] = ld_nc16(src + (size_t)(pix + j * PL) * C);
+    for (int j = 0; j < 4; ++j)
+      u[j] = pix + j * PL < pix1 ? ld_nc16(src + (size_t)(pix + j * PL) * C) : make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
+      const int q = pix + j * PL;
+      if (q >= pix1) break;
       float v[VEC];
       unpack16(u[j], v);
 #pragma unroll
@@ -235,24 +230,10 @@ gn_apply_kernel(const T* __restrict__ x, T* __restrict__ out, const T* __restric
         if (SILU) v[i] = silu_f(v[i]);
       }
       const uint4 o = pack16(v);
-      const int q = pix + j * PL;
       *reinterpret_cast<uint4*>(dst + (size_t)q * C) = o;
       if (halo_mode != 0) write_halos(out, prev_slab, o, p, q, pix_per_patch, last_row0, W, C, vc * VEC,
                                       out_patch_stride, out_off, top_src, bot_src, halo_mode);
     }
-  }
-  for (; pix < pix1; pix += PL) {
-    float v[VEC];
-    unpack16(ld_nc16(src + (size_t)pix * C), v);
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) {
-      v[i] = fmaf(v[i], sc[i], sf[i]);
-      if (SILU) v[i] = silu_f(v[i]);
-    }
-    const uint4 o = pack16(v);
-    *reinterpret_cast<uint4*>(dst + (size_t)pix * C) = o;
-    if (halo_mode != 0) write_halos(out, prev_slab, o, p, pix, pix_per_patch, last_row0, W, C, vc * VEC,
-                                    out_patch_stride, out_off, top_src, bot_src, halo_mode);
   }
 }
 
@@ -348,19 +329,20 @@ cudaError_t launch_gn_stats_merge(const GnArgs& a, cudaStream_t s) {
 }
 
 template <typename T>
-cudaError_t launch_gn_apply(const T* x, T* out, const T* prev_slab, const float* coef, int N,
-                            int pix_per_patch, int C, int W, long long out_patch_stride_pix,
-                            long long out_pix_off, bool silu, int halo_mode, cudaStream_t s) {
+cudaError_t launch_gn_apply(const T* x, T* out, const T* prev_slab, const float* mean_rstd, const float* gamma,
+                            const float* beta, int G, int N, int pix_per_patch, int C, int W,
+                            long long out_patch_stride_pix, long long out_pix_off, bool silu, int halo_mode,
+                            cudaStream_t s) {
   const int per = chunk_pixels(N, pix_per_patch);
   dim3 grid((pix_per_patch + per - 1) / per, N);
   if (silu)
-    gn_apply_kernel<T, true><<<grid, kGnThreads, 0, s>>>(x, out, prev_slab, coef, pix_per_patch, C,
-                                                         out_patch_stride_pix, out_pix_off, per, W, N,
-                                                         halo_mode);
+    gn_apply_kernel<T, true><<<grid, kGnThreads, 0, s>>>(x, out, prev_slab, mean_rstd, gamma, beta, G,
+                                                         pix_per_patch, C, out_patch_stride_pix, out_pix_off,
+                                                         per, W, N, halo_mode);
   else
-    gn_apply_kernel<T, false><<<grid, kGnThreads, 0, s>>>(x, out, prev_slab, coef, pix_per_patch, C,
-                                                          out_patch_stride_pix, out_pix_off, per, W, N,
-                                                          halo_mode);
+    gn_apply_kernel<T, false><<<grid, kGnThreads, 0, s>>>(x, out, prev_slab, mean_rstd, gamma, beta, G,
+                                                          pix_per_patch, C, out_patch_stride_pix, out_pix_off,
+                                                          per, W, N, halo_mode);
   return cudaGetLastError();
 }
 
@@ -393,13 +375,13 @@ cudaError_t launch_layernorm(const void* x, void* y, const float* gamma, const f
 
 template cudaError_t launch_gn_stats_merge<float>(const GnArgs&, cudaStream_t);
 template cudaError_t launch_gn_stats_merge<__nv_bfloat16>(const GnArgs&, cudaStream_t);
-template cudaError_t launch_gn_apply<float>(const float*, float*, const float*, const float*, int,
-                                            int, int, int, long long, long long, bool, int,
-                                            cudaStream_t);
+template cudaError_t launch_gn_apply<float>(const float*, float*, const float*, const float*, const float*,
+                                            const float*, int, int, int, int, int, long long, long long,
+                                            bool, int, cudaStream_t);
 template cudaError_t launch_gn_apply<__nv_bfloat16>(const __nv_bfloat16*, __nv_bfloat16*,
-                                                    const __nv_bfloat16*, const float*, int, int,
-                                                    int, int, long long, long long, bool, int,
-                                                    cudaStream_t);
+                                                    const __nv_bfloat16*, const float*, const float*,
+                                                    const float*, int, int, int, int, int, long long,
+                                                    long long, bool, int, cudaStream_t);
 template cudaError_t launch_halo_refresh<float>(const float*, float*, int, int, int, int,
                                                 cudaStream_t);
 template cudaError_t launch_halo_refresh<__nv_bfloat16>(const __nv_bfloat16*, __nv_bfloat16*, int,

@@ -37,7 +37,7 @@ struct dfp_ctx {
   void* kb[2] = {nullptr, nullptr};
   void* vb[2] = {nullptr, nullptr};
   float *mom1[2] = {nullptr, nullptr}, *mom2[2] = {nullptr, nullptr};
-  float *coef = nullptr, *dbg1 = nullptr, *dbg2 = nullptr, *part = nullptr;
+  float *dbg1 = nullptr, *dbg2 = nullptr, *part = nullptr;   // dbg = (mean, rstd) per (patch, group)
   unsigned* counter = nullptr;
   int* dev_err = nullptr;
   // split-KV attention scratch

@@ -20,8 +20,7 @@ struct GnArgs {
   const float* stale;     // [N][G][2] moments of step t-1 (read on displaced steps)
   const float* gamma;     // [C] fp32
   const float* beta;      // [C] fp32
-  float* coef;            // [N][C][2] per (patch, channel) (scale, shift)
-  float* dbg;             // [N][G][2] (mean, rstd) used, for inspection
+  float* dbg;             // [N][G][2] (mean, rstd) used -- read by the apply kernel
   int is_sync, mode, naive;
 };
 int gn_stats_chunks(int N, int pix_per_patch);
@@ -29,9 +28,10 @@ template <typename T> cudaError_t launch_gn_stats_merge(const GnArgs& a, cudaStr
 // halo_mode: 0 none (plain output), 1 sync (fresh neighbour rows), 2 displaced
 // (the previous step's rows, read from prev_slab)
 template <typename T>
-cudaError_t launch_gn_apply(const T* x, T* out, const T* prev_slab, const float* coef, int N,
-                            int pix_per_patch, int C, int W, long long out_patch_stride_pix,
-                            long long out_pix_off, bool silu, int halo_mode, cudaStream_t s);
+cudaError_t launch_gn_apply(const T* x, T* out, const T* prev_slab, const float* mean_rstd, const float* gamma,
+                            const float* beta, int G, int N, int pix_per_patch, int C, int W,
+                            long long out_patch_stride_pix, long long out_pix_off, bool silu, int halo_mode,
+                            cudaStream_t s);
 template <typename T>
 cudaError_t launch_halo_refresh(const T* src_slab, T* dst_slab, int N, int R, int W, int C,
                                 cudaStream_t s);
@@ -78,6 +78,8 @@ bool encode_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, 
                     uint64_t s1_bytes, uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
 bool encode_tmap_4d(CUtensorMap* m, const void* base, const uint64_t dims[4],
                     const uint64_t strides_bytes[3], const uint32_t box[4]);
+// GEMM operand: row-major [rows][K] bf16, K a multiple of 64; box = box_rows x two 64-wide K chunks
+bool encode_gemm_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows);
 
 struct TcGemmPlan {
   int M, N, K;            // GEMM sizes (conv: M = H*W, K = 9*Cin)
@@ -86,9 +88,14 @@ struct TcGemmPlan {
   // conv geometry
   int P, R, W, Cin;       // patches, rows per patch, width, input channels
   int cols_tile, rows_tile, tiles_per_row;
+  int m_tiles;            // filled by launch_tc_gemm
+  int sms;                // persistent grid size (SM count), filled by launch_tc_gemm
 };
 cudaError_t launch_tc_gemm(const TcGemmPlan& plan, const CUtensorMap& mapA, const CUtensorMap& mapB,
                            const Epilogue& epi, int* err, cudaStream_t s);
+// N-tile width (160, 128 or 64, dividing N) minimising waves x bytes moved per k-block.
+int choose_bn(int N, int m_tiles);
+int gemm_m_tiles_plain(int M);
 
 struct TcAttnArgs {
   int L, Lp, N, heads, C, mode;

@@ -7,12 +7,12 @@
 // region), or a host that must not take the allocator's locks on its critical
 // path.  The regular path (dfp_create / dfp_step) allocates its scratch when the
 // handle is made; this entry point instead takes its scratch -- the per-block
-// partial sums, the block-arrival counter and the per-channel scale/shift -- from
-// one fixed array compiled into the library.  The caller passes only inputs and
-// outputs.
+// partial sums, the block-arrival counter and, when the caller does not want them,
+// the per-(patch, group) mean / rstd -- from one fixed array compiled into the
+// library.  The caller passes only inputs and outputs.
 //
 // The array (g_noalloc_scratch below) is file-scope device memory: every GPU that
-// loads the library holds its 1 MiB until the process exits.  Its host-side name
+// loads the library holds its 256 KiB until the process exits.  Its host-side name
 // is only a stand-in, so the device address is looked up with
 // cudaGetSymbolAddress, once per device, by the first call made with that device
 // current; make that first call before any stream capture begins.  All calls on a
@@ -32,9 +32,9 @@ namespace {
 
 // Layout of the scratch, in floats.
 constexpr size_t kCounterFloats = 64;                 // arrival counter (first word), padded
-constexpr size_t kPartFloats = 98304;                 // per-block partial (sum x, sum x^2)
-constexpr size_t kCoefFloats = 163840;                // per-(patch, channel) (scale, shift)
-constexpr size_t kScratchFloats = kCounterFloats + kPartFloats + kCoefFloats;   // 1 MiB
+constexpr size_t kPartFloats = 64960;                 // per-block partial (sum x, sum x^2)
+constexpr size_t kStatFloats = 512;                   // (mean, rstd) per (patch, group), N*G <= 256
+constexpr size_t kScratchFloats = kCounterFloats + kPartFloats + kStatFloats;   // 256 KiB
 
 static __device__ __align__(256) float g_noalloc_scratch[kScratchFloats];
 
@@ -74,13 +74,9 @@ extern "C" DFP_API dfp_status dfp_group_norm_noalloc(const void* x, void* y, dfp
   const int pix_per_patch = (H / n_patches) * W;
   const int n_chunks = dfp::gn_stats_chunks(n_patches, pix_per_patch);
   const size_t part_need = (size_t)n_patches * n_chunks * groups * 2;
-  const size_t coef_need = (size_t)n_patches * C * 2;
   if (part_need > kPartFloats)
     return fail(DFP_E_ARG, "too many (patch, group, block) partials for the fixed scratch (" +
                                std::to_string(part_need) + " > " + std::to_string(kPartFloats) + " floats)");
-  if (coef_need > kCoefFloats)
-    return fail(DFP_E_ARG, "n_patches * C too large for the fixed scratch (2 * n_patches * C must be <= " +
-                               std::to_string(kCoefFloats) + ")");
 
   // ---- once per device: the device address of the scratch array
   int dev = 0;
@@ -102,7 +98,7 @@ extern "C" DFP_API dfp_status dfp_group_norm_noalloc(const void* x, void* y, dfp
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   unsigned* counter = reinterpret_cast<unsigned*>(base);
   float* part = base + kCounterFloats;
-  float* coef = part + kPartFloats;
+  float* stats = part + kPartFloats;
 
   // the arrival counter must start at zero (the kernel also leaves it at zero)
   e = cudaMemsetAsync(counter, 0, sizeof(unsigned), s);
@@ -112,22 +108,23 @@ extern "C" DFP_API dfp_status dfp_group_norm_noalloc(const void* x, void* y, dfp
   a.x = x; a.N = n_patches; a.pix_per_patch = pix_per_patch; a.C = C; a.G = groups; a.eps = eps;
   a.part = part; a.counter = counter;
   a.fresh_out = fresh_moments; a.stale = stale_moments ? stale_moments : fresh_moments;
-  a.gamma = gamma; a.beta = beta; a.coef = coef;
-  a.dbg = mean_rstd ? mean_rstd : coef + coef_need;   // unused tail of the coef region when not wanted
+  a.gamma = gamma; a.beta = beta;
+  float* mr = mean_rstd ? mean_rstd : stats;  // the (mean, rstd) the apply step reads
+  a.dbg = mr;
   a.is_sync = stale_moments ? 0 : 1; a.mode = (int)mode; a.naive = 0;
-  if (!mean_rstd && coef_need + (size_t)n_patches * groups * 2 > kCoefFloats)
-    return fail(DFP_E_ARG, "pass mean_rstd: no room left in the fixed scratch for the statistics");
   if (dtype == DFP_BF16) {
     e = dfp::launch_gn_stats_merge<__nv_bfloat16>(a, s);
     if (e == cudaSuccess)
       e = dfp::launch_gn_apply<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y),
-                                              nullptr, coef, n_patches, pix_per_patch, C, W, pix_per_patch, 0,
+                                              nullptr, mr, gamma, beta, groups, n_patches, pix_per_patch, C, W,
+                                              pix_per_patch, 0,
                                               apply_silu != 0, 0, s);
   } else {
     e = dfp::launch_gn_stats_merge<float>(a, s);
     if (e == cudaSuccess)
-      e = dfp::launch_gn_apply<float>(static_cast<const float*>(x), static_cast<float*>(y), nullptr, coef,
-                                      n_patches, pix_per_patch, C, W, pix_per_patch, 0, apply_silu != 0, 0, s);
+      e = dfp::launch_gn_apply<float>(static_cast<const float*>(x), static_cast<float*>(y), nullptr, mr, gamma,
+                                      beta, groups, n_patches, pix_per_patch, C, W, pix_per_patch, 0,
+                                      apply_silu != 0, 0, s);
   }
   if (e != cudaSuccess) return fail(DFP_E_CUDA, std::string("launch: ") + cudaGetErrorString(e));
   return DFP_OK;

@@ -58,13 +58,6 @@ struct Stage {
 
 namespace {
 
-int pick_bn_stage(int N) {
-  if (N % 128 == 0 && N / 128 >= 8) return 128;
-  if (N % 160 == 0) return 160;
-  if (N % 128 == 0) return 128;
-  return 64;
-}
-
 uint16_t f32_to_bf16(float f) {
   uint32_t u;
   std::memcpy(&u, &f, 4);
@@ -183,12 +176,13 @@ dfp_status stage_create(dfp_ctx* h) {
     ok &= encode_tmap_4d(&st->m_slab1[i], st->slab1[i], dims, strides, box);
     ok &= encode_tmap_4d(&st->m_slab2[i], st->slab2[i], dims, strides, box);
   }
-  const int bn_c = pick_bn_stage((int)C);
-  ok &= encode_tmap_2d(&st->m_wc1, st->w_c1, 9 * C, C, 9 * C * 2, 64, bn_c);
-  ok &= encode_tmap_2d(&st->m_wc2, st->w_c2, 9 * C, C, 9 * C * 2, 64, bn_c);
-  ok &= encode_tmap_2d(&st->m_u, st->u, C, L, C * 2, 64, 128);
-  ok &= encode_tmap_2d(&st->m_o, h->o, C, L, C * 2, 64, 128);
-  ok &= encode_tmap_2d(&st->m_g, st->g, F, L, F * 2, 64, 128);
+  const int lin_m = gemm_m_tiles_plain((int)L);
+  const int bn_c = choose_bn((int)C, (int)N * ((int)R / rows_tile) * tpr);
+  ok &= encode_gemm_rows(&st->m_wc1, st->w_c1, C, 9 * C, bn_c);
+  ok &= encode_gemm_rows(&st->m_wc2, st->w_c2, C, 9 * C, bn_c);
+  ok &= encode_gemm_rows(&st->m_u, st->u, L, C, 128);
+  ok &= encode_gemm_rows(&st->m_o, h->o, L, C, 128);
+  ok &= encode_gemm_rows(&st->m_g, st->g, L, F, 128);
   ok &= encode_tmap_3d(&h->m_q, h->q, 64, L, heads, 128, L * 128, 64, 128, 1);
   auto plan = [&](TcGemmPlan& p, int M, int Nn, int K, int bn) {
     p = TcGemmPlan{};
@@ -196,13 +190,13 @@ dfp_status stage_create(dfp_ctx* h) {
   };
   for (int b = 0; b < c.n_xformer; ++b) {
     XfBlock& x = st->xf[b];
-    const int bq = pick_bn_stage(3 * (int)C), bc = pick_bn_stage((int)C);
-    ok &= encode_tmap_2d(&x.m_wqkv, x.w_qkv, C, 3 * C, C * 2, 64, bq);
-    ok &= encode_tmap_2d(&x.m_wo1, x.w_o1, C, C, C * 2, 64, bc);
-    ok &= encode_tmap_2d(&x.m_wq2, x.w_q2, C, C, C * 2, 64, bc);
-    ok &= encode_tmap_2d(&x.m_wo2, x.w_o2, C, C, C * 2, 64, bc);
-    ok &= encode_tmap_2d(&x.m_wff1, x.w_ff1, C, 2 * F, C * 2, 64, 128);
-    ok &= encode_tmap_2d(&x.m_wff2, x.w_ff2, F, C, F * 2, 64, bc);
+    const int bq = choose_bn(3 * (int)C, lin_m), bc = choose_bn((int)C, lin_m);
+    ok &= encode_gemm_rows(&x.m_wqkv, x.w_qkv, 3 * C, C, bq);
+    ok &= encode_gemm_rows(&x.m_wo1, x.w_o1, C, C, bc);
+    ok &= encode_gemm_rows(&x.m_wq2, x.w_q2, C, C, bc);
+    ok &= encode_gemm_rows(&x.m_wo2, x.w_o2, C, C, bc);
+    ok &= encode_gemm_rows(&x.m_wff1, x.w_ff1, 2 * F, C, 128);
+    ok &= encode_gemm_rows(&x.m_wff2, x.w_ff2, C, F, bc);   // same N = C as to_out
     for (int i = 0; i < 2; ++i) {
       ok &= encode_tmap_3d(&x.m_k[i], x.kb[i], 64, L, heads, 128, L * 128, 64, 128, 1);
       ok &= encode_tmap_3d(&x.m_v[i], x.vb[i], 64, L, heads, 128, L * 128, 64, 128, 1);
@@ -332,12 +326,13 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   // ---- ResNet block: GN1 + SiLU -> conv1 -> GN2 + SiLU -> conv2 + x
   GnArgs g{};
   g.x = xv; g.N = N; g.pix_per_patch = Lp; g.C = C; g.G = G; g.eps = c.gn_eps;
-  g.part = h->part; g.counter = h->counter; g.coef = h->coef;
+  g.part = h->part; g.counter = h->counter;
   g.is_sync = is_sync; g.mode = (int)c.gn_mode; g.naive = naive ? 1 : 0;
   g.fresh_out = st->mom1[cur]; g.stale = st->mom1[prv]; g.gamma = st->n1_g; g.beta = st->n1_b; g.dbg = h->dbg1;
   DFP_LAUNCH(launch_gn_stats_merge<bf>(g, s), "norm1 statistics");
   DFP_LAUNCH(launch_gn_apply<bf>(static_cast<const bf*>(xv), static_cast<bf*>(st->slab1[cur]),
-                                 static_cast<const bf*>(st->slab1[prv]), h->coef, N, Lp, C, W, (long long)(R + 2) * W,
+                                 static_cast<const bf*>(st->slab1[prv]), h->dbg1, st->n1_g, st->n1_b, G, N, Lp, C, W,
+                                 (long long)(R + 2) * W,
                                  W, true, halo_mode, s), "norm1 apply + halo");
   Epilogue ec{};
   ec.kind = 0; ec.out = st->h1; ec.bias = st->b_c1; ec.ldo = C;
@@ -346,7 +341,8 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   g.dbg = h->dbg2;
   DFP_LAUNCH(launch_gn_stats_merge<bf>(g, s), "norm2 statistics");
   DFP_LAUNCH(launch_gn_apply<bf>(static_cast<const bf*>(st->h1), static_cast<bf*>(st->slab2[cur]),
-                                 static_cast<const bf*>(st->slab2[prv]), h->coef, N, Lp, C, W, (long long)(R + 2) * W,
+                                 static_cast<const bf*>(st->slab2[prv]), h->dbg2, st->n2_g, st->n2_b, G, N, Lp, C, W,
+                                 (long long)(R + 2) * W,
                                  W, true, halo_mode, s), "norm2 apply + halo");
   ec.out = st->r[0]; ec.bias = st->b_c2; ec.residual = xv;
   DFP_LAUNCH(launch_tc_gemm(st->p_c2, st->m_slab2[cur], st->m_wc2, ec, h->dev_err, s), "conv2 + residual (tcgen05)");

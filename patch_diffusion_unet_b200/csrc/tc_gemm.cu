@@ -1,4 +1,7 @@
 // Tensor-core (tcgen05 / TMEM / TMA) GEMM for sm_100a, bf16 operands, fp32 accumulate.
+// A pipeline stage carries two 64-wide K chunks (one TMA box of two chunks for the
+// row-major operands, two 4-D boxes for the conv slab), halving TMA instructions and
+// barrier hand-offs per FLOP.
 //
 // One kernel serves two contractions of the layer step:
 //  * the displaced conv3x3 as an implicit GEMM (DistriConv2dPP, "DistriFusion源码探秘"
@@ -49,13 +52,105 @@ __device__ __forceinline__ TileInfo tile_of(const TcGemmPlan& pl, int m_tile) {
   return t;
 }
 
+// Epilogue of one tile: drain the 128 x BN accumulator at TMEM column `acc` and store.
+template <int BN>
+__device__ __forceinline__ void epilogue_tile(const TcGemmPlan& plan, const Epilogue& epi, const TileInfo& tile,
+                                              int n0, uint32_t taddr, int row, bool valid_tile) {
+  long long gm = -1;
+  if (plan.conv) {
+    const int rr = row / plan.cols_tile, jj = row - rr * plan.cols_tile;
+    if (rr < plan.rows_tile && tile.j0 + jj < plan.W)
+      gm = ((long long)tile.p * plan.R + tile.i0 + rr) * plan.W + tile.j0 + jj;
+  } else if (tile.m0 + row < plan.M) {
+    gm = tile.m0 + row;
+  }
+  if (!valid_tile) gm = -1;
+  if (BN == 128 && epi.kind == 2) {
+    // GEGLU: columns [0, 64) are values, [64, 128) the gates of the same features
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      uint32_t rv[32], rg[32];
+      tmem_ld32(taddr + c * 32, rv);
+      tmem_ld32(taddr + 64 + c * 32, rg);
+      tmem_wait_ld();
+      if (gm < 0) continue;
+      const int nv = n0 + c * 32, ng = n0 + 64 + c * 32;
+      float w[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float av = __uint_as_float(rv[i]) + __ldg(epi.bias + nv + i);
+        const float g = __uint_as_float(rg[i]) + __ldg(epi.bias + ng + i);
+        w[i] = av * (0.5f * g * (1.f + erff(g * 0.70710678118654752f)));
+      }
+      uint4* d4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(epi.out) + gm * epi.ldo + n0 / 2 + c * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float w8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w8[e] = w[i * 8 + e];
+        d4[i] = pack16(w8);
+      }
+    }
+    return;
+  }
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c * 32, r);
+    tmem_wait_ld();
+    const int n = n0 + c * 32;
+    if (gm < 0 || n >= plan.N) continue;
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+    __nv_bfloat16* dst;
+    if (epi.kind == 0) {
+      if (epi.bias) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] += __ldg(epi.bias + n + i);
+      }
+      if (epi.residual) {
+        const uint4* r4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(epi.residual) + gm * epi.ldo + n);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float rr[8];
+          unpack16(r4[i], rr);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[i * 8 + e] += rr[e];
+        }
+      }
+      dst = static_cast<__nv_bfloat16*>(epi.out) + gm * epi.ldo + n;
+    } else {
+      const int which = n / epi.C, cc = n - which * epi.C;
+      const int head = cc >> 6, d0 = cc & 63;
+      void* base = which == 0 ? epi.q : (which == 1 ? epi.k : epi.v);
+      dst = static_cast<__nv_bfloat16*>(base) + ((long long)head * epi.L + gm) * 64 + d0;
+    }
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float w8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w8[e] = v[i * 8 + e];
+      d4[i] = pack16(w8);
+    }
+  }
+}
+
+// Persistent: CTA b takes tiles b, b + gridDim.x, ...  Two TMEM accumulators let the
+// epilogue of tile i overlap the main loop of tile i + 1; the TMA ring runs on across
+// tiles.  Tile t = (m_tile = t / n_tiles_n, n_tile = t % n_tiles_n): the CTAs in flight
+// share A tiles (all N tiles of an M tile are neighbours) and all share the weights.
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                const TcGemmPlan plan, const Epilogue epi, int* err) {
-  constexpr uint32_t kABytes = kBM * kBK * 2;
-  constexpr uint32_t kBBytes = BN * kBK * 2;
-  constexpr uint32_t kCols = TmemCols<BN>::v;
+  // A stage holds two 64-wide K chunks: [chunk][rows][64] for A (16 KB per chunk) and for B
+  constexpr uint32_t kAChunk = kBM * kBK * 2;
+  constexpr uint32_t kBChunk = BN * kBK * 2;
+  constexpr uint32_t kABytes = 2 * kAChunk;
+  constexpr uint32_t kBBytes = 2 * kBChunk;
+  constexpr uint32_t kCols = TmemCols<BN>::v;            // one accumulator
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -63,25 +158,30 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * kBBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
-  uint64_t* accum = bars + 2 * STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
-  __shared__ int s_abort;
+  uint64_t* acc_full = bars + 2 * STAGES;                // [2]
+  uint64_t* acc_empty = bars + 2 * STAGES + 2;           // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  __shared__ volatile int s_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN;
-  const TileInfo tile = tile_of(plan, blockIdx.y);
-  const int num_kb = plan.K / kBK;
+  const int n_tiles_n = plan.N / BN;
+  const int n_tiles = plan.m_tiles * n_tiles_n;
+  // K stages of two chunks; the conv pairs chunks within a tap (an odd last chunk of a
+  // tap reads zeros past the channel count: A is zero there, so B's chunk does not matter)
+  const int cpt = plan.conv ? plan.Cin / kBK : 0;                 // chunks per tap
+  const int ppt = (cpt + 1) / 2;                                  // chunk pairs per tap
+  const int num_kb = plan.conv ? 9 * ppt : (plan.K / kBK + 1) / 2;
   const uint32_t a_box_bytes =
-      plan.conv ? (uint32_t)(plan.rows_tile * plan.cols_tile * kBK * 2) : kABytes;
+      plan.conv ? (uint32_t)(2 * plan.rows_tile * plan.cols_tile * kBK * 2) : kABytes;
 
   if (threadIdx.x == 0) {
     s_abort = 0;
     for (int s = 0; s < STAGES; ++s) { mbar_init(smem_u32(&full[s]), 1); mbar_init(smem_u32(&empty[s]), 1); }
-    mbar_init(smem_u32(accum), 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(&acc_full[i]), 1); mbar_init(smem_u32(&acc_empty[i]), 128); }
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), kCols);
+    tmem_alloc(smem_u32(tmem_slot), 2 * kCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -94,145 +194,85 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     if (lane == 0) {
       tma_prefetch_desc(&mapA);
       tma_prefetch_desc(&mapB);
-      const int kc_per_tap = plan.conv ? plan.Cin / kBK : 1;
-      int issued = 0;
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const int s = kb % STAGES, round = kb / STAGES;
-        if (round > 0 && !mbar_wait(smem_u32(&empty[s]), (round - 1) & 1, err, kErrWaitStageFree)) {
-          s_abort = 1;
-          break;
+      int kg = 0;   // k-stages issued so far (ring position)
+      for (int t = blockIdx.x; t < n_tiles && !s_abort; t += gridDim.x) {
+        const TileInfo tile = tile_of(plan, t / n_tiles_n);
+        const int n0 = (t % n_tiles_n) * BN;
+        for (int kb = 0; kb < num_kb; ++kb, ++kg) {
+          const int s = kg % STAGES, round = kg / STAGES;
+          if (round > 0 && !mbar_wait(smem_u32(&empty[s]), (round - 1) & 1, err, kErrWaitStageFree)) {
+            s_abort = 1;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full[s]);
+          mbar_arrive_expect_tx(fb, a_box_bytes + kBBytes);
+          if (plan.conv) {
+            const int tap = kb / ppt, kc = 2 * (kb - tap * ppt);
+            const int r = tap / 3, sx = tap - 3 * (tap / 3);
+            const uint32_t da = smem_u32(sA + s * kABytes);
+            tma_load_4d(da, &mapA, fb, kc * kBK, tile.j0 + sx - 1, tile.i0 + r, tile.p);
+            tma_load_4d(da + kAChunk, &mapA, fb, (kc + 1) * kBK, tile.j0 + sx - 1, tile.i0 + r, tile.p);
+            tma_load_3d(smem_u32(sB + s * kBBytes), &mapB, fb, 0, n0, tap * cpt + kc);
+          } else {
+            tma_load_3d(smem_u32(sA + s * kABytes), &mapA, fb, 0, tile.m0, 2 * kb);
+            tma_load_3d(smem_u32(sB + s * kBBytes), &mapB, fb, 0, n0, 2 * kb);
+          }
         }
-        const uint32_t fb = smem_u32(&full[s]);
-        mbar_arrive_expect_tx(fb, a_box_bytes + kBBytes);
-        if (plan.conv) {
-          const int tap = kb / kc_per_tap, kc = kb - tap * kc_per_tap;
-          const int r = tap / 3, sx = tap - 3 * (tap / 3);
-          tma_load_4d(smem_u32(sA + s * kABytes), &mapA, fb, kc * kBK, tile.j0 + sx - 1, tile.i0 + r, tile.p);
-        } else {
-          tma_load_2d(smem_u32(sA + s * kABytes), &mapA, fb, kb * kBK, tile.m0);
-        }
-        tma_load_2d(smem_u32(sB + s * kBBytes), &mapB, fb, kb * kBK, n0);
-        ++issued;
       }
       if (s_abort) {
         // let the copies already in flight land before the CTA can exit
-        for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
-          mbar_wait(smem_u32(&full[kb % STAGES]), (kb / STAGES) & 1, err, kErrWaitTmaFull);
+        for (int k = (kg > STAGES ? kg - STAGES : 0); k < kg; ++k)
+          mbar_wait(smem_u32(&full[k % STAGES]), (k / STAGES) & 1, err, kErrWaitTmaFull);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      // The stage ring is unrolled so that every MMA operand is a hoisted descriptor
-      // plus a compile-time offset: runtime arithmetic between tcgen05.mma
-      // instructions stalls their issue.
       constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, false, false);
       const uint64_t ad0 = sw128_kmajor_desc(smem_u32(sA));
       const uint64_t bd0 = sw128_kmajor_desc(smem_u32(sB));
       bool ok = true;
-      for (int kb0 = 0; ok && kb0 < num_kb; kb0 += STAGES) {
-        const uint32_t par = (uint32_t)(kb0 / STAGES) & 1u;
-#pragma unroll
-        for (int s = 0; s < STAGES; ++s) {
-          const int kb = kb0 + s;
-          if (kb >= num_kb) break;
-          if (!mbar_wait(smem_u32(&full[s]), par, err, kErrWaitTmaFull)) { ok = false; break; }
+      int kg = 0, ti = 0;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++ti) {
+        const int buf = ti & 1, use = ti >> 1;
+        if (use > 0 && !mbar_wait(smem_u32(&acc_empty[buf]), (use - 1) & 1, err, kErrWaitAccum)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d = tmem_d + buf * kCols;
+        for (int kb = 0; kb < num_kb; ++kb, ++kg) {
+          const int s = kg % STAGES, round = kg / STAGES;
+          if (!mbar_wait(smem_u32(&full[s]), round & 1, err, kErrWaitTmaFull)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t ad = ad0 + (uint64_t)((s * kABytes) >> 4);
-          const uint64_t bd = bd0 + (uint64_t)((s * kBBytes) >> 4);
-          umma_f16_ss(tmem_d, ad, bd, idesc, kb > 0);
+          // operands: per-stage bases, compile-time offsets per K slice
+          const uint64_t ad = ad0 + (uint64_t)s * (kABytes >> 4);
+          const uint64_t bd = bd0 + (uint64_t)s * (kBBytes >> 4);
+          umma_f16_ss(d, ad, bd, idesc, kb > 0);
 #pragma unroll
-          for (int kk = 1; kk < kBK / 16; ++kk) umma_f16_ss(tmem_d, ad + 2 * kk, bd + 2 * kk, idesc, 1);
+          for (int kk = 1; kk < kBK / 16; ++kk) umma_f16_ss(d, ad + 2 * kk, bd + 2 * kk, idesc, 1);
+          const uint64_t ad1 = ad + (kAChunk >> 4), bd1 = bd + (kBChunk >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) umma_f16_ss(d, ad1 + 2 * kk, bd1 + 2 * kk, idesc, 1);
           umma_commit(smem_u32(&empty[s]));
         }
+        umma_commit(smem_u32(&acc_full[buf]));
       }
       if (!ok) s_abort = 1;
-      umma_commit(smem_u32(accum));
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2..5)
     const int sub = warp & 3;
     const int row = sub * 32 + lane;
-    const bool ready = mbar_wait(smem_u32(accum), 0, err, kErrWaitAccum);
-    tc_fence_after();
-    long long gm = -1;
-    if (plan.conv) {
-      const int rr = row / plan.cols_tile, jj = row - rr * plan.cols_tile;
-      if (rr < plan.rows_tile && tile.j0 + jj < plan.W)
-        gm = ((long long)tile.p * plan.R + tile.i0 + rr) * plan.W + tile.j0 + jj;
-    } else if (tile.m0 + row < plan.M) {
-      gm = tile.m0 + row;
-    }
-    if (!ready || s_abort) gm = -1;
-    const uint32_t taddr = tmem_d + ((uint32_t)(sub * 32) << 16);
-    if (BN == 128 && epi.kind == 2) {
-      // GEGLU: columns [0, 64) are values, [64, 128) the gates of the same features
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t rv[32], rg[32];
-        tmem_ld32(taddr + c * 32, rv);
-        tmem_ld32(taddr + 64 + c * 32, rg);
-        tmem_wait_ld();
-        if (gm < 0) continue;
-        const int nv = n0 + c * 32, ng = n0 + 64 + c * 32;
-        float w[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float a = __uint_as_float(rv[i]) + __ldg(epi.bias + nv + i);
-          const float g = __uint_as_float(rg[i]) + __ldg(epi.bias + ng + i);
-          w[i] = a * (0.5f * g * (1.f + erff(g * 0.70710678118654752f)));
-        }
-        uint4* d4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(epi.out) + gm * epi.ldo + n0 / 2 + c * 32);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float w8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) w8[e] = w[i * 8 + e];
-          d4[i] = pack16(w8);
-        }
-      }
-    } else
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      uint32_t r[32];
-      tmem_ld32(taddr + c * 32, r);
-      tmem_wait_ld();
-      const int n = n0 + c * 32;
-      if (gm < 0 || n >= plan.N) continue;
-      float v[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-      __nv_bfloat16* dst;
-      if (epi.kind == 0) {
-        if (epi.bias) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] += __ldg(epi.bias + n + i);
-        }
-        if (epi.residual) {
-          const uint4* r4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(epi.residual) + gm * epi.ldo + n);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            float rr[8];
-            unpack16(r4[i], rr);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[i * 8 + e] += rr[e];
-          }
-        }
-        dst = static_cast<__nv_bfloat16*>(epi.out) + gm * epi.ldo + n;
-      } else {
-        const int which = n / epi.C, cc = n - which * epi.C;
-        const int head = cc >> 6, d0 = cc & 63;
-        void* base = which == 0 ? epi.q : (which == 1 ? epi.k : epi.v);
-        dst = static_cast<__nv_bfloat16*>(base) + ((long long)head * epi.L + gm) * 64 + d0;
-      }
-      uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float w8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) w8[e] = v[i * 8 + e];
-        d4[i] = pack16(w8);
-      }
+    int ti = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++ti) {
+      const int buf = ti & 1, use = ti >> 1;
+      const bool ready = mbar_wait(smem_u32(&acc_full[buf]), use & 1, err, kErrWaitAccum);
+      tc_fence_after();
+      const TileInfo tile = tile_of(plan, t / n_tiles_n);
+      const int n0 = (t % n_tiles_n) * BN;
+      epilogue_tile<BN>(plan, epi, tile, n0, tmem_d + buf * kCols + ((uint32_t)(sub * 32) << 16), row,
+                        ready && !s_abort);
+      tc_fence_before();
+      mbar_arrive(smem_u32(&acc_empty[buf]));
+      if (!ready) break;
     }
   }
 
@@ -240,35 +280,66 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_d, kCols);
+    tmem_dealloc(tmem_d, 2 * kCols);
   }
 }
 
 template <int BN, int STAGES>
 cudaError_t launch_bn(const TcGemmPlan& plan, const CUtensorMap& mA, const CUtensorMap& mB,
                       const Epilogue& epi, int* err, cudaStream_t s) {
-  const size_t smem = 1024 + (size_t)STAGES * (kBM * kBK * 2 + BN * kBK * 2) + (2 * STAGES + 2) * 8 + 64;
+  const size_t smem = 1024 + (size_t)STAGES * 2 * (kBM * kBK * 2 + BN * kBK * 2) + (2 * STAGES + 6) * 8 + 64;
   auto kern = tc_gemm_kernel<BN, STAGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  int m_tiles;
-  if (plan.conv)
-    m_tiles = plan.P * (plan.R / plan.rows_tile) * plan.tiles_per_row;
-  else
-    m_tiles = (plan.M + kBM - 1) / kBM;
-  dim3 grid(plan.N / BN, m_tiles);
+  const int n_tiles = plan.m_tiles * (plan.N / BN);
+  const int grid = n_tiles < plan.sms ? n_tiles : plan.sms;
   kern<<<grid, kThreads, smem, s>>>(mA, mB, plan, epi, err);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_tc_gemm(const TcGemmPlan& plan, const CUtensorMap& mapA, const CUtensorMap& mapB,
+namespace {
+int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+}  // namespace
+
+int gemm_m_tiles_plain(int M) { return (M + kBM - 1) / kBM; }
+
+int choose_bn(int N, int m_tiles) {
+  const int sms = sm_count();
+  int best = 0;
+  long best_cost = 0;
+  for (int bn : {160, 128, 64}) {
+    if (N % bn) continue;
+    // a k-block moves 16 KB of A and bn * 128 B of B through TMA: time per wave
+    // follows those bytes, not the tile width (narrow tiles are not cheaper per FLOP)
+    const long tiles = (long)m_tiles * (N / bn);
+    const long cost = ((tiles + sms - 1) / sms) * (128 + bn);
+    if (!best || cost < best_cost) { best = bn; best_cost = cost; }
+  }
+  return best ? best : 64;
+}
+
+cudaError_t launch_tc_gemm(const TcGemmPlan& plan_in, const CUtensorMap& mapA, const CUtensorMap& mapB,
                            const Epilogue& epi, int* err, cudaStream_t s) {
+  TcGemmPlan plan = plan_in;
+  plan.m_tiles = plan.conv ? plan.P * (plan.R / plan.rows_tile) * plan.tiles_per_row : (plan.M + kBM - 1) / kBM;
+  plan.sms = sm_count();
+  // as many two-chunk stages as fit in ~220 KB of shared memory
   switch (plan.bn) {
-    case 128: return launch_bn<128, 4>(plan, mapA, mapB, epi, err, s);
-    case 160: return launch_bn<160, 4>(plan, mapA, mapB, epi, err, s);
-    case 64: return launch_bn<64, 6>(plan, mapA, mapB, epi, err, s);
+    case 128: return launch_bn<128, 3>(plan, mapA, mapB, epi, err, s);
+    case 160: return launch_bn<160, 3>(plan, mapA, mapB, epi, err, s);
+    case 64: return launch_bn<64, 4>(plan, mapA, mapB, epi, err, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -300,6 +371,14 @@ bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 }  // namespace
+
+bool encode_gemm_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows) {
+  // view [K/64 chunks][rows][64] of a row-major [rows][K] bf16 matrix; one box = two chunks
+  const cuuint64_t dims[3] = {64, rows, (K + 63) / 64};
+  const cuuint64_t strides[2] = {K * 2, 128};
+  const cuuint32_t box[3] = {64, box_rows, 2};
+  return encode(m, base, 3, dims, strides, box);
+}
 
 bool encode_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                     uint64_t outer_stride_bytes, uint32_t box_inner, uint32_t box_outer) {

@@ -60,7 +60,8 @@ def test_noalloc_group_norm_matches_layer_step_two_calls():
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     from patch_diffusion_unet_b200 import dfp
     null = ctypes.c_void_p(16)                      # never dereferenced: the size check fails first
-    st = dfp.LIB.dfp_group_norm_noalloc(null, null, dfp.BF16, 64, 64, 4096, 64, 4, 1e-5, null, null, None,
+    # one patch, 256 groups over a 64x64 map: 148 blocks x 256 groups x 2 partial sums > 64960
+    st = dfp.LIB.dfp_group_norm_noalloc(null, null, dfp.BF16, 64, 64, 4096, 1, 256, 1e-5, null, null, None,
                                         dfp.GN_CORRECTED, 1, null, null, None)
     assert st == dfp.E_ARG
     assert "scratch" in dfp.LIB.dfp_group_norm_noalloc_error().decode()
