@@ -18,6 +18,7 @@ summed step time.  Rank 0 prints one JSON line.
 the same metric on the same workload, full (unsampled) displaced steps.
 """
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -70,6 +71,30 @@ def work_model(cfg):
     L, d = H * W, cfg["head_dim"]
     e = 2 if cfg["dtype"] == "bf16" else 4
     R = H // N
+    if cfg.get("block") == "sdxl_stage":
+        F, T = cfg["ffn_inner"], cfg["ctx_len"]
+        ln = ("hbm", 2 * L * C * e)
+        wm = {
+            "norm1 statistics": ("hbm", L * C * e),
+            "norm1 apply + halo": ("hbm", 2 * L * C * e + 2 * 2 * (N - 1) * W * C * e),
+            "conv1 (tcgen05)": ("tensor", 2.0 * L * C * 9 * C),
+            "norm2 statistics": ("hbm", L * C * e),
+            "norm2 apply + halo": ("hbm", 2 * L * C * e + 2 * 2 * (N - 1) * W * C * e),
+            "conv2 + residual (tcgen05)": ("tensor", 2.0 * L * C * 9 * C),
+            "layernorm 1": ln, "layernorm 2": ln, "layernorm 3": ln,
+            "self-attn qkv (tcgen05)": ("tensor", 2.0 * L * C * 3 * C),
+            "self-attention (tcgen05)": ("tensor", 4.0 * L * L * d * heads),
+            "self-attn out + residual (tcgen05)": ("tensor", 2.0 * L * C * C),
+            "cross-attn q (tcgen05)": ("tensor", 2.0 * L * C * C),
+            "cross-attention (tcgen05)": ("tensor", 4.0 * L * T * d * heads),
+            "cross-attn out + residual (tcgen05)": ("tensor", 2.0 * L * C * C),
+            "ff proj + GEGLU (tcgen05)": ("tensor", 2.0 * L * C * 2 * F),
+            "ff out + residual (tcgen05)": ("tensor", 2.0 * L * F * C),
+        }
+        per_block = 2.0 * L * C * 6 * C + 4.0 * L * (L + T) * d * heads + 2.0 * L * C * 3 * F
+        wm["_total_flops"] = 2 * 2.0 * L * C * 9 * C + cfg["n_xformer"] * per_block
+        wm["_rows_per_patch"] = R
+        return wm
     return {
         "gn1 statistics": ("hbm", L * C * e),
         "gn1 apply + halo": ("hbm", 2 * L * C * e + 2 * 2 * (N - 1) * W * C * e),
@@ -82,6 +107,29 @@ def work_model(cfg):
         "_total_flops": 2.0 * L * C * 9 * C + 2.0 * L * C * 4 * C + 4.0 * L * L * d * heads,
         "_rows_per_patch": R,
     }
+
+
+# ---------------------------------------------------------------------------- ncu traffic
+
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of one ncu capture
+# (profiles/), keyed by workload and kernel, with a hash of the kernel's sources at
+# capture time: once the kernel changes the figure no longer applies and is reported null.
+NCU_TRAFFIC = {
+    ("sdxl1024-64x64x640-n4-bf16", "attention (tcgen05)"):
+        (27.03e6, ("tc_attention.cu", "dfp_common.cuh"), "7948499bb23f5feb"),
+}
+
+
+def ncu_traffic(workload, kernel):
+    ent = NCU_TRAFFIC.get((workload, kernel))
+    if ent is None:
+        return None
+    nbytes, files, sha = ent
+    m = hashlib.sha256()
+    for fn in files:
+        with open(os.path.join(ROOT, "patch_diffusion_unet_b200", "csrc", fn), "rb") as f:
+            m.update(f.read())
+    return nbytes if m.hexdigest()[:16] == sha else None
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -223,7 +271,7 @@ def main():
     L = cfg["H"] * cfg["W"]
     wl = inputs.SyntheticWorkload(cfg)
     blk = dfp.DisplacedPatchBlock(cfg)
-    blk.load_weights(wl.weights)
+    blk.load_weights(dict(wl.weights, context=wl.context) if wl.context is not None else wl.weights)
     stream = blk.stream
     n_pool = 16
     host_x = [inputs.to_torch(wl.x(t), dtype) for t in range(n_pool)]
@@ -330,13 +378,15 @@ def main():
             ach = work / (us * 1e-6) / 1e12
             peak = pk.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
             roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                    "frac": ach / peak, "traffic": None, "peak_source": f"{pk_src} bf16 burst",
+                    "frac": ach / peak, "traffic": ncu_traffic(cfg["name"], dom),
+                    "peak_source": f"{pk_src} bf16 burst",
                     "work_per_launch": work, "us_per_launch": us}
         else:
             ach = work / (us * 1e-6) / 1e9
             peak = pk.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
             roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
-                    "frac": ach / peak, "traffic": None, "peak_source": f"{pk_src} HBM copy",
+                    "frac": ach / peak, "traffic": ncu_traffic(cfg["name"], dom),
+                    "peak_source": f"{pk_src} HBM copy",
                     "work_per_launch": work, "us_per_launch": us}
 
     blk.close()
