@@ -191,20 +191,26 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // The whole warp walks the loop (coordinates are warp-uniform); one lane issues.
+    const bool leader = elect_one();
+    if (leader) {
       tma_prefetch_desc(&mapA);
       tma_prefetch_desc(&mapB);
-      int kg = 0;   // k-stages issued so far (ring position)
-      for (int t = blockIdx.x; t < n_tiles && !s_abort; t += gridDim.x) {
-        const TileInfo tile = tile_of(plan, t / n_tiles_n);
-        const int n0 = (t % n_tiles_n) * BN;
-        for (int kb = 0; kb < num_kb; ++kb, ++kg) {
-          const int s = kg % STAGES, round = kg / STAGES;
-          if (round > 0 && !mbar_wait(smem_u32(&empty[s]), (round - 1) & 1, err, kErrWaitStageFree)) {
-            s_abort = 1;
-            break;
-          }
-          const uint32_t fb = smem_u32(&full[s]);
+    }
+    int kg = 0;   // k-stages issued so far (ring position)
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+      const TileInfo tile = tile_of(plan, t / n_tiles_n);
+      const int n0 = (t % n_tiles_n) * BN;
+      for (int kb = 0; kb < num_kb; ++kb, ++kg) {
+        const int s = kg % STAGES, round = kg / STAGES;
+        if (round > 0 && !mbar_wait_warp(smem_u32(&empty[s]), (round - 1) & 1, err, kErrWaitStageFree)) {
+          ok = false;
+          break;
+        }
+        if (__any_sync(0xffffffffu, s_abort != 0)) { ok = false; break; }
+        const uint32_t fb = smem_u32(&full[s]);
+        if (leader) {
           mbar_arrive_expect_tx(fb, a_box_bytes + kBBytes);
           if (plan.conv) {
             const int tap = kb / ppt, kc = 2 * (kb - tap * ppt);
@@ -218,45 +224,52 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
             tma_load_3d(smem_u32(sB + s * kBBytes), &mapB, fb, 0, n0, 2 * kb);
           }
         }
+        __syncwarp();
       }
-      if (s_abort) {
-        // let the copies already in flight land before the CTA can exit
-        for (int k = (kg > STAGES ? kg - STAGES : 0); k < kg; ++k)
-          mbar_wait(smem_u32(&full[k % STAGES]), (k / STAGES) & 1, err, kErrWaitTmaFull);
-      }
+    }
+    if (!ok || __any_sync(0xffffffffu, s_abort != 0)) {
+      if (leader) s_abort = 1;
+      // let the copies already in flight land before the CTA can exit
+      for (int k = (kg > STAGES ? kg - STAGES : 0); k < kg; ++k)
+        mbar_wait(smem_u32(&full[k % STAGES]), (k / STAGES) & 1, err, kErrWaitTmaFull);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, false, false);
-      const uint64_t ad0 = sw128_kmajor_desc(smem_u32(sA));
-      const uint64_t bd0 = sw128_kmajor_desc(smem_u32(sB));
-      bool ok = true;
-      int kg = 0, ti = 0;
-      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++ti) {
-        const int buf = ti & 1, use = ti >> 1;
-        if (use > 0 && !mbar_wait(smem_u32(&acc_empty[buf]), (use - 1) & 1, err, kErrWaitAccum)) { ok = false; break; }
+    // The whole warp walks the loop so the descriptors stay warp-uniform; the
+    // elected lane issues the MMAs and the commits (which track that lane's MMAs).
+    const bool leader = elect_one();
+    constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, false, false);
+    const uint64_t ad0 = sw128_kmajor_desc(smem_u32(sA));
+    const uint64_t bd0 = sw128_kmajor_desc(smem_u32(sB));
+    bool ok = true;
+    int kg = 0, ti = 0;
+    for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++ti) {
+      const int buf = ti & 1, use = ti >> 1;
+      if (use > 0 && !mbar_wait_warp(smem_u32(&acc_empty[buf]), (use - 1) & 1, err, kErrWaitAccum)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d = tmem_d + buf * kCols;
+      for (int kb = 0; kb < num_kb; ++kb, ++kg) {
+        const int s = kg % STAGES, round = kg / STAGES;
+        if (!mbar_wait_warp(smem_u32(&full[s]), round & 1, err, kErrWaitTmaFull)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d = tmem_d + buf * kCols;
-        for (int kb = 0; kb < num_kb; ++kb, ++kg) {
-          const int s = kg % STAGES, round = kg / STAGES;
-          if (!mbar_wait(smem_u32(&full[s]), round & 1, err, kErrWaitTmaFull)) { ok = false; break; }
-          tc_fence_after();
-          // operands: per-stage bases, compile-time offsets per K slice
-          const uint64_t ad = ad0 + (uint64_t)s * (kABytes >> 4);
-          const uint64_t bd = bd0 + (uint64_t)s * (kBBytes >> 4);
+        // operands: per-stage bases, compile-time offsets per K slice
+        const uint64_t ad = ad0 + (uint64_t)s * (kABytes >> 4);
+        const uint64_t bd = bd0 + (uint64_t)s * (kBBytes >> 4);
+        const uint64_t ad1 = ad + (kAChunk >> 4), bd1 = bd + (kBChunk >> 4);
+        if (leader) {
           umma_f16_ss(d, ad, bd, idesc, kb > 0);
 #pragma unroll
           for (int kk = 1; kk < kBK / 16; ++kk) umma_f16_ss(d, ad + 2 * kk, bd + 2 * kk, idesc, 1);
-          const uint64_t ad1 = ad + (kAChunk >> 4), bd1 = bd + (kBChunk >> 4);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) umma_f16_ss(d, ad1 + 2 * kk, bd1 + 2 * kk, idesc, 1);
           umma_commit(smem_u32(&empty[s]));
         }
-        umma_commit(smem_u32(&acc_full[buf]));
+        __syncwarp();
       }
-      if (!ok) s_abort = 1;
+      if (ok && leader) umma_commit(smem_u32(&acc_full[buf]));
+      __syncwarp();
     }
+    if (!ok && leader) s_abort = 1;
   } else {
     // ------------------------------------------------------------ epilogue (warps 2..5)
     const int sub = warp & 3;
@@ -299,7 +312,6 @@ cudaError_t launch_bn(const TcGemmPlan& plan, const CUtensorMap& mA, const CUten
 
 }  // namespace
 
-namespace {
 int sm_count() {
   static int cached[64] = {};
   int dev = 0;
@@ -311,7 +323,6 @@ int sm_count() {
   }
   return cached[dev];
 }
-}  // namespace
 
 int gemm_m_tiles_plain(int M) { return (M + kBM - 1) / kBM; }
 
