@@ -230,16 +230,13 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
   ok &= h->alloc((void**)&h->part, N * (size_t)gn_stats_chunks((int)N, (int)(R * W)) * G * 2 * 4);
   ok &= h->alloc((void**)&h->counter, 64);
   ok &= h->alloc((void**)&h->dev_err, 64);
-  const int n_qt = (h->Lp + 127) / 128;
-  const size_t pairs = (size_t)((n_qt + 1) / 2) * N * cfg->heads;
   if (cfg->dtype == DFP_BF16) {
-    const int min_tiles = cfg->context == DFP_CTX_NAIVE ? n_qt : (h->L + 127) / 128;
-    h->attn_splits = attention_splits(h->L, h->Lp, (int)N, cfg->heads, min_tiles);
-    if (h->attn_splits > 1) {
-      ok &= h->alloc((void**)&h->attn_part_o, pairs * h->attn_splits * 256 * 64 * 4);
-      ok &= h->alloc((void**)&h->attn_part_ml, pairs * h->attn_splits * 256 * 2 * 4);
-    }
-    ok &= h->alloc((void**)&h->attn_counters, pairs * 4 + 64);
+    // persistent attention: one CTA per SM, two partial-result slots per CTA
+    h->attn_ctas = sm_count();
+    const size_t f = attention_scratch_floats(h->attn_ctas);
+    ok &= h->alloc((void**)&h->attn_part_o, f * 4);
+    ok &= h->alloc((void**)&h->attn_part_ml, f / 32 * 4);
+    ok &= h->alloc((void**)&h->attn_counters, (size_t)h->attn_ctas * 2 * 4 + 64);
   }
   if (!ok) {
     g_create_error = "device allocation failed";
@@ -259,7 +256,7 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
     if (e == cudaSuccess) e = cudaMemset(p, 0, map);
   if (e == cudaSuccess) e = cudaMemset(h->counter, 0, 64);
   if (e == cudaSuccess) e = cudaMemset(h->dev_err, 0, 64);
-  if (e == cudaSuccess && h->attn_counters) e = cudaMemset(h->attn_counters, 0, pairs * 4 + 64);
+  if (e == cudaSuccess && h->attn_counters) e = cudaMemset(h->attn_counters, 0, (size_t)h->attn_ctas * 2 * 4 + 64);
   if (e != cudaSuccess) {
     g_create_error = std::string("cudaMemset: ") + cudaGetErrorString(e);
     dfp_destroy(h);
@@ -578,7 +575,7 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   if (h->family == 0) {
     TcAttnArgs a{};
     a.L = L; a.Lp = Lp; a.N = N; a.heads = c.heads; a.C = C; a.mode = mode; a.o = h->o; a.err = h->dev_err;
-    a.splits = h->attn_splits; a.n_qtiles = (Lp + 127) / 128;
+    a.ctas = h->attn_ctas; a.n_qtiles = (Lp + 127) / 128;
     a.part_o = h->attn_part_o; a.part_ml = h->attn_part_ml; a.counters = h->attn_counters;
     DFP_LAUNCH(launch_tc_attention(a, h->m_q, h->m_k[cur], h->m_v[cur], h->m_k[prv], h->m_v[prv], s), "attention (tcgen05)");
   } else {

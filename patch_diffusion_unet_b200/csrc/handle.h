@@ -41,7 +41,7 @@ struct dfp_ctx {
   unsigned* counter = nullptr;
   int* dev_err = nullptr;
   // split-KV attention scratch
-  int attn_splits = 1;
+  int attn_ctas = 0;
   float *attn_part_o = nullptr, *attn_part_ml = nullptr;
   unsigned* attn_counters = nullptr;
   std::vector<void*> allocs;

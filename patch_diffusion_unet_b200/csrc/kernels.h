@@ -78,6 +78,8 @@ bool encode_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, 
                     uint64_t s1_bytes, uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
 bool encode_tmap_4d(CUtensorMap* m, const void* base, const uint64_t dims[4],
                     const uint64_t strides_bytes[3], const uint32_t box[4]);
+bool encode_tmap_5d(CUtensorMap* m, const void* base, const uint64_t dims[5],
+                    const uint64_t strides_bytes[4], const uint32_t box[5]);
 // GEMM operand: row-major [rows][K] bf16, K a multiple of 64; box = box_rows x two 64-wide K chunks
 bool encode_gemm_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows);
 
@@ -102,16 +104,22 @@ struct TcAttnArgs {
   int kv_len;             // cross-attention: number of context tokens (mode kAttnCross)
   void* o;                // [L, C] bf16
   int* err;
-  int splits;             // CTAs sharing the KV tile list of one Q-tile pair
   int n_qtiles;           // ceil(Lp / 128)
-  float* part_o;          // scratch [pairs][splits][256][64] (splits > 1)
-  float* part_ml;         // scratch [pairs][splits][256][2]  (running max, row sum)
-  unsigned* counters;     // scratch [pairs], zero between launches
+  int ctas;               // persistent CTAs (one per SM); the scratch below is sized for them
+  float* part_o;          // scratch [ctas][2][256][64]: unnormalised O of a cut pair's piece
+  float* part_ml;         // scratch [ctas][2][256][2]:  (running max, row sum) of the same
+  unsigned* counters;     // scratch [ctas][2], zero between launches
+  int total_tiles;        // set by the launcher
 };
-// Split count for the KV loop: enough CTAs to fill the GPU (148 SMs) in whole waves,
-// keeping at least 2 KV tiles per split.  min_tiles = fewest KV tiles of any mode used.
-int attention_splits(int L, int Lp, int N, int heads, int min_tiles);
-// maps: q [heads][L][64]; k/v fresh and stale, same shape (box 128 rows x 64)
+// floats of part_o for `ctas` CTAs (part_ml needs 1/32 of it)
+size_t attention_scratch_floats(int ctas);
+int sm_count();
+// V operand of the attention: [heads][rows][64] bf16 (rows a multiple of 4, every KV tile
+// starting at a multiple of 4) seen as a 5-D view whose 128-row box lands in shared memory
+// with rows 1 and 2 of every group of 4 swapped -- the key order in which the softmax
+// threads pack P (see the attention kernel).
+bool encode_attn_v(CUtensorMap* m, const void* base, uint64_t rows, uint64_t heads);
+// maps: q [heads][L][64]; k fresh and stale (box 128 rows x 64); v from encode_attn_v
 cudaError_t launch_tc_attention(const TcAttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mkf,
                                 const CUtensorMap& mvf, const CUtensorMap& mks,
                                 const CUtensorMap& mvs, cudaStream_t s);

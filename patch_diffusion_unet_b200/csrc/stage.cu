@@ -160,6 +160,7 @@ dfp_status stage_create(dfp_ctx* h) {
       e = cudaMemset(st->xf[b].kb[i], 0, map);
       if (e == cudaSuccess) e = cudaMemset(st->xf[b].vb[i], 0, map);
     }
+
   if (e != cudaSuccess) return h->cuda_fail(e, "cudaMemset");
   h->y = st->r.back();
 
@@ -362,7 +363,7 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
     DFP_LAUNCH(launch_tc_gemm(x.p_qkv, st->m_u, x.m_wqkv, eq, h->dev_err, s), "self-attn qkv (tcgen05)");
     TcAttnArgs a{};
     a.L = L; a.Lp = Lp; a.N = N; a.heads = c.heads; a.C = C; a.mode = sa_mode; a.o = h->o; a.err = h->dev_err;
-    a.n_qtiles = (Lp + 127) / 128; a.splits = h->attn_splits;
+    a.n_qtiles = (Lp + 127) / 128; a.ctas = h->attn_ctas;
     a.part_o = h->attn_part_o; a.part_ml = h->attn_part_ml; a.counters = h->attn_counters;
     DFP_LAUNCH(launch_tc_attention(a, h->m_q, x.m_k[cur], x.m_v[cur], x.m_k[prv], x.m_v[prv], s),
                "self-attention (tcgen05)");
@@ -376,7 +377,7 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
     DFP_LAUNCH(launch_tc_gemm(x.p_q2, st->m_u, x.m_wq2, e2, h->dev_err, s), "cross-attn q (tcgen05)");
     TcAttnArgs ca{};
     ca.L = L; ca.Lp = L; ca.N = 1; ca.heads = c.heads; ca.C = C; ca.mode = kAttnCross; ca.kv_len = c.ctx_len;
-    ca.o = h->o; ca.err = h->dev_err; ca.n_qtiles = (L + 127) / 128; ca.splits = 1;
+    ca.o = h->o; ca.err = h->dev_err; ca.n_qtiles = (L + 127) / 128; ca.ctas = h->attn_ctas;
     ca.part_o = h->attn_part_o; ca.part_ml = h->attn_part_ml; ca.counters = h->attn_counters;
     DFP_LAUNCH(launch_tc_attention(ca, h->m_q, x.m_ck, x.m_cv, x.m_ck, x.m_cv, s), "cross-attention (tcgen05)");
     eo.out = r_ca; eo.bias = x.b_o2; eo.residual = r_sa;

@@ -18,8 +18,10 @@
 // they exchange their partial row maxima through shared memory -- at head width
 // 64 the softmax work per tile is large next to the MMAs, and two threads per
 // row double the latency hiding.  In the fifth warpgroup warp 16 issues TMA
-// (both Q tiles once, K/V through 3-stage rings shared by the groups) and warp
-// 17 issues the MMAs from one thread.  Per KV tile j and group g:
+// (the Q-tile pair of each piece into a double buffer, K/V through 3-stage rings
+// shared by the groups) and warp 17 issues the MMAs from one elected lane; this
+// warpgroup hands most of its registers to the softmax warpgroups (setmaxnreg).
+// Per KV tile j and group g:
 //   S_g = Q_g K_j^T            tcgen05.mma, A and B from shared memory, D in TMEM
 //   P_g = exp2(S_g * c - m_g)  softmax threads, written back over S_g in TMEM as
 //                              bf16 pairs (byte-permute truncation)
@@ -34,10 +36,19 @@
 // degree-3 polynomial for 2^f fitted by weighted least squares on Chebyshev
 // nodes, max relative error 7.5e-5) to offload the MUFU unit.
 //
-// Split-KV: with few query tiles per SM (small maps) the KV tile list of a Q-tile
-// pair is split over `splits` CTAs; each writes its unnormalised O, m and l to a
-// scratch buffer and the last CTA of the pair (arrival counter) merges them in
-// split order, so the result is deterministic.
+// Work split (stream-K style): a unit of work is one KV tile for one Q-tile pair of
+// one (patch, head).  The units are laid out pair-major within (patch, head) and
+// the whole list is cut into one contiguous range per SM, so every CTA gets the
+// same number of KV tiles whatever the number of pairs.  A CTA walks its range as
+// a sequence of pieces (the part of one pair's KV list that falls in the range);
+// Q is double-buffered so the next piece's queries load while the current piece
+// runs, and the K/V ring does not drain between pieces.  A pair whose KV list is
+// cut between CTAs is finished by the last of them to arrive (arrival counter):
+// each piece leaves its unnormalised O, running max and row sum in a per-CTA slot
+// and the last one merges the pieces in KV order, so the result does not depend
+// on timing.
+#include <algorithm>
+
 #include "dfp_common.cuh"
 #include "kernels.h"
 
@@ -46,7 +57,6 @@ namespace dfp {
 namespace {
 
 constexpr int kThreads = 640;
-constexpr int kSoftmaxThreads = 512;
 constexpr int kWarpTma = 16, kWarpMma = 17;
 constexpr int kTile = 128;
 constexpr uint32_t kTileBytes = 128 * 64 * 2;   // one 128 x 64 bf16 tile
@@ -54,45 +64,90 @@ constexpr int kStages = 3;
 constexpr int kOCols = 80;                      // 64 outputs + 16 row-sum columns
 constexpr uint32_t kTmemCols = 512;             // S/P: [128g, 128g+128), O: [256+128g, +80)
 constexpr float kRescale = 8.f;                 // lazy rescale threshold (log2 units)
-constexpr int kPolyPer8 = 3;                    // of every 8 columns, this many use the polynomial
+constexpr int kPolyPer8 = 3;
+// registers per thread after the split: 128 x 64 + 512 x 104 = 640 x 96 (the launch's)
+constexpr int kRegsTmaMma = 64, kRegsSoftmax = 104;                    // of every 8 columns, this many use the polynomial
 
-struct Segs {
-  int n;
-  int stale[3], start[3], len[3], tiles[3];
-  int total;
+__host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// KV tiles of one query-tile pair of patch p.  The KV list walks the segments
+//   sync       [0, L) fresh
+//   cross      [0, kv_len) (the fixed context)
+//   naive      own patch fresh only
+//   displaced  own patch fresh, then [0, p*Lp) stale, then [(p+1)*Lp, L) stale
+// each rounded up to whole 128-key tiles (the columns past a segment's end are masked).
+__host__ __device__ __forceinline__ int unit_tiles(int mode, int p, int Lp, int L, int kv_len) {
+  if (mode == kAttnSync) return cdiv(L, kTile);
+  if (mode == kAttnCross) return cdiv(kv_len, kTile);
+  int t = cdiv(Lp, kTile);
+  if (mode == kAttnDisplaced) t += cdiv(p * Lp, kTile) + cdiv(L - (p + 1) * Lp, kTile);
+  return t;
+}
+
+// tile j of patch p's KV list -> (stale?, first key row, valid keys)
+__device__ __forceinline__ void tile_src(int mode, int p, int Lp, int L, int kv_len, int j, int& stale,
+                                         int& row, int& valid) {
+  stale = 0;
+  if (mode == kAttnSync || mode == kAttnCross) {
+    row = j * kTile;
+    valid = min(kTile, (mode == kAttnSync ? L : kv_len) - row);
+    return;
+  }
+  const int own = cdiv(Lp, kTile);
+  if (j < own) {
+    row = p * Lp + j * kTile;
+    valid = min(kTile, Lp - j * kTile);
+    return;
+  }
+  stale = 1;
+  j -= own;
+  const int t1 = cdiv(p * Lp, kTile);
+  if (j < t1) {
+    row = j * kTile;
+    valid = min(kTile, p * Lp - row);
+    return;
+  }
+  row = (p + 1) * Lp + (j - t1) * kTile;
+  valid = min(kTile, L - row);
+}
+
+// The unit list: patch-major, then head, then Q-tile pair; unit (p, head, pair) has
+// unit_tiles(p) KV tiles.  Global tile x -> its unit and the unit's first tile.
+// All schedule arithmetic is 32-bit: the launcher checks total_tiles * ctas < 2^31.
+struct Unit {
+  int p, head, pair, T, U0;
 };
-
-__device__ __forceinline__ Segs make_segs(int mode, int p, int Lp, int L, int kv_len) {
-  Segs s{};
-  auto add = [&](int st, int b, int len) {
-    if (len <= 0) return;
-    s.stale[s.n] = st; s.start[s.n] = b; s.len[s.n] = len;
-    s.tiles[s.n] = (len + kTile - 1) / kTile;
-    s.total += s.tiles[s.n];
-    ++s.n;
-  };
-  if (mode == kAttnSync) {
-    add(0, 0, L);
-  } else if (mode == kAttnCross) {
-    add(0, 0, kv_len);        // the fixed context: same for every patch, never stale
-  } else {
-    add(0, p * Lp, Lp);
-    if (mode == kAttnDisplaced) {
-      add(1, 0, p * Lp);
-      add(1, (p + 1) * Lp, L - (p + 1) * Lp);
+__device__ __forceinline__ Unit locate(const TcAttnArgs& a, int n_pairs, int x) {
+  int base = 0;
+  Unit u{};
+  for (int p = 0; p < a.N; ++p) {
+    const int T = unit_tiles(a.mode, p, a.Lp, a.L, a.kv_len);
+    const int blk = T * a.heads * n_pairs;
+    if (x < base + blk) {
+      const int ui = (x - base) / T;
+      u.p = p; u.head = ui / n_pairs; u.pair = ui - u.head * n_pairs; u.T = T;
+      u.U0 = base + ui * T;
+      return u;
+    }
+    base += blk;
+  }
+  return u;   // not reached for x < total
+}
+// the unit after u in the list (no division: pairs, then heads, then patches)
+__device__ __forceinline__ void advance(const TcAttnArgs& a, int n_pairs, Unit& u) {
+  u.U0 += u.T;
+  if (++u.pair == n_pairs) {
+    u.pair = 0;
+    if (++u.head == a.heads) {
+      u.head = 0;
+      ++u.p;
+      u.T = unit_tiles(a.mode, u.p, a.Lp, a.L, a.kv_len);
     }
   }
-  return s;
 }
-
-// tile j of the segment list -> (stale?, first key row, valid keys)
-__device__ __forceinline__ void seg_tile(const Segs& s, int j, int& stale, int& row, int& valid) {
-  int k = 0;
-  while (k < s.n - 1 && j >= s.tiles[k]) { j -= s.tiles[k]; ++k; }
-  stale = s.stale[k];
-  row = s.start[k] + j * kTile;
-  valid = min(kTile, s.len[k] - j * kTile);
-}
+// the CTA whose range [c*TT/G, (c+1)*TT/G) holds global tile x
+__device__ __forceinline__ int cta_of(int x, int TT, int G) { return ((x + 1) * G + TT - 1) / TT - 1; }
+__device__ __forceinline__ int range_start(int c, int TT, int G) { return c * TT / G; }
 
 __device__ __forceinline__ float ex2_mufu(float x) {
   float y;
@@ -175,6 +230,11 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
@@ -203,44 +263,158 @@ __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
+// End of a piece for one softmax group: this thread's half row of O (32 columns)
+// and the row sum, normalised into the output, or -- for a pair cut between CTAs --
+// left as a partial in this CTA's slot, with the last piece to arrive merging all
+// of them in KV order.  O streams through 8-column chunks so the epilogue needs few
+// registers; it is out of line so that none of them count against the KV loop.
+// Returns false if the final P V never completed.
+__device__ __noinline__ bool piece_epilogue(const TcAttnArgs& a, const Unit& u, uint32_t tO, uint32_t o_bar,
+                                               uint32_t o_parity, float m_used, int g, int half, int row,
+                                               bool group_leader, int c, int X0, int* s_last) {
+  const int TT = a.total_tiles, G = gridDim.x;
+  const bool have = mbar_wait(o_bar, o_parity, a.err, kErrWaitAttnO);
+  float l = 1.f;
+  if (have) {
+    tc_fence_after();
+    uint32_t r8[8];
+    tmem_ld8(tO + 64, r8);
+    tmem_wait_ld();
+    l = __uint_as_float(r8[0]);
+  }
+  const int q_local = (2 * u.pair + g) * kTile + row;
+  const bool row_ok = have && q_local < a.Lp;
+  uint4* out_row = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) +
+                                            (size_t)(u.p * a.Lp + q_local) * a.C + u.head * 64 + half * 32);
+  const int c_first = cta_of(u.U0, TT, G);
+  const int npieces = cta_of(u.U0 + u.T - 1, TT, G) - c_first + 1;
+  if (npieces == 1) {
+    if (have) {
+      const float inv = 1.f / l;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t r8[8];
+        tmem_ld8(tO + half * 32 + k * 8, r8);
+        tmem_wait_ld();
+        float w8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w8[e] = __uint_as_float(r8[e]) * inv;
+        if (row_ok) out_row[k] = pack16(w8);
+      }
+    }
+    return have;
+  }
+  // this piece's partial result into the CTA's slot (0: its first piece, 1: its last
+  // piece; X0 < U0 means the pair started after this CTA's range did)
+  const size_t slot = (size_t)c * 2 + (X0 < u.U0 ? 1 : 0);
+  const size_t prow = slot * 256 + g * 128 + row;
+  if (have) {
+    float4* po = reinterpret_cast<float4*>(a.part_o + prow * 64 + half * 32);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t r8[8];
+      tmem_ld8(tO + half * 32 + k * 8, r8);
+      tmem_wait_ld();
+      po[2 * k] = make_float4(__uint_as_float(r8[0]), __uint_as_float(r8[1]), __uint_as_float(r8[2]),
+                              __uint_as_float(r8[3]));
+      po[2 * k + 1] = make_float4(__uint_as_float(r8[4]), __uint_as_float(r8[5]), __uint_as_float(r8[6]),
+                                  __uint_as_float(r8[7]));
+    }
+    if (half == 0) reinterpret_cast<float2*>(a.part_ml)[prow] = make_float2(m_used, l);
+  }
+  __threadfence();
+  named_bar(2 + g, 256);
+  if (group_leader) *s_last = atomicAdd(a.counters + 2 * c_first + g, 1u) == (unsigned)(npieces - 1);
+  named_bar(2 + g, 256);
+  if (*s_last) {
+    __threadfence();
+    if (row_ok) {
+      float mm = -INFINITY;
+      for (int k = 0; k < npieces; ++k) {
+        const int ck = c_first + k;
+        const size_t sr = ((size_t)ck * 2 + (range_start(ck, TT, G) < u.U0 ? 1 : 0)) * 256 + g * 128 + row;
+        mm = fmaxf(mm, __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr).x);
+      }
+      float lsum = 0.f;
+      for (int k = 0; k < npieces; ++k) {
+        const int ck = c_first + k;
+        const size_t sr = ((size_t)ck * 2 + (range_start(ck, TT, G) < u.U0 ? 1 : 0)) * 256 + g * 128 + row;
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr);
+        lsum = fmaf(ml.y, ex2_mufu(ml.x - mm), lsum);
+      }
+      const float inv = 1.f / lsum;
+      // merge 8 columns at a time, pieces in KV order
+      for (int q = 0; q < 4; ++q) {
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        for (int k = 0; k < npieces; ++k) {
+          const int ck = c_first + k;
+          const size_t sr = ((size_t)ck * 2 + (range_start(ck, TT, G) < u.U0 ? 1 : 0)) * 256 + g * 128 + row;
+          const float w = ex2_mufu(__ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr).x - mm);
+          const float4* po = reinterpret_cast<const float4*>(a.part_o + sr * 64 + half * 32 + q * 8);
+          const float4 v0 = __ldcg(po), v1 = __ldcg(po + 1);
+          acc[0] = fmaf(v0.x, w, acc[0]); acc[1] = fmaf(v0.y, w, acc[1]);
+          acc[2] = fmaf(v0.z, w, acc[2]); acc[3] = fmaf(v0.w, w, acc[3]);
+          acc[4] = fmaf(v1.x, w, acc[4]); acc[5] = fmaf(v1.y, w, acc[5]);
+          acc[6] = fmaf(v1.z, w, acc[6]); acc[7] = fmaf(v1.w, w, acc[7]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] *= inv;
+        out_row[q] = pack16(acc);
+      }
+    }
+    if (group_leader) a.counters[2 * c_first + g] = 0u;
+  }
+  return have;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mkf,
                     const __grid_constant__ CUtensorMap mvf, const __grid_constant__ CUtensorMap mks,
                     const __grid_constant__ CUtensorMap mvs, const TcAttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                          // 2 x 16 KB
-  uint8_t* sK = sQ + 2 * kTileBytes;           // kStages x 16 KB
+  uint8_t* sQ = smem;                          // 2 buffers x 2 tiles x 16 KB
+  uint8_t* sK = sQ + 4 * kTileBytes;           // kStages x 16 KB
   uint8_t* sV = sK + kStages * kTileBytes;     // kStages x 16 KB
   uint8_t* sOnes = sV + kStages * kTileBytes;  // 16 KB of bf16 1.0 (the row-sum columns of B)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sOnes + kTileBytes);
-  uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
+  uint64_t* q_full = bars;                     // [2]
+  uint64_t* q_empty = q_full + 2;              // [2]
+  uint64_t* k_full = q_empty + 2;
   uint64_t* k_empty = k_full + kStages;
   uint64_t* v_full = k_empty + kStages;
   uint64_t* v_empty = v_full + kStages;
   uint64_t* s_full = v_empty + kStages;        // [2]
   uint64_t* p_full = s_full + 2;               // [2]
   uint64_t* o_done = p_full + 2;               // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 2);
+  uint64_t* mma_drain = o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
   __shared__ volatile int s_abort;
-  __shared__ int s_last;
-  __shared__ Segs s_segs;
+  __shared__ int s_last[2];
   __shared__ float s_rowmax[2][2][2][128];   // [tile parity][group][half][row]
+  __shared__ int s_piece[2][8];               // per group: p, head, pair, T, U0, piece start
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int splits = a.splits;
-  const int split = blockIdx.x % splits, pair = blockIdx.x / splits;
-  const int p = blockIdx.y, head = blockIdx.z;
-  const int qt0 = 2 * pair;
-  const bool activeB = qt0 + 1 < a.n_qtiles;
-  const Segs& segs = s_segs;   // the KV segment list lives in shared memory (registers are precious)
+  const int G = gridDim.x, c = blockIdx.x;
+  const int TT = a.total_tiles;
+  const int X0 = range_start(c, TT, G), X1 = range_start(c + 1, TT, G);
+  const int NT = X1 - X0;
+  const int n_pairs = (a.n_qtiles + 1) / 2;
   int* err = a.err;
 
   if (threadIdx.x == 0) {
-    s_segs = make_segs(a.mode, p, a.Lp, a.L, a.kv_len);
     s_abort = 0;
-    mbar_init(smem_u32(q_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&q_full[i]), 1); mbar_init(smem_u32(&q_empty[i]), 1);
+    }
     for (int i = 0; i < kStages; ++i) {
       mbar_init(smem_u32(&k_full[i]), 1); mbar_init(smem_u32(&k_empty[i]), 1);
       mbar_init(smem_u32(&v_full[i]), 1); mbar_init(smem_u32(&v_empty[i]), 1);
@@ -250,6 +424,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
       mbar_init(smem_u32(&p_full[g]), 256);
       mbar_init(smem_u32(&o_done[g]), 1);
     }
+    mbar_init(smem_u32(mma_drain), 1);
     fence_mbar_init();
   }
   {
@@ -266,318 +441,345 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int j0 = split * segs.total / splits;
-  const int nt = (split + 1) * segs.total / splits - j0;
 
   if (warp >= kWarpTma) {
+   // Register split: this warpgroup (TMA, MMA and two idle warps) gives registers to
+   // the four softmax warpgroups (the launcher checks the launch's total covers it).
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsTmaMma) : "memory");
+   // Both warps walk their loops with all lanes (addresses and descriptors stay
+   // warp-uniform); the elected lane issues the copies, MMAs and commits.
+   const bool leader = elect_one();
    if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&mq);
-      const int qrow = p * a.Lp + qt0 * kTile;
-      mbar_arrive_expect_tx(smem_u32(q_full), activeB ? 2 * kTileBytes : kTileBytes);
-      tma_load_3d(smem_u32(sQ), &mq, smem_u32(q_full), 0, qrow, head);
-      if (activeB) tma_load_3d(smem_u32(sQ + kTileBytes), &mq, smem_u32(q_full), 0, qrow + kTile, head);
-      int issued = 0;
-      for (int jj = 0; jj < nt; ++jj) {
-        const int s = jj % kStages, round = jj / kStages;
+    if (leader) tma_prefetch_desc(&mq);
+    int gt = 0, pi = 0;   // tiles and pieces issued so far
+    bool ok = true;
+    Unit u = locate(a, n_pairs, X0);
+    for (int x = X0; ok && x < X1; ++pi, advance(a, n_pairs, u)) {
+      const int jl0 = x - u.U0;
+      const int n = min(u.U0 + u.T, X1) - x;
+      // the piece's two query tiles into Q buffer pi & 1
+      const int qb = pi & 1;
+      if (pi >= 2 && !mbar_wait_warp(smem_u32(&q_empty[qb]), ((pi >> 1) - 1) & 1, err, kErrWaitStageFree)) {
+        ok = false;
+        break;
+      }
+      if (leader) {
+        const int qrow = u.p * a.Lp + 2 * u.pair * kTile;
+        const uint32_t qbar = smem_u32(&q_full[qb]);
+        mbar_arrive_expect_tx(qbar, 2 * kTileBytes);
+        tma_load_3d(smem_u32(sQ + 2 * qb * kTileBytes), &mq, qbar, 0, qrow, u.head);
+        tma_load_3d(smem_u32(sQ + (2 * qb + 1) * kTileBytes), &mq, qbar, 0, qrow + kTile, u.head);
+      }
+      __syncwarp();
+      for (int jj = 0; jj < n; ++jj, ++gt) {
+        const int s = gt % kStages, round = gt / kStages;
         int stale, row, valid;
-        seg_tile(segs, j0 + jj, stale, row, valid);
-        if (round > 0 && !mbar_wait(smem_u32(&k_empty[s]), (round - 1) & 1, err, kErrWaitStageFree)) { s_abort = 1; break; }
-        mbar_arrive_expect_tx(smem_u32(&k_full[s]), kTileBytes);
-        tma_load_3d(smem_u32(sK + s * kTileBytes), stale ? &mks : &mkf, smem_u32(&k_full[s]), 0, row, head);
-        if (round > 0 && !mbar_wait(smem_u32(&v_empty[s]), (round - 1) & 1, err, kErrWaitStageFree)) {
-          s_abort = 1;
-          mbar_arrive_expect_tx(smem_u32(&v_full[s]), 0);
-          ++issued;
+        tile_src(a.mode, u.p, a.Lp, a.L, a.kv_len, jl0 + jj, stale, row, valid);
+        if (round > 0 && !mbar_wait_warp(smem_u32(&k_empty[s]), (round - 1) & 1, err, kErrWaitStageFree)) { ok = false; break; }
+        if (leader) {
+          mbar_arrive_expect_tx(smem_u32(&k_full[s]), kTileBytes);
+          tma_load_3d(smem_u32(sK + s * kTileBytes), stale ? &mks : &mkf, smem_u32(&k_full[s]), 0, row, u.head);
+        }
+        if (round > 0 && !mbar_wait_warp(smem_u32(&v_empty[s]), (round - 1) & 1, err, kErrWaitStageFree)) {
+          if (leader) mbar_arrive_expect_tx(smem_u32(&v_full[s]), 0);
+          ++gt;
+          ok = false;
           break;
         }
-        mbar_arrive_expect_tx(smem_u32(&v_full[s]), kTileBytes);
-        tma_load_3d(smem_u32(sV + s * kTileBytes), stale ? &mvs : &mvf, smem_u32(&v_full[s]), 0, row, head);
-        ++issued;
-      }
-      if (s_abort) {
-        for (int jj = (issued > kStages ? issued - kStages : 0); jj < issued; ++jj) {
-          mbar_wait(smem_u32(&k_full[jj % kStages]), (jj / kStages) & 1, err, kErrWaitTmaFull);
-          mbar_wait(smem_u32(&v_full[jj % kStages]), (jj / kStages) & 1, err, kErrWaitTmaFull);
+        if (leader) {
+          mbar_arrive_expect_tx(smem_u32(&v_full[s]), kTileBytes);
+          tma_load_3d(smem_u32(sV + s * kTileBytes), stale ? &mvs : &mvf, smem_u32(&v_full[s]), 0, row, u.head);
         }
+        __syncwarp();
       }
+      x += n;
+    }
+    if (!ok) {
+      if (leader) s_abort = 1;
+      // let the copies already in flight land before the CTA can exit
+      for (int j = (gt > kStages ? gt - kStages : 0); j < gt; ++j) {
+        mbar_wait(smem_u32(&k_full[j % kStages]), (j / kStages) & 1, err, kErrWaitTmaFull);
+        mbar_wait(smem_u32(&v_full[j % kStages]), (j / kStages) & 1, err, kErrWaitTmaFull);
+      }
+      for (int q = (pi > 2 ? pi - 2 : 0); q < pi; ++q)
+        mbar_wait(smem_u32(&q_full[q & 1]), (q >> 1) & 1, err, kErrWaitTmaFull);
     }
    } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      // Per MMA, every operand is a per-tile base plus a compile-time offset (the two
-      // groups and the K slices are unrolled): runtime arithmetic between
-      // tcgen05.mma instructions stalls their issue.
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTile, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, kOCols, false, true);
-      constexpr uint64_t kTileDesc = kTileBytes >> 4;            // one tile in descriptor address units
-      const uint64_t qd0 = sw128_kmajor_desc(smem_u32(sQ));
-      const uint64_t kd0 = sw128_kmajor_desc(smem_u32(sK));
-      // V stage 0 with the ones block as its second 64-column atom (leading byte offset);
-      // stage st: start address + st tiles, leading byte offset - st tiles
-      uint64_t vd0 = sw128_mnmajor_desc(smem_u32(sV));
-      vd0 = (vd0 & ~(uint64_t(0x3FFF) << 16)) |
-            (uint64_t(((smem_u32(sOnes) - smem_u32(sV)) >> 4) & 0x3FFF) << 16);
-      const bool two = activeB;
-      bool ok = mbar_wait(smem_u32(q_full), 0, err, kErrWaitTmaFull);
-      // S_g = Q_g K^T, K tile at descriptor kd
-#define DFP_ISSUE_S(G, KD)                                                   \
-      do {                                                                   \
-        const uint64_t qd = qd0 + (uint64_t)(G) * kTileDesc;                 \
-        umma_f16_ss(tmem + 128 * (G), qd, (KD), idesc_s, 0);                 \
-        umma_f16_ss(tmem + 128 * (G), qd + 2, (KD) + 2, idesc_s, 1);         \
-        umma_f16_ss(tmem + 128 * (G), qd + 4, (KD) + 4, idesc_s, 1);         \
-        umma_f16_ss(tmem + 128 * (G), qd + 6, (KD) + 6, idesc_s, 1);         \
+    // Per MMA, every operand is a per-tile base plus a compile-time offset (the two
+    // groups and the K slices are unrolled): runtime arithmetic between
+    // tcgen05.mma instructions stalls their issue.
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTile, false, false);
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, kOCols, false, true);
+    constexpr uint64_t kTileDesc = kTileBytes >> 4;            // one tile in descriptor address units
+    const uint64_t qd0 = sw128_kmajor_desc(smem_u32(sQ));
+    const uint64_t kd0 = sw128_kmajor_desc(smem_u32(sK));
+    // V stage 0 with the ones block as its second 64-column atom (leading byte offset);
+    // stage st: start address + st tiles, leading byte offset - st tiles
+    uint64_t vd0 = sw128_mnmajor_desc(smem_u32(sV));
+    vd0 = (vd0 & ~(uint64_t(0x3FFF) << 16)) |
+          (uint64_t(((smem_u32(sOnes) - smem_u32(sV)) >> 4) & 0x3FFF) << 16);
+    // S_g = Q_g K^T, Q tile descriptor QD, K tile descriptor KD
+#define DFP_ISSUE_S(G, QD, KD)                                               \
+    do {                                                                     \
+      if (leader) {                                                          \
+        umma_f16_ss(tmem + 128 * (G), (QD), (KD), idesc_s, 0);               \
+        umma_f16_ss(tmem + 128 * (G), (QD) + 2, (KD) + 2, idesc_s, 1);       \
+        umma_f16_ss(tmem + 128 * (G), (QD) + 4, (KD) + 4, idesc_s, 1);       \
+        umma_f16_ss(tmem + 128 * (G), (QD) + 6, (KD) + 6, idesc_s, 1);       \
         umma_commit(smem_u32(&s_full[G]));                                   \
-      } while (0)
-      // O_g += P_g [V | 1], V tile at descriptor vd (P read from TMEM over S_g)
+      }                                                                      \
+      __syncwarp();                                                          \
+    } while (0)
+    // O_g += P_g [V | 1], V tile at descriptor vd (P read from TMEM over S_g)
 #define DFP_ISSUE_PV(G, VD, ACC0)                                                                \
-      do {                                                                                       \
+    do {                                                                                         \
+      if (leader) {                                                                              \
         umma_f16_ts(tmem + 256 + 128 * (G), tmem + 128 * (G), (VD), idesc_o, (ACC0));            \
         _Pragma("unroll") for (int kk = 1; kk < 8; ++kk)                                         \
           umma_f16_ts(tmem + 256 + 128 * (G), tmem + 128 * (G) + kk * 8, (VD) + (uint64_t)kk * 128, idesc_o, 1); \
         umma_commit(smem_u32(&o_done[G]));                                                       \
-      } while (0)
-      if (ok && !mbar_wait(smem_u32(&k_full[0]), 0, err, kErrWaitTmaFull)) ok = false;
+      }                                                                                          \
+      __syncwarp();                                                                              \
+    } while (0)
+    // piece walk: for each tile, is it the first / last of its piece, and which piece
+    int px = X0;
+    int left = 0, pc = -1;
+    Unit mu = locate(a, n_pairs, X0);
+    auto next_tile = [&](bool& first, bool& last, int& piece) {
+      first = left == 0;
+      if (first) {
+        if (pc >= 0) advance(a, n_pairs, mu);
+        left = min(mu.U0 + mu.T, X1) - px;
+        ++pc;
+      }
+      --left;
+      ++px;
+      last = left == 0;
+      piece = pc;
+    };
+    bool ok = true;
+    bool cur_first, cur_last;
+    int cur_piece;
+    next_tile(cur_first, cur_last, cur_piece);
+    {
+      const int qb = cur_piece & 1;
+      ok = mbar_wait_warp(smem_u32(&q_full[qb]), (cur_piece >> 1) & 1, err, kErrWaitTmaFull) &&
+           mbar_wait_warp(smem_u32(&k_full[0]), 0, err, kErrWaitTmaFull);
       if (ok) {
         tc_fence_after();
-        DFP_ISSUE_S(0, kd0);
-        if (two) DFP_ISSUE_S(1, kd0);
-        umma_commit(smem_u32(&k_empty[0]));
+        const uint64_t qd = qd0 + (uint64_t)(2 * qb) * kTileDesc;
+        DFP_ISSUE_S(0, qd, kd0);
+        DFP_ISSUE_S(1, qd + kTileDesc, kd0);
+        if (leader) {
+          if (cur_last) umma_commit(smem_u32(&q_empty[qb]));
+          umma_commit(smem_u32(&k_empty[0]));
+        }
+        __syncwarp();
       }
-      for (int jj = 0; ok && jj < nt; ++jj) {
-        const int st = jj % kStages, st1 = (jj + 1) % kStages;
-        const uint32_t par = (uint32_t)(jj / kStages) & 1u, par1 = (uint32_t)((jj + 1) / kStages) & 1u;
-        const bool more = jj + 1 < nt;
-        const uint32_t acc0 = jj > 0;
-        const uint64_t vd = vd0 + (uint64_t)st * (kTileDesc - (kTileDesc << 16));
-        const uint64_t kd1 = kd0 + (uint64_t)st1 * kTileDesc;
-        if (!mbar_wait(smem_u32(&v_full[st]), par, err, kErrWaitTmaFull)) { ok = false; break; }
-        if (!mbar_wait(smem_u32(&p_full[0]), (uint32_t)jj & 1u, err, kErrWaitAttnP)) { ok = false; break; }
+    }
+    for (int gt = 0; ok && gt < NT; ++gt) {
+      const int st = gt % kStages, st1 = (gt + 1) % kStages;
+      const uint32_t par = (uint32_t)(gt / kStages) & 1u, par1 = (uint32_t)((gt + 1) / kStages) & 1u;
+      const bool more = gt + 1 < NT;
+      const uint32_t acc0 = cur_first ? 0u : 1u;
+      const uint64_t vd = vd0 + (uint64_t)st * (kTileDesc - (kTileDesc << 16));
+      const uint64_t kd1 = kd0 + (uint64_t)st1 * kTileDesc;
+      bool nx_first = false, nx_last = false;
+      int nx_piece = cur_piece;
+      if (more) next_tile(nx_first, nx_last, nx_piece);
+      const int nqb = nx_piece & 1;
+      const uint64_t nqd = qd0 + (uint64_t)(2 * nqb) * kTileDesc;
+      if (!mbar_wait_warp(smem_u32(&v_full[st]), par, err, kErrWaitTmaFull)) { ok = false; break; }
+      if (!mbar_wait_warp(smem_u32(&p_full[0]), (uint32_t)gt & 1u, err, kErrWaitAttnP)) { ok = false; break; }
+      tc_fence_after();
+      DFP_ISSUE_PV(0, vd, acc0);
+      if (more) {
+        if (!mbar_wait_warp(smem_u32(&k_full[st1]), par1, err, kErrWaitTmaFull)) { ok = false; break; }
+        if (nx_first && !mbar_wait_warp(smem_u32(&q_full[nqb]), (nx_piece >> 1) & 1, err, kErrWaitTmaFull)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        DFP_ISSUE_PV(0, vd, acc0);
-        if (more) {
-          if (!mbar_wait(smem_u32(&k_full[st1]), par1, err, kErrWaitTmaFull)) { ok = false; break; }
-          tc_fence_after();
-          DFP_ISSUE_S(0, kd1);
-        }
-        if (two) {
-          if (!mbar_wait(smem_u32(&p_full[1]), (uint32_t)jj & 1u, err, kErrWaitAttnP)) { ok = false; break; }
-          tc_fence_after();
-          DFP_ISSUE_PV(1, vd, acc0);
-          if (more) DFP_ISSUE_S(1, kd1);
-        }
-        umma_commit(smem_u32(&v_empty[st]));
-        if (more) umma_commit(smem_u32(&k_empty[st1]));
+        DFP_ISSUE_S(0, nqd, kd1);
       }
+      if (!mbar_wait_warp(smem_u32(&p_full[1]), (uint32_t)gt & 1u, err, kErrWaitAttnP)) { ok = false; break; }
+      tc_fence_after();
+      DFP_ISSUE_PV(1, vd, acc0);
+      if (more) DFP_ISSUE_S(1, nqd + kTileDesc, kd1);
+      if (leader) {
+        umma_commit(smem_u32(&v_empty[st]));
+        if (more) {
+          umma_commit(smem_u32(&k_empty[st1]));
+          if (nx_last) umma_commit(smem_u32(&q_empty[nqb]));
+        }
+      }
+      __syncwarp();
+      cur_first = nx_first;
+      cur_last = nx_last;
+      cur_piece = nx_piece;
+    }
 #undef DFP_ISSUE_S
 #undef DFP_ISSUE_PV
-      if (!ok) s_abort = 1;
-    }
+    if (!ok && leader) s_abort = 1;
+    // every MMA issued by this CTA completes before its TMEM can be released
+    if (leader) umma_commit(smem_u32(mma_drain));
+    __syncwarp();
+    mbar_wait(smem_u32(mma_drain), 0, err, kErrWaitAccum);
    }
   } else {
     // ------------------------------------------------------------ softmax groups (warps 0..15)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax) : "memory");
     const int g = warp >> 3;                    // query tile of this warp
     const int half = (warp >> 2) & 1;           // key columns [64 half, 64 half + 64)
     const int sub = warp & 3;                   // TMEM lane quadrant
     const int row = sub * 32 + lane;
-    const bool active = g == 0 || activeB;
+    const bool group_leader = (warp & 7) == 0 && lane == 0;
     const uint32_t lane_off = (uint32_t)(sub * 32) << 16;
     const uint32_t tS = tmem + 128 * g + lane_off;
     const uint32_t tO = tmem + 256 + 128 * g + lane_off;
     const float sl2 = 0.125f * 1.4426950408889634f;   // (1/sqrt(64)) * log2(e)
-    float m_used = -INFINITY;
-    bool ok = active;
+    bool ok = true;
     // A failed wait only marks the thread; the group leaves the loop together at the
     // next max-exchange barrier (bar.red.or), so no thread is left waiting there.
     bool carry = false;                         // a failed wait of the previous tile
-    for (int jj = 0; ok && jj < nt; ++jj) {
-      int stale, krow, valid;
-      seg_tile(segs, j0 + jj, stale, krow, valid);
-      bool bad = !mbar_wait(smem_u32(&s_full[g]), jj & 1, err, kErrWaitAttnS) || carry;
-      tc_fence_after();
-      float sc[64];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + half * 64 + c * 32, r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sc[c * 32 + i] = __uint_as_float(r[i]);
-      }
-      tmem_wait_ld();
-      const int vcols = valid - half * 64;     // valid columns of this half (may be <= 0 or >= 64)
-      const bool full_tile = valid == kTile;
-      if (!full_tile) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) sc[i] = i < vcols ? sc[i] : -INFINITY;
-      }
-      float mx[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = max3(sc[i], sc[8 + i], sc[16 + i]);
-#pragma unroll
-      for (int i = 24; i < 64; i += 16) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], sc[i + k], i + 8 + k < 64 ? sc[i + 8 + k] : mx[k]);
-      }
-      const float mhalf = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-      // exchange with the other half of the row (double-buffered by tile parity)
-      s_rowmax[jj & 1][g][half][row] = mhalf;
-      if (named_bar_or(2 + g, 256, bad)) { ok = false; s_abort = 1; break; }
-      const float mrow = fmaxf(mhalf, s_rowmax[jj & 1][g][half ^ 1][row]) * sl2;
-      if (jj == 0) {
-        m_used = mrow;
-      } else {
-        const bool need = mrow > m_used + kRescale;
-        if (__any_sync(0xffffffffu, need)) {
-          // both halves of a row see the same mrow, so they agree on every decision
-          const float m_new = need ? mrow : m_used;
-          const float alpha = ex2_mufu(m_used - m_new);
-          if (!mbar_wait(smem_u32(&o_done[g]), (jj - 1) & 1, err, kErrWaitAttnO)) carry = true;
-          tc_fence_after();
-          // O (64 columns) and its row sums (16): half 0 rescales columns 0-39, half 1 40-79
-#pragma unroll
-          for (int c = 0; c < 5; ++c) {
-            uint32_t r8[8];
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                         : "=r"(r8[0]), "=r"(r8[1]), "=r"(r8[2]), "=r"(r8[3]), "=r"(r8[4]), "=r"(r8[5]),
-                           "=r"(r8[6]), "=r"(r8[7])
-                         : "r"(tO + half * 40 + c * 8));
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 8; ++i) r8[i] = __float_as_uint(__uint_as_float(r8[i]) * alpha);
-            asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
-                         ::"r"(tO + half * 40 + c * 8), "r"(r8[0]), "r"(r8[1]), "r"(r8[2]), "r"(r8[3]),
-                           "r"(r8[4]), "r"(r8[5]), "r"(r8[6]), "r"(r8[7])
-                         : "memory");
-          }
-          tmem_wait_st();
-          m_used = m_new;
-        }
-      }
-      const float nm = -m_used;
-      if (full_tile) {
-        // x = s * c - m on pairs (fp32x2); a fixed share of the pairs through the
-        // polynomial on the FMA pipe, the rest through the MUFU
-        const uint64_t sl2x2 = f2(sl2, sl2), nmx2 = f2(nm, nm);
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const uint64_t x2 = fma2(f2(sc[c * 32 + e], sc[c * 32 + e + 1]), sl2x2, nmx2);
-            if (((e >> 1) & 7) < kPolyPer8) {
-              pk[e >> 1] = ex2_poly_pair_bf16(x2);
-            } else {
-              float x0, x1;
-              f2_split(x2, x0, x1);
-              pk[e >> 1] = pack_trunc(ex2_mufu(x0), ex2_mufu(x1));
-            }
-          }
-          tmem_st16(tS + half * 32 + c * 16, pk);
-        }
-      } else {
-        // partial tile: masked columns are -inf, which only the MUFU maps to exactly 0
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2)
-            pk[e >> 1] = pack_trunc(ex2_mufu(fmaf(sc[c * 32 + e], sl2, nm)),
-                                    ex2_mufu(fmaf(sc[c * 32 + e + 1], sl2, nm)));
-          tmem_st16(tS + half * 32 + c * 16, pk);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(smem_u32(&p_full[g]));
+    // The group's current unit lives in shared memory (the group leader advances it
+    // between pieces): registers across the KV loop are all taken by the scores.
+    volatile int* sp = s_piece[g];
+    if (group_leader) {
+      const Unit u0 = locate(a, n_pairs, X0);
+      sp[0] = u0.p; sp[1] = u0.head; sp[2] = u0.pair; sp[3] = u0.T; sp[4] = u0.U0; sp[5] = X0;
     }
-    // every active thread of the group reaches this barrier exactly once
-    if (active && named_bar_or(2 + g, 256, carry || !ok)) { ok = false; s_abort = 1; }
-    // ---- epilogue: this half's 32 output columns and the row sum
-    float o[32], l = 1.f;
-    bool have = false;
-    if (ok && !s_abort) {
-      if (mbar_wait(smem_u32(&o_done[g]), (nt - 1) & 1, err, kErrWaitAttnO)) {
+    named_bar(2 + g, 256);
+    int gt = 0;
+    while (ok) {
+      int n;
+      {
+        const int x = sp[5];
+        if (x >= X1) break;
+        n = min(sp[4] + sp[3], X1) - x;
+      }
+      float m_used = -INFINITY;
+      for (int jj = 0; jj < n; ++jj, ++gt) {
+        int stale, krow, valid;
+        tile_src(a.mode, sp[0], a.Lp, a.L, a.kv_len, sp[5] - sp[4] + jj, stale, krow, valid);
+        bool bad = !mbar_wait(smem_u32(&s_full[g]), gt & 1, err, kErrWaitAttnS) || carry;
         tc_fence_after();
-        uint32_t r[32], r16[16];
-        tmem_ld32(tO + half * 32, r);
-        tmem_ld16(tO + 64, r16);
+        float sc[64];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(tS + half * 64 + cc * 32, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sc[cc * 32 + i] = __uint_as_float(r[i]);
+        }
         tmem_wait_ld();
+        const int vcols = valid - half * 64;     // valid columns of this half (may be <= 0 or >= 64)
+        const bool full_tile = valid == kTile;
+        if (!full_tile) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(r[i]);
-        l = __uint_as_float(r16[0]);
-        have = true;
-      } else {
-        s_abort = 1;
-      }
-    }
-    const int q_local = (qt0 + g) * kTile + row;
-    const bool row_ok = have && q_local < a.Lp;
-    __nv_bfloat16* out_row = static_cast<__nv_bfloat16*>(a.o) + (size_t)(p * a.Lp + q_local) * a.C + head * 64 + half * 32;
-    if (splits == 1) {
-      if (row_ok) {
-        const float inv = 1.f / l;
-        uint4* dst = reinterpret_cast<uint4*>(out_row);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float w8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) w8[e] = o[c * 8 + e] * inv;
-          dst[c] = pack16(w8);
+          for (int i = 0; i < 64; ++i) sc[i] = i < vcols ? sc[i] : -INFINITY;
         }
-      }
-    } else {
-      // partial results of this split, then the last CTA of the pair merges them
-      const size_t grp = ((size_t)head * a.N + p) * ((a.n_qtiles + 1) / 2) + pair;
-      const size_t slot = (grp * splits + split) * 256 + g * 128 + row;
-      if (have) {
-        float4* po = reinterpret_cast<float4*>(a.part_o + slot * 64 + half * 32);
+        float mx[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) po[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-        if (half == 0) reinterpret_cast<float2*>(a.part_ml)[slot] = make_float2(m_used, l);
-      }
-      __threadfence();
-      named_bar(1, kSoftmaxThreads);
-      if (threadIdx.x == 0) s_last = atomicAdd(a.counters + grp, 1u) == (unsigned)(splits - 1);
-      named_bar(1, kSoftmaxThreads);
-      if (s_last) {
-        __threadfence();
-        if (row_ok) {
-          float mm = -INFINITY;
-          for (int s2 = 0; s2 < splits; ++s2)
-            mm = fmaxf(mm, __ldcg(reinterpret_cast<const float2*>(a.part_ml) + (grp * splits + s2) * 256 + g * 128 + row).x);
-          float acc[32], lsum = 0.f;
+        for (int i = 0; i < 8; ++i) mx[i] = max3(sc[i], sc[8 + i], sc[16 + i]);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-          for (int s2 = 0; s2 < splits; ++s2) {
-            const size_t sl = (grp * splits + s2) * 256 + g * 128 + row;
-            const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sl);
-            const float w = ex2_mufu(ml.x - mm);
-            lsum = fmaf(ml.y, w, lsum);
-            const float4* po = reinterpret_cast<const float4*>(a.part_o + sl * 64 + half * 32);
+        for (int i = 24; i < 64; i += 16) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const float4 v = __ldcg(po + c);
-              acc[4 * c] = fmaf(v.x, w, acc[4 * c]);
-              acc[4 * c + 1] = fmaf(v.y, w, acc[4 * c + 1]);
-              acc[4 * c + 2] = fmaf(v.z, w, acc[4 * c + 2]);
-              acc[4 * c + 3] = fmaf(v.w, w, acc[4 * c + 3]);
+          for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], sc[i + k], i + 8 + k < 64 ? sc[i + 8 + k] : mx[k]);
+        }
+        const float mhalf = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+        // exchange with the other half of the row (double-buffered by tile parity)
+        s_rowmax[gt & 1][g][half][row] = mhalf;
+        if (named_bar_or(2 + g, 256, bad)) { ok = false; break; }
+        const float mrow = fmaxf(mhalf, s_rowmax[gt & 1][g][half ^ 1][row]) * sl2;
+        if (jj == 0) {
+          m_used = mrow;
+        } else {
+          const bool need = mrow > m_used + kRescale;
+          if (__any_sync(0xffffffffu, need)) {
+            // both halves of a row see the same mrow, so they agree on every decision
+            const float m_new = need ? mrow : m_used;
+            const float alpha = ex2_mufu(m_used - m_new);
+            if (!mbar_wait(smem_u32(&o_done[g]), (gt - 1) & 1, err, kErrWaitAttnO)) carry = true;
+            tc_fence_after();
+            // O (64 columns) and its row sums (16): half 0 rescales columns 0-39, half 1 40-79
+#pragma unroll
+            for (int cc = 0; cc < 5; ++cc) {
+              uint32_t r8[8];
+              asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                           : "=r"(r8[0]), "=r"(r8[1]), "=r"(r8[2]), "=r"(r8[3]), "=r"(r8[4]), "=r"(r8[5]),
+                             "=r"(r8[6]), "=r"(r8[7])
+                           : "r"(tO + half * 40 + cc * 8));
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 8; ++i) r8[i] = __float_as_uint(__uint_as_float(r8[i]) * alpha);
+              asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                           ::"r"(tO + half * 40 + cc * 8), "r"(r8[0]), "r"(r8[1]), "r"(r8[2]), "r"(r8[3]),
+                             "r"(r8[4]), "r"(r8[5]), "r"(r8[6]), "r"(r8[7])
+                           : "memory");
             }
-          }
-          const float inv = 1.f / lsum;
-          uint4* dst = reinterpret_cast<uint4*>(out_row);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float w8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w8[e] = acc[c * 8 + e] * inv;
-            dst[c] = pack16(w8);
+            tmem_wait_st();
+            m_used = m_new;
           }
         }
-        if (threadIdx.x == 0) a.counters[grp] = 0u;
+        const float nm = -m_used;
+        if (full_tile) {
+          // x = s * c - m on pairs (fp32x2); a fixed share of the pairs through the
+          // polynomial on the FMA pipe, the rest through the MUFU
+          const uint64_t sl2x2 = f2(sl2, sl2), nmx2 = f2(nm, nm);
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              const uint64_t x2 = fma2(f2(sc[cc * 16 + e], sc[cc * 16 + e + 1]), sl2x2, nmx2);
+              if ((e >> 1) < kPolyPer8) {
+                pk[e >> 1] = ex2_poly_pair_bf16(x2);
+              } else {
+                float x0, x1;
+                f2_split(x2, x0, x1);
+                pk[e >> 1] = pack_trunc(ex2_mufu(x0), ex2_mufu(x1));
+              }
+            }
+            tmem_st8(tS + half * 32 + cc * 8, pk);
+          }
+        } else {
+          // partial tile: masked columns are -inf, which only the MUFU maps to exactly 0
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int e = 0; e < 16; e += 2)
+              pk[e >> 1] = pack_trunc(ex2_mufu(fmaf(sc[cc * 16 + e], sl2, nm)),
+                                      ex2_mufu(fmaf(sc[cc * 16 + e + 1], sl2, nm)));
+            tmem_st8(tS + half * 32 + cc * 8, pk);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&p_full[g]));
       }
+      if (!ok) break;
+      // every thread of the group reaches this barrier once per piece
+      if (named_bar_or(2 + g, 256, carry)) { ok = false; break; }
+      // ---- piece epilogue (out of line: its registers do not add to the KV loop's)
+      Unit u;
+      u.p = sp[0]; u.head = sp[1]; u.pair = sp[2]; u.T = sp[3]; u.U0 = sp[4];
+      if (!piece_epilogue(a, u, tO, smem_u32(&o_done[g]), (uint32_t)(gt - 1) & 1u, m_used, g, half, row,
+                          group_leader, c, X0, &s_last[g]))
+        carry = true;
+      // next piece: every thread of the group is done with s_piece before it changes
+      named_bar(2 + g, 256);
+      if (group_leader) {
+        const int x_next = min(u.U0 + u.T, X1);
+        advance(a, n_pairs, u);
+        sp[0] = u.p; sp[1] = u.head; sp[2] = u.pair; sp[3] = u.T; sp[4] = u.U0; sp[5] = x_next;
+      }
+      named_bar(2 + g, 256);
     }
+    if (!ok || carry) s_abort = 1;
   }
 
   tc_fence_before();
@@ -590,31 +792,38 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
 
 }  // namespace
 
-int attention_splits(int L, int Lp, int N, int heads, int mode_min_tiles) {
-  const int n_qt = (Lp + kTile - 1) / kTile;
-  const int groups = ((n_qt + 1) / 2) * N * heads;
-  int best = 1;
-  double best_eff = 0.0;
-  for (int s = 1; s <= 4; ++s) {
-    if (s > 1 && mode_min_tiles / s < 2) break;
-    const long items = (long)groups * s;
-    const long waves = (items + 147) / 148;
-    const double eff = (double)items / (double)(waves * 148);
-    if (eff > best_eff + 0.03) { best_eff = eff; best = s; }
-    if (eff >= 0.7) break;   // each split adds a CTA prologue and a merge: stop early
-  }
-  return best;
+long long attention_total_tiles(const TcAttnArgs& a) {
+  const int n_pairs = (a.n_qtiles + 1) / 2;
+  long long tt = 0;
+  for (int p = 0; p < a.N; ++p) tt += (long long)unit_tiles(a.mode, p, a.Lp, a.L, a.kv_len) * a.heads * n_pairs;
+  return tt;
 }
 
-cudaError_t launch_tc_attention(const TcAttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mkf,
+size_t attention_scratch_floats(int ctas) { return (size_t)ctas * 2 * 256 * 64; }
+
+cudaError_t launch_tc_attention(const TcAttnArgs& args, const CUtensorMap& mq, const CUtensorMap& mkf,
                                 const CUtensorMap& mvf, const CUtensorMap& mks,
                                 const CUtensorMap& mvs, cudaStream_t s) {
-  const size_t smem = 1024 + (2 + 2 * kStages + 1) * (size_t)kTileBytes + (4 * kStages + 8) * 8 + 64;
+  const size_t smem = 1024 + (4 + 2 * kStages + 1) * (size_t)kTileBytes + (4 * kStages + 12) * 8 + 64;
   cudaError_t e = cudaFuncSetAttribute(tc_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int n_qt = (a.Lp + kTile - 1) / kTile;
-  dim3 grid(((n_qt + 1) / 2) * a.splits, a.N, a.heads);
-  tc_attention_kernel<<<grid, kThreads, smem, s>>>(mq, mkf, mvf, mks, mvs, a);
+  // The register split inside the kernel (setmaxnreg) hands the launch's registers from
+  // one warpgroup to the others; it needs the full 96 per thread at launch.
+  static int regs = 0;
+  if (!regs) {
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, tc_attention_kernel);
+    if (e != cudaSuccess) return e;
+    regs = fa.numRegs;
+  }
+  if (regs * kThreads < 128 * kRegsTmaMma + 512 * kRegsSoftmax) return cudaErrorInvalidConfiguration;
+  TcAttnArgs a = args;
+  const long long tt = attention_total_tiles(a);
+  if (tt <= 0) return cudaSuccess;
+  const int G = (int)std::min<long long>(a.ctas, tt);
+  if (G <= 0 || tt * G >= (1ll << 31)) return cudaErrorInvalidValue;   // 32-bit schedule arithmetic
+  a.total_tiles = (int)tt;
+  tc_attention_kernel<<<G, kThreads, smem, s>>>(mq, mkf, mvf, mks, mvs, a);
   return cudaGetLastError();
 }
 

@@ -405,6 +405,13 @@ bool encode_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, 
   const cuuint32_t box[3] = {b0, b1, b2};
   return encode(m, base, 3, dims, strides, box);
 }
+bool encode_tmap_5d(CUtensorMap* m, const void* base, const uint64_t dims[5],
+                    const uint64_t strides_bytes[4], const uint32_t box[5]) {
+  const cuuint64_t d[5] = {dims[0], dims[1], dims[2], dims[3], dims[4]};
+  const cuuint64_t st[4] = {strides_bytes[0], strides_bytes[1], strides_bytes[2], strides_bytes[3]};
+  const cuuint32_t b[5] = {box[0], box[1], box[2], box[3], box[4]};
+  return encode(m, base, 5, d, st, b);
+}
 bool encode_tmap_4d(CUtensorMap* m, const void* base, const uint64_t dims[4],
                     const uint64_t strides_bytes[3], const uint32_t box[4]) {
   const cuuint64_t d[4] = {dims[0], dims[1], dims[2], dims[3]};
