@@ -117,7 +117,7 @@ dfp_status build_tmaps(dfp_ctx* h) {
   ok &= encode_tmap_3d(&h->m_q, h->q, 64, L, heads, 128, (uint64_t)L * 128, 64, 128, 1);
   for (int i = 0; i < 2; ++i) {
     ok &= encode_tmap_3d(&h->m_k[i], h->kb[i], 64, L, heads, 128, (uint64_t)L * 128, 64, 128, 1);
-    ok &= encode_tmap_3d(&h->m_v[i], h->vb[i], 64, L, heads, 128, (uint64_t)L * 128, 64, 128, 1);
+    ok &= encode_attn_v(&h->m_v[i], h->vb[i], L, heads);
   }
   if (!ok) return h->fail(DFP_E_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
   TcGemmPlan& cp = h->conv_plan;

@@ -58,6 +58,9 @@ struct Stage {
 
 namespace {
 
+// rows per head of the context K/V buffers: ctx_len padded with zeros to whole 128-key tiles
+size_t ctx_rows(size_t ctx_len) { return (ctx_len + 127) / 128 * 128; }
+
 uint16_t f32_to_bf16(float f) {
   uint32_t u;
   std::memcpy(&u, &f, 4);
@@ -147,7 +150,8 @@ dfp_status stage_create(dfp_ctx* h) {
     ok &= h->alloc((void**)&x.b_o1, C * 4) && h->alloc((void**)&x.b_o2, C * 4);
     ok &= h->alloc((void**)&x.b_ff1, 2 * F * 4) && h->alloc((void**)&x.b_ff2, C * 4);
     for (int i = 0; i < 2; ++i) ok &= h->alloc(&x.kb[i], map) && h->alloc(&x.vb[i], map);
-    ok &= h->alloc(&x.ctx_k, heads * T * 64 * 2) && h->alloc(&x.ctx_v, heads * T * 64 * 2);
+    // context K/V: ctx_len rows per head padded with zeros to whole 128-key tiles
+    ok &= h->alloc(&x.ctx_k, heads * ctx_rows(T) * 64 * 2) && h->alloc(&x.ctx_v, heads * ctx_rows(T) * 64 * 2);
   }
   if (!ok) return h->fail(DFP_E_NOMEM, "device allocation failed");
   cudaError_t e = cudaSuccess;
@@ -160,7 +164,10 @@ dfp_status stage_create(dfp_ctx* h) {
       e = cudaMemset(st->xf[b].kb[i], 0, map);
       if (e == cudaSuccess) e = cudaMemset(st->xf[b].vb[i], 0, map);
     }
-
+  for (int b = 0; b < c.n_xformer && e == cudaSuccess; ++b) {
+    e = cudaMemset(st->xf[b].ctx_k, 0, heads * ctx_rows(T) * 64 * 2);
+    if (e == cudaSuccess) e = cudaMemset(st->xf[b].ctx_v, 0, heads * ctx_rows(T) * 64 * 2);
+  }
   if (e != cudaSuccess) return h->cuda_fail(e, "cudaMemset");
   h->y = st->r.back();
 
@@ -200,10 +207,10 @@ dfp_status stage_create(dfp_ctx* h) {
     ok &= encode_gemm_rows(&x.m_wff2, x.w_ff2, C, F, bc);   // same N = C as to_out
     for (int i = 0; i < 2; ++i) {
       ok &= encode_tmap_3d(&x.m_k[i], x.kb[i], 64, L, heads, 128, L * 128, 64, 128, 1);
-      ok &= encode_tmap_3d(&x.m_v[i], x.vb[i], 64, L, heads, 128, L * 128, 64, 128, 1);
+      ok &= encode_attn_v(&x.m_v[i], x.vb[i], L, heads);
     }
-    ok &= encode_tmap_3d(&x.m_ck, x.ctx_k, 64, T, heads, 128, T * 128, 64, 128, 1);
-    ok &= encode_tmap_3d(&x.m_cv, x.ctx_v, 64, T, heads, 128, T * 128, 64, 128, 1);
+    ok &= encode_tmap_3d(&x.m_ck, x.ctx_k, 64, ctx_rows(T), heads, 128, ctx_rows(T) * 128, 64, 128, 1);
+    ok &= encode_attn_v(&x.m_cv, x.ctx_v, ctx_rows(T), heads);
     plan(x.p_qkv, (int)L, 3 * (int)C, (int)C, bq);
     plan(x.p_o1, (int)L, (int)C, (int)C, bc);
     plan(x.p_q2, (int)L, (int)C, (int)C, bc);
@@ -295,7 +302,7 @@ dfp_status stage_finish_load(dfp_ctx* h) {
       continue;
     for (int kv = 0; kv < 2; ++kv) {
       Epilogue e{};
-      e.kind = 1; e.q = kv == 0 ? x.ctx_k : x.ctx_v; e.L = c.ctx_len; e.C = c.C;
+      e.kind = 1; e.q = kv == 0 ? x.ctx_k : x.ctx_v; e.L = (int)ctx_rows(c.ctx_len); e.C = c.C;   // padded head stride
       cudaError_t ce = launch_simt_gemm<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(st->ctx), nullptr,
                                                        static_cast<const __nv_bfloat16*>(kv == 0 ? x.w_k2 : x.w_v2),
                                                        c.ctx_len, c.C, c.ctx_dim, e, h->stream);

@@ -244,6 +244,29 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
+// 16x64b shapes: a warp reads / writes 16 TMEM lanes; lane t of the warp holds row
+// 8*(t%2) + t/4 of those 16 and, per 2-column repeat r, column 2r + (t/2)%2.
+__device__ __forceinline__ void tmem_ld_16x64b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x64b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_16x64b_x8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x64b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st_16x64b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.16x64b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -399,7 +422,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
   __shared__ volatile int s_abort;
   __shared__ int s_last[2];
-  __shared__ float s_rowmax[2][2][2][128];   // [tile parity][group][half][row]
+  __shared__ float s_mrow[2][128];           // [group][row]: running max handed to the piece epilogue
   __shared__ int s_piece[2][8];               // per group: p, head, pair, T, U0, piece start
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -489,7 +512,8 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
         }
         if (leader) {
           mbar_arrive_expect_tx(smem_u32(&v_full[s]), kTileBytes);
-          tma_load_3d(smem_u32(sV + s * kTileBytes), stale ? &mvs : &mvf, smem_u32(&v_full[s]), 0, row, u.head);
+          tma_load_5d(smem_u32(sV + s * kTileBytes), stale ? &mvs : &mvf, smem_u32(&v_full[s]), 0, 0, 0, row >> 2,
+                      u.head);
         }
         __syncwarp();
       }
@@ -632,18 +656,25 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
     // ------------------------------------------------------------ softmax groups (warps 0..15)
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax) : "memory");
     const int g = warp >> 3;                    // query tile of this warp
-    const int half = (warp >> 2) & 1;           // key columns [64 half, 64 half + 64)
-    const int sub = warp & 3;                   // TMEM lane quadrant
-    const int row = sub * 32 + lane;
+    const int q4 = warp & 3;                    // TMEM lane quadrant (fixed by the warp's SM sub-partition)
+    const int h16 = (warp >> 2) & 1;            // which 16 lanes of the quadrant
+    // KV loop (16x64b shapes): two lanes of a warp share a query row, each holding 64 of
+    // its 128 score columns (2r + cq); they exchange row maxima with one shuffle.
+    const int cq = (lane >> 1) & 1;
+    const uint32_t lane16 = (uint32_t)(32 * q4 + 16 * h16) << 16;
+    const uint32_t tS = tmem + 128 * g + lane16;
+    const uint32_t tO = tmem + 256 + 128 * g + lane16;
+    const int srow = 32 * q4 + 16 * h16 + 8 * (lane & 1) + (lane >> 2);
+    // piece epilogue (32x32b shape): lane = row of the quadrant, h16 picks 32 output columns
+    const int erow = 32 * q4 + lane;
+    const uint32_t tOe = tmem + 256 + 128 * g + ((uint32_t)(32 * q4) << 16);
     const bool group_leader = (warp & 7) == 0 && lane == 0;
-    const uint32_t lane_off = (uint32_t)(sub * 32) << 16;
-    const uint32_t tS = tmem + 128 * g + lane_off;
-    const uint32_t tO = tmem + 256 + 128 * g + lane_off;
     const float sl2 = 0.125f * 1.4426950408889634f;   // (1/sqrt(64)) * log2(e)
     bool ok = true;
-    // A failed wait only marks the thread; the group leaves the loop together at the
-    // next max-exchange barrier (bar.red.or), so no thread is left waiting there.
-    bool carry = false;                         // a failed wait of the previous tile
+    // A failed wait makes the whole warp give up the piece (waits are agreed warp-wide,
+    // so the TMEM instructions stay warp-uniform); the group then leaves together at the
+    // piece barrier (bar.red.or), which every thread reaches once per piece.
+    bool carry = false;
     // The group's current unit lives in shared memory (the group leader advances it
     // between pieces): registers across the KV loop are all taken by the scores.
     volatile int* sp = s_piece[g];
@@ -661,25 +692,26 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
         n = min(sp[4] + sp[3], X1) - x;
       }
       float m_used = -INFINITY;
-      for (int jj = 0; jj < n; ++jj, ++gt) {
+      for (int jj = 0; jj < n && !carry; ++jj, ++gt) {
         int stale, krow, valid;
         tile_src(a.mode, sp[0], a.Lp, a.L, a.kv_len, sp[5] - sp[4] + jj, stale, krow, valid);
-        bool bad = !mbar_wait(smem_u32(&s_full[g]), gt & 1, err, kErrWaitAttnS) || carry;
+        if (!mbar_wait_warp(smem_u32(&s_full[g]), gt & 1, err, kErrWaitAttnS)) { carry = true; break; }
         tc_fence_after();
-        float sc[64];
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
+        float sc[64];   // sc[i] = S[row][2i + cq]
+        {
           uint32_t r[32];
-          tmem_ld32(tS + half * 64 + cc * 32, r);
+          tmem_ld_16x64b_x32(tS, r);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) sc[cc * 32 + i] = __uint_as_float(r[i]);
+          for (int i = 0; i < 32; ++i) sc[i] = __uint_as_float(r[i]);
+          tmem_ld_16x64b_x32(tS + 64, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sc[32 + i] = __uint_as_float(r[i]);
         }
         tmem_wait_ld();
-        const int vcols = valid - half * 64;     // valid columns of this half (may be <= 0 or >= 64)
         const bool full_tile = valid == kTile;
         if (!full_tile) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) sc[i] = i < vcols ? sc[i] : -INFINITY;
+          for (int i = 0; i < 64; ++i) sc[i] = 2 * i + cq < valid ? sc[i] : -INFINITY;
         }
         float mx[8];
 #pragma unroll
@@ -689,42 +721,36 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
 #pragma unroll
           for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], sc[i + k], i + 8 + k < 64 ? sc[i + 8 + k] : mx[k]);
         }
-        const float mhalf = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-        // exchange with the other half of the row (double-buffered by tile parity)
-        s_rowmax[gt & 1][g][half][row] = mhalf;
-        if (named_bar_or(2 + g, 256, bad)) { ok = false; break; }
-        const float mrow = fmaxf(mhalf, s_rowmax[gt & 1][g][half ^ 1][row]) * sl2;
+        float mrow = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+        mrow = fmaxf(mrow, __shfl_xor_sync(0xffffffffu, mrow, 2)) * sl2;   // the row's other half
         if (jj == 0) {
           m_used = mrow;
         } else {
           const bool need = mrow > m_used + kRescale;
           if (__any_sync(0xffffffffu, need)) {
-            // both halves of a row see the same mrow, so they agree on every decision
+            // both lanes of a row see the same mrow, so they agree on every decision
             const float m_new = need ? mrow : m_used;
             const float alpha = ex2_mufu(m_used - m_new);
-            if (!mbar_wait(smem_u32(&o_done[g]), (gt - 1) & 1, err, kErrWaitAttnO)) carry = true;
+            if (!mbar_wait_warp(smem_u32(&o_done[g]), (gt - 1) & 1, err, kErrWaitAttnO)) { carry = true; break; }
             tc_fence_after();
-            // O (64 columns) and its row sums (16): half 0 rescales columns 0-39, half 1 40-79
+            // this lane's 40 of the row's 80 O columns (64 outputs + 16 row-sum columns)
 #pragma unroll
             for (int cc = 0; cc < 5; ++cc) {
               uint32_t r8[8];
-              asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                           : "=r"(r8[0]), "=r"(r8[1]), "=r"(r8[2]), "=r"(r8[3]), "=r"(r8[4]), "=r"(r8[5]),
-                             "=r"(r8[6]), "=r"(r8[7])
-                           : "r"(tO + half * 40 + cc * 8));
+              tmem_ld_16x64b_x8(tO + cc * 16, r8);
               tmem_wait_ld();
 #pragma unroll
               for (int i = 0; i < 8; ++i) r8[i] = __float_as_uint(__uint_as_float(r8[i]) * alpha);
-              asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
-                           ::"r"(tO + half * 40 + cc * 8), "r"(r8[0]), "r"(r8[1]), "r"(r8[2]), "r"(r8[3]),
-                             "r"(r8[4]), "r"(r8[5]), "r"(r8[6]), "r"(r8[7])
-                           : "memory");
+              tmem_st_16x64b_x8(tO + cc * 16, r8);
             }
             tmem_wait_st();
             m_used = m_new;
           }
         }
         const float nm = -m_used;
+        // P over S in TMEM: this lane packs its own neighbours sc[2r'], sc[2r'+1] (score
+        // columns 4r'+cq and 4r'+cq+2) into P column 2r'+cq, i.e. the key order within
+        // each group of 4 is 0, 2, 1, 3 -- the order in which V's rows are loaded.
         if (full_tile) {
           // x = s * c - m on pairs (fp32x2); a fixed share of the pairs through the
           // polynomial on the FMA pipe, the rest through the MUFU
@@ -733,17 +759,17 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
           for (int cc = 0; cc < 4; ++cc) {
             uint32_t pk[8];
 #pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              const uint64_t x2 = fma2(f2(sc[cc * 16 + e], sc[cc * 16 + e + 1]), sl2x2, nmx2);
-              if ((e >> 1) < kPolyPer8) {
-                pk[e >> 1] = ex2_poly_pair_bf16(x2);
+            for (int e = 0; e < 8; ++e) {
+              const uint64_t x2 = fma2(f2(sc[cc * 16 + 2 * e], sc[cc * 16 + 2 * e + 1]), sl2x2, nmx2);
+              if (e < kPolyPer8) {
+                pk[e] = ex2_poly_pair_bf16(x2);
               } else {
                 float x0, x1;
                 f2_split(x2, x0, x1);
-                pk[e >> 1] = pack_trunc(ex2_mufu(x0), ex2_mufu(x1));
+                pk[e] = pack_trunc(ex2_mufu(x0), ex2_mufu(x1));
               }
             }
-            tmem_st8(tS + half * 32 + cc * 8, pk);
+            tmem_st_16x64b_x8(tS + cc * 16, pk);
           }
         } else {
           // partial tile: masked columns are -inf, which only the MUFU maps to exactly 0
@@ -751,26 +777,27 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
           for (int cc = 0; cc < 4; ++cc) {
             uint32_t pk[8];
 #pragma unroll
-            for (int e = 0; e < 16; e += 2)
-              pk[e >> 1] = pack_trunc(ex2_mufu(fmaf(sc[cc * 16 + e], sl2, nm)),
-                                      ex2_mufu(fmaf(sc[cc * 16 + e + 1], sl2, nm)));
-            tmem_st8(tS + half * 32 + cc * 8, pk);
+            for (int e = 0; e < 8; ++e)
+              pk[e] = pack_trunc(ex2_mufu(fmaf(sc[cc * 16 + 2 * e], sl2, nm)),
+                                 ex2_mufu(fmaf(sc[cc * 16 + 2 * e + 1], sl2, nm)));
+            tmem_st_16x64b_x8(tS + cc * 16, pk);
           }
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(smem_u32(&p_full[g]));
       }
-      if (!ok) break;
+      // the row's lazily updated maximum, for the epilogue's (32x32b) row owner
+      if (cq == 0) s_mrow[g][srow] = m_used;
       // every thread of the group reaches this barrier once per piece
       if (named_bar_or(2 + g, 256, carry)) { ok = false; break; }
       // ---- piece epilogue (out of line: its registers do not add to the KV loop's)
       Unit u;
       u.p = sp[0]; u.head = sp[1]; u.pair = sp[2]; u.T = sp[3]; u.U0 = sp[4];
-      if (!piece_epilogue(a, u, tO, smem_u32(&o_done[g]), (uint32_t)(gt - 1) & 1u, m_used, g, half, row,
-                          group_leader, c, X0, &s_last[g]))
+      if (!piece_epilogue(a, u, tOe, smem_u32(&o_done[g]), (uint32_t)(gt - 1) & 1u, s_mrow[g][erow], g, h16,
+                          erow, group_leader, c, X0, &s_last[g]))
         carry = true;
-      // next piece: every thread of the group is done with s_piece before it changes
+      // next piece: every thread of the group is done with s_piece (and s_mrow) before it changes
       named_bar(2 + g, 256);
       if (group_leader) {
         const int x_next = min(u.U0 + u.T, X1);
@@ -791,6 +818,15 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
 }
 
 }  // namespace
+
+bool encode_attn_v(CUtensorMap* m, const void* base, uint64_t rows, uint64_t heads) {
+  // key = 4 s + q + 2 e lands in shared-memory row 4 s + 2 q + e: dims (d, e, q, s, head)
+  const uint64_t dims[5] = {64, 2, 2, (rows + 3) / 4, heads};
+  const uint64_t strides[4] = {256, 128, 512, rows * 128};
+  const uint32_t box[5] = {64, 2, 2, 32, 1};
+  if (rows % 4) return false;
+  return encode_tmap_5d(m, base, dims, strides, box);
+}
 
 long long attention_total_tiles(const TcAttnArgs& a) {
   const int n_pairs = (a.n_qtiles + 1) / 2;
