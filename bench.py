@@ -75,11 +75,9 @@ def work_model(cfg):
         F, T = cfg["ffn_inner"], cfg["ctx_len"]
         ln = ("hbm", 2 * L * C * e)
         wm = {
-            "norm1 statistics": ("hbm", L * C * e),
-            "norm1 apply + halo": ("hbm", 2 * L * C * e + 2 * 2 * (N - 1) * W * C * e),
+            "norm1 + SiLU + halo (fused)": ("hbm", 2 * L * C * e + 2 * 2 * (N - 1) * W * C * e),
             "conv1 (tcgen05)": ("tensor", 2.0 * L * C * 9 * C),
-            "norm2 statistics": ("hbm", L * C * e),
-            "norm2 apply + halo": ("hbm", 2 * L * C * e + 2 * 2 * (N - 1) * W * C * e),
+            "norm2 + SiLU + halo (fused)": ("hbm", 2 * L * C * e + 2 * 2 * (N - 1) * W * C * e),
             "conv2 + residual (tcgen05)": ("tensor", 2.0 * L * C * 9 * C),
             "layernorm 1": ln, "layernorm 2": ln, "layernorm 3": ln,
             "self-attn qkv (tcgen05)": ("tensor", 2.0 * L * C * 3 * C),
@@ -96,11 +94,9 @@ def work_model(cfg):
         wm["_rows_per_patch"] = R
         return wm
     return {
-        "gn1 statistics": ("hbm", L * C * e),
-        "gn1 apply + halo": ("hbm", 2 * L * C * e + 2 * 2 * (N - 1) * W * C * e),
+        "gn1 + SiLU + halo (fused)": ("hbm", 2 * L * C * e + 2 * 2 * (N - 1) * W * C * e),
         "conv (tcgen05)": ("tensor", 2.0 * L * C * 9 * C),
-        "gn2 statistics": ("hbm", L * C * e),
-        "gn2 apply": ("hbm", 2 * L * C * e),
+        "gn2 (fused)": ("hbm", 2 * L * C * e),
         "qkv (tcgen05)": ("tensor", 2.0 * L * C * 3 * C),
         "attention (tcgen05)": ("tensor", 4.0 * L * L * d * heads),
         "out projection (tcgen05)": ("tensor", 2.0 * L * C * C),

@@ -116,7 +116,7 @@ dfp_status build_tmaps(dfp_ctx* h) {
   const int heads = c.heads;
   ok &= encode_tmap_3d(&h->m_q, h->q, 64, L, heads, 128, (uint64_t)L * 128, 64, 128, 1);
   for (int i = 0; i < 2; ++i) {
-    ok &= encode_tmap_3d(&h->m_k[i], h->kb[i], 64, L, heads, 128, (uint64_t)L * 128, 64, 128, 1);
+    ok &= encode_attn_k(&h->m_k[i], h->kb[i], L, heads);
     ok &= encode_attn_v(&h->m_v[i], h->vb[i], L, heads);
   }
   if (!ok) return h->fail(DFP_E_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
@@ -541,12 +541,18 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   g.fresh_out = h->mom1[cur]; g.stale = h->mom1[prv];
   g.gamma = h->gn1_g; g.beta = h->gn1_b; g.dbg = h->dbg1;
   g.is_sync = is_sync; g.mode = (int)c.gn_mode; g.naive = naive ? 1 : 0;
-  DFP_LAUNCH(launch_gn_stats_merge<T>(g, s), "gn1 statistics");
-  // the same kernel fills the halo rows: the neighbours' boundary rows of this step
+  // the apply also fills the halo rows: the neighbours' boundary rows of this step
   // (sync) or of the previous step (displaced, read from the other slab buffer)
   const int halo_mode = (naive || N == 1) ? 0 : (displaced ? 2 : 1);
-  DFP_LAUNCH(launch_gn_apply<T>(x, slab, static_cast<const T*>(h->slab[prv]), h->dbg1, h->gn1_g, h->gn1_b, G, N, Lp, C, W,
-                                (long long)(R + 2) * W, W, true, halo_mode, s), "gn1 apply + halo");
+  if (h->family == 0) {
+    // statistics, merge and apply in one cooperative launch
+    const GnOut go{slab, h->slab[prv], (long long)(R + 2) * W, W, W, halo_mode};
+    DFP_LAUNCH(launch_gn_fused<T>(g, go, true, h->dev_err, s), "gn1 + SiLU + halo (fused)");
+  } else {
+    DFP_LAUNCH(launch_gn_stats_merge<T>(g, s), "gn1 statistics");
+    DFP_LAUNCH(launch_gn_apply<T>(x, slab, static_cast<const T*>(h->slab[prv]), h->dbg1, h->gn1_g, h->gn1_b, G, N, Lp,
+                                  C, W, (long long)(R + 2) * W, W, true, halo_mode, s), "gn1 apply + halo");
+  }
   // ---- conv3x3 (+ bias) -> h
   Epilogue ec{};
   ec.kind = 0; ec.out = h->h; ec.bias = h->b_conv; ec.ldo = C;
@@ -559,9 +565,14 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   // ---- GN2 (no SiLU) -> t
   g.x = h->h; g.fresh_out = h->mom2[cur]; g.stale = h->mom2[prv];
   g.gamma = h->gn2_g; g.beta = h->gn2_b; g.dbg = h->dbg2;
-  DFP_LAUNCH(launch_gn_stats_merge<T>(g, s), "gn2 statistics");
-  DFP_LAUNCH(launch_gn_apply<T>(static_cast<const T*>(h->h), static_cast<T*>(h->t), nullptr, h->dbg2, h->gn2_g, h->gn2_b, G, N, Lp,
-                                C, W, (long long)Lp, 0, false, 0, s), "gn2 apply");
+  if (h->family == 0) {
+    const GnOut go{h->t, nullptr, (long long)Lp, 0, W, 0};
+    DFP_LAUNCH(launch_gn_fused<T>(g, go, false, h->dev_err, s), "gn2 (fused)");
+  } else {
+    DFP_LAUNCH(launch_gn_stats_merge<T>(g, s), "gn2 statistics");
+    DFP_LAUNCH(launch_gn_apply<T>(static_cast<const T*>(h->h), static_cast<T*>(h->t), nullptr, h->dbg2, h->gn2_g,
+                                  h->gn2_b, G, N, Lp, C, W, (long long)Lp, 0, false, 0, s), "gn2 apply");
+  }
   // ---- Q, K, V projections; K/V land in this step's cache buffers
   Epilogue eq{};
   eq.kind = 1; eq.q = h->q; eq.k = h->kb[cur]; eq.v = h->vb[cur]; eq.L = L; eq.C = C;

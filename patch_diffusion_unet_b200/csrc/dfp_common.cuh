@@ -20,6 +20,7 @@ enum DeviceError : int {
   kErrWaitAttnS = 4,       // softmax waited too long for S = Q K^T
   kErrWaitAttnP = 5,       // MMA waited too long for P
   kErrWaitAttnO = 6,       // softmax waited too long for P V
+  kErrGridSync = 7,        // a block waited too long at a grid-wide barrier
 };
 
 // Limit of every spin-wait, in SM clock cycles (about 2 s at the B200's maximum

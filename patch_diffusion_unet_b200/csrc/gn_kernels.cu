@@ -13,6 +13,8 @@
 // The reductions are deterministic: per-thread sums in a fixed pixel order, a
 // fixed-order shared-memory tree, and a last-block merge over the chunk partials
 // in a fixed order (no floating-point atomics).
+#include <algorithm>
+
 #include "dfp_common.cuh"
 #include "kernels.h"
 
@@ -237,6 +239,212 @@ gn_apply_kernel(const T* __restrict__ x, T* __restrict__ out, const T* __restric
   }
 }
 
+// ---------------------------------------------------------------- fused GroupNorm
+// Statistics, merge and apply in one cooperative launch (every block resident): each
+// block sums its chunk, all blocks meet at a grid barrier, then every block reduces
+// the chunk partials of the patches it needs (its own; all of them on sync steps) in
+// a fixed order, applies the same merge rule as above and normalises its chunk (the
+// map was just read, so the second read is served by L2).  Block (0, p) publishes
+// patch p's fresh moments and (mean, rstd).  counter[0] counts arrivals at the
+// barrier and counter[1] departures; the last block to leave zeroes both.
+
+__device__ __forceinline__ bool grid_barrier(unsigned* count, unsigned total, int* err) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(count, 1u);
+    int ok = 1;
+    const long long t0 = clock64();
+    while (*reinterpret_cast<volatile unsigned*>(count) < total) {
+      if (clock64() - t0 > kWaitLimitCycles) {
+        atomicCAS(err, 0, kErrGridSync);
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+template <typename T, bool SILU>
+__global__ void __launch_bounds__(kGnThreads, 2)
+gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
+  constexpr int VEC = VecTraits<T>::kN;
+  extern __shared__ float sh[];                 // [2][PL][C] lane sums, then [2][C] channel sums
+  __shared__ float s_mr[256 * 2];               // (mean, rstd) of this patch's groups
+  __shared__ float s_mom[256 * 2];              // fresh moments of the patches needed
+  const int C = a.C, G = a.G, N = a.N;
+  const int V = C / VEC;
+  const int PL = kGnThreads / V;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int vc = tid % V, pl = tid / V;
+  const int p = blockIdx.y, chunk = blockIdx.x;
+  const int pix0 = chunk * pix_per_chunk;
+  const int pix1 = min(pix0 + pix_per_chunk, a.pix_per_patch);
+  const T* base = static_cast<const T*>(a.x) + (size_t)p * a.pix_per_patch * C + vc * VEC;
+  float* chan = sh + 2 * PL * C;
+
+  // ---- phase 1: per-channel partial sums of this chunk (8 loads in flight)
+  {
+    float s1[VEC], s2[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) s1[i] = s2[i] = 0.f;
+    if (pl < PL) {
+      for (int pix = pix0 + pl; pix < pix1; pix += 8 * PL) {
+        uint4 u[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          u[j] = pix + j * PL < pix1 ? ld_nc16(base + (size_t)(pix + j * PL) * C) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float v[VEC];
+          unpack16(u[j], v);
+#pragma unroll
+          for (int i = 0; i < VEC; ++i) { s1[i] += v[i]; s2[i] = fmaf(v[i], v[i], s2[i]); }
+        }
+      }
+      float4* d1 = reinterpret_cast<float4*>(sh + pl * C + vc * VEC);
+      float4* d2 = reinterpret_cast<float4*>(sh + PL * C + pl * C + vc * VEC);
+#pragma unroll
+      for (int i = 0; i < VEC / 4; ++i) {
+        d1[i] = make_float4(s1[4 * i], s1[4 * i + 1], s1[4 * i + 2], s1[4 * i + 3]);
+        d2[i] = make_float4(s2[4 * i], s2[4 * i + 1], s2[4 * i + 2], s2[4 * i + 3]);
+      }
+    }
+  }
+  __syncthreads();
+  for (int c = tid; c < C; c += kGnThreads) {
+    float t1 = 0.f, t2 = 0.f;
+    for (int l = 0; l < PL; ++l) { t1 += sh[l * C + c]; t2 += sh[PL * C + l * C + c]; }
+    chan[c] = t1;
+    chan[C + c] = t2;
+  }
+  __syncthreads();
+  const int cg = C / G;
+  for (int g = warp; g < G; g += kGnThreads / 32) {
+    float t1 = 0.f, t2 = 0.f;
+    for (int c = lane; c < cg; c += 32) { t1 += chan[g * cg + c]; t2 += chan[C + g * cg + c]; }
+    t1 = warp_sum(t1);
+    t2 = warp_sum(t2);
+    if (lane == 0) reinterpret_cast<float2*>(a.part)[((size_t)p * n_chunks + chunk) * G + g] = make_float2(t1, t2);
+  }
+
+  // ---- grid barrier: every chunk partial is written
+  const unsigned total = gridDim.x * gridDim.y;
+  if (!grid_barrier(a.counter, total, err)) return;
+
+  // ---- phase 2: fresh moments of the patches needed, in a fixed order
+  const bool all = a.is_sync && !a.naive;       // sync steps merge every patch's fresh moments
+  const int p_lo = all ? 0 : p, np = all ? N : 1;
+  const int items = np * G;                     // <= 256
+  const int S = kGnThreads / items;             // threads per item, >= 2
+  float* red = sh;                              // [S][items][2]
+  if (tid < S * items) {
+    const int item = tid % items, part_id = tid / items;
+    const int pp = p_lo + item / G, gg = item % G;
+    const float2* src = reinterpret_cast<const float2*>(a.part) + (size_t)pp * n_chunks * G + gg;
+    float2 acc = make_float2(0.f, 0.f);
+    for (int c = part_id; c < n_chunks; c += S) {
+      const float2 v = __ldcg(src + (size_t)c * G);
+      acc.x += v.x; acc.y += v.y;
+    }
+    red[(part_id * items + item) * 2 + 0] = acc.x;
+    red[(part_id * items + item) * 2 + 1] = acc.y;
+  }
+  __syncthreads();
+  const float inv_n = 1.f / ((float)a.pix_per_patch * (float)cg);
+  if (tid < items) {
+    float t1 = 0.f, t2 = 0.f;
+    for (int s2 = 0; s2 < S; ++s2) { t1 += red[(s2 * items + tid) * 2]; t2 += red[(s2 * items + tid) * 2 + 1]; }
+    s_mom[tid * 2] = t1 * inv_n;
+    s_mom[tid * 2 + 1] = t2 * inv_n;
+  }
+  __syncthreads();
+  if (tid < G) {
+    const int gg = tid;
+    const int own = (all ? p : 0) * G + gg;     // this patch's entry in s_mom
+    const float m1 = s_mom[own * 2], m2 = s_mom[own * 2 + 1];
+    float e1, e2;
+    if (a.naive) {
+      e1 = m1; e2 = m2;
+    } else if (a.is_sync) {
+      e1 = 0.f; e2 = 0.f;
+      for (int j = 0; j < N; ++j) { e1 += s_mom[(j * G + gg) * 2]; e2 += s_mom[(j * G + gg) * 2 + 1]; }
+      e1 /= (float)N; e2 /= (float)N;
+    } else {
+      float st1 = 0.f, st2 = 0.f;
+      for (int j = 0; j < N; ++j) { st1 += a.stale[(j * G + gg) * 2]; st2 += a.stale[(j * G + gg) * 2 + 1]; }
+      const float own1 = a.stale[(p * G + gg) * 2], own2 = a.stale[(p * G + gg) * 2 + 1];
+      if (a.mode == 0) {        // corrected
+        e1 = st1 / (float)N + (m1 - own1);
+        e2 = st2 / (float)N + (m2 - own2);
+      } else {                  // stale others
+        e1 = (m1 + (st1 - own1)) / (float)N;
+        e2 = (m2 + (st2 - own2)) / (float)N;
+      }
+    }
+    const float rstd = 1.f / sqrtf(fmaxf(e2 - e1 * e1, 0.f) + a.eps);
+    s_mr[gg * 2] = e1;
+    s_mr[gg * 2 + 1] = rstd;
+    if (chunk == 0) {
+      a.fresh_out[(p * G + gg) * 2] = m1;
+      a.fresh_out[(p * G + gg) * 2 + 1] = m2;
+      a.dbg[(p * G + gg) * 2] = e1;
+      a.dbg[(p * G + gg) * 2 + 1] = rstd;
+    }
+  }
+  __syncthreads();
+
+  // ---- phase 3: normalise (+SiLU) this chunk, with the halo rows
+  if (pl < PL) {
+    float sc[VEC], sf[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+      const int c = vc * VEC + i;
+      sc[i] = __ldg(a.gamma + c) * s_mr[(c / cg) * 2 + 1];
+      sf[i] = __ldg(a.beta + c) - s_mr[(c / cg) * 2] * sc[i];
+    }
+    T* outp = static_cast<T*>(o.out);
+    T* dst = outp + ((size_t)p * o.out_patch_stride + o.out_off) * C + vc * VEC;
+    const int last_row0 = a.pix_per_patch - o.W;
+    const bool top_src = o.halo_mode != 0 && p > 0;
+    const bool bot_src = o.halo_mode != 0 && p < N - 1;
+    for (int pix = pix0 + pl; pix < pix1; pix += 4 * PL) {
+      uint4 u[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        u[j] = pix + j * PL < pix1 ? ld_nc16(base + (size_t)(pix + j * PL) * C) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int q = pix + j * PL;
+        if (q >= pix1) break;
+        float v[VEC];
+        unpack16(u[j], v);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) {
+          v[i] = fmaf(v[i], sc[i], sf[i]);
+          if (SILU) v[i] = silu_f(v[i]);
+        }
+        const uint4 ov = pack16(v);
+        *reinterpret_cast<uint4*>(dst + (size_t)q * C) = ov;
+        if (o.halo_mode != 0)
+          write_halos(outp, static_cast<const T*>(o.prev_slab), ov, p, q, a.pix_per_patch, last_row0, o.W, C,
+                      vc * VEC, o.out_patch_stride, o.out_off, top_src, bot_src, o.halo_mode);
+      }
+    }
+  }
+  // ---- departure: the last block out re-arms the barrier for the next launch
+  if (tid == 0 && atomicAdd(a.counter + 1, 1u) == total - 1) {
+    a.counter[0] = 0u;
+    a.counter[1] = 0u;
+  }
+}
+
 template <typename T>
 __global__ void halo_refresh_kernel(const T* __restrict__ src, T* __restrict__ dst, int R, int W, int C) {
   constexpr int VEC = VecTraits<T>::kN;
@@ -254,9 +462,10 @@ __global__ void halo_refresh_kernel(const T* __restrict__ src, T* __restrict__ d
 
 // Pixels per block: one wave of 512-thread blocks over the whole map.
 // Per-token LayerNorm (transformer blocks of the SDXL-style stage): one warp per
-// token, the token's C channels held in registers (16-byte vectors), mean and
-// biased variance by warp butterflies (deterministic), fp32 math, bf16 in/out.
-template <int KMAX>
+// token, the token's C channels held in registers (NV 16-byte vectors per lane, NV
+// fixed at compile time so nothing is masked), mean and biased variance by warp
+// butterflies (deterministic, two passes over the registers), fp32 math, bf16 in/out.
+template <int NV>
 __global__ void __launch_bounds__(256)
 layernorm_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ y,
                  const float* __restrict__ gamma, const float* __restrict__ beta, int L, int C, float eps) {
@@ -265,35 +474,48 @@ layernorm_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict_
   if (tok >= L) return;
   const int nvec = C / 8;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)tok * C);
-  float v[KMAX][8];
+  uint4 u[NV];
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int i = lane + 32 * k;
+    u[k] = i < nvec ? ld_nc16(src + i) : make_uint4(0, 0, 0, 0);
+  }
   float s = 0.f;
 #pragma unroll
-  for (int k = 0; k < KMAX; ++k) {
-    const int i = lane + 32 * k;
-    if (i < nvec) {
-      unpack16(ld_nc16(src + i), v[k]);
+  for (int k = 0; k < NV; ++k) {
+    float v[8];
+    unpack16(u[k], v);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) s += v[k][e];
-    }
+    for (int e = 0; e < 8; ++e) s += v[e];
   }
   const float mean = warp_sum(s) / (float)C;
   float q = 0.f;
 #pragma unroll
-  for (int k = 0; k < KMAX; ++k) {
+  for (int k = 0; k < NV; ++k) {
     if (lane + 32 * k < nvec) {
+      float v[8];
+      unpack16(u[k], v);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) { const float d = v[k][e] - mean; q = fmaf(d, d, q); }
+      for (int e = 0; e < 8; ++e) { const float d = v[e] - mean; q = fmaf(d, d, q); }
     }
   }
   const float rstd = 1.f / sqrtf(warp_sum(q) / (float)C + eps);
   uint4* dst = reinterpret_cast<uint4*>(y + (size_t)tok * C);
+  const float4* g4 = reinterpret_cast<const float4*>(gamma);
+  const float4* b4 = reinterpret_cast<const float4*>(beta);
 #pragma unroll
-  for (int k = 0; k < KMAX; ++k) {
+  for (int k = 0; k < NV; ++k) {
     const int i = lane + 32 * k;
     if (i < nvec) {
+      float v[8];
+      unpack16(u[k], v);
+      const float4 ga = __ldg(g4 + 2 * i), gb = __ldg(g4 + 2 * i + 1);
+      const float4 ba = __ldg(b4 + 2 * i), bb = __ldg(b4 + 2 * i + 1);
+      const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+      const float bt[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
       float o[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = (v[k][e] - mean) * rstd * __ldg(gamma + i * 8 + e) + __ldg(beta + i * 8 + e);
+      for (int e = 0; e < 8; ++e) o[e] = fmaf((v[e] - mean) * rstd, gg[e], bt[e]);
       dst[i] = pack16(o);
     }
   }
@@ -347,6 +569,40 @@ cudaError_t launch_gn_apply(const T* x, T* out, const T* prev_slab, const float*
 }
 
 template <typename T>
+cudaError_t launch_gn_fused(const GnArgs& a, const GnOut& o, bool silu, int* err, cudaStream_t s) {
+  constexpr int VEC = VecTraits<T>::kN;
+  const int V = a.C / VEC;
+  const int PL = kGnThreads / V;
+  size_t smem = (size_t)(2 * PL + 2) * a.C * sizeof(float);
+  const size_t red = (size_t)kGnThreads * 2 * sizeof(float);
+  if (smem < red) smem = red;
+  auto kern = silu ? gn_fused_kernel<T, true> : gn_fused_kernel<T, false>;
+  // every block must be resident at once (the grid barrier): at most the occupancy
+  // limit, and no more chunks than the partial-sum scratch holds
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGnThreads, smem);
+  if (e != cudaSuccess) return e;
+  const int max_blocks = per_sm * sm_count();
+  if (a.N > max_blocks) return cudaErrorCooperativeLaunchTooLarge;
+  int n_chunks = std::min(gn_stats_chunks(a.N, a.pix_per_patch), max_blocks / a.N);
+  const int per = (a.pix_per_patch + n_chunks - 1) / n_chunks;
+  n_chunks = (a.pix_per_patch + per - 1) / per;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(n_chunks, a.N);
+  cfg.blockDim = dim3(kGnThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;   // every block resident: the grid barrier cannot starve
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, o, n_chunks, per, err);
+}
+
+template <typename T>
 cudaError_t launch_halo_refresh(const T* src_slab, T* dst_slab, int N, int R, int W, int C,
                                 cudaStream_t s) {
   if (N < 2) return cudaSuccess;
@@ -366,10 +622,16 @@ cudaError_t launch_layernorm(const void* x, void* y, const float* gamma, const f
   const dim3 grid((L + 7) / 8);
   const auto* xi = static_cast<const __nv_bfloat16*>(x);
   auto* yo = static_cast<__nv_bfloat16*>(y);
-  if (C <= 1024)
-    layernorm_kernel<4><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps);
-  else
-    layernorm_kernel<8><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps);
+  switch ((C / 8 + 31) / 32) {   // 16-byte vectors per lane
+    case 1: layernorm_kernel<1><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
+    case 2: layernorm_kernel<2><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
+    case 3: layernorm_kernel<3><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
+    case 4: layernorm_kernel<4><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
+    case 5: layernorm_kernel<5><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
+    case 6: layernorm_kernel<6><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
+    case 7: layernorm_kernel<7><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
+    default: layernorm_kernel<8><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
+  }
   return cudaGetLastError();
 }
 
@@ -382,6 +644,8 @@ template cudaError_t launch_gn_apply<__nv_bfloat16>(const __nv_bfloat16*, __nv_b
                                                     const __nv_bfloat16*, const float*, const float*,
                                                     const float*, int, int, int, int, int, long long,
                                                     long long, bool, int, cudaStream_t);
+template cudaError_t launch_gn_fused<float>(const GnArgs&, const GnOut&, bool, int*, cudaStream_t);
+template cudaError_t launch_gn_fused<__nv_bfloat16>(const GnArgs&, const GnOut&, bool, int*, cudaStream_t);
 template cudaError_t launch_halo_refresh<float>(const float*, float*, int, int, int, int,
                                                 cudaStream_t);
 template cudaError_t launch_halo_refresh<__nv_bfloat16>(const __nv_bfloat16*, __nv_bfloat16*, int,

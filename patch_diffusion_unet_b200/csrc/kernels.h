@@ -23,7 +23,19 @@ struct GnArgs {
   float* dbg;             // [N][G][2] (mean, rstd) used -- read by the apply kernel
   int is_sync, mode, naive;
 };
+// Output side of the fused GroupNorm: out [N][out_patch_stride pixels][C] starting at
+// pixel out_off of each patch (the haloed slab, or a plain map with stride pix_per_patch
+// and offset 0), halo_mode as for launch_gn_apply.
+struct GnOut {
+  void* out;
+  const void* prev_slab;
+  long long out_patch_stride, out_off;
+  int W, halo_mode;
+};
 int gn_stats_chunks(int N, int pix_per_patch);
+// statistics + merge + apply (+SiLU) in one cooperative launch; a.counter needs two
+// zeroed words; a.dbg receives (mean, rstd)
+template <typename T> cudaError_t launch_gn_fused(const GnArgs& a, const GnOut& o, bool silu, int* err, cudaStream_t s);
 template <typename T> cudaError_t launch_gn_stats_merge(const GnArgs& a, cudaStream_t s);
 // halo_mode: 0 none (plain output), 1 sync (fresh neighbour rows), 2 displaced
 // (the previous step's rows, read from prev_slab)
@@ -119,6 +131,8 @@ int sm_count();
 // with rows 1 and 2 of every group of 4 swapped -- the key order in which the softmax
 // threads pack P (see the attention kernel).
 bool encode_attn_v(CUtensorMap* m, const void* base, uint64_t rows, uint64_t heads);
+// K operand of the attention: [heads][rows][64] bf16, one box per KV tile
+bool encode_attn_k(CUtensorMap* m, const void* base, uint64_t rows, uint64_t heads);
 // maps: q [heads][L][64]; k fresh and stale (box 128 rows x 64); v from encode_attn_v
 cudaError_t launch_tc_attention(const TcAttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mkf,
                                 const CUtensorMap& mvf, const CUtensorMap& mks,

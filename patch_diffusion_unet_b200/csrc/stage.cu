@@ -206,10 +206,10 @@ dfp_status stage_create(dfp_ctx* h) {
     ok &= encode_gemm_rows(&x.m_wff1, x.w_ff1, 2 * F, C, 128);
     ok &= encode_gemm_rows(&x.m_wff2, x.w_ff2, C, F, bc);   // same N = C as to_out
     for (int i = 0; i < 2; ++i) {
-      ok &= encode_tmap_3d(&x.m_k[i], x.kb[i], 64, L, heads, 128, L * 128, 64, 128, 1);
+      ok &= encode_attn_k(&x.m_k[i], x.kb[i], L, heads);
       ok &= encode_attn_v(&x.m_v[i], x.vb[i], L, heads);
     }
-    ok &= encode_tmap_3d(&x.m_ck, x.ctx_k, 64, ctx_rows(T), heads, 128, ctx_rows(T) * 128, 64, 128, 1);
+    ok &= encode_attn_k(&x.m_ck, x.ctx_k, ctx_rows(T), heads);
     ok &= encode_attn_v(&x.m_cv, x.ctx_v, ctx_rows(T), heads);
     plan(x.p_qkv, (int)L, 3 * (int)C, (int)C, bq);
     plan(x.p_o1, (int)L, (int)C, (int)C, bc);
@@ -337,21 +337,19 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   g.part = h->part; g.counter = h->counter;
   g.is_sync = is_sync; g.mode = (int)c.gn_mode; g.naive = naive ? 1 : 0;
   g.fresh_out = st->mom1[cur]; g.stale = st->mom1[prv]; g.gamma = st->n1_g; g.beta = st->n1_b; g.dbg = h->dbg1;
-  DFP_LAUNCH(launch_gn_stats_merge<bf>(g, s), "norm1 statistics");
-  DFP_LAUNCH(launch_gn_apply<bf>(static_cast<const bf*>(xv), static_cast<bf*>(st->slab1[cur]),
-                                 static_cast<const bf*>(st->slab1[prv]), h->dbg1, st->n1_g, st->n1_b, G, N, Lp, C, W,
-                                 (long long)(R + 2) * W,
-                                 W, true, halo_mode, s), "norm1 apply + halo");
+  {
+    const GnOut go{st->slab1[cur], st->slab1[prv], (long long)(R + 2) * W, W, W, halo_mode};
+    DFP_LAUNCH(launch_gn_fused<bf>(g, go, true, h->dev_err, s), "norm1 + SiLU + halo (fused)");
+  }
   Epilogue ec{};
   ec.kind = 0; ec.out = st->h1; ec.bias = st->b_c1; ec.ldo = C;
   DFP_LAUNCH(launch_tc_gemm(st->p_c1, st->m_slab1[cur], st->m_wc1, ec, h->dev_err, s), "conv1 (tcgen05)");
   g.x = st->h1; g.fresh_out = st->mom2[cur]; g.stale = st->mom2[prv]; g.gamma = st->n2_g; g.beta = st->n2_b;
   g.dbg = h->dbg2;
-  DFP_LAUNCH(launch_gn_stats_merge<bf>(g, s), "norm2 statistics");
-  DFP_LAUNCH(launch_gn_apply<bf>(static_cast<const bf*>(st->h1), static_cast<bf*>(st->slab2[cur]),
-                                 static_cast<const bf*>(st->slab2[prv]), h->dbg2, st->n2_g, st->n2_b, G, N, Lp, C, W,
-                                 (long long)(R + 2) * W,
-                                 W, true, halo_mode, s), "norm2 apply + halo");
+  {
+    const GnOut go{st->slab2[cur], st->slab2[prv], (long long)(R + 2) * W, W, W, halo_mode};
+    DFP_LAUNCH(launch_gn_fused<bf>(g, go, true, h->dev_err, s), "norm2 + SiLU + halo (fused)");
+  }
   ec.out = st->r[0]; ec.bias = st->b_c2; ec.residual = xv;
   DFP_LAUNCH(launch_tc_gemm(st->p_c2, st->m_slab2[cur], st->m_wc2, ec, h->dev_err, s), "conv2 + residual (tcgen05)");
 

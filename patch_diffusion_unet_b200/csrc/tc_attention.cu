@@ -819,6 +819,10 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
 
 }  // namespace
 
+bool encode_attn_k(CUtensorMap* m, const void* base, uint64_t rows, uint64_t heads) {
+  return encode_tmap_3d(m, base, 64, rows, heads, 128, rows * 128, 64, kTile, 1);
+}
+
 bool encode_attn_v(CUtensorMap* m, const void* base, uint64_t rows, uint64_t heads) {
   // key = 4 s + q + 2 e lands in shared-memory row 4 s + 2 q + e: dims (d, e, q, s, head)
   const uint64_t dims[5] = {64, 2, 2, (rows + 3) / 4, heads};
