@@ -335,8 +335,17 @@ def main():
     blk.set_profiling(False)
     kern_us = {k: 1e3 * statistics.mean(v) for k, v in per.items()}
 
-    # ---- sync step time (for context)
-    sync_ms = None
+    # ---- sync steps (every patch fresh), timed the same way, for context
+    n_sync_t = min(args.steps, 50)
+    sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_sync_t)]
+    for i in range(n_sync_t):
+        t += 1
+        sev[i][0].record(stream)
+        blk.step(x_of(t), t, 1)
+        sev[i][1].record(stream)
+        flush.zero_()
+    torch.cuda.synchronize()
+    sync_ms = statistics.mean(a.elapsed_time(b) for a, b in sev)
 
     # ---- end to end through the host-buffer entry point (pinned host memory)
     e2e = None
@@ -404,6 +413,7 @@ def main():
                        "n_patches": cfg["n_patches"], "heads": cfg["heads"], "parallelism": f"replicas{world}",
                        "l2": "flushed between timed steps (512 MB write, outside the events)",
                        "step": "displaced (is_sync=0)"},
+            "sync_ms_per_step": sync_ms,
             "gpu_launches": launches * args.steps,
             "launches_per_step": launches,
             "kernels_us": {k: round(v, 2) for k, v in kern_us.items()},

@@ -289,6 +289,24 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
   const T* base = static_cast<const T*>(a.x) + (size_t)p * a.pix_per_patch * C + vc * VEC;
   float* chan = sh + 2 * PL * C;
 
+  const int last_row0 = a.pix_per_patch - o.W;
+  const bool top_src = o.halo_mode != 0 && p > 0;          // my first row feeds patch p-1
+  const bool bot_src = o.halo_mode != 0 && p < N - 1;      // my last row feeds patch p+1
+  // ---- displaced steps: the halo rows are last step's values, final already -- copy
+  // them now, overlapped with the statistics, instead of after the barrier
+  if (o.halo_mode == 2 && pl < PL) {
+    T* outp = static_cast<T*>(o.out);
+    const T* prev = static_cast<const T*>(o.prev_slab);
+    for (int q = pix0 + pl; q < pix1; q += PL) {
+      if (!((top_src && q < o.W) || (bot_src && q >= last_row0))) continue;
+      const uint4 hv = ld_nc16(prev + ((size_t)p * o.out_patch_stride + o.out_off + q) * C + vc * VEC);
+      if (top_src && q < o.W)
+        *reinterpret_cast<uint4*>(outp + ((size_t)(p - 1) * o.out_patch_stride + o.out_off + a.pix_per_patch + q) * C +
+                                  vc * VEC) = hv;
+      if (bot_src && q >= last_row0)
+        *reinterpret_cast<uint4*>(outp + ((size_t)(p + 1) * o.out_patch_stride + (q - last_row0)) * C + vc * VEC) = hv;
+    }
+  }
   // ---- phase 1: per-channel partial sums of this chunk (8 loads in flight)
   {
     float s1[VEC], s2[VEC];
@@ -411,9 +429,6 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
     }
     T* outp = static_cast<T*>(o.out);
     T* dst = outp + ((size_t)p * o.out_patch_stride + o.out_off) * C + vc * VEC;
-    const int last_row0 = a.pix_per_patch - o.W;
-    const bool top_src = o.halo_mode != 0 && p > 0;
-    const bool bot_src = o.halo_mode != 0 && p < N - 1;
     for (int pix = pix0 + pl; pix < pix1; pix += 4 * PL) {
       uint4 u[4];
 #pragma unroll
@@ -428,11 +443,11 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
 #pragma unroll
         for (int i = 0; i < VEC; ++i) {
           v[i] = fmaf(v[i], sc[i], sf[i]);
-          if (SILU) v[i] = silu_f(v[i]);
+          if (SILU) v[i] = __fdividef(v[i], 1.f + __expf(-v[i]));   // bf16 output: fast forms suffice
         }
         const uint4 ov = pack16(v);
         *reinterpret_cast<uint4*>(dst + (size_t)q * C) = ov;
-        if (o.halo_mode != 0)
+        if (o.halo_mode == 1)   // sync steps: this step's boundary rows (displaced: copied above)
           write_halos(outp, static_cast<const T*>(o.prev_slab), ov, p, q, a.pix_per_patch, last_row0, o.W, C,
                       vc * VEC, o.out_patch_stride, o.out_off, top_src, bot_src, o.halo_mode);
       }

@@ -64,7 +64,7 @@ constexpr int kStages = 3;
 constexpr int kOCols = 80;                      // 64 outputs + 16 row-sum columns
 constexpr uint32_t kTmemCols = 512;             // S/P: [128g, 128g+128), O: [256+128g, +80)
 constexpr float kRescale = 8.f;                 // lazy rescale threshold (log2 units)
-constexpr int kPolyPer8 = 3;
+constexpr int kPolyPer8 = 2;
 // registers per thread after the split: 128 x 64 + 512 x 104 = 640 x 96 (the launch's)
 constexpr int kRegsTmaMma = 64, kRegsSoftmax = 104;                    // of every 8 columns, this many use the polynomial
 
