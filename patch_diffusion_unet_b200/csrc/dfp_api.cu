@@ -106,13 +106,14 @@ dfp_status build_tmaps(dfp_ctx* h) {
     ok &= encode_tmap_4d(&h->m_slab[i], h->slab[i], dims, str, box);
   }
   const int conv_m_tiles = N * (R / rows_tile) * tpr, lin_m_tiles = gemm_m_tiles_plain(L);
-  const int bn_conv = choose_bn(C, conv_m_tiles), bn_qkv = choose_bn(3 * C, lin_m_tiles),
-            bn_out = choose_bn(C, lin_m_tiles);
-  ok &= encode_gemm_rows(&h->m_wconv, h->w_conv, C, 9ull * C, bn_conv);
+  const GemmChoice g_conv = choose_gemm(C, conv_m_tiles, conv_k_stages(C)),
+                   g_qkv = choose_gemm(3 * C, lin_m_tiles, gemm_k_stages(C)),
+                   g_out = choose_gemm(C, lin_m_tiles, gemm_k_stages(C));
+  ok &= encode_gemm_rows(&h->m_wconv, h->w_conv, C, 9ull * C, g_conv.b_box_rows());
   ok &= encode_gemm_rows(&h->m_t, h->t, L, C, 128);
-  ok &= encode_gemm_rows(&h->m_wqkv, h->w_qkv, 3ull * C, C, bn_qkv);
+  ok &= encode_gemm_rows(&h->m_wqkv, h->w_qkv, 3ull * C, C, g_qkv.b_box_rows());
   ok &= encode_gemm_rows(&h->m_o, h->o, L, C, 128);
-  ok &= encode_gemm_rows(&h->m_wo, h->w_o, C, C, bn_out);
+  ok &= encode_gemm_rows(&h->m_wo, h->w_o, C, C, g_out.b_box_rows());
   const int heads = c.heads;
   ok &= encode_tmap_3d(&h->m_q, h->q, 64, L, heads, 128, (uint64_t)L * 128, 64, 128, 1);
   for (int i = 0; i < 2; ++i) {
@@ -122,15 +123,15 @@ dfp_status build_tmaps(dfp_ctx* h) {
   if (!ok) return h->fail(DFP_E_CUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
   TcGemmPlan& cp = h->conv_plan;
   cp = TcGemmPlan{};
-  cp.M = L; cp.N = C; cp.K = 9 * C; cp.bn = bn_conv; cp.conv = 1;
+  cp.M = L; cp.N = C; cp.K = 9 * C; cp.bn = g_conv.bn; cp.pair = g_conv.pair; cp.conv = 1;
   cp.P = N; cp.R = R; cp.W = W; cp.Cin = C;
   cp.cols_tile = cols_tile; cp.rows_tile = rows_tile; cp.tiles_per_row = tpr;
   TcGemmPlan& qp = h->qkv_plan;
   qp = TcGemmPlan{};
-  qp.M = L; qp.N = 3 * C; qp.K = C; qp.bn = bn_qkv;
+  qp.M = L; qp.N = 3 * C; qp.K = C; qp.bn = g_qkv.bn; qp.pair = g_qkv.pair;
   TcGemmPlan& op = h->out_plan;
   op = TcGemmPlan{};
-  op.M = L; op.N = C; op.K = C; op.bn = bn_out;
+  op.M = L; op.N = C; op.K = C; op.bn = g_out.bn; op.pair = g_out.pair;
   return DFP_OK;
 }
 

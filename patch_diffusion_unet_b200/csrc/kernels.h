@@ -102,13 +102,23 @@ struct TcGemmPlan {
   // conv geometry
   int P, R, W, Cin;       // patches, rows per patch, width, input channels
   int cols_tile, rows_tile, tiles_per_row;
+  int pair;               // 1: CTA-pair kernel (256 x bn tiles; B's map boxes bn/2 rows)
   int m_tiles;            // filled by launch_tc_gemm
   int sms;                // persistent grid size (SM count), filled by launch_tc_gemm
 };
 cudaError_t launch_tc_gemm(const TcGemmPlan& plan, const CUtensorMap& mapA, const CUtensorMap& mapB,
                            const Epilogue& epi, int* err, cudaStream_t s);
-// N-tile width (160, 128 or 64, dividing N) minimising waves x bytes moved per k-block.
-int choose_bn(int N, int m_tiles);
+// N-tile width and CTA-pairing (pair: 256-row tiles over two SMs, B's map boxes bn/2
+// rows) minimising waves x operand rows per SM and k-stage; k_stages = two-chunk (128-wide)
+// K stages per tile; force_bn fixes the width.
+struct GemmChoice {
+  int bn, pair;
+  uint32_t b_box_rows() const { return pair ? bn / 2 : bn; }
+};
+GemmChoice choose_gemm(int N, int m_tiles, int k_stages, int force_bn = 0);
+// two-chunk K stages of a plain GEMM (K) and of the conv (Cin): what choose_gemm takes
+inline int gemm_k_stages(int K) { return (K / 64 + 1) / 2; }
+inline int conv_k_stages(int Cin) { return 9 * ((Cin / 64 + 1) / 2); }
 int gemm_m_tiles_plain(int M);
 
 struct TcAttnArgs {

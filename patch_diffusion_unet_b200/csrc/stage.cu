@@ -185,26 +185,30 @@ dfp_status stage_create(dfp_ctx* h) {
     ok &= encode_tmap_4d(&st->m_slab2[i], st->slab2[i], dims, strides, box);
   }
   const int lin_m = gemm_m_tiles_plain((int)L);
-  const int bn_c = choose_bn((int)C, (int)N * ((int)R / rows_tile) * tpr);
-  ok &= encode_gemm_rows(&st->m_wc1, st->w_c1, C, 9 * C, bn_c);
-  ok &= encode_gemm_rows(&st->m_wc2, st->w_c2, C, 9 * C, bn_c);
+  const GemmChoice g_c = choose_gemm((int)C, (int)N * ((int)R / rows_tile) * tpr, conv_k_stages((int)C));
+  ok &= encode_gemm_rows(&st->m_wc1, st->w_c1, C, 9 * C, g_c.b_box_rows());
+  ok &= encode_gemm_rows(&st->m_wc2, st->w_c2, C, 9 * C, g_c.b_box_rows());
   ok &= encode_gemm_rows(&st->m_u, st->u, L, C, 128);
   ok &= encode_gemm_rows(&st->m_o, h->o, L, C, 128);
   ok &= encode_gemm_rows(&st->m_g, st->g, L, F, 128);
   ok &= encode_tmap_3d(&h->m_q, h->q, 64, L, heads, 128, L * 128, 64, 128, 1);
-  auto plan = [&](TcGemmPlan& p, int M, int Nn, int K, int bn) {
+  auto plan = [&](TcGemmPlan& p, int M, int Nn, int K, const GemmChoice& g) {
     p = TcGemmPlan{};
-    p.M = M; p.N = Nn; p.K = K; p.bn = bn;
+    p.M = M; p.N = Nn; p.K = K; p.bn = g.bn; p.pair = g.pair;
   };
   for (int b = 0; b < c.n_xformer; ++b) {
     XfBlock& x = st->xf[b];
-    const int bq = choose_bn(3 * (int)C, lin_m), bc = choose_bn((int)C, lin_m);
-    ok &= encode_gemm_rows(&x.m_wqkv, x.w_qkv, 3 * C, C, bq);
-    ok &= encode_gemm_rows(&x.m_wo1, x.w_o1, C, C, bc);
-    ok &= encode_gemm_rows(&x.m_wq2, x.w_q2, C, C, bc);
-    ok &= encode_gemm_rows(&x.m_wo2, x.w_o2, C, C, bc);
-    ok &= encode_gemm_rows(&x.m_wff1, x.w_ff1, 2 * F, C, 128);
-    ok &= encode_gemm_rows(&x.m_wff2, x.w_ff2, C, F, bc);   // same N = C as to_out
+    const int ks = gemm_k_stages((int)C);
+    const GemmChoice bq = choose_gemm(3 * (int)C, lin_m, ks), bc = choose_gemm((int)C, lin_m, ks);
+    // GEGLU: 128-wide tiles of 64 value + 64 gate columns (the weight rows are interleaved so)
+    const GemmChoice bf = choose_gemm(2 * (int)F, lin_m, ks, 128);
+    const GemmChoice b2 = choose_gemm((int)C, lin_m, gemm_k_stages((int)F));
+    ok &= encode_gemm_rows(&x.m_wqkv, x.w_qkv, 3 * C, C, bq.b_box_rows());
+    ok &= encode_gemm_rows(&x.m_wo1, x.w_o1, C, C, bc.b_box_rows());
+    ok &= encode_gemm_rows(&x.m_wq2, x.w_q2, C, C, bc.b_box_rows());
+    ok &= encode_gemm_rows(&x.m_wo2, x.w_o2, C, C, bc.b_box_rows());
+    ok &= encode_gemm_rows(&x.m_wff1, x.w_ff1, 2 * F, C, bf.b_box_rows());
+    ok &= encode_gemm_rows(&x.m_wff2, x.w_ff2, C, F, b2.b_box_rows());
     for (int i = 0; i < 2; ++i) {
       ok &= encode_attn_k(&x.m_k[i], x.kb[i], L, heads);
       ok &= encode_attn_v(&x.m_v[i], x.vb[i], L, heads);
@@ -215,13 +219,13 @@ dfp_status stage_create(dfp_ctx* h) {
     plan(x.p_o1, (int)L, (int)C, (int)C, bc);
     plan(x.p_q2, (int)L, (int)C, (int)C, bc);
     plan(x.p_o2, (int)L, (int)C, (int)C, bc);
-    plan(x.p_ff1, (int)L, 2 * (int)F, (int)C, 128);
-    plan(x.p_ff2, (int)L, (int)C, (int)F, bc);
+    plan(x.p_ff1, (int)L, 2 * (int)F, (int)C, bf);
+    plan(x.p_ff2, (int)L, (int)C, (int)F, b2);
   }
   if (!ok) return h->fail(DFP_E_CUDA, "cuTensorMapEncodeTiled failed");
   for (TcGemmPlan* p : {&st->p_c1, &st->p_c2}) {
     *p = TcGemmPlan{};
-    p->M = (int)L; p->N = (int)C; p->K = 9 * (int)C; p->bn = bn_c; p->conv = 1;
+    p->M = (int)L; p->N = (int)C; p->K = 9 * (int)C; p->bn = g_c.bn; p->pair = g_c.pair; p->conv = 1;
     p->P = (int)N; p->R = (int)R; p->W = (int)W; p->Cin = (int)C;
     p->cols_tile = cols_tile; p->rows_tile = rows_tile; p->tiles_per_row = tpr;
   }

@@ -297,6 +297,233 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   }
 }
 
+// CTA-pair variant (cluster of 2, cta_group::2): the pair computes 256 x BN tiles.  Each
+// CTA loads its own 128 rows of A and half of B's BN rows into its own shared memory
+// (plain TMA loads whose byte counts land on the leader's barrier), the leader's MMA warp
+// issues M = 256 MMAs that read both CTAs' tiles, and each CTA's epilogue drains its own
+// 128 x BN accumulator.  Per SM that is 128 + BN/2 operand rows per k-stage instead of
+// 128 + BN: the loads, not the tensor core, bound the single-CTA kernel.
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                    const TcGemmPlan plan, const Epilogue epi, int* err) {
+  constexpr int BNH = BN / 2;                             // B rows held by this CTA
+  constexpr uint32_t kAChunk = kBM * kBK * 2;
+  constexpr uint32_t kBChunk = BNH * kBK * 2;
+  constexpr uint32_t kABytes = 2 * kAChunk;
+  constexpr uint32_t kBBytes = 2 * kBChunk;
+  constexpr uint32_t kCols = TmemCols<BN>::v;            // one accumulator
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * kBBytes);
+  uint64_t* full = bars;                                 // leader's: both CTAs' loads
+  uint64_t* empty = bars + STAGES;                       // each CTA's, from the leader's commits
+  uint64_t* acc_full = bars + 2 * STAGES;                // [2] each CTA's
+  uint64_t* acc_empty = bars + 2 * STAGES + 2;           // [2] leader's: one arrival per CTA
+  uint64_t* exit_bar = bars + 2 * STAGES + 4;            // both CTAs arrive on both
+  uint64_t* drain = bars + 2 * STAGES + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 6);
+  __shared__ volatile int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool lead = rank == 0;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int n_tiles_n = plan.N / BN;
+  const int m_pairs = (plan.m_tiles + 1) / 2;
+  const int n_tiles = m_pairs * n_tiles_n;
+  const int cpt = plan.conv ? plan.Cin / kBK : 0;
+  const int ppt = (cpt + 1) / 2;
+  const int num_kb = plan.conv ? 9 * ppt : (plan.K / kBK + 1) / 2;
+  const uint32_t a_box_bytes =
+      plan.conv ? (uint32_t)(2 * plan.rows_tile * plan.cols_tile * kBK * 2) : kABytes;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < STAGES; ++s) { mbar_init(smem_u32(&full[s]), 1); mbar_init(smem_u32(&empty[s]), 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(smem_u32(&acc_full[i]), 1); mbar_init(smem_u32(&acc_empty[i]), 2); }
+    mbar_init(smem_u32(exit_bar), 2);
+    mbar_init(smem_u32(drain), 1);
+    fence_mbar_init_cluster();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), 2 * kCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();          // both CTAs' barriers exist before either touches the other's
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    const bool issuer = elect_one();
+    if (issuer) {
+      tma_prefetch_desc(&mapA);
+      tma_prefetch_desc(&mapB);
+    }
+    int kg = 0;
+    bool ok = true;
+    for (int t = pair; ok && t < n_tiles; t += n_pairs) {
+      const TileInfo tile = tile_of(plan, 2 * (t / n_tiles_n) + (int)rank);   // past the end: TMA zero fill
+      const int n0 = (t % n_tiles_n) * BN + (int)rank * BNH;
+      for (int kb = 0; kb < num_kb; ++kb, ++kg) {
+        const int s = kg % STAGES, round = kg / STAGES;
+        if (round > 0 && !__all_sync(0xffffffffu, mbar_wait_cluster(smem_u32(&empty[s]), (round - 1) & 1, err,
+                                                                   kErrWaitStageFree))) {
+          ok = false;
+          break;
+        }
+        if (__any_sync(0xffffffffu, s_abort != 0)) { ok = false; break; }
+        const uint32_t fb = map_to_rank(smem_u32(&full[s]), 0);
+        if (issuer) {
+          if (lead) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * (a_box_bytes + kBBytes));
+          if (plan.conv) {
+            const int tap = kb / ppt, kc = 2 * (kb - tap * ppt);
+            const int r = tap / 3, sx = tap - 3 * (tap / 3);
+            const uint32_t da = smem_u32(sA + s * kABytes);
+            tma_load_4d_pair(da, &mapA, fb, kc * kBK, tile.j0 + sx - 1, tile.i0 + r, tile.p);
+            tma_load_4d_pair(da + kAChunk, &mapA, fb, (kc + 1) * kBK, tile.j0 + sx - 1, tile.i0 + r, tile.p);
+            tma_load_3d_pair(smem_u32(sB + s * kBBytes), &mapB, fb, 0, n0, tap * cpt + kc);
+          } else {
+            tma_load_3d_pair(smem_u32(sA + s * kABytes), &mapA, fb, 0, tile.m0, 2 * kb);
+            tma_load_3d_pair(smem_u32(sB + s * kBBytes), &mapB, fb, 0, n0, 2 * kb);
+          }
+        }
+        __syncwarp();
+      }
+    }
+    if (!ok || __any_sync(0xffffffffu, s_abort != 0)) {
+      if (issuer) s_abort = 1;
+      // the leader's barriers count both CTAs' copies: let those in flight land
+      if (lead)
+        for (int k = (kg > STAGES ? kg - STAGES : 0); k < kg; ++k)
+          mbar_wait_cluster(smem_u32(&full[k % STAGES]), (k / STAGES) & 1, err, kErrWaitTmaFull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader CTA)
+    if (lead) {
+      const bool issuer = elect_one();
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * kBM, BN, false, false);
+      const uint64_t ad0 = sw128_kmajor_desc(smem_u32(sA));
+      const uint64_t bd0 = sw128_kmajor_desc(smem_u32(sB));
+      bool ok = true;
+      int kg = 0, ti = 0;
+      for (int t = pair; ok && t < n_tiles; t += n_pairs, ++ti) {
+        const int buf = ti & 1, use = ti >> 1;
+        if (use > 0 && !__all_sync(0xffffffffu, mbar_wait_cluster(smem_u32(&acc_empty[buf]), (use - 1) & 1, err,
+                                                                   kErrWaitAccum))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_d + buf * kCols;
+        for (int kb = 0; kb < num_kb; ++kb, ++kg) {
+          const int s = kg % STAGES, round = kg / STAGES;
+          if (!__all_sync(0xffffffffu, mbar_wait_cluster(smem_u32(&full[s]), round & 1, err, kErrWaitTmaFull))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = ad0 + (uint64_t)s * (kABytes >> 4);
+          const uint64_t bd = bd0 + (uint64_t)s * (kBBytes >> 4);
+          const uint64_t ad1 = ad + (kAChunk >> 4), bd1 = bd + (kBChunk >> 4);
+          if (issuer) {
+            umma_f16_ss_pair(d, ad, bd, idesc, kb > 0);
+#pragma unroll
+            for (int kk = 1; kk < kBK / 16; ++kk) umma_f16_ss_pair(d, ad + 2 * kk, bd + 2 * kk, idesc, 1);
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) umma_f16_ss_pair(d, ad1 + 2 * kk, bd1 + 2 * kk, idesc, 1);
+            umma_commit_pair(smem_u32(&empty[s]), 0x3);   // the stage is free in both CTAs
+          }
+          __syncwarp();
+        }
+        if (ok && issuer) umma_commit_pair(smem_u32(&acc_full[buf]), 0x3);
+        __syncwarp();
+      }
+      if (!ok && issuer) s_abort = 1;
+      // every MMA of this CTA pair completes before TMEM can be released
+      if (issuer) umma_commit_pair(smem_u32(drain), 0x1);
+      __syncwarp();
+      mbar_wait(smem_u32(drain), 0, err, kErrWaitAccum);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5, both CTAs)
+    const int sub = warp & 3;
+    const int row = sub * 32 + lane;
+    int ti = 0;
+    for (int t = pair; t < n_tiles; t += n_pairs, ++ti) {
+      const int buf = ti & 1, use = ti >> 1;
+      const bool ready = mbar_wait_cluster(smem_u32(&acc_full[buf]), use & 1, err, kErrWaitAccum);
+      tc_fence_after();
+      const int m_tile = 2 * (t / n_tiles_n) + (int)rank;
+      const TileInfo tile = tile_of(plan, m_tile);
+      const int n0 = (t % n_tiles_n) * BN;
+      epilogue_tile<BN>(plan, epi, tile, n0, tmem_d + buf * kCols + ((uint32_t)(sub * 32) << 16), row,
+                        ready && !s_abort && m_tile < plan.m_tiles);
+      tc_fence_before();
+      // the four epilogue warps of this CTA are done with the accumulator; they also agree
+      // on giving up (a failed wait anywhere ends the loop for all of them)
+      const bool give_up = named_bar_red_or(1, 128, !ready);
+      if (threadIdx.x == 64) {
+        if (lead) mbar_arrive(smem_u32(&acc_empty[buf]));
+        else mbar_arrive_remote(map_to_rank(smem_u32(&acc_empty[buf]), 0));
+      }
+      if (give_up) break;
+    }
+  }
+
+  // ---- exit: neither CTA leaves while the other may still reach into its shared memory
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive(smem_u32(exit_bar));
+    mbar_arrive_remote(map_to_rank(smem_u32(exit_bar), rank ^ 1u));
+    mbar_wait_cluster(smem_u32(exit_bar), 0, err, kErrWaitAccum);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_d, 2 * kCols);
+  }
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_pair(const TcGemmPlan& plan, const CUtensorMap& mA, const CUtensorMap& mB,
+                        const Epilogue& epi, int* err, cudaStream_t s) {
+  const size_t smem = 1024 + (size_t)STAGES * 2 * (kBM * kBK * 2 + (BN / 2) * kBK * 2) + (2 * STAGES + 8) * 8 + 64;
+  auto kern = tc_gemm_pair_kernel<BN, STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int n_tiles = ((plan.m_tiles + 1) / 2) * (plan.N / BN);
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  // persistent: no more pairs than can be resident at once (a GPC with an odd number of
+  // free SMs leaves one idle), so no pair waits for a second wave
+  static int max_pairs = 0;
+  if (!max_pairs) {
+    cfg.gridDim = dim3(2 * (plan.sms / 2));
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    max_pairs = n > 0 ? n : 1;
+  }
+  const int pairs = n_tiles < max_pairs ? n_tiles : max_pairs;
+  cfg.gridDim = dim3(2 * pairs);
+  return cudaLaunchKernelEx(&cfg, kern, mA, mB, plan, epi, err);
+}
+
 template <int BN, int STAGES>
 cudaError_t launch_bn(const TcGemmPlan& plan, const CUtensorMap& mA, const CUtensorMap& mB,
                       const Epilogue& epi, int* err, cudaStream_t s) {
@@ -326,19 +553,31 @@ int sm_count() {
 
 int gemm_m_tiles_plain(int M) { return (M + kBM - 1) / kBM; }
 
-int choose_bn(int N, int m_tiles) {
+GemmChoice choose_gemm(int N, int m_tiles, int k_stages, int force_bn) {
   const int sms = sm_count();
-  int best = 0;
+  GemmChoice best{0, 0};
   long best_cost = 0;
-  for (int bn : {160, 128, 64}) {
-    if (N % bn) continue;
-    // a k-block moves 16 KB of A and bn * 128 B of B through TMA: time per wave
-    // follows those bytes, not the tile width (narrow tiles are not cheaper per FLOP)
-    const long tiles = (long)m_tiles * (N / bn);
-    const long cost = ((tiles + sms - 1) / sms) * (128 + bn);
-    if (!best || cost < best_cost) { best = bn; best_cost = cost; }
+  for (int pair = 1; pair >= 0; --pair) {
+    for (int bn : {160, 128, 64}) {
+      if (N % bn || (force_bn && bn != force_bn)) continue;
+      if (pair && (bn == 64 || m_tiles < 2)) continue;
+      if (pair) {
+        // the pair's set-up (cluster sync, remote arrivals, exit handshake) and its
+        // longer pipeline fill pay off only over enough k-stages per CTA pair (24: measured on the 64x64x640 and SDXL-stage projections)
+        const long ptiles = (long)((m_tiles + 1) / 2) * (N / bn);
+        const long per_pair = (ptiles + sms / 2 - 1) / (sms / 2);
+        if (per_pair * k_stages < 24) continue;
+      }
+      // per SM and k-stage the loads move 128 + bn (single CTA) or 128 + bn/2 (CTA pair)
+      // operand rows; that, times the waves, is the time
+      const long units = pair ? (long)((m_tiles + 1) / 2) * (N / bn) : (long)m_tiles * (N / bn);
+      const long slots = pair ? sms / 2 : sms;
+      const long cost = ((units + slots - 1) / slots) * (pair ? 128 + bn / 2 : 128 + bn);
+      if (!best.bn || cost < best_cost) { best = GemmChoice{bn, pair}; best_cost = cost; }
+    }
   }
-  return best ? best : 64;
+  if (!best.bn) best = GemmChoice{64, 0};
+  return best;
 }
 
 cudaError_t launch_tc_gemm(const TcGemmPlan& plan_in, const CUtensorMap& mapA, const CUtensorMap& mapB,
@@ -347,6 +586,13 @@ cudaError_t launch_tc_gemm(const TcGemmPlan& plan_in, const CUtensorMap& mapA, c
   plan.m_tiles = plan.conv ? plan.P * (plan.R / plan.rows_tile) * plan.tiles_per_row : (plan.M + kBM - 1) / kBM;
   plan.sms = sm_count();
   // as many two-chunk stages as fit in ~220 KB of shared memory
+  if (plan.pair) {
+    switch (plan.bn) {
+      case 128: return launch_pair<128, 4>(plan, mapA, mapB, epi, err, s);
+      case 160: return launch_pair<160, 4>(plan, mapA, mapB, epi, err, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (plan.bn) {
     case 128: return launch_bn<128, 3>(plan, mapA, mapB, epi, err, s);
     case 160: return launch_bn<160, 3>(plan, mapA, mapB, epi, err, s);
