@@ -351,46 +351,59 @@ __device__ __noinline__ bool piece_epilogue(const TcAttnArgs& a, const Unit& u, 
     }
     if (half == 0) reinterpret_cast<float2*>(a.part_ml)[prow] = make_float2(m_used, l);
   }
-  __threadfence();
+  // publish: the group barrier orders every thread's partial stores before the leader's
+  // fence, and the fence orders them before the arrival count (cumulativity)
   named_bar(2 + g, 256);
-  if (group_leader) *s_last = atomicAdd(a.counters + 2 * c_first + g, 1u) == (unsigned)(npieces - 1);
+  if (group_leader) {
+    __threadfence();
+    const bool last = atomicAdd(a.counters + 2 * c_first + g, 1u) == (unsigned)(npieces - 1);
+    if (last) __threadfence();   // acquire: the other pieces' partials before the group reads them
+    *s_last = last;
+  }
   named_bar(2 + g, 256);
   if (*s_last) {
-    __threadfence();
     if (row_ok) {
-      float mm = -INFINITY;
-      for (int k = 0; k < npieces; ++k) {
+      // all loads of up to two pieces go out before any arithmetic (one round trip), then
+      // further pieces one batch each; pieces are combined in KV order
+      float acc[32], lsum = 0.f, mm = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+      auto slot_row = [&](int k) {
         const int ck = c_first + k;
-        const size_t sr = ((size_t)ck * 2 + (range_start(ck, TT, G) < u.U0 ? 1 : 0)) * 256 + g * 128 + row;
-        mm = fmaxf(mm, __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr).x);
-      }
-      float lsum = 0.f;
-      for (int k = 0; k < npieces; ++k) {
-        const int ck = c_first + k;
-        const size_t sr = ((size_t)ck * 2 + (range_start(ck, TT, G) < u.U0 ? 1 : 0)) * 256 + g * 128 + row;
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr);
-        lsum = fmaf(ml.y, ex2_mufu(ml.x - mm), lsum);
+        return ((size_t)ck * 2 + (range_start(ck, TT, G) < u.U0 ? 1 : 0)) * 256 + g * 128 + row;
+      };
+      for (int k0 = 0; k0 < npieces; k0 += 2) {
+        const bool two = k0 + 1 < npieces;
+        const size_t s0 = slot_row(k0), s1 = two ? slot_row(k0 + 1) : s0;
+        float4 v0[8], v1[8];
+        const float4* p0 = reinterpret_cast<const float4*>(a.part_o + s0 * 64 + half * 32);
+        const float4* p1 = reinterpret_cast<const float4*>(a.part_o + s1 * 64 + half * 32);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v0[q] = __ldcg(p0 + q);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v1[q] = __ldcg(p1 + q);
+        const float2 ml0 = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + s0);
+        const float2 ml1 = two ? __ldcg(reinterpret_cast<const float2*>(a.part_ml) + s1) : make_float2(-INFINITY, 0.f);
+        // rescale what is accumulated so far to the new running maximum
+        const float m_new = fmaxf(mm, fmaxf(ml0.x, ml1.x));
+        const float r = ex2_mufu(mm - m_new), w0 = ex2_mufu(ml0.x - m_new), w1 = two ? ex2_mufu(ml1.x - m_new) : 0.f;
+        mm = m_new;
+        lsum = fmaf(ml1.y, w1, fmaf(ml0.y, w0, lsum * r));
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          acc[4 * q] = fmaf(v1[q].x, w1, fmaf(v0[q].x, w0, acc[4 * q] * r));
+          acc[4 * q + 1] = fmaf(v1[q].y, w1, fmaf(v0[q].y, w0, acc[4 * q + 1] * r));
+          acc[4 * q + 2] = fmaf(v1[q].z, w1, fmaf(v0[q].z, w0, acc[4 * q + 2] * r));
+          acc[4 * q + 3] = fmaf(v1[q].w, w1, fmaf(v0[q].w, w0, acc[4 * q + 3] * r));
+        }
       }
       const float inv = 1.f / lsum;
-      // merge 8 columns at a time, pieces in KV order
+#pragma unroll
       for (int q = 0; q < 4; ++q) {
-        float acc[8];
+        float w8[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-        for (int k = 0; k < npieces; ++k) {
-          const int ck = c_first + k;
-          const size_t sr = ((size_t)ck * 2 + (range_start(ck, TT, G) < u.U0 ? 1 : 0)) * 256 + g * 128 + row;
-          const float w = ex2_mufu(__ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr).x - mm);
-          const float4* po = reinterpret_cast<const float4*>(a.part_o + sr * 64 + half * 32 + q * 8);
-          const float4 v0 = __ldcg(po), v1 = __ldcg(po + 1);
-          acc[0] = fmaf(v0.x, w, acc[0]); acc[1] = fmaf(v0.y, w, acc[1]);
-          acc[2] = fmaf(v0.z, w, acc[2]); acc[3] = fmaf(v0.w, w, acc[3]);
-          acc[4] = fmaf(v1.x, w, acc[4]); acc[5] = fmaf(v1.y, w, acc[5]);
-          acc[6] = fmaf(v1.z, w, acc[6]); acc[7] = fmaf(v1.w, w, acc[7]);
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] *= inv;
-        out_row[q] = pack16(acc);
+        for (int e = 0; e < 8; ++e) w8[e] = acc[8 * q + e] * inv;
+        out_row[q] = pack16(w8);
       }
     }
     if (group_leader) a.counters[2 * c_first + g] = 0u;

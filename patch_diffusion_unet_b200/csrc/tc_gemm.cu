@@ -563,10 +563,11 @@ GemmChoice choose_gemm(int N, int m_tiles, int k_stages, int force_bn) {
       if (pair && (bn == 64 || m_tiles < 2)) continue;
       if (pair) {
         // the pair's set-up (cluster sync, remote arrivals, exit handshake) and its
-        // longer pipeline fill pay off only over enough k-stages per CTA pair (24: measured on the 64x64x640 and SDXL-stage projections)
+        // longer pipeline fill pay off with long tiles (K >= 1024) or many of them (measured on the
+        // 64x64x640, 240x240x640 and SDXL-stage projections)
         const long ptiles = (long)((m_tiles + 1) / 2) * (N / bn);
         const long per_pair = (ptiles + sms / 2 - 1) / (sms / 2);
-        if (per_pair * k_stages < 24) continue;
+        if (k_stages < 8 && per_pair * k_stages < 64) continue;
       }
       // per SM and k-stage the loads move 128 + bn (single CTA) or 128 + bn/2 (CTA pair)
       // operand rows; that, times the waves, is the time
