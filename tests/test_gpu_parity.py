@@ -60,6 +60,10 @@ RAGGED = [
     # one row per patch: a row is both the first and the last of its patch
     dict(name="r1", H=4, W=64, C=128, n_patches=4, gn_groups=8, gn_eps=1e-5, heads=2, head_dim=64,
          dtype="bf16", block="res_attn", steps=5, n_sync=2),
+    # an odd number of conv tiles (3 patches x 5 one-row tiles): the last CTA pair of the
+    # conv GEMM has a padding tile (zero-filled loads, no stores)
+    dict(name="r15", H=15, W=40, C=128, n_patches=3, gn_groups=8, gn_eps=1e-5, heads=2, head_dim=64,
+         dtype="bf16", block="res_attn", steps=5, n_sync=2),
     # N = 1 (no cross-patch context at all)
     dict(name="n1", H=16, W=32, C=192, n_patches=1, gn_groups=8, gn_eps=1e-5, heads=3, head_dim=64,
          dtype="bf16", block="res_attn", steps=4, n_sync=1),
