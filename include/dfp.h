@@ -20,7 +20,7 @@
  *     dfp_last_error() text says why (a NULL handle gets a static message).
  *   - Argument checks run on the host before any launch.
  *   - Work is enqueued on the handle's CUDA stream; no call blocks on the device
- *     except dfp_step_host, dfp_copy_out (host destination) and
+ *     except dfp_step_host, dfp_synchronize, dfp_copy_out (host destination) and
  *     dfp_check_device.
  *   - Tensors are row-major.  The feature map is NHWC with batch 1: [H, W, C].
  *     Tokens of attention are the pixels in row-major (h, w) order.
@@ -125,6 +125,20 @@ DFP_API dfp_status dfp_step(dfp_handle h, const void* x, int step, int is_sync);
  * memory gives asynchronous copies) to the device, runs the step, copies the
  * output to y_host and waits for the stream. */
 DFP_API dfp_status dfp_step_host(dfp_handle h, const void* x_host, void* y_host, int step, int is_sync);
+
+/* Pipelined form of dfp_step_host (no counterpart in the pages: a serving loop).  Enqueues
+ * the copy of x_host to the device on a copy stream, the step on the handle's stream and
+ * the copy of its output to y_host on a second copy stream, then returns without waiting:
+ * consecutive calls overlap one step's copies with the neighbouring steps' kernels.
+ * x_host and y_host must be pinned (page-locked) for the copies to overlap.  The caller
+ * must not modify x_host or read y_host of a call until dfp_synchronize returns (or, when
+ * alternating two host buffers, until two calls later plus dfp_synchronize); device-side
+ * buffers are double-buffered and ordered by events.  Errors are as for dfp_step. */
+DFP_API dfp_status dfp_step_host_async(dfp_handle h, const void* x_host, void* y_host, int step, int is_sync);
+
+/* Wait until every step and copy enqueued on the handle (its stream and the copy streams
+ * of dfp_step_host_async) has completed. */
+DFP_API dfp_status dfp_synchronize(dfp_handle h);
 
 /* Library-owned device pointer to the last step's output [H*W, C] (config dtype);
  * valid until the next dfp_step or dfp_destroy. */

@@ -388,6 +388,56 @@ dfp_status dfp_step_host(dfp_handle h, const void* x_host, void* y_host, int ste
   return DFP_OK;
 }
 
+dfp_status dfp_step_host_async(dfp_handle h, const void* x_host, void* y_host, int step, int is_sync) {
+  if (!h) return DFP_E_ARG;
+  if (!x_host || !y_host) return h->fail(DFP_E_ARG, "x_host / y_host is NULL");
+  const size_t bytes = (size_t)h->L * h->cfg.C * h->esz;
+  cudaError_t e = cudaSuccess;
+  if (!h->s_in) {
+    e = cudaStreamCreateWithFlags(&h->s_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->s_out, cudaStreamNonBlocking);
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+      e = cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_done[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) return h->cuda_fail(e, "async host step set-up");
+    bool ok = true;
+    for (int i = 0; i < 2; ++i) ok = ok && h->alloc(&h->xin2[i], bytes) && h->alloc(&h->ystage[i], bytes);
+    if (!ok) return h->fail(DFP_E_NOMEM, "device allocation failed");
+  }
+  const int b = (int)(h->n_async & 1);
+  const bool reuse = h->n_async >= 2;   // buffer b was used two calls ago
+  // input: into xin2[b] once the step two calls ago has finished reading it
+  if (reuse && (e = cudaStreamWaitEvent(h->s_in, h->ev_done[b], 0)) != cudaSuccess) return h->cuda_fail(e, "input order");
+  if ((e = cudaMemcpyAsync(h->xin2[b], x_host, bytes, cudaMemcpyHostToDevice, h->s_in)) != cudaSuccess)
+    return h->cuda_fail(e, "input copy");
+  if ((e = cudaEventRecord(h->ev_in[b], h->s_in)) != cudaSuccess) return h->cuda_fail(e, "input event");
+  if ((e = cudaStreamWaitEvent(h->stream, h->ev_in[b], 0)) != cudaSuccess) return h->cuda_fail(e, "input order");
+  dfp_status st = dfp_step(h, h->xin2[b], step, is_sync);
+  if (st != DFP_OK) return st;
+  // output: staged to ystage[b] (once its previous copy-out is done), copied out on s_out
+  if (reuse && (e = cudaStreamWaitEvent(h->stream, h->ev_out[b], 0)) != cudaSuccess) return h->cuda_fail(e, "output order");
+  if ((e = cudaMemcpyAsync(h->ystage[b], h->y, bytes, cudaMemcpyDeviceToDevice, h->stream)) != cudaSuccess)
+    return h->cuda_fail(e, "output staging");
+  if ((e = cudaEventRecord(h->ev_done[b], h->stream)) != cudaSuccess) return h->cuda_fail(e, "step event");
+  if ((e = cudaStreamWaitEvent(h->s_out, h->ev_done[b], 0)) != cudaSuccess) return h->cuda_fail(e, "output order");
+  if ((e = cudaMemcpyAsync(y_host, h->ystage[b], bytes, cudaMemcpyDeviceToHost, h->s_out)) != cudaSuccess)
+    return h->cuda_fail(e, "output copy");
+  if ((e = cudaEventRecord(h->ev_out[b], h->s_out)) != cudaSuccess) return h->cuda_fail(e, "output event");
+  ++h->n_async;
+  return DFP_OK;
+}
+
+dfp_status dfp_synchronize(dfp_handle h) {
+  if (!h) return DFP_E_ARG;
+  cudaError_t e = cudaStreamSynchronize(h->stream);
+  if (e == cudaSuccess && h->s_in) e = cudaStreamSynchronize(h->s_in);
+  if (e == cudaSuccess && h->s_out) e = cudaStreamSynchronize(h->s_out);
+  if (e != cudaSuccess) return h->cuda_fail(e, "stream synchronize");
+  return DFP_OK;
+}
+
 dfp_status dfp_output(dfp_handle h, const void** y) {
   if (!h) return DFP_E_ARG;
   if (!y) return h->fail(DFP_E_ARG, "y is NULL");
@@ -503,6 +553,11 @@ int dfp_kernel_times(dfp_handle h, float* ms, const char** names, int max_n) {
 dfp_status dfp_destroy(dfp_handle h) {
   if (!h) return DFP_OK;
   cudaStreamSynchronize(h->stream);
+  for (cudaStream_t cs : {h->s_in, h->s_out})
+    if (cs) { cudaStreamSynchronize(cs); cudaStreamDestroy(cs); }
+  for (int i = 0; i < 2; ++i)
+    for (cudaEvent_t ev : {h->ev_in[i], h->ev_done[i], h->ev_out[i]})
+      if (ev) cudaEventDestroy(ev);
   for (int i = 0; i < dfp_ctx::kMaxEv; ++i)
     if (h->ev[i]) cudaEventDestroy(h->ev[i]);
   for (void* p : h->allocs) cudaFree(p);

@@ -19,6 +19,13 @@ size_t dtype_size(dfp_dtype d);
 struct dfp_ctx {
   dfp_config cfg{};
   cudaStream_t stream = nullptr;
+  // dfp_step_host_async: copy streams, double-buffered device input and output staging,
+  // and the events that order them against the compute stream (created on first use)
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  void* xin2[2] = {nullptr, nullptr};
+  void* ystage[2] = {nullptr, nullptr};
+  cudaEvent_t ev_in[2] = {}, ev_done[2] = {}, ev_out[2] = {};
+  long long n_async = 0;       // asynchronous host steps issued so far
   std::string err;
   int R = 0, L = 0, Lp = 0, family = 0;
   size_t esz = 4;

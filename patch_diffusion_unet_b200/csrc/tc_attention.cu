@@ -363,46 +363,40 @@ __device__ __noinline__ bool piece_epilogue(const TcAttnArgs& a, const Unit& u, 
   named_bar(2 + g, 256);
   if (*s_last) {
     if (row_ok) {
-      // all loads of up to two pieces go out before any arithmetic (one round trip), then
-      // further pieces one batch each; pieces are combined in KV order
-      float acc[32], lsum = 0.f, mm = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-      auto slot_row = [&](int k) {
+      // This path runs at most twice per CTA: it is kept small (rolled loops, few registers)
+      // so that it costs the KV loop nothing.  First the pieces' running maxima and row sums,
+      // then 8 columns at a time, every piece's contribution in KV order.
+      float mm = -INFINITY;
+#pragma unroll 1
+      for (int k = 0; k < npieces; ++k) {
         const int ck = c_first + k;
-        return ((size_t)ck * 2 + (range_start(ck, TT, G) < u.U0 ? 1 : 0)) * 256 + g * 128 + row;
-      };
-      for (int k0 = 0; k0 < npieces; k0 += 2) {
-        const bool two = k0 + 1 < npieces;
-        const size_t s0 = slot_row(k0), s1 = two ? slot_row(k0 + 1) : s0;
-        float4 v0[8], v1[8];
-        const float4* p0 = reinterpret_cast<const float4*>(a.part_o + s0 * 64 + half * 32);
-        const float4* p1 = reinterpret_cast<const float4*>(a.part_o + s1 * 64 + half * 32);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) v0[q] = __ldcg(p0 + q);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) v1[q] = __ldcg(p1 + q);
-        const float2 ml0 = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + s0);
-        const float2 ml1 = two ? __ldcg(reinterpret_cast<const float2*>(a.part_ml) + s1) : make_float2(-INFINITY, 0.f);
-        // rescale what is accumulated so far to the new running maximum
-        const float m_new = fmaxf(mm, fmaxf(ml0.x, ml1.x));
-        const float r = ex2_mufu(mm - m_new), w0 = ex2_mufu(ml0.x - m_new), w1 = two ? ex2_mufu(ml1.x - m_new) : 0.f;
-        mm = m_new;
-        lsum = fmaf(ml1.y, w1, fmaf(ml0.y, w0, lsum * r));
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          acc[4 * q] = fmaf(v1[q].x, w1, fmaf(v0[q].x, w0, acc[4 * q] * r));
-          acc[4 * q + 1] = fmaf(v1[q].y, w1, fmaf(v0[q].y, w0, acc[4 * q + 1] * r));
-          acc[4 * q + 2] = fmaf(v1[q].z, w1, fmaf(v0[q].z, w0, acc[4 * q + 2] * r));
-          acc[4 * q + 3] = fmaf(v1[q].w, w1, fmaf(v0[q].w, w0, acc[4 * q + 3] * r));
-        }
+        const size_t sr = ((size_t)ck * 2 + (range_start(ck, TT, G) < u.U0 ? 1 : 0)) * 256 + g * 128 + row;
+        mm = fmaxf(mm, __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr).x);
+      }
+      float lsum = 0.f;
+#pragma unroll 1
+      for (int k = 0; k < npieces; ++k) {
+        const int ck = c_first + k;
+        const size_t sr = ((size_t)ck * 2 + (range_start(ck, TT, G) < u.U0 ? 1 : 0)) * 256 + g * 128 + row;
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr);
+        lsum = fmaf(ml.y, ex2_mufu(ml.x - mm), lsum);
       }
       const float inv = 1.f / lsum;
-#pragma unroll
+#pragma unroll 1
       for (int q = 0; q < 4; ++q) {
-        float w8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) w8[e] = acc[8 * q + e] * inv;
+        float w8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+        for (int k = 0; k < npieces; ++k) {
+          const int ck = c_first + k;
+          const size_t sr = ((size_t)ck * 2 + (range_start(ck, TT, G) < u.U0 ? 1 : 0)) * 256 + g * 128 + row;
+          const float w = ex2_mufu(__ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr).x - mm) * inv;
+          const float4* po = reinterpret_cast<const float4*>(a.part_o + sr * 64 + half * 32) + 2 * q;
+          const float4 v0 = __ldcg(po), v1 = __ldcg(po + 1);
+          w8[0] = fmaf(v0.x, w, w8[0]); w8[1] = fmaf(v0.y, w, w8[1]);
+          w8[2] = fmaf(v0.z, w, w8[2]); w8[3] = fmaf(v0.w, w, w8[3]);
+          w8[4] = fmaf(v1.x, w, w8[4]); w8[5] = fmaf(v1.y, w, w8[5]);
+          w8[6] = fmaf(v1.z, w, w8[6]); w8[7] = fmaf(v1.w, w, w8[7]);
+        }
         out_row[q] = pack16(w8);
       }
     }
@@ -706,8 +700,13 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
       }
       float m_used = -INFINITY;
       for (int jj = 0; jj < n && !carry; ++jj, ++gt) {
-        int stale, krow, valid;
-        tile_src(a.mode, sp[0], a.Lp, a.L, a.kv_len, sp[5] - sp[4] + jj, stale, krow, valid);
+        // every tile is full when all segment lengths are multiples of the tile (parameters
+        // only: no per-tile lookup); otherwise the tile's valid key count
+        int valid = kTile;
+        if (!((a.mode == kAttnCross ? a.kv_len : (a.Lp | a.L)) % kTile == 0)) {
+          int stale, krow;
+          tile_src(a.mode, sp[0], a.Lp, a.L, a.kv_len, sp[5] - sp[4] + jj, stale, krow, valid);
+        }
         if (!mbar_wait_warp(smem_u32(&s_full[g]), gt & 1, err, kErrWaitAttnS)) { carry = true; break; }
         tc_fence_after();
         float sc[64];   // sc[i] = S[row][2i + cq]

@@ -19,7 +19,8 @@ GN_CORRECTED, GN_STALE_OTHERS = 0, 1
 CTX_DISPLACED, CTX_NAIVE = 0, 1
 FAMILY_TENSOR_CORE, FAMILY_SIMT = 0, 1
 
-EXPORTED = ("dfp_create", "dfp_load_weights", "dfp_step", "dfp_step_host", "dfp_output",
+EXPORTED = ("dfp_create", "dfp_load_weights", "dfp_step", "dfp_step_host", "dfp_step_host_async",
+            "dfp_synchronize", "dfp_output",
             "dfp_copy_out", "dfp_buffer_bytes", "dfp_check_device", "dfp_launches_per_step",
             "dfp_set_kernel_family", "dfp_set_profiling", "dfp_kernel_times", "dfp_destroy",
             "dfp_last_error", "dfp_group_norm_noalloc", "dfp_group_norm_noalloc_error")
@@ -51,6 +52,8 @@ def load_library(path=_LIB_PATH):
         "dfp_load_weights": ([H, ctypes.POINTER(Tensor), ctypes.c_int], ctypes.c_int),
         "dfp_step": ([H, ctypes.c_void_p, ctypes.c_int, ctypes.c_int], ctypes.c_int),
         "dfp_step_host": ([H, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int], ctypes.c_int),
+        "dfp_step_host_async": ([H, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int], ctypes.c_int),
+        "dfp_synchronize": ([H], ctypes.c_int),
         "dfp_output": ([H, ctypes.POINTER(ctypes.c_void_p)], ctypes.c_int),
         "dfp_copy_out": ([H, ctypes.c_char_p, ctypes.c_void_p, ctypes.c_longlong], ctypes.c_int),
         "dfp_buffer_bytes": ([H, ctypes.c_char_p, ctypes.POINTER(ctypes.c_longlong)], ctypes.c_int),
@@ -166,6 +169,15 @@ class DisplacedPatchBlock:
         """Host-buffer step: x_host / y_host are CPU tensors (pinned for async copies)."""
         self._check(LIB.dfp_step_host(self.h, ctypes.c_void_p(x_host.data_ptr()),
                                       ctypes.c_void_p(y_host.data_ptr()), int(step), int(is_sync)))
+
+    def step_host_async(self, x_host, y_host, step, is_sync):
+        """Pipelined host-buffer step (pinned CPU tensors): returns once enqueued; x_host
+        must stay unchanged and y_host is filled after synchronize()."""
+        self._check(LIB.dfp_step_host_async(self.h, ctypes.c_void_p(x_host.data_ptr()),
+                                            ctypes.c_void_p(y_host.data_ptr()), int(step), int(is_sync)))
+
+    def synchronize(self):
+        self._check(LIB.dfp_synchronize(self.h))
 
     def buffer(self, name):
         """A fresh torch copy (on the device) of an internal buffer of the last step."""

@@ -185,3 +185,28 @@ def test_host_buffer_step_matches_device_step():
         assert torch.equal(a.output().cpu(), y_host)
     a.close()
     b.close()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg_id", [1, 4])
+def test_pipelined_host_steps_match_device_steps(cfg_id):
+    """dfp_step_host_async: consecutive calls without waiting (copies overlapped with the
+    neighbouring steps), then one synchronize; every step's output equals the device path's."""
+    from patch_diffusion_unet_b200 import dfp
+    cfg = configs.get(cfg_id)
+    wl = inputs.SyntheticWorkload(cfg)
+    weights = dict(wl.weights, context=wl.context) if wl.context is not None else wl.weights
+    a, b = dfp.DisplacedPatchBlock(cfg), dfp.DisplacedPatchBlock(cfg)
+    a.load_weights(weights)
+    b.load_weights(weights)
+    sched = wl.schedule()[:8]
+    xs = [inputs.to_torch(wl.x(t), "bf16").pin_memory() for t, _ in sched]
+    ys = [torch.empty(cfg["H"] * cfg["W"], cfg["C"], dtype=torch.bfloat16).pin_memory() for _ in sched]
+    for i, (t, s) in enumerate(sched):
+        b.step_host_async(xs[i], ys[i], t, s)
+    b.synchronize()
+    for i, (t, s) in enumerate(sched):
+        a.step(xs[i].cuda(), t, s)
+        assert torch.equal(a.output().cpu(), ys[i]), f"step {t}"
+    a.close()
+    b.close()
