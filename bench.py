@@ -112,7 +112,7 @@ def work_model(cfg):
 # capture time: once the kernel changes the figure no longer applies and is reported null.
 NCU_TRAFFIC = {
     ("sdxl1024-64x64x640-n4-bf16", "attention (tcgen05)"):
-        (28.20e6, ("tc_attention.cu", "dfp_common.cuh"), "66c56d18cbbea4e3"),
+        (28.20e6, ("tc_attention.cu", "dfp_common.cuh"), "7aeba0d1c53e3d1c"),
 }
 
 

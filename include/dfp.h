@@ -140,6 +140,16 @@ DFP_API dfp_status dfp_step_host_async(dfp_handle h, const void* x_host, void* y
  * of dfp_step_host_async) has completed. */
 DFP_API dfp_status dfp_synchronize(dfp_handle h);
 
+/* Self-test of failure detection (no counterpart in the pages).  Every spin-wait in the
+ * library's kernels is bounded: after ~4e9 SM clocks (about 2 s) it records an error code in
+ * a device word and the kernel winds down, so a lost arrival surfaces as DFP_E_DEVICE from
+ * dfp_check_device instead of a hung GPU.  This call runs one thread that waits, through the
+ * same code, on an mbarrier nothing arrives on (on the current device and the legacy default
+ * stream), and returns the code it recorded in *code_out (1: a TMA stage never filled) and
+ * the wait's length in SM clocks in *cycles_out (may be NULL).  The context stays usable.
+ * Blocks for the length of the wait.  DFP_E_CUDA if a CUDA call fails. */
+DFP_API dfp_status dfp_selftest_wait_timeout(int* code_out, long long* cycles_out);
+
 /* Library-owned device pointer to the last step's output [H*W, C] (config dtype);
  * valid until the next dfp_step or dfp_destroy. */
 DFP_API dfp_status dfp_output(dfp_handle h, const void** y);

@@ -1,5 +1,6 @@
-// GroupNorm over row patches with stale cross-patch statistics, and the halo
-// refresh of the conv input cache.  All three kernels are HBM-bandwidth bound.
+// GroupNorm over row patches with stale cross-patch statistics (writing the conv input
+// slab with its halo rows), and the per-token LayerNorm of the transformer stage.  All of
+// them move whole feature maps once or twice: HBM (and at small sizes latency) bound.
 //
 // DistriGroupNorm ("DistriFusion源码探秘" source walkthrough, Patch Parallelism
 // section, item 3) with the "corrected asynchronous" default of the --sync_mode
@@ -460,20 +461,6 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
   }
 }
 
-template <typename T>
-__global__ void halo_refresh_kernel(const T* __restrict__ src, T* __restrict__ dst, int R, int W, int C) {
-  constexpr int VEC = VecTraits<T>::kN;
-  const int b = blockIdx.y >> 1, dir = blockIdx.y & 1;
-  const size_t row = (size_t)W * C;
-  const size_t slab = (size_t)(R + 2) * row;
-  // dir 0: top halo of patch b+1 <- last interior row of patch b
-  // dir 1: bottom halo of patch b <- first interior row of patch b+1
-  const T* s = dir == 0 ? src + b * slab + (size_t)R * row : src + (b + 1) * slab + row;
-  T* d = dir == 0 ? dst + (b + 1) * slab : dst + b * slab + (size_t)(R + 1) * row;
-  const int nvec = (int)(row / VEC);
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nvec; i += gridDim.x * blockDim.x)
-    reinterpret_cast<uint4*>(d)[i] = ld_nc16(reinterpret_cast<const uint4*>(s) + i);
-}
 
 // Pixels per block: one wave of 512-thread blocks over the whole map.
 // Per-token LayerNorm (transformer blocks of the SDXL-style stage): one warp per
@@ -617,19 +604,6 @@ cudaError_t launch_gn_fused(const GnArgs& a, const GnOut& o, bool silu, int* err
   return cudaLaunchKernelEx(&cfg, kern, a, o, n_chunks, per, err);
 }
 
-template <typename T>
-cudaError_t launch_halo_refresh(const T* src_slab, T* dst_slab, int N, int R, int W, int C,
-                                cudaStream_t s) {
-  if (N < 2) return cudaSuccess;
-  constexpr int VEC = VecTraits<T>::kN;
-  const int nvec = W * C / VEC;
-  const int threads = 256;
-  int bx = (nvec + threads - 1) / threads;
-  if (bx > 64) bx = 64;
-  dim3 grid(bx, 2 * (N - 1));
-  halo_refresh_kernel<T><<<grid, threads, 0, s>>>(src_slab, dst_slab, R, W, C);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_layernorm(const void* x, void* y, const float* gamma, const float* beta, int L, int C,
                              float eps, cudaStream_t s) {
@@ -661,9 +635,5 @@ template cudaError_t launch_gn_apply<__nv_bfloat16>(const __nv_bfloat16*, __nv_b
                                                     long long, bool, int, cudaStream_t);
 template cudaError_t launch_gn_fused<float>(const GnArgs&, const GnOut&, bool, int*, cudaStream_t);
 template cudaError_t launch_gn_fused<__nv_bfloat16>(const GnArgs&, const GnOut&, bool, int*, cudaStream_t);
-template cudaError_t launch_halo_refresh<float>(const float*, float*, int, int, int, int,
-                                                cudaStream_t);
-template cudaError_t launch_halo_refresh<__nv_bfloat16>(const __nv_bfloat16*, __nv_bfloat16*, int,
-                                                        int, int, int, cudaStream_t);
 
 }  // namespace dfp

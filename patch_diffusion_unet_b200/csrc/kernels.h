@@ -44,9 +44,6 @@ cudaError_t launch_gn_apply(const T* x, T* out, const T* prev_slab, const float*
                             const float* beta, int G, int N, int pix_per_patch, int C, int W,
                             long long out_patch_stride_pix, long long out_pix_off, bool silu, int halo_mode,
                             cudaStream_t s);
-template <typename T>
-cudaError_t launch_halo_refresh(const T* src_slab, T* dst_slab, int N, int R, int W, int C,
-                                cudaStream_t s);
 
 // Per-token LayerNorm over C channels (biased variance), bf16 in / out, fp32 math.
 cudaError_t launch_layernorm(const void* x, void* y, const float* gamma, const float* beta, int L, int C,
