@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Benchmark of the displaced-patch UNet layer step on B200: layer-steps/s and latent px/s.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--batch B] [--impl ours|reference]
 
 One "step" is one displaced layer step (dfp_step with is_sync = 0) of the
 workload: GN1 statistics + corrected merge, GN1 apply + SiLU, halo refresh,
@@ -16,6 +16,10 @@ summed step time.  Rank 0 prints one JSON line.
 
 --impl reference times the CPU oracle (numpy fp64) on the host cores instead:
 the same metric on the same workload, full (unsampled) displaced steps.
+
+--batch B runs B images per layer step (the classifier-free-guidance batch, B = 2):
+a step is still one dfp_step, now over B images; "images_per_s" reports
+value * B and the work model counts all B images.
 """
 import argparse
 import hashlib
@@ -45,12 +49,15 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--batch", type=int, default=1, help="images per step (2: the guidance batch)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--profile-steps", type=int, default=10)
     ap.add_argument("--min-warmup-s", type=float, default=1.5,
                     help="keep warming up until this much wall time has passed (clocks settle)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="launch each kernel only after its predecessor completed (no programmatic dependent launch)")
     return ap.parse_args()
 
 
@@ -66,7 +73,15 @@ def peaks():
 # ---------------------------------------------------------------------------- work model
 
 def work_model(cfg):
-    """Algorithmic FLOPs / bytes per launch of each kernel of one layer step."""
+    """Algorithmic FLOPs / bytes per launch of each kernel of one layer step (all images of
+    a batch: every kernel does each image's work once)."""
+    B = cfg.get("batch", 1)
+    wm = _work_model_one_image(cfg)
+    return {k: (v[0], B * v[1]) if isinstance(v, tuple) else (B * v if k == "_total_flops" else v)
+            for k, v in wm.items()}
+
+
+def _work_model_one_image(cfg):
     H, W, C, N, heads = cfg["H"], cfg["W"], cfg["C"], cfg["n_patches"], cfg["heads"]
     L, d = H * W, cfg["head_dim"]
     e = 2 if cfg["dtype"] == "bf16" else 4
@@ -112,7 +127,7 @@ def work_model(cfg):
 # capture time: once the kernel changes the figure no longer applies and is reported null.
 NCU_TRAFFIC = {
     ("sdxl1024-64x64x640-n4-bf16", "attention (tcgen05)"):
-        (28.20e6, ("tc_attention.cu", "dfp_common.cuh"), "7aeba0d1c53e3d1c"),
+        (28.23e6, ("tc_attention.cu", "dfp_common.cuh"), "036626542f523539"),
 }
 
 
@@ -225,6 +240,7 @@ def dist_setup():
 
 def run_reference(args, cfg):
     world = int(os.environ.get("WORLD_SIZE", "1"))
+    B = cfg.get("batch", 1)
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
     import oracle
@@ -253,9 +269,9 @@ def run_reference(args, cfg):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "latent_px_per_s": value * L,
+        "data": "synthetic", "latent_px_per_s": value * L * B, "images_per_s": value * B,
         "config": {"workload": cfg["name"], "H": cfg["H"], "W": cfg["W"], "C": cfg["C"],
-                   "n_patches": cfg["n_patches"], "l2": "n/a (CPU)"},
+                   "n_patches": cfg["n_patches"], "batch": B, "l2": "n/a (CPU)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": f"{args.steps} full displaced layer steps after {n_sync} sync steps"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -267,6 +283,9 @@ def run_reference(args, cfg):
 def main():
     args = parse()
     cfg = configs.get(args.config)
+    B = max(1, args.batch)
+    if B > 1:
+        cfg = configs.get(cfg, batch=B, name=f"{cfg['name']}-b{B}")
     if args.impl == "reference":
         return run_reference(args, cfg)
 
@@ -281,6 +300,7 @@ def main():
     wl = inputs.SyntheticWorkload(cfg)
     blk = dfp.DisplacedPatchBlock(cfg)
     blk.load_weights(dict(wl.weights, context=wl.context) if wl.context is not None else wl.weights)
+    blk.set_launch_overlap(not args.no_overlap)
     stream = blk.stream
     n_pool = 16
     host_x = [inputs.to_torch(wl.x(t), dtype) for t in range(n_pool)]
@@ -363,7 +383,7 @@ def main():
         # neighbouring steps' kernels; L2 is still flushed between steps, on the step's
         # stream and inside the timed region
         xh = [h.pin_memory() for h in host_x]
-        yh = [torch.empty(L, cfg["C"], dtype=xh[0].dtype).pin_memory() for _ in range(2)]
+        yh = [torch.empty(B * L, cfg["C"], dtype=xh[0].dtype).pin_memory() for _ in range(2)]
         for i in range(4):
             t += 1
             blk.step_host_async(xh[t % n_pool], yh[i & 1], t, 0)
@@ -379,7 +399,7 @@ def main():
         blk.synchronize()
         e_total = time.perf_counter() - w0
         e2e_rate, _ = replica_throughput(e_total * 1e3, n_e, world, "cuda")
-        nbytes = L * cfg["C"] * (2 if dtype == "bf16" else 4)
+        nbytes = B * L * cfg["C"] * (2 if dtype == "bf16" else 4)
         e2e = {"value": e2e_rate, "unit": UNIT, "h2d_bytes_per_step": nbytes,
                "d2h_bytes_per_step": nbytes, "steps": n_e,
                "api": "dfp_step_host_async (pinned host buffers) + dfp_synchronize, wall clock",
@@ -421,10 +441,11 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": n_warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if dtype == "bf16" else "f32", "data": "synthetic",
-            "latent_px_per_s": value * L,
+            "latent_px_per_s": value * L * B, "images_per_s": value * B,
             "tensor_tflops_per_step": wm["_total_flops"] / (ms_step * 1e-3) / 1e12,
             "config": {"workload": cfg["name"], "H": cfg["H"], "W": cfg["W"], "C": cfg["C"],
-                       "n_patches": cfg["n_patches"], "heads": cfg["heads"], "parallelism": f"replicas{world}",
+                       "n_patches": cfg["n_patches"], "heads": cfg["heads"], "batch": B,
+                       "launch_overlap": not args.no_overlap, "parallelism": f"replicas{world}",
                        "l2": "flushed between timed steps (512 MB write, outside the events)",
                        "step": "displaced (is_sync=0)"},
             "sync_ms_per_step": sync_ms,

@@ -22,9 +22,13 @@
  *   - Work is enqueued on the handle's CUDA stream; no call blocks on the device
  *     except dfp_step_host, dfp_synchronize, dfp_copy_out (host destination) and
  *     dfp_check_device.
- *   - Tensors are row-major.  The feature map is NHWC with batch 1: [H, W, C].
- *     Tokens of attention are the pixels in row-major (h, w) order.
- *   - Patch p (0 <= p < N) owns rows [p*H/N, (p+1)*H/N).
+ *   - Tensors are row-major.  The feature map is NHWC: [B, H, W, C] with B =
+ *     dfp_config.batch images (B = 1: [H, W, C]).  Tokens of attention are the
+ *     pixels of one image in row-major (h, w) order; L = H * W per image.
+ *   - Patch p (0 <= p < N) of every image owns rows [p*H/N, (p+1)*H/N).  The images
+ *     of a batch share the weights and the step schedule and nothing else: each has
+ *     its own GroupNorm statistics, halo rows, K/V context and (transformer stage)
+ *     cross-attention context.
  *   - One handle is not thread-safe; distinct handles are independent.
  */
 #ifndef DFP_H
@@ -56,7 +60,7 @@ typedef enum { DFP_F32 = 0, DFP_BF16 = 1 } dfp_dtype;
 
 typedef enum {
   DFP_BLOCK_RES_ATTN = 0,   /* GN+SiLU -> conv3x3 -> GN -> self-attention (Q,K,V,O) */
-  DFP_BLOCK_SDXL_STAGE = 1  /* ResNet block + transformer blocks (not built yet)     */
+  DFP_BLOCK_SDXL_STAGE = 1  /* ResNet block + transformer blocks                     */
 } dfp_block;
 
 typedef enum {
@@ -83,6 +87,13 @@ typedef struct {
   dfp_gn_mode gn_mode;
   dfp_context context;
   int n_xformer, ffn_inner, ctx_len, ctx_dim;  /* DFP_BLOCK_SDXL_STAGE only           */
+  /* Images per step, 1..8 (0 counts as 1).  2 is the classifier-free-guidance batch
+   * (conditional and unconditional branch; guidance scale 5 by default) that the
+   * project README's latency benchmark splits across GPU groups unless
+   * --no_split_batch is given (README, Benchmarks: COCO quality and Latency).  On one
+   * GPU the images run through the same launches, every image-specific step indexed
+   * by image.  The SIMT family (fp32) needs batch * n_patches * gn_groups <= 512. */
+  int batch;
 } dfp_config;
 
 typedef struct {
@@ -107,11 +118,18 @@ DFP_API dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_hand
  * of the block must be named exactly once across calls before the first step;
  * names for DFP_BLOCK_RES_ATTN: gn1.weight gn1.bias conv1.weight conv1.bias
  * gn2.weight gn2.bias attn.to_q.weight attn.to_k.weight attn.to_v.weight
- * attn.to_out.weight attn.to_out.bias.  Blocks until the copies are done.
+ * attn.to_out.weight attn.to_out.bias.  DFP_BLOCK_SDXL_STAGE: resnet.{norm1,conv1,
+ * norm2,conv2}.{weight,bias}, xf<b>.{norm1,norm2,norm3}.{weight,bias},
+ * xf<b>.attn1.to_{q,k,v,out}.weight, xf<b>.attn1.to_out.bias, the same for attn2
+ * (to_k / to_v are [C, ctx_dim]), xf<b>.ff.proj.{weight,bias} ([2F, C], GEGLU value
+ * rows then gate rows), xf<b>.ff.out.{weight,bias}, and "context": the text context,
+ * [ctx_len, ctx_dim] for one image or [B, ctx_len, ctx_dim], one per image, for a
+ * batch (conditional and unconditional context of the guidance batch).  Blocks
+ * until the copies are done.
  * Errors: DFP_E_ARG for an unknown name, wrong shape or dtype. */
 DFP_API dfp_status dfp_load_weights(dfp_handle h, const dfp_tensor* w, int n);
 
-/* One layer step.  x: caller-owned device pointer [H, W, C] of the config dtype,
+/* One layer step.  x: caller-owned device pointer [B, H, W, C] of the config dtype,
  * contiguous; it must stay valid until the stream work completes.
  * step: 0 starts a new run and must be synchronous (is_sync = 1); otherwise
  * step must equal the previous step + 1.  is_sync = 1 uses fresh context
@@ -121,7 +139,7 @@ DFP_API dfp_status dfp_load_weights(dfp_handle h, const dfp_tensor* w, int n);
  * Errors: DFP_E_STATE (order, weights missing), DFP_E_ARG, DFP_E_CUDA. */
 DFP_API dfp_status dfp_step(dfp_handle h, const void* x, int step, int is_sync);
 
-/* Same step with HOST buffers: copies x_host ([H,W,C], config dtype; pinned
+/* Same step with HOST buffers: copies x_host ([B,H,W,C], config dtype; pinned
  * memory gives asynchronous copies) to the device, runs the step, copies the
  * output to y_host and waits for the stream. */
 DFP_API dfp_status dfp_step_host(dfp_handle h, const void* x_host, void* y_host, int step, int is_sync);
@@ -150,17 +168,17 @@ DFP_API dfp_status dfp_synchronize(dfp_handle h);
  * Blocks for the length of the wait.  DFP_E_CUDA if a CUDA call fails. */
 DFP_API dfp_status dfp_selftest_wait_timeout(int* code_out, long long* cycles_out);
 
-/* Library-owned device pointer to the last step's output [H*W, C] (config dtype);
+/* Library-owned device pointer to the last step's output [B*H*W, C] (config dtype);
  * valid until the next dfp_step or dfp_destroy. */
 DFP_API dfp_status dfp_output(dfp_handle h, const void** y);
 
 /* Copy an internal buffer of the last step to dst (device or host pointer,
  * dst_bytes must equal the buffer size, see dfp_buffer_bytes).  Names:
- * "y" output [L,C]; "slab" GN1+SiLU output with its halo rows [N,H/N+2,W,C];
- * "h" conv output [H,W,C];
- * "t" GN2 output [H,W,C]; "q","k","v" this step's projections [heads,L,64];
- * "o" attention output [L,C]; "gn1","gn2" per-(patch,group) (mean, rstd) fp32
- * [N,G,2].  Stream-ordered; a host dst makes the call wait for the stream. */
+ * "y" output [B*L,C]; "slab" GN1+SiLU output with its halo rows [B*N,H/N+2,W,C];
+ * "h" conv output [B,H,W,C];
+ * "t" GN2 output [B,H,W,C]; "q","k","v" this step's projections [heads,B*L,64];
+ * "o" attention output [B*L,C]; "gn1","gn2" per-(image,patch,group) (mean, rstd)
+ * fp32 [B*N,G,2].  Stream-ordered; a host dst makes the call wait for the stream. */
 DFP_API dfp_status dfp_copy_out(dfp_handle h, const char* name, void* dst, long long dst_bytes);
 DFP_API dfp_status dfp_buffer_bytes(dfp_handle h, const char* name, long long* bytes);
 
@@ -171,6 +189,15 @@ DFP_API dfp_status dfp_check_device(dfp_handle h);
 
 /* Number of kernel launches one dfp_step of this handle enqueues. */
 DFP_API int dfp_launches_per_step(dfp_handle h);
+
+/* Launch overlap between the kernels of a step (no counterpart in the pages; on by
+ * default): every tensor-core-family kernel is launched with programmatic stream
+ * serialization, so its blocks are scheduled, and set up their barriers and tensor
+ * memory, while the previous kernel on the stream finishes; each waits for that kernel
+ * to complete before it touches device memory, so results do not change.  enable = 0
+ * launches every kernel only after its predecessor has completed.  DFP_E_ARG unless
+ * enable is 0 or 1. */
+DFP_API dfp_status dfp_set_launch_overlap(dfp_handle h, int enable);
 
 /* Choose the kernel family for the contractions: 0 = tcgen05/TMA tensor-core
  * kernels (default for bf16), 1 = SIMT CUDA-core kernels (the only family for

@@ -364,6 +364,31 @@ class SDXLStage(_StepProtocol):
 
 
 def make_block(cfg, weights, context_tokens=None, gn_mode=GN_CORRECTED, context=CTX_DISPLACED):
+    if cfg.get("batch", 1) > 1:
+        return GuidanceBatch(cfg, weights, context_tokens, gn_mode, context)
     if cfg["block"] == "res_attn":
         return ResAttnBlock(cfg, weights, gn_mode, context)
     return SDXLStage(cfg, weights, context_tokens, gn_mode, context)
+
+
+class GuidanceBatch:
+    """B images through the same layer (or stage) step: the classifier-free-guidance
+    batch, a conditional and an unconditional branch at guidance scale 5 ([CSDN]
+    Implementation details; [README] Benchmarks, --guidance_scale).  The multi-GPU
+    original may send the two branches to separate device groups unless
+    --no_split_batch is given ([README] Benchmarks, Latency); either way every image
+    is its own displaced-patch step -- its own GroupNorm statistics, halo rows and K/V
+    context, and for the transformer stage its own text context -- and the images
+    share only the weights and the step schedule.  x is [B, H, W, C]; contexts is
+    [B, ctx_len, ctx_dim] (transformer stage) or None.  Every returned array gains a
+    leading image axis."""
+
+    def __init__(self, cfg, weights, contexts=None, gn_mode=GN_CORRECTED, context=CTX_DISPLACED):
+        one = dict(cfg, batch=1)
+        self.blocks = [make_block(one, weights, None if contexts is None else contexts[b], gn_mode, context)
+                       for b in range(cfg["batch"])]
+
+    def step(self, x, step, is_sync, **kw):
+        outs = [blk.step(xb, step, is_sync, **kw) for blk, xb in zip(self.blocks, x)]
+        return {k: np.stack([o[k] for o in outs]) if isinstance(outs[0][k], np.ndarray) else [o[k] for o in outs]
+                for k in outs[0]}

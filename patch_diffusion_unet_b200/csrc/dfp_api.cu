@@ -1,15 +1,16 @@
 // libdfp host side: the C ABI of include/dfp.h, the handle with its device
 // buffers, weight re-layout, and the fixed launch sequence of one layer step.
 //
-// Device memory of a handle (row-major, batch 1):
-//   slab[2]     [N][R+2][W][C]   GN1+SiLU output with one halo row above/below each
+// Device memory of a handle (row-major; B images of L = H*W tokens, one after another,
+// each split into N row patches -- patch index b*N + p):
+//   slab[2]     [B*N][R+2][W][C] GN1+SiLU output with one halo row above/below each
 //                                patch; two buffers alternate by step parity, the other
 //                                one holds the previous step's map (stale context)
-//   h, t        [H*W][C]         conv output, GN2 output
-//   q           [heads][L][64]   this step's queries
-//   k[2], v[2]  [heads][L][64]   keys / values, alternating by step parity
-//   o, y        [L][C]           attention output, block output
-//   mom1/2[2]   [N][G][2] fp32   per-(patch, group) (E[x], E[x^2]) of GN1 / GN2, alternating
+//   h, t        [B*H*W][C]       conv output, GN2 output
+//   q           [heads][B*L][64] this step's queries
+//   k[2], v[2]  [heads][B*L][64] keys / values, alternating by step parity
+//   o, y        [B*L][C]         attention output, block output
+//   mom1/2[2]   [B*N][G][2] fp32 per-(patch, group) (E[x], E[x^2]) of GN1 / GN2, alternating
 //   part        fp32 scratch     per-chunk partial sums of the GroupNorm statistics
 #include <cmath>
 #include <cstdio>
@@ -61,6 +62,10 @@ dfp_status check_config(const dfp_config* c, std::string& why) {
   if (c->H % c->n_patches) return bad("H must be a multiple of n_patches");
   if (c->gn_groups <= 0 || c->C % c->gn_groups) return bad("C must be a multiple of gn_groups");
   if (c->n_patches * c->gn_groups > 256) return bad("n_patches * gn_groups must be <= 256");
+  if (c->batch < 0 || c->batch > 8) return bad("batch must be 0..8 (0 counts as 1)");
+  const long long B = c->batch > 1 ? c->batch : 1;
+  if (c->dtype == DFP_F32 && B * c->n_patches * c->gn_groups > 512)
+    return bad("batch * n_patches * gn_groups must be <= 512 for the SIMT kernels (fp32)");
   if (c->head_dim != 64) return bad("head_dim must be 64");
   if (c->heads * c->head_dim != c->C) return bad("heads * head_dim must equal C");
   if (c->C % 64) return bad("C must be a multiple of 64");
@@ -71,7 +76,7 @@ dfp_status check_config(const dfp_config* c, std::string& why) {
   if (!(c->gn_eps >= 0.f)) return bad("gn_eps must be >= 0");
   const long long Lp = (long long)(c->H / c->n_patches) * c->W;
   if (Lp % 8) return bad("(H / n_patches) * W must be a multiple of 8");
-  if ((long long)c->H * c->W * c->C > (1ll << 31)) return bad("feature map too large (H*W*C >= 2^31)");
+  if (B * c->H * c->W * c->C > (1ll << 31)) return bad("feature map too large (batch*H*W*C >= 2^31)");
   if (c->block == DFP_BLOCK_SDXL_STAGE) {
     if (c->dtype != DFP_BF16) { why = "the transformer stage is built for bf16 storage only"; return DFP_E_UNSUPPORTED; }
     if (c->n_xformer < 1 || c->n_xformer > 2) return bad("n_xformer must be 1 or 2");
@@ -95,7 +100,8 @@ void conv_tiles(int R, int W, int& cols_tile, int& rows_tile, int& tiles_per_row
 
 dfp_status build_tmaps(dfp_ctx* h) {
   const dfp_config& c = h->cfg;
-  const int C = c.C, W = c.W, N = c.n_patches, R = h->R, L = h->L;
+  // the batch is B * N patches and B * L tokens: every map and plan spans all images
+  const int C = c.C, W = c.W, N = h->B * c.n_patches, R = h->R, L = h->B * h->L;
   bool ok = true;
   int cols_tile, rows_tile, tpr;
   conv_tiles(R, W, cols_tile, rows_tile, tpr);
@@ -198,7 +204,10 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
   h->Lp = h->R * cfg->W;
   h->esz = dtype_size(cfg->dtype);
   h->family = cfg->dtype == DFP_BF16 ? 0 : 1;
-  const size_t C = cfg->C, N = cfg->n_patches, G = cfg->gn_groups, W = cfg->W, R = h->R, L = h->L;
+  h->B = cfg->batch > 1 ? cfg->batch : 1;
+  // buffers hold all B images: N and L below count patches and tokens over the batch
+  const size_t C = cfg->C, N = (size_t)h->B * cfg->n_patches, G = cfg->gn_groups, W = cfg->W, R = h->R,
+               L = (size_t)h->B * h->L;
   const size_t map = L * C * h->esz;
   const bool is_stage = cfg->block == DFP_BLOCK_SDXL_STAGE;
   bool ok = true;
@@ -376,7 +385,7 @@ dfp_status dfp_step(dfp_handle h, const void* x, int step, int is_sync) {
 dfp_status dfp_step_host(dfp_handle h, const void* x_host, void* y_host, int step, int is_sync) {
   if (!h) return DFP_E_ARG;
   if (!x_host || !y_host) return h->fail(DFP_E_ARG, "x_host / y_host is NULL");
-  const size_t bytes = (size_t)h->L * h->cfg.C * h->esz;
+  const size_t bytes = (size_t)h->B * h->L * h->cfg.C * h->esz;
   cudaError_t e = cudaMemcpyAsync(h->xin, x_host, bytes, cudaMemcpyHostToDevice, h->stream);
   if (e != cudaSuccess) return h->cuda_fail(e, "input copy");
   dfp_status st = dfp_step(h, h->xin, step, is_sync);
@@ -391,7 +400,7 @@ dfp_status dfp_step_host(dfp_handle h, const void* x_host, void* y_host, int ste
 dfp_status dfp_step_host_async(dfp_handle h, const void* x_host, void* y_host, int step, int is_sync) {
   if (!h) return DFP_E_ARG;
   if (!x_host || !y_host) return h->fail(DFP_E_ARG, "x_host / y_host is NULL");
-  const size_t bytes = (size_t)h->L * h->cfg.C * h->esz;
+  const size_t bytes = (size_t)h->B * h->L * h->cfg.C * h->esz;
   cudaError_t e = cudaSuccess;
   if (!h->s_in) {
     e = cudaStreamCreateWithFlags(&h->s_in, cudaStreamNonBlocking);
@@ -446,8 +455,8 @@ dfp_status dfp_output(dfp_handle h, const void** y) {
 }
 
 static bool buffer_of(dfp_handle h, const char* name, const void** ptr, long long* bytes) {
-  const long long map = (long long)h->L * h->cfg.C * (long long)h->esz;
-  const long long st = (long long)h->cfg.n_patches * h->cfg.gn_groups * 2 * 4;
+  const long long map = (long long)h->B * h->L * h->cfg.C * (long long)h->esz;
+  const long long st = (long long)h->B * h->cfg.n_patches * h->cfg.gn_groups * 2 * 4;
   const int cur = h->last_step < 0 ? 0 : (h->last_step & 1);
   const std::string n = name;
   if (h->stage) {
@@ -467,7 +476,7 @@ static bool buffer_of(dfp_handle h, const char* name, const void** ptr, long lon
   else if (n == "gn2") { *ptr = h->dbg2; *bytes = st; }
   else if (n == "slab") {
     *ptr = h->slab[cur];
-    *bytes = (long long)h->cfg.n_patches * (h->R + 2) * h->cfg.W * h->cfg.C * (long long)h->esz;
+    *bytes = (long long)h->B * h->cfg.n_patches * (h->R + 2) * h->cfg.W * h->cfg.C * (long long)h->esz;
   } else return false;
   return true;
 }
@@ -514,11 +523,20 @@ dfp_status dfp_check_device(dfp_handle h) {
 
 int dfp_launches_per_step(dfp_handle h) { return h ? h->launches : -1; }
 
+dfp_status dfp_set_launch_overlap(dfp_handle h, int enable) {
+  if (!h) return DFP_E_ARG;
+  if (enable != 0 && enable != 1) return h->fail(DFP_E_ARG, "enable must be 0 or 1");
+  h->overlap = enable != 0;
+  return DFP_OK;
+}
+
 dfp_status dfp_set_kernel_family(dfp_handle h, int family) {
   if (!h) return DFP_E_ARG;
   if (family != 0 && family != 1) return h->fail(DFP_E_ARG, "family must be 0 or 1");
   if (family == 0 && h->cfg.dtype != DFP_BF16)
     return h->fail(DFP_E_UNSUPPORTED, "tensor-core kernels need bf16 storage");
+  if (family == 1 && h->B * h->cfg.n_patches * h->cfg.gn_groups > 512)
+    return h->fail(DFP_E_UNSUPPORTED, "the SIMT kernels need batch * n_patches * gn_groups <= 512");
   h->family = family;
   return DFP_OK;
 }
@@ -579,7 +597,9 @@ namespace {
 template <typename T>
 dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   const dfp_config& c = h->cfg;
+  // N, L per image; NB, LB over the batch (B images, patch b*N + p, token b*L + i)
   const int N = c.n_patches, C = c.C, G = c.gn_groups, W = c.W, R = h->R, L = h->L, Lp = h->Lp;
+  const int B = h->B, NB = B * N, LB = B * L;
   const int cur = step & 1, prv = cur ^ 1;
   const bool naive = c.context == DFP_CTX_NAIVE;
   const bool displaced = !is_sync && !naive;
@@ -592,11 +612,16 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
 
   // ---- GN1 statistics (+ corrected merge) and apply + SiLU into the slab interior
   GnArgs g{};
-  g.x = x; g.N = N; g.pix_per_patch = Lp; g.C = C; g.G = G; g.eps = c.gn_eps;
+  g.x = x; g.N = NB; g.per_image = N; g.pix_per_patch = Lp; g.C = C; g.G = G; g.eps = c.gn_eps;
   g.part = h->part; g.counter = h->counter;
   g.fresh_out = h->mom1[cur]; g.stale = h->mom1[prv];
   g.gamma = h->gn1_g; g.beta = h->gn1_b; g.dbg = h->dbg1;
   g.is_sync = is_sync; g.mode = (int)c.gn_mode; g.naive = naive ? 1 : 0;
+  // consecutive tensor-core-family kernels overlap launch and set-up with their
+  // predecessor's tail (each waits for the predecessor before touching memory)
+  const int pdl = h->overlap ? 1 : 0;
+  g.pdl = pdl;
+  h->conv_plan.pdl = h->qkv_plan.pdl = h->out_plan.pdl = pdl;
   // the apply also fills the halo rows: the neighbours' boundary rows of this step
   // (sync) or of the previous step (displaced, read from the other slab buffer)
   const int halo_mode = (naive || N == 1) ? 0 : (displaced ? 2 : 1);
@@ -606,8 +631,8 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
     DFP_LAUNCH(launch_gn_fused<T>(g, go, true, h->dev_err, s), "gn1 + SiLU + halo (fused)");
   } else {
     DFP_LAUNCH(launch_gn_stats_merge<T>(g, s), "gn1 statistics");
-    DFP_LAUNCH(launch_gn_apply<T>(x, slab, static_cast<const T*>(h->slab[prv]), h->dbg1, h->gn1_g, h->gn1_b, G, N, Lp,
-                                  C, W, (long long)(R + 2) * W, W, true, halo_mode, s), "gn1 apply + halo");
+    DFP_LAUNCH(launch_gn_apply<T>(x, slab, static_cast<const T*>(h->slab[prv]), h->dbg1, h->gn1_g, h->gn1_b, G, NB, N,
+                                  Lp, C, W, (long long)(R + 2) * W, W, true, halo_mode, s), "gn1 apply + halo");
   }
   // ---- conv3x3 (+ bias) -> h
   Epilogue ec{};
@@ -615,8 +640,8 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   if (h->family == 0) {
     DFP_LAUNCH(launch_tc_gemm(h->conv_plan, h->m_slab[cur], h->m_wconv, ec, h->dev_err, s), "conv (tcgen05)");
   } else {
-    ConvA cv{slab, N, R, W, C};
-    DFP_LAUNCH(launch_simt_gemm<T>(nullptr, &cv, static_cast<const T*>(h->w_conv), L, C, 9 * C, ec, s), "conv (simt)");
+    ConvA cv{slab, NB, R, W, C};
+    DFP_LAUNCH(launch_simt_gemm<T>(nullptr, &cv, static_cast<const T*>(h->w_conv), LB, C, 9 * C, ec, s), "conv (simt)");
   }
   // ---- GN2 (no SiLU) -> t
   g.x = h->h; g.fresh_out = h->mom2[cur]; g.stale = h->mom2[prv];
@@ -627,28 +652,29 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   } else {
     DFP_LAUNCH(launch_gn_stats_merge<T>(g, s), "gn2 statistics");
     DFP_LAUNCH(launch_gn_apply<T>(static_cast<const T*>(h->h), static_cast<T*>(h->t), nullptr, h->dbg2, h->gn2_g,
-                                  h->gn2_b, G, N, Lp, C, W, (long long)Lp, 0, false, 0, s), "gn2 apply");
+                                  h->gn2_b, G, NB, N, Lp, C, W, (long long)Lp, 0, false, 0, s), "gn2 apply");
   }
   // ---- Q, K, V projections; K/V land in this step's cache buffers
   Epilogue eq{};
-  eq.kind = 1; eq.q = h->q; eq.k = h->kb[cur]; eq.v = h->vb[cur]; eq.L = L; eq.C = C;
+  eq.kind = 1; eq.q = h->q; eq.k = h->kb[cur]; eq.v = h->vb[cur]; eq.L = LB; eq.C = C;
   if (h->family == 0) {
     DFP_LAUNCH(launch_tc_gemm(h->qkv_plan, h->m_t, h->m_wqkv, eq, h->dev_err, s), "qkv (tcgen05)");
   } else {
-    DFP_LAUNCH(launch_simt_gemm<T>(static_cast<const T*>(h->t), nullptr, static_cast<const T*>(h->w_qkv), L, 3 * C, C, eq, s), "qkv (simt)");
+    DFP_LAUNCH(launch_simt_gemm<T>(static_cast<const T*>(h->t), nullptr, static_cast<const T*>(h->w_qkv), LB, 3 * C, C, eq, s), "qkv (simt)");
   }
   // ---- displaced attention
   const int mode = naive ? kAttnNaive : (is_sync ? kAttnSync : kAttnDisplaced);
   if (h->family == 0) {
     TcAttnArgs a{};
     a.L = L; a.Lp = Lp; a.N = N; a.heads = c.heads; a.C = C; a.mode = mode; a.o = h->o; a.err = h->dev_err;
+    a.images = B; a.kv_stride = L; a.pdl = pdl;
     a.ctas = h->attn_ctas; a.n_qtiles = (Lp + 127) / 128;
     a.part_o = h->attn_part_o; a.part_ml = h->attn_part_ml; a.counters = h->attn_counters;
     DFP_LAUNCH(launch_tc_attention(a, h->m_q, h->m_k[cur], h->m_v[cur], h->m_k[prv], h->m_v[prv], s), "attention (tcgen05)");
   } else {
     DFP_LAUNCH(launch_simt_attention<T>(static_cast<const T*>(h->q), static_cast<const T*>(h->kb[cur]),
                                         static_cast<const T*>(h->vb[cur]), static_cast<const T*>(h->kb[prv]),
-                                        static_cast<const T*>(h->vb[prv]), static_cast<T*>(h->o), L, Lp, N,
+                                        static_cast<const T*>(h->vb[prv]), static_cast<T*>(h->o), L, Lp, N, B,
                                         c.heads, C, mode, s), "attention (simt)");
   }
   // ---- output projection (+ bias) -> y
@@ -657,7 +683,7 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   if (h->family == 0) {
     DFP_LAUNCH(launch_tc_gemm(h->out_plan, h->m_o, h->m_wo, eo, h->dev_err, s), "out projection (tcgen05)");
   } else {
-    DFP_LAUNCH(launch_simt_gemm<T>(static_cast<const T*>(h->o), nullptr, static_cast<const T*>(h->w_o), L, C, C, eo, s), "out projection (simt)");
+    DFP_LAUNCH(launch_simt_gemm<T>(static_cast<const T*>(h->o), nullptr, static_cast<const T*>(h->w_o), LB, C, C, eo, s), "out projection (simt)");
   }
   DFP_LAUNCH_END();
   return DFP_OK;

@@ -285,6 +285,18 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with the programmatic stream
+// serialization attribute may be scheduled while the kernel before it in the stream is
+// still running.  Every such kernel calls wait_prior_grid() before it reads or writes
+// any buffer another launch touches: it returns once the prior grid has completed and its
+// writes are visible (immediately for a kernel launched without the attribute).  Since
+// every kernel waits, the prior grid's own predecessors have completed too.
+// allow_next_grid() lets the next kernel begin launching; it takes effect once every
+// block of this grid has called it (or exited), so all of this grid's blocks are then
+// resident and the next grid's blocks only take resources this grid no longer needs.
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_next_grid() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // D[tmem] (+)= A[smem desc] * B[smem desc]^T, bf16/f16 operands, one elected thread.
 __device__ __forceinline__ void umma_f16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                             uint32_t idesc, uint32_t accumulate) {

@@ -11,6 +11,8 @@
 //   stale-oth. est_p = (m_p(t) + sum_{j != p} m_j(t-1)) / N
 //   naive      est_p = m_p(t)                             (no cross-patch context)
 //   mean = est.E[x], var = max(est.E[x^2] - mean^2, 0), rstd = 1 / sqrt(var + eps).
+// j runs over the N patches of the same image: a batch of images (the guidance
+// batch) is images x N patches, numbered image-major, with nothing shared across images.
 // The reductions are deterministic: per-thread sums in a fixed pixel order, a
 // fixed-order shared-memory tree, and a last-block merge over the chunk partials
 // in a fixed order (no floating-point atomics).
@@ -36,7 +38,7 @@ __global__ void __launch_bounds__(kGnThreads)
 gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
   constexpr int VEC = VecTraits<T>::kN;
   extern __shared__ float sh[];                 // [2][PL][C] lane sums, then [2][C] channel sums
-  __shared__ float s_mom[256 * 2];              // merged fresh moments  [N*G][2]
+  __shared__ float s_mom[512 * 2];              // merged fresh moments  [N*G][2]
   __shared__ int s_last;
   const int C = a.C, G = a.G, N = a.N;
   const int V = C / VEC;
@@ -103,8 +105,8 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
   if (!s_last) return;
   __threadfence();
 
-  const int NG = N * G;                         // <= 256 (checked on the host)
-  const int S = kGnThreads / NG;                // threads per (patch, group), >= 2
+  const int NG = N * G;                         // <= 512 (checked on the host)
+  const int S = kGnThreads / NG;                // threads per (patch, group), >= 1
   float* red = sh;                              // [S][NG][2]
   if (tid < S * NG) {
     const int item = tid % NG, part_id = tid / NG;
@@ -137,23 +139,24 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
   __syncthreads();
   if (tid < NG) {
     const int pp = tid / G, gg = tid % G;
+    const int NI = a.per_image, j0 = pp / NI * NI;   // the patches of pp's image
     float e1, e2;
     if (a.naive) {
       e1 = s_mom[tid * 2]; e2 = s_mom[tid * 2 + 1];
     } else if (a.is_sync) {
       e1 = 0.f; e2 = 0.f;
-      for (int j = 0; j < N; ++j) { e1 += s_mom[(j * G + gg) * 2]; e2 += s_mom[(j * G + gg) * 2 + 1]; }
-      e1 /= (float)N; e2 /= (float)N;
+      for (int j = j0; j < j0 + NI; ++j) { e1 += s_mom[(j * G + gg) * 2]; e2 += s_mom[(j * G + gg) * 2 + 1]; }
+      e1 /= (float)NI; e2 /= (float)NI;
     } else {
       float st1 = 0.f, st2 = 0.f;
-      for (int j = 0; j < N; ++j) { st1 += a.stale[(j * G + gg) * 2]; st2 += a.stale[(j * G + gg) * 2 + 1]; }
+      for (int j = j0; j < j0 + NI; ++j) { st1 += a.stale[(j * G + gg) * 2]; st2 += a.stale[(j * G + gg) * 2 + 1]; }
       const float own1 = a.stale[(pp * G + gg) * 2], own2 = a.stale[(pp * G + gg) * 2 + 1];
       if (a.mode == 0) {        // corrected
-        e1 = st1 / (float)N + (s_mom[tid * 2] - own1);
-        e2 = st2 / (float)N + (s_mom[tid * 2 + 1] - own2);
+        e1 = st1 / (float)NI + (s_mom[tid * 2] - own1);
+        e2 = st2 / (float)NI + (s_mom[tid * 2 + 1] - own2);
       } else {                  // stale others
-        e1 = (s_mom[tid * 2] + (st1 - own1)) / (float)N;
-        e2 = (s_mom[tid * 2 + 1] + (st2 - own2)) / (float)N;
+        e1 = (s_mom[tid * 2] + (st1 - own1)) / (float)NI;
+        e2 = (s_mom[tid * 2 + 1] + (st2 - own2)) / (float)NI;
       }
     }
     const float var = fmaxf(e2 - e1 * e1, 0.f);
@@ -192,7 +195,7 @@ __global__ void __launch_bounds__(kGnThreads)
 gn_apply_kernel(const T* __restrict__ x, T* __restrict__ out, const T* __restrict__ prev_slab,
                 const float* __restrict__ mean_rstd, const float* __restrict__ gamma,
                 const float* __restrict__ beta, int G, int pix_per_patch, int C, long long out_patch_stride,
-                long long out_off, int pix_per_chunk, int W, int N, int halo_mode) {
+                long long out_off, int pix_per_chunk, int W, int per_image, int halo_mode) {
   constexpr int VEC = VecTraits<T>::kN;
   const int V = C / VEC;
   const int PL = kGnThreads / V;
@@ -214,8 +217,9 @@ gn_apply_kernel(const T* __restrict__ x, T* __restrict__ out, const T* __restric
   const T* src = x + (size_t)p * pix_per_patch * C + vc * VEC;
   T* dst = out + ((size_t)p * out_patch_stride + out_off) * C + vc * VEC;
   const int last_row0 = pix_per_patch - W;
-  const bool top_src = halo_mode != 0 && p > 0;          // my first row feeds patch p-1
-  const bool bot_src = halo_mode != 0 && p < N - 1;      // my last row feeds patch p+1
+  const int pi = p % per_image;                          // patch within its image
+  const bool top_src = halo_mode != 0 && pi > 0;         // my first row feeds patch p-1
+  const bool bot_src = halo_mode != 0 && pi < per_image - 1;   // my last row feeds patch p+1
   for (int pix = pix0 + pl; pix < pix1; pix += 4 * PL) {
     uint4 u[4];
 #pragma unroll
@@ -279,7 +283,7 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
   extern __shared__ float sh[];                 // [2][PL][C] lane sums, then [2][C] channel sums
   __shared__ float s_mr[256 * 2];               // (mean, rstd) of this patch's groups
   __shared__ float s_mom[256 * 2];              // fresh moments of the patches needed
-  const int C = a.C, G = a.G, N = a.N;
+  const int C = a.C, G = a.G;
   const int V = C / VEC;
   const int PL = kGnThreads / V;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -289,10 +293,13 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
   const int pix1 = min(pix0 + pix_per_chunk, a.pix_per_patch);
   const T* base = static_cast<const T*>(a.x) + (size_t)p * a.pix_per_patch * C + vc * VEC;
   float* chan = sh + 2 * PL * C;
+  wait_prior_grid();            // everything below reads or writes buffers of other launches
+  allow_next_grid();
 
   const int last_row0 = a.pix_per_patch - o.W;
-  const bool top_src = o.halo_mode != 0 && p > 0;          // my first row feeds patch p-1
-  const bool bot_src = o.halo_mode != 0 && p < N - 1;      // my last row feeds patch p+1
+  const int NI = a.per_image, pi = p % NI;                 // patch within its image
+  const bool top_src = o.halo_mode != 0 && pi > 0;         // my first row feeds patch p-1
+  const bool bot_src = o.halo_mode != 0 && pi < NI - 1;    // my last row feeds patch p+1
   // ---- displaced steps: the halo rows are last step's values, final already -- copy
   // them now, overlapped with the statistics, instead of after the barrier
   if (o.halo_mode == 2 && pl < PL) {
@@ -358,8 +365,8 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
   if (!grid_barrier(a.counter, total, err)) return;
 
   // ---- phase 2: fresh moments of the patches needed, in a fixed order
-  const bool all = a.is_sync && !a.naive;       // sync steps merge every patch's fresh moments
-  const int p_lo = all ? 0 : p, np = all ? N : 1;
+  const bool all = a.is_sync && !a.naive;       // sync steps merge the image's fresh moments
+  const int p_lo = all ? p - pi : p, np = all ? NI : 1;
   const int items = np * G;                     // <= 256
   const int S = kGnThreads / items;             // threads per item, >= 2
   float* red = sh;                              // [S][items][2]
@@ -386,25 +393,28 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
   __syncthreads();
   if (tid < G) {
     const int gg = tid;
-    const int own = (all ? p : 0) * G + gg;     // this patch's entry in s_mom
+    const int own = (all ? pi : 0) * G + gg;    // this patch's entry in s_mom
     const float m1 = s_mom[own * 2], m2 = s_mom[own * 2 + 1];
     float e1, e2;
     if (a.naive) {
       e1 = m1; e2 = m2;
     } else if (a.is_sync) {
       e1 = 0.f; e2 = 0.f;
-      for (int j = 0; j < N; ++j) { e1 += s_mom[(j * G + gg) * 2]; e2 += s_mom[(j * G + gg) * 2 + 1]; }
-      e1 /= (float)N; e2 /= (float)N;
+      for (int j = 0; j < NI; ++j) { e1 += s_mom[(j * G + gg) * 2]; e2 += s_mom[(j * G + gg) * 2 + 1]; }
+      e1 /= (float)NI; e2 /= (float)NI;
     } else {
       float st1 = 0.f, st2 = 0.f;
-      for (int j = 0; j < N; ++j) { st1 += a.stale[(j * G + gg) * 2]; st2 += a.stale[(j * G + gg) * 2 + 1]; }
+      for (int j = p - pi; j < p - pi + NI; ++j) {
+        st1 += a.stale[(j * G + gg) * 2];
+        st2 += a.stale[(j * G + gg) * 2 + 1];
+      }
       const float own1 = a.stale[(p * G + gg) * 2], own2 = a.stale[(p * G + gg) * 2 + 1];
       if (a.mode == 0) {        // corrected
-        e1 = st1 / (float)N + (m1 - own1);
-        e2 = st2 / (float)N + (m2 - own2);
+        e1 = st1 / (float)NI + (m1 - own1);
+        e2 = st2 / (float)NI + (m2 - own2);
       } else {                  // stale others
-        e1 = (m1 + (st1 - own1)) / (float)N;
-        e2 = (m2 + (st2 - own2)) / (float)N;
+        e1 = (m1 + (st1 - own1)) / (float)NI;
+        e2 = (m2 + (st2 - own2)) / (float)NI;
       }
     }
     const float rstd = 1.f / sqrtf(fmaxf(e2 - e1 * e1, 0.f) + a.eps);
@@ -473,6 +483,8 @@ layernorm_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict_
                  const float* __restrict__ gamma, const float* __restrict__ beta, int L, int C, float eps) {
   const int tok = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
+  wait_prior_grid();
+  allow_next_grid();
   if (tok >= L) return;
   const int nvec = C / 8;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)tok * C);
@@ -554,7 +566,7 @@ cudaError_t launch_gn_stats_merge(const GnArgs& a, cudaStream_t s) {
 
 template <typename T>
 cudaError_t launch_gn_apply(const T* x, T* out, const T* prev_slab, const float* mean_rstd, const float* gamma,
-                            const float* beta, int G, int N, int pix_per_patch, int C, int W,
+                            const float* beta, int G, int N, int per_image, int pix_per_patch, int C, int W,
                             long long out_patch_stride_pix, long long out_pix_off, bool silu, int halo_mode,
                             cudaStream_t s) {
   const int per = chunk_pixels(N, pix_per_patch);
@@ -562,11 +574,11 @@ cudaError_t launch_gn_apply(const T* x, T* out, const T* prev_slab, const float*
   if (silu)
     gn_apply_kernel<T, true><<<grid, kGnThreads, 0, s>>>(x, out, prev_slab, mean_rstd, gamma, beta, G,
                                                          pix_per_patch, C, out_patch_stride_pix, out_pix_off,
-                                                         per, W, N, halo_mode);
+                                                         per, W, per_image, halo_mode);
   else
     gn_apply_kernel<T, false><<<grid, kGnThreads, 0, s>>>(x, out, prev_slab, mean_rstd, gamma, beta, G,
                                                           pix_per_patch, C, out_patch_stride_pix, out_pix_off,
-                                                          per, W, N, halo_mode);
+                                                          per, W, per_image, halo_mode);
   return cudaGetLastError();
 }
 
@@ -596,43 +608,59 @@ cudaError_t launch_gn_fused(const GnArgs& a, const GnOut& o, bool silu, int* err
   cfg.blockDim = dim3(kGnThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;   // every block resident: the grid barrier cannot starve
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, o, n_chunks, per, err);
+  cfg.numAttrs = a.pdl ? 2 : 1;
+  e = cudaLaunchKernelEx(&cfg, kern, a, o, n_chunks, per, err);
+  if (e != cudaSuccess && a.pdl) {
+    // a runtime that does not take both attributes together: launch it plainly
+    cudaGetLastError();
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, a, o, n_chunks, per, err);
+  }
+  return e;
 }
 
 
 cudaError_t launch_layernorm(const void* x, void* y, const float* gamma, const float* beta, int L, int C,
-                             float eps, cudaStream_t s) {
+                             float eps, bool pdl, cudaStream_t s) {
   if (C % 8 || C > 2048) return cudaErrorInvalidValue;
-  const dim3 grid((L + 7) / 8);
   const auto* xi = static_cast<const __nv_bfloat16*>(x);
   auto* yo = static_cast<__nv_bfloat16*>(y);
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3((L + 7) / 8);
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
   switch ((C / 8 + 31) / 32) {   // 16-byte vectors per lane
-    case 1: layernorm_kernel<1><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
-    case 2: layernorm_kernel<2><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
-    case 3: layernorm_kernel<3><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
-    case 4: layernorm_kernel<4><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
-    case 5: layernorm_kernel<5><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
-    case 6: layernorm_kernel<6><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
-    case 7: layernorm_kernel<7><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
-    default: layernorm_kernel<8><<<grid, 256, 0, s>>>(xi, yo, gamma, beta, L, C, eps); break;
+    case 1: return cudaLaunchKernelEx(&cfg, layernorm_kernel<1>, xi, yo, gamma, beta, L, C, eps);
+    case 2: return cudaLaunchKernelEx(&cfg, layernorm_kernel<2>, xi, yo, gamma, beta, L, C, eps);
+    case 3: return cudaLaunchKernelEx(&cfg, layernorm_kernel<3>, xi, yo, gamma, beta, L, C, eps);
+    case 4: return cudaLaunchKernelEx(&cfg, layernorm_kernel<4>, xi, yo, gamma, beta, L, C, eps);
+    case 5: return cudaLaunchKernelEx(&cfg, layernorm_kernel<5>, xi, yo, gamma, beta, L, C, eps);
+    case 6: return cudaLaunchKernelEx(&cfg, layernorm_kernel<6>, xi, yo, gamma, beta, L, C, eps);
+    case 7: return cudaLaunchKernelEx(&cfg, layernorm_kernel<7>, xi, yo, gamma, beta, L, C, eps);
+    default: return cudaLaunchKernelEx(&cfg, layernorm_kernel<8>, xi, yo, gamma, beta, L, C, eps);
   }
-  return cudaGetLastError();
 }
 
 template cudaError_t launch_gn_stats_merge<float>(const GnArgs&, cudaStream_t);
 template cudaError_t launch_gn_stats_merge<__nv_bfloat16>(const GnArgs&, cudaStream_t);
 template cudaError_t launch_gn_apply<float>(const float*, float*, const float*, const float*, const float*,
-                                            const float*, int, int, int, int, int, long long, long long,
-                                            bool, int, cudaStream_t);
+                                            const float*, int, int, int, int, int, int, long long,
+                                            long long, bool, int, cudaStream_t);
 template cudaError_t launch_gn_apply<__nv_bfloat16>(const __nv_bfloat16*, __nv_bfloat16*,
                                                     const __nv_bfloat16*, const float*, const float*,
-                                                    const float*, int, int, int, int, int, long long,
-                                                    long long, bool, int, cudaStream_t);
+                                                    const float*, int, int, int, int, int, int,
+                                                    long long, long long, bool, int, cudaStream_t);
 template cudaError_t launch_gn_fused<float>(const GnArgs&, const GnOut&, bool, int*, cudaStream_t);
 template cudaError_t launch_gn_fused<__nv_bfloat16>(const GnArgs&, const GnOut&, bool, int*, cudaStream_t);
 

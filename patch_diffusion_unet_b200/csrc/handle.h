@@ -28,6 +28,8 @@ struct dfp_ctx {
   long long n_async = 0;       // asynchronous host steps issued so far
   std::string err;
   int R = 0, L = 0, Lp = 0, family = 0;
+  int B = 1;                   // images per step (the guidance batch); L, Lp are per image
+  bool overlap = true;         // programmatic dependent launch between the step's kernels
   size_t esz = 4;
   // weights
   void* w_conv = nullptr;   // [C][9][C]

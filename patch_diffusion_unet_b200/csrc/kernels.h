@@ -13,6 +13,8 @@ enum AttnMode : int { kAttnSync = 0, kAttnDisplaced = 1, kAttnNaive = 2, kAttnCr
 struct GnArgs {
   const void* x;          // [N * pix_per_patch, C] input map, patch-major rows
   int N, pix_per_patch, C, G;
+  int per_image;          // patches per image: N = images * per_image; the merge runs over
+                          // the patches of one image and halos stop at image edges
   float eps;
   float* part;            // scratch [N][n_chunks][G][2] partial (sum x, sum x^2)
   unsigned* counter;      // scratch, one word, zero between launches
@@ -22,6 +24,7 @@ struct GnArgs {
   const float* beta;      // [C] fp32
   float* dbg;             // [N][G][2] (mean, rstd) used -- read by the apply kernel
   int is_sync, mode, naive;
+  int pdl;                // fused kernel: launch with programmatic stream serialization
 };
 // Output side of the fused GroupNorm: out [N][out_patch_stride pixels][C] starting at
 // pixel out_off of each patch (the haloed slab, or a plain map with stride pix_per_patch
@@ -38,16 +41,17 @@ int gn_stats_chunks(int N, int pix_per_patch);
 template <typename T> cudaError_t launch_gn_fused(const GnArgs& a, const GnOut& o, bool silu, int* err, cudaStream_t s);
 template <typename T> cudaError_t launch_gn_stats_merge(const GnArgs& a, cudaStream_t s);
 // halo_mode: 0 none (plain output), 1 sync (fresh neighbour rows), 2 displaced
-// (the previous step's rows, read from prev_slab)
+// (the previous step's rows, read from prev_slab); N patches in all, per_image per image
 template <typename T>
 cudaError_t launch_gn_apply(const T* x, T* out, const T* prev_slab, const float* mean_rstd, const float* gamma,
-                            const float* beta, int G, int N, int pix_per_patch, int C, int W,
+                            const float* beta, int G, int N, int per_image, int pix_per_patch, int C, int W,
                             long long out_patch_stride_pix, long long out_pix_off, bool silu, int halo_mode,
                             cudaStream_t s);
 
 // Per-token LayerNorm over C channels (biased variance), bf16 in / out, fp32 math.
+// pdl: launch with programmatic stream serialization (the kernel waits for its predecessor).
 cudaError_t launch_layernorm(const void* x, void* y, const float* gamma, const float* beta, int L, int C,
-                             float eps, cudaStream_t s);
+                             float eps, bool pdl, cudaStream_t s);
 
 // ---------------------------------------------------------------- GEMM epilogues
 struct Epilogue {
@@ -76,7 +80,7 @@ cudaError_t launch_simt_gemm(const T* A, const ConvA* conv, const T* B, int M, i
                              const Epilogue& epi, cudaStream_t s);
 template <typename T>
 cudaError_t launch_simt_attention(const T* q, const T* kf, const T* vf, const T* ks, const T* vs,
-                                  T* o, int L, int Lp, int N, int heads, int C, int mode,
+                                  T* o, int L, int Lp, int N, int images, int heads, int C, int mode,
                                   cudaStream_t s);
 
 // ---------------------------------------------------------------- tensor-core path (bf16)
@@ -102,6 +106,7 @@ struct TcGemmPlan {
   int pair;               // 1: CTA-pair kernel (256 x bn tiles; B's map boxes bn/2 rows)
   int m_tiles;            // filled by launch_tc_gemm
   int sms;                // persistent grid size (SM count), filled by launch_tc_gemm
+  int pdl;                // launch with programmatic stream serialization
 };
 cudaError_t launch_tc_gemm(const TcGemmPlan& plan, const CUtensorMap& mapA, const CUtensorMap& mapB,
                            const Epilogue& epi, int* err, cudaStream_t s);
@@ -119,9 +124,11 @@ inline int conv_k_stages(int Cin) { return 9 * ((Cin / 64 + 1) / 2); }
 int gemm_m_tiles_plain(int M);
 
 struct TcAttnArgs {
-  int L, Lp, N, heads, C, mode;
+  int L, Lp, N, heads, C, mode;   // per image: L tokens in N patches of Lp
+  int images;             // images of the batch; q, o, k and v hold them one after another
+  int kv_stride;          // K/V rows per image: L, or the padded context rows (kAttnCross)
   int kv_len;             // cross-attention: number of context tokens (mode kAttnCross)
-  void* o;                // [L, C] bf16
+  void* o;                // [images * L, C] bf16
   int* err;
   int n_qtiles;           // ceil(Lp / 128)
   int ctas;               // persistent CTAs (one per SM); the scratch below is sized for them
@@ -129,6 +136,7 @@ struct TcAttnArgs {
   float* part_ml;         // scratch [ctas][2][256][2]:  (running max, row sum) of the same
   unsigned* counters;     // scratch [ctas][2], zero between launches
   int total_tiles;        // set by the launcher
+  int pdl;                // launch with programmatic stream serialization
 };
 // floats of part_o for `ctas` CTAs (part_ml needs 1/32 of it)
 size_t attention_scratch_floats(int ctas);

@@ -105,7 +105,7 @@ extern "C" DFP_API dfp_status dfp_group_norm_noalloc(const void* x, void* y, dfp
   if (e != cudaSuccess) return fail(DFP_E_CUDA, std::string("counter clear: ") + cudaGetErrorString(e));
 
   dfp::GnArgs a{};
-  a.x = x; a.N = n_patches; a.pix_per_patch = pix_per_patch; a.C = C; a.G = groups; a.eps = eps;
+  a.x = x; a.N = n_patches; a.per_image = n_patches; a.pix_per_patch = pix_per_patch; a.C = C; a.G = groups; a.eps = eps;
   a.part = part; a.counter = counter;
   a.fresh_out = fresh_moments; a.stale = stale_moments ? stale_moments : fresh_moments;
   a.gamma = gamma; a.beta = beta;
@@ -116,14 +116,14 @@ extern "C" DFP_API dfp_status dfp_group_norm_noalloc(const void* x, void* y, dfp
     e = dfp::launch_gn_stats_merge<__nv_bfloat16>(a, s);
     if (e == cudaSuccess)
       e = dfp::launch_gn_apply<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y),
-                                              nullptr, mr, gamma, beta, groups, n_patches, pix_per_patch, C, W,
+                                              nullptr, mr, gamma, beta, groups, n_patches, n_patches, pix_per_patch, C, W,
                                               pix_per_patch, 0,
                                               apply_silu != 0, 0, s);
   } else {
     e = dfp::launch_gn_stats_merge<float>(a, s);
     if (e == cudaSuccess)
       e = dfp::launch_gn_apply<float>(static_cast<const float*>(x), static_cast<float*>(y), nullptr, mr, gamma,
-                                      beta, groups, n_patches, pix_per_patch, C, W, pix_per_patch, 0,
+                                      beta, groups, n_patches, n_patches, pix_per_patch, C, W, pix_per_patch, 0,
                                       apply_silu != 0, 0, s);
   }
   if (e != cudaSuccess) return fail(DFP_E_CUDA, std::string("launch: ") + cudaGetErrorString(e));

@@ -91,23 +91,26 @@ simt_gemm_kernel(const T* __restrict__ A, ConvA cv, const T* __restrict__ B, int
 constexpr int kAq = 64;   // queries per block (one per thread)
 constexpr int kAk = 32;   // keys staged per shared-memory tile
 
-// One thread per query row, head width 64, online softmax in fp32.
+// One thread per query row, head width 64, online softmax in fp32.  blockIdx.y runs
+// over images x N patches; q, k, v are [heads][images * L][64] and o [images * L][C],
+// and a patch reads the keys of its own image only.
 template <typename T>
 __global__ void __launch_bounds__(kAq)
 simt_attention_kernel(const T* __restrict__ q, const T* __restrict__ kf, const T* __restrict__ vf,
                       const T* __restrict__ ks, const T* __restrict__ vs, T* __restrict__ o, int L,
-                      int Lp, int C, int mode) {
+                      int Lp, int N, int images, int C, int mode) {
   __shared__ float Ksh[kAk][64];
   __shared__ float Vsh[kAk][64];
-  const int head = blockIdx.z, p = blockIdx.y;
+  const int head = blockIdx.z, pg = blockIdx.y, p = pg % N, img = pg / N;
+  const size_t LT = (size_t)images * L;    // rows per head
   const int local = blockIdx.x * kAq + threadIdx.x;
   const bool valid = local < Lp;
-  const int qi = p * Lp + (valid ? local : 0);
+  const int qi = pg * Lp + (valid ? local : 0);
   const float scale = 0.125f;  // 1 / sqrt(64)
   float qv[64], acc[64];
 #pragma unroll
   for (int j = 0; j < 64; ++j) {
-    qv[j] = to_f32(q[((size_t)head * L + qi) * 64 + j]) * scale;
+    qv[j] = to_f32(q[((size_t)head * LT + qi) * 64 + j]) * scale;
     acc[j] = 0.f;
   }
   float mrun = -INFINITY, lrun = 0.f;
@@ -132,7 +135,7 @@ simt_attention_kernel(const T* __restrict__ q, const T* __restrict__ kf, const T
       const int nk = min(kAk, seg_len[sg] - t0);
       for (int e = threadIdx.x; e < kAk * 64; e += kAq) {
         const int kk = e >> 6, j = e & 63;
-        const size_t row = (size_t)head * L + seg_b[sg] + t0 + kk;
+        const size_t row = (size_t)head * LT + (size_t)img * L + seg_b[sg] + t0 + kk;
         Ksh[kk][j] = kk < nk ? to_f32(Kb[row * 64 + j]) : 0.f;
         Vsh[kk][j] = kk < nk ? to_f32(Vb[row * 64 + j]) : 0.f;
       }
@@ -178,10 +181,10 @@ cudaError_t launch_simt_gemm(const T* A, const ConvA* conv, const T* B, int M, i
 
 template <typename T>
 cudaError_t launch_simt_attention(const T* q, const T* kf, const T* vf, const T* ks, const T* vs,
-                                  T* o, int L, int Lp, int N, int heads, int C, int mode,
+                                  T* o, int L, int Lp, int N, int images, int heads, int C, int mode,
                                   cudaStream_t s) {
-  dim3 grid((Lp + kAq - 1) / kAq, N, heads);
-  simt_attention_kernel<T><<<grid, kAq, 0, s>>>(q, kf, vf, ks, vs, o, L, Lp, C, mode);
+  dim3 grid((Lp + kAq - 1) / kAq, N * images, heads);
+  simt_attention_kernel<T><<<grid, kAq, 0, s>>>(q, kf, vf, ks, vs, o, L, Lp, N, images, C, mode);
   return cudaGetLastError();
 }
 
@@ -192,9 +195,9 @@ template cudaError_t launch_simt_gemm<__nv_bfloat16>(const __nv_bfloat16*, const
                                                      const Epilogue&, cudaStream_t);
 template cudaError_t launch_simt_attention<float>(const float*, const float*, const float*,
                                                   const float*, const float*, float*, int, int,
-                                                  int, int, int, int, cudaStream_t);
+                                                  int, int, int, int, int, cudaStream_t);
 template cudaError_t launch_simt_attention<__nv_bfloat16>(
     const __nv_bfloat16*, const __nv_bfloat16*, const __nv_bfloat16*, const __nv_bfloat16*,
-    const __nv_bfloat16*, __nv_bfloat16*, int, int, int, int, int, int, cudaStream_t);
+    const __nv_bfloat16*, __nv_bfloat16*, int, int, int, int, int, int, int, cudaStream_t);
 
 }  // namespace dfp

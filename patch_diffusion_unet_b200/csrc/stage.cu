@@ -10,15 +10,16 @@
 // Parallelism section items 1-3); LayerNorm, the projections and the feed-forward
 // act per token and need no cross-patch context.
 //
-// Device memory (bf16 storage, fp32 statistics / accumulation):
-//   slab1[2], slab2[2]   [N][R+2][W][C]  conv inputs with halo rows, parity-alternating
-//   h1                   [L][C]          conv1 output
-//   r[1 + 3 n_xformer]   [L][C]          residual stream after the ResNet block and after
-//                                        each attention / feed-forward sub-layer
-//   u                    [L][C]          LayerNorm output (A operand of the projections)
-//   g                    [L][F]          GEGLU output
-//   per block: k[2], v[2] [heads][L][64] self-attention cache; ctx_k, ctx_v
-//                        [heads][ctx_len][64] projected context (computed at load)
+// Device memory (bf16 storage, fp32 statistics / accumulation; B images one after
+// another, L tokens and N patches each, as in the res-attn block):
+//   slab1[2], slab2[2]   [B*N][R+2][W][C]  conv inputs with halo rows, parity-alternating
+//   h1                   [B*L][C]          conv1 output
+//   r[1 + 3 n_xformer]   [B*L][C]          residual stream after the ResNet block and after
+//                                          each attention / feed-forward sub-layer
+//   u                    [B*L][C]          LayerNorm output (A operand of the projections)
+//   g                    [B*L][F]          GEGLU output
+//   per block: k[2], v[2] [heads][B*L][64] self-attention cache; ctx_k, ctx_v
+//                        [heads][B*ctx_rows][64] projected context of each image (at load)
 #include <cmath>
 #include <cstring>
 
@@ -90,7 +91,7 @@ std::vector<WeightSpec> stage_weight_specs(const dfp_config& c, std::vector<std:
       {"resnet.conv1.weight", {C, C, 3, 3}}, {"resnet.conv1.bias", {C}},
       {"resnet.norm2.weight", {C}}, {"resnet.norm2.bias", {C}},
       {"resnet.conv2.weight", {C, C, 3, 3}}, {"resnet.conv2.bias", {C}},
-      {"context", {T, D}},
+      {"context", c.batch > 1 ? std::vector<long long>{c.batch, T, D} : std::vector<long long>{T, D}},
   };
   for (int b = 0; b < c.n_xformer; ++b) {
     const std::string p = "xf" + std::to_string(b) + ".";
@@ -125,9 +126,10 @@ dfp_status stage_create(dfp_ctx* h) {
   Stage* st = new (std::nothrow) Stage();
   if (!st) return h->fail(DFP_E_NOMEM, "host allocation failed");
   h->stage = st;
-  const size_t C = c.C, N = c.n_patches, G = c.gn_groups, W = c.W, R = h->R, L = h->L;
+  // N and L count patches and tokens over the batch; T context tokens per image
+  const size_t B = h->B, C = c.C, N = B * c.n_patches, G = c.gn_groups, W = c.W, R = h->R, L = B * h->L;
   const size_t F = c.ffn_inner, T = c.ctx_len, D = c.ctx_dim, heads = c.heads;
-  const size_t map = L * C * 2, slab = N * (R + 2) * W * C * 2;
+  const size_t map = L * C * 2, slab = N * (R + 2) * W * C * 2, ctx_all = B * ctx_rows(T);
   bool ok = true;
   ok &= h->alloc((void**)&st->n1_g, C * 4) && h->alloc((void**)&st->n1_b, C * 4);
   ok &= h->alloc((void**)&st->n2_g, C * 4) && h->alloc((void**)&st->n2_b, C * 4);
@@ -138,7 +140,7 @@ dfp_status stage_create(dfp_ctx* h) {
     ok &= h->alloc((void**)&st->mom1[i], N * G * 8) && h->alloc((void**)&st->mom2[i], N * G * 8);
   }
   ok &= h->alloc(&st->h1, map) && h->alloc(&st->u, map) && h->alloc(&st->g, L * F * 2);
-  ok &= h->alloc(&st->ctx, T * D * 2);
+  ok &= h->alloc(&st->ctx, B * T * D * 2);
   st->r.assign(1 + 3 * c.n_xformer, nullptr);
   for (auto& p : st->r) ok &= h->alloc(&p, map);
   for (int b = 0; b < c.n_xformer; ++b) {
@@ -151,7 +153,7 @@ dfp_status stage_create(dfp_ctx* h) {
     ok &= h->alloc((void**)&x.b_ff1, 2 * F * 4) && h->alloc((void**)&x.b_ff2, C * 4);
     for (int i = 0; i < 2; ++i) ok &= h->alloc(&x.kb[i], map) && h->alloc(&x.vb[i], map);
     // context K/V: ctx_len rows per head padded with zeros to whole 128-key tiles
-    ok &= h->alloc(&x.ctx_k, heads * ctx_rows(T) * 64 * 2) && h->alloc(&x.ctx_v, heads * ctx_rows(T) * 64 * 2);
+    ok &= h->alloc(&x.ctx_k, heads * ctx_all * 64 * 2) && h->alloc(&x.ctx_v, heads * ctx_all * 64 * 2);
   }
   if (!ok) return h->fail(DFP_E_NOMEM, "device allocation failed");
   cudaError_t e = cudaSuccess;
@@ -165,8 +167,8 @@ dfp_status stage_create(dfp_ctx* h) {
       if (e == cudaSuccess) e = cudaMemset(st->xf[b].vb[i], 0, map);
     }
   for (int b = 0; b < c.n_xformer && e == cudaSuccess; ++b) {
-    e = cudaMemset(st->xf[b].ctx_k, 0, heads * ctx_rows(T) * 64 * 2);
-    if (e == cudaSuccess) e = cudaMemset(st->xf[b].ctx_v, 0, heads * ctx_rows(T) * 64 * 2);
+    e = cudaMemset(st->xf[b].ctx_k, 0, heads * ctx_all * 64 * 2);
+    if (e == cudaSuccess) e = cudaMemset(st->xf[b].ctx_v, 0, heads * ctx_all * 64 * 2);
   }
   if (e != cudaSuccess) return h->cuda_fail(e, "cudaMemset");
   h->y = st->r.back();
@@ -213,8 +215,8 @@ dfp_status stage_create(dfp_ctx* h) {
       ok &= encode_attn_k(&x.m_k[i], x.kb[i], L, heads);
       ok &= encode_attn_v(&x.m_v[i], x.vb[i], L, heads);
     }
-    ok &= encode_attn_k(&x.m_ck, x.ctx_k, ctx_rows(T), heads);
-    ok &= encode_attn_v(&x.m_cv, x.ctx_v, ctx_rows(T), heads);
+    ok &= encode_attn_k(&x.m_ck, x.ctx_k, ctx_all, heads);
+    ok &= encode_attn_v(&x.m_cv, x.ctx_v, ctx_all, heads);
     plan(x.p_qkv, (int)L, 3 * (int)C, (int)C, bq);
     plan(x.p_o1, (int)L, (int)C, (int)C, bc);
     plan(x.p_q2, (int)L, (int)C, (int)C, bc);
@@ -304,14 +306,19 @@ dfp_status stage_finish_load(dfp_ctx* h) {
     const std::string p = "xf" + std::to_string(b) + ".";
     if (x.ctx_ready || !h->loaded.count(p + "attn2.to_k.weight") || !h->loaded.count(p + "attn2.to_v.weight"))
       continue;
-    for (int kv = 0; kv < 2; ++kv) {
-      Epilogue e{};
-      e.kind = 1; e.q = kv == 0 ? x.ctx_k : x.ctx_v; e.L = (int)ctx_rows(c.ctx_len); e.C = c.C;   // padded head stride
-      cudaError_t ce = launch_simt_gemm<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(st->ctx), nullptr,
-                                                       static_cast<const __nv_bfloat16*>(kv == 0 ? x.w_k2 : x.w_v2),
-                                                       c.ctx_len, c.C, c.ctx_dim, e, h->stream);
-      if (ce != cudaSuccess) return h->cuda_fail(ce, "context projection");
-    }
+    // image i's context rows land at rows [i * ctx_rows, i * ctx_rows + ctx_len) of every head
+    const size_t cr = ctx_rows(c.ctx_len);
+    for (int img = 0; img < h->B; ++img)
+      for (int kv = 0; kv < 2; ++kv) {
+        Epilogue e{};
+        e.kind = 1;
+        e.q = static_cast<__nv_bfloat16*>(kv == 0 ? x.ctx_k : x.ctx_v) + img * cr * 64;
+        e.L = (int)(h->B * cr); e.C = c.C;   // head stride: the padded rows of all images
+        cudaError_t ce = launch_simt_gemm<__nv_bfloat16>(
+            static_cast<const __nv_bfloat16*>(st->ctx) + (size_t)img * c.ctx_len * c.ctx_dim, nullptr,
+            static_cast<const __nv_bfloat16*>(kv == 0 ? x.w_k2 : x.w_v2), c.ctx_len, c.C, c.ctx_dim, e, h->stream);
+        if (ce != cudaSuccess) return h->cuda_fail(ce, "context projection");
+      }
     cudaError_t ce = cudaStreamSynchronize(h->stream);
     if (ce != cudaSuccess) return h->cuda_fail(ce, "context projection");
     x.ctx_ready = true;
@@ -322,7 +329,9 @@ dfp_status stage_finish_load(dfp_ctx* h) {
 dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   Stage* st = h->stage;
   const dfp_config& c = h->cfg;
+  // N, L per image; NB, LB over the batch (B images, patch b*N + p, token b*L + i)
   const int N = c.n_patches, C = c.C, G = c.gn_groups, W = c.W, R = h->R, L = h->L, Lp = h->Lp;
+  const int B = h->B, NB = B * N, LB = B * L;
   const int cur = step & 1, prv = cur ^ 1;
   const bool naive = c.context == DFP_CTX_NAIVE;
   const bool displaced = !is_sync && !naive;
@@ -337,7 +346,14 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
 
   // ---- ResNet block: GN1 + SiLU -> conv1 -> GN2 + SiLU -> conv2 + x
   GnArgs g{};
-  g.x = xv; g.N = N; g.pix_per_patch = Lp; g.C = C; g.G = G; g.eps = c.gn_eps;
+  const int pdl = h->overlap ? 1 : 0;   // see run_step: launch overlap between kernels
+  st->p_c1.pdl = st->p_c2.pdl = pdl;
+  for (int b = 0; b < c.n_xformer; ++b)
+    for (TcGemmPlan* p : {&st->xf[b].p_qkv, &st->xf[b].p_o1, &st->xf[b].p_q2, &st->xf[b].p_o2, &st->xf[b].p_ff1,
+                          &st->xf[b].p_ff2})
+      p->pdl = pdl;
+  g.pdl = pdl;
+  g.x = xv; g.N = NB; g.per_image = N; g.pix_per_patch = Lp; g.C = C; g.G = G; g.eps = c.gn_eps;
   g.part = h->part; g.counter = h->counter;
   g.is_sync = is_sync; g.mode = (int)c.gn_mode; g.naive = naive ? 1 : 0;
   g.fresh_out = st->mom1[cur]; g.stale = st->mom1[prv]; g.gamma = st->n1_g; g.beta = st->n1_b; g.dbg = h->dbg1;
@@ -366,12 +382,13 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
     void* r_ca = st->r[3 * b + 2];
     void* r_ff = st->r[3 * b + 3];
     // self-attention on displaced K/V
-    DFP_LAUNCH(launch_layernorm(rin, st->u, x.ln_g[0], x.ln_b[0], L, C, 1e-5f, s), "layernorm 1");
+    DFP_LAUNCH(launch_layernorm(rin, st->u, x.ln_g[0], x.ln_b[0], LB, C, 1e-5f, pdl != 0, s), "layernorm 1");
     Epilogue eq{};
-    eq.kind = 1; eq.q = h->q; eq.k = x.kb[cur]; eq.v = x.vb[cur]; eq.L = L; eq.C = C;
+    eq.kind = 1; eq.q = h->q; eq.k = x.kb[cur]; eq.v = x.vb[cur]; eq.L = LB; eq.C = C;
     DFP_LAUNCH(launch_tc_gemm(x.p_qkv, st->m_u, x.m_wqkv, eq, h->dev_err, s), "self-attn qkv (tcgen05)");
     TcAttnArgs a{};
     a.L = L; a.Lp = Lp; a.N = N; a.heads = c.heads; a.C = C; a.mode = sa_mode; a.o = h->o; a.err = h->dev_err;
+    a.images = B; a.kv_stride = L; a.pdl = pdl;
     a.n_qtiles = (Lp + 127) / 128; a.ctas = h->attn_ctas;
     a.part_o = h->attn_part_o; a.part_ml = h->attn_part_ml; a.counters = h->attn_counters;
     DFP_LAUNCH(launch_tc_attention(a, h->m_q, x.m_k[cur], x.m_v[cur], x.m_k[prv], x.m_v[prv], s),
@@ -380,19 +397,21 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
     eo.kind = 0; eo.out = r_sa; eo.bias = x.b_o1; eo.residual = rin; eo.ldo = C;
     DFP_LAUNCH(launch_tc_gemm(x.p_o1, st->m_o, x.m_wo1, eo, h->dev_err, s), "self-attn out + residual (tcgen05)");
     // cross-attention to the fixed context (same for every patch: no staleness)
-    DFP_LAUNCH(launch_layernorm(r_sa, st->u, x.ln_g[1], x.ln_b[1], L, C, 1e-5f, s), "layernorm 2");
+    DFP_LAUNCH(launch_layernorm(r_sa, st->u, x.ln_g[1], x.ln_b[1], LB, C, 1e-5f, pdl != 0, s), "layernorm 2");
     Epilogue e2{};
-    e2.kind = 1; e2.q = h->q; e2.L = L; e2.C = C;
+    e2.kind = 1; e2.q = h->q; e2.L = LB; e2.C = C;
     DFP_LAUNCH(launch_tc_gemm(x.p_q2, st->m_u, x.m_wq2, e2, h->dev_err, s), "cross-attn q (tcgen05)");
     TcAttnArgs ca{};
     ca.L = L; ca.Lp = L; ca.N = 1; ca.heads = c.heads; ca.C = C; ca.mode = kAttnCross; ca.kv_len = c.ctx_len;
+    ca.images = B; ca.kv_stride = (int)ctx_rows(c.ctx_len);   // image b reads its own context
+    ca.pdl = pdl;
     ca.o = h->o; ca.err = h->dev_err; ca.n_qtiles = (L + 127) / 128; ca.ctas = h->attn_ctas;
     ca.part_o = h->attn_part_o; ca.part_ml = h->attn_part_ml; ca.counters = h->attn_counters;
     DFP_LAUNCH(launch_tc_attention(ca, h->m_q, x.m_ck, x.m_cv, x.m_ck, x.m_cv, s), "cross-attention (tcgen05)");
     eo.out = r_ca; eo.bias = x.b_o2; eo.residual = r_sa;
     DFP_LAUNCH(launch_tc_gemm(x.p_o2, st->m_o, x.m_wo2, eo, h->dev_err, s), "cross-attn out + residual (tcgen05)");
     // GEGLU feed-forward
-    DFP_LAUNCH(launch_layernorm(r_ca, st->u, x.ln_g[2], x.ln_b[2], L, C, 1e-5f, s), "layernorm 3");
+    DFP_LAUNCH(launch_layernorm(r_ca, st->u, x.ln_g[2], x.ln_b[2], LB, C, 1e-5f, pdl != 0, s), "layernorm 3");
     Epilogue ef{};
     ef.kind = 2; ef.out = st->g; ef.bias = x.b_ff1; ef.ldo = c.ffn_inner;
     DFP_LAUNCH(launch_tc_gemm(x.p_ff1, st->m_u, x.m_wff1, ef, h->dev_err, s), "ff proj + GEGLU (tcgen05)");
@@ -406,14 +425,14 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
 bool stage_buffer(dfp_ctx* h, const std::string& name, const void** ptr, long long* bytes) {
   Stage* st = h->stage;
   const dfp_config& c = h->cfg;
-  const long long map = (long long)h->L * c.C * 2;
+  const long long map = (long long)h->B * h->L * c.C * 2;
   const int cur = h->last_step < 0 ? 0 : (h->last_step & 1);
   if (name == "y") { *ptr = st->r.back(); *bytes = map; return true; }
   if (name == "resnet") { *ptr = st->r[0]; *bytes = map; return true; }
   if (name == "h") { *ptr = st->h1; *bytes = map; return true; }
   if (name == "slab" || name == "slab2") {
     *ptr = name == "slab" ? st->slab1[cur] : st->slab2[cur];
-    *bytes = (long long)c.n_patches * (h->R + 2) * c.W * c.C * 2;
+    *bytes = (long long)h->B * c.n_patches * (h->R + 2) * c.W * c.C * 2;
     return true;
   }
   for (int b = 0; b < c.n_xformer; ++b) {

@@ -10,7 +10,10 @@
 //   displaced  own patch fresh, then [0, p*Lp) stale, then [(p+1)*Lp, L) stale
 //   naive      own patch fresh only (the naive-patch baseline, README Overview (b))
 // Segment ends need not be multiples of the 128-key tile: columns past a
-// segment's end are masked.
+// segment's end are masked.  A batch of images (the guidance batch) is images x N
+// patches: Q, O, K and V hold the images one after another (rows img * L + token;
+// cross-attention contexts at img * kv_stride), and a patch reads only the keys of
+// its own image.
 //
 // CTA layout (640 threads, five warpgroups): two softmax groups of 8 warps, each
 // owning one 128-query tile.  Warps w and w+4 of a group read the same 32 TMEM
@@ -37,7 +40,7 @@
 // nodes, max relative error 7.5e-5) to offload the MUFU unit.
 //
 // Work split (stream-K style): a unit of work is one KV tile for one Q-tile pair of
-// one (patch, head).  The units are laid out pair-major within (patch, head) and
+// one (patch, head), the patches of all images of the batch in one list.  The units are laid out pair-major within (patch, head) and
 // the whole list is cut into one contiguous range per SM, so every CTA gets the
 // same number of KV tiles whatever the number of pairs.  A CTA walks its range as
 // a sequence of pieces (the part of one pair's KV list that falls in the range);
@@ -111,17 +114,18 @@ __device__ __forceinline__ void tile_src(int mode, int p, int Lp, int L, int kv_
   valid = min(kTile, L - row);
 }
 
-// The unit list: patch-major, then head, then Q-tile pair; unit (p, head, pair) has
-// unit_tiles(p) KV tiles.  Global tile x -> its unit and the unit's first tile.
+// The unit list: patch-major over the images' patches (patch pg = img * N + p, so Q and O
+// rows start at pg * Lp), then head, then Q-tile pair; unit (pg, head, pair) has
+// unit_tiles(pg % N) KV tiles.  Global tile x -> its unit and the unit's first tile.
 // All schedule arithmetic is 32-bit: the launcher checks total_tiles * ctas < 2^31.
 struct Unit {
-  int p, head, pair, T, U0;
+  int p, head, pair, T, U0;   // p: patch over the batch (img * N + patch within the image)
 };
 __device__ __forceinline__ Unit locate(const TcAttnArgs& a, int n_pairs, int x) {
   int base = 0;
   Unit u{};
-  for (int p = 0; p < a.N; ++p) {
-    const int T = unit_tiles(a.mode, p, a.Lp, a.L, a.kv_len);
+  for (int p = 0; p < a.N * a.images; ++p) {
+    const int T = unit_tiles(a.mode, p % a.N, a.Lp, a.L, a.kv_len);
     const int blk = T * a.heads * n_pairs;
     if (x < base + blk) {
       const int ui = (x - base) / T;
@@ -141,7 +145,7 @@ __device__ __forceinline__ void advance(const TcAttnArgs& a, int n_pairs, Unit& 
     if (++u.head == a.heads) {
       u.head = 0;
       ++u.p;
-      u.T = unit_tiles(a.mode, u.p, a.Lp, a.L, a.kv_len);
+      u.T = unit_tiles(a.mode, u.p % a.N, a.Lp, a.L, a.kv_len);
     }
   }
 }
@@ -449,6 +453,9 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the set-up above touches no global memory: overlap it with the prior kernel's tail
+  wait_prior_grid();
+  allow_next_grid();
 
   if (warp >= kWarpTma) {
    // Register split: this warpgroup (TMA, MMA and two idle warps) gives registers to
@@ -480,10 +487,13 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
         tma_load_3d(smem_u32(sQ + (2 * qb + 1) * kTileBytes), &mq, qbar, 0, qrow + kTile, u.head);
       }
       __syncwarp();
+      // the piece's patch within its image, and the image's first K/V row
+      const int img = u.p / a.N, p_img = u.p - img * a.N, kv0 = img * a.kv_stride;
       for (int jj = 0; jj < n; ++jj, ++gt) {
         const int s = gt % kStages, round = gt / kStages;
         int stale, row, valid;
-        tile_src(a.mode, u.p, a.Lp, a.L, a.kv_len, jl0 + jj, stale, row, valid);
+        tile_src(a.mode, p_img, a.Lp, a.L, a.kv_len, jl0 + jj, stale, row, valid);
+        row += kv0;
         if (round > 0 && !mbar_wait_warp(smem_u32(&k_empty[s]), (round - 1) & 1, err, kErrWaitStageFree)) { ok = false; break; }
         if (leader) {
           mbar_arrive_expect_tx(smem_u32(&k_full[s]), kTileBytes);
@@ -683,7 +693,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
         int valid = kTile;
         if (!((a.mode == kAttnCross ? a.kv_len : (a.Lp | a.L)) % kTile == 0)) {
           int stale, krow;
-          tile_src(a.mode, sp[0], a.Lp, a.L, a.kv_len, sp[5] - sp[4] + jj, stale, krow, valid);
+          tile_src(a.mode, sp[0] % a.N, a.Lp, a.L, a.kv_len, sp[5] - sp[4] + jj, stale, krow, valid);
         }
         if (!mbar_wait_warp(smem_u32(&s_full[g]), gt & 1, err, kErrWaitAttnS)) { carry = true; break; }
         tc_fence_after();
@@ -826,7 +836,7 @@ long long attention_total_tiles(const TcAttnArgs& a) {
   const int n_pairs = (a.n_qtiles + 1) / 2;
   long long tt = 0;
   for (int p = 0; p < a.N; ++p) tt += (long long)unit_tiles(a.mode, p, a.Lp, a.L, a.kv_len) * a.heads * n_pairs;
-  return tt;
+  return tt * a.images;
 }
 
 size_t attention_scratch_floats(int ctas) { return (size_t)ctas * 2 * 256 * 64; }
@@ -848,13 +858,23 @@ cudaError_t launch_tc_attention(const TcAttnArgs& args, const CUtensorMap& mq, c
   }
   if (regs * kThreads < 128 * kRegsTmaMma + 512 * kRegsSoftmax) return cudaErrorInvalidConfiguration;
   TcAttnArgs a = args;
+  if (a.images < 1 || a.kv_stride < 0) return cudaErrorInvalidValue;
   const long long tt = attention_total_tiles(a);
   if (tt <= 0) return cudaSuccess;
   const int G = (int)std::min<long long>(a.ctas, tt);
   if (G <= 0 || tt * G >= (1ll << 31)) return cudaErrorInvalidValue;   // 32-bit schedule arithmetic
   a.total_tiles = (int)tt;
-  tc_attention_kernel<<<G, kThreads, smem, s>>>(mq, mkf, mvf, mks, mvs, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(G);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, tc_attention_kernel, mq, mkf, mvf, mks, mvs, a);
 }
 
 }  // namespace dfp

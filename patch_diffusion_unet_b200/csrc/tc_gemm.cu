@@ -188,6 +188,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  // the set-up above touches no global memory: overlap it with the prior kernel's tail
+  wait_prior_grid();
+  allow_next_grid();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -356,6 +359,8 @@ tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_const
   cluster_sync_all();          // both CTAs' barriers exist before either touches the other's
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  wait_prior_grid();           // the set-up above touches no global memory
+  allow_next_grid();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -499,13 +504,15 @@ cudaError_t launch_pair(const TcGemmPlan& plan, const CUtensorMap& mA, const CUt
   if (e != cudaSuccess) return e;
   const int n_tiles = ((plan.m_tiles + 1) / 2) * (plan.N / BN);
   cudaLaunchConfig_t cfg{};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1;   // the occupancy query sees the cluster shape only
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -521,6 +528,7 @@ cudaError_t launch_pair(const TcGemmPlan& plan, const CUtensorMap& mA, const CUt
   }
   const int pairs = n_tiles < max_pairs ? n_tiles : max_pairs;
   cfg.gridDim = dim3(2 * pairs);
+  cfg.numAttrs = plan.pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, mA, mB, plan, epi, err);
 }
 
@@ -533,8 +541,17 @@ cudaError_t launch_bn(const TcGemmPlan& plan, const CUtensorMap& mA, const CUten
   if (e != cudaSuccess) return e;
   const int n_tiles = plan.m_tiles * (plan.N / BN);
   const int grid = n_tiles < plan.sms ? n_tiles : plan.sms;
-  kern<<<grid, kThreads, smem, s>>>(mA, mB, plan, epi, err);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = plan.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, mA, mB, plan, epi, err);
 }
 
 }  // namespace

@@ -24,7 +24,7 @@ EXPORTED = ("dfp_create", "dfp_load_weights", "dfp_step", "dfp_step_host", "dfp_
             "dfp_copy_out", "dfp_buffer_bytes", "dfp_check_device", "dfp_launches_per_step",
             "dfp_set_kernel_family", "dfp_set_profiling", "dfp_kernel_times", "dfp_destroy",
             "dfp_last_error", "dfp_group_norm_noalloc", "dfp_group_norm_noalloc_error",
-            "dfp_selftest_wait_timeout")
+            "dfp_selftest_wait_timeout", "dfp_set_launch_overlap")
 
 
 class Config(ctypes.Structure):
@@ -33,7 +33,7 @@ class Config(ctypes.Structure):
                 ("heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("block", ctypes.c_int), ("gn_mode", ctypes.c_int), ("context", ctypes.c_int),
                 ("n_xformer", ctypes.c_int), ("ffn_inner", ctypes.c_int), ("ctx_len", ctypes.c_int),
-                ("ctx_dim", ctypes.c_int)]
+                ("ctx_dim", ctypes.c_int), ("batch", ctypes.c_int)]
 
 
 class Tensor(ctypes.Structure):
@@ -61,6 +61,7 @@ def load_library(path=_LIB_PATH):
         "dfp_check_device": ([H], ctypes.c_int),
         "dfp_launches_per_step": ([H], ctypes.c_int),
         "dfp_set_kernel_family": ([H, ctypes.c_int], ctypes.c_int),
+        "dfp_set_launch_overlap": ([H, ctypes.c_int], ctypes.c_int),
         "dfp_set_profiling": ([H, ctypes.c_int], ctypes.c_int),
         "dfp_kernel_times": ([H, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_char_p), ctypes.c_int],
                              ctypes.c_int),
@@ -109,6 +110,7 @@ def make_config(cfg, gn_mode=GN_CORRECTED, context=CTX_DISPLACED):
     c.ffn_inner = cfg.get("ffn_inner", 0)
     c.ctx_len = cfg.get("ctx_len", 0)
     c.ctx_dim = cfg.get("ctx_dim", 0)
+    c.batch = cfg.get("batch", 1)
     return c
 
 
@@ -163,7 +165,8 @@ class DisplacedPatchBlock:
         self._check(LIB.dfp_load_weights(self.h, arr, len(weights)))
 
     def step(self, x, step, is_sync):
-        """x: contiguous CUDA tensor [H, W, C] of the config dtype (must outlive the stream work)."""
+        """x: contiguous CUDA tensor [B, H, W, C] (B = cfg "batch", default 1; [H, W, C] for one
+        image) of the config dtype (must outlive the stream work)."""
         if not (x.is_cuda and x.is_contiguous() and x.dtype == self.tdtype):
             raise ValueError("x must be a contiguous CUDA tensor of the config dtype")
         self._check(LIB.dfp_step(self.h, ctypes.c_void_p(x.data_ptr()), int(step), int(is_sync)))
@@ -194,7 +197,7 @@ class DisplacedPatchBlock:
         return out
 
     def output(self):
-        return self.buffer("y").view(self.cfg["H"] * self.cfg["W"], self.cfg["C"])
+        return self.buffer("y").view(self.cfg.get("batch", 1) * self.cfg["H"] * self.cfg["W"], self.cfg["C"])
 
     def check_device(self):
         self._check(LIB.dfp_check_device(self.h))
@@ -216,3 +219,7 @@ class DisplacedPatchBlock:
 
     def set_kernel_family(self, family):
         self._check(LIB.dfp_set_kernel_family(self.h, int(family)))
+
+    def set_launch_overlap(self, enable=True):
+        """Programmatic dependent launch between the step's kernels (on by default)."""
+        self._check(LIB.dfp_set_launch_overlap(self.h, int(enable)))

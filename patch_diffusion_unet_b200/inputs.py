@@ -16,6 +16,12 @@ Recipe (fixed, seed 0 unless stated):
   round-to-nearest-even, and returned as float32 whose values are exactly
   representable in the storage type.
 
+  A batch of B images (workload key "batch", the classifier-free-guidance batch):
+  image 0 is the single-image workload above, unchanged; image b >= 1 draws its
+  own context (transformer stage) and then its x_0, e_1, e_2, ... from
+  numpy.random.default_rng([seed, b]).  The weights are image 0's.  x(t) is then
+  [B, H, W, C] and the context [B, ctx_len, ctx_dim].
+
 Stand-in for the pages' workload: SDXL latents of COCO-caption prompts
 ("DistriFusion: Distributed Parallel Inference for High-Resolution Diffusion
 Models" README, Benchmarks / COCO quality) are not available; these synthetic
@@ -117,11 +123,14 @@ class SyntheticWorkload:
             else:
                 v = np.full(shape, fill)
             self.weights[name] = round_to(v, self.dtype)
+        self.batch = cfg.get("batch", 1)
+        # image b >= 1 of a batch: its own stream for its context and its inputs
+        self.rngs = [self.rng] + [np.random.default_rng([seed, b]) for b in range(1, self.batch)]
         self.context = None
         if cfg["block"] == "sdxl_stage":
-            self.context = round_to(self.rng.standard_normal((cfg["ctx_len"], cfg["ctx_dim"])),
-                                    self.dtype)
-        self._state = None   # fp64 x_t
+            ctx = [round_to(r.standard_normal((cfg["ctx_len"], cfg["ctx_dim"])), self.dtype) for r in self.rngs]
+            self.context = ctx[0] if self.batch == 1 else np.stack(ctx)
+        self._state = None   # fp64 x_t, one per image
         self._t = -1
 
     def x(self, t):
@@ -132,11 +141,12 @@ class SyntheticWorkload:
             raise ValueError(f"inputs are drawn sequentially: asked for step {t} after {self._t}")
         shape = (self.cfg["H"], self.cfg["W"], self.cfg["C"])
         if t == 0:
-            self._state = self.rng.standard_normal(shape)
+            self._state = [r.standard_normal(shape) for r in self.rngs]
         else:
-            self._state = RHO * self._state + NOISE * self.rng.standard_normal(shape)
+            self._state = [RHO * s + NOISE * r.standard_normal(shape) for s, r in zip(self._state, self.rngs)]
         self._t = t
-        self._cur = round_to(self._state, self.dtype)
+        cur = [round_to(s, self.dtype) for s in self._state]
+        self._cur = cur[0] if self.batch == 1 else np.stack(cur)
         return self._cur
 
     def schedule(self):

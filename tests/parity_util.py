@@ -23,20 +23,23 @@ def host(t):
 
 
 def gpu_stage_views(blk, cfg):
-    """Internal buffers of the last GPU step, reshaped like the oracle's intermediates."""
+    """Internal buffers of the last GPU step, reshaped like the oracle's intermediates
+    (with a leading image axis for a batch; the slab keeps its [B*N, R+2, W, C] rows)."""
     H, W, C, N, heads = cfg["H"], cfg["W"], cfg["C"], cfg["n_patches"], cfg["heads"]
+    B = cfg.get("batch", 1)
     R, L = H // N, H * W
-    slab = host(blk.buffer("slab")).reshape(N, R + 2, W, C)
+    lead = (B,) if B > 1 else ()
+    slab = host(blk.buffer("slab")).reshape(B * N, R + 2, W, C)
     out = dict(
         slab=slab,
-        y1=slab[:, 1:R + 1].reshape(H, W, C),
-        h=host(blk.buffer("h")).reshape(H, W, C),
-        t=host(blk.buffer("t")).reshape(H, W, C),
-        o=host(blk.buffer("o")).reshape(L, C),
-        y=host(blk.buffer("y")).reshape(L, C),
+        y1=slab[:, 1:R + 1].reshape(lead + (H, W, C)),
+        h=host(blk.buffer("h")).reshape(lead + (H, W, C)),
+        t=host(blk.buffer("t")).reshape(lead + (H, W, C)),
+        o=host(blk.buffer("o")).reshape(lead + (L, C)),
+        y=host(blk.buffer("y")).reshape(lead + (L, C)),
     )
     for n in ("q", "k", "v"):
-        out[n] = host(blk.buffer(n)).reshape(heads, L, 64).transpose(1, 0, 2).reshape(L, C)
+        out[n] = host(blk.buffer(n)).reshape(heads, B, L, 64).transpose(1, 2, 0, 3).reshape(lead + (L, C))
     return out
 
 
@@ -71,12 +74,13 @@ def run_parity(cfg, n_steps, oracle_from=0, query_tokens=None, gn_mode=0, contex
         ref = orc.step(x, t - oracle_from, is_sync, query_tokens=query_tokens)
         g = gpu_stage_views(blk, cfg) if stages else dict(y=host(blk.output()))
         res = {}
-        yg = g["y"] if query_tokens is None else g["y"][query_tokens]
+        qsel = (query_tokens,) if cfg.get("batch", 1) == 1 else (slice(None), query_tokens)
+        yg = g["y"] if query_tokens is None else g["y"][qsel]
         res["y"] = (rel_l2(yg, ref["y"]), max_abs(yg, ref["y"]))
         if stages:
             for n in ("y1", "h", "t", "q", "k", "v"):
                 res[n] = (rel_l2(g[n], ref[n]), max_abs(g[n], ref[n]))
-            og = g["o"] if query_tokens is None else g["o"][query_tokens]
+            og = g["o"] if query_tokens is None else g["o"][qsel]
             res["o"] = (rel_l2(og, ref["o"]), max_abs(og, ref["o"]))
             res["halo_ok"] = check_halos(cfg, g["slab"], prev_slab, is_sync, context)
             prev_slab = g["slab"]
@@ -88,8 +92,16 @@ def run_parity(cfg, n_steps, oracle_from=0, query_tokens=None, gn_mode=0, contex
 
 
 def check_halos(cfg, slab, prev_slab, is_sync, context):
-    """Halo rows are copies: bit-exact against the source rows (stale = previous GPU step)."""
+    """Halo rows are copies: bit-exact against the source rows (stale = previous GPU step).
+    A batch's slab holds B images of N patches each; every image is checked on its own
+    (its first and last patch get zero halos: the image edges)."""
     N = cfg["n_patches"]
+    B = cfg.get("batch", 1)
+    if B > 1:
+        per = slab.shape[0] // B
+        return all(check_halos(dict(cfg, batch=1), slab[b * per:(b + 1) * per],
+                               None if prev_slab is None else prev_slab[b * per:(b + 1) * per], is_sync, context)
+                   for b in range(B))
     R = cfg["H"] // N
     if N == 1 or context == 1:
         return bool(np.all(slab[:, 0] == 0) and np.all(slab[:, R + 1] == 0))

@@ -74,3 +74,65 @@ def sdxl_stage_full(x, w, ctx, cfg):
         a, gate = hg.chunk(2, dim=-1)
         r = r + F.linear(a * F.gelu(gate), _t(w[p + "ff.out.weight"]), _t(w[p + "ff.out.bias"]))
     return dict(y=r.numpy())
+
+
+# ---------------------------------------------------------------- batched (guidance batch)
+# The same layers on a batch [B, H, W, C] with PyTorch's batched routines: group_norm
+# takes its statistics per sample, conv2d runs per sample, and scaled_dot_product_attention
+# attends within each batch element -- so these pin that a batch of images never mixes.
+
+def _mha_batched(tok, wq, wk, wv, wo, bo, heads, ctx=None):
+    ctx = tok if ctx is None else ctx
+    B, L, C = tok.shape
+    d = C // heads
+
+    def split(u):
+        return u.view(B, u.shape[1], heads, d).transpose(1, 2)
+
+    q, k, v = split(F.linear(tok, _t(wq))), split(F.linear(ctx, _t(wk))), split(F.linear(ctx, _t(wv)))
+    o = F.scaled_dot_product_attention(q, k, v).transpose(1, 2).reshape(B, L, C)
+    return F.linear(o, _t(wo), _t(bo)), o
+
+
+def res_attn_full_batched(xs, w, cfg):
+    """res_attn_full on a batch xs [B, H, W, C]; arrays come back with a leading batch axis."""
+    G, eps = cfg["gn_groups"], cfg["gn_eps"]
+    B, H, W, C = xs.shape
+    X = _t(xs).permute(0, 3, 1, 2)
+    y1 = F.silu(F.group_norm(X, G, _t(w["gn1.weight"]), _t(w["gn1.bias"]), eps))
+    h = F.conv2d(y1, _t(w["conv1.weight"]), _t(w["conv1.bias"]), padding=1)
+    t = F.group_norm(h, G, _t(w["gn2.weight"]), _t(w["gn2.bias"]), eps)
+    tok = t.permute(0, 2, 3, 1).reshape(B, H * W, C)
+    y, o = _mha_batched(tok, w["attn.to_q.weight"], w["attn.to_k.weight"], w["attn.to_v.weight"],
+                        w["attn.to_out.weight"], w["attn.to_out.bias"], cfg["heads"])
+    nhwc = lambda a: a.permute(0, 2, 3, 1).numpy()  # noqa: E731
+    return dict(y=y.numpy(), y1=nhwc(y1), h=nhwc(h), t=nhwc(t), o=o.numpy())
+
+
+def sdxl_stage_full_batched(xs, w, ctxs, cfg):
+    """sdxl_stage_full on a batch xs [B, H, W, C] with one context per image ctxs [B, T, D]."""
+    G, eps, C = cfg["gn_groups"], cfg["gn_eps"], cfg["C"]
+    B, H, W, _ = xs.shape
+    X = _t(xs).permute(0, 3, 1, 2)
+    h = F.conv2d(F.silu(F.group_norm(X, G, _t(w["resnet.norm1.weight"]), _t(w["resnet.norm1.bias"]), eps)),
+                 _t(w["resnet.conv1.weight"]), _t(w["resnet.conv1.bias"]), padding=1)
+    h = F.conv2d(F.silu(F.group_norm(h, G, _t(w["resnet.norm2.weight"]), _t(w["resnet.norm2.bias"]), eps)),
+                 _t(w["resnet.conv2.weight"]), _t(w["resnet.conv2.bias"]), padding=1)
+    r = (X + h).permute(0, 2, 3, 1).reshape(B, H * W, C)
+    c = _t(ctxs)
+    for b in range(cfg["n_xformer"]):
+        p = f"xf{b}."
+
+        def ln(u, n):
+            return F.layer_norm(u, (C,), _t(w[p + n + ".weight"]), _t(w[p + n + ".bias"]), 1e-5)
+
+        r = r + _mha_batched(ln(r, "norm1"), w[p + "attn1.to_q.weight"], w[p + "attn1.to_k.weight"],
+                             w[p + "attn1.to_v.weight"], w[p + "attn1.to_out.weight"],
+                             w[p + "attn1.to_out.bias"], cfg["heads"])[0]
+        r = r + _mha_batched(ln(r, "norm2"), w[p + "attn2.to_q.weight"], w[p + "attn2.to_k.weight"],
+                             w[p + "attn2.to_v.weight"], w[p + "attn2.to_out.weight"],
+                             w[p + "attn2.to_out.bias"], cfg["heads"], ctx=c)[0]
+        hg = F.linear(ln(r, "norm3"), _t(w[p + "ff.proj.weight"]), _t(w[p + "ff.proj.bias"]))
+        a, gate = hg.chunk(2, dim=-1)
+        r = r + F.linear(a * F.gelu(gate), _t(w[p + "ff.out.weight"]), _t(w[p + "ff.out.bias"]))
+    return dict(y=r.numpy())
