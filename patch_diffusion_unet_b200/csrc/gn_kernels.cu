@@ -253,12 +253,19 @@ gn_apply_kernel(const T* __restrict__ x, T* __restrict__ out, const T* __restric
 // patch p's fresh moments and (mean, rstd).  counter[0] counts arrivals at the
 // barrier and counter[1] departures; the last block to leave zeroes both.
 
-__device__ __forceinline__ bool grid_barrier(unsigned* count, unsigned total, int* err) {
-  __shared__ int s_ok;
+// Arrive at the grid barrier: once every thread of the block has finished the writes the
+// barrier publishes, one thread counts the block in.  grid_wait() then waits for all blocks;
+// work in between overlaps the wait.
+__device__ __forceinline__ void grid_arrive(unsigned* count) {
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
     atomicAdd(count, 1u);
+  }
+}
+__device__ __forceinline__ bool grid_wait(unsigned* count, unsigned total, int* err) {
+  __shared__ int s_ok;
+  if (threadIdx.x == 0) {
     int ok = 1;
     const long long t0 = clock64();
     while (*reinterpret_cast<volatile unsigned*>(count) < total) {
@@ -300,21 +307,6 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
   const int NI = a.per_image, pi = p % NI;                 // patch within its image
   const bool top_src = o.halo_mode != 0 && pi > 0;         // my first row feeds patch p-1
   const bool bot_src = o.halo_mode != 0 && pi < NI - 1;    // my last row feeds patch p+1
-  // ---- displaced steps: the halo rows are last step's values, final already -- copy
-  // them now, overlapped with the statistics, instead of after the barrier
-  if (o.halo_mode == 2 && pl < PL) {
-    T* outp = static_cast<T*>(o.out);
-    const T* prev = static_cast<const T*>(o.prev_slab);
-    for (int q = pix0 + pl; q < pix1; q += PL) {
-      if (!((top_src && q < o.W) || (bot_src && q >= last_row0))) continue;
-      const uint4 hv = ld_nc16(prev + ((size_t)p * o.out_patch_stride + o.out_off + q) * C + vc * VEC);
-      if (top_src && q < o.W)
-        *reinterpret_cast<uint4*>(outp + ((size_t)(p - 1) * o.out_patch_stride + o.out_off + a.pix_per_patch + q) * C +
-                                  vc * VEC) = hv;
-      if (bot_src && q >= last_row0)
-        *reinterpret_cast<uint4*>(outp + ((size_t)(p + 1) * o.out_patch_stride + (q - last_row0)) * C + vc * VEC) = hv;
-    }
-  }
   // ---- phase 1: per-channel partial sums of this chunk (8 loads in flight)
   {
     float s1[VEC], s2[VEC];
@@ -362,7 +354,36 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
 
   // ---- grid barrier: every chunk partial is written
   const unsigned total = gridDim.x * gridDim.y;
-  if (!grid_barrier(a.counter, total, err)) return;
+  grid_arrive(a.counter);
+  // displaced steps: the halo rows are last step's values, final already -- copy them
+  // while the other blocks reach the barrier (eight 16-byte loads in flight per thread;
+  // only the blocks whose chunk holds a patch's first or last row have any)
+  if (o.halo_mode == 2 && pl < PL && ((top_src && pix0 < o.W) || (bot_src && pix1 > last_row0))) {
+    T* outp = static_cast<T*>(o.out);
+    const T* prev = static_cast<const T*>(o.prev_slab);
+    for (int q0 = pix0 + pl; q0 < pix1; q0 += 8 * PL) {
+      uint4 hv[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int q = q0 + j * PL;
+        const bool need = q < pix1 && ((top_src && q < o.W) || (bot_src && q >= last_row0));
+        hv[j] = need ? ld_nc16(prev + ((size_t)p * o.out_patch_stride + o.out_off + q) * C + vc * VEC)
+                     : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int q = q0 + j * PL;
+        if (q >= pix1) break;
+        if (top_src && q < o.W)   // bottom halo row (slab row R+1) of patch p-1
+          *reinterpret_cast<uint4*>(outp + ((size_t)(p - 1) * o.out_patch_stride + o.out_off + a.pix_per_patch + q) *
+                                               C + vc * VEC) = hv[j];
+        if (bot_src && q >= last_row0)   // top halo row (slab row 0) of patch p+1
+          *reinterpret_cast<uint4*>(outp + ((size_t)(p + 1) * o.out_patch_stride + (q - last_row0)) * C + vc * VEC) =
+              hv[j];
+      }
+    }
+  }
+  if (!grid_wait(a.counter, total, err)) return;
 
   // ---- phase 2: fresh moments of the patches needed, in a fixed order
   const bool all = a.is_sync && !a.naive;       // sync steps merge the image's fresh moments
@@ -374,10 +395,15 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
     const int item = tid % items, part_id = tid / items;
     const int pp = p_lo + item / G, gg = item % G;
     const float2* src = reinterpret_cast<const float2*>(a.part) + (size_t)pp * n_chunks * G + gg;
+    // chunks part_id, part_id + S, ... summed in that order, eight loads in flight (the
+    // zeros past the end leave the sum unchanged)
     float2 acc = make_float2(0.f, 0.f);
-    for (int c = part_id; c < n_chunks; c += S) {
-      const float2 v = __ldcg(src + (size_t)c * G);
-      acc.x += v.x; acc.y += v.y;
+    for (int c = part_id; c < n_chunks; c += 8 * S) {
+      float2 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = c + u * S < n_chunks ? __ldcg(src + (size_t)(c + u * S) * G) : make_float2(0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) { acc.x += v[u].x; acc.y += v[u].y; }
     }
     red[(part_id * items + item) * 2 + 0] = acc.x;
     red[(part_id * items + item) * 2 + 1] = acc.y;
