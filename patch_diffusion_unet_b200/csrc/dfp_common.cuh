@@ -21,6 +21,7 @@ enum DeviceError : int {
   kErrWaitAttnP = 5,       // MMA waited too long for P
   kErrWaitAttnO = 6,       // softmax waited too long for P V
   kErrGridSync = 7,        // a block waited too long at a grid-wide barrier
+  kErrWaitAttnMerge = 8,   // a split query tile's merge waited too long for another piece
 };
 
 // Limit of every spin-wait, in SM clock cycles (about 2 s at the B200's maximum
@@ -294,6 +295,17 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // allow_next_grid() lets the next kernel begin launching; it takes effect once every
 // block of this grid has called it (or exited), so all of this grid's blocks are then
 // resident and the next grid's blocks only take resources this grid no longer needs.
+// Release / acquire flag accesses at GPU scope (a flag published after a block-level
+// barrier makes every write of the barrier's threads visible to an acquiring reader).
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void allow_next_grid() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 

@@ -132,10 +132,12 @@ struct TcAttnArgs {
   int* err;
   int n_qtiles;           // ceil(Lp / 128)
   int ctas;               // persistent CTAs (one per SM); the scratch below is sized for them
-  float* part_o;          // scratch [ctas][2][256][64]: unnormalised O of a cut pair's piece
-  float* part_ml;         // scratch [ctas][2][256][2]:  (running max, row sum) of the same
-  unsigned* counters;     // scratch [ctas][2], zero between launches
+  float* part_o;          // scratch [ctas][256][64]: unnormalised O of the CTA's first piece when
+                          // it continues a pair another CTA started
+  float* part_ml;         // scratch [ctas][256][2]:  (running max, row sum) of the same
+  unsigned* counters;     // scratch [ctas][2]: publish flags of the CTAs' first pieces (zeroed once)
   int total_tiles;        // set by the launcher
+  unsigned epoch;         // set by the launcher: this launch's flag value (never 0, never reused)
   int pdl;                // launch with programmatic stream serialization
 };
 // floats of part_o for `ctas` CTAs (part_ml needs 1/32 of it)

@@ -46,11 +46,14 @@
 // a sequence of pieces (the part of one pair's KV list that falls in the range);
 // Q is double-buffered so the next piece's queries load while the current piece
 // runs, and the K/V ring does not drain between pieces.  A pair whose KV list is
-// cut between CTAs is finished by the last of them to arrive (arrival counter):
-// each piece leaves its unnormalised O, running max and row sum in a per-CTA slot
-// and the last one merges the pieces in KV order, so the result does not depend
-// on timing.
+// cut between CTAs is finished by the CTA holding its first KV tiles (the end of that
+// CTA's range, so processed after the other pieces, which open their CTAs' ranges):
+// the other pieces leave their unnormalised O, running max and row sum in a per-CTA
+// slot and publish a flag; the first piece merges them with its own O in KV order,
+// so the result does not depend on timing.  Only a merging piece ever waits, and only
+// for pieces that wait for nothing: with one resident CTA per SM this cannot cycle.
 #include <algorithm>
+#include <atomic>
 
 #include "dfp_common.cuh"
 #include "kernels.h"
@@ -276,13 +279,18 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
 
 // End of a piece for one softmax group: this thread's half row of O (32 columns)
 // and the row sum, normalised into the output, or -- for a pair cut between CTAs --
-// left as a partial in this CTA's slot, with the last piece to arrive merging all
-// of them in KV order.  O streams through 8-column chunks so the epilogue needs few
-// registers; it is out of line so that none of them count against the KV loop.
-// Returns false if the final P V never completed.
+// merged.  The pieces of a cut pair lie in consecutive CTAs' ranges; the first CTA's
+// piece (the pair's first KV tiles) is the end of that CTA's range, so it is processed
+// last there, after the later pieces, which open their CTAs' ranges.  That CTA merges:
+// the later pieces leave their unnormalised O, running max and row sum in their CTA's
+// slot and publish a flag (a release store of the launch's epoch, no round trip); the
+// first piece waits for the flags (already set, as a rule) and merges in KV order, its
+// own O straight from TMEM.  O streams through 8-column chunks so the epilogue needs
+// few registers; it is out of line so that none of them count against the KV loop.
+// Returns false if the final P V never completed or a merge waited in vain.
 __device__ __noinline__ bool piece_epilogue(const TcAttnArgs& a, const Unit& u, uint32_t tO, uint32_t o_bar,
                                                uint32_t o_parity, float m_used, int g, int half, int row,
-                                               bool group_leader, int c, int X0, int* s_last) {
+                                               bool group_leader, int c) {
   const int TT = a.total_tiles, G = gridDim.x;
   const bool have = mbar_wait(o_bar, o_parity, a.err, kErrWaitAttnO);
   float l = 1.f;
@@ -315,76 +323,96 @@ __device__ __noinline__ bool piece_epilogue(const TcAttnArgs& a, const Unit& u, 
     }
     return have;
   }
-  // this piece's partial result into the CTA's slot (0: its first piece, 1: its last
-  // piece; X0 < U0 means the pair started after this CTA's range did)
-  const size_t slot = (size_t)c * 2 + (X0 < u.U0 ? 1 : 0);
-  const size_t prow = slot * 256 + g * 128 + row;
-  if (have) {
-    float4* po = reinterpret_cast<float4*>(a.part_o + prow * 64 + half * 32);
+  if (c != c_first) {
+    // a later piece: this CTA's first piece, into the CTA's slot
+    const size_t prow = (size_t)c * 256 + g * 128 + row;
+    if (have) {
+      float4* po = reinterpret_cast<float4*>(a.part_o + prow * 64 + half * 32);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      uint32_t r8[8];
-      tmem_ld8(tO + half * 32 + k * 8, r8);
-      tmem_wait_ld();
-      po[2 * k] = make_float4(__uint_as_float(r8[0]), __uint_as_float(r8[1]), __uint_as_float(r8[2]),
-                              __uint_as_float(r8[3]));
-      po[2 * k + 1] = make_float4(__uint_as_float(r8[4]), __uint_as_float(r8[5]), __uint_as_float(r8[6]),
-                                  __uint_as_float(r8[7]));
+      for (int k = 0; k < 4; ++k) {
+        uint32_t r8[8];
+        tmem_ld8(tO + half * 32 + k * 8, r8);
+        tmem_wait_ld();
+        po[2 * k] = make_float4(__uint_as_float(r8[0]), __uint_as_float(r8[1]), __uint_as_float(r8[2]),
+                                __uint_as_float(r8[3]));
+        po[2 * k + 1] = make_float4(__uint_as_float(r8[4]), __uint_as_float(r8[5]), __uint_as_float(r8[6]),
+                                    __uint_as_float(r8[7]));
+      }
+      if (half == 0) reinterpret_cast<float2*>(a.part_ml)[prow] = make_float2(m_used, l);
     }
-    if (half == 0) reinterpret_cast<float2*>(a.part_ml)[prow] = make_float2(m_used, l);
+    // publish: the group barrier orders every thread's partial stores before the
+    // leader's release store of the flag
+    named_bar(2 + g, 256);
+    if (group_leader) st_release_gpu(a.counters + 2 * c + g, a.epoch);
+    return have;
   }
-  // publish: the group barrier orders every thread's partial stores before the leader's
-  // fence, and the fence orders them before the arrival count (cumulativity)
-  named_bar(2 + g, 256);
+  // the first piece: wait for the later pieces' flags (bounded), then merge
+  int failed = 0;
   if (group_leader) {
-    __threadfence();
-    const bool last = atomicAdd(a.counters + 2 * c_first + g, 1u) == (unsigned)(npieces - 1);
-    if (last) __threadfence();   // acquire: the other pieces' partials before the group reads them
-    *s_last = last;
-  }
-  named_bar(2 + g, 256);
-  if (*s_last) {
-    if (row_ok) {
-      // This path runs at most twice per CTA: it is kept small (rolled loops, few registers)
-      // so that it costs the KV loop nothing.  First the pieces' running maxima and row sums,
-      // then 8 columns at a time, every piece's contribution in KV order.
-      float mm = -INFINITY;
-#pragma unroll 1
-      for (int k = 0; k < npieces; ++k) {
-        const int ck = c_first + k;
-        const size_t sr = ((size_t)ck * 2 + (range_start(ck, TT, G) < u.U0 ? 1 : 0)) * 256 + g * 128 + row;
-        mm = fmaxf(mm, __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr).x);
-      }
-      float lsum = 0.f;
-#pragma unroll 1
-      for (int k = 0; k < npieces; ++k) {
-        const int ck = c_first + k;
-        const size_t sr = ((size_t)ck * 2 + (range_start(ck, TT, G) < u.U0 ? 1 : 0)) * 256 + g * 128 + row;
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr);
-        lsum = fmaf(ml.y, ex2_mufu(ml.x - mm), lsum);
-      }
-      const float inv = 1.f / lsum;
-#pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        float w8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-        for (int k = 0; k < npieces; ++k) {
-          const int ck = c_first + k;
-          const size_t sr = ((size_t)ck * 2 + (range_start(ck, TT, G) < u.U0 ? 1 : 0)) * 256 + g * 128 + row;
-          const float w = ex2_mufu(__ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr).x - mm) * inv;
-          const float4* po = reinterpret_cast<const float4*>(a.part_o + sr * 64 + half * 32) + 2 * q;
-          const float4 v0 = __ldcg(po), v1 = __ldcg(po + 1);
-          w8[0] = fmaf(v0.x, w, w8[0]); w8[1] = fmaf(v0.y, w, w8[1]);
-          w8[2] = fmaf(v0.z, w, w8[2]); w8[3] = fmaf(v0.w, w, w8[3]);
-          w8[4] = fmaf(v1.x, w, w8[4]); w8[5] = fmaf(v1.y, w, w8[5]);
-          w8[6] = fmaf(v1.z, w, w8[6]); w8[7] = fmaf(v1.w, w, w8[7]);
+    for (int k = 1; k < npieces && !failed; ++k) {
+      const unsigned* flag = a.counters + 2 * (c_first + k) + g;
+      const long long t0 = clock64();
+      while (ld_acquire_gpu(flag) != a.epoch) {
+        if (clock64() - t0 > kWaitLimitCycles) {
+          atomicCAS(a.err, 0, kErrWaitAttnMerge);
+          failed = 1;
+          break;
         }
-        out_row[q] = pack16(w8);
+        __nanosleep(32);
       }
     }
-    if (group_leader) a.counters[2 * c_first + g] = 0u;
   }
-  return have;
+  if (named_bar_or(2 + g, 256, failed != 0) || !have) return false;
+  // running maxima and row sums of every piece in KV order (this piece first)
+  float mm = m_used;
+#pragma unroll 1
+  for (int k = 1; k < npieces; ++k) {
+    const size_t sr = (size_t)(c_first + k) * 256 + g * 128 + row;
+    mm = fmaxf(mm, __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr).x);
+  }
+  float lsum = fmaf(l, ex2_mufu(m_used - mm), 0.f);
+#pragma unroll 1
+  for (int k = 1; k < npieces; ++k) {
+    const size_t sr = (size_t)(c_first + k) * 256 + g * 128 + row;
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr);
+    lsum = fmaf(ml.y, ex2_mufu(ml.x - mm), lsum);
+  }
+  const float inv = 1.f / lsum;
+  // this piece's O from TMEM, then each later piece's 32 columns (eight 16-byte loads in
+  // flight), every output element accumulated over the pieces in KV order
+  float acc[4][8];
+  {
+    const float w = ex2_mufu(m_used - mm) * inv;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t r8[8];
+      tmem_ld8(tO + half * 32 + q * 8, r8);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[q][e] = fmaf(__uint_as_float(r8[e]), w, 0.f);
+    }
+  }
+#pragma unroll 1
+  for (int k = 1; k < npieces; ++k) {
+    const size_t sr = (size_t)(c_first + k) * 256 + g * 128 + row;
+    const float w = ex2_mufu(__ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr).x - mm) * inv;
+    const float4* po = reinterpret_cast<const float4*>(a.part_o + sr * 64 + half * 32);
+    float4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __ldcg(po + i);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc[q][0] = fmaf(v[2 * q].x, w, acc[q][0]); acc[q][1] = fmaf(v[2 * q].y, w, acc[q][1]);
+      acc[q][2] = fmaf(v[2 * q].z, w, acc[q][2]); acc[q][3] = fmaf(v[2 * q].w, w, acc[q][3]);
+      acc[q][4] = fmaf(v[2 * q + 1].x, w, acc[q][4]); acc[q][5] = fmaf(v[2 * q + 1].y, w, acc[q][5]);
+      acc[q][6] = fmaf(v[2 * q + 1].z, w, acc[q][6]); acc[q][7] = fmaf(v[2 * q + 1].w, w, acc[q][7]);
+    }
+  }
+  if (row_ok) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) out_row[q] = pack16(acc[q]);
+  }
+  return true;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -410,7 +438,6 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
   uint64_t* mma_drain = o_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
   __shared__ volatile int s_abort;
-  __shared__ int s_last[2];
   __shared__ float s_mrow[2][128];           // [group][row]: running max handed to the piece epilogue
   __shared__ int s_piece[2][8];               // per group: p, head, pair, T, U0, piece start
 
@@ -795,7 +822,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
       Unit u;
       u.p = sp[0]; u.head = sp[1]; u.pair = sp[2]; u.T = sp[3]; u.U0 = sp[4];
       if (!piece_epilogue(a, u, tOe, smem_u32(&o_done[g]), (uint32_t)(gt - 1) & 1u, s_mrow[g][erow], g, h16,
-                          erow, group_leader, c, X0, &s_last[g]))
+                          erow, group_leader, c))
         carry = true;
       // next piece: every thread of the group is done with s_piece (and s_mrow) before it changes
       named_bar(2 + g, 256);
@@ -839,7 +866,7 @@ long long attention_total_tiles(const TcAttnArgs& a) {
   return tt * a.images;
 }
 
-size_t attention_scratch_floats(int ctas) { return (size_t)ctas * 2 * 256 * 64; }
+size_t attention_scratch_floats(int ctas) { return (size_t)ctas * 256 * 64; }
 
 cudaError_t launch_tc_attention(const TcAttnArgs& args, const CUtensorMap& mq, const CUtensorMap& mkf,
                                 const CUtensorMap& mvf, const CUtensorMap& mks,
@@ -859,6 +886,9 @@ cudaError_t launch_tc_attention(const TcAttnArgs& args, const CUtensorMap& mq, c
   if (regs * kThreads < 128 * kRegsTmaMma + 512 * kRegsSoftmax) return cudaErrorInvalidConfiguration;
   TcAttnArgs a = args;
   if (a.images < 1 || a.kv_stride < 0) return cudaErrorInvalidValue;
+  // a fresh flag value per launch (flags hold the epoch of the launch that last set them)
+  static std::atomic<unsigned> epoch{0};
+  do a.epoch = ++epoch; while (a.epoch == 0);
   const long long tt = attention_total_tiles(a);
   if (tt <= 0) return cudaSuccess;
   const int G = (int)std::min<long long>(a.ctas, tt);
