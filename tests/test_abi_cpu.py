@@ -74,4 +74,8 @@ def test_null_arguments():
     assert L.dfp_step(None, None, 0, 1) == dfp.E_ARG
     assert L.dfp_check_device(None) == dfp.E_ARG
     assert L.dfp_launches_per_step(None) == -1
+    assert L.dfp_set_launch_overlap(None, 1) == dfp.E_ARG
+    assert L.dfp_set_kernel_family(None, 0) == dfp.E_ARG
+    assert L.dfp_synchronize(None) == dfp.E_ARG
+    assert L.dfp_step_host_async(None, None, None, 0, 1) == dfp.E_ARG
     assert isinstance(L.dfp_last_error(None), bytes)
