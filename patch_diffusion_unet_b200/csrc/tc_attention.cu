@@ -290,7 +290,8 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
 // Returns false if the final P V never completed or a merge waited in vain.
 __device__ __noinline__ bool piece_epilogue(const TcAttnArgs& a, const Unit& u, uint32_t tO, uint32_t o_bar,
                                                uint32_t o_parity, float m_used, int g, int half, int row,
-                                               bool group_leader, int c) {
+                                               int c, uint32_t pub_bar, uint32_t mrg_bar,
+                                               const volatile int* merge_fail) {
   const int TT = a.total_tiles, G = gridDim.x;
   const bool have = mbar_wait(o_bar, o_parity, a.err, kErrWaitAttnO);
   float l = 1.f;
@@ -340,39 +341,35 @@ __device__ __noinline__ bool piece_epilogue(const TcAttnArgs& a, const Unit& u, 
       }
       if (half == 0) reinterpret_cast<float2*>(a.part_ml)[prow] = make_float2(m_used, l);
     }
-    // publish: the group barrier orders every thread's partial stores before the
-    // leader's release store of the flag
-    named_bar(2 + g, 256);
-    if (group_leader) st_release_gpu(a.counters + 2 * c + g, a.epoch);
+    // publish: every thread's arrival (release, CTA scope) hands its partial stores to the
+    // publisher warp, which releases the flag at GPU scope -- the group does not wait
+    mbar_arrive(pub_bar);
     return have;
   }
-  // the first piece: wait for the later pieces' flags (bounded), then merge
-  int failed = 0;
-  if (group_leader) {
-    for (int k = 1; k < npieces && !failed; ++k) {
-      const unsigned* flag = a.counters + 2 * (c_first + k) + g;
-      const long long t0 = clock64();
-      while (ld_acquire_gpu(flag) != a.epoch) {
-        if (clock64() - t0 > kWaitLimitCycles) {
-          atomicCAS(a.err, 0, kErrWaitAttnMerge);
-          failed = 1;
-          break;
-        }
-        __nanosleep(32);
-      }
-    }
+  // the first piece: the flag warp has acquired the later pieces' flags (normally set long
+  // before) and lets the groups in; then merge
+  const bool flags_ok = mbar_wait(mrg_bar, 0, a.err, kErrWaitAttnMerge) && *merge_fail == 0;
+  if (!flags_ok || !have) return false;
+  // running maxima and row sums of every piece in KV order (this piece first); the second
+  // piece's statistics and partial O are loaded together (one round trip for two pieces)
+  const size_t sr1 = (size_t)(c_first + 1) * 256 + g * 128 + row;
+  const float2 ml1 = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr1);
+  float4 v1[8];
+  {
+    const float4* po = reinterpret_cast<const float4*>(a.part_o + sr1 * 64 + half * 32);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v1[i] = __ldcg(po + i);
   }
-  if (named_bar_or(2 + g, 256, failed != 0) || !have) return false;
-  // running maxima and row sums of every piece in KV order (this piece first)
-  float mm = m_used;
+  float mm = fmaxf(m_used, ml1.x);
 #pragma unroll 1
-  for (int k = 1; k < npieces; ++k) {
+  for (int k = 2; k < npieces; ++k) {
     const size_t sr = (size_t)(c_first + k) * 256 + g * 128 + row;
     mm = fmaxf(mm, __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr).x);
   }
   float lsum = fmaf(l, ex2_mufu(m_used - mm), 0.f);
+  lsum = fmaf(ml1.y, ex2_mufu(ml1.x - mm), lsum);
 #pragma unroll 1
-  for (int k = 1; k < npieces; ++k) {
+  for (int k = 2; k < npieces; ++k) {
     const size_t sr = (size_t)(c_first + k) * 256 + g * 128 + row;
     const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr);
     lsum = fmaf(ml.y, ex2_mufu(ml.x - mm), lsum);
@@ -392,8 +389,18 @@ __device__ __noinline__ bool piece_epilogue(const TcAttnArgs& a, const Unit& u, 
       for (int e = 0; e < 8; ++e) acc[q][e] = fmaf(__uint_as_float(r8[e]), w, 0.f);
     }
   }
+  {
+    const float w = ex2_mufu(ml1.x - mm) * inv;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc[q][0] = fmaf(v1[2 * q].x, w, acc[q][0]); acc[q][1] = fmaf(v1[2 * q].y, w, acc[q][1]);
+      acc[q][2] = fmaf(v1[2 * q].z, w, acc[q][2]); acc[q][3] = fmaf(v1[2 * q].w, w, acc[q][3]);
+      acc[q][4] = fmaf(v1[2 * q + 1].x, w, acc[q][4]); acc[q][5] = fmaf(v1[2 * q + 1].y, w, acc[q][5]);
+      acc[q][6] = fmaf(v1[2 * q + 1].z, w, acc[q][6]); acc[q][7] = fmaf(v1[2 * q + 1].w, w, acc[q][7]);
+    }
+  }
 #pragma unroll 1
-  for (int k = 1; k < npieces; ++k) {
+  for (int k = 2; k < npieces; ++k) {
     const size_t sr = (size_t)(c_first + k) * 256 + g * 128 + row;
     const float w = ex2_mufu(__ldcg(reinterpret_cast<const float2*>(a.part_ml) + sr).x - mm) * inv;
     const float4* po = reinterpret_cast<const float4*>(a.part_o + sr * 64 + half * 32);
@@ -440,6 +447,9 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
   __shared__ volatile int s_abort;
   __shared__ float s_mrow[2][128];           // [group][row]: running max handed to the piece epilogue
   __shared__ int s_piece[2][8];               // per group: p, head, pair, T, U0, piece start
+  __shared__ __align__(8) uint64_t s_pub[2];   // [group]: the partial of the CTA's first piece is written
+  __shared__ __align__(8) uint64_t s_mrg;      // the later pieces of the pair this CTA merges are published
+  __shared__ volatile int s_merge_fail;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, c = blockIdx.x;
@@ -464,6 +474,10 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
       mbar_init(smem_u32(&o_done[g]), 1);
     }
     mbar_init(smem_u32(mma_drain), 1);
+    mbar_init(smem_u32(&s_pub[0]), 256);
+    mbar_init(smem_u32(&s_pub[1]), 256);
+    mbar_init(smem_u32(&s_mrg), 1);
+    s_merge_fail = 0;
     fence_mbar_init();
   }
   {
@@ -673,6 +687,43 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
     if (leader) umma_commit(smem_u32(mma_drain));
     __syncwarp();
     mbar_wait(smem_u32(mma_drain), 0, err, kErrWaitAccum);
+   } else if (warp == kWarpMma + 1) {
+    // ------------------------------------------------------------ publisher
+    // The CTA's first piece continues a pair an earlier CTA started: once a group has
+    // written its partial (its 256 threads arrived on s_pub[g], release at CTA scope),
+    // release the group's flag at GPU scope for the merging CTA.
+    const Unit u0 = locate(a, n_pairs, X0);
+    const int cf = cta_of(u0.U0, TT, G), np = cta_of(u0.U0 + u0.T - 1, TT, G) - cf + 1;
+    if (NT > 0 && np > 1 && c != cf && leader) {
+      for (int g = 0; g < 2; ++g)
+        if (mbar_wait(smem_u32(&s_pub[g]), 0, err, kErrWaitAttnMerge)) st_release_gpu(a.counters + 2 * c + g, a.epoch);
+    }
+    __syncwarp();
+   } else if (warp == kWarpMma + 2) {
+    // ------------------------------------------------------------ merge flags
+    // The CTA's last piece holds the first KV tiles of a cut pair: acquire the later
+    // pieces' flags of both groups while the CTA works, then let the groups merge.
+    const Unit ul = locate(a, n_pairs, X1 - 1);
+    const int cf = cta_of(ul.U0, TT, G), np = cta_of(ul.U0 + ul.T - 1, TT, G) - cf + 1;
+    if (NT > 0 && np > 1 && c == cf && leader) {
+      int failed = 0;
+      for (int k = 1; k < np && !failed; ++k)
+        for (int g = 0; g < 2 && !failed; ++g) {
+          const unsigned* flag = a.counters + 2 * (cf + k) + g;
+          const long long t0 = clock64();
+          while (ld_acquire_gpu(flag) != a.epoch) {
+            if (clock64() - t0 > kWaitLimitCycles) {
+              atomicCAS(err, 0, kErrWaitAttnMerge);
+              failed = 1;
+              break;
+            }
+            __nanosleep(256);
+          }
+        }
+      s_merge_fail = failed;
+      mbar_arrive(smem_u32(&s_mrg));
+    }
+    __syncwarp();
    }
   } else {
     // ------------------------------------------------------------ softmax groups (warps 0..15)
@@ -822,7 +873,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
       Unit u;
       u.p = sp[0]; u.head = sp[1]; u.pair = sp[2]; u.T = sp[3]; u.U0 = sp[4];
       if (!piece_epilogue(a, u, tOe, smem_u32(&o_done[g]), (uint32_t)(gt - 1) & 1u, s_mrow[g][erow], g, h16,
-                          erow, group_leader, c))
+                          erow, c, smem_u32(&s_pub[g]), smem_u32(&s_mrg), &s_merge_fail))
         carry = true;
       // next piece: every thread of the group is done with s_piece (and s_mrow) before it changes
       named_bar(2 + g, 256);
