@@ -22,7 +22,8 @@
 // 64 the softmax work per tile is large next to the MMAs, and two threads per
 // row double the latency hiding.  In the fifth warpgroup warp 16 issues TMA
 // (the Q-tile pair of each piece into a double buffer, K/V through 3-stage rings
-// shared by the groups) and warp 17 issues the MMAs from one elected lane; this
+// shared by the groups) and warp 17 issues the MMAs from one elected lane; warps 18
+// and 19 publish and acquire the flags of cut query-tile pairs (below); this
 // warpgroup hands most of its registers to the softmax warpgroups (setmaxnreg).
 // Per KV tile j and group g:
 //   S_g = Q_g K_j^T            tcgen05.mma, A and B from shared memory, D in TMEM
@@ -499,7 +500,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
   allow_next_grid();
 
   if (warp >= kWarpTma) {
-   // Register split: this warpgroup (TMA, MMA and two idle warps) gives registers to
+   // Register split: this warpgroup (TMA, MMA, publisher and flag warps) gives registers to
    // the four softmax warpgroups (the launcher checks the launch's total covers it).
    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsTmaMma) : "memory");
    // Both warps walk their loops with all lanes (addresses and descriptors stay
