@@ -183,8 +183,9 @@ DFP_API dfp_status dfp_copy_out(dfp_handle h, const char* name, void* dst, long 
 DFP_API dfp_status dfp_buffer_bytes(dfp_handle h, const char* name, long long* bytes);
 
 /* Wait for the stream and read the device error flag that bounded waits inside
- * the kernels set instead of hanging.  DFP_OK if clean, DFP_E_DEVICE (flag is
- * cleared) otherwise, DFP_E_CUDA if a launch failed asynchronously. */
+ * the kernels set instead of hanging.  DFP_OK if clean, DFP_E_DEVICE otherwise (the
+ * flag is cleared and the GroupNorm grid-barrier counters are re-armed, so further
+ * steps run normally), DFP_E_CUDA if a launch failed asynchronously. */
 DFP_API dfp_status dfp_check_device(dfp_handle h);
 
 /* Number of kernel launches one dfp_step of this handle enqueues. */

@@ -515,7 +515,10 @@ dfp_status dfp_check_device(dfp_handle h) {
   e = cudaMemcpy(&flag, h->dev_err, sizeof(int), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return h->cuda_fail(e, "error flag read");
   if (flag != 0) {
+    // a kernel that gave up left its grid-barrier counters mid-count: re-arm them (no kernel
+    // is in flight after the synchronize above) so the next step starts clean
     cudaMemset(h->dev_err, 0, sizeof(int));
+    cudaMemset(h->counter, 0, 64);
     return h->fail(DFP_E_DEVICE, "a kernel wait ran past its limit (device error code " + std::to_string(flag) + ")");
   }
   return DFP_OK;
