@@ -52,7 +52,7 @@ typedef enum {
   DFP_E_STATE = 2,        /* call out of order (e.g. displaced step, empty cache) */
   DFP_E_CUDA = 3,         /* a CUDA runtime/driver call or a kernel launch failed */
   DFP_E_NOMEM = 4,        /* device or host allocation failed                     */
-  DFP_E_UNSUPPORTED = 5,  /* valid request this build does not implement          */
+  DFP_E_UNSUPPORTED = 5,  /* valid request the library does not implement         */
   DFP_E_DEVICE = 6        /* a kernel reported an error through the device flag   */
 } dfp_status;
 

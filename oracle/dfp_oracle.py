@@ -29,7 +29,7 @@ Sources are web pages about DistriFusion (CVPR 2024):
 * GroupNorm defaults to a "corrected asynchronous" mode ([README] Benchmarks,
   ``--sync_mode`` flag).  The pages name the mode but print no formula.
 
-Readings adopted where the pages are silent (each also listed in the design doc):
+Readings adopted where the pages are silent:
   R1  conv3x3 context: the one row above / below a patch comes from the
       previous step's conv-input map on displaced steps, from the current map
       on synchronous steps; zero outside the image; zero padding left/right.
@@ -46,6 +46,10 @@ Readings adopted where the pages are silent (each also listed in the design doc):
   R6  "naive" context (the pages' naive-patch baseline, [README] Overview (b);
       [CSDN] Baselines): no cross-patch context at all -- zero halo rows,
       patch-local GroupNorm moments, attention within the patch only.
+  R7  guidance batch (classifier-free guidance at scale 5, [CSDN] Implementation
+      details; [README] Benchmarks, --no_split_batch): each image of a batch is
+      its own displaced-patch step -- own GroupNorm statistics, halo rows, K/V
+      and text context -- sharing only the weights and the step schedule.
 """
 import numpy as np
 
