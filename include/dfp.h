@@ -191,6 +191,19 @@ DFP_API dfp_status dfp_check_device(dfp_handle h);
 /* Number of kernel launches one dfp_step of this handle enqueues. */
 DFP_API int dfp_launches_per_step(dfp_handle h);
 
+/* Host-side check of the tensor-core attention's work split (no counterpart in the
+ * pages; no GPU needed).  Walks the list of (image, patch, head, query-tile pair, KV tile)
+ * units as the kernel does, cut into `ctas` contiguous ranges, and checks: every range is
+ * non-empty and its pieces stay inside their units; every unit is covered once; a pair
+ * cut between CTAs has its first KV tiles at the end of one CTA's range (that CTA merges)
+ * and its other pieces each at the start of a range; the kernel's publisher and flag
+ * warps predict exactly those pieces.  L tokens per image in n_patches patches of Lp
+ * tokens; mode 0 sync, 1 displaced, 2 naive, 3 cross-attention (Lp = L, n_patches = 1,
+ * kv_len context tokens).  Returns 0 if every property holds, else the number of the
+ * first that fails (1: bad arguments). */
+DFP_API int dfp_attention_schedule_check(int L, int Lp, int n_patches, int heads, int mode, int kv_len, int images,
+                                         int ctas);
+
 /* Launch overlap between the kernels of a step (no counterpart in the pages; on by
  * default): every tensor-core-family kernel is launched with programmatic stream
  * serialization, so its blocks are scheduled, and set up their barriers and tensor

@@ -526,6 +526,12 @@ dfp_status dfp_check_device(dfp_handle h) {
 
 int dfp_launches_per_step(dfp_handle h) { return h ? h->launches : -1; }
 
+int dfp_attention_schedule_check(int L, int Lp, int n_patches, int heads, int mode, int kv_len, int images,
+                                 int ctas) {
+  if (mode < kAttnSync || mode > kAttnCross) return 1;
+  return attention_schedule_check(L, Lp, n_patches, heads, mode, kv_len, images, ctas);
+}
+
 dfp_status dfp_set_launch_overlap(dfp_handle h, int enable) {
   if (!h) return DFP_E_ARG;
   if (enable != 0 && enable != 1) return h->fail(DFP_E_ARG, "enable must be 0 or 1");

@@ -142,6 +142,8 @@ struct TcAttnArgs {
 };
 // floats of part_o for `ctas` CTAs (part_ml needs 1/32 of it)
 size_t attention_scratch_floats(int ctas);
+// Host walk of the attention work split over `ctas` CTAs (0: every property holds)
+int attention_schedule_check(int L, int Lp, int N, int heads, int mode, int kv_len, int images, int ctas);
 int sm_count();
 // V operand of the attention: [heads][rows][64] bf16 (rows a multiple of 4, every KV tile
 // starting at a multiple of 4) seen as a 5-D view whose 128-row box lands in shared memory

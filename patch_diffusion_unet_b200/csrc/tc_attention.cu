@@ -55,6 +55,7 @@
 // for pieces that wait for nothing: with one resident CTA per SM this cannot cycle.
 #include <algorithm>
 #include <atomic>
+#include <vector>
 
 #include "dfp_common.cuh"
 #include "kernels.h"
@@ -125,7 +126,7 @@ __device__ __forceinline__ void tile_src(int mode, int p, int Lp, int L, int kv_
 struct Unit {
   int p, head, pair, T, U0;   // p: patch over the batch (img * N + patch within the image)
 };
-__device__ __forceinline__ Unit locate(const TcAttnArgs& a, int n_pairs, int x) {
+__host__ __device__ __forceinline__ Unit locate(const TcAttnArgs& a, int n_pairs, int x) {
   int base = 0;
   Unit u{};
   for (int p = 0; p < a.N * a.images; ++p) {
@@ -142,7 +143,7 @@ __device__ __forceinline__ Unit locate(const TcAttnArgs& a, int n_pairs, int x) 
   return u;   // not reached for x < total
 }
 // the unit after u in the list (no division: pairs, then heads, then patches)
-__device__ __forceinline__ void advance(const TcAttnArgs& a, int n_pairs, Unit& u) {
+__host__ __device__ __forceinline__ void advance(const TcAttnArgs& a, int n_pairs, Unit& u) {
   u.U0 += u.T;
   if (++u.pair == n_pairs) {
     u.pair = 0;
@@ -154,8 +155,8 @@ __device__ __forceinline__ void advance(const TcAttnArgs& a, int n_pairs, Unit& 
   }
 }
 // the CTA whose range [c*TT/G, (c+1)*TT/G) holds global tile x
-__device__ __forceinline__ int cta_of(int x, int TT, int G) { return ((x + 1) * G + TT - 1) / TT - 1; }
-__device__ __forceinline__ int range_start(int c, int TT, int G) { return c * TT / G; }
+__host__ __device__ __forceinline__ int cta_of(int x, int TT, int G) { return ((x + 1) * G + TT - 1) / TT - 1; }
+__host__ __device__ __forceinline__ int range_start(int c, int TT, int G) { return c * TT / G; }
 
 __device__ __forceinline__ float ex2_mufu(float x) {
   float y;
@@ -957,6 +958,59 @@ cudaError_t launch_tc_attention(const TcAttnArgs& args, const CUtensorMap& mq, c
   cfg.attrs = attr;
   cfg.numAttrs = a.pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, tc_attention_kernel, mq, mkf, mvf, mks, mvs, a);
+}
+
+// Host walk of the work split exactly as the kernel's three walkers do it (the same
+// locate / advance / cta_of / range_start), checking what the cut-pair merge relies on.
+int attention_schedule_check(int L, int Lp, int N, int heads, int mode, int kv_len, int images, int ctas) {
+  TcAttnArgs a{};
+  a.L = L; a.Lp = Lp; a.N = N; a.heads = heads; a.mode = mode; a.kv_len = kv_len; a.images = images;
+  a.n_qtiles = cdiv(Lp, kTile);
+  if (L <= 0 || Lp <= 0 || N <= 0 || heads <= 0 || images < 1 || ctas < 1) return 1;
+  const int n_pairs = (a.n_qtiles + 1) / 2;
+  const long long tt = attention_total_tiles(a);
+  if (tt <= 0) return 1;
+  const int G = (int)std::min<long long>(ctas, tt);
+  if (tt * G >= (1ll << 31)) return 2;
+  const int TT = (int)tt;
+  std::vector<int> cover(TT, 0);   // tiles of the unit starting at index U0, summed over pieces
+  for (int c = 0; c < G; ++c) {
+    const int X0 = range_start(c, TT, G), X1 = range_start(c + 1, TT, G);
+    if (X1 <= X0) return 3;                         // every CTA has work
+    // what the publisher and flag warps conclude from the range's ends
+    const Unit u0 = locate(a, n_pairs, X0), ul = locate(a, n_pairs, X1 - 1);
+    const int cf0 = cta_of(u0.U0, TT, G), np0 = cta_of(u0.U0 + u0.T - 1, TT, G) - cf0 + 1;
+    const int cfl = cta_of(ul.U0, TT, G), npl = cta_of(ul.U0 + ul.T - 1, TT, G) - cfl + 1;
+    const int expect_publish = np0 > 1 && c != cf0, expect_merge = npl > 1 && c == cfl;
+    int publishes = 0, merges = 0;
+    Unit u = u0;
+    for (int x = X0; x < X1;) {
+      if (!(u.U0 <= x && x < u.U0 + u.T)) return 4;   // the walk stays inside its unit
+      const int x_end = std::min(u.U0 + u.T, X1);
+      cover[u.U0] += x_end - x;
+      const int cf = cta_of(u.U0, TT, G), np = cta_of(u.U0 + u.T - 1, TT, G) - cf + 1;
+      if (c < cf || c >= cf + np) return 5;           // this CTA holds part of the unit
+      if (np > 1) {
+        if (c == cf) {                                 // the first KV tiles end the range
+          if (x_end != X1) return 6;
+          ++merges;
+        } else {                                       // a later piece opens the range
+          if (x != X0) return 7;
+          ++publishes;
+        }
+      }
+      x = x_end;
+      if (x < X1) advance(a, n_pairs, u);
+    }
+    if (publishes != expect_publish || merges != expect_merge) return 8;
+  }
+  // every unit covered exactly once, whole
+  Unit v = locate(a, n_pairs, 0);
+  for (int x = 0; x < TT; x += v.T, advance(a, n_pairs, v)) {
+    if (v.U0 != x || v.T <= 0) return 9;
+    if (cover[x] != v.T) return 10;
+  }
+  return 0;
 }
 
 }  // namespace dfp

@@ -24,7 +24,7 @@ EXPORTED = ("dfp_create", "dfp_load_weights", "dfp_step", "dfp_step_host", "dfp_
             "dfp_copy_out", "dfp_buffer_bytes", "dfp_check_device", "dfp_launches_per_step",
             "dfp_set_kernel_family", "dfp_set_profiling", "dfp_kernel_times", "dfp_destroy",
             "dfp_last_error", "dfp_group_norm_noalloc", "dfp_group_norm_noalloc_error",
-            "dfp_selftest_wait_timeout", "dfp_set_launch_overlap")
+            "dfp_selftest_wait_timeout", "dfp_set_launch_overlap", "dfp_attention_schedule_check")
 
 
 class Config(ctypes.Structure):
@@ -62,6 +62,7 @@ def load_library(path=_LIB_PATH):
         "dfp_launches_per_step": ([H], ctypes.c_int),
         "dfp_set_kernel_family": ([H, ctypes.c_int], ctypes.c_int),
         "dfp_set_launch_overlap": ([H, ctypes.c_int], ctypes.c_int),
+        "dfp_attention_schedule_check": ([ctypes.c_int] * 8, ctypes.c_int),
         "dfp_set_profiling": ([H, ctypes.c_int], ctypes.c_int),
         "dfp_kernel_times": ([H, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_char_p), ctypes.c_int],
                              ctypes.c_int),
