@@ -235,8 +235,8 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
   ok &= h->alloc(&h->q, map);
   ok &= h->alloc(&h->o, map);
   ok &= h->alloc(&h->xin, map);
-  ok &= h->alloc((void**)&h->dbg1, N * G * 2 * 4);
-  ok &= h->alloc((void**)&h->dbg2, N * G * 2 * 4);
+  ok &= h->alloc((void**)&h->mr1, N * G * 2 * 4);
+  ok &= h->alloc((void**)&h->mr2, N * G * 2 * 4);
   ok &= h->alloc((void**)&h->part, N * (size_t)gn_stats_chunks((int)N, (int)(R * W)) * G * 2 * 4);
   ok &= h->alloc((void**)&h->counter, 64);
   ok &= h->alloc((void**)&h->dev_err, 64);
@@ -246,7 +246,7 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
     const size_t f = attention_scratch_floats(h->attn_ctas);
     ok &= h->alloc((void**)&h->attn_part_o, f * 4);
     ok &= h->alloc((void**)&h->attn_part_ml, f / 32 * 4);
-    ok &= h->alloc((void**)&h->attn_counters, (size_t)h->attn_ctas * 2 * 4 + 64);
+    ok &= h->alloc((void**)&h->attn_flags, (size_t)h->attn_ctas * 2 * 4 + 64);
   }
   if (!ok) {
     g_create_error = "device allocation failed";
@@ -266,7 +266,7 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
     if (e == cudaSuccess) e = cudaMemset(p, 0, map);
   if (e == cudaSuccess) e = cudaMemset(h->counter, 0, 64);
   if (e == cudaSuccess) e = cudaMemset(h->dev_err, 0, 64);
-  if (e == cudaSuccess && h->attn_counters) e = cudaMemset(h->attn_counters, 0, (size_t)h->attn_ctas * 2 * 4 + 64);
+  if (e == cudaSuccess && h->attn_flags) e = cudaMemset(h->attn_flags, 0, (size_t)h->attn_ctas * 2 * 4 + 64);
   if (e != cudaSuccess) {
     g_create_error = std::string("cudaMemset: ") + cudaGetErrorString(e);
     dfp_destroy(h);
@@ -461,7 +461,7 @@ static bool buffer_of(dfp_handle h, const char* name, const void** ptr, long lon
   const std::string n = name;
   if (h->stage) {
     if (stage_buffer(h, n, ptr, bytes)) return true;
-    if (n == "gn1" || n == "gn2") { *ptr = n == "gn1" ? h->dbg1 : h->dbg2; *bytes = st; return true; }
+    if (n == "gn1" || n == "gn2") { *ptr = n == "gn1" ? h->mr1 : h->mr2; *bytes = st; return true; }
     if (n == "q" || n == "o") { *ptr = n == "q" ? h->q : h->o; *bytes = map; return true; }
     return false;
   }
@@ -472,8 +472,8 @@ static bool buffer_of(dfp_handle h, const char* name, const void** ptr, long lon
   else if (n == "q") { *ptr = h->q; *bytes = map; }
   else if (n == "k") { *ptr = h->kb[cur]; *bytes = map; }
   else if (n == "v") { *ptr = h->vb[cur]; *bytes = map; }
-  else if (n == "gn1") { *ptr = h->dbg1; *bytes = st; }
-  else if (n == "gn2") { *ptr = h->dbg2; *bytes = st; }
+  else if (n == "gn1") { *ptr = h->mr1; *bytes = st; }
+  else if (n == "gn2") { *ptr = h->mr2; *bytes = st; }
   else if (n == "slab") {
     *ptr = h->slab[cur];
     *bytes = (long long)h->B * h->cfg.n_patches * (h->R + 2) * h->cfg.W * h->cfg.C * (long long)h->esz;
@@ -624,7 +624,7 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   g.x = x; g.N = NB; g.per_image = N; g.pix_per_patch = Lp; g.C = C; g.G = G; g.eps = c.gn_eps;
   g.part = h->part; g.counter = h->counter;
   g.fresh_out = h->mom1[cur]; g.stale = h->mom1[prv];
-  g.gamma = h->gn1_g; g.beta = h->gn1_b; g.dbg = h->dbg1;
+  g.gamma = h->gn1_g; g.beta = h->gn1_b; g.mean_rstd = h->mr1;
   g.is_sync = is_sync; g.mode = (int)c.gn_mode; g.naive = naive ? 1 : 0;
   // consecutive tensor-core-family kernels overlap launch and set-up with their
   // predecessor's tail (each waits for the predecessor before touching memory)
@@ -640,7 +640,7 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
     DFP_LAUNCH(launch_gn_fused<T>(g, go, true, h->dev_err, s), "gn1 + SiLU + halo (fused)");
   } else {
     DFP_LAUNCH(launch_gn_stats_merge<T>(g, s), "gn1 statistics");
-    DFP_LAUNCH(launch_gn_apply<T>(x, slab, static_cast<const T*>(h->slab[prv]), h->dbg1, h->gn1_g, h->gn1_b, G, NB, N,
+    DFP_LAUNCH(launch_gn_apply<T>(x, slab, static_cast<const T*>(h->slab[prv]), h->mr1, h->gn1_g, h->gn1_b, G, NB, N,
                                   Lp, C, W, (long long)(R + 2) * W, W, true, halo_mode, s), "gn1 apply + halo");
   }
   // ---- conv3x3 (+ bias) -> h
@@ -654,13 +654,13 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   }
   // ---- GN2 (no SiLU) -> t
   g.x = h->h; g.fresh_out = h->mom2[cur]; g.stale = h->mom2[prv];
-  g.gamma = h->gn2_g; g.beta = h->gn2_b; g.dbg = h->dbg2;
+  g.gamma = h->gn2_g; g.beta = h->gn2_b; g.mean_rstd = h->mr2;
   if (h->family == 0) {
     const GnOut go{h->t, nullptr, (long long)Lp, 0, W, 0};
     DFP_LAUNCH(launch_gn_fused<T>(g, go, false, h->dev_err, s), "gn2 (fused)");
   } else {
     DFP_LAUNCH(launch_gn_stats_merge<T>(g, s), "gn2 statistics");
-    DFP_LAUNCH(launch_gn_apply<T>(static_cast<const T*>(h->h), static_cast<T*>(h->t), nullptr, h->dbg2, h->gn2_g,
+    DFP_LAUNCH(launch_gn_apply<T>(static_cast<const T*>(h->h), static_cast<T*>(h->t), nullptr, h->mr2, h->gn2_g,
                                   h->gn2_b, G, NB, N, Lp, C, W, (long long)Lp, 0, false, 0, s), "gn2 apply");
   }
   // ---- Q, K, V projections; K/V land in this step's cache buffers
@@ -678,7 +678,7 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
     a.L = L; a.Lp = Lp; a.N = N; a.heads = c.heads; a.C = C; a.mode = mode; a.o = h->o; a.err = h->dev_err;
     a.images = B; a.kv_stride = L; a.pdl = pdl;
     a.ctas = h->attn_ctas; a.n_qtiles = (Lp + 127) / 128;
-    a.part_o = h->attn_part_o; a.part_ml = h->attn_part_ml; a.counters = h->attn_counters;
+    a.part_o = h->attn_part_o; a.part_ml = h->attn_part_ml; a.flags = h->attn_flags;
     DFP_LAUNCH(launch_tc_attention(a, h->m_q, h->m_k[cur], h->m_v[cur], h->m_k[prv], h->m_v[prv], s), "attention (tcgen05)");
   } else {
     DFP_LAUNCH(launch_simt_attention<T>(static_cast<const T*>(h->q), static_cast<const T*>(h->kb[cur]),

@@ -161,8 +161,8 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
     }
     const float var = fmaxf(e2 - e1 * e1, 0.f);
     const float rstd = 1.f / sqrtf(var + a.eps);
-    a.dbg[tid * 2] = e1;
-    a.dbg[tid * 2 + 1] = rstd;
+    a.mean_rstd[tid * 2] = e1;
+    a.mean_rstd[tid * 2 + 1] = rstd;
   }
   if (tid == 0) *a.counter = 0u;
 }
@@ -449,8 +449,8 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
     if (chunk == 0) {
       a.fresh_out[(p * G + gg) * 2] = m1;
       a.fresh_out[(p * G + gg) * 2 + 1] = m2;
-      a.dbg[(p * G + gg) * 2] = e1;
-      a.dbg[(p * G + gg) * 2 + 1] = rstd;
+      a.mean_rstd[(p * G + gg) * 2] = e1;
+      a.mean_rstd[(p * G + gg) * 2 + 1] = rstd;
     }
   }
   __syncthreads();

@@ -46,13 +46,13 @@ struct dfp_ctx {
   void* kb[2] = {nullptr, nullptr};
   void* vb[2] = {nullptr, nullptr};
   float *mom1[2] = {nullptr, nullptr}, *mom2[2] = {nullptr, nullptr};
-  float *dbg1 = nullptr, *dbg2 = nullptr, *part = nullptr;   // dbg = (mean, rstd) per (patch, group)
+  float *mr1 = nullptr, *mr2 = nullptr, *part = nullptr;   // mr = (mean, rstd) per (patch, group)
   unsigned* counter = nullptr;
   int* dev_err = nullptr;
   // split-KV attention scratch
   int attn_ctas = 0;
   float *attn_part_o = nullptr, *attn_part_ml = nullptr;
-  unsigned* attn_counters = nullptr;
+  unsigned* attn_flags = nullptr;
   std::vector<void*> allocs;
   int last_step = -1;
   int launches = 0;

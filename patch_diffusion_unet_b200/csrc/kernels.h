@@ -22,7 +22,7 @@ struct GnArgs {
   const float* stale;     // [N][G][2] moments of step t-1 (read on displaced steps)
   const float* gamma;     // [C] fp32
   const float* beta;      // [C] fp32
-  float* dbg;             // [N][G][2] (mean, rstd) used -- read by the apply kernel
+  float* mean_rstd;       // [N][G][2] (mean, rstd) applied -- also read by the separate apply kernel
   int is_sync, mode, naive;
   int pdl;                // fused kernel: launch with programmatic stream serialization
 };
@@ -37,7 +37,7 @@ struct GnOut {
 };
 int gn_stats_chunks(int N, int pix_per_patch);
 // statistics + merge + apply (+SiLU) in one cooperative launch; a.counter needs two
-// zeroed words; a.dbg receives (mean, rstd)
+// zeroed words; a.mean_rstd receives (mean, rstd)
 template <typename T> cudaError_t launch_gn_fused(const GnArgs& a, const GnOut& o, bool silu, int* err, cudaStream_t s);
 template <typename T> cudaError_t launch_gn_stats_merge(const GnArgs& a, cudaStream_t s);
 // halo_mode: 0 none (plain output), 1 sync (fresh neighbour rows), 2 displaced
@@ -135,7 +135,7 @@ struct TcAttnArgs {
   float* part_o;          // scratch [ctas][256][64]: unnormalised O of the CTA's first piece when
                           // it continues a pair another CTA started
   float* part_ml;         // scratch [ctas][256][2]:  (running max, row sum) of the same
-  unsigned* counters;     // scratch [ctas][2]: publish flags of the CTAs' first pieces (zeroed once)
+  unsigned* flags;        // scratch [ctas][2]: publish flags of the CTAs' first pieces (zeroed once)
   int total_tiles;        // set by the launcher
   unsigned epoch;         // set by the launcher: this launch's flag value (never 0, never reused)
   int pdl;                // launch with programmatic stream serialization

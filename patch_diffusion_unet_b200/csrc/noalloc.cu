@@ -110,7 +110,7 @@ extern "C" DFP_API dfp_status dfp_group_norm_noalloc(const void* x, void* y, dfp
   a.fresh_out = fresh_moments; a.stale = stale_moments ? stale_moments : fresh_moments;
   a.gamma = gamma; a.beta = beta;
   float* mr = mean_rstd ? mean_rstd : stats;  // the (mean, rstd) the apply step reads
-  a.dbg = mr;
+  a.mean_rstd = mr;
   a.is_sync = stale_moments ? 0 : 1; a.mode = (int)mode; a.naive = 0;
   if (dtype == DFP_BF16) {
     e = dfp::launch_gn_stats_merge<__nv_bfloat16>(a, s);

@@ -356,7 +356,7 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   g.x = xv; g.N = NB; g.per_image = N; g.pix_per_patch = Lp; g.C = C; g.G = G; g.eps = c.gn_eps;
   g.part = h->part; g.counter = h->counter;
   g.is_sync = is_sync; g.mode = (int)c.gn_mode; g.naive = naive ? 1 : 0;
-  g.fresh_out = st->mom1[cur]; g.stale = st->mom1[prv]; g.gamma = st->n1_g; g.beta = st->n1_b; g.dbg = h->dbg1;
+  g.fresh_out = st->mom1[cur]; g.stale = st->mom1[prv]; g.gamma = st->n1_g; g.beta = st->n1_b; g.mean_rstd = h->mr1;
   {
     const GnOut go{st->slab1[cur], st->slab1[prv], (long long)(R + 2) * W, W, W, halo_mode};
     DFP_LAUNCH(launch_gn_fused<bf>(g, go, true, h->dev_err, s), "norm1 + SiLU + halo (fused)");
@@ -365,7 +365,7 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   ec.kind = 0; ec.out = st->h1; ec.bias = st->b_c1; ec.ldo = C;
   DFP_LAUNCH(launch_tc_gemm(st->p_c1, st->m_slab1[cur], st->m_wc1, ec, h->dev_err, s), "conv1 (tcgen05)");
   g.x = st->h1; g.fresh_out = st->mom2[cur]; g.stale = st->mom2[prv]; g.gamma = st->n2_g; g.beta = st->n2_b;
-  g.dbg = h->dbg2;
+  g.mean_rstd = h->mr2;
   {
     const GnOut go{st->slab2[cur], st->slab2[prv], (long long)(R + 2) * W, W, W, halo_mode};
     DFP_LAUNCH(launch_gn_fused<bf>(g, go, true, h->dev_err, s), "norm2 + SiLU + halo (fused)");
@@ -390,7 +390,7 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
     a.L = L; a.Lp = Lp; a.N = N; a.heads = c.heads; a.C = C; a.mode = sa_mode; a.o = h->o; a.err = h->dev_err;
     a.images = B; a.kv_stride = L; a.pdl = pdl;
     a.n_qtiles = (Lp + 127) / 128; a.ctas = h->attn_ctas;
-    a.part_o = h->attn_part_o; a.part_ml = h->attn_part_ml; a.counters = h->attn_counters;
+    a.part_o = h->attn_part_o; a.part_ml = h->attn_part_ml; a.flags = h->attn_flags;
     DFP_LAUNCH(launch_tc_attention(a, h->m_q, x.m_k[cur], x.m_v[cur], x.m_k[prv], x.m_v[prv], s),
                "self-attention (tcgen05)");
     Epilogue eo{};
@@ -406,7 +406,7 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
     ca.images = B; ca.kv_stride = (int)ctx_rows(c.ctx_len);   // image b reads its own context
     ca.pdl = pdl;
     ca.o = h->o; ca.err = h->dev_err; ca.n_qtiles = (L + 127) / 128; ca.ctas = h->attn_ctas;
-    ca.part_o = h->attn_part_o; ca.part_ml = h->attn_part_ml; ca.counters = h->attn_counters;
+    ca.part_o = h->attn_part_o; ca.part_ml = h->attn_part_ml; ca.flags = h->attn_flags;
     DFP_LAUNCH(launch_tc_attention(ca, h->m_q, x.m_ck, x.m_cv, x.m_ck, x.m_cv, s), "cross-attention (tcgen05)");
     eo.out = r_ca; eo.bias = x.b_o2; eo.residual = r_sa;
     DFP_LAUNCH(launch_tc_gemm(x.p_o2, st->m_o, x.m_wo2, eo, h->dev_err, s), "cross-attn out + residual (tcgen05)");

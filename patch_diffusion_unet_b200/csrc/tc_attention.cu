@@ -698,7 +698,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
     const int cf = cta_of(u0.U0, TT, G), np = cta_of(u0.U0 + u0.T - 1, TT, G) - cf + 1;
     if (NT > 0 && np > 1 && c != cf && leader) {
       for (int g = 0; g < 2; ++g)
-        if (mbar_wait(smem_u32(&s_pub[g]), 0, err, kErrWaitAttnMerge)) st_release_gpu(a.counters + 2 * c + g, a.epoch);
+        if (mbar_wait(smem_u32(&s_pub[g]), 0, err, kErrWaitAttnMerge)) st_release_gpu(a.flags + 2 * c + g, a.epoch);
     }
     __syncwarp();
    } else if (warp == kWarpMma + 2) {
@@ -711,7 +711,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
       int failed = 0;
       for (int k = 1; k < np && !failed; ++k)
         for (int g = 0; g < 2 && !failed; ++g) {
-          const unsigned* flag = a.counters + 2 * (cf + k) + g;
+          const unsigned* flag = a.flags + 2 * (cf + k) + g;
           const long long t0 = clock64();
           while (ld_acquire_gpu(flag) != a.epoch) {
             if (clock64() - t0 > kWaitLimitCycles) {
