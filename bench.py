@@ -1,21 +1,24 @@
 #!/usr/bin/env python
 """Benchmark of the displaced-patch UNet layer step on B200: layer-steps/s and latent px/s.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--batch B] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 3] [--batch B] [--impl ours|reference]
 
 One "step" is one displaced layer step (dfp_step with is_sync = 0) of the
 workload: GN1 statistics + corrected merge, GN1 apply + SiLU, halo refresh,
 conv3x3, GN2 statistics + merge + apply, Q/K/V projection, displaced attention,
-output projection.  The run first executes the synchronous warm-up steps of the
-schedule (untimed), then W displaced warm-up steps, then K timed displaced steps,
-each bracketed by CUDA events on the library's stream; L2 is flushed (a 512 MB
-write) between timed steps, outside the events.  With N > 1 (torchrun) every
-rank runs an independent replica (the layer step does not shard on one GPU
-each: replicas only); value = total steps of all ranks / max over ranks of the
-summed step time.  Rank 0 prints one JSON line.
+output projection.  The default workload is the largest one that fits a GPU:
+the 240x240x640 map of a 3840 px image in 8 row patches.  The run first executes
+the synchronous steps of the schedule (untimed), then exactly W displaced
+warm-up steps, then K timed displaced steps, each bracketed by CUDA events on the
+library's stream; L2 is flushed (a 512 MB write) between timed steps, outside
+the events.  With N > 1 (torchrun) every rank runs an independent replica (the
+layer step does not shard on one GPU each: replicas only); value = total steps
+of all ranks / max over ranks of the summed step time.  Rank 0 prints one JSON
+line.
 
 --impl reference times the CPU oracle (numpy fp64) on the host cores instead:
-the same metric on the same workload, full (unsampled) displaced steps.
+the same metric on the same workload.  Maps up to 64x64 run full steps; on the
+larger maps every oracle step is a bounded sample (see oracle_query_sample).
 
 --batch B runs B images per layer step (the classifier-free-guidance batch, B = 2):
 a step is still one dfp_step, now over B images; "images_per_s" reports
@@ -48,12 +51,13 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--config", type=int, default=3)
     ap.add_argument("--batch", type=int, default=1, help="images per step (2: the guidance batch)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--profile-steps", type=int, default=10)
-    ap.add_argument("--min-warmup-s", type=float, default=1.5,
-                    help="keep warming up until this much wall time has passed (clocks settle)")
+    ap.add_argument("--min-warmup-s", type=float, default=0.0,
+                    help="keep warming up past W steps until this much wall time has passed "
+                         "(the line's \"warmup\" then reports the steps actually run)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-overlap", action="store_true",
@@ -192,22 +196,82 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------- CPU oracle leg
 
-def oracle_displaced_rate(cfg, n_disp=2):
-    """Time the oracle as it stands on full displaced steps of the workload (after one sync step)."""
-    import oracle
+def _oracle_threads():
     try:
         from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
-        threads = os.cpu_count()
+        return os.cpu_count()
+
+
+def oracle_query_sample(cfg, per_patch=32):
+    """Query tokens whose attention the oracle computes in one bounded step.
+
+    Maps up to 64x64 (4096 tokens) run whole steps (None).  On larger maps a whole
+    fp64 step is minutes of CPU work (the 240x240 map's attention alone is 8.5 TFLOP
+    and 33 G exponentials), so each step computes GroupNorm, conv and the Q/K/V
+    projections in full and the attention for `per_patch` evenly spaced query tokens
+    of every patch; oracle_step_seconds adds the time of the skipped queries."""
+    L = cfg["H"] * cfg["W"]
+    if L <= 4096:
+        return None
+    N = cfg["n_patches"]
+    Lp = L // N
+    return np.concatenate([p * Lp + np.linspace(0, Lp - 1, per_patch).round().astype(np.int64) for p in range(N)])
+
+
+def oracle_step_seconds(blk, cfg, x, t, is_sync, sample):
+    """Seconds for one oracle layer step.  With a query sample of n of the L tokens the
+    step runs with attention for those n queries only; the attention of the other L - n
+    queries is accounted by timing the oracle's own softmax_attention on the same n
+    queries (per patch and head, against full-length K/V, as the step calls it) and
+    scaling that time by (L - n) / n."""
+    import oracle
+    t0 = time.perf_counter()
+    blk.step(x, t, is_sync, **({} if sample is None else {"query_tokens": sample}))
+    dt = time.perf_counter() - t0
+    if sample is None:
+        return dt
+    L, heads, N = cfg["H"] * cfg["W"], cfg["heads"], cfg["n_patches"]
+    Lp, n = L // N, len(sample)
+    extra = 0.0
+    for b in getattr(blk, "blocks", [blk]):
+        last = b.attn.last
+        q, k, v = last["q"], last["k"], last["v"]
+        d = q.shape[1] // heads
+        t1 = time.perf_counter()
+        for p in range(N):
+            sel = sample[(sample >= p * Lp) & (sample < (p + 1) * Lp)]
+            for h in range(heads):
+                c = slice(h * d, (h + 1) * d)
+                oracle.softmax_attention(q[sel, c], k[:, c], v[:, c], 1.0 / np.sqrt(d))
+        extra += (time.perf_counter() - t1) * (L - n) / n
+    return dt + extra
+
+
+def oracle_sample_text(cfg, sample):
+    if sample is None:
+        return "full layer steps"
+    L = cfg["H"] * cfg["W"]
+    return (f"bounded steps: GroupNorms, conv and Q/K/V/O projections in full, attention output for "
+            f"{len(sample)} of {L} query tokens ({len(sample) // cfg['n_patches']} evenly spaced per patch); "
+            f"the other queries' attention time added from the oracle's softmax_attention timed on the "
+            f"same queries, scaled by (L - n) / n")
+
+
+def oracle_displaced_rate(cfg, n_disp=2):
+    """Time the oracle as it stands on displaced steps of the workload (after one sync step)."""
+    import oracle
     wl = inputs.SyntheticWorkload(cfg)
     blk = oracle.make_block(cfg, wl.weights, wl.context)
-    blk.step(wl.x(0), 0, 1)
-    t0 = time.perf_counter()
+    sample = oracle_query_sample(cfg)
+    oracle_step_seconds(blk, cfg, wl.x(0), 0, 1, sample)
+    dt = 0.0
+    w0 = time.perf_counter()
     for t in range(1, 1 + n_disp):
-        blk.step(wl.x(t), t, 0)
-    dt = time.perf_counter() - t0
-    return n_disp / dt, threads, dt
+        dt += oracle_step_seconds(blk, cfg, wl.x(t), t, 0, sample)
+    wall = time.perf_counter() - w0
+    return n_disp / dt, _oracle_threads(), wall, sample
 
 
 # ---------------------------------------------------------------------------- main
@@ -239,6 +303,9 @@ def dist_setup():
 
 
 def run_reference(args, cfg):
+    """The reference arm: the oracle on the host cores, rank 0 only, on the same workload,
+    metric and unit; the synchronous steps of the schedule, then W displaced warm-up steps
+    and K timed displaced steps, each bounded as oracle_step_seconds says."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     B = cfg.get("batch", 1)
     if int(os.environ.get("RANK", "0")) != 0:
@@ -246,25 +313,23 @@ def run_reference(args, cfg):
     import oracle
     wl = inputs.SyntheticWorkload(cfg)
     blk = oracle.make_block(cfg, wl.weights, wl.context)
+    sample = oracle_query_sample(cfg)
     n_sync = cfg["n_sync"]
     t = 0
     for t in range(n_sync):
-        blk.step(wl.x(t), t, 1)
+        oracle_step_seconds(blk, cfg, wl.x(t), t, 1, sample)
     for _ in range(args.warmup):
         t += 1
-        blk.step(wl.x(t), t, 0)
-    t0 = time.perf_counter()
+        oracle_step_seconds(blk, cfg, wl.x(t), t, 0, sample)
+    dt = 0.0
     for _ in range(args.steps):
         t += 1
-        blk.step(wl.x(t), t, 0)
-    dt = time.perf_counter() - t0
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        threads = os.cpu_count()
+        dt += oracle_step_seconds(blk, cfg, wl.x(t), t, 0, sample)
+    threads = _oracle_threads()
     value = args.steps / dt
     L = cfg["H"] * cfg["W"]
+    text = f"{args.steps} displaced layer steps after {n_sync} sync and {args.warmup} warm-up steps; " + \
+        oracle_sample_text(cfg, sample)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
@@ -272,8 +337,7 @@ def run_reference(args, cfg):
         "data": "synthetic", "latent_px_per_s": value * L * B, "images_per_s": value * B,
         "config": {"workload": cfg["name"], "H": cfg["H"], "W": cfg["W"], "C": cfg["C"],
                    "n_patches": cfg["n_patches"], "batch": B, "l2": "n/a (CPU)"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": f"{args.steps} full displaced layer steps after {n_sync} sync steps"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": text},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -302,7 +366,8 @@ def main():
     blk.load_weights(dict(wl.weights, context=wl.context) if wl.context is not None else wl.weights)
     blk.set_launch_overlap(not args.no_overlap)
     stream = blk.stream
-    n_pool = 16
+    # a pool of distinct inputs (the steps cycle through it); fewer of the large maps
+    n_pool = 16 if L <= 16384 else 4
     host_x = [inputs.to_torch(wl.x(t), dtype) for t in range(n_pool)]
     xs = [h.cuda() for h in host_x]
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
@@ -314,7 +379,7 @@ def main():
     for t in range(n_sync):
         blk.step(x_of(t), t, 1)
     t = n_sync - 1
-    # warm-up: at least W displaced steps and at least ~1.5 s (clocks settle, sampler sees load)
+    # warm-up: exactly W displaced steps (more only if --min-warmup-s asks for a minimum time)
     gpu_index = os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local] if \
         os.environ.get("CUDA_VISIBLE_DEVICES") else str(local)
     sampler = ClockSampler(gpu_index)
@@ -431,9 +496,10 @@ def main():
     blk.close()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, threads, dt = oracle_displaced_rate(cfg)
+        rate, threads, wall, sample = oracle_displaced_rate(cfg)
         cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"2 full displaced layer steps of {cfg['name']} after 1 sync step ({dt:.1f} s)"}
+               "sample": f"2 displaced layer steps of {cfg['name']} after 1 sync step ({wall:.1f} s wall); " +
+                         oracle_sample_text(cfg, sample)}
 
     if rank == 0:
         ms_step = total_ms_max / args.steps

@@ -106,7 +106,11 @@ typedef struct {
 } dfp_tensor;
 
 /* Create a handle for one layer (or stage) configuration and allocate its device
- * buffers: the double-buffered context caches, intermediates and the output.
+ * buffers: the double-buffered context caches, intermediates and the output.  The
+ * configuration plays the part of the pages' DistriConfig (project README, Usage:
+ * height, width, warmup_steps; Benchmarks: --sync_mode, --parallelism naive_patch),
+ * reduced to one layer: the map size, the patch count, the GroupNorm merge mode and
+ * the context mode; the caller passes which steps are synchronous (dfp_step).
  * cuda_stream: a cudaStream_t (NULL = legacy default stream); all work of this
  * handle is enqueued on it.  *out receives the handle (NULL on failure).
  * Errors: DFP_E_ARG for invalid sizes (see dfp_config), DFP_E_UNSUPPORTED for a
@@ -114,7 +118,11 @@ typedef struct {
 DFP_API dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out);
 
 /* Copy the weights in (host or device source; the library keeps its own re-laid
- * copy, the caller's memory may be freed after the call returns).  Every weight
+ * copy, the caller's memory may be freed after the call returns).  The counterpart of
+ * the pages' from_pretrained (project README, Usage: the SDXL pipeline loads its fp16
+ * weights) for one layer, with the PyTorch module names the wrapped layers keep
+ * (source walkthrough, Patch Parallelism section: DistriConv2dPP, DistriGroupNorm and
+ * DistriSelfAttentionPP replace the UNet's conv, norm and attention modules in place).  Every weight
  * of the block must be named exactly once across calls before the first step;
  * names for DFP_BLOCK_RES_ATTN: gn1.weight gn1.bias conv1.weight conv1.bias
  * gn2.weight gn2.bias attn.to_q.weight attn.to_k.weight attn.to_v.weight
@@ -129,7 +137,12 @@ DFP_API dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_hand
  * Errors: DFP_E_ARG for an unknown name, wrong shape or dtype. */
 DFP_API dfp_status dfp_load_weights(dfp_handle h, const dfp_tensor* w, int n);
 
-/* One layer step.  x: caller-owned device pointer [B, H, W, C] of the config dtype,
+/* One layer step (project README, Overview (c): every patch computes its own rows
+ * fresh and reuses the previous step's activations of the other patches as context;
+ * the first steps are synchronous -- paper reading blog, Implementation details: step 0
+ * plus the warm-up steps; source walkthrough, forward-pass section: split the input
+ * into patches, compute, gather the patch outputs into the full map).
+ * x: caller-owned device pointer [B, H, W, C] of the config dtype,
  * contiguous; it must stay valid until the stream work completes.
  * step: 0 starts a new run and must be synchronous (is_sync = 1); otherwise
  * step must equal the previous step + 1.  is_sync = 1 uses fresh context
@@ -168,8 +181,20 @@ DFP_API dfp_status dfp_synchronize(dfp_handle h);
  * Blocks for the length of the wait.  DFP_E_CUDA if a CUDA call fails. */
 DFP_API dfp_status dfp_selftest_wait_timeout(int* code_out, long long* cycles_out);
 
-/* Library-owned device pointer to the last step's output [B*H*W, C] (config dtype);
- * valid until the next dfp_step or dfp_destroy. */
+/* Self-test of the softmax's polynomial exponential (no counterpart in the pages).  Part of
+ * the attention's exponentials run on the FMA pipe as 2^x = 2^j * p(f), j = rint(x),
+ * |f| <= 1/2, p the degree-3 minimax fit of 2^f in relative error (max 7.48e-5), x clamped
+ * to >= -125.  This call evaluates that same device code: y[i] = 2^x[i] as fp32 and, if
+ * y_bf16 is not NULL, as the truncated bf16 the softmax stores.  x, y: device fp32 [n];
+ * y_bf16: device bf16 [n], 4-byte aligned, or NULL.  Enqueued on cuda_stream (a
+ * cudaStream_t; NULL = legacy default stream).  DFP_E_ARG for n < 0, n > 2^30, NULL x / y
+ * (n > 0) or a misaligned y_bf16; DFP_E_CUDA if the launch fails. */
+DFP_API dfp_status dfp_selftest_exp2_poly(const float* x, float* y, void* y_bf16, int n, void* cuda_stream);
+
+/* Library-owned device pointer to the last step's output [B*H*W, C] (config dtype):
+ * the N patch outputs assembled into the full map, as the wrapped UNet's forward pass
+ * gathers them (source walkthrough, forward-pass section); valid until the next
+ * dfp_step or dfp_destroy. */
 DFP_API dfp_status dfp_output(dfp_handle h, const void** y);
 
 /* Copy an internal buffer of the last step to dst (device or host pointer,
@@ -232,13 +257,21 @@ DFP_API int dfp_kernel_times(dfp_handle h, float* ms, const char** names, int ma
  * allocate device memory when they need the op (a fixed memory pool that bans the
  * CUDA allocator, a pre-planned or capped memory region, a latency-critical host
  * path that must not take allocator locks).
- *   x, y            device [H, W, C] of dtype (input, output; y may not alias x)
+ *   x, y            device [H, W, C] of dtype (input, output; the two ranges must not
+ *                   overlap: the op does not run in place)
  *   gamma, beta     device fp32 [C]
- *   stale_moments   device fp32 [N, G, 2] (E[x], E[x^2]) per (patch, group) of the
- *                   previous step -- pass the previous call's fresh_moments -- or
- *                   NULL for a synchronous step (exact full-map statistics)
- *   fresh_moments   device fp32 [N, G, 2], out: this call's moments
- *   mean_rstd       device fp32 [N, G, 2], out: the (mean, 1/std) applied, or NULL
+ *   stale_moments   device fp32 [N, G, 2] (mean, variance) per (patch, group) of the
+ *                   previous step -- the previous call's fresh_moments -- or NULL for a
+ *                   synchronous step (exact full-map statistics).  It is read after
+ *                   this call's fresh_moments are written, so the two must be distinct
+ *                   buffers: alternate two buffers between consecutive calls
+ *   fresh_moments   device fp32 [N, G, 2], out: this call's moments (mean, variance):
+ *                   the merge rules of dfp_gn_mode are evaluated on these central
+ *                   moments (the same value as on (E[x], E[x^2]) in exact arithmetic,
+ *                   without the fp32 cancellation of E[x^2] - mean^2 at large means)
+ *   mean_rstd       device fp32 [N, G, 2], out: the (mean, 1/std) applied, or NULL;
+ *                   must not overlap the two moment buffers
+ * Overlapping buffers among these return DFP_E_ARG before anything is enqueued.
  *   cuda_stream     cudaStream_t the work is enqueued on (asynchronous)
  * Scratch comes from a fixed 256 KiB array in the library's device memory (held by
  * every GPU that loads the library until exit).  The first call on a device, with

@@ -10,7 +10,7 @@
 //   q           [heads][B*L][64] this step's queries
 //   k[2], v[2]  [heads][B*L][64] keys / values, alternating by step parity
 //   o, y        [B*L][C]         attention output, block output
-//   mom1/2[2]   [B*N][G][2] fp32 per-(patch, group) (E[x], E[x^2]) of GN1 / GN2, alternating
+//   mom1/2[2]   [B*N][G][2] fp32 per-(patch, group) (mean, variance) of GN1 / GN2, alternating
 //   part        fp32 scratch     per-chunk partial sums of the GroupNorm statistics
 #include <cmath>
 #include <cstdio>

@@ -5,7 +5,7 @@
 // DistriGroupNorm ("DistriFusion源码探秘" source walkthrough, Patch Parallelism
 // section, item 3) with the "corrected asynchronous" default of the --sync_mode
 // flag (DistriFusion project README, Benchmarks).  Per (patch p, group g) the
-// step's moments m_p = (E[x], E[x^2]) are merged with the previous step's:
+// step's moments (E[x], E[x^2]) are merged with the previous step's:
 //   sync       est_p = mean_j m_j(t)                      (exact full-map GroupNorm)
 //   corrected  est_p = mean_j m_j(t-1) + (m_p(t) - m_p(t-1))
 //   stale-oth. est_p = (m_p(t) + sum_{j != p} m_j(t-1)) / N
@@ -13,9 +13,23 @@
 //   mean = est.E[x], var = max(est.E[x^2] - mean^2, 0), rstd = 1 / sqrt(var + eps).
 // j runs over the N patches of the same image: a batch of images (the guidance
 // batch) is images x N patches, numbered image-major, with nothing shared across images.
+//
+// Numerics.  In fp32, E[x^2] - mean^2 loses every digit of the variance when the mean
+// is large next to the spread (at mean 30 and unit variance E[x^2] ~ 901 has an ulp of
+// 6e-5).  So the kernels never form E[x^2]: each (patch, group) is summed as x - K with
+// K the patch's first pixel in the group's first channel (one shift for every chunk and
+// channel of the group, so the shifted sums still add across them), and the moments
+// kept per (patch, group) are (mean, variance) = (K + S1/n, S2/n - (S1/n)^2).  Every merge
+// rule above is a mixture of per-patch distributions, and is evaluated in that central
+// form, which is the same value in exact arithmetic without the cancellation:
+//   sync       mean = avg_j m_j, var = avg_j v_j + avg_j (m_j - mean)^2
+//   corrected  with M, V the previous step's moments, d = m_p - M_p, M~ = avg_j M_j:
+//              mean = M~ + d, var = avg_j V_j + (v_p - V_p) + avg_j (M_j - M~)^2 + 2 d (M_p - M~)
+//   stale-oth. the components (m_p, v_p) and (M_j, V_j) for j != p:
+//              mean = avg c, var = avg w + avg (c - mean)^2
 // The reductions are deterministic: per-thread sums in a fixed pixel order, a
-// fixed-order shared-memory tree, and a last-block merge over the chunk partials
-// in a fixed order (no floating-point atomics).
+// fixed-order shared-memory tree, and a merge over the chunk partials in a fixed order
+// (no floating-point atomics).
 #include <algorithm>
 
 #include "dfp_common.cuh"
@@ -33,6 +47,65 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+__device__ __forceinline__ float load_f32(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float load_f32(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+// The shift of (patch p, group g): the patch's first pixel in the group's first channel.
+template <typename T>
+__device__ __forceinline__ float gn_shift(const void* x, int p, int pix_per_patch, int C, int g, int cg) {
+  return load_f32(static_cast<const T*>(x) + (size_t)p * pix_per_patch * C + (size_t)g * cg);
+}
+
+// Shifts of one thread's VEC channels c0 .. c0+VEC-1 (each the shift of its group).
+template <typename T, int VEC>
+__device__ __forceinline__ void gn_thread_shifts(const void* x, int p, int pix_per_patch, int C, int c0, int cg,
+                                                 float (&k)[VEC]) {
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) k[i] = gn_shift<T>(x, p, pix_per_patch, C, (c0 + i) / cg, cg);
+}
+
+// Merge rules of DistriGroupNorm on per-patch (mean, var) moments (see the file header).
+enum GnRule : int { kGnNaive = 0, kGnSync = 1, kGnCorrected = 2, kGnStaleOthers = 3 };
+__device__ __forceinline__ int gn_rule(const GnArgs& a) {
+  return a.naive ? kGnNaive : a.is_sync ? kGnSync : a.mode == 0 ? kGnCorrected : kGnStaleOthers;
+}
+// own: this step's moments of patch pi (of NI in its image); img: moments of the image's
+// patches (this step's for kGnSync, the previous step's otherwise), `stride` float2 apart.
+// Returns (mean, var) of the estimate, var clamped at 0.
+__device__ __forceinline__ float2 gn_estimate(int rule, int NI, int pi, float2 own, const float2* img, int stride) {
+  const float inv = 1.f / (float)NI;
+  float mu, var;
+  if (rule == kGnNaive) {
+    mu = own.x;
+    var = own.y;
+  } else if (rule == kGnCorrected) {
+    float sm = 0.f, sv = 0.f;
+    for (int j = 0; j < NI; ++j) { const float2 q = img[j * stride]; sm += q.x; sv += q.y; }
+    const float mb = sm * inv;
+    float ss = 0.f;
+    for (int j = 0; j < NI; ++j) { const float e = img[j * stride].x - mb; ss = fmaf(e, e, ss); }
+    const float2 st = img[pi * stride];
+    const float d = own.x - st.x;
+    mu = mb + d;
+    var = sv * inv + (own.y - st.y) + ss * inv + 2.f * d * (st.x - mb);
+  } else {
+    // sync: every component is this step's; stale-others: all but patch pi are the previous step's
+    float sm = 0.f, sv = 0.f;
+    for (int j = 0; j < NI; ++j) {
+      const float2 q = (rule == kGnStaleOthers && j == pi) ? own : img[j * stride];
+      sm += q.x; sv += q.y;
+    }
+    mu = sm * inv;
+    float ss = 0.f;
+    for (int j = 0; j < NI; ++j) {
+      const float e = ((rule == kGnStaleOthers && j == pi) ? own : img[j * stride]).x - mu;
+      ss = fmaf(e, e, ss);
+    }
+    var = sv * inv + ss * inv;
+  }
+  return make_float2(mu, fmaxf(var, 0.f));
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kGnThreads)
 gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
@@ -48,11 +121,14 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
   const int p = blockIdx.y, chunk = blockIdx.x;
   float* chan = sh + 2 * PL * C;
 
-  // ---- phase 1: per-channel partial sums of this chunk of patch p (8 loads in flight)
+  // ---- phase 1: per-channel partial sums of x - K (K: the group's shift) over this chunk
+  // of patch p (8 loads in flight)
   float s1[VEC], s2[VEC];
 #pragma unroll
   for (int i = 0; i < VEC; ++i) s1[i] = s2[i] = 0.f;
   if (pl < PL) {
+    float k[VEC];
+    gn_thread_shifts<T, VEC>(a.x, p, a.pix_per_patch, C, vc * VEC, C / G, k);
     const int pix0 = chunk * pix_per_chunk;
     const int pix1 = min(pix0 + pix_per_chunk, a.pix_per_patch);
     const T* base = static_cast<const T*>(a.x) + (size_t)p * a.pix_per_patch * C + vc * VEC;
@@ -67,7 +143,11 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
         float v[VEC];
         unpack16(u[j], v);
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) { s1[i] += v[i]; s2[i] = fmaf(v[i], v[i], s2[i]); }
+        for (int i = 0; i < VEC; ++i) {
+          const float d = v[i] - k[i];
+          s1[i] += d;
+          s2[i] = fmaf(d, d, s2[i]);
+        }
       }
     }
     float4* d1 = reinterpret_cast<float4*>(sh + pl * C + vc * VEC);
@@ -131,38 +211,24 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
   if (tid < NG) {
     float t1 = 0.f, t2 = 0.f;
     for (int s = 0; s < S; ++s) { t1 += red[(s * NG + tid) * 2]; t2 += red[(s * NG + tid) * 2 + 1]; }
-    s_mom[tid * 2] = t1 * inv_n;
-    s_mom[tid * 2 + 1] = t2 * inv_n;
-    a.fresh_out[tid * 2] = s_mom[tid * 2];
-    a.fresh_out[tid * 2 + 1] = s_mom[tid * 2 + 1];
+    // (mean, var) of patch tid / G, group tid % G from the shifted sums
+    const float m1 = t1 * inv_n;
+    const float mean = gn_shift<T>(a.x, tid / G, a.pix_per_patch, C, tid % G, cg) + m1;
+    const float var = fmaxf(fmaf(-m1, m1, t2 * inv_n), 0.f);
+    s_mom[tid * 2] = mean;
+    s_mom[tid * 2 + 1] = var;
+    a.fresh_out[tid * 2] = mean;
+    a.fresh_out[tid * 2 + 1] = var;
   }
   __syncthreads();
   if (tid < NG) {
     const int pp = tid / G, gg = tid % G;
     const int NI = a.per_image, j0 = pp / NI * NI;   // the patches of pp's image
-    float e1, e2;
-    if (a.naive) {
-      e1 = s_mom[tid * 2]; e2 = s_mom[tid * 2 + 1];
-    } else if (a.is_sync) {
-      e1 = 0.f; e2 = 0.f;
-      for (int j = j0; j < j0 + NI; ++j) { e1 += s_mom[(j * G + gg) * 2]; e2 += s_mom[(j * G + gg) * 2 + 1]; }
-      e1 /= (float)NI; e2 /= (float)NI;
-    } else {
-      float st1 = 0.f, st2 = 0.f;
-      for (int j = j0; j < j0 + NI; ++j) { st1 += a.stale[(j * G + gg) * 2]; st2 += a.stale[(j * G + gg) * 2 + 1]; }
-      const float own1 = a.stale[(pp * G + gg) * 2], own2 = a.stale[(pp * G + gg) * 2 + 1];
-      if (a.mode == 0) {        // corrected
-        e1 = st1 / (float)NI + (s_mom[tid * 2] - own1);
-        e2 = st2 / (float)NI + (s_mom[tid * 2 + 1] - own2);
-      } else {                  // stale others
-        e1 = (s_mom[tid * 2] + (st1 - own1)) / (float)NI;
-        e2 = (s_mom[tid * 2 + 1] + (st2 - own2)) / (float)NI;
-      }
-    }
-    const float var = fmaxf(e2 - e1 * e1, 0.f);
-    const float rstd = 1.f / sqrtf(var + a.eps);
-    a.mean_rstd[tid * 2] = e1;
-    a.mean_rstd[tid * 2 + 1] = rstd;
+    const int rule = gn_rule(a);
+    const float2* img = reinterpret_cast<const float2*>(rule == kGnSync ? s_mom : a.stale) + j0 * G + gg;
+    const float2 e = gn_estimate(rule, NI, pp - j0, make_float2(s_mom[tid * 2], s_mom[tid * 2 + 1]), img, G);
+    a.mean_rstd[tid * 2] = e.x;
+    a.mean_rstd[tid * 2 + 1] = 1.f / sqrtf(e.y + a.eps);
   }
   if (tid == 0) *a.counter = 0u;
 }
@@ -307,12 +373,15 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
   const int NI = a.per_image, pi = p % NI;                 // patch within its image
   const bool top_src = o.halo_mode != 0 && pi > 0;         // my first row feeds patch p-1
   const bool bot_src = o.halo_mode != 0 && pi < NI - 1;    // my last row feeds patch p+1
-  // ---- phase 1: per-channel partial sums of this chunk (8 loads in flight)
+  // ---- phase 1: per-channel partial sums of x - K (K: the group's shift) over this chunk
+  // (8 loads in flight)
   {
     float s1[VEC], s2[VEC];
 #pragma unroll
     for (int i = 0; i < VEC; ++i) s1[i] = s2[i] = 0.f;
     if (pl < PL) {
+      float k[VEC];
+      gn_thread_shifts<T, VEC>(a.x, p, a.pix_per_patch, C, vc * VEC, C / G, k);
       for (int pix = pix0 + pl; pix < pix1; pix += 8 * PL) {
         uint4 u[8];
 #pragma unroll
@@ -323,7 +392,11 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
           float v[VEC];
           unpack16(u[j], v);
 #pragma unroll
-          for (int i = 0; i < VEC; ++i) { s1[i] += v[i]; s2[i] = fmaf(v[i], v[i], s2[i]); }
+          for (int i = 0; i < VEC; ++i) {
+            const float d = v[i] - k[i];
+            s1[i] += d;
+            s2[i] = fmaf(d, d, s2[i]);
+          }
         }
       }
       float4* d1 = reinterpret_cast<float4*>(sh + pl * C + vc * VEC);
@@ -413,43 +486,27 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
   if (tid < items) {
     float t1 = 0.f, t2 = 0.f;
     for (int s2 = 0; s2 < S; ++s2) { t1 += red[(s2 * items + tid) * 2]; t2 += red[(s2 * items + tid) * 2 + 1]; }
-    s_mom[tid * 2] = t1 * inv_n;
-    s_mom[tid * 2 + 1] = t2 * inv_n;
+    // (mean, var) of patch p_lo + tid / G, group tid % G from the shifted sums
+    const float m1 = t1 * inv_n;
+    s_mom[tid * 2] = gn_shift<T>(a.x, p_lo + tid / G, a.pix_per_patch, C, tid % G, cg) + m1;
+    s_mom[tid * 2 + 1] = fmaxf(fmaf(-m1, m1, t2 * inv_n), 0.f);
   }
   __syncthreads();
   if (tid < G) {
     const int gg = tid;
     const int own = (all ? pi : 0) * G + gg;    // this patch's entry in s_mom
-    const float m1 = s_mom[own * 2], m2 = s_mom[own * 2 + 1];
-    float e1, e2;
-    if (a.naive) {
-      e1 = m1; e2 = m2;
-    } else if (a.is_sync) {
-      e1 = 0.f; e2 = 0.f;
-      for (int j = 0; j < NI; ++j) { e1 += s_mom[(j * G + gg) * 2]; e2 += s_mom[(j * G + gg) * 2 + 1]; }
-      e1 /= (float)NI; e2 /= (float)NI;
-    } else {
-      float st1 = 0.f, st2 = 0.f;
-      for (int j = p - pi; j < p - pi + NI; ++j) {
-        st1 += a.stale[(j * G + gg) * 2];
-        st2 += a.stale[(j * G + gg) * 2 + 1];
-      }
-      const float own1 = a.stale[(p * G + gg) * 2], own2 = a.stale[(p * G + gg) * 2 + 1];
-      if (a.mode == 0) {        // corrected
-        e1 = st1 / (float)NI + (m1 - own1);
-        e2 = st2 / (float)NI + (m2 - own2);
-      } else {                  // stale others
-        e1 = (m1 + (st1 - own1)) / (float)NI;
-        e2 = (m2 + (st2 - own2)) / (float)NI;
-      }
-    }
-    const float rstd = 1.f / sqrtf(fmaxf(e2 - e1 * e1, 0.f) + a.eps);
-    s_mr[gg * 2] = e1;
+    const float2 mo = make_float2(s_mom[own * 2], s_mom[own * 2 + 1]);
+    const int rule = gn_rule(a);
+    const float2* img = rule == kGnSync ? reinterpret_cast<const float2*>(s_mom) + gg
+                                        : reinterpret_cast<const float2*>(a.stale) + (p - pi) * G + gg;
+    const float2 e = gn_estimate(rule, NI, pi, mo, img, G);
+    const float rstd = 1.f / sqrtf(e.y + a.eps);
+    s_mr[gg * 2] = e.x;
     s_mr[gg * 2 + 1] = rstd;
     if (chunk == 0) {
-      a.fresh_out[(p * G + gg) * 2] = m1;
-      a.fresh_out[(p * G + gg) * 2 + 1] = m2;
-      a.mean_rstd[(p * G + gg) * 2] = e1;
+      a.fresh_out[(p * G + gg) * 2] = mo.x;
+      a.fresh_out[(p * G + gg) * 2 + 1] = mo.y;
+      a.mean_rstd[(p * G + gg) * 2] = e.x;
       a.mean_rstd[(p * G + gg) * 2 + 1] = rstd;
     }
   }
@@ -586,6 +643,9 @@ cudaError_t launch_gn_stats_merge(const GnArgs& a, cudaStream_t s) {
   const size_t red = (size_t)kGnThreads * 2 * sizeof(float);
   if (smem < red) smem = red;
   dim3 grid(n_chunks, a.N);
+  // wide maps (bf16 C > 3072: one pixel lane of 16 C floats) need more than the default 48 KiB
+  cudaError_t e = cudaFuncSetAttribute(gn_stats_merge_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   gn_stats_merge_kernel<T><<<grid, kGnThreads, smem, s>>>(a, n_chunks, per);
   return cudaGetLastError();
 }

@@ -18,8 +18,8 @@ struct GnArgs {
   float eps;
   float* part;            // scratch [N][n_chunks][G][2] partial (sum x, sum x^2)
   unsigned* counter;      // scratch, one word, zero between launches
-  float* fresh_out;       // [N][G][2] this step's (E[x], E[x^2]) per (patch, group)
-  const float* stale;     // [N][G][2] moments of step t-1 (read on displaced steps)
+  float* fresh_out;       // [N][G][2] this step's (mean, variance) per (patch, group)
+  const float* stale;     // [N][G][2] (mean, variance) of step t-1 (read on displaced steps)
   const float* gamma;     // [C] fp32
   const float* beta;      // [C] fp32
   float* mean_rstd;       // [N][G][2] (mean, rstd) applied -- also read by the separate apply kernel

@@ -19,6 +19,7 @@
 // device share the array and it keeps the last call's contents: the counter that
 // must start at zero is cleared by every call, and calls whose work overlaps on
 // the GPU (different streams without ordering) race on the array.
+#include <cstdint>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -43,6 +44,12 @@ std::mutex g_mu;
 float* g_ptr[kMaxDevices] = {};
 
 thread_local std::string g_noalloc_error;
+
+// Byte ranges [a, a + na) and [b, b + nb) share at least one byte.
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
 
 dfp_status fail(dfp_status s, const std::string& m) {
   g_noalloc_error = m;
@@ -71,6 +78,17 @@ extern "C" DFP_API dfp_status dfp_group_norm_noalloc(const void* x, void* y, dfp
   if (mode != DFP_GN_CORRECTED && mode != DFP_GN_STALE_OTHERS) return fail(DFP_E_ARG, "unknown gn mode");
   if (!(eps >= 0.f)) return fail(DFP_E_ARG, "eps must be >= 0");
   if ((long long)H * W * C >= (1ll << 31)) return fail(DFP_E_ARG, "feature map too large");
+  // the kernels read x while writing y, and read stale_moments after writing fresh_moments
+  // (and before writing mean_rstd): no two of these may share memory
+  const size_t map_bytes = (size_t)H * W * C * (dtype == DFP_BF16 ? 2 : 4);
+  const size_t mom_bytes = (size_t)n_patches * groups * 2 * sizeof(float);
+  if (overlaps(x, map_bytes, y, map_bytes)) return fail(DFP_E_ARG, "x and y overlap (the op does not run in place)");
+  if (stale_moments && overlaps(stale_moments, mom_bytes, fresh_moments, mom_bytes))
+    return fail(DFP_E_ARG, "stale_moments and fresh_moments overlap: alternate two buffers between calls");
+  if (mean_rstd && overlaps(mean_rstd, mom_bytes, fresh_moments, mom_bytes))
+    return fail(DFP_E_ARG, "mean_rstd and fresh_moments overlap");
+  if (mean_rstd && stale_moments && overlaps(mean_rstd, mom_bytes, stale_moments, mom_bytes))
+    return fail(DFP_E_ARG, "mean_rstd and stale_moments overlap");
   const int pix_per_patch = (H / n_patches) * W;
   const int n_chunks = dfp::gn_stats_chunks(n_patches, pix_per_patch);
   const size_t part_need = (size_t)n_patches * n_chunks * groups * 2;

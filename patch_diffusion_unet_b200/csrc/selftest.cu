@@ -10,6 +10,7 @@
 
 #include "../../include/dfp.h"
 #include "dfp_common.cuh"
+#include "exp2_poly.cuh"
 
 namespace {
 
@@ -24,7 +25,37 @@ __global__ void wait_for_nothing_kernel(int* err, long long* cycles) {
   if (ok) atomicExch(err, -1);   // would mean the wait returned without its phase completing
 }
 
+// 2^x of consecutive pairs through the attention softmax's polynomial (exp2_poly.cuh),
+// as fp32 and as the truncated bf16 pairs the softmax stores.
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, uint32_t* __restrict__ y_bf16,
+                                 int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const bool two = i + 1 < n;
+  const uint64_t x2 = dfp::f2(x[i], two ? x[i + 1] : 0.f);
+  uint32_t r0, r1;
+  dfp::ex2_poly_pair_f32(x2, r0, r1);
+  y[i] = __uint_as_float(r0);
+  if (two) y[i + 1] = __uint_as_float(r1);
+  if (y_bf16) {
+    const uint32_t b = dfp::ex2_poly_pair_bf16(x2);
+    if (two) y_bf16[i / 2] = b;
+    else reinterpret_cast<uint16_t*>(y_bf16)[i] = (uint16_t)(b & 0xFFFFu);
+  }
+}
+
 }  // namespace
+
+extern "C" DFP_API dfp_status dfp_selftest_exp2_poly(const float* x, float* y, void* y_bf16, int n, void* stream) {
+  if (n < 0 || n > (1 << 30)) return DFP_E_ARG;
+  if (n == 0) return DFP_OK;
+  if (!x || !y) return DFP_E_ARG;
+  if (y_bf16 && (reinterpret_cast<uintptr_t>(y_bf16) & 3)) return DFP_E_ARG;
+  const int pairs = (n + 1) / 2;
+  exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      x, y, static_cast<uint32_t*>(y_bf16), n);
+  return cudaGetLastError() == cudaSuccess ? DFP_OK : DFP_E_CUDA;
+}
 
 extern "C" DFP_API dfp_status dfp_selftest_wait_timeout(int* code_out, long long* cycles_out) {
   if (!code_out) return DFP_E_ARG;

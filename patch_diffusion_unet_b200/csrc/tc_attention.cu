@@ -37,8 +37,8 @@
 // softmax.  The running maximum is lazy: O and l are rescaled (in TMEM) only
 // when a row's maximum grows by more than 2^8.  Part of the exponentials run as
 // a polynomial on the FMA pipe (range reduction to 2^j * 2^f, |f| <= 1/2, with a
-// degree-3 polynomial for 2^f fitted by weighted least squares on Chebyshev
-// nodes, max relative error 7.5e-5) to offload the MUFU unit.
+// degree-3 minimax polynomial for 2^f, max relative error 7.48e-5; exp2_poly.cuh)
+// to offload the MUFU unit.
 //
 // Work split (stream-K style): a unit of work is one KV tile for one Q-tile pair of
 // one (patch, head), the patches of all images of the batch in one list.  The units are laid out pair-major within (patch, head) and
@@ -58,6 +58,7 @@
 #include <vector>
 
 #include "dfp_common.cuh"
+#include "exp2_poly.cuh"
 #include "kernels.h"
 
 namespace dfp {
@@ -162,50 +163,6 @@ __device__ __forceinline__ float ex2_mufu(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// ---- packed fp32x2 arithmetic (two lanes per 64-bit register pair)
-__device__ __forceinline__ uint64_t f2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
-// 2^x for a pair on the FMA pipe, returned as a truncated bf16 pair (lo = first
-// lane): x = j + f with j = rint(x) by magic-constant rounding (1.5 * 2^23 puts j
-// in the low mantissa bits), 2^f by a degree-3 polynomial, 2^j added into the
-// exponent field.  x is clamped to >= -125 so the exponent cannot wrap.
-__device__ __forceinline__ uint32_t ex2_poly_pair_bf16(uint64_t x2) {
-  float x0, x1;
-  f2_split(x2, x0, x1);
-  const uint64_t x = f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-  const uint64_t t = add2(x, f2(12582912.f, 12582912.f));
-  const uint64_t j = add2(t, f2(-12582912.f, -12582912.f));
-  const uint64_t f = fma2(j, f2(-1.f, -1.f), x);
-  uint64_t p = fma2(f2(0.0551716648f, 0.0551716648f), f, f2(0.242611125f, 0.242611125f));
-  p = fma2(p, f, f2(0.693260968f, 0.693260968f));
-  p = fma2(p, f, f2(0.999928057f, 0.999928057f));
-  float p0, p1, t0, t1;
-  f2_split(p, p0, p1);
-  f2_split(t, t0, t1);
-  const uint32_t r0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
-  const uint32_t r1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(r0), "r"(r1));
-  return r;
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {

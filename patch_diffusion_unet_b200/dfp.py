@@ -24,7 +24,8 @@ EXPORTED = ("dfp_create", "dfp_load_weights", "dfp_step", "dfp_step_host", "dfp_
             "dfp_copy_out", "dfp_buffer_bytes", "dfp_check_device", "dfp_launches_per_step",
             "dfp_set_kernel_family", "dfp_set_profiling", "dfp_kernel_times", "dfp_destroy",
             "dfp_last_error", "dfp_group_norm_noalloc", "dfp_group_norm_noalloc_error",
-            "dfp_selftest_wait_timeout", "dfp_set_launch_overlap", "dfp_attention_schedule_check")
+            "dfp_selftest_wait_timeout", "dfp_selftest_exp2_poly", "dfp_set_launch_overlap",
+            "dfp_attention_schedule_check")
 
 
 class Config(ctypes.Structure):
@@ -75,6 +76,8 @@ def load_library(path=_LIB_PATH):
         "dfp_last_error": ([H], ctypes.c_char_p),
         "dfp_selftest_wait_timeout": ([ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_longlong)],
                                       ctypes.c_int),
+        "dfp_selftest_exp2_poly": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                    ctypes.c_void_p], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)

@@ -44,10 +44,12 @@ def gpu_stage_views(blk, cfg):
 
 
 def run_parity(cfg, n_steps, oracle_from=0, query_tokens=None, gn_mode=0, context=0, family=None,
-               weight_scale=None, random_affine=False, stages=True, seed=0):
+               weight_scale=None, random_affine=False, stages=True, seed=0, x_fn=None, orc_out=None):
     """Run steps 0..n_steps-1 on the GPU; the oracle joins at step `oracle_from` (which must be
     a sync step, so no earlier state is needed) and is compared at every step from there.
-    Returns a list of per-step dicts {stage: (rel_l2, max_abs)}."""
+    x_fn(t, x) -> x' changes the workload's input of step t before both sides see it (values
+    exactly representable in the storage type).  orc_out, a list, receives the oracle's
+    per-step outputs.  Returns a list of per-step dicts {stage: (rel_l2, max_abs)}."""
     from patch_diffusion_unet_b200 import dfp
 
     wl = inputs.SyntheticWorkload(cfg, seed=seed, weight_scale=weight_scale, random_affine=random_affine)
@@ -64,6 +66,8 @@ def run_parity(cfg, n_steps, oracle_from=0, query_tokens=None, gn_mode=0, contex
     prev_slab = None
     for t, is_sync in sched:
         x = wl.x(t)
+        if x_fn is not None:
+            x = x_fn(t, x)
         xd = inputs.to_torch(x, cfg["dtype"]).cuda()
         blk.step(xd, t, is_sync)
         blk.check_device()
@@ -72,6 +76,8 @@ def run_parity(cfg, n_steps, oracle_from=0, query_tokens=None, gn_mode=0, contex
                 prev_slab = gpu_stage_views(blk, cfg)["slab"]
             continue
         ref = orc.step(x, t - oracle_from, is_sync, query_tokens=query_tokens)
+        if orc_out is not None:
+            orc_out.append(ref)
         g = gpu_stage_views(blk, cfg) if stages else dict(y=host(blk.output()))
         res = {}
         qsel = (query_tokens,) if cfg.get("batch", 1) == 1 else (slice(None), query_tokens)

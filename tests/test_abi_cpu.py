@@ -79,3 +79,57 @@ def test_null_arguments():
     assert L.dfp_synchronize(None) == dfp.E_ARG
     assert L.dfp_step_host_async(None, None, None, 0, 1) == dfp.E_ARG
     assert isinstance(L.dfp_last_error(None), bytes)
+
+
+def _noalloc(x, y, stale, fresh, mr, H=64, W=64, C=640, N=4, G=32):
+    from patch_diffusion_unet_b200 import dfp
+    p = ctypes.c_void_p
+    return dfp.LIB.dfp_group_norm_noalloc(p(x), p(y), dfp.BF16, H, W, C, N, G, 1e-5, p(1 << 20), p(2 << 20),
+                                          None if stale is None else p(stale), dfp.GN_CORRECTED, 1, p(fresh),
+                                          None if mr is None else p(mr), None)
+
+
+@pytest.mark.parametrize("case,frag", [
+    # the displaced call reads stale_moments after writing fresh_moments: one buffer for
+    # both would silently turn every displaced call into the synchronous statistics
+    ("stale_is_fresh", "stale_moments and fresh_moments overlap"),
+    ("stale_overlaps_fresh", "stale_moments and fresh_moments overlap"),
+    ("y_is_x", "x and y overlap"),
+    ("y_overlaps_x", "x and y overlap"),
+    ("mean_rstd_is_fresh", "mean_rstd and fresh_moments overlap"),
+    ("mean_rstd_is_stale", "mean_rstd and stale_moments overlap"),
+])
+def test_noalloc_rejects_overlapping_buffers(case, frag):
+    """Host checks of dfp_group_norm_noalloc, before anything touches a GPU (the
+    addresses are never dereferenced)."""
+    from patch_diffusion_unet_b200 import dfp
+    x, y = 1 << 30, 2 << 30                       # 64x64x640 bf16 maps: 5.2 MB each
+    stale, fresh, mr = 3 << 30, 4 << 30, 5 << 30  # [4, 32, 2] fp32: 1 KiB each
+    if case == "stale_is_fresh":
+        stale = fresh
+    elif case == "stale_overlaps_fresh":
+        stale = fresh + 512
+    elif case == "y_is_x":
+        y = x
+    elif case == "y_overlaps_x":
+        y = x + 64 * 64 * 640 * 2 - 16
+    elif case == "mean_rstd_is_fresh":
+        mr = fresh
+    elif case == "mean_rstd_is_stale":
+        mr = stale
+    assert _noalloc(x, y, stale, fresh, mr) == dfp.E_ARG
+    assert frag in dfp.LIB.dfp_group_norm_noalloc_error().decode()
+
+
+def test_noalloc_adjacent_buffers_pass_the_overlap_checks():
+    """Buffers that only touch (one ends where the next starts) do not overlap: the call
+    gets past every overlap check and stops at the scratch-size check that follows them
+    (one patch of 64x64x4096 in 256 groups needs more partial sums than the fixed
+    scratch holds), still before any CUDA call."""
+    from patch_diffusion_unet_b200 import dfp
+    H, W, C, N, G = 64, 64, 4096, 1, 256
+    mb, nb = H * W * C * 2, N * G * 2 * 4
+    x, fresh = 1 << 30, 4 << 30
+    st = _noalloc(x, x + mb, fresh - nb, fresh, fresh + nb, H=H, W=W, C=C, N=N, G=G)
+    assert st == dfp.E_ARG
+    assert "scratch" in dfp.LIB.dfp_group_norm_noalloc_error().decode()

@@ -60,9 +60,16 @@ def test_batch_scales_every_launch():
 
 def test_traffic_only_for_the_captured_source(monkeypatch):
     """A recorded ncu traffic figure applies only while the kernel's sources hash the same."""
-    key = ("sdxl1024-64x64x640-n4-bf16", "attention (tcgen05)")
-    assert bench.ncu_traffic(*key) == bench.NCU_TRAFFIC[key][0]
+    import hashlib
+    import os
+    files = ("tc_attention.cu", "dfp_common.cuh", "exp2_poly.cuh")
+    m = hashlib.sha256()
+    for fn in files:
+        with open(os.path.join(bench.ROOT, "patch_diffusion_unet_b200", "csrc", fn), "rb") as f:
+            m.update(f.read())
+    key = ("some-workload", "attention (tcgen05)")
+    monkeypatch.setitem(bench.NCU_TRAFFIC, key, (123.0e6, files, m.hexdigest()[:16]))
+    assert bench.ncu_traffic(*key) == 123.0e6
     assert bench.ncu_traffic("some-other-workload", "attention (tcgen05)") is None
-    nbytes, files, _ = bench.NCU_TRAFFIC[key]
-    monkeypatch.setitem(bench.NCU_TRAFFIC, key, (nbytes, files, "0" * 16))
+    monkeypatch.setitem(bench.NCU_TRAFFIC, key, (123.0e6, files, "0" * 16))
     assert bench.ncu_traffic(*key) is None

@@ -48,6 +48,57 @@ def test_config0_fp32_random_affine_longer_run():
     _assert(run_parity(cfg, 8, random_affine=True), TOL["f32"])
 
 
+# ------------------------------------------------------------------ GroupNorm edge cases
+
+def _jump_patch0(cfg, scale=10.0):
+    """Step 0 with patch 0 scaled by `scale`, later steps unchanged: on step 1 (the first
+    displaced step) the corrected estimate of patch 0's variance, avg_j V_j + (v_0 - V_0),
+    is negative (the stale V_0 is scale^2 times the fresh v_0), so the clamp at 0 decides it."""
+    R = cfg["H"] // cfg["n_patches"]
+
+    def fn(t, x):
+        if t != 0:
+            return x
+        x = np.array(x, copy=True)
+        x[..., :R, :, :] = inputs.round_to(scale * x[..., :R, :, :], cfg["dtype"])
+        return x
+    return fn
+
+
+@pytest.mark.parametrize("cfg", [configs.get(0), dict(configs.get(0), name="r40-bf16", H=24, W=40, C=128,
+                                                      n_patches=3, gn_groups=8, heads=2, dtype="bf16",
+                                                      steps=4, n_sync=1)],
+                         ids=["fp32-16x16x64", "bf16-24x40x128"])
+def test_groupnorm_variance_clamp(cfg):
+    """A displaced step right after an input jump: the oracle clamps patch 0's GN1 variance
+    (asserted here on the CPU side), and the GPU path matches it at every stage."""
+    orc = []
+    res = run_parity(cfg, cfg["steps"], x_fn=_jump_patch0(cfg), orc_out=orc)
+    mu, var = orc[1]["gn1"]
+    assert np.all(var[0] == 0.0), "the oracle did not clamp: the test input does not reach the clamp"
+    assert np.all(var[1:] > 0.0)
+    _assert(res, TOL[cfg["dtype"]])
+
+
+def test_groupnorm_large_mean_fp32():
+    """x + 30 (mean 30, spread about 1) at the fp32 bar: the statistics must not lose the
+    variance to the cancellation of E[x^2] - E[x]^2 (at mean 30, E[x^2] ~ 901)."""
+    cfg = configs.get(0)
+    shift = lambda t, x: inputs.round_to(np.asarray(x, np.float64) + 30.0, "f32")  # noqa: E731
+    _assert(run_parity(cfg, cfg["steps"], x_fn=shift), TOL["f32"])
+    _assert(run_parity(cfg, cfg["steps"], x_fn=shift, gn_mode=1), TOL["f32"])
+
+
+def test_groupnorm_large_mean_bf16_tcgen05():
+    cfg = RAGGED_MEAN
+    shift = lambda t, x: inputs.round_to(np.asarray(x, np.float64) + 30.0, "bf16")  # noqa: E731
+    _assert(run_parity(cfg, cfg["steps"], x_fn=shift, random_affine=True), TOL["bf16"])
+
+
+RAGGED_MEAN = dict(name="r40m", H=24, W=40, C=128, n_patches=3, gn_groups=8, gn_eps=1e-5, heads=2, head_dim=64,
+                   dtype="bf16", block="res_attn", steps=5, n_sync=2)
+
+
 # ------------------------------------------------------------------ small bf16 shapes (ragged tiles)
 
 RAGGED = [

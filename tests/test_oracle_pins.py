@@ -81,6 +81,22 @@ def test_gn_hand_example_through_layer():
         _close(out[0, :, 0], (np.array(g["patch0_fresh_values"]) - exp["mu"]) / math.sqrt(exp["var"]))
 
 
+def test_gn_clamp_hand_example():
+    """A displaced step whose corrected variance estimate is negative: the oracle clamps it
+    to 0, so patch 0 is normalised by 1/sqrt(eps) (eps = 1/4 here: outputs are x * 2)."""
+    g = json.load(open(os.path.join(GOLDEN, "gn_clamp_hand_example.json")))
+    prev = np.array(g["patch0_stale_values"] + g["patch1_stale_values"]).reshape(2, 2, 1)
+    cur = np.array(g["patch0_fresh_values"] + g["patch1_fresh_values"]).reshape(2, 2, 1)
+    for mode in ("corrected", "stale_others"):
+        gn = oracle.DisplacedGroupNorm(2, 1, g["eps"], np.ones(1), np.zeros(1), mode)
+        gn(prev, is_sync=True)
+        out = gn(cur, is_sync=False)
+        exp = g["expected"][mode]
+        assert gn.last[0][0, 0] == pytest.approx(exp["mu"], abs=1e-12)
+        assert gn.last[1][0, 0] == exp["var"]
+        _close(out[0, :, 0], np.array(exp["patch0_out"]))
+
+
 # --------------------------------------------------------------------------- library pins
 
 @pytest.mark.parametrize("cfg", [configs.get(0), SMALL, configs.get(SMALL, n_patches=2),
