@@ -67,7 +67,13 @@ typedef enum {
   /* est_p = mean_j m_j(t-1) + (m_p(t) - m_p(t-1)), m = (E[x], E[x^2]) per (patch, group) */
   DFP_GN_CORRECTED = 0,
   /* est_p = (m_p(t) + sum_{j != p} m_j(t-1)) / N */
-  DFP_GN_STALE_OTHERS = 1
+  DFP_GN_STALE_OTHERS = 1,
+  /* GroupNorm-only variants of the pages' --sync_mode flag (project README, Benchmarks),
+   * conv halos and attention K/V still displaced:
+   * est_p = mean_j m_j(t): this step's full-map statistics on displaced steps too */
+  DFP_GN_SYNC = 2,
+  /* est_p = m_p(t): patch-local statistics on displaced steps (sync steps stay exact) */
+  DFP_GN_SEPARATE = 3
 } dfp_gn_mode;
 
 typedef enum {
@@ -152,6 +158,33 @@ DFP_API dfp_status dfp_load_weights(dfp_handle h, const dfp_tensor* w, int n);
  * Errors: DFP_E_STATE (order, weights missing), DFP_E_ARG, DFP_E_CUDA. */
 DFP_API dfp_status dfp_step(dfp_handle h, const void* x, int step, int is_sync);
 
+/* Patch parallelism across GPUs (project README, Overview (c): one patch per device, the
+ * other patches' activations of the previous step as context, exchanged asynchronously;
+ * paper reading blog, Ablation: patch parallelism gathers activations with AllGather).
+ * A rank holds a handle for the whole map and computes only its patches [p_begin, p_end)
+ * on displaced steps; between steps the ranks all-gather what each computed -- this
+ * step's K/V rows, GroupNorm moments, the boundary rows of the conv input and the output
+ * rows -- into every rank's buffers (dfp_context_buffer), so the next displaced step finds
+ * the other patches' context of the previous step in place.  Synchronous steps run the
+ * whole map on every rank (dfp_step).  Requirements: DFP_BLOCK_RES_ATTN, bf16, the
+ * tensor-core kernels, batch 1, a gn_mode that needs no statistics of other patches of
+ * the same step (not DFP_GN_SYNC), step >= 1 following the previous step; else
+ * DFP_E_UNSUPPORTED / DFP_E_STATE / DFP_E_ARG (bad range).  Only the range's rows of the
+ * outputs are written: y, this step's K/V, moments and slab rows of the range; the
+ * conv input's halo rows at the range's ends must hold the neighbours' boundary rows of
+ * the previous step (the exchange puts them there).  Asynchronous like dfp_step. */
+DFP_API dfp_status dfp_step_patches(dfp_handle h, const void* x, int step, int p_begin, int p_end);
+
+/* Device pointer and size of a library-owned buffer that the patch-parallel exchange
+ * reads and fills (no counterpart in the pages beyond the all_gather buffers).  parity =
+ * step & 1 selects the step's buffer of the alternating pairs.  Names and layouts:
+ * "k", "v"      [heads][B*L][64] the step's keys / values
+ * "mom1","mom2" [B*N][G][2] fp32 (mean, variance) of GN1 / GN2 per (patch, group)
+ * "slab"        [B*N][R+2][W][C] the conv input with one halo row above / below each patch
+ * "y"           [B*L][C] the block output (parity ignored)
+ * Valid until dfp_destroy.  DFP_E_ARG for an unknown name or a parity other than 0 / 1. */
+DFP_API dfp_status dfp_context_buffer(dfp_handle h, const char* name, int parity, void** ptr, long long* bytes);
+
 /* Same step with HOST buffers: copies x_host ([B,H,W,C], config dtype; pinned
  * memory gives asynchronous copies) to the device, runs the step, copies the
  * output to y_host and waits for the stream. */
@@ -224,10 +257,12 @@ DFP_API int dfp_launches_per_step(dfp_handle h);
  * and its other pieces each at the start of a range; the kernel's publisher and flag
  * warps predict exactly those pieces.  L tokens per image in n_patches patches of Lp
  * tokens; mode 0 sync, 1 displaced, 2 naive, 3 cross-attention (Lp = L, n_patches = 1,
- * kv_len context tokens).  Returns 0 if every property holds, else the number of the
- * first that fails (1: bad arguments). */
+ * kv_len context tokens).  Only the query patches [p_begin, p_end) of the image-major
+ * patch list are listed (p_begin = p_end = 0: all), as for a patch-parallel rank's range.
+ * Returns 0 if every property holds, else the number of the first that fails (1: bad
+ * arguments). */
 DFP_API int dfp_attention_schedule_check(int L, int Lp, int n_patches, int heads, int mode, int kv_len, int images,
-                                         int ctas);
+                                         int ctas, int p_begin, int p_end);
 
 /* Launch overlap between the kernels of a step (no counterpart in the pages; on by
  * default): every tensor-core-family kernel is launched with programmatic stream

@@ -50,11 +50,19 @@ Readings adopted where the pages are silent:
       details; [README] Benchmarks, --no_split_batch): each image of a batch is
       its own displaced-patch step -- own GroupNorm statistics, halo rows, K/V
       and text context -- sharing only the weights and the step schedule.
+  R8  GroupNorm-only variants of --sync_mode ([README] Benchmarks: the flag picks
+      among GroupNorm synchronisation modes and names only the default): "sync" uses this step's
+      moments of every patch (the exact full-map GroupNorm) on displaced steps too,
+      "separate" uses only the patch's own moments of this step (patch-local
+      GroupNorm) on displaced steps; conv halos and attention K/V stay displaced in
+      both.  Sync steps are exact in every mode.
 """
 import numpy as np
 
 GN_CORRECTED = "corrected"
 GN_STALE_OTHERS = "stale_others"
+GN_SYNC = "sync"
+GN_SEPARATE = "separate"
 CTX_DISPLACED = "displaced"
 CTX_NAIVE = "naive"
 
@@ -78,11 +86,11 @@ def group_moments(xp, G):
 
 
 def merge_moments(fresh, stale, is_sync, mode, context=CTX_DISPLACED):
-    """Per-patch GroupNorm mean and variance from fresh / stale moments [N, G, 2] (R3, R6)."""
+    """Per-patch GroupNorm mean and variance from fresh / stale moments [N, G, 2] (R3, R6, R8)."""
     N = fresh.shape[0]
-    if context == CTX_NAIVE:
+    if context == CTX_NAIVE or (mode == GN_SEPARATE and not is_sync):
         est = fresh
-    elif is_sync:
+    elif is_sync or mode == GN_SYNC:
         est = np.broadcast_to(fresh.mean(axis=0), fresh.shape)
     elif mode == GN_CORRECTED:
         est = stale.mean(axis=0)[None] + (fresh - stale)
@@ -163,7 +171,8 @@ class DisplacedGroupNorm:
         H = x.shape[0]
         bounds = patch_bounds(H, self.N)
         fresh = np.stack([group_moments(x[r0:r1], self.G) for r0, r1 in bounds])
-        if not is_sync and self.context != CTX_NAIVE and self.prev is None:
+        reads_stale = self.mode in (GN_CORRECTED, GN_STALE_OTHERS) and self.context != CTX_NAIVE
+        if not is_sync and reads_stale and self.prev is None:
             raise RuntimeError("displaced GroupNorm needs the previous step's statistics")
         mu, var = merge_moments(fresh, self.prev, is_sync, self.mode, self.context)
         out = np.empty_like(x)

@@ -71,7 +71,7 @@ dfp_status check_config(const dfp_config* c, std::string& why) {
   if (c->C % 64) return bad("C must be a multiple of 64");
   if (c->C > 4096) return bad("C must be <= 4096");
   if (c->dtype != DFP_F32 && c->dtype != DFP_BF16) return bad("unknown dtype");
-  if (c->gn_mode != DFP_GN_CORRECTED && c->gn_mode != DFP_GN_STALE_OTHERS) return bad("unknown gn_mode");
+  if (c->gn_mode < DFP_GN_CORRECTED || c->gn_mode > DFP_GN_SEPARATE) return bad("unknown gn_mode");
   if (c->context != DFP_CTX_DISPLACED && c->context != DFP_CTX_NAIVE) return bad("unknown context");
   if (!(c->gn_eps >= 0.f)) return bad("gn_eps must be >= 0");
   const long long Lp = (long long)(c->H / c->n_patches) * c->W;
@@ -181,7 +181,7 @@ std::vector<uint8_t> to_storage(const std::vector<float>& v, dfp_dtype dt) {
 }
 
 template <typename T>
-dfp_status run_step(dfp_ctx* h, const void* x, int step, int is_sync);
+dfp_status run_step(dfp_ctx* h, const void* x, int step, int is_sync, int p0 = 0, int p1 = -1);
 
 }  // namespace
 
@@ -237,7 +237,7 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
   ok &= h->alloc(&h->xin, map);
   ok &= h->alloc((void**)&h->mr1, N * G * 2 * 4);
   ok &= h->alloc((void**)&h->mr2, N * G * 2 * 4);
-  ok &= h->alloc((void**)&h->part, N * (size_t)gn_stats_chunks((int)N, (int)(R * W)) * G * 2 * 4);
+  ok &= h->alloc((void**)&h->part, gn_part_floats((int)N, (int)(R * W), (int)G) * 4);
   ok &= h->alloc((void**)&h->counter, 64);
   ok &= h->alloc((void**)&h->dev_err, 64);
   if (cfg->dtype == DFP_BF16) {
@@ -380,6 +380,45 @@ dfp_status dfp_step(dfp_handle h, const void* x, int step, int is_sync) {
                                             : run_step<float>(h, x, step, is_sync);
   if (st == DFP_OK) h->last_step = step;
   return st;
+}
+
+dfp_status dfp_step_patches(dfp_handle h, const void* x, int step, int p_begin, int p_end) {
+  if (!h) return DFP_E_ARG;
+  if (!x) return h->fail(DFP_E_ARG, "x is NULL");
+  const dfp_config& c = h->cfg;
+  if (h->stage || c.dtype != DFP_BF16 || h->family != 0 || h->B != 1)
+    return h->fail(DFP_E_UNSUPPORTED, "a patch range runs the layer block of one bf16 image on the tensor-core kernels");
+  if (c.gn_mode == DFP_GN_SYNC && c.context != DFP_CTX_NAIVE)
+    return h->fail(DFP_E_UNSUPPORTED, "the GroupNorm sync mode needs every patch's statistics of this step");
+  if (p_begin < 0 || p_end > c.n_patches || p_begin >= p_end) return h->fail(DFP_E_ARG, "bad patch range");
+  if (h->loaded.size() != weight_specs(h).size())
+    return h->fail(DFP_E_STATE, "weights not loaded (every weight must be given before the first step)");
+  if (step <= 0 || step != h->last_step + 1)
+    return h->fail(DFP_E_STATE, "a patch-range step is displaced: it must follow the previous step (step >= 1)");
+  dfp_status st = run_step<__nv_bfloat16>(h, x, step, 0, p_begin, p_end);
+  if (st == DFP_OK) h->last_step = step;
+  return st;
+}
+
+dfp_status dfp_context_buffer(dfp_handle h, const char* name, int parity, void** ptr, long long* bytes) {
+  if (!h) return DFP_E_ARG;
+  if (!name || !ptr || !bytes) return h->fail(DFP_E_ARG, "NULL argument");
+  if (parity != 0 && parity != 1) return h->fail(DFP_E_ARG, "parity must be 0 or 1");
+  if (h->stage) return h->fail(DFP_E_UNSUPPORTED, "context buffers of the layer block only");
+  const dfp_config& c = h->cfg;
+  const long long map = (long long)h->B * h->L * c.C * (long long)h->esz;
+  const long long mom = (long long)h->B * c.n_patches * c.gn_groups * 2 * 4;
+  const std::string n = name;
+  if (n == "k") { *ptr = h->kb[parity]; *bytes = map; }
+  else if (n == "v") { *ptr = h->vb[parity]; *bytes = map; }
+  else if (n == "mom1") { *ptr = h->mom1[parity]; *bytes = mom; }
+  else if (n == "mom2") { *ptr = h->mom2[parity]; *bytes = mom; }
+  else if (n == "slab") {
+    *ptr = h->slab[parity];
+    *bytes = (long long)h->B * c.n_patches * (h->R + 2) * c.W * c.C * (long long)h->esz;
+  } else if (n == "y") { *ptr = h->y; *bytes = map; }
+  else return h->fail(DFP_E_ARG, std::string("unknown context buffer ") + name);
+  return DFP_OK;
 }
 
 dfp_status dfp_step_host(dfp_handle h, const void* x_host, void* y_host, int step, int is_sync) {
@@ -527,9 +566,9 @@ dfp_status dfp_check_device(dfp_handle h) {
 int dfp_launches_per_step(dfp_handle h) { return h ? h->launches : -1; }
 
 int dfp_attention_schedule_check(int L, int Lp, int n_patches, int heads, int mode, int kv_len, int images,
-                                 int ctas) {
+                                 int ctas, int p_begin, int p_end) {
   if (mode < kAttnSync || mode > kAttnCross) return 1;
-  return attention_schedule_check(L, Lp, n_patches, heads, mode, kv_len, images, ctas);
+  return attention_schedule_check(L, Lp, n_patches, heads, mode, kv_len, images, ctas, p_begin, p_end);
 }
 
 dfp_status dfp_set_launch_overlap(dfp_handle h, int enable) {
@@ -603,12 +642,17 @@ const char* dfp_last_error(dfp_handle h) {
 // ====================================================================== step scheduler
 namespace {
 
+// p0, p1: the patches computed, [p0, p1) of the one image (a patch-parallel rank's range;
+// the whole map when p1 < 0).  Range steps are displaced tensor-core steps of one image.
 template <typename T>
-dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
+dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync, int p0, int p1) {
   const dfp_config& c = h->cfg;
   // N, L per image; NB, LB over the batch (B images, patch b*N + p, token b*L + i)
   const int N = c.n_patches, C = c.C, G = c.gn_groups, W = c.W, R = h->R, L = h->L, Lp = h->Lp;
   const int B = h->B, NB = B * N, LB = B * L;
+  const bool range = p1 >= 0;
+  if (!range) { p0 = 0; p1 = NB; }
+  const int n_run = p1 - p0;
   const int cur = step & 1, prv = cur ^ 1;
   const bool naive = c.context == DFP_CTX_NAIVE;
   const bool displaced = !is_sync && !naive;
@@ -626,6 +670,7 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   g.fresh_out = h->mom1[cur]; g.stale = h->mom1[prv];
   g.gamma = h->gn1_g; g.beta = h->gn1_b; g.mean_rstd = h->mr1;
   g.is_sync = is_sync; g.mode = (int)c.gn_mode; g.naive = naive ? 1 : 0;
+  g.p0 = p0; g.n_run = n_run;
   // consecutive tensor-core-family kernels overlap launch and set-up with their
   // predecessor's tail (each waits for the predecessor before touching memory)
   const int pdl = h->overlap ? 1 : 0;
@@ -646,8 +691,13 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   // ---- conv3x3 (+ bias) -> h
   Epilogue ec{};
   ec.kind = 0; ec.out = h->h; ec.bias = h->b_conv; ec.ldo = C;
+  // a patch range computes the conv tiles of its patches and the projections of its rows
+  TcGemmPlan conv_plan = h->conv_plan, qkv_plan = h->qkv_plan, out_plan = h->out_plan;
+  conv_plan.p0 = p0; conv_plan.P = n_run;
+  qkv_plan.m_base = out_plan.m_base = p0 * Lp;
+  qkv_plan.M = out_plan.M = p1 * Lp;
   if (h->family == 0) {
-    DFP_LAUNCH(launch_tc_gemm(h->conv_plan, h->m_slab[cur], h->m_wconv, ec, h->dev_err, s), "conv (tcgen05)");
+    DFP_LAUNCH(launch_tc_gemm(conv_plan, h->m_slab[cur], h->m_wconv, ec, h->dev_err, s), "conv (tcgen05)");
   } else {
     ConvA cv{slab, NB, R, W, C};
     DFP_LAUNCH(launch_simt_gemm<T>(nullptr, &cv, static_cast<const T*>(h->w_conv), LB, C, 9 * C, ec, s), "conv (simt)");
@@ -667,7 +717,7 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   Epilogue eq{};
   eq.kind = 1; eq.q = h->q; eq.k = h->kb[cur]; eq.v = h->vb[cur]; eq.L = LB; eq.C = C;
   if (h->family == 0) {
-    DFP_LAUNCH(launch_tc_gemm(h->qkv_plan, h->m_t, h->m_wqkv, eq, h->dev_err, s), "qkv (tcgen05)");
+    DFP_LAUNCH(launch_tc_gemm(qkv_plan, h->m_t, h->m_wqkv, eq, h->dev_err, s), "qkv (tcgen05)");
   } else {
     DFP_LAUNCH(launch_simt_gemm<T>(static_cast<const T*>(h->t), nullptr, static_cast<const T*>(h->w_qkv), LB, 3 * C, C, eq, s), "qkv (simt)");
   }
@@ -677,6 +727,7 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
     TcAttnArgs a{};
     a.L = L; a.Lp = Lp; a.N = N; a.heads = c.heads; a.C = C; a.mode = mode; a.o = h->o; a.err = h->dev_err;
     a.images = B; a.kv_stride = L; a.pdl = pdl;
+    a.p_lo = p0; a.p_hi = p1;
     a.ctas = h->attn_ctas; a.n_qtiles = (Lp + 127) / 128;
     a.part_o = h->attn_part_o; a.part_ml = h->attn_part_ml; a.flags = h->attn_flags;
     DFP_LAUNCH(launch_tc_attention(a, h->m_q, h->m_k[cur], h->m_v[cur], h->m_k[prv], h->m_v[prv], s), "attention (tcgen05)");
@@ -690,7 +741,7 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
   Epilogue eo{};
   eo.kind = 0; eo.out = h->y; eo.bias = h->b_o; eo.ldo = C;
   if (h->family == 0) {
-    DFP_LAUNCH(launch_tc_gemm(h->out_plan, h->m_o, h->m_wo, eo, h->dev_err, s), "out projection (tcgen05)");
+    DFP_LAUNCH(launch_tc_gemm(out_plan, h->m_o, h->m_wo, eo, h->dev_err, s), "out projection (tcgen05)");
   } else {
     DFP_LAUNCH(launch_simt_gemm<T>(static_cast<const T*>(h->o), nullptr, static_cast<const T*>(h->w_o), LB, C, C, eo, s), "out projection (simt)");
   }

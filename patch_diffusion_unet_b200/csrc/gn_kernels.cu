@@ -10,6 +10,8 @@
 //   corrected  est_p = mean_j m_j(t-1) + (m_p(t) - m_p(t-1))
 //   stale-oth. est_p = (m_p(t) + sum_{j != p} m_j(t-1)) / N
 //   naive      est_p = m_p(t)                             (no cross-patch context)
+// The GroupNorm-only variants of --sync_mode apply the sync rule (mode "sync") or the
+// naive rule (mode "separate") on displaced steps too, the other layers staying displaced.
 //   mean = est.E[x], var = max(est.E[x^2] - mean^2, 0), rstd = 1 / sqrt(var + eps).
 // j runs over the N patches of the same image: a batch of images (the guidance
 // batch) is images x N patches, numbered image-major, with nothing shared across images.
@@ -66,8 +68,17 @@ __device__ __forceinline__ void gn_thread_shifts(const void* x, int p, int pix_p
 
 // Merge rules of DistriGroupNorm on per-patch (mean, var) moments (see the file header).
 enum GnRule : int { kGnNaive = 0, kGnSync = 1, kGnCorrected = 2, kGnStaleOthers = 3 };
+// a.mode is the dfp_gn_mode: 0 corrected, 1 stale-others, 2 sync, 3 separate (the last two
+// are GroupNorm-only variants: every step this step's full-map / patch-local statistics)
 __device__ __forceinline__ int gn_rule(const GnArgs& a) {
-  return a.naive ? kGnNaive : a.is_sync ? kGnSync : a.mode == 0 ? kGnCorrected : kGnStaleOthers;
+  if (a.naive) return kGnNaive;
+  if (a.is_sync) return kGnSync;
+  switch (a.mode) {
+    case 0: return kGnCorrected;
+    case 1: return kGnStaleOthers;
+    case 2: return kGnSync;
+    default: return kGnNaive;
+  }
 }
 // own: this step's moments of patch pi (of NI in its image); img: moments of the image's
 // patches (this step's for kGnSync, the previous step's otherwise), `stride` float2 apart.
@@ -361,7 +372,7 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
   const int PL = kGnThreads / V;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int vc = tid % V, pl = tid / V;
-  const int p = blockIdx.y, chunk = blockIdx.x;
+  const int lp = blockIdx.y, p = a.p0 + lp, chunk = blockIdx.x;   // lp: place in the computed range
   const int pix0 = chunk * pix_per_chunk;
   const int pix1 = min(pix0 + pix_per_chunk, a.pix_per_patch);
   const T* base = static_cast<const T*>(a.x) + (size_t)p * a.pix_per_patch * C + vc * VEC;
@@ -422,7 +433,7 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
     for (int c = lane; c < cg; c += 32) { t1 += chan[g * cg + c]; t2 += chan[C + g * cg + c]; }
     t1 = warp_sum(t1);
     t2 = warp_sum(t2);
-    if (lane == 0) reinterpret_cast<float2*>(a.part)[((size_t)p * n_chunks + chunk) * G + g] = make_float2(t1, t2);
+    if (lane == 0) reinterpret_cast<float2*>(a.part)[((size_t)lp * n_chunks + chunk) * G + g] = make_float2(t1, t2);
   }
 
   // ---- grid barrier: every chunk partial is written
@@ -459,14 +470,14 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
   if (!grid_wait(a.counter, total, err)) return;
 
   // ---- phase 2: fresh moments of the patches needed, in a fixed order
-  const bool all = a.is_sync && !a.naive;       // sync steps merge the image's fresh moments
+  const bool all = gn_rule(a) == kGnSync;       // the sync rule merges the image's fresh moments
   const int p_lo = all ? p - pi : p, np = all ? NI : 1;
   const int items = np * G;                     // <= 256
   const int S = kGnThreads / items;             // threads per item, >= 2
   float* red = sh;                              // [S][items][2]
   if (tid < S * items) {
     const int item = tid % items, part_id = tid / items;
-    const int pp = p_lo + item / G, gg = item % G;
+    const int pp = p_lo + item / G - a.p0, gg = item % G;   // place in the computed range
     const float2* src = reinterpret_cast<const float2*>(a.part) + (size_t)pp * n_chunks * G + gg;
     // chunks part_id, part_id + S, ... summed in that order, eight loads in flight (the
     // zeros past the end leave the sum unchanged)
@@ -632,6 +643,12 @@ int gn_stats_chunks(int N, int pix_per_patch) {
   return (pix_per_patch + per - 1) / per;
 }
 
+size_t gn_part_floats(int N, int pix_per_patch, int G) {
+  size_t most = 0;
+  for (int n = 1; n <= N; ++n) most = std::max(most, (size_t)n * gn_stats_chunks(n, pix_per_patch));
+  return most * G * 2;
+}
+
 template <typename T>
 cudaError_t launch_gn_stats_merge(const GnArgs& a, cudaStream_t s) {
   constexpr int VEC = VecTraits<T>::kN;
@@ -685,12 +702,17 @@ cudaError_t launch_gn_fused(const GnArgs& a, const GnOut& o, bool silu, int* err
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGnThreads, smem);
   if (e != cudaSuccess) return e;
   const int max_blocks = per_sm * sm_count();
-  if (a.N > max_blocks) return cudaErrorCooperativeLaunchTooLarge;
-  int n_chunks = std::min(gn_stats_chunks(a.N, a.pix_per_patch), max_blocks / a.N);
+  const int n_run = a.n_run > 0 ? a.n_run : a.N;   // patches computed
+  if (a.p0 < 0 || a.p0 + n_run > a.N) return cudaErrorInvalidValue;
+  // the sync rule merges every patch of an image from this launch's partial sums
+  const bool all = !a.naive && (a.is_sync || a.mode == 2);
+  if (all && n_run != a.N) return cudaErrorInvalidValue;
+  if (n_run > max_blocks) return cudaErrorCooperativeLaunchTooLarge;
+  int n_chunks = std::min(gn_stats_chunks(n_run, a.pix_per_patch), max_blocks / n_run);
   const int per = (a.pix_per_patch + n_chunks - 1) / n_chunks;
   n_chunks = (a.pix_per_patch + per - 1) / per;
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(n_chunks, a.N);
+  cfg.gridDim = dim3(n_chunks, n_run);
   cfg.blockDim = dim3(kGnThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;

@@ -25,6 +25,8 @@ struct GnArgs {
   float* mean_rstd;       // [N][G][2] (mean, rstd) applied -- also read by the separate apply kernel
   int is_sync, mode, naive;
   int pdl;                // fused kernel: launch with programmatic stream serialization
+  int p0, n_run;          // fused kernel: patches [p0, p0 + n_run) are computed (0, 0: all N);
+                          // part is indexed by the patch's place in that range
 };
 // Output side of the fused GroupNorm: out [N][out_patch_stride pixels][C] starting at
 // pixel out_off of each patch (the haloed slab, or a plain map with stride pix_per_patch
@@ -36,6 +38,8 @@ struct GnOut {
   int W, halo_mode;
 };
 int gn_stats_chunks(int N, int pix_per_patch);
+// floats of GroupNorm partial sums any patch range of N patches needs (the part scratch)
+size_t gn_part_floats(int N, int pix_per_patch, int G);
 // statistics + merge + apply (+SiLU) in one cooperative launch; a.counter needs two
 // zeroed words; a.mean_rstd receives (mean, rstd)
 template <typename T> cudaError_t launch_gn_fused(const GnArgs& a, const GnOut& o, bool silu, int* err, cudaStream_t s);
@@ -97,11 +101,13 @@ bool encode_tmap_5d(CUtensorMap* m, const void* base, const uint64_t dims[5],
 bool encode_gemm_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows);
 
 struct TcGemmPlan {
-  int M, N, K;            // GEMM sizes (conv: M = H*W, K = 9*Cin)
+  int M, N, K;            // GEMM sizes (conv: M = H*W, K = 9*Cin); plain: rows [m_base, M) are computed
   int bn;                 // N tile (64, 128, 160 or 256)
   int conv;               // 1: A is the haloed slab (4-D map), 0: plain [M, K] (2-D map)
+  int m_base;             // plain: first row computed (a patch range of a patch-parallel rank; else 0)
+  int p0;                 // conv: first patch computed; P patches from there
   // conv geometry
-  int P, R, W, Cin;       // patches, rows per patch, width, input channels
+  int P, R, W, Cin;       // patches computed, rows per patch, width, input channels
   int cols_tile, rows_tile, tiles_per_row;
   int pair;               // 1: CTA-pair kernel (256 x bn tiles; B's map boxes bn/2 rows)
   int m_tiles;            // filled by launch_tc_gemm
@@ -125,6 +131,7 @@ int gemm_m_tiles_plain(int M);
 
 struct TcAttnArgs {
   int L, Lp, N, heads, C, mode;   // per image: L tokens in N patches of Lp
+  int p_lo, p_hi;         // query patches [p_lo, p_hi) of the image-major patch list (0, 0: all)
   int images;             // images of the batch; q, o, k and v hold them one after another
   int kv_stride;          // K/V rows per image: L, or the padded context rows (kAttnCross)
   int kv_len;             // cross-attention: number of context tokens (mode kAttnCross)
@@ -143,7 +150,8 @@ struct TcAttnArgs {
 // floats of part_o for `ctas` CTAs (part_ml needs 1/32 of it)
 size_t attention_scratch_floats(int ctas);
 // Host walk of the attention work split over `ctas` CTAs (0: every property holds)
-int attention_schedule_check(int L, int Lp, int N, int heads, int mode, int kv_len, int images, int ctas);
+int attention_schedule_check(int L, int Lp, int N, int heads, int mode, int kv_len, int images, int ctas,
+                             int p_lo = 0, int p_hi = 0);
 int sm_count();
 // V operand of the attention: [heads][rows][64] bf16 (rows a multiple of 4, every KV tile
 // starting at a multiple of 4) seen as a 5-D view whose 128-row box lands in shared memory

@@ -75,7 +75,7 @@ extern "C" DFP_API dfp_status dfp_group_norm_noalloc(const void* x, void* y, dfp
   const int vec = dtype == DFP_BF16 ? 8 : 4;
   if (C % vec || C / vec > 512) return fail(DFP_E_ARG, "C must be a multiple of 16 bytes of elements and C/vector <= 512");
   if (n_patches * groups > 256) return fail(DFP_E_ARG, "n_patches * groups must be <= 256");
-  if (mode != DFP_GN_CORRECTED && mode != DFP_GN_STALE_OTHERS) return fail(DFP_E_ARG, "unknown gn mode");
+  if (mode < DFP_GN_CORRECTED || mode > DFP_GN_SEPARATE) return fail(DFP_E_ARG, "unknown gn mode");
   if (!(eps >= 0.f)) return fail(DFP_E_ARG, "eps must be >= 0");
   if ((long long)H * W * C >= (1ll << 31)) return fail(DFP_E_ARG, "feature map too large");
   // the kernels read x while writing y, and read stale_moments after writing fresh_moments

@@ -122,7 +122,9 @@ __device__ __forceinline__ void tile_src(int mode, int p, int Lp, int L, int kv_
 
 // The unit list: patch-major over the images' patches (patch pg = img * N + p, so Q and O
 // rows start at pg * Lp), then head, then Q-tile pair; unit (pg, head, pair) has
-// unit_tiles(pg % N) KV tiles.  Global tile x -> its unit and the unit's first tile.
+// unit_tiles(pg % N) KV tiles.  Only the query patches [p_lo, p_hi) are listed (all of them
+// unless a patch-parallel rank computes a range).  Global tile x -> its unit and the unit's
+// first tile.
 // All schedule arithmetic is 32-bit: the launcher checks total_tiles * ctas < 2^31.
 struct Unit {
   int p, head, pair, T, U0;   // p: patch over the batch (img * N + patch within the image)
@@ -130,7 +132,7 @@ struct Unit {
 __host__ __device__ __forceinline__ Unit locate(const TcAttnArgs& a, int n_pairs, int x) {
   int base = 0;
   Unit u{};
-  for (int p = 0; p < a.N * a.images; ++p) {
+  for (int p = a.p_lo; p < a.p_hi; ++p) {
     const int T = unit_tiles(a.mode, p % a.N, a.Lp, a.L, a.kv_len);
     const int blk = T * a.heads * n_pairs;
     if (x < base + blk) {
@@ -872,8 +874,8 @@ bool encode_attn_v(CUtensorMap* m, const void* base, uint64_t rows, uint64_t hea
 long long attention_total_tiles(const TcAttnArgs& a) {
   const int n_pairs = (a.n_qtiles + 1) / 2;
   long long tt = 0;
-  for (int p = 0; p < a.N; ++p) tt += (long long)unit_tiles(a.mode, p, a.Lp, a.L, a.kv_len) * a.heads * n_pairs;
-  return tt * a.images;
+  for (int p = a.p_lo; p < a.p_hi; ++p) tt += (long long)unit_tiles(a.mode, p % a.N, a.Lp, a.L, a.kv_len) * a.heads * n_pairs;
+  return tt;
 }
 
 size_t attention_scratch_floats(int ctas) { return (size_t)ctas * 256 * 64; }
@@ -896,6 +898,8 @@ cudaError_t launch_tc_attention(const TcAttnArgs& args, const CUtensorMap& mq, c
   if (regs * kThreads < 128 * kRegsTmaMma + 512 * kRegsSoftmax) return cudaErrorInvalidConfiguration;
   TcAttnArgs a = args;
   if (a.images < 1 || a.kv_stride < 0) return cudaErrorInvalidValue;
+  if (a.p_lo == 0 && a.p_hi == 0) a.p_hi = a.N * a.images;   // every query patch
+  if (a.p_lo < 0 || a.p_hi > a.N * a.images || a.p_lo >= a.p_hi) return cudaErrorInvalidValue;
   // a fresh flag value per launch (flags hold the epoch of the launch that last set them)
   static std::atomic<unsigned> epoch{0};
   do a.epoch = ++epoch; while (a.epoch == 0);
@@ -919,11 +923,14 @@ cudaError_t launch_tc_attention(const TcAttnArgs& args, const CUtensorMap& mq, c
 
 // Host walk of the work split exactly as the kernel's three walkers do it (the same
 // locate / advance / cta_of / range_start), checking what the cut-pair merge relies on.
-int attention_schedule_check(int L, int Lp, int N, int heads, int mode, int kv_len, int images, int ctas) {
+int attention_schedule_check(int L, int Lp, int N, int heads, int mode, int kv_len, int images, int ctas,
+                             int p_lo, int p_hi) {
   TcAttnArgs a{};
   a.L = L; a.Lp = Lp; a.N = N; a.heads = heads; a.mode = mode; a.kv_len = kv_len; a.images = images;
+  a.p_lo = p_lo; a.p_hi = p_hi > 0 ? p_hi : N * images;
   a.n_qtiles = cdiv(Lp, kTile);
   if (L <= 0 || Lp <= 0 || N <= 0 || heads <= 0 || images < 1 || ctas < 1) return 1;
+  if (a.p_lo < 0 || a.p_hi > N * images || a.p_lo >= a.p_hi) return 1;
   const int n_pairs = (a.n_qtiles + 1) / 2;
   const long long tt = attention_total_tiles(a);
   if (tt <= 0) return 1;

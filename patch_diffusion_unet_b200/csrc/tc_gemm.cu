@@ -40,14 +40,15 @@ __device__ __forceinline__ TileInfo tile_of(const TcGemmPlan& pl, int m_tile) {
   TileInfo t{};
   if (pl.conv) {
     const int per_patch = (pl.R / pl.rows_tile) * pl.tiles_per_row;
-    t.p = m_tile / per_patch;
-    const int rem = m_tile - t.p * per_patch;
+    const int lp = m_tile / per_patch;
+    t.p = pl.p0 + lp;
+    const int rem = m_tile - lp * per_patch;
     const int it = rem / pl.tiles_per_row;
     const int jt = rem - it * pl.tiles_per_row;
     t.i0 = it * pl.rows_tile;
     t.j0 = jt * pl.cols_tile;
   } else {
-    t.m0 = m_tile * kBM;
+    t.m0 = pl.m_base + m_tile * kBM;
   }
   return t;
 }
@@ -601,7 +602,10 @@ GemmChoice choose_gemm(int N, int m_tiles, int k_stages, int force_bn) {
 cudaError_t launch_tc_gemm(const TcGemmPlan& plan_in, const CUtensorMap& mapA, const CUtensorMap& mapB,
                            const Epilogue& epi, int* err, cudaStream_t s) {
   TcGemmPlan plan = plan_in;
-  plan.m_tiles = plan.conv ? plan.P * (plan.R / plan.rows_tile) * plan.tiles_per_row : (plan.M + kBM - 1) / kBM;
+  // conv: tiles of patches [p0, p0 + P); plain: rows [m_base, M)
+  plan.m_tiles = plan.conv ? plan.P * (plan.R / plan.rows_tile) * plan.tiles_per_row
+                           : (plan.M - plan.m_base + kBM - 1) / kBM;
+  if (plan.m_tiles <= 0) return cudaErrorInvalidValue;
   plan.sms = sm_count();
   // as many two-chunk stages as fit in ~220 KB of shared memory
   if (plan.pair) {

@@ -15,7 +15,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdfp.so"
 OK, E_ARG, E_STATE, E_CUDA, E_NOMEM, E_UNSUPPORTED, E_DEVICE = range(7)
 F32, BF16 = 0, 1
 BLOCK_RES_ATTN, BLOCK_SDXL_STAGE = 0, 1
-GN_CORRECTED, GN_STALE_OTHERS = 0, 1
+GN_CORRECTED, GN_STALE_OTHERS, GN_SYNC, GN_SEPARATE = 0, 1, 2, 3
 CTX_DISPLACED, CTX_NAIVE = 0, 1
 FAMILY_TENSOR_CORE, FAMILY_SIMT = 0, 1
 
@@ -25,7 +25,7 @@ EXPORTED = ("dfp_create", "dfp_load_weights", "dfp_step", "dfp_step_host", "dfp_
             "dfp_set_kernel_family", "dfp_set_profiling", "dfp_kernel_times", "dfp_destroy",
             "dfp_last_error", "dfp_group_norm_noalloc", "dfp_group_norm_noalloc_error",
             "dfp_selftest_wait_timeout", "dfp_selftest_exp2_poly", "dfp_set_launch_overlap",
-            "dfp_attention_schedule_check")
+            "dfp_attention_schedule_check", "dfp_step_patches", "dfp_context_buffer")
 
 
 class Config(ctypes.Structure):
@@ -63,7 +63,10 @@ def load_library(path=_LIB_PATH):
         "dfp_launches_per_step": ([H], ctypes.c_int),
         "dfp_set_kernel_family": ([H, ctypes.c_int], ctypes.c_int),
         "dfp_set_launch_overlap": ([H, ctypes.c_int], ctypes.c_int),
-        "dfp_attention_schedule_check": ([ctypes.c_int] * 8, ctypes.c_int),
+        "dfp_attention_schedule_check": ([ctypes.c_int] * 10, ctypes.c_int),
+        "dfp_step_patches": ([H, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int], ctypes.c_int),
+        "dfp_context_buffer": ([H, ctypes.c_char_p, ctypes.c_int, ctypes.POINTER(ctypes.c_void_p),
+                                ctypes.POINTER(ctypes.c_longlong)], ctypes.c_int),
         "dfp_set_profiling": ([H, ctypes.c_int], ctypes.c_int),
         "dfp_kernel_times": ([H, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_char_p), ctypes.c_int],
                              ctypes.c_int),

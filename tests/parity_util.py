@@ -57,7 +57,7 @@ def run_parity(cfg, n_steps, oracle_from=0, query_tokens=None, gn_mode=0, contex
     if family is not None:
         blk.set_kernel_family(family)
     blk.load_weights(wl.weights)
-    omode = ["corrected", "stale_others"][gn_mode]
+    omode = ["corrected", "stale_others", "sync", "separate"][gn_mode]
     octx = ["displaced", "naive"][context]
     orc = oracle.make_block(cfg, wl.weights, wl.context, gn_mode=omode, context=octx)
     sched = wl.schedule()[:n_steps]

@@ -13,9 +13,9 @@ SYNC, DISPLACED, NAIVE, CROSS = 0, 1, 2, 3
 CTAS = [148, 147, 132, 100, 64, 37, 7, 2, 1]
 
 
-def _check(L, Lp, N, heads, mode, kv_len=0, images=1, ctas=148):
+def _check(L, Lp, N, heads, mode, kv_len=0, images=1, ctas=148, p_lo=0, p_hi=0):
     from patch_diffusion_unet_b200 import dfp
-    return dfp.LIB.dfp_attention_schedule_check(L, Lp, N, heads, mode, kv_len, images, ctas)
+    return dfp.LIB.dfp_attention_schedule_check(L, Lp, N, heads, mode, kv_len, images, ctas, p_lo, p_hi)
 
 
 # (L, Lp, N, heads) of the workloads: 64x64 / 128x128 / 240x240 maps, the stage's 20 heads,
@@ -53,7 +53,23 @@ def test_random_splits():
         assert _check(N * Lp, Lp, N, heads, mode, images=images, ctas=ctas) == 0, (N, Lp, heads, mode, images, ctas)
 
 
+@pytest.mark.parametrize("shape", SHAPES[:3], ids=["L4096", "L16384", "L57600"])
+@pytest.mark.parametrize("world", [2, 4, 8])
+def test_patch_range_split(shape, world):
+    """A patch-parallel rank lists only its own query patches: every rank's range of the
+    displaced step splits as cleanly as the whole list."""
+    L, Lp, N, heads = shape
+    if N % world:
+        pytest.skip("patches do not divide among the ranks")
+    per = N // world
+    for r in range(world):
+        for ctas in CTAS:
+            assert _check(L, Lp, N, heads, DISPLACED, ctas=ctas, p_lo=r * per, p_hi=(r + 1) * per) == 0, (r, ctas)
+
+
 def test_bad_arguments():
+    assert _check(4096, 1024, 4, 10, DISPLACED, p_lo=3, p_hi=3) == 1
+    assert _check(4096, 1024, 4, 10, DISPLACED, p_lo=0, p_hi=5) == 1
     assert _check(0, 0, 1, 1, SYNC) == 1
     assert _check(4096, 1024, 4, 10, 9) == 1
     assert _check(4096, 1024, 4, 10, SYNC, ctas=0) == 1

@@ -36,7 +36,8 @@ def _sample(L, n, seed=1):
 
 # ------------------------------------------------------------------ config 0 (fp32, SIMT)
 
-@pytest.mark.parametrize("gn_mode,context", [(0, 0), (1, 0), (0, 1)], ids=["corrected", "stale_others", "naive"])
+@pytest.mark.parametrize("gn_mode,context", [(0, 0), (1, 0), (2, 0), (3, 0), (0, 1)],
+                         ids=["corrected", "stale_others", "gn_sync", "gn_separate", "naive"])
 def test_config0_fp32_all_steps(gn_mode, context):
     cfg = configs.get(0)
     res = run_parity(cfg, cfg["steps"], gn_mode=gn_mode, context=context)
@@ -134,10 +135,12 @@ def test_peaked_attention_bf16():
     _assert(run_parity(cfg, cfg["steps"], weight_scale=scale), TOL["bf16"])
 
 
-@pytest.mark.parametrize("gn_mode,context", [(1, 0), (0, 1)], ids=["stale_others", "naive"])
-def test_modes_bf16(gn_mode, context):
+@pytest.mark.parametrize("gn_mode,context", [(1, 0), (2, 0), (3, 0), (0, 1)],
+                         ids=["stale_others", "gn_sync", "gn_separate", "naive"])
+@pytest.mark.parametrize("family", [0, 1], ids=["tcgen05", "simt"])
+def test_modes_bf16(gn_mode, context, family):
     cfg = RAGGED[1]
-    _assert(run_parity(cfg, cfg["steps"], gn_mode=gn_mode, context=context), TOL["bf16"])
+    _assert(run_parity(cfg, cfg["steps"], gn_mode=gn_mode, context=context, family=family), TOL["bf16"])
 
 
 # ------------------------------------------------------------------ configs 1-3 (full sizes)

@@ -162,6 +162,71 @@ def test_naive_context_equals_independent_patches():
         _close(y[p * R:(p + 1) * R].reshape(-1, cfg["C"]), ref)
 
 
+# --------------------------------------------------------------------------- GroupNorm-only modes (R8)
+
+def _gn_lib(x, G, gamma, beta, eps, silu):
+    """PyTorch's group_norm (+ SiLU) on one [rows, W, C] map, fp64."""
+    X = torch_ref._nchw(x)
+    y = torch.nn.functional.group_norm(X, G, torch_ref._t(gamma), torch_ref._t(beta), eps)
+    return torch_ref._nhwc(torch.nn.functional.silu(y) if silu else y)
+
+
+@pytest.mark.parametrize("N", [2, 4])
+def test_gn_sync_mode_displaced_step_normalises_with_the_full_map(N):
+    """GroupNorm 'sync' mode: on a displaced step both GroupNorms equal PyTorch's group_norm
+    over the whole map of this step, while the conv and the attention stay displaced
+    (the output differs from the full layer)."""
+    cfg = configs.get(SMALL, n_patches=N)
+    wl = inputs.SyntheticWorkload(cfg, random_affine=True)
+    w = wl.weights
+    blk = _block(cfg, wl, gn_mode="sync")
+    blk.step(wl.x(0), 0, 1)
+    x = wl.x(1).astype(np.float64)
+    out = blk.step(x, 1, 0)
+    G, eps = cfg["gn_groups"], cfg["gn_eps"]
+    _close(out["y1"], _gn_lib(x, G, w["gn1.weight"], w["gn1.bias"], eps, True))
+    _close(out["t"], _gn_lib(out["h"], G, w["gn2.weight"], w["gn2.bias"], eps, False))
+    assert np.abs(out["y"] - _full(cfg, x, wl)["y"]).max() > 1e-6
+
+
+@pytest.mark.parametrize("N", [2, 4])
+def test_gn_separate_mode_displaced_step_normalises_each_patch_alone(N):
+    """GroupNorm 'separate' mode: on a displaced step each patch's GroupNorm equals
+    PyTorch's group_norm of that patch alone; the synchronous step stays the full layer."""
+    cfg = configs.get(SMALL, n_patches=N)
+    wl = inputs.SyntheticWorkload(cfg, random_affine=True)
+    w = wl.weights
+    blk = _block(cfg, wl, gn_mode="separate")
+    x0 = wl.x(0).astype(np.float64)
+    _close(blk.step(x0, 0, 1)["y"], _full(cfg, x0, wl)["y"])
+    x = wl.x(1).astype(np.float64)
+    out = blk.step(x, 1, 0)
+    G, eps, R = cfg["gn_groups"], cfg["gn_eps"], cfg["H"] // N
+    for p in range(N):
+        rows = slice(p * R, (p + 1) * R)
+        _close(out["y1"][rows], _gn_lib(x[rows], G, w["gn1.weight"], w["gn1.bias"], eps, True))
+        _close(out["t"][rows], _gn_lib(out["h"][rows], G, w["gn2.weight"], w["gn2.bias"], eps, False))
+
+
+@pytest.mark.parametrize("mode", ["sync", "separate"])
+def test_gn_modes_n1_and_stale_equal_fresh_give_full_layer(mode):
+    """N = 1 at every step, and a displaced step whose cache holds this very map (sync
+    mode), reproduce the full layer."""
+    cfg = configs.get(SMALL, n_patches=1)
+    wl = inputs.SyntheticWorkload(cfg, random_affine=True)
+    blk = _block(cfg, wl, gn_mode=mode)
+    for t in range(3):
+        x = wl.x(t).astype(np.float64)
+        _close(blk.step(x, t, int(t == 0))["y"], _full(cfg, x, wl)["y"])
+    if mode == "sync":
+        cfg = configs.get(SMALL, n_patches=4)
+        wl = inputs.SyntheticWorkload(cfg, random_affine=True)
+        blk = _block(cfg, wl, gn_mode=mode)
+        x = wl.x(0).astype(np.float64)
+        blk.step(x, 0, 1)
+        _close(blk.step(x, 1, 0)["y"], _full(cfg, x, wl)["y"])
+
+
 # --------------------------------------------------------------------------- layer-level pins
 
 def test_conv_halo_locality():

@@ -23,7 +23,7 @@ from tests.parity_util import TOL, rel_l2
 
 pytestmark = pytest.mark.gpu
 
-MODES = {0: oracle.GN_CORRECTED, 1: oracle.GN_STALE_OTHERS}
+MODES = {0: oracle.GN_CORRECTED, 1: oracle.GN_STALE_OTHERS, 2: oracle.GN_SYNC, 3: oracle.GN_SEPARATE}
 
 
 def _call(dfp, x, y, dtype, cfg, gamma, beta, stale, mode, silu, fresh, mr):
@@ -36,7 +36,7 @@ def _call(dfp, x, y, dtype, cfg, gamma, beta, stale, mode, silu, fresh, mr):
 
 
 @pytest.mark.parametrize("cid", [0, 1], ids=["fp32-16x16x64", "bf16-64x64x640"])
-@pytest.mark.parametrize("mode", [0, 1], ids=["corrected", "stale_others"])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3], ids=["corrected", "stale_others", "gn_sync", "gn_separate"])
 @pytest.mark.parametrize("silu,keep_mr", [(True, True), (False, False)], ids=["silu", "no-silu-no-mean_rstd"])
 def test_noalloc_matches_oracle_two_calls(cid, mode, silu, keep_mr):
     from patch_diffusion_unet_b200 import dfp
