@@ -12,8 +12,10 @@
 //   o, y        [B*L][C]         attention output, block output
 //   mom1/2[2]   [B*N][G][2] fp32 per-(patch, group) (mean, variance) of GN1 / GN2, alternating
 //   part        fp32 scratch     per-chunk partial sums of the GroupNorm statistics
+#include <atomic>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <new>
@@ -31,6 +33,17 @@ using namespace dfp;
 
 namespace dfp {
 size_t dtype_size(dfp_dtype d) { return d == DFP_BF16 ? 2 : 4; }
+
+bool alloc_fault_injected() {
+  static std::atomic<long long> attempts{0};
+  const char* v = std::getenv("DFP_FAULT_ALLOC_AFTER");
+  if (!v || !*v) {
+    attempts.store(0);
+    return false;
+  }
+  const long long k = std::atoll(v);
+  return attempts.fetch_add(1) >= k;
+}
 }  // namespace dfp
 
 namespace {
@@ -441,18 +454,23 @@ dfp_status dfp_step_host_async(dfp_handle h, const void* x_host, void* y_host, i
   if (!x_host || !y_host) return h->fail(DFP_E_ARG, "x_host / y_host is NULL");
   const size_t bytes = (size_t)h->B * h->L * h->cfg.C * h->esz;
   cudaError_t e = cudaSuccess;
-  if (!h->s_in) {
-    e = cudaStreamCreateWithFlags(&h->s_in, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->s_out, cudaStreamNonBlocking);
+  if (!h->async_ready) {
+    // set up on first use; a failed set-up leaves nothing behind, so a later call retries
+    if (!h->s_in) e = cudaStreamCreateWithFlags(&h->s_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess && !h->s_out) e = cudaStreamCreateWithFlags(&h->s_out, cudaStreamNonBlocking);
     for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
-      e = cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming);
-      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_done[i], cudaEventDisableTiming);
-      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming);
+      if (!h->ev_in[i]) e = cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming);
+      if (e == cudaSuccess && !h->ev_done[i]) e = cudaEventCreateWithFlags(&h->ev_done[i], cudaEventDisableTiming);
+      if (e == cudaSuccess && !h->ev_out[i]) e = cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming);
     }
     if (e != cudaSuccess) return h->cuda_fail(e, "async host step set-up");
     bool ok = true;
     for (int i = 0; i < 2; ++i) ok = ok && h->alloc(&h->xin2[i], bytes) && h->alloc(&h->ystage[i], bytes);
-    if (!ok) return h->fail(DFP_E_NOMEM, "device allocation failed");
+    if (!ok) {
+      for (int i = 0; i < 2; ++i) { h->release(h->xin2[i]); h->release(h->ystage[i]); }
+      return h->fail(DFP_E_NOMEM, "device allocation failed");
+    }
+    h->async_ready = true;
   }
   const int b = (int)(h->n_async & 1);
   const bool reuse = h->n_async >= 2;   // buffer b was used two calls ago

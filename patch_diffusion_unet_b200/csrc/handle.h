@@ -14,6 +14,11 @@ namespace dfp {
 struct Stage;
 void delete_stage(Stage* s);
 size_t dtype_size(dfp_dtype d);
+// Host-side fault injection for allocation failure: while the environment variable
+// DFP_FAULT_ALLOC_AFTER=k is set, the first k device allocations the library attempts
+// succeed and every later one fails as if the device were out of memory (the count
+// restarts when the variable is unset).  Returns true if this attempt must fail.
+bool alloc_fault_injected();
 }  // namespace dfp
 
 struct dfp_ctx {
@@ -26,6 +31,7 @@ struct dfp_ctx {
   void* ystage[2] = {nullptr, nullptr};
   cudaEvent_t ev_in[2] = {}, ev_done[2] = {}, ev_out[2] = {};
   long long n_async = 0;       // asynchronous host steps issued so far
+  bool async_ready = false;    // the streams, events and buffers above are all set up
   std::string err;
   int R = 0, L = 0, Lp = 0, family = 0;
   int B = 1;                   // images per step (the guidance batch); L, Lp are per image
@@ -77,9 +83,17 @@ struct dfp_ctx {
     return DFP_E_CUDA;
   }
   bool alloc(void** p, size_t bytes) {
-    if (cudaMalloc(p, bytes) != cudaSuccess) { *p = nullptr; return false; }
+    if (dfp::alloc_fault_injected() || cudaMalloc(p, bytes) != cudaSuccess) { *p = nullptr; return false; }
     allocs.push_back(*p);
     return true;
+  }
+  // Free one allocation made by alloc() (and forget it).
+  void release(void*& p) {
+    if (!p) return;
+    for (size_t i = 0; i < allocs.size(); ++i)
+      if (allocs[i] == p) { allocs.erase(allocs.begin() + i); break; }
+    cudaFree(p);
+    p = nullptr;
   }
 };
 
