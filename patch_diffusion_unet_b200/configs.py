@@ -13,10 +13,13 @@ n_patches   number of row patches N (patch p owns rows [p*H/N, (p+1)*H/N))
 gn_groups   GroupNorm groups G;  gn_eps the GroupNorm epsilon
 heads, head_dim   self-attention heads x head width (heads*head_dim == C)
 dtype       storage / MMA operand type ("f32" or "bf16")
-block       "res_attn" (GN+SiLU, conv3x3, GN, self-attention)
-            or "sdxl_stage" (ResNet block + transformer blocks)
+block       "res_attn" (GN+SiLU, conv3x3, GN, self-attention),
+            "sdxl_stage" (ResNet block + transformer blocks)
+            or "unet" (the multi-level UNet of a whole denoising step)
 steps, n_sync     denoising steps in a run and how many of the first are synchronous
 n_xformer, ffn_inner, ctx_len, ctx_dim   transformer-stage extras (sdxl_stage only)
+widths, latent_c    UNet level widths (full, half, quarter resolution) and latent channels;
+ddim_train_steps, beta_start, beta_end   the DDIM schedule (unet only)
 """
 
 CONFIGS = {
@@ -35,6 +38,12 @@ CONFIGS = {
     4: dict(name="sdxl-stage-64x64x1280-n8-bf16", H=64, W=64, C=1280, n_patches=8, gn_groups=32,
             gn_eps=1e-5, heads=20, head_dim=64, dtype="bf16", block="sdxl_stage",
             steps=50, n_sync=5, n_xformer=2, ffn_inner=5120, ctx_len=77, ctx_dim=2048),
+    # the multi-level UNet of a 1024 px image and its 50-step DDIM loop (latent 128x128x4;
+    # levels 128^2 / 64^2 / 32^2 with 320 / 640 / 1280 channels, 8 row patches at every level)
+    5: dict(name="sdxl-unet-1024-128x128-n8-bf16", H=128, W=128, C=320, n_patches=8, gn_groups=32,
+            gn_eps=1e-5, heads=5, head_dim=64, dtype="bf16", block="unet", steps=50, n_sync=5,
+            widths=(320, 640, 1280), latent_c=4, ctx_len=77, ctx_dim=2048,
+            ddim_train_steps=1000, beta_start=0.00085, beta_end=0.012),
 }
 
 

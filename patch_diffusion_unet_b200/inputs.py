@@ -53,6 +53,8 @@ def to_torch(a32, dtype):
 
 def fixed_specs(cfg):
     """Norm affine parameters (not drawn): list of (name, shape, fill)."""
+    if cfg["block"] == "unet":
+        return unet_fixed_specs(cfg)
     C = cfg["C"]
     out = []
     if cfg["block"] == "res_attn":
@@ -70,6 +72,8 @@ def fixed_specs(cfg):
 def weight_specs(cfg):
     """Drawn weights in declaration order: list of (name, shape), PyTorch layouts
     (conv [Cout, Cin, 3, 3], linear [out, in])."""
+    if cfg["block"] == "unet":
+        return unet_weight_specs(cfg)
     C = cfg["C"]
     if cfg["block"] == "res_attn":
         return [
@@ -96,6 +100,61 @@ def weight_specs(cfg):
             (p + "ff.out.weight", (C, F)), (p + "ff.out.bias", (C,)),
         ]
     return specs
+
+
+def unet_weight_specs(cfg):
+    """Drawn weights of the multi-level UNet (name, shape) in declaration order, PyTorch
+    layouts: timestep MLP, conv_in, per level a ResNet block (1x1 shortcut when the width
+    changes), transformer blocks at the two lower levels, down / up convs, conv_out."""
+    c0, c1, c2 = cfg["widths"]
+    D, lat = cfg["ctx_dim"], cfg["latent_c"]
+    specs = [("time_embedding.linear_1.weight", (4 * c0, c0)), ("time_embedding.linear_1.bias", (4 * c0,)),
+             ("time_embedding.linear_2.weight", (4 * c0, 4 * c0)), ("time_embedding.linear_2.bias", (4 * c0,)),
+             ("conv_in.weight", (c0, lat, 3, 3)), ("conv_in.bias", (c0,))]
+
+    def resnet(p, ci, co):
+        s = [(p + "conv1.weight", (co, ci, 3, 3)), (p + "conv1.bias", (co,)),
+             (p + "time_emb_proj.weight", (co, 4 * c0)), (p + "time_emb_proj.bias", (co,)),
+             (p + "conv2.weight", (co, co, 3, 3)), (p + "conv2.bias", (co,))]
+        if ci != co:
+            s += [(p + "conv_shortcut.weight", (co, ci)), (p + "conv_shortcut.bias", (co,))]
+        return s
+
+    def xf(p, c):
+        F = 4 * c
+        return [(p + "attn1.to_q.weight", (c, c)), (p + "attn1.to_k.weight", (c, c)), (p + "attn1.to_v.weight", (c, c)),
+                (p + "attn1.to_out.weight", (c, c)), (p + "attn1.to_out.bias", (c,)),
+                (p + "attn2.to_q.weight", (c, c)), (p + "attn2.to_k.weight", (c, D)), (p + "attn2.to_v.weight", (c, D)),
+                (p + "attn2.to_out.weight", (c, c)), (p + "attn2.to_out.bias", (c,)),
+                (p + "ff.proj.weight", (2 * F, c)), (p + "ff.proj.bias", (2 * F,)),
+                (p + "ff.out.weight", (c, F)), (p + "ff.out.bias", (c,))]
+
+    specs += resnet("down0.resnet.", c0, c0)
+    specs += [("down0.downsample.weight", (c0, c0, 3, 3)), ("down0.downsample.bias", (c0,))]
+    specs += resnet("down1.resnet.", c0, c1) + xf("down1.xf.", c1)
+    specs += [("down1.downsample.weight", (c1, c1, 3, 3)), ("down1.downsample.bias", (c1,))]
+    specs += resnet("down2.resnet.", c1, c2) + xf("down2.xf.", c2)
+    specs += [("up1.upsample.weight", (c2, c2, 3, 3)), ("up1.upsample.bias", (c2,))]
+    specs += resnet("up1.resnet.", c2 + c1, c1) + xf("up1.xf.", c1)
+    specs += [("up0.upsample.weight", (c1, c1, 3, 3)), ("up0.upsample.bias", (c1,))]
+    specs += resnet("up0.resnet.", c1 + c0, c0)
+    specs += [("conv_out.weight", (lat, c0, 3, 3)), ("conv_out.bias", (lat,))]
+    return specs
+
+
+def unet_fixed_specs(cfg):
+    """Norm scales / shifts of the UNet (name, shape, fill): 1 and 0, not drawn."""
+    c0, c1, c2 = cfg["widths"]
+    out = []
+    for p, ci, co in (("down0.resnet.", c0, c0), ("down1.resnet.", c0, c1), ("down2.resnet.", c1, c2),
+                      ("up1.resnet.", c2 + c1, c1), ("up0.resnet.", c1 + c0, c0)):
+        out += [(p + "norm1.weight", (ci,), 1.0), (p + "norm1.bias", (ci,), 0.0),
+                (p + "norm2.weight", (co,), 1.0), (p + "norm2.bias", (co,), 0.0)]
+    for p, c in (("down1.xf.", c1), ("down2.xf.", c2), ("up1.xf.", c1)):
+        for n in ("norm1", "norm2", "norm3"):
+            out += [(p + n + ".weight", (c,), 1.0), (p + n + ".bias", (c,), 0.0)]
+    out += [("norm_out.weight", (c0,), 1.0), ("norm_out.bias", (c0,), 0.0)]
+    return out
 
 
 class SyntheticWorkload:
@@ -127,11 +186,19 @@ class SyntheticWorkload:
         # image b >= 1 of a batch: its own stream for its context and its inputs
         self.rngs = [self.rng] + [np.random.default_rng([seed, b]) for b in range(1, self.batch)]
         self.context = None
-        if cfg["block"] == "sdxl_stage":
+        if cfg["block"] in ("sdxl_stage", "unet"):
             ctx = [round_to(r.standard_normal((cfg["ctx_len"], cfg["ctx_dim"])), self.dtype) for r in self.rngs]
             self.context = ctx[0] if self.batch == 1 else np.stack(ctx)
         self._state = None   # fp64 x_t, one per image
         self._t = -1
+
+    def latent(self):
+        """The UNet workload's starting latent x_T ~ N(0, 1), [H, W, latent_c] (drawn after the
+        context from the main stream; the DDIM loop evolves it from there)."""
+        if not hasattr(self, "_latent"):
+            shape = (self.cfg["H"], self.cfg["W"], self.cfg["latent_c"])
+            self._latent = round_to(self.rng.standard_normal(shape), self.dtype)
+        return self._latent
 
     def x(self, t):
         """Layer input of step t (must be requested in order 0, 1, 2, ...; repeats allowed)."""

@@ -136,3 +136,63 @@ def sdxl_stage_full_batched(xs, w, ctxs, cfg):
         a, gate = hg.chunk(2, dim=-1)
         r = r + F.linear(a * F.gelu(gate), _t(w[p + "ff.out.weight"]), _t(w[p + "ff.out.bias"]))
     return dict(y=r.numpy())
+
+
+# ---------------------------------------------------------------- the multi-level UNet
+# The whole (unpatched) network of the UNet workload with PyTorch's routines: strided
+# conv2d for the downsampling, interpolate(nearest) for the upsampling, cat for the skips.
+
+def unet_full(x, w, ctx, cfg, tau):
+    """Predicted noise of the UNet for latent x [H, W, latent_c] at timestep tau."""
+    import math
+    G, eps = cfg["gn_groups"], cfg["gn_eps"]
+    c0, c1, c2 = cfg["widths"]
+    half = c0 // 2
+    f = torch.exp(-math.log(10000.0) * torch.arange(half, dtype=torch.float64) / half)
+    e = torch.cat([torch.cos(float(tau) * f), torch.sin(float(tau) * f)])
+    temb = F.linear(F.silu(F.linear(e, _t(w["time_embedding.linear_1.weight"]), _t(w["time_embedding.linear_1.bias"]))),
+                    _t(w["time_embedding.linear_2.weight"]), _t(w["time_embedding.linear_2.bias"]))
+    ta = F.silu(temb)
+    c = _t(ctx)
+
+    def gn_silu(h, n):
+        return F.silu(F.group_norm(h, G, _t(w[n + ".weight"]), _t(w[n + ".bias"]), eps))
+
+    def conv(h, n, stride=1):
+        return F.conv2d(h, _t(w[n + ".weight"]), _t(w[n + ".bias"]), stride=stride, padding=1)
+
+    def resnet(h, p):
+        y = conv(gn_silu(h, p + "norm1"), p + "conv1") + \
+            F.linear(ta, _t(w[p + "time_emb_proj.weight"]), _t(w[p + "time_emb_proj.bias"]))[None, :, None, None]
+        y = conv(gn_silu(y, p + "norm2"), p + "conv2")
+        if p + "conv_shortcut.weight" in w:
+            h = F.conv2d(h, _t(w[p + "conv_shortcut.weight"])[:, :, None, None], _t(w[p + "conv_shortcut.bias"]))
+        return h + y
+
+    def xf(h, p):
+        _, C, H, W = h.shape
+        r = h[0].permute(1, 2, 0).reshape(H * W, C)
+
+        def ln(u, n):
+            return F.layer_norm(u, (C,), _t(w[p + n + ".weight"]), _t(w[p + n + ".bias"]), 1e-5)
+
+        r = r + _mha(ln(r, "norm1"), w[p + "attn1.to_q.weight"], w[p + "attn1.to_k.weight"], w[p + "attn1.to_v.weight"],
+                     w[p + "attn1.to_out.weight"], w[p + "attn1.to_out.bias"], C // 64)[0]
+        r = r + _mha(ln(r, "norm2"), w[p + "attn2.to_q.weight"], w[p + "attn2.to_k.weight"], w[p + "attn2.to_v.weight"],
+                     w[p + "attn2.to_out.weight"], w[p + "attn2.to_out.bias"], C // 64, ctx=c)[0]
+        hg = F.linear(ln(r, "norm3"), _t(w[p + "ff.proj.weight"]), _t(w[p + "ff.proj.bias"]))
+        a, gate = hg.chunk(2, dim=-1)
+        r = r + F.linear(a * F.gelu(gate), _t(w[p + "ff.out.weight"]), _t(w[p + "ff.out.bias"]))
+        return r.reshape(H, W, C).permute(2, 0, 1)[None]
+
+    up = lambda h: F.interpolate(h, scale_factor=2, mode="nearest")  # noqa: E731
+    h = conv(_nchw(x), "conv_in")
+    s0 = h = resnet(h, "down0.resnet.")
+    h = conv(h, "down0.downsample", stride=2)
+    s1 = h = xf(resnet(h, "down1.resnet."), "down1.xf.")
+    h = conv(h, "down1.downsample", stride=2)
+    mid = h = xf(resnet(h, "down2.resnet."), "down2.xf.")
+    h = xf(resnet(torch.cat([conv(up(h), "up1.upsample"), s1], 1), "up1.resnet."), "up1.xf.")
+    h = resnet(torch.cat([conv(up(h), "up0.upsample"), s0], 1), "up0.resnet.")
+    out = conv(gn_silu(h, "norm_out"), "conv_out")
+    return dict(eps=_nhwc(out), mid=_nhwc(mid), s0=_nhwc(s0), s1=_nhwc(s1), up0=_nhwc(h))
