@@ -85,6 +85,37 @@ def work_model(cfg):
             for k, v in wm.items()}
 
 
+def unet_flops(cfg):
+    """Algorithmic FLOPs of one UNet evaluation (2 per multiply-add; the stride-2 convs at
+    their own cost, the latent's 4 channels unpadded; the timestep MLP and the norms are
+    not counted): {part: FLOPs} and the total."""
+    H, W, lat = cfg["H"], cfg["W"], cfg["latent_c"]
+    c0, c1, c2 = cfg["widths"]
+    T = cfg["ctx_len"]
+    L0, L1, L2 = H * W, H * W // 4, H * W // 16
+
+    def conv(L, ci, co):
+        return 2.0 * L * 9 * ci * co
+
+    def res(L, ci, co):
+        return conv(L, ci, co) + conv(L, co, co) + (2.0 * L * ci * co if ci != co else 0.0)
+
+    def xf(L, c):
+        F = 4 * c
+        heads = c // 64
+        return (2.0 * L * c * 3 * c + 4.0 * L * L * 64 * heads + 2.0 * L * c * c +          # self-attention
+                2.0 * L * c * c + 4.0 * L * T * 64 * heads + 2.0 * L * c * c +             # cross-attention
+                2.0 * L * c * 2 * F + 2.0 * L * F * c)                                     # GEGLU feed-forward
+    parts = {
+        "conv_in": conv(L0, lat, c0), "res0": res(L0, c0, c0), "down0": conv(L1, c0, c0),
+        "res1": res(L1, c0, c1), "xf1": xf(L1, c1), "down1": conv(L2, c1, c1),
+        "res2": res(L2, c1, c2), "xf2": xf(L2, c2), "up1": conv(L1, c2, c2),
+        "ures1": res(L1, c2 + c1, c1), "uxf1": xf(L1, c1), "up0": conv(L0, c1, c1),
+        "ures0": res(L0, c1 + c0, c0), "conv_out": conv(L0, c0, lat),
+    }
+    return parts, sum(parts.values())
+
+
 def _work_model_one_image(cfg):
     H, W, C, N, heads = cfg["H"], cfg["W"], cfg["C"], cfg["n_patches"], cfg["heads"]
     L, d = H * W, cfg["head_dim"]
@@ -312,19 +343,34 @@ def run_reference(args, cfg):
         return 0
     import oracle
     wl = inputs.SyntheticWorkload(cfg)
-    blk = oracle.make_block(cfg, wl.weights, wl.context)
-    sample = oracle_query_sample(cfg)
     n_sync = cfg["n_sync"]
+    if cfg["block"] == "unet":
+        # the oracle UNet, whole steps (one UNet evaluation each) at the DDIM timesteps
+        from oracle import unet_oracle
+        net = unet_oracle.DisplacedUNet(cfg, wl.weights, wl.context)
+        taus, x = ddim_taus(cfg), wl.latent()
+        sample = None
+
+        def run(t, is_sync):
+            t0 = time.perf_counter()
+            net.step(x, t, is_sync, taus[t % len(taus)])
+            return time.perf_counter() - t0
+    else:
+        blk = oracle.make_block(cfg, wl.weights, wl.context)
+        sample = oracle_query_sample(cfg)
+
+        def run(t, is_sync):
+            return oracle_step_seconds(blk, cfg, wl.x(t), t, is_sync, sample)
     t = 0
     for t in range(n_sync):
-        oracle_step_seconds(blk, cfg, wl.x(t), t, 1, sample)
+        run(t, 1)
     for _ in range(args.warmup):
         t += 1
-        oracle_step_seconds(blk, cfg, wl.x(t), t, 0, sample)
+        run(t, 0)
     dt = 0.0
     for _ in range(args.steps):
         t += 1
-        dt += oracle_step_seconds(blk, cfg, wl.x(t), t, 0, sample)
+        dt += run(t, 0)
     threads = _oracle_threads()
     value = args.steps / dt
     L = cfg["H"] * cfg["W"]
@@ -344,6 +390,153 @@ def run_reference(args, cfg):
     return 0
 
 
+def ddim_taus(cfg, n_steps=50):
+    """The DDIM timesteps visited, largest first: (n - 1 - k) n_train / n + 1."""
+    ratio = cfg["ddim_train_steps"] // n_steps
+    return [(n_steps - 1 - k) * ratio + 1 for k in range(n_steps)]
+
+
+def oracle_unet_rate(cfg):
+    """The oracle UNet on the host cores: one displaced step after one synchronous step."""
+    from oracle import unet_oracle
+    wl = inputs.SyntheticWorkload(cfg)
+    net = unet_oracle.DisplacedUNet(cfg, wl.weights, wl.context)
+    taus = ddim_taus(cfg)
+    x = wl.latent()
+    net.step(x, 0, 1, taus[0])
+    t0 = time.perf_counter()
+    net.step(x, 1, 0, taus[1])
+    dt = time.perf_counter() - t0
+    return 1.0 / dt, _oracle_threads(), dt
+
+
+def run_unet(args, cfg):
+    """The multi-level UNet: a step is one displaced UNet evaluation (dfp_step at a DDIM
+    timestep); e2e is a whole DDIM run through dfp_ddim_sample with the starting latent
+    copied in from pinned host memory and the result copied out inside the timed region."""
+    import torch
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    import torch.distributed as dist
+    from patch_diffusion_unet_b200 import dfp
+    H, W = cfg["H"], cfg["W"]
+    wl = inputs.SyntheticWorkload(cfg)
+    blk = dfp.DisplacedPatchBlock(cfg)
+    blk.load_weights(dict(wl.weights, context=wl.context))
+    blk.set_launch_overlap(not args.no_overlap)
+    stream = blk.stream
+    rng = np.random.default_rng(1)
+    xs = [inputs.to_torch(inputs.round_to(rng.standard_normal((H, W, cfg["latent_c"])), "bf16"), "bf16").cuda()
+          for _ in range(4)]
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    taus = ddim_taus(cfg)
+
+    def step(t, is_sync):
+        blk.set_timestep(taus[t % len(taus)])
+        blk.step(xs[t % len(xs)], t, is_sync)
+
+    for t in range(cfg["n_sync"]):
+        step(t, 1)
+    t = cfg["n_sync"] - 1
+    gpu_index = os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local] if \
+        os.environ.get("CUDA_VISIBLE_DEVICES") else str(local)
+    sampler = ClockSampler(gpu_index)
+    for _ in range(args.warmup):
+        t += 1
+        step(t, 0)
+        flush.zero_()
+    blk.check_device()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        t += 1
+        ev[i][0].record(stream)
+        step(t, 0)
+        ev[i][1].record(stream)
+        flush.zero_()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    blk.check_device()
+    value, total_ms_max = replica_throughput(float(sum(a.elapsed_time(b) for a, b in ev)), args.steps, world, "cuda")
+    launches = blk.launches_per_step()
+    # per-kernel time shares (kernel names repeat across layers: summed per name and step)
+    blk.set_profiling(True)
+    per = {}
+    for _ in range(args.profile_steps):
+        t += 1
+        step(t, 0)
+        sums = {}
+        for name, ms in blk.kernel_times():
+            sums[name] = sums.get(name, 0.0) + ms
+        for k, v in sums.items():
+            per.setdefault(k, []).append(v)
+        flush.zero_()
+    blk.set_profiling(False)
+    kern_us = {k: 1e3 * statistics.mean(v) for k, v in per.items()}
+    # end to end: a DDIM run of the whole schedule through the public entry point
+    e2e = None
+    if not args.no_e2e:
+        n_steps = 50
+        xh = torch.from_numpy(np.ascontiguousarray(wl.latent(), np.float32)).pin_memory()
+        yh = torch.empty_like(xh).pin_memory()
+        xd = torch.empty_like(xh, device="cuda")
+        for rep in range(2):   # the first run warms up
+            torch.cuda.synchronize()
+            w0 = time.perf_counter()
+            with torch.cuda.stream(stream):
+                xd.copy_(xh, non_blocking=True)
+            out = blk.ddim_sample(xd, n_steps, cfg["n_sync"], cfg["ddim_train_steps"], cfg["beta_start"],
+                                  cfg["beta_end"])
+            with torch.cuda.stream(stream):
+                yh.copy_(out, non_blocking=True)
+            blk.synchronize()
+            e_total = time.perf_counter() - w0
+        e2e_rate, _ = replica_throughput(e_total * 1e3, n_steps, world, "cuda")
+        nbytes = H * W * cfg["latent_c"] * 4
+        e2e = {"value": e2e_rate, "unit": "unet-steps/s", "h2d_bytes_per_step": nbytes / n_steps,
+               "d2h_bytes_per_step": nbytes / n_steps, "steps": n_steps,
+               "api": "dfp_ddim_sample (50 DDIM steps, first n_sync synchronous), latent in and out through pinned host memory, wall clock",
+               "images_per_s": e2e_rate / n_steps}
+    pk, pk_src = peaks()
+    parts, total = unet_flops(cfg)
+    ms_step = total_ms_max / args.steps
+    ach = total / (ms_step * 1e-3) / 1e12
+    peak = pk.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    roof = {"kernel": "whole UNet step", "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+            "frac": ach / peak, "traffic": None, "peak_source": f"{pk_src} bf16 burst", "work_per_launch": total,
+            "us_per_launch": 1e3 * ms_step}
+    blk.close()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, threads, dt = oracle_unet_rate(cfg)
+        cpu = {"value": rate, "unit": "unet-steps/s", "cores": threads, "kind": "oracle",
+               "sample": f"1 displaced UNet step of {cfg['name']} after 1 sync step ({dt:.1f} s)"}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "unet-steps/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random weights, random latents)",
+            "latent_px_per_s": value * H * W, "tensor_tflops_per_step": ach,
+            "config": {"workload": cfg["name"], "H": H, "W": W, "widths": list(cfg["widths"]),
+                       "n_patches": cfg["n_patches"], "parallelism": f"replicas{world}",
+                       "l2": "flushed between timed steps (512 MB write, outside the events)",
+                       "step": "displaced UNet evaluation (is_sync=0)"},
+            "gpu_launches": launches * args.steps, "launches_per_step": launches,
+            "kernels_us": {k: round(v, 2) for k, v in kern_us.items()},
+            "flops_per_part_g": {k: round(v / 1e9, 2) for k, v in parts.items()},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     cfg = configs.get(args.config)
@@ -352,6 +545,8 @@ def main():
         cfg = configs.get(cfg, batch=B, name=f"{cfg['name']}-b{B}")
     if args.impl == "reference":
         return run_reference(args, cfg)
+    if cfg["block"] == "unet":
+        return run_unet(args, cfg)
 
     import torch
     world, rank, local = dist_setup()

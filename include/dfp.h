@@ -60,7 +60,20 @@ typedef enum { DFP_F32 = 0, DFP_BF16 = 1 } dfp_dtype;
 
 typedef enum {
   DFP_BLOCK_RES_ATTN = 0,   /* GN+SiLU -> conv3x3 -> GN -> self-attention (Q,K,V,O) */
-  DFP_BLOCK_SDXL_STAGE = 1  /* ResNet block + transformer blocks                     */
+  DFP_BLOCK_SDXL_STAGE = 1, /* ResNet block + transformer blocks                     */
+  /* A whole SDXL-shaped UNet (project README, Performance: SDXL, 50-step DDIM; source
+   * walkthrough, Patch Parallelism: every conv, norm and attention layer of the UNet is
+   * wrapped): latent [H, W, 4]; levels H, H/2, H/4 with widths C, 2C, 4C; one ResNet block
+   * per level (timestep embedding added after its first conv), transformer blocks at the
+   * two lower levels, stride-2 convs down, nearest x2 + conv up, skip concatenation;
+   * every conv, GroupNorm and self-attention displaced, the same N row patches at every
+   * level.  A step is one UNet evaluation at the timestep set by dfp_set_timestep; its
+   * output (dfp_output) is the predicted noise [H*W, 4] bf16.  Weights: the names and
+   * PyTorch shapes of the workload's generator (time_embedding.linear_{1,2}, conv_in,
+   * down{0,1,2}.resnet.*, down{1,2}.xf.*, down{0,1}.downsample, up{1,0}.upsample,
+   * up1.resnet.*, up1.xf.*, up0.resnet.*, norm_out, conv_out, and "context").  bf16,
+   * batch 1, heads * 64 == C, H a multiple of 4 N, W of 4, 6 C <= 4096. */
+  DFP_BLOCK_UNET = 2
 } dfp_block;
 
 typedef enum {
@@ -185,6 +198,21 @@ DFP_API dfp_status dfp_step_patches(dfp_handle h, const void* x, int step, int p
  * Valid until dfp_destroy.  DFP_E_ARG for an unknown name or a parity other than 0 / 1. */
 DFP_API dfp_status dfp_context_buffer(dfp_handle h, const char* name, int parity, void** ptr, long long* bytes);
 
+/* The timestep the next DFP_BLOCK_UNET step embeds (DFP_E_UNSUPPORTED for other blocks). */
+DFP_API dfp_status dfp_set_timestep(dfp_handle h, float timestep);
+
+/* The DDIM loop around a DFP_BLOCK_UNET handle (paper reading blog, Implementation details:
+ * 50-step DDIM, the first steps synchronous; project README, Performance): deterministic
+ * DDIM (eta = 0) on a scaled-linear beta schedule of n_train training steps (beta_i =
+ * (sqrt(beta_start) + i (sqrt(beta_end) - sqrt(beta_start)) / (n_train - 1))^2), visiting
+ * timesteps (n_steps - 1 - k) floor(n_train / n_steps) + 1 for k = 0 .. n_steps - 1; step k runs the
+ * UNet at step index k, synchronous for k < n_sync, then x <- sqrt(ab') (x - sqrt(1 - ab) eps)
+ * / sqrt(ab) + sqrt(1 - ab') eps in fp32.  x_T, x_out: device fp32 [H, W, 4] (may be the
+ * same buffer).  Asynchronous on the handle's stream.  DFP_E_ARG unless n_steps >= 1,
+ * 1 <= n_sync, n_steps <= n_train <= 100000 and 0 < beta_start < beta_end < 1. */
+DFP_API dfp_status dfp_ddim_sample(dfp_handle h, const float* x_T, int n_steps, int n_sync, int n_train,
+                                   float beta_start, float beta_end, float* x_out);
+
 /* Same step with HOST buffers: copies x_host ([B,H,W,C], config dtype; pinned
  * memory gives asynchronous copies) to the device, runs the step, copies the
  * output to y_host and waits for the stream. */
@@ -281,8 +309,9 @@ DFP_API dfp_status dfp_set_kernel_family(dfp_handle h, int family);
 /* Per-kernel timing.  With profiling on, dfp_step brackets every kernel launch
  * with CUDA events recorded on the handle's stream.  dfp_kernel_times waits for
  * the last step's events and writes up to max_n durations (milliseconds) and the
- * matching static kernel names; it returns the number of launches timed (0 when
- * profiling is off or no step ran), or -1 on a CUDA error. */
+ * matching static kernel names; it returns the number of durations written (at
+ * most max_n; 0 when profiling is off, no step ran or the step made more than 127
+ * launches), or -1 on a CUDA error. */
 DFP_API dfp_status dfp_set_profiling(dfp_handle h, int enable);
 DFP_API int dfp_kernel_times(dfp_handle h, float* ms, const char** names, int max_n);
 

@@ -96,6 +96,15 @@ dfp_status check_config(const dfp_config* c, std::string& why) {
     if (c->ffn_inner <= 0 || c->ffn_inner % 64) return bad("ffn_inner must be a positive multiple of 64");
     if (c->ctx_len <= 0 || c->ctx_dim <= 0 || c->ctx_dim % 8) return bad("ctx_len > 0 and ctx_dim a positive multiple of 8");
     if (c->C > 2048) return bad("C must be <= 2048 for the transformer stage");
+  } else if (c->block == DFP_BLOCK_UNET) {
+    if (c->dtype != DFP_BF16) { why = "the UNet is built for bf16 storage only"; return DFP_E_UNSUPPORTED; }
+    if (B != 1) { why = "the UNet runs one image per handle"; return DFP_E_UNSUPPORTED; }
+    if (c->H % (4 * c->n_patches) || c->W % 4) return bad("the UNet needs H a multiple of 4 n_patches and W of 4");
+    const long long R1 = c->H / c->n_patches / 2, R2 = R1 / 2;
+    if ((R1 * (c->W / 2)) % 8 || (R2 * (c->W / 4)) % 8)
+      return bad("the UNet's lower levels need a multiple of 8 tokens per patch");
+    if (6 * c->C > 4096) return bad("the UNet needs 6 C <= 4096 (its widest concatenation)");
+    if (c->ctx_len <= 0 || c->ctx_dim <= 0 || c->ctx_dim % 8) return bad("ctx_len > 0 and ctx_dim a positive multiple of 8");
   } else if (c->block != DFP_BLOCK_RES_ATTN) {
     return bad("unknown block type");
   }
@@ -159,6 +168,7 @@ dfp_status build_tmaps(dfp_ctx* h) {
 std::vector<WeightSpec> res_attn_weight_specs(const dfp_config& c);
 std::vector<WeightSpec> weight_specs(dfp_ctx* h) {
   if (h->cfg.block == DFP_BLOCK_SDXL_STAGE) return stage_weight_specs(h->cfg, h->spec_names);
+  if (h->cfg.block == DFP_BLOCK_UNET) return unet_weight_specs(h);
   return res_attn_weight_specs(h->cfg);
 }
 std::vector<WeightSpec> res_attn_weight_specs(const dfp_config& c) {
@@ -222,9 +232,9 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
   const size_t C = cfg->C, N = (size_t)h->B * cfg->n_patches, G = cfg->gn_groups, W = cfg->W, R = h->R,
                L = (size_t)h->B * h->L;
   const size_t map = L * C * h->esz;
-  const bool is_stage = cfg->block == DFP_BLOCK_SDXL_STAGE;
+  const bool is_stage = cfg->block == DFP_BLOCK_SDXL_STAGE, is_unet = cfg->block == DFP_BLOCK_UNET;
   bool ok = true;
-  if (!is_stage) {
+  if (!is_stage && !is_unet) {
     ok &= h->alloc(&h->w_conv, 9 * C * C * h->esz);
     ok &= h->alloc((void**)&h->b_conv, C * 4);
     ok &= h->alloc(&h->w_qkv, 3 * C * C * h->esz);
@@ -269,7 +279,7 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
   // zero everything the kernels rely on: slab halo rows at the image edges, the
   // GroupNorm block counter, the device error word, and all caches
   cudaError_t e = cudaSuccess;
-  if (!is_stage) {
+  if (!is_stage && !is_unet) {
     for (void* p : {h->slab[0], h->slab[1]})
       if (e == cudaSuccess) e = cudaMemset(p, 0, N * (R + 2) * W * C * h->esz);
     for (void* p : {h->kb[0], h->kb[1], h->vb[0], h->vb[1], h->h, h->t, h->y})
@@ -287,6 +297,8 @@ dfp_status dfp_create(const dfp_config* cfg, void* cuda_stream, dfp_handle* out)
   }
   if (is_stage) {
     st = stage_create(h);
+  } else if (is_unet) {
+    st = unet_create(h);
   } else if (cfg->dtype == DFP_BF16) {
     st = build_tmaps(h);
   }
@@ -331,9 +343,10 @@ dfp_status dfp_load_weights(dfp_handle h, const dfp_tensor* w, int n) {
     std::vector<float> v;
     read_as_float(src, t.dtype, numel, v);
     const std::string name = t.name;
-    if (h->stage) {
+    if (h->stage || h->unet) {
       dfp_status lst = DFP_OK;
-      if (!stage_load_weight(h, name, v, lst)) return h->fail(DFP_E_ARG, "unknown weight name " + name);
+      const bool known = h->stage ? stage_load_weight(h, name, v, lst) : unet_load_weight(h, name, v, lst);
+      if (!known) return h->fail(DFP_E_ARG, "unknown weight name " + name);
       if (lst != DFP_OK) return lst;
       h->loaded.insert(name);
       continue;
@@ -375,6 +388,7 @@ dfp_status dfp_load_weights(dfp_handle h, const dfp_tensor* w, int n) {
     h->loaded.insert(name);
   }
   if (h->stage) return stage_finish_load(h);
+  if (h->unet) return unet_finish_load(h);
   return DFP_OK;
 }
 
@@ -389,6 +403,7 @@ dfp_status dfp_step(dfp_handle h, const void* x, int step, int is_sync) {
   if (step != 0 && step != h->last_step + 1)
     return h->fail(DFP_E_STATE, "steps must be consecutive (or restart at 0)");
   dfp_status st = h->stage ? stage_step(h, x, step, is_sync)
+                 : h->unet ? unet_step(h, x, step, is_sync)
                  : h->cfg.dtype == DFP_BF16 ? run_step<__nv_bfloat16>(h, x, step, is_sync)
                                             : run_step<float>(h, x, step, is_sync);
   if (st == DFP_OK) h->last_step = step;
@@ -399,7 +414,7 @@ dfp_status dfp_step_patches(dfp_handle h, const void* x, int step, int p_begin, 
   if (!h) return DFP_E_ARG;
   if (!x) return h->fail(DFP_E_ARG, "x is NULL");
   const dfp_config& c = h->cfg;
-  if (h->stage || c.dtype != DFP_BF16 || h->family != 0 || h->B != 1)
+  if (h->stage || h->unet || c.dtype != DFP_BF16 || h->family != 0 || h->B != 1)
     return h->fail(DFP_E_UNSUPPORTED, "a patch range runs the layer block of one bf16 image on the tensor-core kernels");
   if (c.gn_mode == DFP_GN_SYNC && c.context != DFP_CTX_NAIVE)
     return h->fail(DFP_E_UNSUPPORTED, "the GroupNorm sync mode needs every patch's statistics of this step");
@@ -417,7 +432,7 @@ dfp_status dfp_context_buffer(dfp_handle h, const char* name, int parity, void**
   if (!h) return DFP_E_ARG;
   if (!name || !ptr || !bytes) return h->fail(DFP_E_ARG, "NULL argument");
   if (parity != 0 && parity != 1) return h->fail(DFP_E_ARG, "parity must be 0 or 1");
-  if (h->stage) return h->fail(DFP_E_UNSUPPORTED, "context buffers of the layer block only");
+  if (h->stage || h->unet) return h->fail(DFP_E_UNSUPPORTED, "context buffers of the layer block only");
   const dfp_config& c = h->cfg;
   const long long map = (long long)h->B * h->L * c.C * (long long)h->esz;
   const long long mom = (long long)h->B * c.n_patches * c.gn_groups * 2 * 4;
@@ -434,8 +449,30 @@ dfp_status dfp_context_buffer(dfp_handle h, const char* name, int parity, void**
   return DFP_OK;
 }
 
+dfp_status dfp_set_timestep(dfp_handle h, float timestep) {
+  if (!h) return DFP_E_ARG;
+  if (!h->unet) return h->fail(DFP_E_UNSUPPORTED, "timesteps belong to the UNet block");
+  if (!(timestep >= 0.f)) return h->fail(DFP_E_ARG, "timestep must be >= 0");
+  unet_set_timestep(h, timestep);
+  return DFP_OK;
+}
+
+dfp_status dfp_ddim_sample(dfp_handle h, const float* x_T, int n_steps, int n_sync, int n_train, float beta_start,
+                           float beta_end, float* x_out) {
+  if (!h) return DFP_E_ARG;
+  if (!h->unet) return h->fail(DFP_E_UNSUPPORTED, "DDIM runs the UNet block");
+  if (!x_T || !x_out) return h->fail(DFP_E_ARG, "x_T / x_out is NULL");
+  if (n_steps < 1 || n_sync < 1 || n_train < n_steps || n_train > 100000)
+    return h->fail(DFP_E_ARG, "need n_steps >= 1, n_sync >= 1 and n_steps <= n_train <= 100000");
+  if (!(beta_start > 0.f && beta_start < beta_end && beta_end < 1.f)) return h->fail(DFP_E_ARG, "bad beta range");
+  if (h->loaded.size() != weight_specs(h).size())
+    return h->fail(DFP_E_STATE, "weights not loaded (every weight must be given before the first step)");
+  return unet_ddim(h, x_T, n_steps, n_sync, n_train, beta_start, beta_end, x_out, dfp_step);
+}
+
 dfp_status dfp_step_host(dfp_handle h, const void* x_host, void* y_host, int step, int is_sync) {
   if (!h) return DFP_E_ARG;
+  if (h->unet) return h->fail(DFP_E_UNSUPPORTED, "host-buffer steps of the layer blocks only");
   if (!x_host || !y_host) return h->fail(DFP_E_ARG, "x_host / y_host is NULL");
   const size_t bytes = (size_t)h->B * h->L * h->cfg.C * h->esz;
   cudaError_t e = cudaMemcpyAsync(h->xin, x_host, bytes, cudaMemcpyHostToDevice, h->stream);
@@ -451,6 +488,7 @@ dfp_status dfp_step_host(dfp_handle h, const void* x_host, void* y_host, int ste
 
 dfp_status dfp_step_host_async(dfp_handle h, const void* x_host, void* y_host, int step, int is_sync) {
   if (!h) return DFP_E_ARG;
+  if (h->unet) return h->fail(DFP_E_UNSUPPORTED, "host-buffer steps of the layer blocks only");
   if (!x_host || !y_host) return h->fail(DFP_E_ARG, "x_host / y_host is NULL");
   const size_t bytes = (size_t)h->B * h->L * h->cfg.C * h->esz;
   cudaError_t e = cudaSuccess;
@@ -516,6 +554,7 @@ static bool buffer_of(dfp_handle h, const char* name, const void** ptr, long lon
   const long long st = (long long)h->B * h->cfg.n_patches * h->cfg.gn_groups * 2 * 4;
   const int cur = h->last_step < 0 ? 0 : (h->last_step & 1);
   const std::string n = name;
+  if (h->unet) return unet_buffer(h, n, ptr, bytes);
   if (h->stage) {
     if (stage_buffer(h, n, ptr, bytes)) return true;
     if (n == "gn1" || n == "gn2") { *ptr = n == "gn1" ? h->mr1 : h->mr2; *bytes = st; return true; }
@@ -624,8 +663,8 @@ int dfp_kernel_times(dfp_handle h, float* ms, const char** names, int max_n) {
   if (!h) return -1;
   if (!h->profiling || h->n_ev < 2) return 0;
   if (cudaEventSynchronize(h->ev[h->n_ev - 1]) != cudaSuccess) return -1;
-  const int n = h->n_ev - 1;
-  for (int i = 0; i < n && i < max_n; ++i) {
+  const int n = h->n_ev - 1 < max_n ? h->n_ev - 1 : max_n;
+  for (int i = 0; i < n; ++i) {
     float t = 0.f;
     if (cudaEventElapsedTime(&t, h->ev[i], h->ev[i + 1]) != cudaSuccess) return -1;
     if (ms) ms[i] = t;
@@ -646,6 +685,7 @@ dfp_status dfp_destroy(dfp_handle h) {
     if (h->ev[i]) cudaEventDestroy(h->ev[i]);
   for (void* p : h->allocs) cudaFree(p);
   delete_stage(h->stage);
+  delete_unet(h->unet);
   delete h;
   return DFP_OK;
 }

@@ -80,10 +80,14 @@ __device__ __forceinline__ int gn_rule(const GnArgs& a) {
     default: return kGnNaive;
   }
 }
-// own: this step's moments of patch pi (of NI in its image); img: moments of the image's
-// patches (this step's for kGnSync, the previous step's otherwise), `stride` float2 apart.
-// Returns (mean, var) of the estimate, var clamped at 0.
-__device__ __forceinline__ float2 gn_estimate(int rule, int NI, int pi, float2 own, const float2* img, int stride) {
+// own: this step's moments of patch pi (of NI in its image); img: moments (mean, var) of
+// the image's patches (this step's for kGnSync, the previous step's otherwise), patch j's
+// pair at img[2 j stride] (scalar reads: no alignment assumed).  Returns (mean, var) of
+// the estimate, var clamped at 0.
+__device__ __forceinline__ float2 mom_at(const float* img, int j, int stride) {
+  return make_float2(img[2 * j * stride], img[2 * j * stride + 1]);
+}
+__device__ __forceinline__ float2 gn_estimate(int rule, int NI, int pi, float2 own, const float* img, int stride) {
   const float inv = 1.f / (float)NI;
   float mu, var;
   if (rule == kGnNaive) {
@@ -91,11 +95,11 @@ __device__ __forceinline__ float2 gn_estimate(int rule, int NI, int pi, float2 o
     var = own.y;
   } else if (rule == kGnCorrected) {
     float sm = 0.f, sv = 0.f;
-    for (int j = 0; j < NI; ++j) { const float2 q = img[j * stride]; sm += q.x; sv += q.y; }
+    for (int j = 0; j < NI; ++j) { const float2 q = mom_at(img, j, stride); sm += q.x; sv += q.y; }
     const float mb = sm * inv;
     float ss = 0.f;
-    for (int j = 0; j < NI; ++j) { const float e = img[j * stride].x - mb; ss = fmaf(e, e, ss); }
-    const float2 st = img[pi * stride];
+    for (int j = 0; j < NI; ++j) { const float e = mom_at(img, j, stride).x - mb; ss = fmaf(e, e, ss); }
+    const float2 st = mom_at(img, pi, stride);
     const float d = own.x - st.x;
     mu = mb + d;
     var = sv * inv + (own.y - st.y) + ss * inv + 2.f * d * (st.x - mb);
@@ -103,13 +107,13 @@ __device__ __forceinline__ float2 gn_estimate(int rule, int NI, int pi, float2 o
     // sync: every component is this step's; stale-others: all but patch pi are the previous step's
     float sm = 0.f, sv = 0.f;
     for (int j = 0; j < NI; ++j) {
-      const float2 q = (rule == kGnStaleOthers && j == pi) ? own : img[j * stride];
+      const float2 q = (rule == kGnStaleOthers && j == pi) ? own : mom_at(img, j, stride);
       sm += q.x; sv += q.y;
     }
     mu = sm * inv;
     float ss = 0.f;
     for (int j = 0; j < NI; ++j) {
-      const float e = ((rule == kGnStaleOthers && j == pi) ? own : img[j * stride]).x - mu;
+      const float e = ((rule == kGnStaleOthers && j == pi) ? own : mom_at(img, j, stride)).x - mu;
       ss = fmaf(e, e, ss);
     }
     var = sv * inv + ss * inv;
@@ -122,7 +126,7 @@ __global__ void __launch_bounds__(kGnThreads)
 gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
   constexpr int VEC = VecTraits<T>::kN;
   extern __shared__ float sh[];                 // [2][PL][C] lane sums, then [2][C] channel sums
-  __shared__ float s_mom[512 * 2];              // merged fresh moments  [N*G][2]
+  __shared__ __align__(16) float s_mom[512 * 2];   // fresh moments (mean, var) [N*G][2]
   __shared__ int s_last;
   const int C = a.C, G = a.G, N = a.N;
   const int V = C / VEC;
@@ -151,6 +155,7 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
         u[j] = pix + j * PL < pix1 ? ld_nc16(base + (size_t)(pix + j * PL) * C) : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
+        if (pix + j * PL >= pix1) break;   // past the chunk: a zero would add -K, K^2 to the sums
         float v[VEC];
         unpack16(u[j], v);
 #pragma unroll
@@ -236,7 +241,7 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
     const int pp = tid / G, gg = tid % G;
     const int NI = a.per_image, j0 = pp / NI * NI;   // the patches of pp's image
     const int rule = gn_rule(a);
-    const float2* img = reinterpret_cast<const float2*>(rule == kGnSync ? s_mom : a.stale) + j0 * G + gg;
+    const float* img = (rule == kGnSync ? s_mom : a.stale) + 2 * (j0 * G + gg);
     const float2 e = gn_estimate(rule, NI, pp - j0, make_float2(s_mom[tid * 2], s_mom[tid * 2 + 1]), img, G);
     a.mean_rstd[tid * 2] = e.x;
     a.mean_rstd[tid * 2 + 1] = 1.f / sqrtf(e.y + a.eps);
@@ -245,6 +250,11 @@ gn_stats_merge_kernel(GnArgs a, int n_chunks, int pix_per_chunk) {
 }
 
 __device__ __forceinline__ float silu_f(float y) { return y / (1.f + expf(-y)); }
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // Normalise (+SiLU) one chunk of patch p.  With halo_mode != 0 the output is the
 // haloed slab and the kernel also fills the neighbours' halo rows: a patch's
@@ -361,12 +371,12 @@ __device__ __forceinline__ bool grid_wait(unsigned* count, unsigned total, int* 
 }
 
 template <typename T, bool SILU>
-__global__ void __launch_bounds__(kGnThreads, 2)
+__global__ void __launch_bounds__(kGnThreads, 1)
 gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
   constexpr int VEC = VecTraits<T>::kN;
   extern __shared__ float sh[];                 // [2][PL][C] lane sums, then [2][C] channel sums
-  __shared__ float s_mr[256 * 2];               // (mean, rstd) of this patch's groups
-  __shared__ float s_mom[256 * 2];              // fresh moments of the patches needed
+  __shared__ __align__(16) float s_mr[256 * 2];    // (mean, rstd) of this patch's groups
+  __shared__ __align__(16) float s_mom[256 * 2];   // fresh moments (mean, var) of the patches needed
   const int C = a.C, G = a.G;
   const int V = C / VEC;
   const int PL = kGnThreads / V;
@@ -393,13 +403,17 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
     if (pl < PL) {
       float k[VEC];
       gn_thread_shifts<T, VEC>(a.x, p, a.pix_per_patch, C, vc * VEC, C / G, k);
-      for (int pix = pix0 + pl; pix < pix1; pix += 8 * PL) {
-        uint4 u[8];
+      // the chunk is read again after the barrier: ask L2 to keep it; sixteen loads in flight
+      // per thread (one block per SM: the map's first read is DRAM latency bound)
+      const uint64_t keep = l2_evict_last_policy();
+      for (int pix = pix0 + pl; pix < pix1; pix += 16 * PL) {
+        uint4 u[16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          u[j] = pix + j * PL < pix1 ? ld_nc16(base + (size_t)(pix + j * PL) * C) : make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < 16; ++j)
+          u[j] = pix + j * PL < pix1 ? ld_nc16_policy(base + (size_t)(pix + j * PL) * C, keep) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 16; ++j) {
+          if (pix + j * PL >= pix1) break;   // past the chunk: a zero would add -K, K^2 to the sums
           float v[VEC];
           unpack16(u[j], v);
 #pragma unroll
@@ -508,8 +522,7 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
     const int own = (all ? pi : 0) * G + gg;    // this patch's entry in s_mom
     const float2 mo = make_float2(s_mom[own * 2], s_mom[own * 2 + 1]);
     const int rule = gn_rule(a);
-    const float2* img = rule == kGnSync ? reinterpret_cast<const float2*>(s_mom) + gg
-                                        : reinterpret_cast<const float2*>(a.stale) + (p - pi) * G + gg;
+    const float* img = rule == kGnSync ? s_mom + 2 * gg : a.stale + 2 * ((p - pi) * G + gg);
     const float2 e = gn_estimate(rule, NI, pi, mo, img, G);
     const float rstd = 1.f / sqrtf(e.y + a.eps);
     s_mr[gg * 2] = e.x;
@@ -534,13 +547,16 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
     }
     T* outp = static_cast<T*>(o.out);
     T* dst = outp + ((size_t)p * o.out_patch_stride + o.out_off) * C + vc * VEC;
-    for (int pix = pix0 + pl; pix < pix1; pix += 4 * PL) {
-      uint4 u[4];
+    // the last read of the chunk: let L2 drop it first (the output is what the next kernel reads)
+    const uint64_t drop = l2_evict_first_policy();
+    auto load8 = [&](uint4 (&u)[8], int pix) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        u[j] = pix + j * PL < pix1 ? ld_nc16(base + (size_t)(pix + j * PL) * C) : make_uint4(0, 0, 0, 0);
+      for (int j = 0; j < 8; ++j)
+        u[j] = pix + j * PL < pix1 ? ld_nc16_policy(base + (size_t)(pix + j * PL) * C, drop) : make_uint4(0, 0, 0, 0);
+    };
+    auto apply8 = [&](const uint4 (&u)[8], int pix) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 8; ++j) {
         const int q = pix + j * PL;
         if (q >= pix1) break;
         float v[VEC];
@@ -548,7 +564,16 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
 #pragma unroll
         for (int i = 0; i < VEC; ++i) {
           v[i] = fmaf(v[i], sc[i], sf[i]);
-          if (SILU) v[i] = __fdividef(v[i], 1.f + __expf(-v[i]));   // bf16 output: fast forms suffice
+          // SiLU as v/2 (1 + tanh(v/2)): one MUFU operation for a bf16 output (the approximate
+          // tanh, relative error below 2^-10, is finer than the output's rounding); exact for fp32
+          if (SILU) {
+            if (sizeof(T) == 2) {
+              const float hv = 0.5f * v[i];
+              v[i] = fmaf(hv, tanh_approx(hv), hv);
+            } else {
+              v[i] = silu_f(v[i]);
+            }
+          }
         }
         const uint4 ov = pack16(v);
         *reinterpret_cast<uint4*>(dst + (size_t)q * C) = ov;
@@ -556,6 +581,15 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
           write_halos(outp, static_cast<const T*>(o.prev_slab), ov, p, q, a.pix_per_patch, last_row0, o.W, C,
                       vc * VEC, o.out_patch_stride, o.out_off, top_src, bot_src, o.halo_mode);
       }
+    };
+    // two batches of eight in flight: the next batch loads while this one is written
+    uint4 ua[8], ub[8];
+    load8(ua, pix0 + pl);
+    for (int pix = pix0 + pl; pix < pix1; pix += 16 * PL) {
+      load8(ub, pix + 8 * PL);
+      apply8(ua, pix);
+      load8(ua, pix + 16 * PL);
+      apply8(ub, pix + 8 * PL);
     }
   }
   // ---- departure: the last block out re-arms the barrier for the next launch

@@ -13,6 +13,8 @@
 namespace dfp {
 struct Stage;
 void delete_stage(Stage* s);
+struct Unet;
+void delete_unet(Unet* u);
 size_t dtype_size(dfp_dtype d);
 // Host-side fault injection for allocation failure: while the environment variable
 // DFP_FAULT_ALLOC_AFTER=k is set, the first k device allocations the library attempts
@@ -63,7 +65,7 @@ struct dfp_ctx {
   int last_step = -1;
   int launches = 0;
   // per-launch timing (dfp_set_profiling)
-  static constexpr int kMaxEv = 40;
+  static constexpr int kMaxEv = 128;
   bool profiling = false;
   cudaEvent_t ev[kMaxEv] = {};
   const char* ev_name[kMaxEv] = {};
@@ -73,6 +75,8 @@ struct dfp_ctx {
   dfp::TcGemmPlan conv_plan{}, qkv_plan{}, out_plan{};
   // the SDXL-style stage (DFP_BLOCK_SDXL_STAGE): its own buffers and weights
   dfp::Stage* stage = nullptr;
+  // the multi-level UNet (DFP_BLOCK_UNET)
+  dfp::Unet* unet = nullptr;
 
   dfp_status fail(dfp_status s, const std::string& msg) {
     err = msg;
@@ -114,6 +118,8 @@ struct dfp_ctx {
     if (h->profiling && launches < dfp_ctx::kMaxEv) {            \
       cudaEventRecord(h->ev[launches], s);                       \
       h->n_ev = launches + 1;                                    \
+    } else if (h->profiling) {                                   \
+      h->n_ev = 0;  /* more launches than events: no timing */   \
     }                                                            \
     h->launches = launches;                                      \
   } while (0)
@@ -131,4 +137,14 @@ bool stage_load_weight(dfp_ctx* h, const std::string& name, const std::vector<fl
 dfp_status stage_finish_load(dfp_ctx* h);
 dfp_status stage_step(dfp_ctx* h, const void* x, int step, int is_sync);
 bool stage_buffer(dfp_ctx* h, const std::string& name, const void** ptr, long long* bytes);
+// multi-level UNet (csrc/unet.cu)
+dfp_status unet_create(dfp_ctx* h);
+std::vector<WeightSpec> unet_weight_specs(dfp_ctx* h);
+bool unet_load_weight(dfp_ctx* h, const std::string& name, const std::vector<float>& v, dfp_status& st);
+dfp_status unet_finish_load(dfp_ctx* h);
+dfp_status unet_step(dfp_ctx* h, const void* x, int step, int is_sync);
+void unet_set_timestep(dfp_ctx* h, float tau);
+dfp_status unet_ddim(dfp_ctx* h, const float* x_T, int n_steps, int n_sync, int n_train, float beta_start,
+                     float beta_end, float* x_out, dfp_status (*step_fn)(dfp_ctx*, const void*, int, int));
+bool unet_buffer(dfp_ctx* h, const std::string& name, const void** ptr, long long* bytes);
 }  // namespace dfp

@@ -57,6 +57,24 @@ cudaError_t launch_gn_apply(const T* x, T* out, const T* prev_slab, const float*
 cudaError_t launch_layernorm(const void* x, void* y, const float* gamma, const float* beta, int L, int C,
                              float eps, bool pdl, cudaStream_t s);
 
+// ---------------------------------------------------------------- multi-level UNet helpers
+// The haloed conv input slab [N][R+2][W][C] filled from a map [N*R][W][src_C] (upsample:
+// from the map at half resolution, each pixel repeated 2 x 2); channels past src_C zero;
+// halo_mode as for launch_gn_apply (2 reads the neighbours' rows from prev_slab).
+cudaError_t launch_slab_fill(const void* src, int src_C, void* slab, const void* prev_slab, int C, int N, int R,
+                             int W, int halo_mode, bool upsample, bool pdl, cudaStream_t s);
+// out [L][Ca+Cb] = a [L][Ca] then b [L][Cb], bf16
+cudaError_t launch_concat(const void* a, int Ca, const void* b, int Cb, void* out, long long L, bool pdl,
+                          cudaStream_t s);
+// y = act(W x + b (+ add)), fp32, W [rows][cols]; x_tau >= 0: x is the sinusoidal
+// embedding of timestep x_tau (cols entries)
+cudaError_t launch_gemv(const float* W, const float* b, const float* add, const float* x, float x_tau, float* y,
+                        int rows, int cols, bool silu_out, bool pdl, cudaStream_t s);
+// DDIM update lat = c1 lat + c2 eps (fp32 latent, bf16 eps), and its bf16 copy
+cudaError_t launch_ddim_update(float* lat, const void* eps, void* x_bf, long long n, float c1, float c2, bool pdl,
+                               cudaStream_t s);
+cudaError_t launch_to_bf16(const float* a, void* b, long long n, cudaStream_t s);
+
 // ---------------------------------------------------------------- GEMM epilogues
 struct Epilogue {
   // 0: out[m, n] = acc + bias[n] (+ residual[m, n]); bias / residual may be null
@@ -68,6 +86,9 @@ struct Epilogue {
   const float* bias;
   const void* residual;   // kind 0: [M, ldo] bf16, may alias out (same element read then written)
   int ldo;
+  int subsample;          // kind 0, conv: store only even (row, column) pixels, into the
+                          // half-resolution map (a stride-2 conv)
+  int n_store;            // kind 0: columns stored (0: all); a layer padded to a wider tile
   void* q; void* k; void* v;
   int L, C;
 };

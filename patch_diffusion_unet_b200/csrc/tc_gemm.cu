@@ -66,6 +66,12 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmPlan& plan, const Epil
     gm = tile.m0 + row;
   }
   if (!valid_tile) gm = -1;
+  if (epi.subsample && gm >= 0) {
+    // a stride-2 conv as the stride-1 conv sampled at even rows and columns: keep those
+    // pixels, stored at their place in the half-resolution map
+    const long long prow = gm / plan.W, col = gm - prow * plan.W;
+    gm = ((prow | col) & 1) ? -1 : (prow >> 1) * (plan.W >> 1) + (col >> 1);
+  }
   if (BN == 128 && epi.kind == 2) {
     // GEGLU: columns [0, 64) are values, [64, 128) the gates of the same features
 #pragma unroll 1
@@ -121,6 +127,11 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmPlan& plan, const Epil
         }
       }
       dst = static_cast<__nv_bfloat16*>(epi.out) + gm * epi.ldo + n;
+      if (epi.n_store && n + 32 > epi.n_store) {
+        // only the first n_store columns exist in the output (a padded narrow layer)
+        for (int i = 0; i < 32 && n + i < epi.n_store; ++i) dst[i] = __float2bfloat16_rn(v[i]);
+        continue;
+      }
     } else {
       const int which = n / epi.C, cc = n - which * epi.C;
       const int head = cc >> 6, d0 = cc & 63;

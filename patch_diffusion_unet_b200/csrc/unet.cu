@@ -1,0 +1,721 @@
+// The multi-level UNet (DFP_BLOCK_UNET): one denoising step of an SDXL-shaped network on
+// the displaced-patch path, and the DDIM loop around it.
+//
+// The pages run SDXL's UNet for 50 DDIM steps with every convolution, GroupNorm and
+// self-attention replaced by its displaced form and the latent split into the same row
+// patches at every resolution ("DistriFusion" project README, Overview (c) and
+// Performance; paper reading blog, Implementation details; source walkthrough, Patch
+// Parallelism: DistriUNetPP wraps the UNet's conv, norm and attention layers).  With
+// widths c, 2c, 4c at H, H/2, H/4 (latent H x W x 4):
+//   conv_in -> ResNet(c) = s0 -> down -> ResNet(c->2c) + transformer = s1 -> down
+//   -> ResNet(2c->4c) + transformer -> up -> [., s1] -> ResNet(6c->2c) + transformer
+//   -> up -> [., s0] -> ResNet(3c->c) -> GN + SiLU -> conv_out = predicted noise
+// ResNet(x): h = conv1(SiLU(GN1 x)) + W_t SiLU(temb) + b_t; h = conv2(SiLU(GN2 h));
+// out = h + x, or h + a 1x1 projection of x when the width changes.  The timestep
+// embedding is a sinusoid through Linear - SiLU - Linear.  "down" is a stride-2 3x3 conv,
+// computed as the displaced stride-1 conv whose epilogue keeps the even rows and columns
+// (the same value, and the same halo: a patch's first output row reads the row above it);
+// "up" repeats each pixel 2 x 2 into the next conv's haloed input slab.
+//
+// Every conv reads a haloed slab [N][R+2][W][C] of its level, filled either by the fused
+// GroupNorm (+SiLU) kernel or by the slab-fill kernel (conv_in, down, up); the stale halo
+// rows and the GroupNorm moments alternate by step parity exactly as in the layer block,
+// and each transformer's self-attention keeps its own K/V pair.  conv_in reads the
+// 4-channel latent padded to 64 channels, conv_out computes 64 channels of which 4 are
+// stored.  The narrow kernels (slab fill, concatenation, timestep MLP, DDIM update) are in
+// unet_kernels.cu.
+#include <cmath>
+#include <cstring>
+#include <functional>
+#include <string>
+#include <vector>
+
+#include "handle.h"
+
+namespace dfp {
+
+namespace {
+
+using bf = __nv_bfloat16;
+
+struct Level {
+  int H, W, R, L, Lp;   // rows, columns, rows per patch, tokens, tokens per patch
+};
+
+struct UConv {          // displaced 3x3 conv Cin -> Cout on one level (Cout padded to >= 64)
+  Level lv{};
+  int Cin = 0, Cout = 0;
+  void* slab[2] = {};
+  void* w = nullptr;    // [Cout][9][Cin] bf16
+  float* b = nullptr;
+  CUtensorMap m_slab[2], m_w;
+  TcGemmPlan plan{};
+};
+
+struct UGn {
+  int C = 0;
+  float *g = nullptr, *b = nullptr;
+  float* mom[2] = {};
+};
+
+struct URes {
+  Level lv{};
+  int Cin = 0, Cout = 0;
+  const void* in = nullptr;   // [L][Cin]
+  UGn n1, n2;
+  UConv c1, c2;
+  float *wt = nullptr, *bt = nullptr;   // time projection [Cout][temb] fp32, bias
+  float* bias1 = nullptr;               // per step: conv1 bias + time projection
+  void* h1 = nullptr;                   // [L][Cout] conv1 output
+  void* out = nullptr;                  // [L][Cout]
+  bool sc = false;                      // 1x1 projection of the input (width change)
+  void* w_sc = nullptr;                 // [Cout][Cin] bf16
+  float* b_sc = nullptr;
+  void* sc_out = nullptr;               // [L][Cout]
+  CUtensorMap m_in, m_wsc;
+  TcGemmPlan p_sc{};
+};
+
+struct UXf {                            // transformer block, in place on r [L][C]
+  Level lv{};
+  int C = 0, heads = 0, F = 0;
+  void* r = nullptr;
+  float *ln_g[3] = {}, *ln_b[3] = {};
+  void *w_qkv = nullptr, *w_o1 = nullptr, *w_q2 = nullptr, *w_o2 = nullptr, *w_k2 = nullptr, *w_v2 = nullptr;
+  void *w_ff1 = nullptr, *w_ff2 = nullptr;
+  float *b_o1 = nullptr, *b_o2 = nullptr, *b_ff1 = nullptr, *b_ff2 = nullptr;
+  void* kb[2] = {};
+  void* vb[2] = {};
+  void *ctx_k = nullptr, *ctx_v = nullptr;
+  bool ctx_ready = false;
+  CUtensorMap m_wqkv, m_wo1, m_wq2, m_wo2, m_wff1, m_wff2, m_k[2], m_v[2], m_ck, m_cv, m_q, m_u, m_o, m_g;
+  TcGemmPlan p_qkv{}, p_o1{}, p_q2{}, p_o2{}, p_ff1{}, p_ff2{};
+};
+
+// rows per head of the context K/V buffers: ctx_len padded with zeros to whole 128-key tiles
+size_t ctx_rows(size_t ctx_len) { return (ctx_len + 127) / 128 * 128; }
+
+uint16_t to_bf16_bits(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  return (uint16_t)((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
+}
+
+}  // namespace
+
+struct Unet {
+  int c0 = 0, c1 = 0, c2 = 0, temb = 0;
+  Level lv[3];
+  float *t_w1 = nullptr, *t_b1 = nullptr, *t_w2 = nullptr, *t_b2 = nullptr;
+  float *t_h = nullptr, *t_act = nullptr;   // hidden layer, SiLU(embedding)
+  UConv conv_in, down0, down1, up1, up0, conv_out;
+  URes res0, res1, res2, ures1, ures0;
+  UXf xf1, xf2, uxf1;
+  UGn gn_out;
+  void *h0 = nullptr, *s0 = nullptr, *d0 = nullptr, *d1 = nullptr, *u1 = nullptr, *u0 = nullptr;
+  void *cat1 = nullptr, *cat0 = nullptr, *eps = nullptr, *x_in = nullptr;
+  void *u = nullptr, *g = nullptr, *ctx = nullptr;
+  float* lat = nullptr;                     // DDIM latent, fp32 [L0][4]
+  bool ctx_loaded = false;
+  float tau = 0.f;
+  // weight name -> (shape, loader)
+  struct Entry {
+    std::string name;
+    std::vector<long long> shape;
+    std::function<dfp_status(dfp_ctx*, const std::vector<float>&)> load;
+  };
+  std::vector<Entry> entries;
+};
+
+void delete_unet(Unet* u) { delete u; }
+
+namespace {
+
+dfp_status up_bf16(dfp_ctx* h, void* dst, const std::vector<float>& v) {
+  std::vector<uint16_t> b(v.size());
+  for (size_t i = 0; i < v.size(); ++i) b[i] = to_bf16_bits(v[i]);
+  cudaError_t e = cudaMemcpy(dst, b.data(), b.size() * 2, cudaMemcpyHostToDevice);
+  return e == cudaSuccess ? DFP_OK : h->cuda_fail(e, "weight copy to device");
+}
+dfp_status up_f32(dfp_ctx* h, void* dst, const std::vector<float>& v) {
+  cudaError_t e = cudaMemcpy(dst, v.data(), v.size() * 4, cudaMemcpyHostToDevice);
+  return e == cudaSuccess ? DFP_OK : h->cuda_fail(e, "weight copy to device");
+}
+// conv weight [co][ci][3][3] -> [Cout][tap][Cin] bf16, zero-padded to the layer's widths
+dfp_status up_conv(dfp_ctx* h, const UConv& cv, int co_real, int ci_real, const std::vector<float>& v) {
+  std::vector<float> r((size_t)cv.Cout * 9 * cv.Cin, 0.f);
+  for (int co = 0; co < co_real; ++co)
+    for (int ci = 0; ci < ci_real; ++ci)
+      for (int tap = 0; tap < 9; ++tap) r[((size_t)co * 9 + tap) * cv.Cin + ci] = v[((size_t)co * ci_real + ci) * 9 + tap];
+  return up_bf16(h, cv.w, r);
+}
+
+bool alloc_conv(dfp_ctx* h, UConv& cv, const Level& lv, int N, int Cin, int Cout) {
+  cv.lv = lv;
+  cv.Cin = Cin;
+  cv.Cout = Cout;
+  const size_t slab = (size_t)N * (lv.R + 2) * lv.W * Cin * 2;
+  bool ok = h->alloc(&cv.slab[0], slab) && h->alloc(&cv.slab[1], slab);
+  ok = ok && h->alloc(&cv.w, (size_t)Cout * 9 * Cin * 2) && h->alloc((void**)&cv.b, (size_t)Cout * 4);
+  if (ok) ok = cudaMemset(cv.slab[0], 0, slab) == cudaSuccess && cudaMemset(cv.slab[1], 0, slab) == cudaSuccess &&
+               cudaMemset(cv.b, 0, (size_t)Cout * 4) == cudaSuccess;
+  return ok;
+}
+
+bool alloc_gn(dfp_ctx* h, UGn& gn, int C, int N, int G) {
+  gn.C = C;
+  return h->alloc((void**)&gn.g, C * 4) && h->alloc((void**)&gn.b, C * 4) &&
+         h->alloc((void**)&gn.mom[0], (size_t)N * G * 8) && h->alloc((void**)&gn.mom[1], (size_t)N * G * 8);
+}
+
+bool alloc_res(dfp_ctx* h, URes& r, const Level& lv, int N, int G, int Cin, int Cout, int temb) {
+  r.lv = lv;
+  r.Cin = Cin;
+  r.Cout = Cout;
+  r.sc = Cin != Cout;
+  const size_t map = (size_t)lv.L * Cout * 2;
+  bool ok = alloc_gn(h, r.n1, Cin, N, G) && alloc_gn(h, r.n2, Cout, N, G) && alloc_conv(h, r.c1, lv, N, Cin, Cout) &&
+            alloc_conv(h, r.c2, lv, N, Cout, Cout);
+  ok = ok && h->alloc((void**)&r.wt, (size_t)Cout * temb * 4) && h->alloc((void**)&r.bt, Cout * 4) &&
+       h->alloc((void**)&r.bias1, Cout * 4) && h->alloc(&r.h1, map) && h->alloc(&r.out, map);
+  if (ok && r.sc)
+    ok = h->alloc(&r.w_sc, (size_t)Cout * Cin * 2) && h->alloc((void**)&r.b_sc, Cout * 4) && h->alloc(&r.sc_out, map);
+  return ok;
+}
+
+bool alloc_xf(dfp_ctx* h, UXf& x, const Level& lv, int C, size_t ctx_all, int D) {
+  x.lv = lv;
+  x.C = C;
+  x.heads = C / 64;
+  x.F = 4 * C;
+  const size_t map = (size_t)lv.L * C * 2, F = x.F;
+  bool ok = true;
+  for (int k = 0; k < 3; ++k) ok = ok && h->alloc((void**)&x.ln_g[k], C * 4) && h->alloc((void**)&x.ln_b[k], C * 4);
+  ok = ok && h->alloc(&x.w_qkv, 3ull * C * C * 2) && h->alloc(&x.w_o1, (size_t)C * C * 2) &&
+       h->alloc(&x.w_q2, (size_t)C * C * 2) && h->alloc(&x.w_o2, (size_t)C * C * 2) &&
+       h->alloc(&x.w_k2, (size_t)C * D * 2) && h->alloc(&x.w_v2, (size_t)C * D * 2) &&
+       h->alloc(&x.w_ff1, 2 * F * C * 2) && h->alloc(&x.w_ff2, (size_t)C * F * 2);
+  ok = ok && h->alloc((void**)&x.b_o1, C * 4) && h->alloc((void**)&x.b_o2, C * 4) &&
+       h->alloc((void**)&x.b_ff1, 2 * F * 4) && h->alloc((void**)&x.b_ff2, C * 4);
+  for (int i = 0; i < 2 && ok; ++i) {
+    ok = h->alloc(&x.kb[i], map) && h->alloc(&x.vb[i], map);
+    if (ok) ok = cudaMemset(x.kb[i], 0, map) == cudaSuccess && cudaMemset(x.vb[i], 0, map) == cudaSuccess;
+  }
+  const size_t cbytes = (size_t)x.heads * ctx_all * 64 * 2;
+  ok = ok && h->alloc(&x.ctx_k, cbytes) && h->alloc(&x.ctx_v, cbytes);
+  if (ok) ok = cudaMemset(x.ctx_k, 0, cbytes) == cudaSuccess && cudaMemset(x.ctx_v, 0, cbytes) == cudaSuccess;
+  return ok;
+}
+
+// TMA maps and plan of a conv over its slab (tile geometry as in the layer block)
+bool plan_conv(UConv& cv, int N) {
+  const Level& lv = cv.lv;
+  int cols_tile = lv.W < 128 ? lv.W : 128;
+  const int tpr = (lv.W + cols_tile - 1) / cols_tile;
+  int rows_tile = 128 / cols_tile;
+  if (rows_tile < 1) rows_tile = 1;
+  while (lv.R % rows_tile) --rows_tile;
+  bool ok = true;
+  for (int i = 0; i < 2; ++i) {
+    const uint64_t dims[4] = {(uint64_t)cv.Cin, (uint64_t)lv.W, (uint64_t)(lv.R + 2), (uint64_t)N};
+    const uint64_t str[3] = {(uint64_t)cv.Cin * 2, (uint64_t)lv.W * cv.Cin * 2, (uint64_t)(lv.R + 2) * lv.W * cv.Cin * 2};
+    const uint32_t box[4] = {64, (uint32_t)cols_tile, (uint32_t)rows_tile, 1};
+    ok &= encode_tmap_4d(&cv.m_slab[i], cv.slab[i], dims, str, box);
+  }
+  const int m_tiles = N * (lv.R / rows_tile) * tpr;
+  const GemmChoice gc = choose_gemm(cv.Cout, m_tiles, conv_k_stages(cv.Cin));
+  ok &= encode_gemm_rows(&cv.m_w, cv.w, cv.Cout, 9ull * cv.Cin, gc.b_box_rows());
+  TcGemmPlan& p = cv.plan;
+  p = TcGemmPlan{};
+  p.M = lv.L; p.N = cv.Cout; p.K = 9 * cv.Cin; p.bn = gc.bn; p.pair = gc.pair; p.conv = 1;
+  p.P = N; p.R = lv.R; p.W = lv.W; p.Cin = cv.Cin;
+  p.cols_tile = cols_tile; p.rows_tile = rows_tile; p.tiles_per_row = tpr;
+  return ok;
+}
+
+void plain_plan(TcGemmPlan& p, int M, int Nn, int K, const GemmChoice& g) {
+  p = TcGemmPlan{};
+  p.M = M; p.N = Nn; p.K = K; p.bn = g.bn; p.pair = g.pair;
+}
+
+bool plan_res(URes& r, int N) {
+  bool ok = plan_conv(r.c1, N) && plan_conv(r.c2, N);
+  if (r.sc) {
+    const GemmChoice g = choose_gemm(r.Cout, gemm_m_tiles_plain(r.lv.L), gemm_k_stages(r.Cin));
+    ok &= encode_gemm_rows(&r.m_in, r.in, r.lv.L, r.Cin, 128);
+    ok &= encode_gemm_rows(&r.m_wsc, r.w_sc, r.Cout, r.Cin, g.b_box_rows());
+    plain_plan(r.p_sc, r.lv.L, r.Cout, r.Cin, g);
+  }
+  return ok;
+}
+
+bool plan_xf(UXf& x, void* q, void* o, void* u, void* g, size_t ctx_all) {
+  const int L = x.lv.L, C = x.C, F = x.F, heads = x.heads;
+  const int lin_m = gemm_m_tiles_plain(L), ks = gemm_k_stages(C);
+  const GemmChoice bq = choose_gemm(3 * C, lin_m, ks), bc = choose_gemm(C, lin_m, ks);
+  const GemmChoice bf1 = choose_gemm(2 * F, lin_m, ks, 128);
+  const GemmChoice b2 = choose_gemm(C, lin_m, gemm_k_stages(F));
+  bool ok = true;
+  ok &= encode_gemm_rows(&x.m_wqkv, x.w_qkv, 3ull * C, C, bq.b_box_rows());
+  ok &= encode_gemm_rows(&x.m_wo1, x.w_o1, C, C, bc.b_box_rows());
+  ok &= encode_gemm_rows(&x.m_wq2, x.w_q2, C, C, bc.b_box_rows());
+  ok &= encode_gemm_rows(&x.m_wo2, x.w_o2, C, C, bc.b_box_rows());
+  ok &= encode_gemm_rows(&x.m_wff1, x.w_ff1, 2ull * F, C, bf1.b_box_rows());
+  ok &= encode_gemm_rows(&x.m_wff2, x.w_ff2, C, F, b2.b_box_rows());
+  for (int i = 0; i < 2; ++i) {
+    ok &= encode_attn_k(&x.m_k[i], x.kb[i], L, heads);
+    ok &= encode_attn_v(&x.m_v[i], x.vb[i], L, heads);
+  }
+  ok &= encode_attn_k(&x.m_ck, x.ctx_k, ctx_all, heads);
+  ok &= encode_attn_v(&x.m_cv, x.ctx_v, ctx_all, heads);
+  ok &= encode_tmap_3d(&x.m_q, q, 64, L, heads, 128, (uint64_t)L * 128, 64, 128, 1);
+  ok &= encode_gemm_rows(&x.m_u, u, L, C, 128);
+  ok &= encode_gemm_rows(&x.m_o, o, L, C, 128);
+  ok &= encode_gemm_rows(&x.m_g, g, L, F, 128);
+  plain_plan(x.p_qkv, L, 3 * C, C, bq);
+  plain_plan(x.p_o1, L, C, C, bc);
+  plain_plan(x.p_q2, L, C, C, bc);
+  plain_plan(x.p_o2, L, C, C, bc);
+  plain_plan(x.p_ff1, L, 2 * F, C, bf1);
+  plain_plan(x.p_ff2, L, C, F, b2);
+  return ok;
+}
+
+// Register the weights of a ResNet block under prefix p (names and PyTorch shapes).
+void reg_res(Unet* u, const std::string& p, URes& r) {
+  const long long ci = r.Cin, co = r.Cout, te = u->temb;
+  auto& E = u->entries;
+  URes* R = &r;
+  E.push_back({p + "norm1.weight", {ci}, [R](dfp_ctx* h, const std::vector<float>& v) { return up_f32(h, R->n1.g, v); }});
+  E.push_back({p + "norm1.bias", {ci}, [R](dfp_ctx* h, const std::vector<float>& v) { return up_f32(h, R->n1.b, v); }});
+  E.push_back({p + "conv1.weight", {co, ci, 3, 3},
+               [R](dfp_ctx* h, const std::vector<float>& v) { return up_conv(h, R->c1, R->Cout, R->Cin, v); }});
+  E.push_back({p + "conv1.bias", {co}, [R](dfp_ctx* h, const std::vector<float>& v) { return up_f32(h, R->c1.b, v); }});
+  E.push_back({p + "time_emb_proj.weight", {co, te},
+               [R](dfp_ctx* h, const std::vector<float>& v) { return up_f32(h, R->wt, v); }});
+  E.push_back({p + "time_emb_proj.bias", {co}, [R](dfp_ctx* h, const std::vector<float>& v) { return up_f32(h, R->bt, v); }});
+  E.push_back({p + "norm2.weight", {co}, [R](dfp_ctx* h, const std::vector<float>& v) { return up_f32(h, R->n2.g, v); }});
+  E.push_back({p + "norm2.bias", {co}, [R](dfp_ctx* h, const std::vector<float>& v) { return up_f32(h, R->n2.b, v); }});
+  E.push_back({p + "conv2.weight", {co, co, 3, 3},
+               [R](dfp_ctx* h, const std::vector<float>& v) { return up_conv(h, R->c2, R->Cout, R->Cout, v); }});
+  E.push_back({p + "conv2.bias", {co}, [R](dfp_ctx* h, const std::vector<float>& v) { return up_f32(h, R->c2.b, v); }});
+  if (r.sc) {
+    E.push_back({p + "conv_shortcut.weight", {co, ci},
+                 [R](dfp_ctx* h, const std::vector<float>& v) { return up_bf16(h, R->w_sc, v); }});
+    E.push_back({p + "conv_shortcut.bias", {co},
+                 [R](dfp_ctx* h, const std::vector<float>& v) { return up_f32(h, R->b_sc, v); }});
+  }
+}
+
+void reg_xf(Unet* u, const std::string& p, UXf& x, long long D) {
+  const long long C = x.C, F = x.F;
+  auto& E = u->entries;
+  UXf* X = &x;
+  const char* norms[3] = {"norm1", "norm2", "norm3"};
+  for (int k = 0; k < 3; ++k) {
+    E.push_back({p + norms[k] + ".weight", {C},
+                 [X, k](dfp_ctx* h, const std::vector<float>& v) { return up_f32(h, X->ln_g[k], v); }});
+    E.push_back({p + norms[k] + ".bias", {C},
+                 [X, k](dfp_ctx* h, const std::vector<float>& v) { return up_f32(h, X->ln_b[k], v); }});
+  }
+  const char* qkv[3] = {"attn1.to_q.weight", "attn1.to_k.weight", "attn1.to_v.weight"};
+  for (int k = 0; k < 3; ++k)
+    E.push_back({p + qkv[k], {C, C}, [X, k](dfp_ctx* h, const std::vector<float>& v) {
+                   return up_bf16(h, static_cast<uint8_t*>(X->w_qkv) + (size_t)k * X->C * X->C * 2, v);
+                 }});
+  E.push_back({p + "attn1.to_out.weight", {C, C}, [X](dfp_ctx* h, const std::vector<float>& v) { return up_bf16(h, X->w_o1, v); }});
+  E.push_back({p + "attn1.to_out.bias", {C}, [X](dfp_ctx* h, const std::vector<float>& v) { return up_f32(h, X->b_o1, v); }});
+  E.push_back({p + "attn2.to_q.weight", {C, C}, [X](dfp_ctx* h, const std::vector<float>& v) { return up_bf16(h, X->w_q2, v); }});
+  E.push_back({p + "attn2.to_k.weight", {C, D}, [X](dfp_ctx* h, const std::vector<float>& v) {
+                 X->ctx_ready = false;
+                 return up_bf16(h, X->w_k2, v);
+               }});
+  E.push_back({p + "attn2.to_v.weight", {C, D}, [X](dfp_ctx* h, const std::vector<float>& v) {
+                 X->ctx_ready = false;
+                 return up_bf16(h, X->w_v2, v);
+               }});
+  E.push_back({p + "attn2.to_out.weight", {C, C}, [X](dfp_ctx* h, const std::vector<float>& v) { return up_bf16(h, X->w_o2, v); }});
+  E.push_back({p + "attn2.to_out.bias", {C}, [X](dfp_ctx* h, const std::vector<float>& v) { return up_f32(h, X->b_o2, v); }});
+  // GEGLU projection: per 128-row tile, 64 value rows (f0..f0+63) then their 64 gate rows
+  auto interleave = [](const std::vector<float>& v, size_t F2, size_t cols) {
+    const size_t Fh = F2 / 2;
+    std::vector<float> r(v.size());
+    for (size_t t = 0; t < F2 / 128; ++t)
+      for (size_t j = 0; j < 128; ++j) {
+        const size_t src = j < 64 ? 64 * t + j : Fh + 64 * t + (j - 64);
+        std::memcpy(&r[(t * 128 + j) * cols], &v[src * cols], cols * 4);
+      }
+    return r;
+  };
+  E.push_back({p + "ff.proj.weight", {2 * F, C}, [X, interleave](dfp_ctx* h, const std::vector<float>& v) {
+                 return up_bf16(h, X->w_ff1, interleave(v, 2 * X->F, X->C));
+               }});
+  E.push_back({p + "ff.proj.bias", {2 * F}, [X, interleave](dfp_ctx* h, const std::vector<float>& v) {
+                 return up_f32(h, X->b_ff1, interleave(v, 2 * X->F, 1));
+               }});
+  E.push_back({p + "ff.out.weight", {C, F}, [X](dfp_ctx* h, const std::vector<float>& v) { return up_bf16(h, X->w_ff2, v); }});
+  E.push_back({p + "ff.out.bias", {C}, [X](dfp_ctx* h, const std::vector<float>& v) { return up_f32(h, X->b_ff2, v); }});
+}
+
+}  // namespace
+
+dfp_status unet_create(dfp_ctx* h) {
+  const dfp_config& c = h->cfg;
+  Unet* u = new (std::nothrow) Unet();
+  if (!u) return h->fail(DFP_E_NOMEM, "host allocation failed");
+  h->unet = u;
+  const int N = c.n_patches, G = c.gn_groups, D = c.ctx_dim;
+  u->c0 = c.C; u->c1 = 2 * c.C; u->c2 = 4 * c.C; u->temb = 4 * c.C;
+  for (int l = 0; l < 3; ++l) {
+    Level& lv = u->lv[l];
+    lv.H = c.H >> l; lv.W = c.W >> l; lv.R = lv.H / N; lv.L = lv.H * lv.W; lv.Lp = lv.R * lv.W;
+  }
+  const Level &l0 = u->lv[0], &l1 = u->lv[1], &l2 = u->lv[2];
+  const int c0 = u->c0, c1 = u->c1, c2 = u->c2, te = u->temb;
+  const size_t ctx_all = ctx_rows(c.ctx_len);
+  bool ok = h->alloc((void**)&u->t_w1, (size_t)te * c0 * 4) && h->alloc((void**)&u->t_b1, te * 4) &&
+            h->alloc((void**)&u->t_w2, (size_t)te * te * 4) && h->alloc((void**)&u->t_b2, te * 4) &&
+            h->alloc((void**)&u->t_h, te * 4) && h->alloc((void**)&u->t_act, te * 4);
+  ok = ok && alloc_conv(h, u->conv_in, l0, N, 64, c0);
+  ok = ok && alloc_res(h, u->res0, l0, N, G, c0, c0, te);
+  ok = ok && alloc_conv(h, u->down0, l0, N, c0, c0);
+  ok = ok && alloc_res(h, u->res1, l1, N, G, c0, c1, te) && alloc_xf(h, u->xf1, l1, c1, ctx_all, D);
+  ok = ok && alloc_conv(h, u->down1, l1, N, c1, c1);
+  ok = ok && alloc_res(h, u->res2, l2, N, G, c1, c2, te) && alloc_xf(h, u->xf2, l2, c2, ctx_all, D);
+  ok = ok && alloc_conv(h, u->up1, l1, N, c2, c2);
+  ok = ok && alloc_res(h, u->ures1, l1, N, G, c2 + c1, c1, te) && alloc_xf(h, u->uxf1, l1, c1, ctx_all, D);
+  ok = ok && alloc_conv(h, u->up0, l0, N, c1, c1);
+  ok = ok && alloc_res(h, u->ures0, l0, N, G, c1 + c0, c0, te);
+  ok = ok && alloc_gn(h, u->gn_out, c0, N, G) && alloc_conv(h, u->conv_out, l0, N, c0, 64);
+  ok = ok && h->alloc(&u->h0, (size_t)l0.L * c0 * 2) && h->alloc(&u->d0, (size_t)l1.L * c0 * 2) &&
+       h->alloc(&u->d1, (size_t)l2.L * c1 * 2) && h->alloc(&u->u1, (size_t)l1.L * c2 * 2) &&
+       h->alloc(&u->u0, (size_t)l0.L * c1 * 2) && h->alloc(&u->cat1, (size_t)l1.L * (c2 + c1) * 2) &&
+       h->alloc(&u->cat0, (size_t)l0.L * (c1 + c0) * 2) && h->alloc(&u->eps, (size_t)l0.L * 4 * 2) &&
+       h->alloc(&u->x_in, (size_t)l0.L * 4 * 2) && h->alloc((void**)&u->lat, (size_t)l0.L * 4 * 4);
+  const size_t umax = std::max((size_t)l1.L * c1, (size_t)l2.L * c2);
+  const size_t gmax = std::max((size_t)l1.L * 4 * c1, (size_t)l2.L * 4 * c2);
+  ok = ok && h->alloc(&u->u, umax * 2) && h->alloc(&u->g, gmax * 2) && h->alloc(&u->ctx, (size_t)c.ctx_len * D * 2);
+  if (!ok) return h->fail(DFP_E_NOMEM, "device allocation failed");
+  // the blocks' inputs and outputs: the transformers run in place on their ResNet's output
+  u->s0 = u->res0.out;
+  u->res0.in = u->h0;
+  u->res1.in = u->d0;
+  u->xf1.r = u->res1.out;
+  u->res2.in = u->d1;
+  u->xf2.r = u->res2.out;
+  u->ures1.in = u->cat1;
+  u->uxf1.r = u->ures1.out;
+  u->ures0.in = u->cat0;
+  ok = plan_conv(u->conv_in, N) && plan_res(u->res0, N) && plan_conv(u->down0, N) && plan_res(u->res1, N) &&
+       plan_conv(u->down1, N) && plan_res(u->res2, N) && plan_conv(u->up1, N) && plan_res(u->ures1, N) &&
+       plan_conv(u->up0, N) && plan_res(u->ures0, N) && plan_conv(u->conv_out, N);
+  ok = ok && plan_xf(u->xf1, h->q, h->o, u->u, u->g, ctx_all) && plan_xf(u->xf2, h->q, h->o, u->u, u->g, ctx_all) &&
+       plan_xf(u->uxf1, h->q, h->o, u->u, u->g, ctx_all);
+  if (!ok) return h->fail(DFP_E_CUDA, "cuTensorMapEncodeTiled failed");
+  h->y = u->eps;
+  // ---- weight names (PyTorch shapes) and their loaders, in declaration order
+  auto& E = u->entries;
+  Unet* U = u;
+  E.push_back({"time_embedding.linear_1.weight", {te, c0}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_f32(hh, U->t_w1, v); }});
+  E.push_back({"time_embedding.linear_1.bias", {te}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_f32(hh, U->t_b1, v); }});
+  E.push_back({"time_embedding.linear_2.weight", {te, te}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_f32(hh, U->t_w2, v); }});
+  E.push_back({"time_embedding.linear_2.bias", {te}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_f32(hh, U->t_b2, v); }});
+  E.push_back({"conv_in.weight", {c0, 4, 3, 3}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_conv(hh, U->conv_in, U->c0, 4, v); }});
+  E.push_back({"conv_in.bias", {c0}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_f32(hh, U->conv_in.b, v); }});
+  reg_res(u, "down0.resnet.", u->res0);
+  E.push_back({"down0.downsample.weight", {c0, c0, 3, 3}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_conv(hh, U->down0, U->c0, U->c0, v); }});
+  E.push_back({"down0.downsample.bias", {c0}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_f32(hh, U->down0.b, v); }});
+  reg_res(u, "down1.resnet.", u->res1);
+  reg_xf(u, "down1.xf.", u->xf1, D);
+  E.push_back({"down1.downsample.weight", {c1, c1, 3, 3}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_conv(hh, U->down1, U->c1, U->c1, v); }});
+  E.push_back({"down1.downsample.bias", {c1}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_f32(hh, U->down1.b, v); }});
+  reg_res(u, "down2.resnet.", u->res2);
+  reg_xf(u, "down2.xf.", u->xf2, D);
+  E.push_back({"up1.upsample.weight", {c2, c2, 3, 3}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_conv(hh, U->up1, U->c2, U->c2, v); }});
+  E.push_back({"up1.upsample.bias", {c2}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_f32(hh, U->up1.b, v); }});
+  reg_res(u, "up1.resnet.", u->ures1);
+  reg_xf(u, "up1.xf.", u->uxf1, D);
+  E.push_back({"up0.upsample.weight", {c1, c1, 3, 3}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_conv(hh, U->up0, U->c1, U->c1, v); }});
+  E.push_back({"up0.upsample.bias", {c1}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_f32(hh, U->up0.b, v); }});
+  reg_res(u, "up0.resnet.", u->ures0);
+  E.push_back({"norm_out.weight", {c0}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_f32(hh, U->gn_out.g, v); }});
+  E.push_back({"norm_out.bias", {c0}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_f32(hh, U->gn_out.b, v); }});
+  E.push_back({"conv_out.weight", {4, c0, 3, 3}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_conv(hh, U->conv_out, 4, U->c0, v); }});
+  E.push_back({"conv_out.bias", {4}, [U](dfp_ctx* hh, const std::vector<float>& v) { return up_f32(hh, U->conv_out.b, v); }});
+  E.push_back({"context", {(long long)c.ctx_len, (long long)D}, [U](dfp_ctx* hh, const std::vector<float>& v) {
+                 U->ctx_loaded = true;
+                 for (UXf* x : {&U->xf1, &U->xf2, &U->uxf1}) x->ctx_ready = false;
+                 return up_bf16(hh, U->ctx, v);
+               }});
+  return DFP_OK;
+}
+
+std::vector<WeightSpec> unet_weight_specs(dfp_ctx* h) {
+  std::vector<WeightSpec> out;
+  for (const auto& e : h->unet->entries) out.push_back(WeightSpec{e.name.c_str(), e.shape});
+  return out;
+}
+
+bool unet_load_weight(dfp_ctx* h, const std::string& name, const std::vector<float>& v, dfp_status& st) {
+  for (auto& e : h->unet->entries)
+    if (e.name == name) {
+      st = e.load(h, v);
+      return true;
+    }
+  return false;
+}
+
+dfp_status unet_finish_load(dfp_ctx* h) {
+  // context K/V of every transformer: [ctx_len, ctx_dim] x W^T -> head-major, padded rows zero
+  Unet* u = h->unet;
+  const dfp_config& c = h->cfg;
+  if (!u->ctx_loaded) return DFP_OK;
+  const std::string names[3] = {"down1.xf.", "down2.xf.", "up1.xf."};
+  UXf* xs[3] = {&u->xf1, &u->xf2, &u->uxf1};
+  for (int i = 0; i < 3; ++i) {
+    UXf& x = *xs[i];
+    if (x.ctx_ready || !h->loaded.count(names[i] + "attn2.to_k.weight") ||
+        !h->loaded.count(names[i] + "attn2.to_v.weight"))
+      continue;
+    for (int kv = 0; kv < 2; ++kv) {
+      Epilogue e{};
+      e.kind = 1;
+      e.q = kv == 0 ? x.ctx_k : x.ctx_v;
+      e.L = (int)ctx_rows(c.ctx_len);
+      e.C = x.C;
+      cudaError_t ce = launch_simt_gemm<bf>(static_cast<const bf*>(u->ctx), nullptr,
+                                            static_cast<const bf*>(kv == 0 ? x.w_k2 : x.w_v2), c.ctx_len, x.C,
+                                            c.ctx_dim, e, h->stream);
+      if (ce != cudaSuccess) return h->cuda_fail(ce, "context projection");
+    }
+    cudaError_t ce = cudaStreamSynchronize(h->stream);
+    if (ce != cudaSuccess) return h->cuda_fail(ce, "context projection");
+    x.ctx_ready = true;
+  }
+  return DFP_OK;
+}
+
+namespace {
+
+struct StepCtx {
+  int cur, prv, is_sync, naive, halo_mode, sa_mode, pdl, N, G, gn_mode;
+  float eps;
+};
+
+// GroupNorm (+SiLU) of x [L][C] into conv cv's input slab (with its halo rows)
+cudaError_t gn_into(dfp_ctx* h, const StepCtx& k, UGn& gn, const void* x, UConv& cv) {
+  const Level& lv = cv.lv;
+  GnArgs g{};
+  g.x = x; g.N = k.N; g.per_image = k.N; g.pix_per_patch = lv.Lp; g.C = gn.C; g.G = k.G; g.eps = k.eps;
+  g.part = h->part; g.counter = h->counter;
+  g.fresh_out = gn.mom[k.cur]; g.stale = gn.mom[k.prv]; g.gamma = gn.g; g.beta = gn.b; g.mean_rstd = h->mr1;
+  g.is_sync = k.is_sync; g.mode = k.gn_mode; g.naive = k.naive; g.pdl = k.pdl;
+  const GnOut go{cv.slab[k.cur], cv.slab[k.prv], (long long)(lv.R + 2) * lv.W, lv.W, lv.W, k.halo_mode};
+  return launch_gn_fused<bf>(g, go, true, h->dev_err, h->stream);
+}
+
+cudaError_t conv_run(dfp_ctx* h, const StepCtx& k, UConv& cv, const Epilogue& ep) {
+  cv.plan.pdl = k.pdl;
+  return launch_tc_gemm(cv.plan, cv.m_slab[k.cur], cv.m_w, ep, h->dev_err, h->stream);
+}
+
+Epilogue plain_out(void* out, const float* bias, int ldo, const void* residual = nullptr) {
+  Epilogue e{};
+  e.kind = 0; e.out = out; e.bias = bias; e.ldo = ldo; e.residual = residual;
+  return e;
+}
+
+// Kernel names of one layer's launches (static strings: the profiling events keep them).
+struct ResNames { const char *n1, *c1, *n2, *sc, *c2; };
+struct XfNames { const char *ln1, *qkv, *sa, *o1, *ln2, *q2, *ca, *o2, *ln3, *ff1, *ff2; };
+#define DFP_RES_NAMES(P) {P " norm1 + SiLU (fused)", P " conv1 + time (tcgen05)", P " norm2 + SiLU (fused)", \
+                          P " shortcut (tcgen05)", P " conv2 + residual (tcgen05)"}
+#define DFP_XF_NAMES(P) {P " layernorm 1", P " self-attn qkv (tcgen05)", P " self-attention (tcgen05)",          \
+                         P " self-attn out + residual (tcgen05)", P " layernorm 2", P " cross-attn q (tcgen05)",   \
+                         P " cross-attention (tcgen05)", P " cross-attn out + residual (tcgen05)",               \
+                         P " layernorm 3", P " ff proj + GEGLU (tcgen05)", P " ff out + residual (tcgen05)"}
+const ResNames kRes0 = DFP_RES_NAMES("res0"), kRes1 = DFP_RES_NAMES("res1"), kRes2 = DFP_RES_NAMES("res2"),
+               kURes1 = DFP_RES_NAMES("up1 res"), kURes0 = DFP_RES_NAMES("up0 res");
+const XfNames kXf1 = DFP_XF_NAMES("xf1"), kXf2 = DFP_XF_NAMES("xf2"), kUXf1 = DFP_XF_NAMES("up1 xf");
+#undef DFP_RES_NAMES
+#undef DFP_XF_NAMES
+
+dfp_status run_res(dfp_ctx* h, const StepCtx& k, URes& r, const ResNames& nm, int& launches) {
+  cudaStream_t s = h->stream;
+  cudaError_t e;
+  DFP_LAUNCH(gn_into(h, k, r.n1, r.in, r.c1), nm.n1);
+  DFP_LAUNCH(conv_run(h, k, r.c1, plain_out(r.h1, r.bias1, r.Cout)), nm.c1);
+  DFP_LAUNCH(gn_into(h, k, r.n2, r.h1, r.c2), nm.n2);
+  if (r.sc) {
+    r.p_sc.pdl = k.pdl;
+    DFP_LAUNCH(launch_tc_gemm(r.p_sc, r.m_in, r.m_wsc, plain_out(r.sc_out, r.b_sc, r.Cout), h->dev_err, s), nm.sc);
+  }
+  DFP_LAUNCH(conv_run(h, k, r.c2, plain_out(r.out, r.c2.b, r.Cout, r.sc ? r.sc_out : r.in)), nm.c2);
+  return DFP_OK;
+}
+
+dfp_status run_xf(dfp_ctx* h, const StepCtx& k, UXf& x, const XfNames& nm, int& launches) {
+  cudaStream_t s = h->stream;
+  cudaError_t e;
+  const dfp_config& c = h->cfg;
+  const int L = x.lv.L, C = x.C, pdl = k.pdl;
+  Unet* u = h->unet;
+  for (TcGemmPlan* p : {&x.p_qkv, &x.p_o1, &x.p_q2, &x.p_o2, &x.p_ff1, &x.p_ff2}) p->pdl = pdl;
+  // self-attention on displaced K/V
+  DFP_LAUNCH(launch_layernorm(x.r, u->u, x.ln_g[0], x.ln_b[0], L, C, 1e-5f, pdl != 0, s), nm.ln1);
+  Epilogue eq{};
+  eq.kind = 1; eq.q = h->q; eq.k = x.kb[k.cur]; eq.v = x.vb[k.cur]; eq.L = L; eq.C = C;
+  DFP_LAUNCH(launch_tc_gemm(x.p_qkv, x.m_u, x.m_wqkv, eq, h->dev_err, s), nm.qkv);
+  TcAttnArgs a{};
+  a.L = L; a.Lp = x.lv.Lp; a.N = k.N; a.heads = x.heads; a.C = C; a.mode = k.sa_mode; a.o = h->o; a.err = h->dev_err;
+  a.images = 1; a.kv_stride = L; a.pdl = pdl; a.n_qtiles = (x.lv.Lp + 127) / 128; a.ctas = h->attn_ctas;
+  a.part_o = h->attn_part_o; a.part_ml = h->attn_part_ml; a.flags = h->attn_flags;
+  DFP_LAUNCH(launch_tc_attention(a, x.m_q, x.m_k[k.cur], x.m_v[k.cur], x.m_k[k.prv], x.m_v[k.prv], s),
+             nm.sa);
+  DFP_LAUNCH(launch_tc_gemm(x.p_o1, x.m_o, x.m_wo1, plain_out(x.r, x.b_o1, C, x.r), h->dev_err, s),
+             nm.o1);
+  // cross-attention to the fixed context
+  DFP_LAUNCH(launch_layernorm(x.r, u->u, x.ln_g[1], x.ln_b[1], L, C, 1e-5f, pdl != 0, s), nm.ln2);
+  Epilogue e2{};
+  e2.kind = 1; e2.q = h->q; e2.L = L; e2.C = C;
+  DFP_LAUNCH(launch_tc_gemm(x.p_q2, x.m_u, x.m_wq2, e2, h->dev_err, s), nm.q2);
+  TcAttnArgs ca{};
+  ca.L = L; ca.Lp = L; ca.N = 1; ca.heads = x.heads; ca.C = C; ca.mode = kAttnCross; ca.kv_len = c.ctx_len;
+  ca.images = 1; ca.kv_stride = (int)ctx_rows(c.ctx_len); ca.pdl = pdl;
+  ca.o = h->o; ca.err = h->dev_err; ca.n_qtiles = (L + 127) / 128; ca.ctas = h->attn_ctas;
+  ca.part_o = h->attn_part_o; ca.part_ml = h->attn_part_ml; ca.flags = h->attn_flags;
+  DFP_LAUNCH(launch_tc_attention(ca, x.m_q, x.m_ck, x.m_cv, x.m_ck, x.m_cv, s), nm.ca);
+  DFP_LAUNCH(launch_tc_gemm(x.p_o2, x.m_o, x.m_wo2, plain_out(x.r, x.b_o2, C, x.r), h->dev_err, s),
+             nm.o2);
+  // GEGLU feed-forward
+  DFP_LAUNCH(launch_layernorm(x.r, u->u, x.ln_g[2], x.ln_b[2], L, C, 1e-5f, pdl != 0, s), nm.ln3);
+  Epilogue ef{};
+  ef.kind = 2; ef.out = u->g; ef.bias = x.b_ff1; ef.ldo = x.F;
+  DFP_LAUNCH(launch_tc_gemm(x.p_ff1, x.m_u, x.m_wff1, ef, h->dev_err, s), nm.ff1);
+  DFP_LAUNCH(launch_tc_gemm(x.p_ff2, x.m_g, x.m_wff2, plain_out(x.r, x.b_ff2, C, x.r), h->dev_err, s),
+             nm.ff2);
+  return DFP_OK;
+}
+
+}  // namespace
+
+dfp_status unet_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
+  Unet* u = h->unet;
+  const dfp_config& c = h->cfg;
+  for (UXf* x : {&u->xf1, &u->xf2, &u->uxf1})
+    if (!x->ctx_ready) return h->fail(DFP_E_STATE, "cross-attention context not projected (load the context)");
+  StepCtx k{};
+  k.cur = step & 1; k.prv = k.cur ^ 1; k.is_sync = is_sync;
+  k.naive = c.context == DFP_CTX_NAIVE ? 1 : 0;
+  const bool displaced = !is_sync && !k.naive;
+  k.N = c.n_patches; k.G = c.gn_groups; k.eps = c.gn_eps; k.gn_mode = (int)c.gn_mode;
+  k.halo_mode = (k.naive || k.N == 1) ? 0 : (displaced ? 2 : 1);
+  k.sa_mode = k.naive ? kAttnNaive : (is_sync ? kAttnSync : kAttnDisplaced);
+  k.pdl = h->overlap ? 1 : 0;
+  cudaStream_t s = h->stream;
+  int launches = 0;
+  cudaError_t e;
+  h->n_ev = 0;
+  dfp_status st;
+  const int c0 = u->c0, c1 = u->c1, c2 = u->c2, te = u->temb, N = k.N;
+  const Level &l0 = u->lv[0], &l1 = u->lv[1];
+  // ---- timestep embedding, and every ResNet's conv1 bias for this step
+  DFP_LAUNCH(launch_gemv(u->t_w1, u->t_b1, nullptr, nullptr, u->tau, u->t_h, te, c0, true, k.pdl != 0, s),
+             "timestep embedding 1");
+  DFP_LAUNCH(launch_gemv(u->t_w2, u->t_b2, nullptr, u->t_h, -1.f, u->t_act, te, te, true, k.pdl != 0, s),
+             "timestep embedding 2");
+  for (URes* r : {&u->res0, &u->res1, &u->res2, &u->ures1, &u->ures0})
+    DFP_LAUNCH(launch_gemv(r->wt, r->bt, r->c1.b, u->t_act, -1.f, r->bias1, r->Cout, te, false, k.pdl != 0, s),
+               "time projections");
+  // ---- down path
+  DFP_LAUNCH(launch_slab_fill(xv, 4, u->conv_in.slab[k.cur], u->conv_in.slab[k.prv], 64, N, l0.R, l0.W, k.halo_mode,
+                              false, k.pdl != 0, s), "conv_in input");
+  DFP_LAUNCH(conv_run(h, k, u->conv_in, plain_out(u->h0, u->conv_in.b, c0)), "conv_in (tcgen05)");
+  if ((st = run_res(h, k, u->res0, kRes0, launches)) != DFP_OK) return st;
+  DFP_LAUNCH(launch_slab_fill(u->s0, c0, u->down0.slab[k.cur], u->down0.slab[k.prv], c0, N, l0.R, l0.W, k.halo_mode,
+                              false, k.pdl != 0, s), "down0 input");
+  {
+    Epilogue ed = plain_out(u->d0, u->down0.b, c0);
+    ed.subsample = 1;
+    DFP_LAUNCH(conv_run(h, k, u->down0, ed), "down0 stride-2 conv (tcgen05)");
+  }
+  if ((st = run_res(h, k, u->res1, kRes1, launches)) != DFP_OK) return st;
+  if ((st = run_xf(h, k, u->xf1, kXf1, launches)) != DFP_OK) return st;
+  DFP_LAUNCH(launch_slab_fill(u->xf1.r, c1, u->down1.slab[k.cur], u->down1.slab[k.prv], c1, N, l1.R, l1.W,
+                              k.halo_mode, false, k.pdl != 0, s), "down1 input");
+  {
+    Epilogue ed = plain_out(u->d1, u->down1.b, c1);
+    ed.subsample = 1;
+    DFP_LAUNCH(conv_run(h, k, u->down1, ed), "down1 stride-2 conv (tcgen05)");
+  }
+  if ((st = run_res(h, k, u->res2, kRes2, launches)) != DFP_OK) return st;
+  if ((st = run_xf(h, k, u->xf2, kXf2, launches)) != DFP_OK) return st;
+  // ---- up path
+  DFP_LAUNCH(launch_slab_fill(u->xf2.r, c2, u->up1.slab[k.cur], u->up1.slab[k.prv], c2, N, l1.R, l1.W, k.halo_mode,
+                              true, k.pdl != 0, s), "up1 input (x2)");
+  DFP_LAUNCH(conv_run(h, k, u->up1, plain_out(u->u1, u->up1.b, c2)), "up1 conv (tcgen05)");
+  DFP_LAUNCH(launch_concat(u->u1, c2, u->xf1.r, c1, u->cat1, l1.L, k.pdl != 0, s), "concat skip 1");
+  if ((st = run_res(h, k, u->ures1, kURes1, launches)) != DFP_OK) return st;
+  if ((st = run_xf(h, k, u->uxf1, kUXf1, launches)) != DFP_OK) return st;
+  DFP_LAUNCH(launch_slab_fill(u->uxf1.r, c1, u->up0.slab[k.cur], u->up0.slab[k.prv], c1, N, l0.R, l0.W, k.halo_mode,
+                              true, k.pdl != 0, s), "up0 input (x2)");
+  DFP_LAUNCH(conv_run(h, k, u->up0, plain_out(u->u0, u->up0.b, c1)), "up0 conv (tcgen05)");
+  DFP_LAUNCH(launch_concat(u->u0, c1, u->s0, c0, u->cat0, l0.L, k.pdl != 0, s), "concat skip 0");
+  if ((st = run_res(h, k, u->ures0, kURes0, launches)) != DFP_OK) return st;
+  // ---- output: GN + SiLU -> conv_out (4 of 64 computed channels stored)
+  DFP_LAUNCH(gn_into(h, k, u->gn_out, u->ures0.out, u->conv_out), "norm_out + SiLU (fused)");
+  {
+    Epilogue eo = plain_out(u->eps, u->conv_out.b, 4);
+    eo.n_store = 4;
+    DFP_LAUNCH(conv_run(h, k, u->conv_out, eo), "conv_out (tcgen05)");
+  }
+  DFP_LAUNCH_END();
+  return DFP_OK;
+}
+
+void unet_set_timestep(dfp_ctx* h, float tau) { h->unet->tau = tau; }
+
+dfp_status unet_ddim(dfp_ctx* h, const float* x_T, int n_steps, int n_sync, int n_train, float beta_start,
+                     float beta_end, float* x_out, dfp_status (*step_fn)(dfp_ctx*, const void*, int, int)) {
+  Unet* u = h->unet;
+  const long long n = (long long)u->lv[0].L * 4;
+  std::vector<double> ab(n_train);
+  double acc = 1.0;
+  for (int i = 0; i < n_train; ++i) {
+    const double sb = std::sqrt((double)beta_start) +
+                      (std::sqrt((double)beta_end) - std::sqrt((double)beta_start)) * i / (n_train - 1);
+    acc *= 1.0 - sb * sb;
+    ab[i] = acc;
+  }
+  const int ratio = n_train / n_steps;
+  cudaError_t e = cudaMemcpyAsync(u->lat, x_T, n * 4, cudaMemcpyDeviceToDevice, h->stream);
+  if (e == cudaSuccess) e = launch_to_bf16(u->lat, u->x_in, n, h->stream);
+  if (e != cudaSuccess) return h->cuda_fail(e, "DDIM start");
+  for (int k = 0; k < n_steps; ++k) {
+    const int tau = (n_steps - 1 - k) * ratio + 1;
+    u->tau = (float)tau;
+    dfp_status st = step_fn(h, u->x_in, k, k < n_sync ? 1 : 0);
+    if (st != DFP_OK) return st;
+    const double a = ab[tau], ap = k + 1 < n_steps ? ab[tau - ratio] : 1.0;
+    const double c1 = std::sqrt(ap / a), c2 = std::sqrt(1.0 - ap) - std::sqrt(ap * (1.0 - a) / a);
+    e = launch_ddim_update(u->lat, u->eps, u->x_in, n, (float)c1, (float)c2, h->overlap, h->stream);
+    if (e != cudaSuccess) return h->cuda_fail(e, "DDIM update");
+  }
+  e = cudaMemcpyAsync(x_out, u->lat, n * 4, cudaMemcpyDeviceToDevice, h->stream);
+  if (e != cudaSuccess) return h->cuda_fail(e, "DDIM result copy");
+  return DFP_OK;
+}
+
+bool unet_buffer(dfp_ctx* h, const std::string& name, const void** ptr, long long* bytes) {
+  Unet* u = h->unet;
+  const Level &l0 = u->lv[0], &l1 = u->lv[1], &l2 = u->lv[2];
+  if (name == "y" || name == "eps") { *ptr = u->eps; *bytes = (long long)l0.L * 4 * 2; return true; }
+  if (name == "lat") { *ptr = u->lat; *bytes = (long long)l0.L * 4 * 4; return true; }
+  if (name == "s0") { *ptr = u->s0; *bytes = (long long)l0.L * u->c0 * 2; return true; }
+  if (name == "s1") { *ptr = u->xf1.r; *bytes = (long long)l1.L * u->c1 * 2; return true; }
+  if (name == "mid") { *ptr = u->xf2.r; *bytes = (long long)l2.L * u->c2 * 2; return true; }
+  if (name == "up0") { *ptr = u->ures0.out; *bytes = (long long)l0.L * u->c0 * 2; return true; }
+  return false;
+}
+
+}  // namespace dfp

@@ -14,7 +14,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdfp.so"
 
 OK, E_ARG, E_STATE, E_CUDA, E_NOMEM, E_UNSUPPORTED, E_DEVICE = range(7)
 F32, BF16 = 0, 1
-BLOCK_RES_ATTN, BLOCK_SDXL_STAGE = 0, 1
+BLOCK_RES_ATTN, BLOCK_SDXL_STAGE, BLOCK_UNET = 0, 1, 2
 GN_CORRECTED, GN_STALE_OTHERS, GN_SYNC, GN_SEPARATE = 0, 1, 2, 3
 CTX_DISPLACED, CTX_NAIVE = 0, 1
 FAMILY_TENSOR_CORE, FAMILY_SIMT = 0, 1
@@ -25,7 +25,8 @@ EXPORTED = ("dfp_create", "dfp_load_weights", "dfp_step", "dfp_step_host", "dfp_
             "dfp_set_kernel_family", "dfp_set_profiling", "dfp_kernel_times", "dfp_destroy",
             "dfp_last_error", "dfp_group_norm_noalloc", "dfp_group_norm_noalloc_error",
             "dfp_selftest_wait_timeout", "dfp_selftest_exp2_poly", "dfp_set_launch_overlap",
-            "dfp_attention_schedule_check", "dfp_step_patches", "dfp_context_buffer")
+            "dfp_attention_schedule_check", "dfp_step_patches", "dfp_context_buffer", "dfp_set_timestep",
+            "dfp_ddim_sample")
 
 
 class Config(ctypes.Structure):
@@ -65,6 +66,9 @@ def load_library(path=_LIB_PATH):
         "dfp_set_launch_overlap": ([H, ctypes.c_int], ctypes.c_int),
         "dfp_attention_schedule_check": ([ctypes.c_int] * 10, ctypes.c_int),
         "dfp_step_patches": ([H, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int], ctypes.c_int),
+        "dfp_set_timestep": ([H, ctypes.c_float], ctypes.c_int),
+        "dfp_ddim_sample": ([H, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                             ctypes.c_float, ctypes.c_void_p], ctypes.c_int),
         "dfp_context_buffer": ([H, ctypes.c_char_p, ctypes.c_int, ctypes.POINTER(ctypes.c_void_p),
                                 ctypes.POINTER(ctypes.c_longlong)], ctypes.c_int),
         "dfp_set_profiling": ([H, ctypes.c_int], ctypes.c_int),
@@ -111,7 +115,7 @@ def make_config(cfg, gn_mode=GN_CORRECTED, context=CTX_DISPLACED):
     c.n_patches, c.gn_groups, c.gn_eps = cfg["n_patches"], cfg["gn_groups"], cfg["gn_eps"]
     c.heads, c.head_dim = cfg["heads"], cfg["head_dim"]
     c.dtype = _dtype_code(cfg["dtype"])
-    c.block = BLOCK_RES_ATTN if cfg["block"] == "res_attn" else BLOCK_SDXL_STAGE
+    c.block = {"res_attn": BLOCK_RES_ATTN, "sdxl_stage": BLOCK_SDXL_STAGE, "unet": BLOCK_UNET}[cfg["block"]]
     c.gn_mode, c.context = gn_mode, context
     c.n_xformer = cfg.get("n_xformer", 0)
     c.ffn_inner = cfg.get("ffn_inner", 0)
@@ -196,7 +200,7 @@ class DisplacedPatchBlock:
         """A fresh torch copy (on the device) of an internal buffer of the last step."""
         nbytes = ctypes.c_longlong()
         self._check(LIB.dfp_buffer_bytes(self.h, name.encode(), ctypes.byref(nbytes)))
-        if name.startswith("gn"):
+        if name.startswith("gn") or name == "lat":
             out = torch.empty(nbytes.value // 4, dtype=torch.float32, device="cuda")
         else:
             out = torch.empty(nbytes.value // (2 if self.dtype == BF16 else 4), dtype=self.tdtype, device="cuda")
@@ -204,7 +208,23 @@ class DisplacedPatchBlock:
         return out
 
     def output(self):
-        return self.buffer("y").view(self.cfg.get("batch", 1) * self.cfg["H"] * self.cfg["W"], self.cfg["C"])
+        cols = self.cfg["latent_c"] if self.cfg["block"] == "unet" else self.cfg["C"]
+        return self.buffer("y").view(self.cfg.get("batch", 1) * self.cfg["H"] * self.cfg["W"], cols)
+
+    def set_timestep(self, tau):
+        """UNet block: the timestep the next step embeds."""
+        self._check(LIB.dfp_set_timestep(self.h, float(tau)))
+
+    def ddim_sample(self, x_T, n_steps, n_sync, n_train=1000, beta_start=0.00085, beta_end=0.012, out=None):
+        """UNet block: the DDIM loop from x_T (CUDA fp32 [H, W, 4]); returns the final latent
+        (asynchronous on the handle's stream)."""
+        if not (x_T.is_cuda and x_T.is_contiguous() and x_T.dtype == torch.float32):
+            raise ValueError("x_T must be a contiguous CUDA fp32 tensor")
+        out = torch.empty_like(x_T) if out is None else out
+        self._check(LIB.dfp_ddim_sample(self.h, ctypes.c_void_p(x_T.data_ptr()), int(n_steps), int(n_sync),
+                                        int(n_train), float(beta_start), float(beta_end),
+                                        ctypes.c_void_p(out.data_ptr())))
+        return out
 
     def check_device(self):
         self._check(LIB.dfp_check_device(self.h))
@@ -217,9 +237,9 @@ class DisplacedPatchBlock:
 
     def kernel_times(self):
         """[(kernel name, milliseconds)] of the last profiled step."""
-        ms = (ctypes.c_float * 32)()
-        names = (ctypes.c_char_p * 32)()
-        n = LIB.dfp_kernel_times(self.h, ms, names, 32)
+        ms = (ctypes.c_float * 128)()
+        names = (ctypes.c_char_p * 128)()
+        n = LIB.dfp_kernel_times(self.h, ms, names, 128)
         if n < 0:
             raise DfpError(E_CUDA, "kernel timing failed")
         return [(names[i].decode(), float(ms[i])) for i in range(n)]
