@@ -278,19 +278,23 @@ DFP_API dfp_status dfp_check_device(dfp_handle h);
 DFP_API int dfp_launches_per_step(dfp_handle h);
 
 /* Host-side check of the tensor-core attention's work split (no counterpart in the
- * pages; no GPU needed).  Walks the list of (image, patch, head, query-tile pair, KV tile)
- * units as the kernel does, cut into `ctas` contiguous ranges, and checks: every range is
- * non-empty and its pieces stay inside their units; every unit is covered once; a pair
- * cut between CTAs has its first KV tiles at the end of one CTA's range (that CTA merges)
- * and its other pieces each at the start of a range; the kernel's publisher and flag
- * warps predict exactly those pieces.  L tokens per image in n_patches patches of Lp
- * tokens; mode 0 sync, 1 displaced, 2 naive, 3 cross-attention (Lp = L, n_patches = 1,
- * kv_len context tokens).  Only the query patches [p_begin, p_end) of the image-major
- * patch list are listed (p_begin = p_end = 0: all), as for a patch-parallel rank's range.
- * Returns 0 if every property holds, else the number of the first that fails (1: bad
- * arguments). */
+ * pages; no GPU needed).  The units of work are (head, image patch, query-tile pair), each
+ * a list of KV tiles, in head-major order.  When the K/V the list reads (every head, fresh
+ * and stale rows) exceed kv_budget_bytes (< 0: the kernel's own budget, 48 MB), the first
+ * whole_rounds * ctas units are dealt whole, unit k * ctas + c to CTA c, so the CTAs' units
+ * in flight share one or two heads' K/V in L2; the remaining units (the tail) are cut into
+ * `ctas` contiguous ranges of KV tiles (stream-K).  Walks every CTA's pieces as the kernel
+ * does and checks: every CTA has work and every piece stays inside its unit; every unit is
+ * covered once; a pair cut between CTAs has its first KV tiles at the end of one CTA's
+ * tail range (that CTA merges) and its other pieces each at the start of a range; the
+ * kernel's publisher and flag warps predict exactly those pieces.  L tokens per image in
+ * n_patches patches of Lp tokens; mode 0 sync, 1 displaced, 2 naive, 3 cross-attention
+ * (Lp = L, n_patches = 1, kv_len context tokens).  Only the query patches [p_begin, p_end)
+ * of the image-major patch list are listed (p_begin = p_end = 0: all), as for a
+ * patch-parallel rank's range.  Returns 0 if every property holds, else the number of the
+ * first that fails (1: bad arguments). */
 DFP_API int dfp_attention_schedule_check(int L, int Lp, int n_patches, int heads, int mode, int kv_len, int images,
-                                         int ctas, int p_begin, int p_end);
+                                         int ctas, int p_begin, int p_end, long long kv_budget_bytes);
 
 /* Launch overlap between the kernels of a step (no counterpart in the pages; on by
  * default): every tensor-core-family kernel is launched with programmatic stream

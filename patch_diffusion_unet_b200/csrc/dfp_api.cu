@@ -623,9 +623,10 @@ dfp_status dfp_check_device(dfp_handle h) {
 int dfp_launches_per_step(dfp_handle h) { return h ? h->launches : -1; }
 
 int dfp_attention_schedule_check(int L, int Lp, int n_patches, int heads, int mode, int kv_len, int images,
-                                 int ctas, int p_begin, int p_end) {
+                                 int ctas, int p_begin, int p_end, long long kv_budget_bytes) {
   if (mode < kAttnSync || mode > kAttnCross) return 1;
-  return attention_schedule_check(L, Lp, n_patches, heads, mode, kv_len, images, ctas, p_begin, p_end);
+  return attention_schedule_check(L, Lp, n_patches, heads, mode, kv_len, images, ctas, p_begin, p_end,
+                                  kv_budget_bytes);
 }
 
 dfp_status dfp_set_launch_overlap(dfp_handle h, int enable) {

@@ -164,15 +164,20 @@ struct TcAttnArgs {
                           // it continues a pair another CTA started
   float* part_ml;         // scratch [ctas][256][2]:  (running max, row sum) of the same
   unsigned* flags;        // scratch [ctas][2]: publish flags of the CTAs' first pieces (zeroed once)
-  int total_tiles;        // set by the launcher
+  // set by the launcher: the work split (whole-unit rounds, then a stream-K tail)
+  int whole_rounds;       // rounds of whole units dealt one per CTA
+  int total_tiles;        // tiles of the tail (the units after whole_rounds * ctas)
+  int tail_base;          // tiles of the units before the tail
+  int head_tiles;         // tiles of one head's units
   unsigned epoch;         // set by the launcher: this launch's flag value (never 0, never reused)
   int pdl;                // launch with programmatic stream serialization
 };
 // floats of part_o for `ctas` CTAs (part_ml needs 1/32 of it)
 size_t attention_scratch_floats(int ctas);
 // Host walk of the attention work split over `ctas` CTAs (0: every property holds)
+// kv_budget: K/V bytes above which whole-unit rounds are used (< 0: the launcher's own)
 int attention_schedule_check(int L, int Lp, int N, int heads, int mode, int kv_len, int images, int ctas,
-                             int p_lo = 0, int p_hi = 0);
+                             int p_lo = 0, int p_hi = 0, long long kv_budget = -1);
 int sm_count();
 // V operand of the attention: [heads][rows][64] bf16 (rows a multiple of 4, every KV tile
 // starting at a multiple of 4) seen as a 5-D view whose 128-row box lands in shared memory

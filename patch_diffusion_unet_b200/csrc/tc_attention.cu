@@ -40,15 +40,21 @@
 // degree-3 minimax polynomial for 2^f, max relative error 7.48e-5; exp2_poly.cuh)
 // to offload the MUFU unit.
 //
-// Work split (stream-K style): a unit of work is one KV tile for one Q-tile pair of
-// one (patch, head), the patches of all images of the batch in one list.  The units are laid out pair-major within (patch, head) and
-// the whole list is cut into one contiguous range per SM, so every CTA gets the
-// same number of KV tiles whatever the number of pairs.  A CTA walks its range as
-// a sequence of pieces (the part of one pair's KV list that falls in the range);
+// Work split: a unit of work is the KV list of one Q-tile pair of one (head, patch), the
+// patches of all images of the batch in one head-major list.  When the K and V the list
+// reads do not fit in L2 (the 240 x 240 map reads 295 MB of them), rounds of whole units
+// are dealt one per CTA, unit k * G + c to CTA c: the units in flight are then neighbours
+// in the list and share one or two heads' K and V in L2.  The rest (the tail; all of the
+// list for smaller maps) is stream-K: its KV tiles are cut into one contiguous range per
+// SM, so every CTA gets the same number of KV tiles whatever the number of pairs.  A CTA
+// walks its work as a sequence of pieces (a whole unit, or the part of one pair's KV list
+// that falls in its tail range): the first piece of its tail range, then its whole units,
+// then the rest of its tail range.
 // Q is double-buffered so the next piece's queries load while the current piece
 // runs, and the K/V ring does not drain between pieces.  A pair whose KV list is
 // cut between CTAs is finished by the CTA holding its first KV tiles (the end of that
-// CTA's range, so processed after the other pieces, which open their CTAs' ranges):
+// CTA's tail range, so processed last there, after the other pieces, which open their
+// CTAs' sequences):
 // the other pieces leave their unnormalised O, running max and row sum in a per-CTA
 // slot and publish a flag; the first piece merges them with its own O in KV order,
 // so the result does not depend on timing.  Only a merging piece ever waits, and only
@@ -120,46 +126,137 @@ __device__ __forceinline__ void tile_src(int mode, int p, int Lp, int L, int kv_
   valid = min(kTile, L - row);
 }
 
-// The unit list: patch-major over the images' patches (patch pg = img * N + p, so Q and O
-// rows start at pg * Lp), then head, then Q-tile pair; unit (pg, head, pair) has
+// The unit list: head-major over (head, query patch, Q-tile pair) -- patch pg = img * N + p
+// over the images' patches, so Q and O rows start at pg * Lp -- unit (head, pg, pair) has
 // unit_tiles(pg % N) KV tiles.  Only the query patches [p_lo, p_hi) are listed (all of them
-// unless a patch-parallel rank computes a range).  Global tile x -> its unit and the unit's
-// first tile.
-// All schedule arithmetic is 32-bit: the launcher checks total_tiles * ctas < 2^31.
+// unless a patch-parallel rank computes a range).
+// All schedule arithmetic is 32-bit: the launcher checks total tiles * ctas < 2^31.
 struct Unit {
-  int p, head, pair, T, U0;   // p: patch over the batch (img * N + patch within the image)
+  int p, head, pair, T;   // p: patch over the batch (img * N + patch within the image)
+  int U0;                 // tail units: tail index of the unit's first tile; whole units: -1
 };
-__host__ __device__ __forceinline__ Unit locate(const TcAttnArgs& a, int n_pairs, int x) {
-  int base = 0;
+__host__ __device__ __forceinline__ int patch_tiles(const TcAttnArgs& a, int p) {
+  return unit_tiles(a.mode, p % a.N, a.Lp, a.L, a.kv_len);
+}
+// unit `idx` of the list
+__host__ __device__ __forceinline__ Unit unit_at(const TcAttnArgs& a, int n_pairs, int idx) {
+  const int per_head = (a.p_hi - a.p_lo) * n_pairs;
   Unit u{};
+  u.head = idx / per_head;
+  const int r = idx - u.head * per_head;
+  u.p = a.p_lo + r / n_pairs;
+  u.pair = r - (r / n_pairs) * n_pairs;
+  u.T = patch_tiles(a, u.p);
+  u.U0 = -1;
+  return u;
+}
+// the unit holding tail tile x, its U0 the tail index of its first tile
+__host__ __device__ __forceinline__ Unit locate(const TcAttnArgs& a, int n_pairs, int x) {
+  const int X = x + a.tail_base;          // index among all tiles of the list
+  Unit u{};
+  u.head = X / a.head_tiles;
+  int base = u.head * a.head_tiles;
   for (int p = a.p_lo; p < a.p_hi; ++p) {
-    const int T = unit_tiles(a.mode, p % a.N, a.Lp, a.L, a.kv_len);
-    const int blk = T * a.heads * n_pairs;
-    if (x < base + blk) {
-      const int ui = (x - base) / T;
-      u.p = p; u.head = ui / n_pairs; u.pair = ui - u.head * n_pairs; u.T = T;
-      u.U0 = base + ui * T;
+    const int T = patch_tiles(a, p);
+    if (X < base + T * n_pairs) {
+      u.p = p; u.pair = (X - base) / T; u.T = T;
+      u.U0 = base + u.pair * T - a.tail_base;
       return u;
     }
-    base += blk;
+    base += T * n_pairs;
   }
   return u;   // not reached for x < total
 }
-// the unit after u in the list (no division: pairs, then heads, then patches)
+// the tail unit after u (no division: pairs, then patches, then heads)
 __host__ __device__ __forceinline__ void advance(const TcAttnArgs& a, int n_pairs, Unit& u) {
   u.U0 += u.T;
   if (++u.pair == n_pairs) {
     u.pair = 0;
-    if (++u.head == a.heads) {
-      u.head = 0;
-      ++u.p;
-      u.T = unit_tiles(a.mode, u.p % a.N, a.Lp, a.L, a.kv_len);
+    if (++u.p == a.p_hi) {
+      u.p = a.p_lo;
+      ++u.head;
     }
+    u.T = patch_tiles(a, u.p);
   }
 }
-// the CTA whose range [c*TT/G, (c+1)*TT/G) holds global tile x
+// the CTA whose tail range [c*TT/G, (c+1)*TT/G) holds tail tile x
 __host__ __device__ __forceinline__ int cta_of(int x, int TT, int G) { return ((x + 1) * G + TT - 1) / TT - 1; }
 __host__ __device__ __forceinline__ int range_start(int c, int TT, int G) { return c * TT / G; }
+
+// The pieces of CTA c, in order (phase 0, 1, 2): the first piece of its tail range [X0, X1)
+// (the tail: the units from whole_rounds * G on, their tiles numbered from 0), its
+// whole_rounds whole units (units k * G + c, one piece each, merged by nobody), then the
+// rest of its tail range, one piece per unit the range touches.  With every CTA on whole
+// units at once the units in flight are consecutive in the list and share one or two
+// heads' K and V in L2 whatever the map size; a piece that continues a pair another CTA
+// started opens the sequence, so its partial is published early, and a pair this CTA
+// merges ends it.
+struct Walk {
+  Unit tu;       // the tail unit last walked (the tail resumes after it)
+  int j0, n;     // the piece: its unit's KV tiles [j0, j0 + n)
+  int k;         // the piece's index in the CTA's sequence
+  int x;         // the tail tile after the last tail piece walked
+  int kw;        // whole units walked (phase 1: the current one)
+  int phase;
+};
+struct Sched {
+  int n_pairs, G, c, X0, X1;
+};
+// the unit of the current piece
+__host__ __device__ __forceinline__ Unit walk_unit(const TcAttnArgs& a, const Sched& s, const Walk& w) {
+  return w.phase == 1 ? unit_at(a, s.n_pairs, w.kw * s.G + s.c) : w.tu;
+}
+__host__ __device__ __forceinline__ void walk_whole(const TcAttnArgs& a, const Sched& s, Walk& w) {
+  w.j0 = 0;
+  w.n = unit_at(a, s.n_pairs, w.kw * s.G + s.c).T;
+}
+__host__ __device__ __forceinline__ bool walk_tail_next(const TcAttnArgs& a, const Sched& s, Walk& w) {
+  if (w.x >= s.X1) return false;
+  advance(a, s.n_pairs, w.tu);
+  w.j0 = 0;
+  w.n = min(w.tu.U0 + w.tu.T, s.X1) - w.x;
+  w.x += w.n;
+  return true;
+}
+__host__ __device__ __forceinline__ bool walk_first(const TcAttnArgs& a, const Sched& s, Walk& w) {
+  w.k = 0;
+  w.kw = 0;
+  w.x = s.X0;
+  if (s.X0 < s.X1) {
+    w.tu = locate(a, s.n_pairs, s.X0);
+    w.j0 = s.X0 - w.tu.U0;
+    w.n = min(w.tu.U0 + w.tu.T, s.X1) - s.X0;
+    w.x = s.X0 + w.n;
+    w.phase = 0;
+    return true;
+  }
+  if (a.whole_rounds > 0) {
+    w.phase = 1;
+    walk_whole(a, s, w);
+    return true;
+  }
+  return false;
+}
+__host__ __device__ __forceinline__ bool walk_next(const TcAttnArgs& a, const Sched& s, Walk& w) {
+  ++w.k;
+  if (w.phase == 0 && a.whole_rounds > 0) {
+    w.phase = 1;
+    walk_whole(a, s, w);
+    return true;
+  }
+  if (w.phase == 1 && ++w.kw < a.whole_rounds) {
+    walk_whole(a, s, w);
+    return true;
+  }
+  w.phase = 2;
+  return walk_tail_next(a, s, w);
+}
+// KV tiles of CTA c in all
+__host__ __device__ __forceinline__ int cta_tiles(const TcAttnArgs& a, const Sched& s) {
+  int t = s.X1 - s.X0;
+  for (int k = 0; k < a.whole_rounds; ++k) t += unit_at(a, s.n_pairs, k * s.G + s.c).T;
+  return t;
+}
 
 __device__ __forceinline__ float ex2_mufu(float x) {
   float y;
@@ -267,8 +364,9 @@ __device__ __noinline__ bool piece_epilogue(const TcAttnArgs& a, const Unit& u, 
   const bool row_ok = have && q_local < a.Lp;
   uint4* out_row = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) +
                                             (size_t)(u.p * a.Lp + q_local) * a.C + u.head * 64 + half * 32);
-  const int c_first = cta_of(u.U0, TT, G);
-  const int npieces = cta_of(u.U0 + u.T - 1, TT, G) - c_first + 1;
+  // whole units are one piece; a tail unit spans the CTAs holding its first and last tiles
+  const int c_first = u.U0 < 0 ? c : cta_of(u.U0, TT, G);
+  const int npieces = u.U0 < 0 ? 1 : cta_of(u.U0 + u.T - 1, TT, G) - c_first + 1;
   if (npieces == 1) {
     if (have) {
       const float inv = 1.f / l;
@@ -407,17 +505,19 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
   __shared__ volatile int s_abort;
   __shared__ float s_mrow[2][128];           // [group][row]: running max handed to the piece epilogue
-  __shared__ int s_piece[2][8];               // per group: p, head, pair, T, U0, piece start
+  __shared__ int s_ring[4][8];                // pieces pi (slot pi % 4): p, head, pair, T, U0, first tile, tiles
+  __shared__ __align__(8) uint64_t s_ready[4]; // slot filled (the TMA warp arrives once per piece)
   __shared__ __align__(8) uint64_t s_pub[2];   // [group]: the partial of the CTA's first piece is written
   __shared__ __align__(8) uint64_t s_mrg;      // the later pieces of the pair this CTA merges are published
   __shared__ volatile int s_merge_fail;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, c = blockIdx.x;
-  const int TT = a.total_tiles;
-  const int X0 = range_start(c, TT, G), X1 = range_start(c + 1, TT, G);
-  const int NT = X1 - X0;
+  const int TT = a.total_tiles;                // tiles of the stream-K tail
   const int n_pairs = (a.n_qtiles + 1) / 2;
+  const Sched sc{n_pairs, G, c, range_start(c, TT, G), range_start(c + 1, TT, G)};
+  const int X0 = sc.X0, X1 = sc.X1;
+  const int NT = cta_tiles(a, sc);             // every KV tile of this CTA, whole units included
   int* err = a.err;
 
   if (threadIdx.x == 0) {
@@ -435,6 +535,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
       mbar_init(smem_u32(&o_done[g]), 1);
     }
     mbar_init(smem_u32(mma_drain), 1);
+    for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&s_ready[i]), 1);
     mbar_init(smem_u32(&s_pub[0]), 256);
     mbar_init(smem_u32(&s_pub[1]), 256);
     mbar_init(smem_u32(&s_mrg), 1);
@@ -471,10 +572,11 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
     if (leader) tma_prefetch_desc(&mq);
     int gt = 0, pi = 0;   // tiles and pieces issued so far
     bool ok = true;
-    Unit u = locate(a, n_pairs, X0);
-    for (int x = X0; ok && x < X1; ++pi, advance(a, n_pairs, u)) {
-      const int jl0 = x - u.U0;
-      const int n = min(u.U0 + u.T, X1) - x;
+    Walk w;
+    for (bool have = walk_first(a, sc, w); ok && have; ++pi, have = walk_next(a, sc, w)) {
+      const Unit u = walk_unit(a, sc, w);
+      const int jl0 = w.j0;
+      const int n = w.n;
       // the piece's two query tiles into Q buffer pi & 1
       const int qb = pi & 1;
       if (pi >= 2 && !mbar_wait_warp(smem_u32(&q_empty[qb]), ((pi >> 1) - 1) & 1, err, kErrWaitStageFree)) {
@@ -482,6 +584,11 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
         break;
       }
       if (leader) {
+        // the piece for the softmax groups (slot pi % 4 is free: the groups have started
+        // piece pi - 3, which needs this warp's piece pi - 2 queries loaded and consumed)
+        volatile int* r = s_ring[pi & 3];
+        r[0] = u.p; r[1] = u.head; r[2] = u.pair; r[3] = u.T; r[4] = u.U0; r[5] = jl0; r[6] = n;
+        mbar_arrive(smem_u32(&s_ready[pi & 3]));
         const int qrow = u.p * a.Lp + 2 * u.pair * kTile;
         const uint32_t qbar = smem_u32(&q_full[qb]);
         mbar_arrive_expect_tx(qbar, 2 * kTileBytes);
@@ -514,7 +621,6 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
         }
         __syncwarp();
       }
-      x += n;
     }
     if (!ok) {
       if (leader) s_abort = 1;
@@ -565,18 +671,19 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
       __syncwarp();                                                                              \
     } while (0)
     // piece walk: for each tile, is it the first / last of its piece, and which piece
-    int px = X0;
+    // (called once per tile of the CTA, so a piece always follows).  The pieces' lengths come
+    // from the TMA warp's descriptor ring (this warp is at most one piece ahead of the
+    // softmax groups, the TMA warp at most two ahead of this one, so the slot is current).
     int left = 0, pc = -1;
-    Unit mu = locate(a, n_pairs, X0);
+    bool walk_ok = true;
     auto next_tile = [&](bool& first, bool& last, int& piece) {
       first = left == 0;
       if (first) {
-        if (pc >= 0) advance(a, n_pairs, mu);
-        left = min(mu.U0 + mu.T, X1) - px;
         ++pc;
+        walk_ok = walk_ok && mbar_wait_warp(smem_u32(&s_ready[pc & 3]), (uint32_t)(pc >> 2) & 1u, err, kErrWaitTmaFull);
+        left = walk_ok ? s_ring[pc & 3][6] : 1;
       }
       --left;
-      ++px;
       last = left == 0;
       piece = pc;
     };
@@ -584,7 +691,8 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
     bool cur_first, cur_last;
     int cur_piece;
     next_tile(cur_first, cur_last, cur_piece);
-    {
+    ok = walk_ok;
+    if (ok) {
       const int qb = cur_piece & 1;
       ok = mbar_wait_warp(smem_u32(&q_full[qb]), (cur_piece >> 1) & 1, err, kErrWaitTmaFull) &&
            mbar_wait_warp(smem_u32(&k_full[0]), 0, err, kErrWaitTmaFull);
@@ -610,6 +718,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
       bool nx_first = false, nx_last = false;
       int nx_piece = cur_piece;
       if (more) next_tile(nx_first, nx_last, nx_piece);
+      if (!walk_ok) { ok = false; break; }
       const int nqb = nx_piece & 1;
       const uint64_t nqd = qd0 + (uint64_t)(2 * nqb) * kTileDesc;
       if (!mbar_wait_warp(smem_u32(&v_full[st]), par, err, kErrWaitTmaFull)) { ok = false; break; }
@@ -650,23 +759,25 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
     mbar_wait(smem_u32(mma_drain), 0, err, kErrWaitAccum);
    } else if (warp == kWarpMma + 1) {
     // ------------------------------------------------------------ publisher
-    // The CTA's first piece continues a pair an earlier CTA started: once a group has
+    // The CTA's first tail piece continues a pair an earlier CTA started: once a group has
     // written its partial (its 256 threads arrived on s_pub[g], release at CTA scope),
     // release the group's flag at GPU scope for the merging CTA.
     const Unit u0 = locate(a, n_pairs, X0);
-    const int cf = cta_of(u0.U0, TT, G), np = cta_of(u0.U0 + u0.T - 1, TT, G) - cf + 1;
-    if (NT > 0 && np > 1 && c != cf && leader) {
+    const int cf = X1 > X0 ? cta_of(u0.U0, TT, G) : c;
+    const int np = X1 > X0 ? cta_of(u0.U0 + u0.T - 1, TT, G) - cf + 1 : 1;
+    if (np > 1 && c != cf && leader) {
       for (int g = 0; g < 2; ++g)
         if (mbar_wait(smem_u32(&s_pub[g]), 0, err, kErrWaitAttnMerge)) st_release_gpu(a.flags + 2 * c + g, a.epoch);
     }
     __syncwarp();
    } else if (warp == kWarpMma + 2) {
     // ------------------------------------------------------------ merge flags
-    // The CTA's last piece holds the first KV tiles of a cut pair: acquire the later
+    // The CTA's last tail piece holds the first KV tiles of a cut pair: acquire the later
     // pieces' flags of both groups while the CTA works, then let the groups merge.
     const Unit ul = locate(a, n_pairs, X1 - 1);
-    const int cf = cta_of(ul.U0, TT, G), np = cta_of(ul.U0 + ul.T - 1, TT, G) - cf + 1;
-    if (NT > 0 && np > 1 && c == cf && leader) {
+    const int cf = X1 > X0 ? cta_of(ul.U0, TT, G) : c;
+    const int np = X1 > X0 ? cta_of(ul.U0 + ul.T - 1, TT, G) - cf + 1 : 1;
+    if (np > 1 && c == cf && leader) {
       int failed = 0;
       for (int k = 1; k < np && !failed; ++k)
         for (int g = 0; g < 2 && !failed; ++g) {
@@ -702,29 +813,21 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
     // piece epilogue (32x32b shape): lane = row of the quadrant, h16 picks 32 output columns
     const int erow = 32 * q4 + lane;
     const uint32_t tOe = tmem + 256 + 128 * g + ((uint32_t)(32 * q4) << 16);
-    const bool group_leader = (warp & 7) == 0 && lane == 0;
     const float sl2 = 0.125f * 1.4426950408889634f;   // (1/sqrt(64)) * log2(e)
     bool ok = true;
     // A failed wait makes the whole warp give up the piece (waits are agreed warp-wide,
     // so the TMEM instructions stay warp-uniform); the group then leaves together at the
     // piece barrier (bar.red.or), which every thread reaches once per piece.
     bool carry = false;
-    // The group's current unit lives in shared memory (the group leader advances it
-    // between pieces): registers across the KV loop are all taken by the scores.
-    volatile int* sp = s_piece[g];
-    if (group_leader) {
-      const Unit u0 = locate(a, n_pairs, X0);
-      sp[0] = u0.p; sp[1] = u0.head; sp[2] = u0.pair; sp[3] = u0.T; sp[4] = u0.U0; sp[5] = X0;
-    }
-    named_bar(2 + g, 256);
-    int gt = 0;
-    while (ok) {
-      int n;
-      {
-        const int x = sp[5];
-        if (x >= X1) break;
-        n = min(sp[4] + sp[3], X1) - x;
+    // The pieces come from the TMA warp (a ring of four descriptors in shared memory, each
+    // published with a release arrival): the groups do no walking of their own.
+    int gt = 0, pi = 0;
+    while (ok && gt < NT) {
+      if (!mbar_wait_warp(smem_u32(&s_ready[pi & 3]), (uint32_t)(pi >> 2) & 1u, err, kErrWaitTmaFull)) {
+        carry = true;
       }
+      volatile int* sp = s_ring[pi & 3];
+      const int n = carry ? 0 : sp[6];
       float m_used = -INFINITY;
       for (int jj = 0; jj < n && !carry; ++jj, ++gt) {
         // every tile is full when all segment lengths are multiples of the tile (parameters
@@ -732,7 +835,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
         int valid = kTile;
         if (!((a.mode == kAttnCross ? a.kv_len : (a.Lp | a.L)) % kTile == 0)) {
           int stale, krow;
-          tile_src(a.mode, sp[0] % a.N, a.Lp, a.L, a.kv_len, sp[5] - sp[4] + jj, stale, krow, valid);
+          tile_src(a.mode, sp[0] % a.N, a.Lp, a.L, a.kv_len, sp[5] + jj, stale, krow, valid);
         }
         if (!mbar_wait_warp(smem_u32(&s_full[g]), gt & 1, err, kErrWaitAttnS)) { carry = true; break; }
         tc_fence_after();
@@ -836,14 +939,9 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
       if (!piece_epilogue(a, u, tOe, smem_u32(&o_done[g]), (uint32_t)(gt - 1) & 1u, s_mrow[g][erow], g, h16,
                           erow, c, smem_u32(&s_pub[g]), smem_u32(&s_mrg), &s_merge_fail))
         carry = true;
-      // next piece: every thread of the group is done with s_piece (and s_mrow) before it changes
+      // next piece: every thread of the group is done with s_mrow before it changes
       named_bar(2 + g, 256);
-      if (group_leader) {
-        const int x_next = min(u.U0 + u.T, X1);
-        advance(a, n_pairs, u);
-        sp[0] = u.p; sp[1] = u.head; sp[2] = u.pair; sp[3] = u.T; sp[4] = u.U0; sp[5] = x_next;
-      }
-      named_bar(2 + g, 256);
+      ++pi;
     }
     if (!ok || carry) s_abort = 1;
   }
@@ -871,11 +969,39 @@ bool encode_attn_v(CUtensorMap* m, const void* base, uint64_t rows, uint64_t hea
   return encode_tmap_5d(m, base, dims, strides, box);
 }
 
-long long attention_total_tiles(const TcAttnArgs& a) {
+// K/V bytes above which the whole-unit rounds are used: the list's K and V (every head,
+// fresh and stale rows) no longer fit next to the Q and O streams in the 126 MB L2.
+constexpr long long kL2KvBudget = 48ll << 20;
+
+// The work split of `a` over at most `ctas` CTAs: fills whole_rounds, total_tiles (the tail),
+// tail_base and head_tiles and returns the CTA count (0: no work; -1: too large for the
+// kernel's 32-bit schedule arithmetic).
+int plan_schedule(TcAttnArgs& a, int ctas, long long kv_budget = kL2KvBudget) {
   const int n_pairs = (a.n_qtiles + 1) / 2;
-  long long tt = 0;
-  for (int p = a.p_lo; p < a.p_hi; ++p) tt += (long long)unit_tiles(a.mode, p % a.N, a.Lp, a.L, a.kv_len) * a.heads * n_pairs;
-  return tt;
+  const int np = a.p_hi - a.p_lo;
+  long long per_head = 0;
+  for (int p = a.p_lo; p < a.p_hi; ++p) per_head += (long long)patch_tiles(a, p) * n_pairs;
+  const long long all = per_head * a.heads;
+  if (all <= 0 || np <= 0 || n_pairs <= 0) return 0;
+  const int G = (int)std::min<long long>(ctas, all);
+  if (G <= 0 || all * G >= (1ll << 31)) return -1;
+  const long long units = (long long)a.heads * np * n_pairs;
+  const long long kv_rows =
+      (long long)(a.mode == kAttnCross ? a.kv_len : a.mode == kAttnDisplaced ? 2 * a.L : a.L) * a.images;
+  const long long kv_bytes = kv_rows * a.heads * 64 * 2 * 2;
+  const int F = kv_bytes > kv_budget ? (int)(units / G) : 0;
+  // tiles of the units before the tail (the first F * G of the head-major list)
+  const long long fg = (long long)F * G, per_head_units = (long long)np * n_pairs;
+  const long long h = fg / per_head_units, r = fg - h * per_head_units;
+  long long base = h * per_head;
+  const int lp = (int)(r / n_pairs), pair = (int)(r - (long long)lp * n_pairs);
+  for (int q = 0; q < lp; ++q) base += (long long)patch_tiles(a, a.p_lo + q) * n_pairs;
+  if (lp < np) base += (long long)pair * patch_tiles(a, a.p_lo + lp);
+  a.whole_rounds = F;
+  a.head_tiles = (int)per_head;
+  a.tail_base = (int)base;
+  a.total_tiles = (int)(all - base);
+  return G;
 }
 
 size_t attention_scratch_floats(int ctas) { return (size_t)ctas * 256 * 64; }
@@ -903,11 +1029,9 @@ cudaError_t launch_tc_attention(const TcAttnArgs& args, const CUtensorMap& mq, c
   // a fresh flag value per launch (flags hold the epoch of the launch that last set them)
   static std::atomic<unsigned> epoch{0};
   do a.epoch = ++epoch; while (a.epoch == 0);
-  const long long tt = attention_total_tiles(a);
-  if (tt <= 0) return cudaSuccess;
-  const int G = (int)std::min<long long>(a.ctas, tt);
-  if (G <= 0 || tt * G >= (1ll << 31)) return cudaErrorInvalidValue;   // 32-bit schedule arithmetic
-  a.total_tiles = (int)tt;
+  const int G = plan_schedule(a, a.ctas);
+  if (G == 0) return cudaSuccess;
+  if (G < 0) return cudaErrorInvalidValue;   // 32-bit schedule arithmetic
   cudaLaunchConfig_t cfg{};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -921,59 +1045,77 @@ cudaError_t launch_tc_attention(const TcAttnArgs& args, const CUtensorMap& mq, c
   return cudaLaunchKernelEx(&cfg, tc_attention_kernel, mq, mkf, mvf, mks, mvs, a);
 }
 
-// Host walk of the work split exactly as the kernel's three walkers do it (the same
-// locate / advance / cta_of / range_start), checking what the cut-pair merge relies on.
+// Host walk of the work split exactly as the kernel's walkers do it (the same plan,
+// walk_first / walk_next, locate, cta_of, range_start), checking what the cut-pair merge
+// relies on.
 int attention_schedule_check(int L, int Lp, int N, int heads, int mode, int kv_len, int images, int ctas,
-                             int p_lo, int p_hi) {
+                             int p_lo, int p_hi, long long kv_budget) {
   TcAttnArgs a{};
   a.L = L; a.Lp = Lp; a.N = N; a.heads = heads; a.mode = mode; a.kv_len = kv_len; a.images = images;
   a.p_lo = p_lo; a.p_hi = p_hi > 0 ? p_hi : N * images;
   a.n_qtiles = cdiv(Lp, kTile);
   if (L <= 0 || Lp <= 0 || N <= 0 || heads <= 0 || images < 1 || ctas < 1) return 1;
   if (a.p_lo < 0 || a.p_hi > N * images || a.p_lo >= a.p_hi) return 1;
-  const int n_pairs = (a.n_qtiles + 1) / 2;
-  const long long tt = attention_total_tiles(a);
-  if (tt <= 0) return 1;
-  const int G = (int)std::min<long long>(ctas, tt);
-  if (tt * G >= (1ll << 31)) return 2;
-  const int TT = (int)tt;
-  std::vector<int> cover(TT, 0);   // tiles of the unit starting at index U0, summed over pieces
+  const int G = plan_schedule(a, ctas, kv_budget < 0 ? kL2KvBudget : kv_budget);
+  if (G == 0) return 1;
+  if (G < 0) return 2;
+  const int n_pairs = (a.n_qtiles + 1) / 2, np = a.p_hi - a.p_lo;
+  const int TT = a.total_tiles;
+  auto index_of = [&](const Unit& u) { return ((size_t)u.head * np + (u.p - a.p_lo)) * n_pairs + u.pair; };
+  std::vector<long long> cover((size_t)heads * np * n_pairs, 0);   // tiles of each unit, summed over pieces
   for (int c = 0; c < G; ++c) {
-    const int X0 = range_start(c, TT, G), X1 = range_start(c + 1, TT, G);
-    if (X1 <= X0) return 3;                         // every CTA has work
-    // what the publisher and flag warps conclude from the range's ends
-    const Unit u0 = locate(a, n_pairs, X0), ul = locate(a, n_pairs, X1 - 1);
-    const int cf0 = cta_of(u0.U0, TT, G), np0 = cta_of(u0.U0 + u0.T - 1, TT, G) - cf0 + 1;
-    const int cfl = cta_of(ul.U0, TT, G), npl = cta_of(ul.U0 + ul.T - 1, TT, G) - cfl + 1;
-    const int expect_publish = np0 > 1 && c != cf0, expect_merge = npl > 1 && c == cfl;
-    int publishes = 0, merges = 0;
-    Unit u = u0;
-    for (int x = X0; x < X1;) {
-      if (!(u.U0 <= x && x < u.U0 + u.T)) return 4;   // the walk stays inside its unit
-      const int x_end = std::min(u.U0 + u.T, X1);
-      cover[u.U0] += x_end - x;
-      const int cf = cta_of(u.U0, TT, G), np = cta_of(u.U0 + u.T - 1, TT, G) - cf + 1;
-      if (c < cf || c >= cf + np) return 5;           // this CTA holds part of the unit
-      if (np > 1) {
-        if (c == cf) {                                 // the first KV tiles end the range
+    const Sched sc{n_pairs, G, c, range_start(c, TT, G), range_start(c + 1, TT, G)};
+    const int X0 = sc.X0, X1 = sc.X1;
+    if (cta_tiles(a, sc) <= 0) return 3;            // every CTA has work
+    // what the publisher and flag warps conclude from the tail range's ends
+    int expect_publish = 0, expect_merge = 0;
+    if (X1 > X0) {
+      const Unit u0 = locate(a, n_pairs, X0), ul = locate(a, n_pairs, X1 - 1);
+      const int cf0 = cta_of(u0.U0, TT, G), np0 = cta_of(u0.U0 + u0.T - 1, TT, G) - cf0 + 1;
+      const int cfl = cta_of(ul.U0, TT, G), npl = cta_of(ul.U0 + ul.T - 1, TT, G) - cfl + 1;
+      expect_publish = np0 > 1 && c != cf0;
+      expect_merge = npl > 1 && c == cfl;
+    }
+    int publishes = 0, merges = 0, whole = 0, pieces = 0, merge_k = -1;
+    Walk w;
+    for (bool have = walk_first(a, sc, w); have; have = walk_next(a, sc, w), ++pieces) {
+      if (w.k != pieces) return 4;
+      const Unit wu = walk_unit(a, sc, w);
+      if (w.n <= 0 || w.j0 < 0 || w.j0 + w.n > wu.T) return 4;   // the piece stays inside its unit
+      cover[index_of(wu)] += w.n;
+      if (wu.U0 < 0) {                              // a whole unit
+        if (w.j0 != 0 || w.n != wu.T) return 4;
+        ++whole;
+        continue;
+      }
+      const int x = wu.U0 + w.j0, x_end = x + w.n;
+      if (x < X0 || x_end > X1) return 4;
+      const int cf = cta_of(wu.U0, TT, G), npc = cta_of(wu.U0 + wu.T - 1, TT, G) - cf + 1;
+      if (c < cf || c >= cf + npc) return 5;        // this CTA holds part of the unit
+      if (npc > 1) {
+        if (c == cf) {                               // the first KV tiles end the range
           if (x_end != X1) return 6;
+          merge_k = w.k;
           ++merges;
-        } else {                                       // a later piece opens the range
-          if (x != X0) return 7;
+        } else {                                     // a later piece opens the range, and the sequence
+          if (x != X0 || w.k != 0) return 7;
           ++publishes;
         }
       }
-      x = x_end;
-      if (x < X1) advance(a, n_pairs, u);
     }
+    if (whole != a.whole_rounds) return 11;
     if (publishes != expect_publish || merges != expect_merge) return 8;
+    // the merging piece is the CTA's last, or its only tail piece (then it opens the sequence)
+    if (merges && merge_k != pieces - 1 && !(merge_k == 0 && pieces - whole == 1)) return 12;
   }
   // every unit covered exactly once, whole
-  Unit v = locate(a, n_pairs, 0);
-  for (int x = 0; x < TT; x += v.T, advance(a, n_pairs, v)) {
-    if (v.U0 != x || v.T <= 0) return 9;
-    if (cover[x] != v.T) return 10;
-  }
+  for (int h = 0; h < heads; ++h)
+    for (int p = a.p_lo; p < a.p_hi; ++p)
+      for (int q = 0; q < n_pairs; ++q) {
+        Unit u{};
+        u.head = h; u.p = p; u.pair = q;
+        if (cover[index_of(u)] != patch_tiles(a, p)) return 10;
+      }
   return 0;
 }
 

@@ -53,10 +53,9 @@ __device__ __forceinline__ TileInfo tile_of(const TcGemmPlan& pl, int m_tile) {
   return t;
 }
 
-// Epilogue of one tile: drain the 128 x BN accumulator at TMEM column `acc` and store.
-template <int BN>
-__device__ __forceinline__ void epilogue_tile(const TcGemmPlan& plan, const Epilogue& epi, const TileInfo& tile,
-                                              int n0, uint32_t taddr, int row, bool valid_tile) {
+// Output row of this thread's accumulator lane (row) in tile `tile`, or -1 for none.
+__device__ __forceinline__ long long out_row(const TcGemmPlan& plan, const Epilogue& epi, const TileInfo& tile,
+                                             int row, bool valid_tile) {
   long long gm = -1;
   if (plan.conv) {
     const int rr = row / plan.cols_tile, jj = row - rr * plan.cols_tile;
@@ -72,6 +71,26 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmPlan& plan, const Epil
     const long long prow = gm / plan.W, col = gm - prow * plan.W;
     gm = ((prow | col) & 1) ? -1 : (prow >> 1) * (plan.W >> 1) + (col >> 1);
   }
+  return gm;
+}
+
+// The residual of this thread's output row, read before the accumulator is ready (the
+// loads overlap the tile's MMAs instead of stalling the epilogue chunk by chunk).
+template <int BN>
+__device__ __forceinline__ void prefetch_residual(const Epilogue& epi, long long gm, int n0, int N,
+                                                  uint4 (&res)[BN / 8]) {
+  if (epi.kind != 0 || !epi.residual || gm < 0) return;
+  const uint4* r4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(epi.residual) + gm * epi.ldo + n0);
+#pragma unroll
+  for (int i = 0; i < BN / 8; ++i)
+    if (n0 + 8 * i < N) res[i] = __ldg(r4 + i);
+}
+
+// Epilogue of one tile: drain the 128 x BN accumulator at TMEM address taddr (this warp's
+// lanes) and store row gm (-1: nothing to store; the TMEM reads still run warp-wide).
+template <int BN>
+__device__ __forceinline__ void epilogue_tile(const TcGemmPlan& plan, const Epilogue& epi, long long gm, int n0,
+                                              uint32_t taddr, const uint4 (&res)[BN / 8]) {
   if (BN == 128 && epi.kind == 2) {
     // GEGLU: columns [0, 64) are values, [64, 128) the gates of the same features
 #pragma unroll 1
@@ -100,7 +119,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmPlan& plan, const Epil
     }
     return;
   }
-#pragma unroll 1
+#pragma unroll
   for (int c = 0; c < BN / 32; ++c) {
     uint32_t r[32];
     tmem_ld32(taddr + c * 32, r);
@@ -117,11 +136,10 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmPlan& plan, const Epil
         for (int i = 0; i < 32; ++i) v[i] += __ldg(epi.bias + n + i);
       }
       if (epi.residual) {
-        const uint4* r4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(epi.residual) + gm * epi.ldo + n);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           float rr[8];
-          unpack16(r4[i], rr);
+          unpack16(res[c * 4 + i], rr);
 #pragma unroll
           for (int e = 0; e < 8; ++e) v[i * 8 + e] += rr[e];
         }
@@ -292,12 +310,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     int ti = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++ti) {
       const int buf = ti & 1, use = ti >> 1;
-      const bool ready = mbar_wait(smem_u32(&acc_full[buf]), use & 1, err, kErrWaitAccum);
-      tc_fence_after();
       const TileInfo tile = tile_of(plan, t / n_tiles_n);
       const int n0 = (t % n_tiles_n) * BN;
-      epilogue_tile<BN>(plan, epi, tile, n0, tmem_d + buf * kCols + ((uint32_t)(sub * 32) << 16), row,
-                        ready && !s_abort);
+      const long long gm = out_row(plan, epi, tile, row, true);
+      uint4 res[BN / 8];
+      prefetch_residual<BN>(epi, gm, n0, plan.N, res);
+      const bool ready = mbar_wait(smem_u32(&acc_full[buf]), use & 1, err, kErrWaitAccum);
+      tc_fence_after();
+      epilogue_tile<BN>(plan, epi, ready && !s_abort ? gm : -1, n0,
+                        tmem_d + buf * kCols + ((uint32_t)(sub * 32) << 16), res);
       tc_fence_before();
       mbar_arrive(smem_u32(&acc_empty[buf]));
       if (!ready) break;
@@ -473,13 +494,16 @@ tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_const
     int ti = 0;
     for (int t = pair; t < n_tiles; t += n_pairs, ++ti) {
       const int buf = ti & 1, use = ti >> 1;
-      const bool ready = mbar_wait_cluster(smem_u32(&acc_full[buf]), use & 1, err, kErrWaitAccum);
-      tc_fence_after();
       const int m_tile = 2 * (t / n_tiles_n) + (int)rank;
       const TileInfo tile = tile_of(plan, m_tile);
       const int n0 = (t % n_tiles_n) * BN;
-      epilogue_tile<BN>(plan, epi, tile, n0, tmem_d + buf * kCols + ((uint32_t)(sub * 32) << 16), row,
-                        ready && !s_abort && m_tile < plan.m_tiles);
+      const long long gm = out_row(plan, epi, tile, row, m_tile < plan.m_tiles);
+      uint4 res[BN / 8];
+      prefetch_residual<BN>(epi, gm, n0, plan.N, res);
+      const bool ready = mbar_wait_cluster(smem_u32(&acc_full[buf]), use & 1, err, kErrWaitAccum);
+      tc_fence_after();
+      epilogue_tile<BN>(plan, epi, ready && !s_abort ? gm : -1, n0,
+                        tmem_d + buf * kCols + ((uint32_t)(sub * 32) << 16), res);
       tc_fence_before();
       // the four epilogue warps of this CTA are done with the accumulator; they also agree
       // on giving up (a failed wait anywhere ends the loop for all of them)

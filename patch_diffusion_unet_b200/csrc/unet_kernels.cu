@@ -91,6 +91,16 @@ __device__ __forceinline__ float warp_sum(float v) {
 // y[r] = act(W[r] . x + b[r] (+ add[r])), one warp per output row; fp32 weights [rows][cols].
 // x_tau >= 0: x is the sinusoidal embedding of the timestep, [cos(tau f_k), sin(tau f_k)],
 // f_k = 10000^(-k / (cols/2)), computed here instead of read.
+__device__ __forceinline__ float gemv_x(const float* x, float x_tau, int c, int half) {
+  if (x_tau < 0.f) return x[c];
+  const int k = c < half ? c : c - half;
+  const float f = expf(-9.210340371976184f * (float)k / (float)half);   // ln(10000) = 9.2103...
+  return c < half ? cosf(x_tau * f) : sinf(x_tau * f);
+}
+
+// VEC4: cols % 4 == 0 and 16-byte aligned rows: each lane reads 16-byte vectors of the row,
+// four of them in flight (a row of 1280 weights is ten vectors a lane).
+template <bool VEC4>
 __global__ void gemv_kernel(const float* __restrict__ Wt, const float* __restrict__ b,
                             const float* __restrict__ add, const float* __restrict__ x, float x_tau,
                             float* __restrict__ y, int rows, int cols, int silu_out) {
@@ -101,16 +111,20 @@ __global__ void gemv_kernel(const float* __restrict__ Wt, const float* __restric
   const float* w = Wt + (size_t)r * cols;
   const int half = cols / 2;
   float s = 0.f;
-  for (int c = lane; c < cols; c += 32) {
-    float xv;
-    if (x_tau >= 0.f) {
-      const int k = c < half ? c : c - half;
-      const float f = expf(-9.210340371976184f * (float)k / (float)half);   // ln(10000) = 9.2103...
-      xv = c < half ? cosf(x_tau * f) : sinf(x_tau * f);
-    } else {
-      xv = x[c];
+  if (VEC4) {
+    const float4* w4 = reinterpret_cast<const float4*>(w);
+    const int n4 = cols / 4;
+#pragma unroll 4
+    for (int c4 = lane; c4 < n4; c4 += 32) {
+      const float4 wv = __ldg(w4 + c4);
+      const int c = 4 * c4;
+      s = fmaf(wv.x, gemv_x(x, x_tau, c, half), s);
+      s = fmaf(wv.y, gemv_x(x, x_tau, c + 1, half), s);
+      s = fmaf(wv.z, gemv_x(x, x_tau, c + 2, half), s);
+      s = fmaf(wv.w, gemv_x(x, x_tau, c + 3, half), s);
     }
-    s = fmaf(__ldg(w + c), xv, s);
+  } else {
+    for (int c = lane; c < cols; c += 32) s = fmaf(__ldg(w + c), gemv_x(x, x_tau, c, half), s);
   }
   s = warp_sum(s);
   if (lane == 0) {
@@ -175,8 +189,9 @@ cudaError_t launch_concat(const void* a, int Ca, const void* b, int Cb, void* ou
 
 cudaError_t launch_gemv(const float* W, const float* b, const float* add, const float* x, float x_tau, float* y,
                         int rows, int cols, bool silu_out, bool pdl, cudaStream_t s) {
-  return launch_pdl(gemv_kernel, (rows * 32 + 255) / 256, 256, pdl, s, W, b, add, x, x_tau, y, rows, cols,
-                    silu_out ? 1 : 0);
+  const bool vec4 = cols % 4 == 0 && reinterpret_cast<uintptr_t>(W) % 16 == 0;
+  return launch_pdl(vec4 ? gemv_kernel<true> : gemv_kernel<false>, (rows * 32 + 255) / 256, 256, pdl, s, W, b, add,
+                    x, x_tau, y, rows, cols, silu_out ? 1 : 0);
 }
 
 cudaError_t launch_ddim_update(float* lat, const void* eps, void* x_bf, long long n, float c1, float c2, bool pdl,

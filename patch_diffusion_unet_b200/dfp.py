@@ -64,7 +64,7 @@ def load_library(path=_LIB_PATH):
         "dfp_launches_per_step": ([H], ctypes.c_int),
         "dfp_set_kernel_family": ([H, ctypes.c_int], ctypes.c_int),
         "dfp_set_launch_overlap": ([H, ctypes.c_int], ctypes.c_int),
-        "dfp_attention_schedule_check": ([ctypes.c_int] * 10, ctypes.c_int),
+        "dfp_attention_schedule_check": ([ctypes.c_int] * 10 + [ctypes.c_longlong], ctypes.c_int),
         "dfp_step_patches": ([H, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int], ctypes.c_int),
         "dfp_set_timestep": ([H, ctypes.c_float], ctypes.c_int),
         "dfp_ddim_sample": ([H, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,

@@ -13,9 +13,9 @@ SYNC, DISPLACED, NAIVE, CROSS = 0, 1, 2, 3
 CTAS = [148, 147, 132, 100, 64, 37, 7, 2, 1]
 
 
-def _check(L, Lp, N, heads, mode, kv_len=0, images=1, ctas=148, p_lo=0, p_hi=0):
+def _check(L, Lp, N, heads, mode, kv_len=0, images=1, ctas=148, p_lo=0, p_hi=0, budget=-1):
     from patch_diffusion_unet_b200 import dfp
-    return dfp.LIB.dfp_attention_schedule_check(L, Lp, N, heads, mode, kv_len, images, ctas, p_lo, p_hi)
+    return dfp.LIB.dfp_attention_schedule_check(L, Lp, N, heads, mode, kv_len, images, ctas, p_lo, p_hi, budget)
 
 
 # (L, Lp, N, heads) of the workloads: 64x64 / 128x128 / 240x240 maps, the stage's 20 heads,
@@ -26,13 +26,16 @@ SHAPES = [
 ]
 
 
+@pytest.mark.parametrize("budget", [-1, 0], ids=["own-budget", "whole-rounds"])
 @pytest.mark.parametrize("shape", SHAPES, ids=[f"L{s[0]}-N{s[2]}" for s in SHAPES])
 @pytest.mark.parametrize("mode", [SYNC, DISPLACED, NAIVE], ids=["sync", "displaced", "naive"])
-def test_self_attention_split(shape, mode):
+def test_self_attention_split(shape, mode, budget):
+    """budget 0 deals whole units whenever there are at least as many units as CTAs (the
+    large-map split); -1 takes the kernel's own choice (whole rounds at the 240 x 240 map)."""
     L, Lp, N, heads = shape
     for images in (1, 2):
         for ctas in CTAS:
-            assert _check(L, Lp, N, heads, mode, images=images, ctas=ctas) == 0, (images, ctas)
+            assert _check(L, Lp, N, heads, mode, images=images, ctas=ctas, budget=budget) == 0, (images, ctas)
 
 
 @pytest.mark.parametrize("images", [1, 2, 3])
@@ -50,7 +53,9 @@ def test_random_splits():
         mode = int(rng.integers(0, 3))
         images = int(rng.integers(1, 4))
         ctas = int(rng.integers(1, 200))
-        assert _check(N * Lp, Lp, N, heads, mode, images=images, ctas=ctas) == 0, (N, Lp, heads, mode, images, ctas)
+        for budget in (-1, 0):
+            assert _check(N * Lp, Lp, N, heads, mode, images=images, ctas=ctas, budget=budget) == 0, \
+                (N, Lp, heads, mode, images, ctas, budget)
 
 
 @pytest.mark.parametrize("shape", SHAPES[:3], ids=["L4096", "L16384", "L57600"])
@@ -64,7 +69,9 @@ def test_patch_range_split(shape, world):
     per = N // world
     for r in range(world):
         for ctas in CTAS:
-            assert _check(L, Lp, N, heads, DISPLACED, ctas=ctas, p_lo=r * per, p_hi=(r + 1) * per) == 0, (r, ctas)
+            for budget in (-1, 0):
+                assert _check(L, Lp, N, heads, DISPLACED, ctas=ctas, p_lo=r * per, p_hi=(r + 1) * per,
+                              budget=budget) == 0, (r, ctas, budget)
 
 
 def test_bad_arguments():
