@@ -161,8 +161,8 @@ def _work_model_one_image(cfg):
 # (profiles/), keyed by workload and kernel, with a hash of the kernel's sources at
 # capture time: once the kernel changes the figure no longer applies and is reported null.
 NCU_TRAFFIC = {
-    ("sdxl1024-64x64x640-n4-bf16", "attention (tcgen05)"):
-        (27.19e6, ("tc_attention.cu", "dfp_common.cuh"), "1c605708c6212bac"),
+    ("sdxl3840-240x240x640-n8-bf16", "attention (tcgen05)"):
+        (521.33e6, ("tc_attention.cu", "dfp_common.cuh", "exp2_poly.cuh"), "73f6d37f6d5fab18"),
 }
 
 

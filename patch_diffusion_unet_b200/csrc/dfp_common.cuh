@@ -304,6 +304,33 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- untiled bulk copies
+// (no multicast; addresses and sizes multiples of 16 bytes)
+// global -> this CTA's shared memory, completing `bytes` on the mbarrier, with an L2 policy
+__device__ __forceinline__ void bulk_load_policy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+      ::"r"(dst), "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+// shared -> global, in the issuing thread's current bulk group
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// every bulk group of this thread has finished reading its shared-memory source
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// every bulk group of this thread but the latest has finished reading its source
+__device__ __forceinline__ void bulk_wait_read_prev() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+// every bulk group of this thread has completed (its writes performed)
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Programmatic dependent launch.  A kernel launched with the programmatic stream
 // serialization attribute may be scheduled while the kernel before it in the stream is
 // still running.  Every such kernel calls wait_prior_grid() before it reads or writes
@@ -317,6 +344,9 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // barrier makes every write of the barrier's threads visible to an acquiring reader).
 __device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_release_gpu_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;

@@ -341,29 +341,27 @@ gn_apply_kernel(const T* __restrict__ x, T* __restrict__ out, const T* __restric
 // barrier and counter[1] departures; the last block to leave zeroes both.
 
 // Arrive at the grid barrier: once every thread of the block has finished the writes the
-// barrier publishes, one thread counts the block in.  grid_wait() then waits for all blocks;
-// work in between overlaps the wait.
+// barrier publishes (the block barrier orders them before thread 0), thread 0 counts the
+// block in with a release reduction at GPU scope.  grid_wait() then waits for all blocks
+// (an acquire load, so the other blocks' published writes are visible after the block
+// barrier); work in between overlaps the wait.
 __device__ __forceinline__ void grid_arrive(unsigned* count) {
   __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(count, 1u);
-  }
+  if (threadIdx.x == 0) red_release_gpu_add(count, 1u);
 }
 __device__ __forceinline__ bool grid_wait(unsigned* count, unsigned total, int* err) {
   __shared__ int s_ok;
   if (threadIdx.x == 0) {
     int ok = 1;
     const long long t0 = clock64();
-    while (*reinterpret_cast<volatile unsigned*>(count) < total) {
+    while (ld_acquire_gpu(count) < total) {
       if (clock64() - t0 > kWaitLimitCycles) {
         atomicCAS(err, 0, kErrGridSync);
         ok = 0;
         break;
       }
-      __nanosleep(64);
+      __nanosleep(32);
     }
-    __threadfence();
     s_ok = ok;
   }
   __syncthreads();
@@ -599,6 +597,310 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
   }
 }
 
+// ---------------------------------------------------------------- streamed GroupNorm (bf16)
+// The fused GroupNorm with its two passes over the chunk moved by the copy engine: one
+// thread streams the chunk (contiguous: pixels [pix0, pix1) of patch p, all channels)
+// through a ring of kGsStages shared-memory stages with bulk copies completing on
+// mbarriers, so the threads only read shared memory and the memory system always has
+// kGsStages - 1 stages (~96 KB per SM) in flight.  Statistics pass: the stages are summed
+// as in gn_fused_kernel (the same shifts, the same fixed per-thread pixel order, so the
+// same partial sums).  Apply pass: its first stages are requested before the grid barrier
+// (the reads do not depend on it), each stage is normalised in place, and written back
+// with a bulk store (plus the stores of the rows that are a neighbour's halo on sync
+// steps).  The first pass's copies ask L2 to keep the lines (the chunk is read again),
+// the second's to drop them first.
+constexpr int kGsStages = 3;
+constexpr int kGsStageBytes = 49152;
+
+int gs_stage_pixels(int C) { return std::max(1, kGsStageBytes / (C * 2)); }
+size_t gs_smem_bytes(int C) {
+  const int PL = kGnThreads / (C / 8);
+  return (size_t)kGsStages * gs_stage_pixels(C) * C * 2 + (size_t)(2 * PL + 2) * C * sizeof(float);
+}
+
+template <bool SILU>
+__global__ void __launch_bounds__(kGnThreads, 1)
+gn_stream_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int stage_pix, int* err) {
+  using T = __nv_bfloat16;
+  constexpr int VEC = 8;
+  constexpr int S = kGsStages;
+  extern __shared__ __align__(128) uint8_t gs_smem[];
+  __shared__ __align__(8) uint64_t full[S];
+  __shared__ __align__(16) float s_mr[256 * 2];    // (mean, rstd) of this patch's groups
+  __shared__ __align__(16) float s_mom[256 * 2];   // fresh moments (mean, var) of the patches needed
+  __shared__ float s_shift[256];                   // their shifts K
+  __shared__ __align__(16) float s_stale[256 * 2]; // previous step's moments of the image's patches
+  const int C = a.C, G = a.G;
+  const int V = C / VEC;
+  const int PL = kGnThreads / V;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int vc = tid % V, pl = tid / V;
+  const int lp = blockIdx.y, p = a.p0 + lp, chunk = blockIdx.x;
+  const int pix0 = chunk * pix_per_chunk;
+  const int pix1 = min(pix0 + pix_per_chunk, a.pix_per_patch);
+  const int nst = (pix1 - pix0 + stage_pix - 1) / stage_pix;   // stages of the chunk
+  const size_t stage_elems = (size_t)stage_pix * C;
+  T* ring = reinterpret_cast<T*>(gs_smem);
+  float* sh = reinterpret_cast<float*>(gs_smem + (size_t)S * stage_elems * sizeof(T));
+  float* chan = sh + 2 * PL * C;
+  const T* src = static_cast<const T*>(a.x) + (size_t)p * a.pix_per_patch * C;
+
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) mbar_init(smem_u32(&full[i]), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  wait_prior_grid();            // everything below reads or writes buffers of other launches
+  allow_next_grid();
+
+  // load number L (stage L of the first pass, stage L - nst of the second) into slot L % S
+  auto issue = [&](int L, uint64_t pol) {
+    const int k = L < nst ? L : L - nst;
+    const int s0 = pix0 + k * stage_pix, n = min(stage_pix, pix1 - s0);
+    const uint32_t bytes = (uint32_t)n * C * 2, bar = smem_u32(&full[L % S]);
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load_policy(smem_u32(ring + (size_t)(L % S) * stage_elems), src + (size_t)s0 * C, bytes, bar, pol);
+  };
+  // every thread waits for load L (a failed wait ends the kernel's work, recorded in err)
+  auto ready = [&](int L) { return mbar_wait(smem_u32(&full[L % S]), (uint32_t)(L / S) & 1u, err, kErrWaitTmaFull); };
+  const uint64_t keep = l2_evict_last_policy(), drop = l2_evict_first_policy();
+
+  const int last_row0 = a.pix_per_patch - o.W;
+  const int NI = a.per_image, pi = p % NI;                 // patch within its image
+  const bool top_src = o.halo_mode != 0 && pi > 0;         // my first row feeds patch p-1
+  const bool bot_src = o.halo_mode != 0 && pi < NI - 1;    // my last row feeds patch p+1
+  // ---- pass 1: per-channel partial sums of x - K (K: the group's shift) over this chunk
+  // Loads 0 .. 2 nst - 1 (both passes) in order; load L + S goes into L's slot once load L is
+  // consumed, so the first pass's last slots already bring in the second pass's first stages.
+  bool ok = true;
+  int issued = 0;               // thread 0: loads issued
+  if (tid == 0)
+    for (; issued < min(S, 2 * nst); ++issued) issue(issued, issued < nst ? keep : drop);
+  {
+    float s1[VEC], s2[VEC], k[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) s1[i] = s2[i] = 0.f;
+    if (pl < PL) gn_thread_shifts<T, VEC>(a.x, p, a.pix_per_patch, C, vc * VEC, C / G, k);
+    for (int L = 0; L < nst; ++L) {
+      ok = ok && ready(L);
+      const T* st = ring + (size_t)(L % S) * stage_elems;
+      const int n = min(stage_pix, pix1 - (pix0 + L * stage_pix));
+      if (ok && pl < PL) {
+        for (int q = pl; q < n; q += PL) {
+          float v[VEC];
+          unpack16(*reinterpret_cast<const uint4*>(st + (size_t)q * C + vc * VEC), v);
+#pragma unroll
+          for (int i = 0; i < VEC; ++i) {
+            const float d = v[i] - k[i];
+            s1[i] += d;
+            s2[i] = fmaf(d, d, s2[i]);
+          }
+        }
+      }
+      __syncthreads();   // the slot is consumed
+      if (tid == 0 && ok && L + S < 2 * nst) {
+        issue(L + S, L + S < nst ? keep : drop);
+        issued = L + S + 1;
+      }
+    }
+    if (pl < PL) {
+      float4* d1 = reinterpret_cast<float4*>(sh + pl * C + vc * VEC);
+      float4* d2 = reinterpret_cast<float4*>(sh + PL * C + pl * C + vc * VEC);
+#pragma unroll
+      for (int i = 0; i < VEC / 4; ++i) {
+        d1[i] = make_float4(s1[4 * i], s1[4 * i + 1], s1[4 * i + 2], s1[4 * i + 3]);
+        d2[i] = make_float4(s2[4 * i], s2[4 * i + 1], s2[4 * i + 2], s2[4 * i + 3]);
+      }
+    }
+  }
+  __syncthreads();
+  for (int c = tid; c < C; c += kGnThreads) {
+    float t1 = 0.f, t2 = 0.f;
+    for (int l = 0; l < PL; ++l) { t1 += sh[l * C + c]; t2 += sh[PL * C + l * C + c]; }
+    chan[c] = t1;
+    chan[C + c] = t2;
+  }
+  __syncthreads();
+  const int cg = C / G;
+  for (int g = warp; g < G; g += kGnThreads / 32) {
+    float t1 = 0.f, t2 = 0.f;
+    for (int c = lane; c < cg; c += 32) { t1 += chan[g * cg + c]; t2 += chan[C + g * cg + c]; }
+    t1 = warp_sum(t1);
+    t2 = warp_sum(t2);
+    if (lane == 0) reinterpret_cast<float2*>(a.part)[((size_t)lp * n_chunks + chunk) * G + g] = make_float2(t1, t2);
+  }
+  // what the merge and the normalisation need besides the other blocks' partials, read
+  // before the barrier: this thread's gamma and beta, the shifts of the patches merged and
+  // the previous step's moments of the image's patches
+  float gm[VEC], bt[VEC];
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) {
+    gm[i] = pl < PL ? __ldg(a.gamma + vc * VEC + i) : 0.f;
+    bt[i] = pl < PL ? __ldg(a.beta + vc * VEC + i) : 0.f;
+  }
+  const int rule = gn_rule(a);
+  const bool all = rule == kGnSync;             // the sync rule merges the image's fresh moments
+  const int p_lo = all ? p - pi : p, np = all ? NI : 1;
+  const int items = np * G;                     // <= 256
+
+  // ---- grid barrier: every chunk partial is written
+  const unsigned total = gridDim.x * gridDim.y;
+  grid_arrive(a.counter);
+  // the merge's other inputs, read while the other blocks reach the barrier
+  if (tid < items) s_shift[tid] = gn_shift<T>(a.x, p_lo + tid / G, a.pix_per_patch, C, tid % G, cg);
+  if (rule == kGnCorrected || rule == kGnStaleOthers)
+    for (int i = tid; i < NI * G * 2; i += kGnThreads) s_stale[i] = a.stale[(size_t)(p - pi) * G * 2 + i];
+  // displaced steps: the halo rows are last step's values, final already -- copy them
+  // while the other blocks reach the barrier
+  if (o.halo_mode == 2 && pl < PL && ((top_src && pix0 < o.W) || (bot_src && pix1 > last_row0))) {
+    T* outp = static_cast<T*>(o.out);
+    const T* prev = static_cast<const T*>(o.prev_slab);
+    for (int q0 = pix0 + pl; q0 < pix1; q0 += 8 * PL) {
+      uint4 hv[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int q = q0 + j * PL;
+        const bool need = q < pix1 && ((top_src && q < o.W) || (bot_src && q >= last_row0));
+        hv[j] = need ? ld_nc16(prev + ((size_t)p * o.out_patch_stride + o.out_off + q) * C + vc * VEC)
+                     : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int q = q0 + j * PL;
+        if (q >= pix1) break;
+        if (top_src && q < o.W)
+          *reinterpret_cast<uint4*>(outp + ((size_t)(p - 1) * o.out_patch_stride + o.out_off + a.pix_per_patch + q) *
+                                               C + vc * VEC) = hv[j];
+        if (bot_src && q >= last_row0)
+          *reinterpret_cast<uint4*>(outp + ((size_t)(p + 1) * o.out_patch_stride + (q - last_row0)) * C + vc * VEC) =
+              hv[j];
+      }
+    }
+  }
+  if (!grid_wait(a.counter, total, err)) ok = false;
+
+  // ---- merge: fresh moments of the patches needed, in a fixed order
+  const int SP = kGnThreads / items;            // threads per item, >= 2
+  float* red = sh;                              // [SP][items][2]
+  if (ok && tid < SP * items) {
+    const int item = tid % items, part_id = tid / items;
+    const int pp = p_lo + item / G - a.p0, gg = item % G;
+    const float2* srcp = reinterpret_cast<const float2*>(a.part) + (size_t)pp * n_chunks * G + gg;
+    float2 acc = make_float2(0.f, 0.f);
+    for (int c = part_id; c < n_chunks; c += 8 * SP) {
+      float2 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = c + u * SP < n_chunks ? __ldcg(srcp + (size_t)(c + u * SP) * G) : make_float2(0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) { acc.x += v[u].x; acc.y += v[u].y; }
+    }
+    red[(part_id * items + item) * 2 + 0] = acc.x;
+    red[(part_id * items + item) * 2 + 1] = acc.y;
+  }
+  __syncthreads();
+  const float inv_n = 1.f / ((float)a.pix_per_patch * (float)cg);
+  if (ok && tid < items) {
+    float t1 = 0.f, t2 = 0.f;
+    for (int s2 = 0; s2 < SP; ++s2) { t1 += red[(s2 * items + tid) * 2]; t2 += red[(s2 * items + tid) * 2 + 1]; }
+    const float m1 = t1 * inv_n;
+    s_mom[tid * 2] = s_shift[tid] + m1;
+    s_mom[tid * 2 + 1] = fmaxf(fmaf(-m1, m1, t2 * inv_n), 0.f);
+  }
+  __syncthreads();
+  if (ok && tid < G) {
+    const int gg = tid;
+    const int own = (all ? pi : 0) * G + gg;
+    const float2 mo = make_float2(s_mom[own * 2], s_mom[own * 2 + 1]);
+    const float* img = (rule == kGnSync ? s_mom : s_stale) + 2 * gg;
+    const float2 e = gn_estimate(rule, NI, pi, mo, img, G);
+    const float rstd = 1.f / sqrtf(e.y + a.eps);
+    s_mr[gg * 2] = e.x;
+    s_mr[gg * 2 + 1] = rstd;
+    if (chunk == 0) {
+      a.fresh_out[(p * G + gg) * 2] = mo.x;
+      a.fresh_out[(p * G + gg) * 2 + 1] = mo.y;
+      a.mean_rstd[(p * G + gg) * 2] = e.x;
+      a.mean_rstd[(p * G + gg) * 2 + 1] = rstd;
+    }
+  }
+  __syncthreads();
+
+  // ---- pass 2: normalise (+SiLU) each stage in place and store it back
+  float scl[VEC], sft[VEC];
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) {
+    const int c = vc * VEC + i;
+    scl[i] = gm[i] * s_mr[(c / cg) * 2 + 1];
+    sft[i] = bt[i] - s_mr[(c / cg) * 2] * scl[i];
+  }
+  T* outp = static_cast<T*>(o.out);
+  for (int k = 0; k < nst; ++k) {
+    const int L = nst + k;
+    ok = ok && ready(L);
+    T* st = ring + (size_t)(L % S) * stage_elems;
+    const int s0 = pix0 + k * stage_pix, n = min(stage_pix, pix1 - s0);
+    if (ok && pl < PL) {
+      for (int q = pl; q < n; q += PL) {
+        uint4* cell = reinterpret_cast<uint4*>(st + (size_t)q * C + vc * VEC);
+        float v[VEC];
+        unpack16(*cell, v);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) {
+          v[i] = fmaf(v[i], scl[i], sft[i]);
+          if (SILU) {
+            // SiLU as v/2 (1 + tanh(v/2)): one MUFU operation (the approximate tanh, relative
+            // error below 2^-10, is finer than the bf16 output's rounding)
+            const float hv = 0.5f * v[i];
+            v[i] = fmaf(hv, tanh_approx(hv), hv);
+          }
+        }
+        *cell = pack16(v);
+      }
+    }
+    fence_proxy_async_smem();   // this thread's writes, before the copy engine reads them
+    __syncthreads();
+    if (tid == 0 && ok) {
+      const uint32_t sa = smem_u32(st);
+      bulk_store(outp + ((size_t)p * o.out_patch_stride + o.out_off + s0) * C, sa, (uint32_t)n * C * 2);
+      if (o.halo_mode == 1) {
+        // sync steps: this step's boundary rows are also the neighbours' halo rows
+        if (top_src && s0 < o.W) {
+          const int e = min(s0 + n, o.W);
+          bulk_store(outp + ((size_t)(p - 1) * o.out_patch_stride + o.out_off + a.pix_per_patch + s0) * C, sa,
+                     (uint32_t)(e - s0) * C * 2);
+        }
+        if (bot_src && s0 + n > last_row0) {
+          const int b = max(s0, last_row0);
+          bulk_store(outp + ((size_t)(p + 1) * o.out_patch_stride + (b - last_row0)) * C,
+                     sa + (uint32_t)(b - s0) * C * 2, (uint32_t)(s0 + n - b) * C * 2);
+        }
+      }
+      bulk_commit();
+      // refill the previous stage's slot (its stores have read it by now, as a rule), so two
+      // stages stay in flight while this one's stores run
+      if (L - 1 >= nst && L - 1 + S < 2 * nst) {
+        bulk_wait_read_prev();
+        issue(L - 1 + S, drop);
+        issued = L - 1 + S + 1;
+      }
+    }
+  }
+  if (tid == 0) {
+    bulk_wait_all();
+    if (!ok) {
+      // a wait gave up: let the loads still in flight land before the block exits (the last
+      // load issued into each slot; the earlier ones of a slot completed before it)
+      for (int L = max(0, issued - S); L < issued; ++L)
+        mbar_wait(smem_u32(&full[L % S]), (uint32_t)(L / S) & 1u, err, kErrWaitTmaFull);
+    }
+  }
+  // ---- departure: the last block out re-arms the barrier for the next launch
+  if (tid == 0 && atomicAdd(a.counter + 1, 1u) == total - 1) {
+    a.counter[0] = 0u;
+    a.counter[1] = 0u;
+  }
+}
+
 
 // Pixels per block: one wave of 512-thread blocks over the whole map.
 // Per-token LayerNorm (transformer blocks of the SDXL-style stage): one warp per
@@ -722,18 +1024,23 @@ cudaError_t launch_gn_apply(const T* x, T* out, const T* prev_slab, const float*
 template <typename T>
 cudaError_t launch_gn_fused(const GnArgs& a, const GnOut& o, bool silu, int* err, cudaStream_t s) {
   constexpr int VEC = VecTraits<T>::kN;
+  constexpr bool kStream = sizeof(T) == 2;   // bf16: the streamed kernel
   const int V = a.C / VEC;
   const int PL = kGnThreads / V;
-  size_t smem = (size_t)(2 * PL + 2) * a.C * sizeof(float);
+  size_t smem = kStream ? gs_smem_bytes(a.C) : (size_t)(2 * PL + 2) * a.C * sizeof(float);
   const size_t red = (size_t)kGnThreads * 2 * sizeof(float);
   if (smem < red) smem = red;
-  auto kern = silu ? gn_fused_kernel<T, true> : gn_fused_kernel<T, false>;
+  using Kern = void (*)(GnArgs, GnOut, int, int, int*);
+  using SKern = void (*)(GnArgs, GnOut, int, int, int, int*);
+  Kern kern = silu ? gn_fused_kernel<T, true> : gn_fused_kernel<T, false>;
+  SKern skern = silu ? gn_stream_kernel<true> : gn_stream_kernel<false>;
+  const void* kfn = kStream ? reinterpret_cast<const void*>(skern) : reinterpret_cast<const void*>(kern);
   // every block must be resident at once (the grid barrier): at most the occupancy
   // limit, and no more chunks than the partial-sum scratch holds
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGnThreads, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, kGnThreads, smem);
   if (e != cudaSuccess) return e;
   const int max_blocks = per_sm * sm_count();
   const int n_run = a.n_run > 0 ? a.n_run : a.N;   // patches computed
@@ -757,12 +1064,17 @@ cudaError_t launch_gn_fused(const GnArgs& a, const GnOut& o, bool silu, int* err
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = a.pdl ? 2 : 1;
-  e = cudaLaunchKernelEx(&cfg, kern, a, o, n_chunks, per, err);
+  const int stage_pix = gs_stage_pixels(a.C);
+  auto go = [&]() {
+    return kStream ? cudaLaunchKernelEx(&cfg, skern, a, o, n_chunks, per, stage_pix, err)
+                   : cudaLaunchKernelEx(&cfg, kern, a, o, n_chunks, per, err);
+  };
+  e = go();
   if (e != cudaSuccess && a.pdl) {
     // a runtime that does not take both attributes together: launch it plainly
     cudaGetLastError();
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, a, o, n_chunks, per, err);
+    e = go();
   }
   return e;
 }

@@ -119,13 +119,10 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmPlan& plan, const Epil
     }
     return;
   }
-#pragma unroll
-  for (int c = 0; c < BN / 32; ++c) {
-    uint32_t r[32];
-    tmem_ld32(taddr + c * 32, r);
-    tmem_wait_ld();
+  // store the 32 columns of chunk c (registers r, already loaded)
+  auto store_chunk = [&](int c, const uint32_t (&r)[32]) {
     const int n = n0 + c * 32;
-    if (gm < 0 || n >= plan.N) continue;
+    if (gm < 0 || n >= plan.N) return;
     float v[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
@@ -148,7 +145,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmPlan& plan, const Epil
       if (epi.n_store && n + 32 > epi.n_store) {
         // only the first n_store columns exist in the output (a padded narrow layer)
         for (int i = 0; i < 32 && n + i < epi.n_store; ++i) dst[i] = __float2bfloat16_rn(v[i]);
-        continue;
+        return;
       }
     } else {
       const int which = n / epi.C, cc = n - which * epi.C;
@@ -164,6 +161,16 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmPlan& plan, const Epil
       for (int e = 0; e < 8; ++e) w8[e] = v[i * 8 + e];
       d4[i] = pack16(w8);
     }
+  };
+  // the next chunk's TMEM load is in flight while this one is converted and stored
+  uint32_t r[2][32];
+  tmem_ld32(taddr, r[0]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    if (c + 1 < BN / 32) tmem_ld32(taddr + (c + 1) * 32, r[(c + 1) & 1]);
+    store_chunk(c, r[c & 1]);
+    tmem_wait_ld();
   }
 }
 
