@@ -29,6 +29,7 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kThreads = 192;
+constexpr uint32_t kStageBytes = 4 * 2048;   // the epilogue warps' transpose buffers
 
 template <int BN> struct TmemCols { static constexpr uint32_t v = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256; };
 
@@ -88,9 +89,13 @@ __device__ __forceinline__ void prefetch_residual(const Epilogue& epi, long long
 
 // Epilogue of one tile: drain the 128 x BN accumulator at TMEM address taddr (this warp's
 // lanes) and store row gm (-1: nothing to store; the TMEM reads still run warp-wide).
+// stage: this warp's 2 KB of shared memory.  A warp's 32 x 32 chunk goes through it so that
+// each store instruction writes 8 whole 64-byte row segments rather than 32 scattered 16-byte
+// pieces (the rows of a warp are 32 output rows, each lane holds one).
 template <int BN>
 __device__ __forceinline__ void epilogue_tile(const TcGemmPlan& plan, const Epilogue& epi, long long gm, int n0,
-                                              uint32_t taddr, const uint4 (&res)[BN / 8]) {
+                                              uint32_t taddr, const uint4 (&res)[BN / 8], uint4* stage) {
+  const int lane = threadIdx.x & 31;
   if (BN == 128 && epi.kind == 2) {
     // GEGLU: columns [0, 64) are values, [64, 128) the gates of the same features
 #pragma unroll 1
@@ -119,10 +124,10 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmPlan& plan, const Epil
     }
     return;
   }
-  // store the 32 columns of chunk c (registers r, already loaded)
+  // store the 32 columns of chunk c (registers r, already loaded); warp-wide
   auto store_chunk = [&](int c, const uint32_t (&r)[32]) {
     const int n = n0 + c * 32;
-    if (gm < 0 || n >= plan.N) return;
+    if (n >= plan.N) return;   // warp-uniform
     float v[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
@@ -141,26 +146,44 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmPlan& plan, const Epil
           for (int e = 0; e < 8; ++e) v[i * 8 + e] += rr[e];
         }
       }
-      dst = static_cast<__nv_bfloat16*>(epi.out) + gm * epi.ldo + n;
       if (epi.n_store && n + 32 > epi.n_store) {
         // only the first n_store columns exist in the output (a padded narrow layer)
+        if (gm < 0) return;
+        dst = static_cast<__nv_bfloat16*>(epi.out) + gm * epi.ldo + n;
         for (int i = 0; i < 32 && n + i < epi.n_store; ++i) dst[i] = __float2bfloat16_rn(v[i]);
         return;
       }
-    } else {
-      const int which = n / epi.C, cc = n - which * epi.C;
-      const int head = cc >> 6, d0 = cc & 63;
-      void* base = which == 0 ? epi.q : (which == 1 ? epi.k : epi.v);
-      dst = static_cast<__nv_bfloat16*>(base) + ((long long)head * epi.L + gm) * 64 + d0;
     }
-    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    // the row through shared memory: 16-byte pieces swizzled by row (conflict-free both ways)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       float w8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) w8[e] = v[i * 8 + e];
-      d4[i] = pack16(w8);
+      stage[lane * 4 + (i ^ ((lane >> 1) & 3))] = pack16(w8);
     }
+    __syncwarp();
+    // lane 4 rr + ch stores piece ch of rows rr, rr + 8, rr + 16, rr + 24
+    const int ch = lane & 3;
+    long long head_base = 0;
+    void* base = epi.out;
+    if (epi.kind != 0) {
+      const int which = n / epi.C, cc = n - which * epi.C;
+      base = which == 0 ? epi.q : (which == 1 ? epi.k : epi.v);
+      head_base = (long long)(cc >> 6) * epi.L * 64 + (cc & 63);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int rr = k * 8 + (lane >> 2);
+      const long long g = __shfl_sync(0xffffffffu, gm, rr);
+      const uint4 piece = stage[rr * 4 + (ch ^ ((rr >> 1) & 3))];
+      if (g >= 0) {
+        __nv_bfloat16* d = static_cast<__nv_bfloat16*>(base) +
+                           (epi.kind == 0 ? g * epi.ldo + n : head_base + g * 64) + ch * 8;
+        *reinterpret_cast<uint4*>(d) = piece;
+      }
+    }
+    __syncwarp();   // the stage is read before the next chunk rewrites it
   };
   // the next chunk's TMEM load is in flight while this one is converted and stored
   uint32_t r[2][32];
@@ -192,7 +215,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * kABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * kBBytes);
+  uint4* sStage = reinterpret_cast<uint4*>(sB + STAGES * kBBytes);   // 4 epilogue warps x 2 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * kBBytes + kStageBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* acc_full = bars + 2 * STAGES;                // [2]
@@ -325,7 +349,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       const bool ready = mbar_wait(smem_u32(&acc_full[buf]), use & 1, err, kErrWaitAccum);
       tc_fence_after();
       epilogue_tile<BN>(plan, epi, ready && !s_abort ? gm : -1, n0,
-                        tmem_d + buf * kCols + ((uint32_t)(sub * 32) << 16), res);
+                        tmem_d + buf * kCols + ((uint32_t)(sub * 32) << 16), res, sStage + sub * 128);
       tc_fence_before();
       mbar_arrive(smem_u32(&acc_empty[buf]));
       if (!ready) break;
@@ -360,7 +384,8 @@ tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * kABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * kBBytes);
+  uint4* sStage = reinterpret_cast<uint4*>(sB + STAGES * kBBytes);   // 4 epilogue warps x 2 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * kBBytes + kStageBytes);
   uint64_t* full = bars;                                 // leader's: both CTAs' loads
   uint64_t* empty = bars + STAGES;                       // each CTA's, from the leader's commits
   uint64_t* acc_full = bars + 2 * STAGES;                // [2] each CTA's
@@ -510,7 +535,7 @@ tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_const
       const bool ready = mbar_wait_cluster(smem_u32(&acc_full[buf]), use & 1, err, kErrWaitAccum);
       tc_fence_after();
       epilogue_tile<BN>(plan, epi, ready && !s_abort ? gm : -1, n0,
-                        tmem_d + buf * kCols + ((uint32_t)(sub * 32) << 16), res);
+                        tmem_d + buf * kCols + ((uint32_t)(sub * 32) << 16), res, sStage + sub * 128);
       tc_fence_before();
       // the four epilogue warps of this CTA are done with the accumulator; they also agree
       // on giving up (a failed wait anywhere ends the loop for all of them)
@@ -541,7 +566,8 @@ tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_const
 template <int BN, int STAGES>
 cudaError_t launch_pair(const TcGemmPlan& plan, const CUtensorMap& mA, const CUtensorMap& mB,
                         const Epilogue& epi, int* err, cudaStream_t s) {
-  const size_t smem = 1024 + (size_t)STAGES * 2 * (kBM * kBK * 2 + (BN / 2) * kBK * 2) + (2 * STAGES + 8) * 8 + 64;
+  const size_t smem = 1024 + (size_t)STAGES * 2 * (kBM * kBK * 2 + (BN / 2) * kBK * 2) + kStageBytes +
+                      (2 * STAGES + 8) * 8 + 64;
   auto kern = tc_gemm_pair_kernel<BN, STAGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -578,7 +604,8 @@ cudaError_t launch_pair(const TcGemmPlan& plan, const CUtensorMap& mA, const CUt
 template <int BN, int STAGES>
 cudaError_t launch_bn(const TcGemmPlan& plan, const CUtensorMap& mA, const CUtensorMap& mB,
                       const Epilogue& epi, int* err, cudaStream_t s) {
-  const size_t smem = 1024 + (size_t)STAGES * 2 * (kBM * kBK * 2 + BN * kBK * 2) + (2 * STAGES + 6) * 8 + 64;
+  const size_t smem = 1024 + (size_t)STAGES * 2 * (kBM * kBK * 2 + BN * kBK * 2) + kStageBytes +
+                      (2 * STAGES + 6) * 8 + 64;
   auto kern = tc_gemm_kernel<BN, STAGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
