@@ -310,6 +310,15 @@ DFP_API dfp_status dfp_set_launch_overlap(dfp_handle h, int enable);
  * fp32).  Returns DFP_E_UNSUPPORTED for tensor cores with fp32. */
 DFP_API dfp_status dfp_set_kernel_family(dfp_handle h, int family);
 
+/* Work split of the tensor-core attention (no counterpart in the pages; a tuning knob): when
+ * the K/V bytes one launch reads (every head, fresh and stale rows) exceed `bytes`, the launch
+ * deals rounds of whole (head, patch, query-tile pair) units to its CTAs, so the CTAs in
+ * flight share one or two heads' K/V in L2; below it, every KV tile is split stream-K.
+ * 0 (the default) takes the kernel's own budget, 48 MB; 1 forces the whole-unit rounds
+ * wherever there are at least as many units as CTAs.  Results do not depend on it beyond
+ * rounding order.  DFP_E_ARG for bytes < 0. */
+DFP_API dfp_status dfp_set_attention_kv_budget(dfp_handle h, long long bytes);
+
 /* Per-kernel timing.  With profiling on, dfp_step brackets every kernel launch
  * with CUDA events recorded on the handle's stream.  dfp_kernel_times waits for
  * the last step's events and writes up to max_n durations (milliseconds) and the

@@ -636,6 +636,13 @@ dfp_status dfp_set_launch_overlap(dfp_handle h, int enable) {
   return DFP_OK;
 }
 
+dfp_status dfp_set_attention_kv_budget(dfp_handle h, long long bytes) {
+  if (!h) return DFP_E_ARG;
+  if (bytes < 0) return h->fail(DFP_E_ARG, "the K/V budget must be >= 0");
+  h->attn_kv_budget = bytes;
+  return DFP_OK;
+}
+
 dfp_status dfp_set_kernel_family(dfp_handle h, int family) {
   if (!h) return DFP_E_ARG;
   if (family != 0 && family != 1) return h->fail(DFP_E_ARG, "family must be 0 or 1");
@@ -789,6 +796,7 @@ dfp_status run_step(dfp_ctx* h, const void* xv, int step, int is_sync, int p0, i
     a.p_lo = p0; a.p_hi = p1;
     a.ctas = h->attn_ctas; a.n_qtiles = (Lp + 127) / 128;
     a.part_o = h->attn_part_o; a.part_ml = h->attn_part_ml; a.flags = h->attn_flags;
+    a.kv_budget = h->attn_kv_budget;
     DFP_LAUNCH(launch_tc_attention(a, h->m_q, h->m_k[cur], h->m_v[cur], h->m_k[prv], h->m_v[prv], s), "attention (tcgen05)");
   } else {
     DFP_LAUNCH(launch_simt_attention<T>(static_cast<const T*>(h->q), static_cast<const T*>(h->kb[cur]),

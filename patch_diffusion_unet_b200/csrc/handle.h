@@ -38,6 +38,7 @@ struct dfp_ctx {
   int R = 0, L = 0, Lp = 0, family = 0;
   int B = 1;                   // images per step (the guidance batch); L, Lp are per image
   bool overlap = true;         // programmatic dependent launch between the step's kernels
+  long long attn_kv_budget = 0;   // attention whole-unit rounds above this many K/V bytes (0: default)
   size_t esz = 4;
   // weights
   void* w_conv = nullptr;   // [C][9][C]

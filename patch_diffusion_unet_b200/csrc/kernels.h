@@ -70,6 +70,21 @@ cudaError_t launch_concat(const void* a, int Ca, const void* b, int Cb, void* ou
 // embedding of timestep x_tau (cols entries)
 cudaError_t launch_gemv(const float* W, const float* b, const float* add, const float* x, float x_tau, float* y,
                         int rows, int cols, bool silu_out, bool pdl, cudaStream_t s);
+// y_s = W_s x + b_s (+ add_s) for up to kGemvSegs segments over one x [cols] (cols % 4 == 0,
+// 16-byte aligned W and x), one launch
+constexpr int kGemvSegs = 8;
+struct GemvSeg {
+  const float* W;     // [rows][cols]
+  const float* b;
+  const float* add;   // may be null
+  float* y;
+  int rows;
+};
+struct GemvBatch {
+  GemvSeg seg[kGemvSegs];
+  int n;
+};
+cudaError_t launch_gemv_multi(const GemvBatch& batch, const float* x, int cols, bool pdl, cudaStream_t s);
 // DDIM update lat = c1 lat + c2 eps (fp32 latent, bf16 eps), and its bf16 copy
 cudaError_t launch_ddim_update(float* lat, const void* eps, void* x_bf, long long n, float c1, float c2, bool pdl,
                                cudaStream_t s);
@@ -171,6 +186,7 @@ struct TcAttnArgs {
   int head_tiles;         // tiles of one head's units
   unsigned epoch;         // set by the launcher: this launch's flag value (never 0, never reused)
   int pdl;                // launch with programmatic stream serialization
+  long long kv_budget;    // K/V bytes above which whole-unit rounds are used (0: the kernel's own)
 };
 // floats of part_o for `ctas` CTAs (part_ml needs 1/32 of it)
 size_t attention_scratch_floats(int ctas);

@@ -391,6 +391,7 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
     a.images = B; a.kv_stride = L; a.pdl = pdl;
     a.n_qtiles = (Lp + 127) / 128; a.ctas = h->attn_ctas;
     a.part_o = h->attn_part_o; a.part_ml = h->attn_part_ml; a.flags = h->attn_flags;
+    a.kv_budget = h->attn_kv_budget;
     DFP_LAUNCH(launch_tc_attention(a, h->m_q, x.m_k[cur], x.m_v[cur], x.m_k[prv], x.m_v[prv], s),
                "self-attention (tcgen05)");
     Epilogue eo{};
@@ -407,6 +408,7 @@ dfp_status stage_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
     ca.pdl = pdl;
     ca.o = h->o; ca.err = h->dev_err; ca.n_qtiles = (L + 127) / 128; ca.ctas = h->attn_ctas;
     ca.part_o = h->attn_part_o; ca.part_ml = h->attn_part_ml; ca.flags = h->attn_flags;
+    ca.kv_budget = h->attn_kv_budget;
     DFP_LAUNCH(launch_tc_attention(ca, h->m_q, x.m_ck, x.m_cv, x.m_ck, x.m_cv, s), "cross-attention (tcgen05)");
     eo.out = r_ca; eo.bias = x.b_o2; eo.residual = r_sa;
     DFP_LAUNCH(launch_tc_gemm(x.p_o2, st->m_o, x.m_wo2, eo, h->dev_err, s), "cross-attn out + residual (tcgen05)");

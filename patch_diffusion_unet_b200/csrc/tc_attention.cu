@@ -1029,7 +1029,7 @@ cudaError_t launch_tc_attention(const TcAttnArgs& args, const CUtensorMap& mq, c
   // a fresh flag value per launch (flags hold the epoch of the launch that last set them)
   static std::atomic<unsigned> epoch{0};
   do a.epoch = ++epoch; while (a.epoch == 0);
-  const int G = plan_schedule(a, a.ctas);
+  const int G = plan_schedule(a, a.ctas, a.kv_budget > 0 ? a.kv_budget : kL2KvBudget);
   if (G == 0) return cudaSuccess;
   if (G < 0) return cudaErrorInvalidValue;   // 32-bit schedule arithmetic
   cudaLaunchConfig_t cfg{};

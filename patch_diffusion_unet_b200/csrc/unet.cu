@@ -570,6 +570,7 @@ dfp_status run_xf(dfp_ctx* h, const StepCtx& k, UXf& x, const XfNames& nm, int& 
   a.L = L; a.Lp = x.lv.Lp; a.N = k.N; a.heads = x.heads; a.C = C; a.mode = k.sa_mode; a.o = h->o; a.err = h->dev_err;
   a.images = 1; a.kv_stride = L; a.pdl = pdl; a.n_qtiles = (x.lv.Lp + 127) / 128; a.ctas = h->attn_ctas;
   a.part_o = h->attn_part_o; a.part_ml = h->attn_part_ml; a.flags = h->attn_flags;
+  a.kv_budget = h->attn_kv_budget;
   DFP_LAUNCH(launch_tc_attention(a, x.m_q, x.m_k[k.cur], x.m_v[k.cur], x.m_k[k.prv], x.m_v[k.prv], s),
              nm.sa);
   DFP_LAUNCH(launch_tc_gemm(x.p_o1, x.m_o, x.m_wo1, plain_out(x.r, x.b_o1, C, x.r), h->dev_err, s),
@@ -584,6 +585,7 @@ dfp_status run_xf(dfp_ctx* h, const StepCtx& k, UXf& x, const XfNames& nm, int& 
   ca.images = 1; ca.kv_stride = (int)ctx_rows(c.ctx_len); ca.pdl = pdl;
   ca.o = h->o; ca.err = h->dev_err; ca.n_qtiles = (L + 127) / 128; ca.ctas = h->attn_ctas;
   ca.part_o = h->attn_part_o; ca.part_ml = h->attn_part_ml; ca.flags = h->attn_flags;
+  ca.kv_budget = h->attn_kv_budget;
   DFP_LAUNCH(launch_tc_attention(ca, x.m_q, x.m_ck, x.m_cv, x.m_ck, x.m_cv, s), nm.ca);
   DFP_LAUNCH(launch_tc_gemm(x.p_o2, x.m_o, x.m_wo2, plain_out(x.r, x.b_o2, C, x.r), h->dev_err, s),
              nm.o2);
@@ -624,9 +626,12 @@ dfp_status unet_step(dfp_ctx* h, const void* xv, int step, int is_sync) {
              "timestep embedding 1");
   DFP_LAUNCH(launch_gemv(u->t_w2, u->t_b2, nullptr, u->t_h, -1.f, u->t_act, te, te, true, k.pdl != 0, s),
              "timestep embedding 2");
-  for (URes* r : {&u->res0, &u->res1, &u->res2, &u->ures1, &u->ures0})
-    DFP_LAUNCH(launch_gemv(r->wt, r->bt, r->c1.b, u->t_act, -1.f, r->bias1, r->Cout, te, false, k.pdl != 0, s),
-               "time projections");
+  {
+    GemvBatch tb{};
+    for (URes* r : {&u->res0, &u->res1, &u->res2, &u->ures1, &u->ures0})
+      tb.seg[tb.n++] = GemvSeg{r->wt, r->bt, r->c1.b, r->bias1, r->Cout};
+    DFP_LAUNCH(launch_gemv_multi(tb, u->t_act, te, k.pdl != 0, s), "time projections");
+  }
   // ---- down path
   DFP_LAUNCH(launch_slab_fill(xv, 4, u->conv_in.slab[k.cur], u->conv_in.slab[k.prv], 64, N, l0.R, l0.W, k.halo_mode,
                               false, k.pdl != 0, s), "conv_in input");

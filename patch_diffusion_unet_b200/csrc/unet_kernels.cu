@@ -133,6 +133,32 @@ __global__ void gemv_kernel(const float* __restrict__ Wt, const float* __restric
   }
 }
 
+// Several y_s = W_s x + b_s (+ add_s) over the same x in one launch (the ResNets' time
+// projections): the warps of the grid take the segments' rows one after another.
+__global__ void gemv_multi_kernel(const GemvBatch batch, const float* __restrict__ x, int cols) {
+  wait_prior_grid();
+  allow_next_grid();
+  int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  int sgi = 0;
+  while (sgi < batch.n && r >= batch.seg[sgi].rows) r -= batch.seg[sgi++].rows;
+  if (sgi >= batch.n) return;
+  const GemvSeg& sg = batch.seg[sgi];
+  const float4* w4 = reinterpret_cast<const float4*>(sg.W + (size_t)r * cols);
+  const float4* x4 = reinterpret_cast<const float4*>(x);
+  float s = 0.f;
+#pragma unroll 4
+  for (int c4 = lane; c4 < cols / 4; c4 += 32) {
+    const float4 wv = __ldg(w4 + c4), xv = __ldg(x4 + c4);
+    s = fmaf(wv.x, xv.x, s);
+    s = fmaf(wv.y, xv.y, s);
+    s = fmaf(wv.z, xv.z, s);
+    s = fmaf(wv.w, xv.w, s);
+  }
+  s = warp_sum(s);
+  if (lane == 0) sg.y[r] = s + sg.b[r] + (sg.add ? sg.add[r] : 0.f);
+}
+
 // DDIM (eta = 0): lat = c1 * lat + c2 * eps over [L][4]; x_bf = bf16(lat) for the next UNet.
 __global__ void ddim_update_kernel(float* __restrict__ lat, const bf* __restrict__ eps, bf* __restrict__ x_bf,
                                    long long n, float c1, float c2) {
@@ -192,6 +218,16 @@ cudaError_t launch_gemv(const float* W, const float* b, const float* add, const 
   const bool vec4 = cols % 4 == 0 && reinterpret_cast<uintptr_t>(W) % 16 == 0;
   return launch_pdl(vec4 ? gemv_kernel<true> : gemv_kernel<false>, (rows * 32 + 255) / 256, 256, pdl, s, W, b, add,
                     x, x_tau, y, rows, cols, silu_out ? 1 : 0);
+}
+
+cudaError_t launch_gemv_multi(const GemvBatch& batch, const float* x, int cols, bool pdl, cudaStream_t s) {
+  if (cols % 4 || reinterpret_cast<uintptr_t>(x) % 16 || batch.n < 1 || batch.n > kGemvSegs) return cudaErrorInvalidValue;
+  int rows = 0;
+  for (int i = 0; i < batch.n; ++i) {
+    if (reinterpret_cast<uintptr_t>(batch.seg[i].W) % 16) return cudaErrorInvalidValue;
+    rows += batch.seg[i].rows;
+  }
+  return launch_pdl(gemv_multi_kernel, (rows * 32 + 255) / 256, 256, pdl, s, batch, x, cols);
 }
 
 cudaError_t launch_ddim_update(float* lat, const void* eps, void* x_bf, long long n, float c1, float c2, bool pdl,

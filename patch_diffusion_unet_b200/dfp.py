@@ -22,7 +22,7 @@ FAMILY_TENSOR_CORE, FAMILY_SIMT = 0, 1
 EXPORTED = ("dfp_create", "dfp_load_weights", "dfp_step", "dfp_step_host", "dfp_step_host_async",
             "dfp_synchronize", "dfp_output",
             "dfp_copy_out", "dfp_buffer_bytes", "dfp_check_device", "dfp_launches_per_step",
-            "dfp_set_kernel_family", "dfp_set_profiling", "dfp_kernel_times", "dfp_destroy",
+            "dfp_set_kernel_family", "dfp_set_attention_kv_budget", "dfp_set_profiling", "dfp_kernel_times", "dfp_destroy",
             "dfp_last_error", "dfp_group_norm_noalloc", "dfp_group_norm_noalloc_error",
             "dfp_selftest_wait_timeout", "dfp_selftest_exp2_poly", "dfp_set_launch_overlap",
             "dfp_attention_schedule_check", "dfp_step_patches", "dfp_context_buffer", "dfp_set_timestep",
@@ -63,6 +63,7 @@ def load_library(path=_LIB_PATH):
         "dfp_check_device": ([H], ctypes.c_int),
         "dfp_launches_per_step": ([H], ctypes.c_int),
         "dfp_set_kernel_family": ([H, ctypes.c_int], ctypes.c_int),
+        "dfp_set_attention_kv_budget": ([H, ctypes.c_longlong], ctypes.c_int),
         "dfp_set_launch_overlap": ([H, ctypes.c_int], ctypes.c_int),
         "dfp_attention_schedule_check": ([ctypes.c_int] * 10 + [ctypes.c_longlong], ctypes.c_int),
         "dfp_step_patches": ([H, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int], ctypes.c_int),
@@ -246,6 +247,10 @@ class DisplacedPatchBlock:
 
     def set_kernel_family(self, family):
         self._check(LIB.dfp_set_kernel_family(self.h, int(family)))
+
+    def set_attention_kv_budget(self, nbytes):
+        """K/V bytes above which the attention deals whole-unit rounds (0: the kernel's own)."""
+        self._check(LIB.dfp_set_attention_kv_budget(self.h, int(nbytes)))
 
     def set_launch_overlap(self, enable=True):
         """Programmatic dependent launch between the step's kernels (on by default)."""

@@ -44,18 +44,22 @@ def gpu_stage_views(blk, cfg):
 
 
 def run_parity(cfg, n_steps, oracle_from=0, query_tokens=None, gn_mode=0, context=0, family=None,
-               weight_scale=None, random_affine=False, stages=True, seed=0, x_fn=None, orc_out=None):
+               weight_scale=None, random_affine=False, stages=True, seed=0, x_fn=None, orc_out=None,
+               kv_budget=None):
     """Run steps 0..n_steps-1 on the GPU; the oracle joins at step `oracle_from` (which must be
     a sync step, so no earlier state is needed) and is compared at every step from there.
     x_fn(t, x) -> x' changes the workload's input of step t before both sides see it (values
     exactly representable in the storage type).  orc_out, a list, receives the oracle's
-    per-step outputs.  Returns a list of per-step dicts {stage: (rel_l2, max_abs)}."""
+    per-step outputs.  kv_budget sets the attention's K/V budget (1: whole-unit rounds wherever
+    there are enough units).  Returns a list of per-step dicts {stage: (rel_l2, max_abs)}."""
     from patch_diffusion_unet_b200 import dfp
 
     wl = inputs.SyntheticWorkload(cfg, seed=seed, weight_scale=weight_scale, random_affine=random_affine)
     blk = dfp.DisplacedPatchBlock(cfg, gn_mode=gn_mode, context=context)
     if family is not None:
         blk.set_kernel_family(family)
+    if kv_budget is not None:
+        blk.set_attention_kv_budget(kv_budget)
     blk.load_weights(wl.weights)
     omode = ["corrected", "stale_others", "sync", "separate"][gn_mode]
     octx = ["displaced", "naive"][context]

@@ -59,6 +59,13 @@ def test_config1_batch2_first_steps_all_stages():
     _assert(run_parity(cfg, 7), TOL["bf16"])
 
 
+def test_config1_batch2_whole_unit_rounds():
+    """Two images with the attention's large-map split forced (K/V budget of one byte): the
+    320 units (2 images x 4 patches x 10 heads x 4 pairs) make two whole rounds and a tail."""
+    cfg = configs.get(1, batch=2)
+    _assert(run_parity(cfg, 4, kv_budget=1), TOL["bf16"])
+
+
 def test_batch_image0_matches_single_image_run():
     """Image 0 of a batch is the single-image workload: its output agrees with the
     single-image handle's at the bf16 bar (the launch shapes differ, so not bitwise)."""

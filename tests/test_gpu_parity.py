@@ -150,6 +150,14 @@ def test_config1_first_steps_all_stages():
     _assert(run_parity(cfg, 8), TOL["bf16"])
 
 
+def test_config1_whole_unit_rounds():
+    """The attention's large-map split forced onto config 1 (a K/V budget of one byte): one
+    round of whole (head, patch, pair) units dealt one per CTA, then the 12 remaining units
+    split stream-K, each CTA's first tail piece first and its merging piece last."""
+    cfg = configs.get(1)
+    _assert(run_parity(cfg, 5, kv_budget=1), TOL["bf16"])
+
+
 def test_config1_simt_cross_check():
     cfg = configs.get(1)
     _assert(run_parity(cfg, 7, family=1), TOL["bf16"])
