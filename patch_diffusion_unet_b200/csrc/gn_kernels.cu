@@ -598,34 +598,64 @@ gn_fused_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int* err) {
 }
 
 // ---------------------------------------------------------------- streamed GroupNorm (bf16)
-// The fused GroupNorm with its two passes over the chunk moved by the copy engine: one
-// thread streams the chunk (contiguous: pixels [pix0, pix1) of patch p, all channels)
-// through a ring of kGsStages shared-memory stages with bulk copies completing on
-// mbarriers, so the threads only read shared memory and the memory system always has
-// kGsStages - 1 stages (~96 KB per SM) in flight.  Statistics pass: the stages are summed
-// as in gn_fused_kernel (the same shifts, the same fixed per-thread pixel order, so the
-// same partial sums).  Apply pass: its first stages are requested before the grid barrier
-// (the reads do not depend on it), each stage is normalised in place, and written back
-// with a bulk store (plus the stores of the rows that are a neighbour's halo on sync
-// steps).  The first pass's copies ask L2 to keep the lines (the chunk is read again),
-// the second's to drop them first.
-constexpr int kGsStages = 3;
-constexpr int kGsStageBytes = 49152;
+// The fused GroupNorm with its two passes over the chunk moved by the copy engine.  A copy
+// warp streams the chunk (contiguous: pixels [pix0, pix1) of patch p, all channels) through
+// a ring of kGsStages shared-memory stages with untiled bulk copies completing on `full`
+// mbarriers; the 16 compute warps only read shared memory and release each stage with one
+// arrival per warp on its `empty` mbarrier, so neither side waits for the other except on
+// the stage it needs.  Statistics pass: the stages are summed as in gn_fused_kernel (the
+// same shifts, the same fixed per-thread pixel order, so the same partial sums).  Apply
+// pass: the copy warp requests its first stages as soon as first-pass slots free up (the
+// reads do not depend on the grid barrier); the compute warps normalise each stage in place,
+// and the copy warp writes it back with a bulk store (plus, on sync steps, the rows that are a
+// neighbour's halo) before it reuses the slot.  The first pass's copies ask L2 to keep the
+// lines (the chunk is read again), the second's to drop them first.
+constexpr int kGsStages = 4;
+constexpr int kGsStageBytes = 40960;
+constexpr int kGsThreads = kGnThreads + 32;   // 16 compute warps and the copy warp
 
-int gs_stage_pixels(int C) { return std::max(1, kGsStageBytes / (C * 2)); }
-size_t gs_smem_bytes(int C) {
-  const int PL = kGnThreads / (C / 8);
-  return (size_t)kGsStages * gs_stage_pixels(C) * C * 2 + (size_t)(2 * PL + 2) * C * sizeof(float);
+// stage size: kGsStageBytes, less for very wide maps so that the ring and the partial sums
+// stay within 192 KB of dynamic shared memory
+size_t gs_sums_bytes(int C) { return (size_t)(2 * (kGnThreads / (C / 8)) + 2) * C * sizeof(float); }
+int gs_stage_pixels(int C) {
+  const long long room = (196608ll - (long long)gs_sums_bytes(C)) / kGsStages;
+  return (int)std::max(1ll, std::min<long long>(kGsStageBytes, room) / (C * 2));
+}
+size_t gs_smem_bytes(int C) { return (size_t)kGsStages * gs_stage_pixels(C) * C * 2 + gs_sums_bytes(C); }
+
+// barrier over the compute warps only (the copy warp runs its own loop)
+__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kGnThreads) : "memory"); }
+__device__ __forceinline__ void grid_arrive_c(unsigned* count) {
+  compute_sync();
+  if (threadIdx.x == 0) red_release_gpu_add(count, 1u);
+}
+__device__ __forceinline__ bool grid_wait_c(unsigned* count, unsigned total, int* err) {
+  __shared__ int s_ok;
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const long long t0 = clock64();
+    while (ld_acquire_gpu(count) < total) {
+      if (clock64() - t0 > kWaitLimitCycles) {
+        atomicCAS(err, 0, kErrGridSync);
+        ok = 0;
+        break;
+      }
+      __nanosleep(32);
+    }
+    s_ok = ok;
+  }
+  compute_sync();
+  return s_ok != 0;
 }
 
 template <bool SILU>
-__global__ void __launch_bounds__(kGnThreads, 1)
+__global__ void __launch_bounds__(kGsThreads, 1)
 gn_stream_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int stage_pix, int* err) {
   using T = __nv_bfloat16;
   constexpr int VEC = 8;
   constexpr int S = kGsStages;
   extern __shared__ __align__(128) uint8_t gs_smem[];
-  __shared__ __align__(8) uint64_t full[S];
+  __shared__ __align__(8) uint64_t full[S], empty[S];
   __shared__ __align__(16) float s_mr[256 * 2];    // (mean, rstd) of this patch's groups
   __shared__ __align__(16) float s_mom[256 * 2];   // fresh moments (mean, var) of the patches needed
   __shared__ float s_shift[256];                   // their shifts K
@@ -644,38 +674,102 @@ gn_stream_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int stage_p
   float* sh = reinterpret_cast<float*>(gs_smem + (size_t)S * stage_elems * sizeof(T));
   float* chan = sh + 2 * PL * C;
   const T* src = static_cast<const T*>(a.x) + (size_t)p * a.pix_per_patch * C;
+  const int last_row0 = a.pix_per_patch - o.W;
+  const int NI = a.per_image, pi = p % NI;                 // patch within its image
+  const bool top_src = o.halo_mode != 0 && pi > 0;         // my first row feeds patch p-1
+  const bool bot_src = o.halo_mode != 0 && pi < NI - 1;    // my last row feeds patch p+1
 
   if (tid == 0) {
-    for (int i = 0; i < S; ++i) mbar_init(smem_u32(&full[i]), 1);
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), kGnThreads / 32);
+    }
     fence_mbar_init();
   }
   __syncthreads();
   wait_prior_grid();            // everything below reads or writes buffers of other launches
   allow_next_grid();
 
-  // load number L (stage L of the first pass, stage L - nst of the second) into slot L % S
-  auto issue = [&](int L, uint64_t pol) {
-    const int k = L < nst ? L : L - nst;
-    const int s0 = pix0 + k * stage_pix, n = min(stage_pix, pix1 - s0);
-    const uint32_t bytes = (uint32_t)n * C * 2, bar = smem_u32(&full[L % S]);
-    mbar_arrive_expect_tx(bar, bytes);
-    bulk_load_policy(smem_u32(ring + (size_t)(L % S) * stage_elems), src + (size_t)s0 * C, bytes, bar, pol);
-  };
-  // every thread waits for load L (a failed wait ends the kernel's work, recorded in err)
-  auto ready = [&](int L) { return mbar_wait(smem_u32(&full[L % S]), (uint32_t)(L / S) & 1u, err, kErrWaitTmaFull); };
-  const uint64_t keep = l2_evict_last_policy(), drop = l2_evict_first_policy();
+  if (warp == kGnThreads / 32) {
+    // ------------------------------------------------------------ copy warp
+    if (lane == 0) {
+      const uint64_t keep = l2_evict_last_policy(), drop = l2_evict_first_policy();
+      T* outp = static_cast<T*>(o.out);
+      // load number L: stage L of the first pass, stage L - nst of the second, into slot L % S
+      auto issue = [&](int L) {
+        const int k = L < nst ? L : L - nst;
+        const int s0 = pix0 + k * stage_pix, n = min(stage_pix, pix1 - s0);
+        const uint32_t bytes = (uint32_t)n * C * 2, bar = smem_u32(&full[L % S]);
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_load_policy(smem_u32(ring + (size_t)(L % S) * stage_elems), src + (size_t)s0 * C, bytes, bar,
+                         L < nst ? keep : drop);
+      };
+      // the normalised second-pass stage of load L back to the output (and the halo rows)
+      auto store = [&](int L) {
+        const int k = L - nst;
+        const int s0 = pix0 + k * stage_pix, n = min(stage_pix, pix1 - s0);
+        const uint32_t sa = smem_u32(ring + (size_t)(L % S) * stage_elems);
+        bulk_store(outp + ((size_t)p * o.out_patch_stride + o.out_off + s0) * C, sa, (uint32_t)n * C * 2);
+        if (o.halo_mode == 1) {
+          // sync steps: this step's boundary rows are also the neighbours' halo rows
+          if (top_src && s0 < o.W) {
+            const int e = min(s0 + n, o.W);
+            bulk_store(outp + ((size_t)(p - 1) * o.out_patch_stride + o.out_off + a.pix_per_patch + s0) * C, sa,
+                       (uint32_t)(e - s0) * C * 2);
+          }
+          if (bot_src && s0 + n > last_row0) {
+            const int b = max(s0, last_row0);
+            bulk_store(outp + ((size_t)(p + 1) * o.out_patch_stride + (b - last_row0)) * C,
+                       sa + (uint32_t)(b - s0) * C * 2, (uint32_t)(s0 + n - b) * C * 2);
+          }
+        }
+        bulk_commit();
+      };
+      // the slot of load L is free once its previous occupant (load L - S) is released by the
+      // compute warps and, for a second-pass stage, stored and read out by the copy engine
+      bool ok = true;
+      int issued = 0;
+      for (int L = 0; L < 2 * nst; ++L) {
+        if (L >= S) {
+          const int occ = L - S;
+          ok = mbar_wait(smem_u32(&empty[occ % S]), (uint32_t)(occ / S) & 1u, err, kErrWaitStageFree);
+          if (!ok) break;
+          if (occ >= nst) {
+            store(occ);
+            bulk_wait_read_all();
+          }
+        }
+        issue(L);
+        issued = L + 1;
+      }
+      // the second-pass stages no later load displaces
+      for (int occ = max(nst, 2 * nst - S); ok && occ < 2 * nst; ++occ) {
+        ok = mbar_wait(smem_u32(&empty[occ % S]), (uint32_t)(occ / S) & 1u, err, kErrWaitStageFree);
+        if (ok) store(occ);
+      }
+      // the block's shared memory must outlive the stores' reads of it; their writes complete
+      // with the grid, before any later launch that waits for it reads them
+      bulk_wait_read_all();
+      if (!ok) {
+        // a wait gave up: let the loads still in flight land before the block exits (the last
+        // load issued into each slot; the earlier ones of a slot completed before it)
+        for (int L = max(0, issued - S); L < issued; ++L)
+          mbar_wait(smem_u32(&full[L % S]), (uint32_t)(L / S) & 1u, err, kErrWaitTmaFull);
+      }
+    }
+    return;
+  }
 
-  const int last_row0 = a.pix_per_patch - o.W;
-  const int NI = a.per_image, pi = p % NI;                 // patch within its image
-  const bool top_src = o.halo_mode != 0 && pi > 0;         // my first row feeds patch p-1
-  const bool bot_src = o.halo_mode != 0 && pi < NI - 1;    // my last row feeds patch p+1
-  // ---- pass 1: per-channel partial sums of x - K (K: the group's shift) over this chunk
-  // Loads 0 .. 2 nst - 1 (both passes) in order; load L + S goes into L's slot once load L is
-  // consumed, so the first pass's last slots already bring in the second pass's first stages.
+  // ------------------------------------------------------------ compute warps (512 threads)
+  // a failed wait ends this thread's work (the code is in err); arrivals continue, so the
+  // copy warp is never left waiting on a warp that gave up
+  auto ready = [&](int L) { return mbar_wait(smem_u32(&full[L % S]), (uint32_t)(L / S) & 1u, err, kErrWaitTmaFull); };
+  auto release = [&](int L) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&empty[L % S]));
+  };
   bool ok = true;
-  int issued = 0;               // thread 0: loads issued
-  if (tid == 0)
-    for (; issued < min(S, 2 * nst); ++issued) issue(issued, issued < nst ? keep : drop);
+  // ---- pass 1: per-channel partial sums of x - K (K: the group's shift) over this chunk
   {
     float s1[VEC], s2[VEC], k[VEC];
 #pragma unroll
@@ -697,11 +791,7 @@ gn_stream_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int stage_p
           }
         }
       }
-      __syncthreads();   // the slot is consumed
-      if (tid == 0 && ok && L + S < 2 * nst) {
-        issue(L + S, L + S < nst ? keep : drop);
-        issued = L + S + 1;
-      }
+      release(L);
     }
     if (pl < PL) {
       float4* d1 = reinterpret_cast<float4*>(sh + pl * C + vc * VEC);
@@ -713,14 +803,14 @@ gn_stream_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int stage_p
       }
     }
   }
-  __syncthreads();
+  compute_sync();
   for (int c = tid; c < C; c += kGnThreads) {
     float t1 = 0.f, t2 = 0.f;
     for (int l = 0; l < PL; ++l) { t1 += sh[l * C + c]; t2 += sh[PL * C + l * C + c]; }
     chan[c] = t1;
     chan[C + c] = t2;
   }
-  __syncthreads();
+  compute_sync();
   const int cg = C / G;
   for (int g = warp; g < G; g += kGnThreads / 32) {
     float t1 = 0.f, t2 = 0.f;
@@ -729,9 +819,7 @@ gn_stream_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int stage_p
     t2 = warp_sum(t2);
     if (lane == 0) reinterpret_cast<float2*>(a.part)[((size_t)lp * n_chunks + chunk) * G + g] = make_float2(t1, t2);
   }
-  // what the merge and the normalisation need besides the other blocks' partials, read
-  // before the barrier: this thread's gamma and beta, the shifts of the patches merged and
-  // the previous step's moments of the image's patches
+  // this thread's gamma and beta (read while the other blocks finish)
   float gm[VEC], bt[VEC];
 #pragma unroll
   for (int i = 0; i < VEC; ++i) {
@@ -745,7 +833,7 @@ gn_stream_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int stage_p
 
   // ---- grid barrier: every chunk partial is written
   const unsigned total = gridDim.x * gridDim.y;
-  grid_arrive(a.counter);
+  grid_arrive_c(a.counter);
   // the merge's other inputs, read while the other blocks reach the barrier
   if (tid < items) s_shift[tid] = gn_shift<T>(a.x, p_lo + tid / G, a.pix_per_patch, C, tid % G, cg);
   if (rule == kGnCorrected || rule == kGnStaleOthers)
@@ -777,7 +865,7 @@ gn_stream_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int stage_p
       }
     }
   }
-  if (!grid_wait(a.counter, total, err)) ok = false;
+  if (!grid_wait_c(a.counter, total, err)) ok = false;
 
   // ---- merge: fresh moments of the patches needed, in a fixed order
   const int SP = kGnThreads / items;            // threads per item, >= 2
@@ -797,7 +885,7 @@ gn_stream_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int stage_p
     red[(part_id * items + item) * 2 + 0] = acc.x;
     red[(part_id * items + item) * 2 + 1] = acc.y;
   }
-  __syncthreads();
+  compute_sync();
   const float inv_n = 1.f / ((float)a.pix_per_patch * (float)cg);
   if (ok && tid < items) {
     float t1 = 0.f, t2 = 0.f;
@@ -806,7 +894,7 @@ gn_stream_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int stage_p
     s_mom[tid * 2] = s_shift[tid] + m1;
     s_mom[tid * 2 + 1] = fmaxf(fmaf(-m1, m1, t2 * inv_n), 0.f);
   }
-  __syncthreads();
+  compute_sync();
   if (ok && tid < G) {
     const int gg = tid;
     const int own = (all ? pi : 0) * G + gg;
@@ -823,9 +911,9 @@ gn_stream_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int stage_p
       a.mean_rstd[(p * G + gg) * 2 + 1] = rstd;
     }
   }
-  __syncthreads();
+  compute_sync();
 
-  // ---- pass 2: normalise (+SiLU) each stage in place and store it back
+  // ---- pass 2: normalise (+SiLU) each stage in place; the copy warp stores it back
   float scl[VEC], sft[VEC];
 #pragma unroll
   for (int i = 0; i < VEC; ++i) {
@@ -833,12 +921,11 @@ gn_stream_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int stage_p
     scl[i] = gm[i] * s_mr[(c / cg) * 2 + 1];
     sft[i] = bt[i] - s_mr[(c / cg) * 2] * scl[i];
   }
-  T* outp = static_cast<T*>(o.out);
   for (int k = 0; k < nst; ++k) {
     const int L = nst + k;
     ok = ok && ready(L);
     T* st = ring + (size_t)(L % S) * stage_elems;
-    const int s0 = pix0 + k * stage_pix, n = min(stage_pix, pix1 - s0);
+    const int n = min(stage_pix, pix1 - (pix0 + k * stage_pix));
     if (ok && pl < PL) {
       for (int q = pl; q < n; q += PL) {
         uint4* cell = reinterpret_cast<uint4*>(st + (size_t)q * C + vc * VEC);
@@ -858,41 +945,7 @@ gn_stream_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int stage_p
       }
     }
     fence_proxy_async_smem();   // this thread's writes, before the copy engine reads them
-    __syncthreads();
-    if (tid == 0 && ok) {
-      const uint32_t sa = smem_u32(st);
-      bulk_store(outp + ((size_t)p * o.out_patch_stride + o.out_off + s0) * C, sa, (uint32_t)n * C * 2);
-      if (o.halo_mode == 1) {
-        // sync steps: this step's boundary rows are also the neighbours' halo rows
-        if (top_src && s0 < o.W) {
-          const int e = min(s0 + n, o.W);
-          bulk_store(outp + ((size_t)(p - 1) * o.out_patch_stride + o.out_off + a.pix_per_patch + s0) * C, sa,
-                     (uint32_t)(e - s0) * C * 2);
-        }
-        if (bot_src && s0 + n > last_row0) {
-          const int b = max(s0, last_row0);
-          bulk_store(outp + ((size_t)(p + 1) * o.out_patch_stride + (b - last_row0)) * C,
-                     sa + (uint32_t)(b - s0) * C * 2, (uint32_t)(s0 + n - b) * C * 2);
-        }
-      }
-      bulk_commit();
-      // refill the previous stage's slot (its stores have read it by now, as a rule), so two
-      // stages stay in flight while this one's stores run
-      if (L - 1 >= nst && L - 1 + S < 2 * nst) {
-        bulk_wait_read_prev();
-        issue(L - 1 + S, drop);
-        issued = L - 1 + S + 1;
-      }
-    }
-  }
-  if (tid == 0) {
-    bulk_wait_all();
-    if (!ok) {
-      // a wait gave up: let the loads still in flight land before the block exits (the last
-      // load issued into each slot; the earlier ones of a slot completed before it)
-      for (int L = max(0, issued - S); L < issued; ++L)
-        mbar_wait(smem_u32(&full[L % S]), (uint32_t)(L / S) & 1u, err, kErrWaitTmaFull);
-    }
+    release(L);
   }
   // ---- departure: the last block out re-arms the barrier for the next launch
   if (tid == 0 && atomicAdd(a.counter + 1, 1u) == total - 1) {
@@ -900,7 +953,6 @@ gn_stream_kernel(GnArgs a, GnOut o, int n_chunks, int pix_per_chunk, int stage_p
     a.counter[1] = 0u;
   }
 }
-
 
 // Pixels per block: one wave of 512-thread blocks over the whole map.
 // Per-token LayerNorm (transformer blocks of the SDXL-style stage): one warp per
@@ -1040,7 +1092,8 @@ cudaError_t launch_gn_fused(const GnArgs& a, const GnOut& o, bool silu, int* err
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, kGnThreads, smem);
+  const int threads = kStream ? kGsThreads : kGnThreads;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, threads, smem);
   if (e != cudaSuccess) return e;
   const int max_blocks = per_sm * sm_count();
   const int n_run = a.n_run > 0 ? a.n_run : a.N;   // patches computed
@@ -1054,7 +1107,7 @@ cudaError_t launch_gn_fused(const GnArgs& a, const GnOut& o, bool silu, int* err
   n_chunks = (a.pix_per_patch + per - 1) / per;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(n_chunks, n_run);
-  cfg.blockDim = dim3(kGnThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
