@@ -324,12 +324,7 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
-// every bulk group of this thread but the latest has finished reading its source
-__device__ __forceinline__ void bulk_wait_read_prev() {
-  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
-// every bulk group of this thread has completed (its writes performed)
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 
 // Programmatic dependent launch.  A kernel launched with the programmatic stream
 // serialization attribute may be scheduled while the kernel before it in the stream is
