@@ -1084,8 +1084,11 @@ cudaError_t launch_gn_fused(const GnArgs& a, const GnOut& o, bool silu, int* err
   if (smem < red) smem = red;
   using Kern = void (*)(GnArgs, GnOut, int, int, int*);
   using SKern = void (*)(GnArgs, GnOut, int, int, int, int*);
-  Kern kern = silu ? gn_fused_kernel<T, true> : gn_fused_kernel<T, false>;
-  SKern skern = silu ? gn_stream_kernel<true> : gn_stream_kernel<false>;
+  // bf16 takes the streamed kernel, fp32 the register-streaming one (only one is instantiated)
+  Kern kern = nullptr;
+  SKern skern = nullptr;
+  if constexpr (kStream) skern = silu ? gn_stream_kernel<true> : gn_stream_kernel<false>;
+  else kern = silu ? gn_fused_kernel<T, true> : gn_fused_kernel<T, false>;
   const void* kfn = kStream ? reinterpret_cast<const void*>(skern) : reinterpret_cast<const void*>(kern);
   // every block must be resident at once (the grid barrier): at most the occupancy
   // limit, and no more chunks than the partial-sum scratch holds
@@ -1119,8 +1122,8 @@ cudaError_t launch_gn_fused(const GnArgs& a, const GnOut& o, bool silu, int* err
   cfg.numAttrs = a.pdl ? 2 : 1;
   const int stage_pix = gs_stage_pixels(a.C);
   auto go = [&]() {
-    return kStream ? cudaLaunchKernelEx(&cfg, skern, a, o, n_chunks, per, stage_pix, err)
-                   : cudaLaunchKernelEx(&cfg, kern, a, o, n_chunks, per, err);
+    if constexpr (kStream) return cudaLaunchKernelEx(&cfg, skern, a, o, n_chunks, per, stage_pix, err);
+    else return cudaLaunchKernelEx(&cfg, kern, a, o, n_chunks, per, err);
   };
   e = go();
   if (e != cudaSuccess && a.pdl) {
