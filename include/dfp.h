@@ -287,7 +287,9 @@ DFP_API int dfp_launches_per_step(dfp_handle h);
  * does and checks: every CTA has work and every piece stays inside its unit; every unit is
  * covered once; a pair cut between CTAs has its first KV tiles at the end of one CTA's
  * tail range (that CTA merges) and its other pieces each at the start of a range; the
- * kernel's publisher and flag warps predict exactly those pieces.  L tokens per image in
+ * kernel's publisher and flag warps predict exactly those pieces; the softmax's per-piece
+ * table of partial tiles gives every KV tile the valid key count of the TMA warp's per-tile
+ * walk.  L tokens per image in
  * n_patches patches of Lp tokens; mode 0 sync, 1 displaced, 2 naive, 3 cross-attention
  * (Lp = L, n_patches = 1, kv_len context tokens).  Only the query patches [p_begin, p_end)
  * of the image-major patch list are listed (p_begin = p_end = 0: all), as for a

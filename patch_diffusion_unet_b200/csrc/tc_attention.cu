@@ -100,7 +100,7 @@ __host__ __device__ __forceinline__ int unit_tiles(int mode, int p, int Lp, int 
 }
 
 // tile j of patch p's KV list -> (stale?, first key row, valid keys)
-__device__ __forceinline__ void tile_src(int mode, int p, int Lp, int L, int kv_len, int j, int& stale,
+__host__ __device__ __forceinline__ void tile_src(int mode, int p, int Lp, int L, int kv_len, int j, int& stale,
                                          int& row, int& valid) {
   stale = 0;
   if (mode == kAttnSync || mode == kAttnCross) {
@@ -124,6 +124,38 @@ __device__ __forceinline__ void tile_src(int mode, int p, int Lp, int L, int kv_
   }
   row = (p + 1) * Lp + (j - t1) * kTile;
   valid = min(kTile, L - row);
+}
+
+// Only the last tile of each of the (at most three) segments of patch p's KV list can be
+// partial: their indices in the list (-1: no such segment) and valid key counts, the same
+// counts tile_src gives, taken once per piece instead of per tile.
+struct TileEnds {
+  int e0, v0, e1, v1, e2, v2;
+};
+__host__ __device__ __forceinline__ TileEnds tile_ends(int mode, int p, int Lp, int L, int kv_len) {
+  TileEnds t{-1, kTile, -1, kTile, -1, kTile};
+  if (mode == kAttnSync || mode == kAttnCross) {
+    const int len = mode == kAttnSync ? L : kv_len;
+    const int T = cdiv(len, kTile);
+    t.e0 = T - 1;
+    t.v0 = len - (T - 1) * kTile;
+    return t;
+  }
+  const int own = cdiv(Lp, kTile);
+  t.e0 = own - 1;
+  t.v0 = Lp - (own - 1) * kTile;
+  if (mode == kAttnDisplaced) {
+    const int t1 = cdiv(p * Lp, kTile), t2 = cdiv(L - (p + 1) * Lp, kTile);
+    if (t1 > 0) {
+      t.e1 = own + t1 - 1;
+      t.v1 = p * Lp - (t1 - 1) * kTile;
+    }
+    if (t2 > 0) {
+      t.e2 = own + t1 + t2 - 1;
+      t.v2 = L - (p + 1) * Lp - (t2 - 1) * kTile;
+    }
+  }
+  return t;
 }
 
 // The unit list: head-major over (head, query patch, Q-tile pair) -- patch pg = img * N + p
@@ -828,15 +860,13 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constan
       }
       volatile int* sp = s_ring[pi & 3];
       const int n = carry ? 0 : sp[6];
+      const int j0 = sp[5];
+      const TileEnds te = tile_ends(a.mode, sp[0] % a.N, a.Lp, a.L, a.kv_len);
       float m_used = -INFINITY;
       for (int jj = 0; jj < n && !carry; ++jj, ++gt) {
-        // every tile is full when all segment lengths are multiples of the tile (parameters
-        // only: no per-tile lookup); otherwise the tile's valid key count
-        int valid = kTile;
-        if (!((a.mode == kAttnCross ? a.kv_len : (a.Lp | a.L)) % kTile == 0)) {
-          int stale, krow;
-          tile_src(a.mode, sp[0] % a.N, a.Lp, a.L, a.kv_len, sp[5] + jj, stale, krow, valid);
-        }
+        // the tile's valid key count (a segment's last tile may be partial)
+        const int jt = j0 + jj;
+        const int valid = jt == te.e0 ? te.v0 : jt == te.e1 ? te.v1 : jt == te.e2 ? te.v2 : kTile;
         if (!mbar_wait_warp(smem_u32(&s_full[g]), gt & 1, err, kErrWaitAttnS)) { carry = true; break; }
         tc_fence_after();
         float sc[64];   // sc[i] = S[row][2i + cq]
@@ -1107,6 +1137,17 @@ int attention_schedule_check(int L, int Lp, int N, int heads, int mode, int kv_l
     if (publishes != expect_publish || merges != expect_merge) return 8;
     // the merging piece is the CTA's last, or its only tail piece (then it opens the sequence)
     if (merges && merge_k != pieces - 1 && !(merge_k == 0 && pieces - whole == 1)) return 12;
+  }
+  // the softmax's per-piece partial-tile table gives every tile the valid key count the
+  // TMA warp's per-tile walk gives
+  for (int p = 0; p < N; ++p) {
+    const TileEnds te = tile_ends(mode, p, Lp, L, kv_len);
+    for (int j = 0; j < unit_tiles(mode, p, Lp, L, kv_len); ++j) {
+      int stale, row, valid;
+      tile_src(mode, p, Lp, L, kv_len, j, stale, row, valid);
+      const int v = j == te.e0 ? te.v0 : j == te.e1 ? te.v1 : j == te.e2 ? te.v2 : kTile;
+      if (v != valid || valid < 1 || valid > kTile) return 13;
+    }
   }
   // every unit covered exactly once, whole
   for (int h = 0; h < heads; ++h)
