@@ -282,7 +282,7 @@ def oracle_step_seconds(blk, cfg, x, t, is_sync, sample):
 
 def oracle_sample_text(cfg, sample):
     if sample is None:
-        return "full layer steps"
+        return "full UNet evaluations" if cfg.get("block") == "unet" else "full layer steps"
     L = cfg["H"] * cfg["W"]
     return (f"bounded steps: GroupNorms, conv and Q/K/V/O projections in full, attention output for "
             f"{len(sample)} of {L} query tokens ({len(sample) // cfg['n_patches']} evenly spaced per patch); "
@@ -333,6 +333,15 @@ def dist_setup():
     return world, rank, local
 
 
+def workload_config(cfg, B):
+    """The keys of a line's `config` that name the workload, the same in both arms."""
+    if cfg["block"] == "unet":
+        return {"workload": cfg["name"], "H": cfg["H"], "W": cfg["W"], "widths": list(cfg["widths"]),
+                "n_patches": cfg["n_patches"], "step": "displaced UNet evaluation (is_sync=0)"}
+    return {"workload": cfg["name"], "H": cfg["H"], "W": cfg["W"], "C": cfg["C"], "n_patches": cfg["n_patches"],
+            "heads": cfg["heads"], "batch": B, "step": "displaced (is_sync=0)"}
+
+
 def run_reference(args, cfg):
     """The reference arm: the oracle on the host cores, rank 0 only, on the same workload,
     metric and unit; the synchronous steps of the schedule, then W displaced warm-up steps
@@ -374,17 +383,18 @@ def run_reference(args, cfg):
     threads = _oracle_threads()
     value = args.steps / dt
     L = cfg["H"] * cfg["W"]
-    text = f"{args.steps} displaced layer steps after {n_sync} sync and {args.warmup} warm-up steps; " + \
+    unit = "unet-steps/s" if cfg["block"] == "unet" else UNIT
+    what = "displaced UNet evaluations" if cfg["block"] == "unet" else "displaced layer steps"
+    text = f"{args.steps} {what} after {n_sync} sync and {args.warmup} warm-up steps; " + \
         oracle_sample_text(cfg, sample)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "latent_px_per_s": value * L * B, "images_per_s": value * B,
-        "config": {"workload": cfg["name"], "H": cfg["H"], "W": cfg["W"], "C": cfg["C"],
-                   "n_patches": cfg["n_patches"], "batch": B, "l2": "n/a (CPU)"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": text},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "config": {**workload_config(cfg, B), "parallelism": "rank 0 on the host cores", "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": text},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -521,10 +531,8 @@ def run_unet(args, cfg):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random weights, random latents)",
             "latent_px_per_s": value * H * W, "tensor_tflops_per_step": ach,
-            "config": {"workload": cfg["name"], "H": H, "W": W, "widths": list(cfg["widths"]),
-                       "n_patches": cfg["n_patches"], "parallelism": f"replicas{world}",
-                       "l2": "flushed between timed steps (512 MB write, outside the events)",
-                       "step": "displaced UNet evaluation (is_sync=0)"},
+            "config": {**workload_config(cfg, 1), "parallelism": f"replicas{world}",
+                       "l2": "flushed between timed steps (512 MB write, outside the events)"},
             "gpu_launches": launches * args.steps, "launches_per_step": launches,
             "kernels_us": {k: round(v, 2) for k, v in kern_us.items()},
             "flops_per_part_g": {k: round(v / 1e9, 2) for k, v in parts.items()},
@@ -704,11 +712,9 @@ def main():
             "vs_baseline": None, "dtype": "bf16" if dtype == "bf16" else "f32", "data": "synthetic",
             "latent_px_per_s": value * L * B, "images_per_s": value * B,
             "tensor_tflops_per_step": wm["_total_flops"] / (ms_step * 1e-3) / 1e12,
-            "config": {"workload": cfg["name"], "H": cfg["H"], "W": cfg["W"], "C": cfg["C"],
-                       "n_patches": cfg["n_patches"], "heads": cfg["heads"], "batch": B,
-                       "launch_overlap": not args.no_overlap, "parallelism": f"replicas{world}",
-                       "l2": "flushed between timed steps (512 MB write, outside the events)",
-                       "step": "displaced (is_sync=0)"},
+            "config": {**workload_config(cfg, B), "launch_overlap": not args.no_overlap,
+                       "parallelism": f"replicas{world}",
+                       "l2": "flushed between timed steps (512 MB write, outside the events)"},
             "sync_ms_per_step": sync_ms,
             "gpu_launches": launches * args.steps,
             "launches_per_step": launches,
