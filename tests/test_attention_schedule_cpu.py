@@ -38,10 +38,12 @@ def test_self_attention_split(shape, mode, budget):
             assert _check(L, Lp, N, heads, mode, images=images, ctas=ctas, budget=budget) == 0, (images, ctas)
 
 
+@pytest.mark.parametrize("kv_len", [1, 77, 128, 129, 300])
 @pytest.mark.parametrize("images", [1, 2, 3])
-def test_cross_attention_split(images):
+def test_cross_attention_split(images, kv_len):
+    """The context's key count sets the one partial tile (none at 128)."""
     for ctas in CTAS:
-        assert _check(4096, 4096, 1, 20, CROSS, kv_len=77, images=images, ctas=ctas) == 0
+        assert _check(4096, 4096, 1, 20, CROSS, kv_len=kv_len, images=images, ctas=ctas) == 0
 
 
 def test_random_splits():
